@@ -1,0 +1,187 @@
+/*
+ * iskv.h -- C ABI of libiskv, the B200 (sm_100a) hot path of iS-KV online low-rank KV-cache
+ * compression.
+ *
+ * Sources: "iS-KV reading notes" (zhongzhuzhou.org notes on "iS-KV: Online Low-Rank KV Cache
+ * Compression via Block-Incremental SVD"), cited by section / algorithm / equation.
+ *
+ * Conventions for every entry point
+ *  - All array arguments are DEVICE pointers unless a comment says "host". The caller owns all
+ *    memory: the library never allocates on these paths; every call that needs scratch takes a
+ *    caller workspace sized by the matching *_workspace_size() query.
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed as void*; NULL = the
+ *    legacy default stream). The return value reports argument errors found on the host
+ *    (ISKV_ERR_ARG / ISKV_ERR_SHAPE / ISKV_ERR_WORKSPACE) or a failed kernel launch
+ *    (ISKV_ERR_CUDA); nothing is launched when an error is returned.
+ *  - Conditions found on the device (capacity, non-finite values, an unconverged Jacobi sweep, a
+ *    bounded wait that ran out) are OR-ed into the history's device status word
+ *    (meta[ISKV_META_STATUS], bit (1 << code)) and read back with iskv_get_status(), which syncs.
+ *  - Matrices are row-major. Element types are given by iskv_dtype values.
+ */
+#ifndef ISKV_H
+#define ISKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ISKV_ABI_VERSION 1
+
+typedef enum {
+  ISKV_OK = 0,
+  ISKV_ERR_ARG = 1,            /* null pointer, bad enum, misaligned pointer                  */
+  ISKV_ERR_SHAPE = 2,          /* inconsistent or unsupported sizes                           */
+  ISKV_ERR_CUDA = 3,           /* a CUDA runtime call or kernel launch failed                 */
+  ISKV_ERR_CAPACITY = 4,       /* device: n + b > n_cap, the fold was skipped                 */
+  ISKV_ERR_NONFINITE = 5,      /* device: a non-finite singular value came out of a fold      */
+  ISKV_ERR_NOT_CONVERGED = 6,  /* device: Jacobi / Newton-Schulz hit its iteration cap        */
+  ISKV_ERR_TIMEOUT = 7,        /* device: a bounded cluster wait gave up                      */
+  ISKV_ERR_WORKSPACE = 8       /* workspace pointer null, misaligned or too small             */
+} iskv_status;
+
+typedef enum { ISKV_F32 = 0, ISKV_BF16 = 1 } iskv_dtype;
+
+/* Indices into the device meta word of a history. */
+enum { ISKV_META_K = 0, ISKV_META_N = 1, ISKV_META_FOLDS = 2, ISKV_META_STATUS = 3 };
+
+/*
+ * One compressed history: one (sequence, layer, K|V) path, the factors U diag(sigma) B^T of
+ * Section 2.2 ("iS-KV reading notes"), rank k <= r_max, n compressed rows.
+ *   U      [n_cap][r_max]  storage dtype; row i = coordinates of compressed row i. Must be
+ *                          zero-initialised (columns >= k are read as zero).
+ *   sigma  [r_max]         float32, descending; entries >= k are zero.
+ *   B      [d][r_max]      storage dtype; column j = basis vector j. Zero-initialised.
+ *   pos    [n_cap]         int32 original token position of U row i (Section 3.2: K and V
+ *                          histories index different tokens, so rows are scattered by position).
+ *   meta   [4]             int64 {k, n, folds since last reorth, status bits}; zero at creation.
+ * All five pointers are device pointers, 16-byte aligned. d must be a multiple of 16 and r_max a
+ * multiple of 16, 16 <= r_max <= min(d, 512).
+ */
+typedef struct {
+  int32_t d;
+  int32_t r_max;
+  int64_t n_cap;
+  int32_t storage; /* iskv_dtype of U and B */
+  int32_t reserved;
+  void *U;
+  float *sigma;
+  void *B;
+  int32_t *pos;
+  int64_t *meta;
+} iskv_lowrank;
+
+/* ABI version (ISKV_ABI_VERSION) and a static string naming a status code. */
+int32_t iskv_abi_version(void);
+const char *iskv_status_string(int32_t status);
+
+/* Detail of the last host-side error on the calling thread (empty string if none). */
+const char *iskv_last_error(void);
+
+/*
+ * Block fold -- Algorithm 2 of Section 4 ("iS-KV reading notes"): merge the pending block F of b
+ * exact rows into the history, rotating the basis and EVERY history coordinate row together:
+ *   C = F B;  E = F - C B^T;  E <- E - (E B) B^T;  Householder QR  E^T = Q_R R_R;  SVD of R_R;
+ *   P = kept residual directions (rho_i > tol, tol = max(tau_rel, 2^-23 max(b,d)) * max(sigma_1,
+ *   rho_1));  Z = [[diag sigma, 0], [F B, F P]];  Z = G diag(sigma+) H^T truncated to
+ *   k' = min(r_max, k + p);  U[0:n] <- U[0:n] G[0:k];  U[n:n+b] <- G[k:];  B <- [B, P] H;
+ *   pos[n:n+b] <- f_pos;  k <- k';  n <- n + b;  folds += 1.
+ * F      [b][d] f_dtype (device). f_pos [b] int32 (device).
+ * Sizes: 1 <= b <= min(d, 128), b % 8 == 0.
+ * ws     caller workspace of at least iskv_fold_workspace_size(1, d, r_max, b) bytes, 256-byte
+ *        aligned; its contents need no initialisation and are scratch after the call returns.
+ * Device errors: n + b > n_cap -> the fold is a no-op and ISKV_ERR_CAPACITY is recorded;
+ * non-finite new singular values -> ISKV_ERR_NONFINITE; Jacobi sweep cap -> ISKV_ERR_NOT_CONVERGED
+ * (best-so-far result is kept).
+ */
+size_t iskv_fold_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t b);
+iskv_status iskv_fold_block(const iskv_lowrank *h, const void *F, int32_t f_dtype, int32_t b,
+                            const int32_t *f_pos, float tau_rel, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/*
+ * The same fold for `count` independent histories in one set of launches (e.g. every layer's K
+ * and V path when their pending queues fill on the same decode step, Algorithm 3 step 4).
+ * hs, F, f_pos are HOST arrays of `count` entries (F[i], f_pos[i] are device pointers). All
+ * histories share d, r_max, storage; all blocks share b and f_dtype. 1 <= count <= 4096.
+ */
+iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const void *const *F,
+                                    int32_t f_dtype, int32_t b, const int32_t *const *f_pos,
+                                    float tau_rel, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Re-orthogonalisation -- Section 4.4: with orthonormal-basis factorisations U = Q_U R_U,
+ * B = Q_B R_B, decompose R_U diag(sigma) R_B^T = X diag(sigma') Y^T and set U <- Q_U X,
+ * sigma <- sigma', B <- Q_B Y. The product U diag(sigma) B^T is unchanged in exact arithmetic;
+ * k and n are unchanged; meta[FOLDS] is reset to 0. hs is a HOST array of `count` handles sharing
+ * d, r_max, storage and n_cap.
+ */
+size_t iskv_reorth_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap);
+iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t ws_bytes,
+                        void *stream);
+
+/*
+ * Reconstruction -- Algorithm 3 steps 7-8: out[pos[i], :] = (U[i] * sigma) B^T for the n
+ * compressed rows, out[exact_pos[e], :] = exact_rows[e] for the n_exact exact rows; when
+ * apply_rope != 0 every written row is then rotated by its own position with rotate-half RoPE
+ * (pairs (j, j + head_dim/2) inside each head, angle pos * rope_theta^(-2j/head_dim)).
+ * out          [n_total][d] out_dtype; rows not named by either set are left untouched.
+ * exact_rows   [n_exact][d] exact_dtype (may be NULL when n_exact == 0); exact_pos [n_exact].
+ * Positions must lie in [0, n_total) and be distinct across both sets (not checked on device).
+ * d == n_heads * head_dim, head_dim even and <= 256.
+ * ws           iskv_reconstruct_workspace_size(1, d, r_max) bytes (sigma-scaled basis).
+ * hs and the per-job arrays of the batched form are HOST arrays of `count` entries.
+ */
+size_t iskv_reconstruct_workspace_size(int32_t count, int32_t d, int32_t r_max);
+iskv_status iskv_reconstruct(const iskv_lowrank *h, const void *exact_rows, int32_t exact_dtype,
+                             const int32_t *exact_pos, int64_t n_exact, int64_t n_total,
+                             int32_t n_heads, int32_t head_dim, int32_t apply_rope,
+                             double rope_theta, void *out, int32_t out_dtype, void *ws,
+                             size_t ws_bytes, void *stream);
+iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
+                                     const void *const *exact_rows, int32_t exact_dtype,
+                                     const int32_t *const *exact_pos, const int64_t *n_exact,
+                                     const int64_t *n_total, int32_t n_heads, int32_t head_dim,
+                                     const int32_t *apply_rope, double rope_theta,
+                                     void *const *out, int32_t out_dtype, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/*
+ * Prompt-block protection -- Section 3.1 and Algorithm 1 steps 2-4: blocks of `block` prompt
+ * tokens; the last `suffix_blocks` full blocks and the partial tail are the local suffix; for each
+ * KV head, score(block) = min over its tokens of cos(post-RoPE key, block-mean key) (float64,
+ * cos = dot / max(|k||m|, 1e-30)); each head picks its `per_head` lowest (score, block index)
+ * candidates (all if fewer); P_K = union over heads of the picked blocks' tokens plus the suffix;
+ * P_V = every prompt position q with |p - q| <= v_radius for some p in P_K.
+ * keys            [L][n_heads][head_dim] k_dtype, post-RoPE.
+ * pk_out, pv_out  [L] int32: ascending positions (first n_pk / n_pv entries valid).
+ * head_blocks_out [n_heads][per_head] int32: each head's picked blocks ascending, -1 padded.
+ * counts_out      [2 + n_heads] int64: {n_pk, n_pv, n_picked[h]...}.
+ * Limits: 1 <= L <= 2^24, n_heads <= 64, head_dim <= 256 and even, block in [1, 64],
+ * per_head <= 4096.
+ */
+size_t iskv_select_workspace_size(int64_t L, int32_t n_heads, int32_t block);
+iskv_status iskv_select_prompt_blocks(const void *keys, int32_t k_dtype, int64_t L,
+                                      int32_t n_heads, int32_t head_dim, int32_t block,
+                                      int32_t per_head, int32_t suffix_blocks, int32_t v_radius,
+                                      int32_t *pk_out, int32_t *pv_out, int32_t *head_blocks_out,
+                                      int64_t *counts_out, void *ws, size_t ws_bytes,
+                                      void *stream);
+
+/* Zero a history's meta word and sigma (stream-ordered). U and B are not touched. */
+iskv_status iskv_reset(const iskv_lowrank *h, void *stream);
+
+/*
+ * Synchronously read a history's meta word (waits for all work on the device to finish).
+ * Any output pointer may be NULL (host pointers).
+ */
+iskv_status iskv_get_status(const iskv_lowrank *h, int64_t *k, int64_t *n, int64_t *folds,
+                            int64_t *status_bits);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISKV_H */

@@ -1,0 +1,243 @@
+"""kv_cache_online_b200 -- B200 (sm_100a) hot path of iS-KV online low-rank KV-cache compression.
+
+Thin Python binding over ``libiskv.so`` (C ABI in ``include/iskv.h``). PyTorch provides device
+memory and streams; every step of the fold, re-orthogonalisation, reconstruction and prompt-block
+selection runs in the library's CUDA kernels. There is no CPU or PyTorch fallback: if the library is
+missing, every call raises.
+
+Sources: "iS-KV reading notes" (zhongzhuzhou.org), Sections 3-5 and Algorithms 1-3.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import ISKV_BF16, ISKV_F32, IskvError, IskvLowRank  # noqa: F401
+
+_DT = {torch.float32: ISKV_F32, torch.bfloat16: ISKV_BF16}
+_TD = {ISKV_F32: torch.float32, ISKV_BF16: torch.bfloat16}
+
+
+def _dt(t: torch.Tensor) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16") from None
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must live on a CUDA device")
+
+
+class Workspace:
+    """A reusable, 256-byte aligned device byte buffer grown on demand."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        nbytes = max(int(nbytes), 256)
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=self.device)
+        off = (-self.buf.data_ptr()) % 256
+        return self.buf[off:off + nbytes]
+
+
+_default_ws = {}
+
+
+def _ws(device, nbytes):
+    key = (str(device), "ws")
+    w = _default_ws.get(key)
+    if w is None:
+        w = _default_ws[key] = Workspace(device)
+    return w.get(nbytes)
+
+
+class LowRankHistory:
+    """One compressed history (a (sequence, layer, K|V) path): ``U diag(sigma) B^T`` with the
+    original token position of every compressed row (Section 2.2 and Section 3.2).
+
+    Device tensors: ``U`` (n_cap, r_max), ``sigma`` (r_max,) float32, ``B`` (d, r_max), ``pos``
+    (n_cap,) int32, ``meta`` (4,) int64 = {k, n, folds since reorth, status bits}.
+    """
+
+    def __init__(self, d: int, r_max: int, n_cap: int, storage=torch.bfloat16, device="cuda"):
+        self.d, self.r_max, self.n_cap = int(d), int(r_max), int(n_cap)
+        self.storage = storage
+        self.U = torch.zeros(self.n_cap, self.r_max, dtype=storage, device=device)
+        self.sigma = torch.zeros(self.r_max, dtype=torch.float32, device=device)
+        self.B = torch.zeros(self.d, self.r_max, dtype=storage, device=device)
+        self.pos = torch.zeros(max(self.n_cap, 1), dtype=torch.int32, device=device)
+        self.meta = torch.zeros(4, dtype=torch.int64, device=device)
+
+    @property
+    def device(self):
+        return self.U.device
+
+    def handle(self) -> IskvLowRank:
+        return IskvLowRank(self.d, self.r_max, self.n_cap, _DT[self.storage], 0, _ptr(self.U),
+                           _ptr(self.sigma), _ptr(self.B), _ptr(self.pos), _ptr(self.meta))
+
+    def status(self):
+        """(k, n, folds since reorth, status bits); synchronises the device."""
+        k, n, f, s = (ctypes.c_int64() for _ in range(4))
+        h = self.handle()
+        _lib.check(_lib.load().iskv_get_status(ctypes.byref(h), ctypes.byref(k), ctypes.byref(n),
+                                               ctypes.byref(f), ctypes.byref(s)), "get_status")
+        return k.value, n.value, f.value, s.value
+
+    def reset(self, stream=None):
+        h = self.handle()
+        _lib.check(_lib.load().iskv_reset(ctypes.byref(h), _stream(stream)), "reset")
+
+
+def _handles(hists):
+    arr = (IskvLowRank * len(hists))()
+    for i, h in enumerate(hists):
+        arr[i] = h.handle()
+    return arr
+
+
+def fold_workspace_size(count, d, r_max, b) -> int:
+    return int(_lib.load().iskv_fold_workspace_size(count, d, r_max, b))
+
+
+def fold_block_batched(hists, Fs, f_poss, tau_rel: float = 0.0, ws=None, stream=None):
+    """Algorithm 2 for every history in ``hists`` (one pending block each), in one launch set."""
+    lib = _lib.load()
+    n = len(hists)
+    if n == 0:
+        return
+    b = int(Fs[0].shape[0])
+    fdt = _dt(Fs[0])
+    for F, p in zip(Fs, f_poss):
+        _need_cuda(F, p)
+        if F.shape != (b, hists[0].d) or _dt(F) != fdt or not F.is_contiguous():
+            raise ValueError("every F must be a contiguous (b, d) tensor of one dtype")
+        if p.dtype != torch.int32 or p.numel() != b or not p.is_contiguous():
+            raise ValueError("f_pos must be a contiguous int32 tensor of b entries")
+    need = lib.iskv_fold_workspace_size(n, hists[0].d, hists[0].r_max, b)
+    w = ws if ws is not None else _ws(hists[0].device, need)
+    hs = _handles(hists)
+    Fp = (ctypes.c_void_p * n)(*[F.data_ptr() for F in Fs])
+    Pp = (ctypes.c_void_p * n)(*[p.data_ptr() for p in f_poss])
+    _lib.check(lib.iskv_fold_block_batched(hs, n, Fp, fdt, b, Pp, float(tau_rel), w.data_ptr(),
+                                           w.numel(), _stream(stream)), "fold_block")
+
+
+def fold_block(hist, F, f_pos, tau_rel: float = 0.0, ws=None, stream=None):
+    """Algorithm 2: merge the pending block ``F`` (b, d) at positions ``f_pos`` into ``hist``."""
+    fold_block_batched([hist], [F], [f_pos], tau_rel, ws, stream)
+
+
+def reorth_workspace_size(count, d, r_max, n_cap) -> int:
+    return int(_lib.load().iskv_reorth_workspace_size(count, d, r_max, n_cap))
+
+
+def reorth(hists, ws=None, stream=None):
+    """Section 4.4 re-orthogonalisation of every history in ``hists``."""
+    if isinstance(hists, LowRankHistory):
+        hists = [hists]
+    lib = _lib.load()
+    n = len(hists)
+    need = lib.iskv_reorth_workspace_size(n, hists[0].d, hists[0].r_max, hists[0].n_cap)
+    w = ws if ws is not None else _ws(hists[0].device, need)
+    _lib.check(lib.iskv_reorth(_handles(hists), n, w.data_ptr(), w.numel(), _stream(stream)),
+               "reorth")
+
+
+def reconstruct_workspace_size(count, d, r_max) -> int:
+    return int(_lib.load().iskv_reconstruct_workspace_size(count, d, r_max))
+
+
+def reconstruct_batched(hists, exact_rows, exact_pos, n_total, n_heads, head_dim, rope,
+                        theta=500000.0, outs=None, out_dtype=torch.bfloat16, ws=None, stream=None):
+    """Algorithm 3 steps 7-8 for every history: dense (n_total, d) caches with compressed rows at
+    their positions, exact rows copied, keys rotated (``rope[i]``)."""
+    lib = _lib.load()
+    n = len(hists)
+    d = hists[0].d
+    if isinstance(n_total, int):
+        n_total = [n_total] * n
+    if isinstance(rope, bool):
+        rope = [rope] * n
+    if outs is None:
+        outs = [torch.empty(nt, d, dtype=out_dtype, device=h.device) for h, nt in zip(hists, n_total)]
+    odt = _dt(outs[0])
+    edt = ISKV_F32
+    er, ep, ne = [], [], []
+    for x, p in zip(exact_rows, exact_pos):
+        if x is None or p is None or p.numel() == 0:
+            er.append(None)
+            ep.append(None)
+            ne.append(0)
+            continue
+        _need_cuda(x, p)
+        edt = _dt(x)
+        if p.dtype != torch.int32 or x.shape != (p.numel(), d) or not x.is_contiguous():
+            raise ValueError("exact rows must be (n_exact, d) contiguous with int32 positions")
+        er.append(x.data_ptr())
+        ep.append(p.data_ptr())
+        ne.append(p.numel())
+    need = lib.iskv_reconstruct_workspace_size(n, d, hists[0].r_max)
+    w = ws if ws is not None else _ws(hists[0].device, need)
+    _lib.check(lib.iskv_reconstruct_batched(
+        _handles(hists), n, (ctypes.c_void_p * n)(*er), edt, (ctypes.c_void_p * n)(*ep),
+        (ctypes.c_int64 * n)(*ne), (ctypes.c_int64 * n)(*n_total), n_heads, head_dim,
+        (ctypes.c_int32 * n)(*[1 if r else 0 for r in rope]), float(theta),
+        (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs]), odt, w.data_ptr(), w.numel(),
+        _stream(stream)), "reconstruct")
+    return outs
+
+
+def reconstruct(hist, exact_rows, exact_pos, n_total, n_heads, head_dim, rope, theta=500000.0,
+                out=None, out_dtype=torch.bfloat16, ws=None, stream=None):
+    """Single-history form of :func:`reconstruct_batched`."""
+    return reconstruct_batched([hist], [exact_rows], [exact_pos], [n_total], n_heads, head_dim,
+                               [rope], theta, None if out is None else [out], out_dtype, ws,
+                               stream)[0]
+
+
+def select_workspace_size(L, n_heads, block=8) -> int:
+    return int(_lib.load().iskv_select_workspace_size(L, n_heads, block))
+
+
+def select_prompt_blocks(keys, block=8, per_head=128, suffix_blocks=4, v_radius=32, ws=None,
+                         stream=None, out=None):
+    """Algorithm 1 steps 2-4 on post-RoPE prompt keys ``(L, H, hd)``. Returns device tensors
+    ``P_K``, ``P_V`` (int32, length L, first ``counts[0]`` / ``counts[1]`` valid), ``head_blocks``
+    (H, per_head) int32 (-1 padded) and ``counts`` (2 + H,) int64."""
+    lib = _lib.load()
+    _need_cuda(keys)
+    if keys.dim() != 3 or not keys.is_contiguous():
+        raise ValueError("keys must be a contiguous (L, H, hd) tensor")
+    L, H, hd = keys.shape
+    dev = keys.device
+    if out is None:
+        out = {"P_K": torch.empty(L, dtype=torch.int32, device=dev),
+               "P_V": torch.empty(L, dtype=torch.int32, device=dev),
+               "head_blocks": torch.empty(H, max(per_head, 1), dtype=torch.int32, device=dev),
+               "counts": torch.zeros(2 + H, dtype=torch.int64, device=dev)}
+    need = lib.iskv_select_workspace_size(L, H, block)
+    w = ws if ws is not None else _ws(dev, need)
+    _lib.check(lib.iskv_select_prompt_blocks(
+        keys.data_ptr(), _dt(keys), L, H, hd, block, per_head, suffix_blocks, v_radius,
+        out["P_K"].data_ptr(), out["P_V"].data_ptr(), out["head_blocks"].data_ptr(),
+        out["counts"].data_ptr(), w.data_ptr(), w.numel(), _stream(stream)), "select_prompt_blocks")
+    return out

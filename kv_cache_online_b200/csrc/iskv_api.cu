@@ -1,0 +1,415 @@
+// C ABI of libiskv: argument validation on the host, workspace carving and the launch sequence of
+// each entry point. Every numerical step runs in the kernels of the other translation units.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "iskv.h"
+#include "kernels.h"
+#include "recon.h"
+#include "reorth.h"
+#include "select.h"
+
+using namespace iskv;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+iskv_status fail(iskv_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+iskv_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(ISKV_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_dtype(int32_t t) { return t == ISKV_F32 || t == ISKV_BF16; }
+
+iskv_status check_handle(const iskv_lowrank *h, const char *who) {
+  if (!h) return fail(ISKV_ERR_ARG, "%s: null history handle", who);
+  if (!h->U || !h->sigma || !h->B || !h->pos || !h->meta)
+    return fail(ISKV_ERR_ARG, "%s: null pointer in history handle", who);
+  if (!aligned(h->U, 16) || !aligned(h->sigma, 16) || !aligned(h->B, 16) || !aligned(h->pos, 16) ||
+      !aligned(h->meta, 16))
+    return fail(ISKV_ERR_ARG, "%s: history pointers must be 16-byte aligned", who);
+  if (!valid_dtype(h->storage)) return fail(ISKV_ERR_ARG, "%s: bad storage dtype", who);
+  if (h->d <= 0 || h->d % 16 || h->r_max < 16 || h->r_max % 16 || h->r_max > 512 ||
+      h->r_max > h->d)
+    return fail(ISKV_ERR_SHAPE, "%s: need d %% 16 == 0, r_max %% 16 == 0, 16 <= r_max <= "
+                "min(d, 512) (got d=%d r_max=%d)", who, h->d, h->r_max);
+  if (h->n_cap < 0 || h->n_cap >= (int64_t)1 << 31)
+    return fail(ISKV_ERR_SHAPE, "%s: n_cap out of range", who);
+  return ISKV_OK;
+}
+
+iskv_status check_ws(const void *ws, size_t have, size_t need, const char *who) {
+  if (need == 0) return ISKV_OK;
+  if (!ws) return fail(ISKV_ERR_WORKSPACE, "%s: null workspace", who);
+  if (!aligned(ws, 256)) return fail(ISKV_ERR_WORKSPACE, "%s: workspace must be 256-byte aligned", who);
+  if (have < need)
+    return fail(ISKV_ERR_WORKSPACE, "%s: workspace too small (%zu < %zu bytes)", who, have, need);
+  return ISKV_OK;
+}
+
+size_t jobs_bytes(int32_t count, size_t each) { return align_up((size_t)count * each, 256); }
+
+}  // namespace
+
+extern "C" {
+
+int32_t iskv_abi_version(void) { return ISKV_ABI_VERSION; }
+
+const char *iskv_status_string(int32_t st) {
+  switch (st) {
+    case ISKV_OK: return "ok";
+    case ISKV_ERR_ARG: return "invalid argument";
+    case ISKV_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case ISKV_ERR_CUDA: return "CUDA error";
+    case ISKV_ERR_CAPACITY: return "history capacity exceeded";
+    case ISKV_ERR_NONFINITE: return "non-finite singular value";
+    case ISKV_ERR_NOT_CONVERGED: return "iteration did not converge";
+    case ISKV_ERR_TIMEOUT: return "bounded wait timed out";
+    case ISKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+  }
+}
+
+const char *iskv_last_error(void) { return g_last_error.c_str(); }
+
+// ------------------------------------------------------------------------------------------------
+// Fold
+size_t iskv_fold_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t b) {
+  if (count < 1 || d < 1 || r_max < 1 || b < 1) return 0;
+  const FoldWsLayout L = fold_ws_layout(d, r_max, b);
+  return jobs_bytes(count, sizeof(FoldJob)) + (size_t)count * L.total;
+}
+
+iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const void *const *F,
+                                    int32_t f_dtype, int32_t b, const int32_t *const *f_pos,
+                                    float tau_rel, void *ws, size_t ws_bytes, void *stream) {
+  const char *who = "iskv_fold_block";
+  g_last_error.clear();
+  if (!hs || !F || !f_pos) return fail(ISKV_ERR_ARG, "%s: null host array", who);
+  if (count < 1 || count > 4096) return fail(ISKV_ERR_SHAPE, "%s: count must be in [1, 4096]", who);
+  if (!valid_dtype(f_dtype)) return fail(ISKV_ERR_ARG, "%s: bad F dtype", who);
+  if (!(tau_rel >= 0.f)) return fail(ISKV_ERR_ARG, "%s: tau_rel must be >= 0", who);
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_status st = check_handle(&hs[i], who);
+    if (st != ISKV_OK) return st;
+    if (hs[i].d != hs[0].d || hs[i].r_max != hs[0].r_max || hs[i].storage != hs[0].storage)
+      return fail(ISKV_ERR_SHAPE, "%s: batched histories must share d, r_max, storage", who);
+    if (!F[i] || !f_pos[i]) return fail(ISKV_ERR_ARG, "%s: null F or f_pos", who);
+    if (!aligned(F[i], 16) || !aligned(f_pos[i], 4))
+      return fail(ISKV_ERR_ARG, "%s: F must be 16-byte aligned", who);
+  }
+  const int d = hs[0].d, r = hs[0].r_max;
+  if (b < 8 || b % 8 || b > 128 || b > d)
+    return fail(ISKV_ERR_SHAPE, "%s: need 8 <= b <= min(d, 128), b %% 8 == 0 (got %d)", who, b);
+  if (fold_residual_smem(d, b) > 200 * 1024)
+    return fail(ISKV_ERR_SHAPE, "%s: d = %d with b = %d exceeds the residual QR cluster", who, d, b);
+  {
+    const JacobiCfg jc = jacobi_cfg(r + b, r + 2 * b);
+    if (jc.smem > 200 * 1024 || 32 * jc.w > 640)
+      return fail(ISKV_ERR_SHAPE, "%s: r_max + b too large for the core SVD cluster", who);
+  }
+  const size_t need = iskv_fold_workspace_size(count, d, r, b);
+  iskv_status st = check_ws(ws, ws_bytes, need, who);
+  if (st != ISKV_OK) return st;
+
+  FoldParams p;
+  p.d = d;
+  p.r = r;
+  p.b = b;
+  p.f_dtype = f_dtype;
+  p.storage = hs[0].storage;
+  p.count = count;
+  p.tau_rel = tau_rel;
+  p.ws = fold_ws_layout(d, r, b);
+  char *base = static_cast<char *>(ws);
+  const size_t jb = jobs_bytes(count, sizeof(FoldJob));
+  std::vector<FoldJob> jobs(count);
+  int64_t ncap_max = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    FoldJob &j = jobs[i];
+    j.h.U = hs[i].U;
+    j.h.sigma = hs[i].sigma;
+    j.h.B = hs[i].B;
+    j.h.pos = hs[i].pos;
+    j.h.meta = hs[i].meta;
+    j.h.ws = base + jb + (size_t)i * p.ws.total;
+    j.F = F[i];
+    j.f_pos = f_pos[i];
+    j.n_cap = hs[i].n_cap;
+    j.pad_ = 0;
+    if (hs[i].n_cap > ncap_max) ncap_max = hs[i].n_cap;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FoldJob *djobs = reinterpret_cast<FoldJob *>(base);
+  cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(FoldJob) * count, s);
+  if (e != cudaSuccess) return cuda_fail(e, "fold: upload");
+  if ((e = launch_fold_prepare(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: prepare");
+  if ((e = launch_fold_project(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: project");
+  if ((e = launch_fold_residual(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: residual");
+  const char *cj = reinterpret_cast<const char *>(djobs);
+  if ((e = launch_core(cj, fold_core_params(p), s)) != cudaSuccess)
+    return cuda_fail(e, "fold: core svd");
+  const RotParams rp = fold_rot_params(p);
+  if ((e = launch_rotate_basis(cj, rp, s)) != cudaSuccess)
+    return cuda_fail(e, "fold: basis rotation");
+  if ((e = launch_rotate_coords(cj, rp, ncap_max, s)) != cudaSuccess)
+    return cuda_fail(e, "fold: coordinate rotation");
+  if ((e = launch_fold_finalize(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: finalize");
+  return ISKV_OK;
+}
+
+iskv_status iskv_fold_block(const iskv_lowrank *h, const void *F, int32_t f_dtype, int32_t b,
+                            const int32_t *f_pos, float tau_rel, void *ws, size_t ws_bytes,
+                            void *stream) {
+  const void *Fs[1] = {F};
+  const int32_t *ps[1] = {f_pos};
+  if (!h) return fail(ISKV_ERR_ARG, "iskv_fold_block: null history handle");
+  return iskv_fold_block_batched(h, 1, Fs, f_dtype, b, ps, tau_rel, ws, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Re-orthogonalisation
+size_t iskv_reorth_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap) {
+  if (count < 1 || d < 1 || r_max < 1 || n_cap < 0) return 0;
+  const ReorthWsLayout L = reorth_ws_layout(d, r_max, n_cap);
+  return jobs_bytes(count, sizeof(ReorthJob)) + (size_t)count * L.total;
+}
+
+iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t ws_bytes,
+                        void *stream) {
+  const char *who = "iskv_reorth";
+  g_last_error.clear();
+  if (!hs) return fail(ISKV_ERR_ARG, "%s: null host array", who);
+  if (count < 1 || count > 4096) return fail(ISKV_ERR_SHAPE, "%s: count must be in [1, 4096]", who);
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_status st = check_handle(&hs[i], who);
+    if (st != ISKV_OK) return st;
+    if (hs[i].d != hs[0].d || hs[i].r_max != hs[0].r_max || hs[i].storage != hs[0].storage ||
+        hs[i].n_cap != hs[0].n_cap)
+      return fail(ISKV_ERR_SHAPE, "%s: batched histories must share d, r_max, storage, n_cap", who);
+  }
+  const int d = hs[0].d, r = hs[0].r_max;
+  const int64_t ncap = hs[0].n_cap;
+  const size_t need = iskv_reorth_workspace_size(count, d, r, ncap);
+  iskv_status st = check_ws(ws, ws_bytes, need, who);
+  if (st != ISKV_OK) return st;
+  ReorthParams p;
+  p.d = d;
+  p.r = r;
+  p.storage = hs[0].storage;
+  p.count = count;
+  p.n_cap = ncap;
+  p.ws = reorth_ws_layout(d, r, ncap);
+  char *base = static_cast<char *>(ws);
+  const size_t jb = jobs_bytes(count, sizeof(ReorthJob));
+  std::vector<ReorthJob> jobs(count);
+  for (int32_t i = 0; i < count; ++i) {
+    ReorthJob &j = jobs[i];
+    j.h.U = hs[i].U;
+    j.h.sigma = hs[i].sigma;
+    j.h.B = hs[i].B;
+    j.h.pos = hs[i].pos;
+    j.h.meta = hs[i].meta;
+    j.h.ws = base + jb + (size_t)i * p.ws.total;
+    j.n_cap = hs[i].n_cap;
+    j.pad_ = 0;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ReorthJob *djobs = reinterpret_cast<ReorthJob *>(base);
+  cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReorthJob) * count, s);
+  if (e != cudaSuccess) return cuda_fail(e, "reorth: upload");
+  if ((e = launch_reorth(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "reorth");
+  return ISKV_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Reconstruction
+size_t iskv_reconstruct_workspace_size(int32_t count, int32_t d, int32_t r_max) {
+  if (count < 1 || d < 1 || r_max < 1) return 0;
+  return jobs_bytes(count, sizeof(ReconJob)) + (size_t)count * align_up((size_t)d * r_max * 2, 256);
+}
+
+iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
+                                     const void *const *exact_rows, int32_t exact_dtype,
+                                     const int32_t *const *exact_pos, const int64_t *n_exact,
+                                     const int64_t *n_total, int32_t n_heads, int32_t head_dim,
+                                     const int32_t *apply_rope, double rope_theta,
+                                     void *const *out, int32_t out_dtype, void *ws,
+                                     size_t ws_bytes, void *stream) {
+  const char *who = "iskv_reconstruct";
+  g_last_error.clear();
+  if (!hs || !exact_rows || !exact_pos || !n_exact || !n_total || !apply_rope || !out)
+    return fail(ISKV_ERR_ARG, "%s: null host array", who);
+  if (count < 1 || count > 4096) return fail(ISKV_ERR_SHAPE, "%s: count must be in [1, 4096]", who);
+  if (!valid_dtype(exact_dtype) || !valid_dtype(out_dtype))
+    return fail(ISKV_ERR_ARG, "%s: bad dtype", who);
+  if (n_heads < 1 || head_dim < 2 || head_dim % 2 || head_dim > 256)
+    return fail(ISKV_ERR_SHAPE, "%s: need even head_dim <= 256", who);
+  if (!(rope_theta > 0.0)) return fail(ISKV_ERR_ARG, "%s: rope_theta must be > 0", who);
+  int64_t max_exact = 0, ncap_max = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_status st = check_handle(&hs[i], who);
+    if (st != ISKV_OK) return st;
+    if (hs[i].d != hs[0].d || hs[i].r_max != hs[0].r_max || hs[i].storage != hs[0].storage)
+      return fail(ISKV_ERR_SHAPE, "%s: batched histories must share d, r_max, storage", who);
+    if (hs[i].d != n_heads * head_dim)
+      return fail(ISKV_ERR_SHAPE, "%s: d must equal n_heads * head_dim", who);
+    if (!out[i]) return fail(ISKV_ERR_ARG, "%s: null output", who);
+    if (n_exact[i] < 0 || n_total[i] < 0) return fail(ISKV_ERR_SHAPE, "%s: negative size", who);
+    if (n_exact[i] > 0 && (!exact_rows[i] || !exact_pos[i]))
+      return fail(ISKV_ERR_ARG, "%s: null exact rows", who);
+    if (n_exact[i] > max_exact) max_exact = n_exact[i];
+    if (hs[i].n_cap > ncap_max) ncap_max = hs[i].n_cap;
+  }
+  const int d = hs[0].d, r = hs[0].r_max;
+  const size_t need = iskv_reconstruct_workspace_size(count, d, r);
+  iskv_status st = check_ws(ws, ws_bytes, need, who);
+  if (st != ISKV_OK) return st;
+  ReconParams p;
+  p.d = d;
+  p.r = r;
+  p.storage = hs[0].storage;
+  p.exact_dtype = exact_dtype;
+  p.out_dtype = out_dtype;
+  p.n_heads = n_heads;
+  p.head_dim = head_dim;
+  p.count = count;
+  p.theta = rope_theta;
+  p.n_cap_max = ncap_max;
+  char *base = static_cast<char *>(ws);
+  const size_t jb = jobs_bytes(count, sizeof(ReconJob));
+  std::vector<ReconJob> jobs(count);
+  for (int32_t i = 0; i < count; ++i) {
+    ReconJob &j = jobs[i];
+    j.U = hs[i].U;
+    j.sigma = hs[i].sigma;
+    j.B = hs[i].B;
+    j.pos = hs[i].pos;
+    j.meta = hs[i].meta;
+    j.exact_rows = exact_rows[i];
+    j.exact_pos = exact_pos[i];
+    j.out = out[i];
+    j.bsig = base + jb + (size_t)i * align_up((size_t)d * r * 2, 256);
+    j.n_exact = n_exact[i];
+    j.n_total = n_total[i];
+    j.apply_rope = apply_rope[i];
+    j.pad_ = 0;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ReconJob *djobs = reinterpret_cast<ReconJob *>(base);
+  cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReconJob) * count, s);
+  if (e != cudaSuccess) return cuda_fail(e, "reconstruct: upload");
+  if ((e = launch_recon_compressed(djobs, p, s)) != cudaSuccess)
+    return cuda_fail(e, "reconstruct: compressed rows");
+  if ((e = launch_recon_exact(djobs, p, max_exact, s)) != cudaSuccess)
+    return cuda_fail(e, "reconstruct: exact rows");
+  return ISKV_OK;
+}
+
+iskv_status iskv_reconstruct(const iskv_lowrank *h, const void *exact_rows, int32_t exact_dtype,
+                             const int32_t *exact_pos, int64_t n_exact, int64_t n_total,
+                             int32_t n_heads, int32_t head_dim, int32_t apply_rope,
+                             double rope_theta, void *out, int32_t out_dtype, void *ws,
+                             size_t ws_bytes, void *stream) {
+  if (!h) return fail(ISKV_ERR_ARG, "iskv_reconstruct: null history handle");
+  const void *er[1] = {exact_rows};
+  const int32_t *ep[1] = {exact_pos};
+  const int64_t ne[1] = {n_exact};
+  const int64_t nt[1] = {n_total};
+  const int32_t ar[1] = {apply_rope};
+  void *o[1] = {out};
+  return iskv_reconstruct_batched(h, 1, er, exact_dtype, ep, ne, nt, n_heads, head_dim, ar,
+                                  rope_theta, o, out_dtype, ws, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Prompt-block selection
+size_t iskv_select_workspace_size(int64_t L, int32_t n_heads, int32_t block) {
+  if (L < 1 || n_heads < 1 || block < 1) return 0;
+  return select_ws_layout(L, n_heads, block).total;
+}
+
+iskv_status iskv_select_prompt_blocks(const void *keys, int32_t k_dtype, int64_t L,
+                                      int32_t n_heads, int32_t head_dim, int32_t block,
+                                      int32_t per_head, int32_t suffix_blocks, int32_t v_radius,
+                                      int32_t *pk_out, int32_t *pv_out, int32_t *head_blocks_out,
+                                      int64_t *counts_out, void *ws, size_t ws_bytes,
+                                      void *stream) {
+  const char *who = "iskv_select_prompt_blocks";
+  g_last_error.clear();
+  if (!keys || !pk_out || !pv_out || !head_blocks_out || !counts_out)
+    return fail(ISKV_ERR_ARG, "%s: null pointer", who);
+  if (!valid_dtype(k_dtype)) return fail(ISKV_ERR_ARG, "%s: bad key dtype", who);
+  if (L < 1 || L > ((int64_t)1 << 24)) return fail(ISKV_ERR_SHAPE, "%s: need 1 <= L <= 2^24", who);
+  if (n_heads < 1 || n_heads > 64 || head_dim < 2 || head_dim > 256 || head_dim % 2)
+    return fail(ISKV_ERR_SHAPE, "%s: need n_heads <= 64, even head_dim <= 256", who);
+  if (block < 1 || block > 64 || per_head < 0 || per_head > 4096 || suffix_blocks < 0 ||
+      v_radius < 0)
+    return fail(ISKV_ERR_SHAPE, "%s: bad block / per_head / suffix / radius", who);
+  const size_t need = iskv_select_workspace_size(L, n_heads, block);
+  iskv_status st = check_ws(ws, ws_bytes, need, who);
+  if (st != ISKV_OK) return st;
+  SelectArgs a;
+  a.keys = keys;
+  a.k_dtype = k_dtype;
+  a.L = L;
+  a.H = n_heads;
+  a.hd = head_dim;
+  a.block = block;
+  a.per_head = per_head;
+  a.suffix_blocks = suffix_blocks;
+  a.v_radius = v_radius;
+  a.pk_out = pk_out;
+  a.pv_out = pv_out;
+  a.head_blocks = head_blocks_out;
+  a.counts = counts_out;
+  a.ws = ws;
+  cudaError_t e = launch_select(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select");
+  return ISKV_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+iskv_status iskv_reset(const iskv_lowrank *h, void *stream) {
+  g_last_error.clear();
+  iskv_status st = check_handle(h, "iskv_reset");
+  if (st != ISKV_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(h->meta, 0, 4 * sizeof(int64_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->sigma, 0, sizeof(float) * h->r_max, s);
+  if (e != cudaSuccess) return cuda_fail(e, "iskv_reset");
+  return ISKV_OK;
+}
+
+iskv_status iskv_get_status(const iskv_lowrank *h, int64_t *k, int64_t *n, int64_t *folds,
+                            int64_t *status_bits) {
+  g_last_error.clear();
+  iskv_status st = check_handle(h, "iskv_get_status");
+  if (st != ISKV_OK) return st;
+  int64_t m[4];
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(m, h->meta, sizeof m, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "iskv_get_status");
+  if (k) *k = m[ISKV_META_K];
+  if (n) *n = m[ISKV_META_N];
+  if (folds) *folds = m[ISKV_META_FOLDS];
+  if (status_bits) *status_bits = m[ISKV_META_STATUS];
+  return ISKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,168 @@
+// Per-step reconstruction (iS-KV reading notes, Algorithm 3 steps 7-8): compressed row i of a
+// history is (U[i] * sigma) B^T, written to its original position pos[i]; exact rows are copied to
+// their own positions; keys are rotated by their own position with rotate-half RoPE.
+//
+// RoPE angles: pos * theta^(-2j/hd) reaches tens of thousands of radians, where one float32 ulp is
+// ~4e-3 rad. The angle is therefore formed and reduced modulo 2 pi in float64 and only the reduced
+// angle (|a| <= pi) goes to sincosf.
+#include "recon.h"
+
+namespace iskv {
+
+ISKV_DEV double rope_inv_freq(int j, int hd, double log_theta) {
+  return exp(-2.0 * (double)j / (double)hd * log_theta);
+}
+
+ISKV_DEV void rope_sincos(int64_t pos, double inv_freq, float &c, float &s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  double a = (double)pos * inv_freq;
+  a -= two_pi * rint(a / two_pi);
+  sincosf((float)a, &s, &c);
+}
+
+// ------------------------------------------------------------------------------------------------
+// CUDA-core path (float32 storage, and any storage when the tensor-core path is not selected).
+// Tile: 32 rows x one head; thread = (row, pair group); each thread owns pairs (c, c + hd/2).
+constexpr int RRM = 32, RBK = 16;
+
+template <typename TS, typename TO>
+__global__ void __launch_bounds__(256) k_recon_ffma(const ReconJob *jobs, ReconParams p) {
+  const ReconJob &jb = jobs[blockIdx.z];
+  const int64_t n = jb.meta[ISKV_META_N];
+  const int k = (int)jb.meta[ISKV_META_K];
+  const int i0 = blockIdx.x * RRM;
+  if (i0 >= n) return;
+  const int h = blockIdx.y, hd = p.head_dim, half = hd / 2, r = p.r, d = p.d;
+  __shared__ float Us[RBK][RRM + 1];
+  __shared__ float Bs[RBK][256 + 1];
+  __shared__ double invf[128];
+  const int tid = threadIdx.x;
+  if (jb.apply_rope)
+    for (int j = tid; j < half; j += 256) invf[j] = rope_inv_freq(j, hd, log(p.theta));
+  __syncthreads();
+  const TS *U = static_cast<const TS *>(jb.U);
+  const TS *B = static_cast<const TS *>(jb.B);
+  const float *sg = jb.sigma;
+  const int row = tid / 8, g = tid % 8;
+  constexpr int HPMAX = 16;  // pairs per thread for head_dim <= 256
+  float lo[HPMAX], hi[HPMAX];
+#pragma unroll
+  for (int u = 0; u < HPMAX; ++u) lo[u] = hi[u] = 0.f;
+  for (int l0 = 0; l0 < k; l0 += RBK) {
+    for (int e = tid; e < RRM * RBK; e += 256) {
+      const int i = e / RBK, ll = e % RBK;
+      Us[ll][i] = (i0 + i < n && l0 + ll < k) ? to_f<TS>(U[(size_t)(i0 + i) * r + l0 + ll]) : 0.f;
+    }
+    for (int e = tid; e < hd * RBK; e += 256) {
+      const int c = e / RBK, ll = e % RBK;
+      const int l = l0 + ll;
+      Bs[ll][c] = l < k ? sg[l] * to_f<TS>(B[(size_t)(h * hd + c) * r + l]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int ll = 0; ll < RBK; ++ll) {
+      const float a = Us[ll][row];
+#pragma unroll
+      for (int u = 0; u < HPMAX; ++u) {
+        const int c = g + 8 * u;
+        if (c < half) {
+          lo[u] = fmaf(a, Bs[ll][c], lo[u]);
+          hi[u] = fmaf(a, Bs[ll][c + half], hi[u]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const int64_t gi = i0 + row;
+  if (gi >= n) return;
+  const int64_t ps = jb.pos[gi];
+  if (ps < 0 || ps >= jb.n_total) {  // a position outside the output: skip and flag
+    if (g == 0) record_status(jb.meta, ISKV_ERR_SHAPE);
+    return;
+  }
+  TO *out = static_cast<TO *>(jb.out) + (size_t)ps * d + (size_t)h * hd;
+#pragma unroll
+  for (int u = 0; u < HPMAX; ++u) {
+    const int c = g + 8 * u;
+    if (c >= half) continue;
+    float x1 = lo[u], x2 = hi[u];
+    if (jb.apply_rope) {
+      float cs, sn;
+      rope_sincos(ps, invf[c], cs, sn);
+      const float y1 = x1 * cs - x2 * sn, y2 = x2 * cs + x1 * sn;
+      x1 = y1;
+      x2 = y2;
+    }
+    out[c] = from_f<TO>(x1);
+    out[c + half] = from_f<TO>(x2);
+  }
+}
+
+// Exact rows: copy (and rotate) exact_rows[e] to out[exact_pos[e]].
+template <typename TE, typename TO>
+__global__ void k_recon_exact(const ReconJob *jobs, ReconParams p) {
+  const ReconJob &jb = jobs[blockIdx.y];
+  const int hd = p.head_dim, half = hd / 2, d = p.d, H = p.n_heads;
+  const int64_t npairs = jb.n_exact * (int64_t)H * half;
+  const double lt = log(p.theta);
+  const TE *X = static_cast<const TE *>(jb.exact_rows);
+  TO *out = static_cast<TO *>(jb.out);
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < npairs;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = t / (H * half);
+    const int rem = (int)(t % (H * half));
+    const int h = rem / half, c = rem % half;
+    const int64_t ps = jb.exact_pos[e];
+    if (ps < 0 || ps >= jb.n_total) {
+      record_status(jb.meta, ISKV_ERR_SHAPE);
+      continue;
+    }
+    float x1 = to_f<TE>(X[(size_t)e * d + h * hd + c]);
+    float x2 = to_f<TE>(X[(size_t)e * d + h * hd + c + half]);
+    if (jb.apply_rope) {
+      float cs, sn;
+      rope_sincos(ps, rope_inv_freq(c, hd, lt), cs, sn);
+      const float y1 = x1 * cs - x2 * sn, y2 = x2 * cs + x1 * sn;
+      x1 = y1;
+      x2 = y2;
+    }
+    out[(size_t)ps * d + h * hd + c] = from_f<TO>(x1);
+    out[(size_t)ps * d + h * hd + c + half] = from_f<TO>(x2);
+  }
+}
+
+template <typename TS, typename TO>
+static cudaError_t recon_ffma_t(const ReconJob *jobs, const ReconParams &p, cudaStream_t s) {
+  const dim3 g((unsigned)((p.n_cap_max + RRM - 1) / RRM), p.n_heads, p.count);
+  k_recon_ffma<TS, TO><<<g, 256, 0, s>>>(jobs, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_recon_compressed_ffma(const ReconJob *jobs, const ReconParams &p,
+                                         cudaStream_t s) {
+  const bool sb = p.storage == ISKV_BF16, ob = p.out_dtype == ISKV_BF16;
+  if (sb && ob) return recon_ffma_t<__nv_bfloat16, __nv_bfloat16>(jobs, p, s);
+  if (sb) return recon_ffma_t<__nv_bfloat16, float>(jobs, p, s);
+  if (ob) return recon_ffma_t<float, __nv_bfloat16>(jobs, p, s);
+  return recon_ffma_t<float, float>(jobs, p, s);
+}
+
+cudaError_t launch_recon_compressed(const ReconJob *jobs, const ReconParams &p, cudaStream_t s) {
+  return launch_recon_compressed_ffma(jobs, p, s);
+}
+
+cudaError_t launch_recon_exact(const ReconJob *jobs, const ReconParams &p, int64_t max_exact,
+                               cudaStream_t s) {
+  if (max_exact <= 0) return cudaSuccess;
+  const int64_t work = max_exact * (int64_t)p.n_heads * (p.head_dim / 2);
+  const unsigned gx = (unsigned)((work + 255) / 256 < 4096 ? (work + 255) / 256 : 4096);
+  const dim3 g(gx, p.count);
+  const bool eb = p.exact_dtype == ISKV_BF16, ob = p.out_dtype == ISKV_BF16;
+  if (eb && ob) k_recon_exact<__nv_bfloat16, __nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
+  else if (eb) k_recon_exact<__nv_bfloat16, float><<<g, 256, 0, s>>>(jobs, p);
+  else if (ob) k_recon_exact<float, __nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
+  else k_recon_exact<float, float><<<g, 256, 0, s>>>(jobs, p);
+  return cudaGetLastError();
+}
+
+}  // namespace iskv

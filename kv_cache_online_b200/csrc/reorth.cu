@@ -1,0 +1,313 @@
+// Re-orthogonalisation (iS-KV reading notes, Section 4.4).
+//
+// The pages take thin QR factorisations U = Q_U R_U, B = Q_B R_B, decompose
+// R_U diag(sigma) R_B^T = X diag(sigma') Y^T and set U <- Q_U X, sigma <- sigma', B <- Q_B Y.
+// Any factorisation with an orthonormal Q gives the same product and the same sigma', and the new
+// U, B are the singular vectors of the product. Here R is the symmetric square root of the Gram
+// matrix (the polar factor): R_U = (U^T U)^(1/2), Q_U = U R_U^(-1). Both roots come from the
+// coupled Newton-Schulz iteration (Higham 1997), which is GEMM-only and converges quadratically
+// for the near-orthonormal factors seen here:
+//   Y_0 = A / c, Z_0 = I;  T = (3I - Z Y) / 2;  Y <- Y T;  Z <- T Z   ->  Y = (A/c)^(1/2),
+//   Z = (A/c)^(-1/2), with c = trace(A) / k.
+// Then M = R_U diag(sigma) R_B goes through the cluster Jacobi SVD (dense mode), and the two
+// rotations U <- U (R_U^-1 X), B <- B (R_B^-1 Y) reuse the fold's rotation kernels.
+#include "gemm_tile.cuh"
+#include "reorth.h"
+
+namespace iskv {
+
+enum { RS_CU = 8, RS_CB = 9 };  // scalar slots holding the Newton-Schulz scales (float bits)
+
+ReorthWsLayout reorth_ws_layout(int d, int r, int64_t n_cap) {
+  ReorthWsLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  const size_t rr = sizeof(float) * (size_t)r * r;
+  L.nsplit_u = (int)((n_cap + REORTH_SPLIT - 1) / REORTH_SPLIT);
+  if (L.nsplit_u < 1) L.nsplit_u = 1;
+  L.nsplit_b = (d + REORTH_SPLIT - 1) / REORTH_SPLIT;
+  L.scal = take(FS_COUNT * sizeof(int32_t));
+  L.gpart_u = take(rr * L.nsplit_u);
+  L.gpart_b = take(rr * L.nsplit_b);
+  for (int w = 0; w < 2; ++w) {
+    L.G[w] = take(rr);
+    L.Y[w] = take(rr);
+    L.Z[w] = take(rr);
+    L.T[w] = take(rr);
+    L.Y2[w] = take(rr);
+    L.Z2[w] = take(rr);
+  }
+  L.M = take(rr);
+  L.Gt = take(rr);
+  L.Gtb = take(sizeof(__nv_bfloat16) * (size_t)r * r);
+  L.Ht = take(rr);
+  L.sig = take(sizeof(float) * r);
+  L.TUt = take(rr);
+  L.TUtb = take(sizeof(__nv_bfloat16) * (size_t)r * r);
+  L.TBt = take(rr);
+  L.Bn = take(sizeof(float) * (size_t)d * r);
+  L.total = o;
+  return L;
+}
+
+__global__ void k_reorth_prepare(const ReorthJob *jobs, ReorthParams p) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= p.count) return;
+  const ReorthJob &jb = jobs[j];
+  int32_t *sc = reinterpret_cast<int32_t *>(jb.h.ws);
+  const int64_t k = jb.h.meta[ISKV_META_K], n = jb.h.meta[ISKV_META_N];
+  sc[FS_K_OLD] = (int32_t)k;
+  sc[FS_N_OLD] = (int32_t)n;
+  sc[FS_P] = 0;
+  sc[FS_K_NEW] = (int32_t)k;
+  sc[FS_SKIP] = (k <= 0 || k > p.r || n < 0 || n > jb.n_cap) ? 1 : 0;
+  sc[FS_SWEEPS] = 0;
+}
+
+constexpr int GBM = 32, GBN = 64, GBK = 16, GTM = 2, GTN = 4;
+
+// Gram partial: Gpart[s] = X[rows of split s]^T X[rows of split s] (k x k), X = U (n rows) or B.
+template <typename TS>
+__global__ void __launch_bounds__(256) k_gram_partial(const ReorthJob *jobs, ReorthParams p,
+                                                      int which, int nsplit) {
+  const int job = blockIdx.z / nsplit, s = blockIdx.z % nsplit;
+  const ReorthJob &jb = jobs[job];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], r = p.r;
+  const int rows = which == 0 ? sc[FS_N_OLD] : p.d;
+  const TS *X = static_cast<const TS *>(which == 0 ? jb.h.U : jb.h.B);
+  float *G = reinterpret_cast<float *>(jb.h.ws + (which == 0 ? p.ws.gpart_u : p.ws.gpart_b)) +
+             (size_t)s * r * r;
+  const int r0 = s * REORTH_SPLIT;
+  const int nrows = max(0, min(REORTH_SPLIT, rows - r0));
+  const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
+  if (m0 >= k || n0 >= k) return;
+  tile_gemm<GBM, GBN, GBK, GTM, GTN, false, true>(
+      m0, n0, k, k, nrows,
+      [&](int m, int kk) { return to_f<TS>(X[(size_t)(r0 + kk) * r + m]); },
+      [&](int kk, int n) { return to_f<TS>(X[(size_t)(r0 + kk) * r + n]); },
+      [&](int m, int n, float acc) { G[(size_t)m * r + n] = acc; });
+}
+
+// Sum the partials; then the scale c = trace / k and the Newton-Schulz start Y = G / c, Z = I.
+__global__ void k_gram_reduce(const ReorthJob *jobs, ReorthParams p) {
+  const int job = blockIdx.y >> 1, which = blockIdx.y & 1;
+  const ReorthJob &jb = jobs[job];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], r = p.r;
+  const int ns = which == 0 ? p.ws.nsplit_u : p.ws.nsplit_b;
+  const float *part = reinterpret_cast<const float *>(jb.h.ws + (which == 0 ? p.ws.gpart_u : p.ws.gpart_b));
+  float *G = reinterpret_cast<float *>(jb.h.ws + p.ws.G[which]);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < k * k; e += gridDim.x * blockDim.x) {
+    const int i = e / k, j = e % k;
+    float s = 0.f;
+    for (int q = 0; q < ns; ++q) s += part[(size_t)q * r * r + (size_t)i * r + j];
+    G[(size_t)i * r + j] = s;
+  }
+}
+
+__global__ void k_ns_init(const ReorthJob *jobs, ReorthParams p) {
+  const int job = blockIdx.y >> 1, which = blockIdx.y & 1;
+  const ReorthJob &jb = jobs[job];
+  int32_t *sc = reinterpret_cast<int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], r = p.r;
+  const float *G = reinterpret_cast<const float *>(jb.h.ws + p.ws.G[which]);
+  __shared__ double s_tr;
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < k; ++i) t += G[(size_t)i * r + i];
+    s_tr = t / k;
+    if (blockIdx.x == 0) sc[which == 0 ? RS_CU : RS_CB] = __float_as_int((float)(t / k));
+  }
+  __syncthreads();
+  const float c = (float)s_tr;
+  const float inv = c > 0.f ? 1.f / c : 0.f;
+  float *Y = reinterpret_cast<float *>(jb.h.ws + p.ws.Y[which]);
+  float *Z = reinterpret_cast<float *>(jb.h.ws + p.ws.Z[which]);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < k * k; e += gridDim.x * blockDim.x) {
+    const int i = e / k, j = e % k;
+    Y[(size_t)i * r + j] = G[(size_t)i * r + j] * inv;
+    Z[(size_t)i * r + j] = i == j ? 1.f : 0.f;
+  }
+}
+
+// Newton-Schulz stages. STAGE 0: T = 1.5 I - 0.5 Z Y. STAGE 1: Y2 = Y T (g = 0), Z2 = T Z (g = 1).
+template <int STAGE>
+__global__ void __launch_bounds__(256) k_ns_step(const ReorthJob *jobs, ReorthParams p,
+                                                 size_t y0, size_t z0, size_t y1, size_t z1,
+                                                 size_t yb0, size_t zb0, size_t yb1, size_t zb1) {
+  const int per = STAGE == 0 ? 2 : 4;
+  const int job = blockIdx.z / per, rem = blockIdx.z % per, which = rem & 1, g = rem >> 1;
+  const ReorthJob &jb = jobs[job];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], r = p.r;
+  char *ws = jb.h.ws;
+  const float *Y = reinterpret_cast<const float *>(ws + (which == 0 ? y0 : yb0));
+  const float *Z = reinterpret_cast<const float *>(ws + (which == 0 ? z0 : zb0));
+  float *T = reinterpret_cast<float *>(ws + p.ws.T[which]);
+  const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
+  if (m0 >= k || n0 >= k) return;
+  if (STAGE == 0) {
+    tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
+        m0, n0, k, k, k, [&](int m, int kk) { return Z[(size_t)m * r + kk]; },
+        [&](int kk, int n) { return Y[(size_t)kk * r + n]; },
+        [&](int m, int n, float acc) { T[(size_t)m * r + n] = (m == n ? 1.5f : 0.f) - 0.5f * acc; });
+  } else if (g == 0) {
+    float *Yo = reinterpret_cast<float *>(ws + (which == 0 ? y1 : yb1));
+    tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
+        m0, n0, k, k, k, [&](int m, int kk) { return Y[(size_t)m * r + kk]; },
+        [&](int kk, int n) { return T[(size_t)kk * r + n]; },
+        [&](int m, int n, float acc) { Yo[(size_t)m * r + n] = acc; });
+  } else {
+    float *Zo = reinterpret_cast<float *>(ws + (which == 0 ? z1 : zb1));
+    tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
+        m0, n0, k, k, k, [&](int m, int kk) { return T[(size_t)m * r + kk]; },
+        [&](int kk, int n) { return Z[(size_t)kk * r + n]; },
+        [&](int m, int n, float acc) { Zo[(size_t)m * r + n] = acc; });
+  }
+}
+
+// M = sqrt(c_u c_b) Y_u diag(sigma) Y_b  (= R_U diag(sigma) R_B^T with symmetric R_B).
+__global__ void __launch_bounds__(256) k_reorth_M(const ReorthJob *jobs, ReorthParams p,
+                                                  size_t yu, size_t yb) {
+  const ReorthJob &jb = jobs[blockIdx.z];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], r = p.r;
+  const float scale = sqrtf(__int_as_float(sc[RS_CU]) * __int_as_float(sc[RS_CB]));
+  const float *Yu = reinterpret_cast<const float *>(jb.h.ws + yu);
+  const float *Yb = reinterpret_cast<const float *>(jb.h.ws + yb);
+  const float *sg = jb.h.sigma;
+  float *M = reinterpret_cast<float *>(jb.h.ws + p.ws.M);
+  const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
+  if (m0 >= k || n0 >= k) return;
+  tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
+      m0, n0, k, k, k, [&](int m, int l) { return Yu[(size_t)m * r + l] * sg[l]; },
+      [&](int l, int n) { return Yb[(size_t)l * r + n]; },
+      [&](int m, int n, float acc) { M[(size_t)m * r + n] = scale * acc; });
+}
+
+// Rotations: TUt[q][l] = (Z_u X)[l][q] / sqrt(c_u) with X[j][q] = Gt[q][j];
+//            TBt[q][l] = (Z_b Y)[l][q] / sqrt(c_b) with Y[j][q] = Ht[q][j].
+__global__ void __launch_bounds__(256) k_reorth_T(const ReorthJob *jobs, ReorthParams p, size_t zu,
+                                                  size_t zb) {
+  const int job = blockIdx.z >> 1, which = blockIdx.z & 1;
+  const ReorthJob &jb = jobs[job];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], r = p.r;
+  const float inv = rsqrtf(__int_as_float(sc[which == 0 ? RS_CU : RS_CB]));
+  const float *Z = reinterpret_cast<const float *>(jb.h.ws + (which == 0 ? zu : zb));
+  const float *V = reinterpret_cast<const float *>(jb.h.ws + (which == 0 ? p.ws.Gt : p.ws.Ht));
+  float *out = reinterpret_cast<float *>(jb.h.ws + (which == 0 ? p.ws.TUt : p.ws.TBt));
+  __nv_bfloat16 *outb = reinterpret_cast<__nv_bfloat16 *>(jb.h.ws + p.ws.TUtb);
+  const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
+  if (m0 >= k || n0 >= k) return;
+  tile_gemm<GBM, GBN, GBK, GTM, GTN, true, false>(
+      m0, n0, k, k, k, [&](int l, int j) { return Z[(size_t)l * r + j]; },
+      [&](int j, int q) { return V[(size_t)q * r + j]; },
+      [&](int l, int q, float acc) {
+        const float v = acc * inv;
+        out[(size_t)q * r + l] = v;
+        if (which == 0) outb[(size_t)q * r + l] = __float2bfloat16_rn(v);
+      });
+}
+
+template <typename TS>
+__global__ void k_reorth_finalize(const ReorthJob *jobs, ReorthParams p) {
+  const ReorthJob &jb = jobs[blockIdx.y];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], r = p.r, d = p.d;
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x, nth = gridDim.x * blockDim.x;
+  TS *B = static_cast<TS *>(jb.h.B);
+  const float *Bn = reinterpret_cast<const float *>(jb.h.ws + p.ws.Bn);
+  const float *sig = reinterpret_cast<const float *>(jb.h.ws + p.ws.sig);
+  for (int e = tid; e < d * r; e += nth) {
+    const int q = e % r;
+    B[e] = from_f<TS>(q < k ? Bn[e] : 0.f);
+  }
+  for (int e = tid; e < r; e += nth) jb.h.sigma[e] = e < k ? sig[e] : 0.f;
+  if (tid == 0) jb.h.meta[ISKV_META_FOLDS] = 0;
+}
+
+cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s) {
+  const int r = p.r;
+  const ReorthWsLayout &W = p.ws;
+  k_reorth_prepare<<<(p.count + 127) / 128, 128, 0, s>>>(jobs, p);
+  const unsigned tn = (r + GBN - 1) / GBN, tm = (r + GBM - 1) / GBM;
+  if (p.storage == ISKV_BF16) {
+    k_gram_partial<__nv_bfloat16><<<dim3(tn, tm, p.count * W.nsplit_u), 256, 0, s>>>(jobs, p, 0, W.nsplit_u);
+    k_gram_partial<__nv_bfloat16><<<dim3(tn, tm, p.count * W.nsplit_b), 256, 0, s>>>(jobs, p, 1, W.nsplit_b);
+  } else {
+    k_gram_partial<float><<<dim3(tn, tm, p.count * W.nsplit_u), 256, 0, s>>>(jobs, p, 0, W.nsplit_u);
+    k_gram_partial<float><<<dim3(tn, tm, p.count * W.nsplit_b), 256, 0, s>>>(jobs, p, 1, W.nsplit_b);
+  }
+  k_gram_reduce<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
+  k_ns_init<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
+  size_t y0[2] = {W.Y[0], W.Y[1]}, z0[2] = {W.Z[0], W.Z[1]};
+  size_t y1[2] = {W.Y2[0], W.Y2[1]}, z1[2] = {W.Z2[0], W.Z2[1]};
+  for (int it = 0; it < NS_ITERS; ++it) {
+    k_ns_step<0><<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p, y0[0], z0[0], y1[0], z1[0],
+                                                         y0[1], z0[1], y1[1], z1[1]);
+    k_ns_step<1><<<dim3(tn, tm, p.count * 4), 256, 0, s>>>(jobs, p, y0[0], z0[0], y1[0], z1[0],
+                                                         y0[1], z0[1], y1[1], z1[1]);
+    for (int w = 0; w < 2; ++w) {
+      size_t t = y0[w]; y0[w] = y1[w]; y1[w] = t;
+      t = z0[w]; z0[w] = z1[w]; z1[w] = t;
+    }
+  }
+  k_reorth_M<<<dim3(tn, tm, p.count), 256, 0, s>>>(jobs, p, y0[0], y0[1]);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  CoreParams c;
+  c.r = r;
+  c.b = 0;
+  c.count = p.count;
+  c.job_stride = sizeof(ReorthJob);
+  c.mode = 1;
+  c.C = 0;
+  c.FP = 0;
+  c.M = W.M;
+  c.Gt = W.Gt;
+  c.Gtb = W.Gtb;
+  c.Gbot = W.Gt;  // unused in dense mode (b = 0)
+  c.Ht = W.Ht;
+  c.sig = W.sig;
+  c.hs = r;
+  c.ldm = r;
+  c.max_sweeps = 40;
+  e = launch_core(reinterpret_cast<const char *>(jobs), c, s);
+  if (e != cudaSuccess) return e;
+  k_reorth_T<<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p, z0[0], z0[1]);
+
+  RotParams q;
+  q.d = p.d;
+  q.r = r;
+  q.storage = p.storage;
+  q.count = p.count;
+  q.job_stride = sizeof(ReorthJob);
+  q.gt = W.TUt;
+  q.gtb = W.TUtb;
+  q.ht = W.TBt;
+  q.pmat = W.TBt;  // unused: p = 0
+  q.bn = W.Bn;
+  q.hs = r;
+  q.pld = 1;
+  e = launch_rotate_coords(reinterpret_cast<const char *>(jobs), q, p.n_cap, s);
+  if (e != cudaSuccess) return e;
+  e = launch_rotate_basis(reinterpret_cast<const char *>(jobs), q, s);
+  if (e != cudaSuccess) return e;
+  if (p.storage == ISKV_BF16)
+    k_reorth_finalize<__nv_bfloat16><<<dim3(32, p.count), 256, 0, s>>>(jobs, p);
+  else
+    k_reorth_finalize<float><<<dim3(32, p.count), 256, 0, s>>>(jobs, p);
+  return cudaGetLastError();
+}
+
+}  // namespace iskv

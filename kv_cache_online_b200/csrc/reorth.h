@@ -1,0 +1,27 @@
+// Re-orthogonalisation: workspace layout and launcher.
+#pragma once
+
+#include "kernels.h"
+
+namespace iskv {
+
+constexpr int REORTH_SPLIT = 1024;  // rows per Gram partial
+constexpr int NS_ITERS = 8;         // coupled Newton-Schulz iterations
+
+struct ReorthWsLayout {
+  size_t scal, gpart_u, gpart_b, G[2], Y[2], Z[2], T[2], Y2[2], Z2[2], M, Gt, Gtb, Ht, sig, TUt,
+      TUtb, TBt, Bn, total;
+  int nsplit_u, nsplit_b;
+};
+
+ReorthWsLayout reorth_ws_layout(int d, int r, int64_t n_cap);
+
+struct ReorthParams {
+  int d, r, storage, count;
+  int64_t n_cap;
+  ReorthWsLayout ws;
+};
+
+cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s);
+
+}  // namespace iskv

@@ -1,0 +1,50 @@
+"""GPU parity of re-orthogonalisation (Section 4.4) against the float64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import kv, set_state, state, stored
+from oracle import fold as of
+from oracle import reorth as oreo
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("storage,tol", [(torch.float32, 1e-4), (torch.bfloat16, 2e-2)])
+def test_reorth_parity(storage, tol):
+    m = kv()
+    n, d, r, k = 4096, 1024, 256, 256
+    g = np.random.Generator(np.random.PCG64(31))
+    U = stored(np.linalg.qr(g.standard_normal((n, k)))[0] + 2e-3 * g.standard_normal((n, k)) /
+               np.sqrt(n), storage)
+    B = stored(np.linalg.qr(g.standard_normal((d, k)))[0] + 2e-3 * g.standard_normal((d, k)) /
+               np.sqrt(d), storage)
+    s = stored(np.sqrt(n) * np.arange(1, k + 1) ** -1.0, torch.float32)
+    h = m.LowRankHistory(d, r, n, storage=storage)
+    set_state(h, U, s, B, np.arange(n), folds=16)
+    m.reorth(h)
+    U2, s2, B2, _, (k2, n2, folds, st) = state(h)
+    assert (k2, n2, folds, st) == (k, n, 0, 0)
+    Ur, sr, Br = oreo.reorth(U, s, B)
+    np.testing.assert_allclose(s2, sr, rtol=1e-4)
+    assert of.rel_fro(of.low_rank_product(U2, s2, B2), of.low_rank_product(U, s, B)) < tol
+    if storage == torch.float32:
+        assert oreo.orthogonality_error(U2) < 1e-4
+        assert oreo.orthogonality_error(B2) < 1e-4
+
+
+def test_reorth_partial_rank_after_folds():
+    m = kv()
+    import synth
+    X = stored(synth.lowrank_rows(512, 128, 1.0, 0.0, seed=0, rank=12), torch.float32)
+    h = m.LowRankHistory(128, 16, 512, storage=torch.float32)
+    Xd = torch.as_tensor(X, dtype=torch.float32, device="cuda")
+    for i in range(10):
+        m.fold_block(h, Xd[i * 16:(i + 1) * 16].contiguous(),
+                     torch.arange(i * 16, (i + 1) * 16, dtype=torch.int32, device="cuda"))
+    U, s, B, _, (k, n, _, _) = state(h)
+    m.reorth(h)
+    U2, s2, B2, _, (k2, n2, folds, st) = state(h)
+    assert (k2, n2, folds, st) == (k, n, 0, 0)
+    assert of.rel_fro(of.low_rank_product(U2, s2, B2), of.low_rank_product(U, s, B)) < 1e-4
