@@ -182,14 +182,16 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
     if (tid < b) {
       double s = 0.0;
       for (int i = 0; i < b; ++i) s = fma((double)Rm[tid * b + i], (double)Rm[tid * b + i], s);
-      nrm[tid] = (float)sqrt(s);
+      const float v = (float)sqrt(s);
+      nrm[tid] = isfinite(v) ? v : -1.f;  // non-finite input ranks last; the order stays total
+      if (!isfinite(v)) record_status(jb.h.meta, ISKV_ERR_NONFINITE);
     }
     __syncthreads();
-    if (tid < b) {  // rank by (norm desc, index asc)
+    if (tid < b) {  // rank by (norm desc, index asc): a permutation of 0..b-1
       int rk = 0;
       for (int c = 0; c < b; ++c)
         rk += (nrm[c] > nrm[tid]) || (nrm[c] == nrm[tid] && c < tid);
-      order[rk] = tid;
+      order[min(rk, b - 1)] = tid;
     }
     __syncthreads();
     if (tid == 0) {
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
     // W[i][q] = Rm[:, order[q]] / rho for q < p (row-major b x b).
     for (int e = tid; e < b * pp; e += RES_NTH) {
       const int i = e / pp, q = e % pp;
-      const int c = order[q];
+      const int c = min(max(order[q], 0), b - 1);
       W[i * b + q] = Rm[c * b + i] / nrm[c];
     }
     __syncthreads();

@@ -263,10 +263,14 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
     if (warp >= w) continue;
     const int j = pairs[(0 * cj + rank) * 2 + slot] * w + warp;
     const float nj = nrm_all[j];
+    // Rank by (norm desc, index asc) on a key where a non-finite norm sorts last, so the ranks
+    // form a permutation even for NaN input.
+    const float kj = isfinite(nj) ? nj : -1.f;
     int cnt = 0;
     for (int i = lane; i < npad; i += 32) {
       const float ni = nrm_all[i];
-      cnt += (ni > nj) || (ni == nj && i < j);
+      const float ki = isfinite(ni) ? ni : -1.f;
+      cnt += (ki > kj) || (ki == kj && i < j);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
