@@ -129,7 +129,8 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
  * (pairs (j, j + head_dim/2) inside each head, angle pos * rope_theta^(-2j/head_dim)).
  * out          [n_total][d] out_dtype; rows not named by either set are left untouched.
  * exact_rows   [n_exact][d] exact_dtype (may be NULL when n_exact == 0); exact_pos [n_exact].
- * Positions must lie in [0, n_total) and be distinct across both sets (not checked on device).
+ * Positions must be distinct across both sets; a position outside [0, n_total) is not written and
+ * ISKV_ERR_SHAPE is recorded in the history's status word.
  * d == n_heads * head_dim, head_dim even and <= 256.
  * ws           iskv_reconstruct_workspace_size(1, d, r_max) bytes (sigma-scaled basis).
  * hs and the per-job arrays of the batched form are HOST arrays of `count` entries.
@@ -179,6 +180,22 @@ iskv_status iskv_reset(const iskv_lowrank *h, void *stream);
  */
 iskv_status iskv_get_status(const iskv_lowrank *h, int64_t *k, int64_t *n, int64_t *folds,
                             int64_t *status_bits);
+
+/*
+ * Instrumentation (no counterpart on the pages; measurement support). When stage timing is on,
+ * every entry point records CUDA events on its own stream around each internal stage (fold:
+ * projection, residual QR + SVD, core SVD, basis rotation, coordinate rotation, write-back;
+ * reorth; reconstruction; selection). iskv_stage_read() waits for those events and returns the
+ * accumulated milliseconds and call counts per stage (arrays of iskv_stage_count() entries, host
+ * memory). iskv_stage_timing() returns the previous setting. iskv_launch_count() is the number of
+ * kernels the library has launched in this process (always counted).
+ */
+int32_t iskv_stage_timing(int32_t enable);
+int32_t iskv_stage_count(void);
+const char *iskv_stage_name(int32_t i);
+iskv_status iskv_stage_read(double *ms, int64_t *calls);
+void iskv_stage_reset(void);
+int64_t iskv_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -241,3 +241,29 @@ def select_prompt_blocks(keys, block=8, per_head=128, suffix_blocks=4, v_radius=
         out["P_K"].data_ptr(), out["P_V"].data_ptr(), out["head_blocks"].data_ptr(),
         out["counts"].data_ptr(), w.data_ptr(), w.numel(), _stream(stream)), "select_prompt_blocks")
     return out
+
+
+# ------------------------------------------------------------------------------------------------
+# Instrumentation (measurement support, not part of the method).
+
+def stage_timing(enable: bool) -> bool:
+    """Turn per-stage CUDA-event timing inside the library on or off; returns the old setting."""
+    return bool(_lib.load().iskv_stage_timing(1 if enable else 0))
+
+
+def stage_times(reset: bool = False):
+    """{stage name: (total ms, calls)} accumulated since the last reset (waits for the events)."""
+    lib = _lib.load()
+    n = lib.iskv_stage_count()
+    ms = (ctypes.c_double * n)()
+    calls = (ctypes.c_int64 * n)()
+    _lib.check(lib.iskv_stage_read(ms, calls), "stage_read")
+    out = {lib.iskv_stage_name(i).decode(): (ms[i], calls[i]) for i in range(n)}
+    if reset:
+        lib.iskv_stage_reset()
+    return out
+
+
+def launch_count() -> int:
+    """Number of kernels the library has launched in this process."""
+    return int(_lib.load().iskv_launch_count())

@@ -53,6 +53,12 @@ SIGNATURES = {
     "iskv_get_status": (c_i32, [ctypes.POINTER(IskvLowRank), ctypes.POINTER(c_i64),
                                 ctypes.POINTER(c_i64), ctypes.POINTER(c_i64),
                                 ctypes.POINTER(c_i64)]),
+    "iskv_stage_timing": (c_i32, [c_i32]),
+    "iskv_stage_count": (c_i32, []),
+    "iskv_stage_name": (ctypes.c_char_p, [c_i32]),
+    "iskv_stage_read": (c_i32, [ctypes.POINTER(c_f64), ctypes.POINTER(c_i64)]),
+    "iskv_stage_reset": (None, []),
+    "iskv_launch_count": (c_i64, []),
 }
 
 _lib = None

@@ -13,6 +13,7 @@
 
 #include "jacobi_small.cuh"
 #include "kernels.h"
+#include "profiling.h"
 
 namespace cg = cooperative_groups;
 
@@ -306,6 +307,7 @@ cudaError_t launch_fold_residual(const FoldJob *jobs, const FoldParams &p, cudaS
     if (e != cudaSuccess) return e;
     e = cudaLaunchKernelEx(&cfg, k_fold_residual<float>, jobs, p);
   }
+  count_launches(1);
   return e;
 }
 

@@ -7,6 +7,7 @@
 
 #include "gemm_tile.cuh"
 #include "kernels.h"
+#include "profiling.h"
 
 namespace iskv {
 
@@ -28,6 +29,7 @@ cudaError_t upload_jobs(void *dst, const void *src, size_t bytes, cudaStream_t s
     const size_t n = bytes - off < sizeof(UploadChunk) ? bytes - off : sizeof(UploadChunk);
     std::memcpy(c.data, p + off, n);
     k_upload<<<1, 256, 0, s>>>(static_cast<unsigned char *>(dst) + off, c, (int)n);
+    count_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -70,6 +72,7 @@ __global__ void k_fold_prepare(const FoldJob *jobs, FoldParams p) {
 
 cudaError_t launch_fold_prepare(const FoldJob *jobs, const FoldParams &p, cudaStream_t s) {
   k_fold_prepare<<<(p.count + 127) / 128, 128, 0, s>>>(jobs, p);
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -123,6 +126,7 @@ static cudaError_t project_t(const FoldJob *jobs, const FoldParams &p, cudaStrea
   k_fold_project<1, TF, TS><<<gd, 256, 0, s>>>(jobs, p);
   k_fold_project<2, TF, TS><<<gk, 256, 0, s>>>(jobs, p);
   k_fold_project<3, TF, TS><<<gd, 256, 0, s>>>(jobs, p);
+  count_launches(4);
   return cudaGetLastError();
 }
 
@@ -165,6 +169,7 @@ cudaError_t launch_rotate_basis(const char *jobs, const RotParams &p, cudaStream
     k_rotate_basis<__nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
   else
     k_rotate_basis<float><<<g, 256, 0, s>>>(jobs, p);
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -242,6 +247,7 @@ cudaError_t launch_rotate_coords_ffma(const char *jobs, const RotParams &p, int6
     if (e != cudaSuccess) return e;
     k_rotate_coords_ffma<float><<<g, 256, smem, s>>>(jobs, p);
   }
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -287,6 +293,7 @@ cudaError_t launch_fold_finalize(const FoldJob *jobs, const FoldParams &p, cudaS
     k_fold_finalize<__nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
   else
     k_fold_finalize<float><<<g, 256, 0, s>>>(jobs, p);
+  count_launches(1);
   return cudaGetLastError();
 }
 

@@ -8,6 +8,7 @@
 
 #include "iskv.h"
 #include "kernels.h"
+#include "profiling.h"
 #include "recon.h"
 #include "reorth.h"
 #include "select.h"
@@ -156,20 +157,28 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   FoldJob *djobs = reinterpret_cast<FoldJob *>(base);
+  stage_begin(s);
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(FoldJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "fold: upload");
   if ((e = launch_fold_prepare(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: prepare");
+  stage_mark(s, ST_UPLOAD);
   if ((e = launch_fold_project(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: project");
+  stage_mark(s, ST_FOLD_PROJECT);
   if ((e = launch_fold_residual(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: residual");
+  stage_mark(s, ST_FOLD_RESIDUAL);
   const char *cj = reinterpret_cast<const char *>(djobs);
   if ((e = launch_core(cj, fold_core_params(p), s)) != cudaSuccess)
     return cuda_fail(e, "fold: core svd");
+  stage_mark(s, ST_FOLD_CORE);
   const RotParams rp = fold_rot_params(p);
   if ((e = launch_rotate_basis(cj, rp, s)) != cudaSuccess)
     return cuda_fail(e, "fold: basis rotation");
+  stage_mark(s, ST_FOLD_BASIS);
   if ((e = launch_rotate_coords(cj, rp, ncap_max, s)) != cudaSuccess)
     return cuda_fail(e, "fold: coordinate rotation");
+  stage_mark(s, ST_FOLD_COORDS);
   if ((e = launch_fold_finalize(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: finalize");
+  stage_mark(s, ST_FOLD_FINALIZE);
   return ISKV_OK;
 }
 
@@ -231,8 +240,10 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ReorthJob *djobs = reinterpret_cast<ReorthJob *>(base);
+  stage_begin(s);
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReorthJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "reorth: upload");
+  stage_mark(s, ST_UPLOAD);
   if ((e = launch_reorth(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "reorth");
   return ISKV_OK;
 }
@@ -312,12 +323,16 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ReconJob *djobs = reinterpret_cast<ReconJob *>(base);
+  stage_begin(s);
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReconJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "reconstruct: upload");
+  stage_mark(s, ST_UPLOAD);
   if ((e = launch_recon_compressed(djobs, p, s)) != cudaSuccess)
     return cuda_fail(e, "reconstruct: compressed rows");
+  stage_mark(s, ST_RECON_COMPRESSED);
   if ((e = launch_recon_exact(djobs, p, max_exact, s)) != cudaSuccess)
     return cuda_fail(e, "reconstruct: exact rows");
+  stage_mark(s, ST_RECON_EXACT);
   return ISKV_OK;
 }
 
@@ -379,8 +394,11 @@ iskv_status iskv_select_prompt_blocks(const void *keys, int32_t k_dtype, int64_t
   a.head_blocks = head_blocks_out;
   a.counts = counts_out;
   a.ws = ws;
-  cudaError_t e = launch_select(a, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  stage_begin(s);
+  cudaError_t e = launch_select(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "select");
+  stage_mark(s, ST_SELECT);
   return ISKV_OK;
 }
 

@@ -20,6 +20,7 @@
 
 #include "jacobi_small.cuh"
 #include "kernels.h"
+#include "profiling.h"
 
 namespace cg = cooperative_groups;
 
@@ -335,6 +336,7 @@ static cudaError_t core_launch(const char *jobs, const CoreParams &p, const Jaco
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  count_launches(1);
   return cudaLaunchKernelEx(&cfg, kern, jobs, p, c.w);
 }
 

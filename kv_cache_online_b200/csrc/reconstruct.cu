@@ -5,6 +5,7 @@
 // RoPE angles: pos * theta^(-2j/hd) reaches tens of thousands of radians, where one float32 ulp is
 // ~4e-3 rad. The angle is therefore formed and reduced modulo 2 pi in float64 and only the reduced
 // angle (|a| <= pi) goes to sincosf.
+#include "profiling.h"
 #include "recon.h"
 
 namespace iskv {
@@ -135,6 +136,7 @@ template <typename TS, typename TO>
 static cudaError_t recon_ffma_t(const ReconJob *jobs, const ReconParams &p, cudaStream_t s) {
   const dim3 g((unsigned)((p.n_cap_max + RRM - 1) / RRM), p.n_heads, p.count);
   k_recon_ffma<TS, TO><<<g, 256, 0, s>>>(jobs, p);
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -162,6 +164,7 @@ cudaError_t launch_recon_exact(const ReconJob *jobs, const ReconParams &p, int64
   else if (eb) k_recon_exact<__nv_bfloat16, float><<<g, 256, 0, s>>>(jobs, p);
   else if (ob) k_recon_exact<float, __nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
   else k_recon_exact<float, float><<<g, 256, 0, s>>>(jobs, p);
+  count_launches(1);
   return cudaGetLastError();
 }
 

@@ -12,6 +12,7 @@
 // Then M = R_U diag(sigma) R_B goes through the cluster Jacobi SVD (dense mode), and the two
 // rotations U <- U (R_U^-1 X), B <- B (R_B^-1 Y) reuse the fold's rotation kernels.
 #include "gemm_tile.cuh"
+#include "profiling.h"
 #include "reorth.h"
 
 namespace iskv {
@@ -248,6 +249,8 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
     k_gram_partial<float><<<dim3(tn, tm, p.count * W.nsplit_b), 256, 0, s>>>(jobs, p, 1, W.nsplit_b);
   }
   k_gram_reduce<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
+  count_launches(4);
+  stage_mark(s, ST_REORTH_GRAM);
   k_ns_init<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
   size_t y0[2] = {W.Y[0], W.Y[1]}, z0[2] = {W.Z[0], W.Z[1]};
   size_t y1[2] = {W.Y2[0], W.Y2[1]}, z1[2] = {W.Z2[0], W.Z2[1]};
@@ -262,6 +265,8 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
     }
   }
   k_reorth_M<<<dim3(tn, tm, p.count), 256, 0, s>>>(jobs, p, y0[0], y0[1]);
+  count_launches(2 + 2 * NS_ITERS);
+  stage_mark(s, ST_REORTH_NS);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -285,6 +290,8 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   e = launch_core(reinterpret_cast<const char *>(jobs), c, s);
   if (e != cudaSuccess) return e;
   k_reorth_T<<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p, z0[0], z0[1]);
+  count_launches(1);
+  stage_mark(s, ST_REORTH_CORE);
 
   RotParams q;
   q.d = p.d;
@@ -301,12 +308,15 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   q.pld = 1;
   e = launch_rotate_coords(reinterpret_cast<const char *>(jobs), q, p.n_cap, s);
   if (e != cudaSuccess) return e;
+  stage_mark(s, ST_REORTH_COORDS);
   e = launch_rotate_basis(reinterpret_cast<const char *>(jobs), q, s);
   if (e != cudaSuccess) return e;
   if (p.storage == ISKV_BF16)
     k_reorth_finalize<__nv_bfloat16><<<dim3(32, p.count), 256, 0, s>>>(jobs, p);
   else
     k_reorth_finalize<float><<<dim3(32, p.count), 256, 0, s>>>(jobs, p);
+  count_launches(1);
+  stage_mark(s, ST_REORTH_BASIS);
   return cudaGetLastError();
 }
 

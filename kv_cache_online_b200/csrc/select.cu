@@ -8,6 +8,7 @@
 // Kernels: block scores (one warp per (head, block)), an exact radix select per head (one CTA
 // per head; 8 passes of 8-bit digits over an order-preserving 64-bit key, ties taken in block
 // order), and a three-phase scan that compacts P_K and P_V.
+#include "profiling.h"
 #include "select.h"
 
 namespace iskv {
@@ -241,6 +242,7 @@ static cudaError_t scan_u8(const uint8_t *f, int64_t L, int32_t *chunk, int32_t 
   k_scan_chunk_sums<<<(unsigned)nchunks, 256, 0, s>>>(f, L, chunk);
   k_scan_chunk_offsets<<<1, SEL_NTH, 0, s>>>(chunk, nchunks);
   k_scan_apply<<<(unsigned)nchunks, SEL_NTH, 0, s>>>(f, L, chunk, cnt);
+  count_launches(3);
   return cudaGetLastError();
 }
 
@@ -291,17 +293,21 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t s) {
     else
       k_block_scores<<<g, 256, 0, s>>>(static_cast<const float *>(a.keys), n_cand, a.H, a.hd,
                                        a.block, scores);
+    count_launches(1);
   }
   k_select_head<<<a.H, SEL_NTH, 0, s>>>(scores, n_cand, a.per_head, a.head_blocks, a.counts,
                                         blkflag);
   const unsigned gL = (unsigned)((a.L + 255) / 256 < 65535 ? (a.L + 255) / 256 : 65535);
   k_mark_protected<<<gL, 256, 0, s>>>(blkflag, a.L, a.block, n_cand, prot);
+  count_launches(2);
   e = scan_u8(prot, a.L, chunk, cntK, s);
   if (e != cudaSuccess) return e;
   k_compact_pk_near<<<gL, 256, 0, s>>>(prot, cntK, a.L, a.v_radius, a.pk_out, nearf, a.counts);
+  count_launches(1);
   e = scan_u8(nearf, a.L, chunk, cntV, s);
   if (e != cudaSuccess) return e;
   k_compact_pv<<<gL, 256, 0, s>>>(nearf, cntV, a.L, a.pv_out, a.counts);
+  count_launches(1);
   return cudaGetLastError();
 }
 
