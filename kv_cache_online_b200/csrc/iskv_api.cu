@@ -12,6 +12,7 @@
 #include "recon.h"
 #include "reorth.h"
 #include "select.h"
+#include "tc.h"
 
 using namespace iskv;
 
@@ -93,7 +94,7 @@ const char *iskv_last_error(void) { return g_last_error.c_str(); }
 size_t iskv_fold_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t b) {
   if (count < 1 || d < 1 || r_max < 1 || b < 1) return 0;
   const FoldWsLayout L = fold_ws_layout(d, r_max, b);
-  return jobs_bytes(count, sizeof(FoldJob)) + (size_t)count * L.total;
+  return jobs_bytes(count, sizeof(FoldJob)) + tc_table_bytes(count) + (size_t)count * L.total;
 }
 
 iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const void *const *F,
@@ -138,7 +139,8 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   p.tau_rel = tau_rel;
   p.ws = fold_ws_layout(d, r, b);
   char *base = static_cast<char *>(ws);
-  const size_t jb = jobs_bytes(count, sizeof(FoldJob));
+  TcJob *tc_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(FoldJob)));
+  const size_t jb = jobs_bytes(count, sizeof(FoldJob)) + tc_table_bytes(count);
   std::vector<FoldJob> jobs(count);
   int64_t ncap_max = 0;
   for (int32_t i = 0; i < count; ++i) {
@@ -174,8 +176,18 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   if ((e = launch_rotate_basis(cj, rp, s)) != cudaSuccess)
     return cuda_fail(e, "fold: basis rotation");
   stage_mark(s, ST_FOLD_BASIS);
-  if ((e = launch_rotate_coords(cj, rp, ncap_max, s)) != cudaSuccess)
-    return cuda_fail(e, "fold: coordinate rotation");
+  if (tc_rotation_supported(r, p.storage)) {
+    std::vector<TcJob> tj(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_rotation_job(tj[i], hs[i].U, hs[i].n_cap, r, jobs[i].h.ws + p.ws.Gtb,
+                               reinterpret_cast<const int32_t *>(jobs[i].h.ws + p.ws.scal),
+                               hs[i].meta))
+        return fail(ISKV_ERR_CUDA, "fold: tensor map encoding failed");
+    e = launch_tc_rotation(tj.data(), count, tc_dev, r, ncap_max, s);
+  } else {
+    e = launch_rotate_coords_ffma(cj, rp, ncap_max, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "fold: coordinate rotation");
   stage_mark(s, ST_FOLD_COORDS);
   if ((e = launch_fold_finalize(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: finalize");
   stage_mark(s, ST_FOLD_FINALIZE);
@@ -196,7 +208,7 @@ iskv_status iskv_fold_block(const iskv_lowrank *h, const void *F, int32_t f_dtyp
 size_t iskv_reorth_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap) {
   if (count < 1 || d < 1 || r_max < 1 || n_cap < 0) return 0;
   const ReorthWsLayout L = reorth_ws_layout(d, r_max, n_cap);
-  return jobs_bytes(count, sizeof(ReorthJob)) + (size_t)count * L.total;
+  return jobs_bytes(count, sizeof(ReorthJob)) + tc_table_bytes(count) + (size_t)count * L.total;
 }
 
 iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t ws_bytes,
@@ -225,7 +237,8 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   p.n_cap = ncap;
   p.ws = reorth_ws_layout(d, r, ncap);
   char *base = static_cast<char *>(ws);
-  const size_t jb = jobs_bytes(count, sizeof(ReorthJob));
+  TcJob *tc_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReorthJob)));
+  const size_t jb = jobs_bytes(count, sizeof(ReorthJob)) + tc_table_bytes(count);
   std::vector<ReorthJob> jobs(count);
   for (int32_t i = 0; i < count; ++i) {
     ReorthJob &j = jobs[i];
@@ -237,6 +250,18 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
     j.h.ws = base + jb + (size_t)i * p.ws.total;
     j.n_cap = hs[i].n_cap;
     j.pad_ = 0;
+  }
+  std::vector<TcJob> tj;
+  p.tc_host = nullptr;
+  p.tc_dev = tc_dev;
+  if (tc_rotation_supported(r, p.storage)) {
+    tj.resize(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_rotation_job(tj[i], hs[i].U, hs[i].n_cap, r, jobs[i].h.ws + p.ws.TUtb,
+                               reinterpret_cast<const int32_t *>(jobs[i].h.ws + p.ws.scal),
+                               hs[i].meta))
+        return fail(ISKV_ERR_CUDA, "reorth: tensor map encoding failed");
+    p.tc_host = tj.data();
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ReorthJob *djobs = reinterpret_cast<ReorthJob *>(base);
@@ -252,7 +277,8 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
 // Reconstruction
 size_t iskv_reconstruct_workspace_size(int32_t count, int32_t d, int32_t r_max) {
   if (count < 1 || d < 1 || r_max < 1) return 0;
-  return jobs_bytes(count, sizeof(ReconJob)) + (size_t)count * align_up((size_t)d * r_max * 2, 256);
+  return jobs_bytes(count, sizeof(ReconJob)) + tc_table_bytes(count) +
+         (size_t)count * align_up((size_t)d * r_max * 2, 256);
 }
 
 iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
@@ -303,7 +329,8 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
   p.theta = rope_theta;
   p.n_cap_max = ncap_max;
   char *base = static_cast<char *>(ws);
-  const size_t jb = jobs_bytes(count, sizeof(ReconJob));
+  TcJob *tc_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReconJob)));
+  const size_t jb = jobs_bytes(count, sizeof(ReconJob)) + tc_table_bytes(count);
   std::vector<ReconJob> jobs(count);
   for (int32_t i = 0; i < count; ++i) {
     ReconJob &j = jobs[i];
@@ -327,8 +354,17 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReconJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "reconstruct: upload");
   stage_mark(s, ST_UPLOAD);
-  if ((e = launch_recon_compressed(djobs, p, s)) != cudaSuccess)
-    return cuda_fail(e, "reconstruct: compressed rows");
+  if (tc_recon_supported(r, p.storage, out_dtype, head_dim)) {
+    std::vector<TcJob> tj(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_recon_job(tj[i], hs[i].U, hs[i].n_cap, r, jobs[i].bsig, d, out[i], hs[i].pos,
+                            hs[i].meta, n_total[i], apply_rope[i]))
+        return fail(ISKV_ERR_CUDA, "reconstruct: tensor map encoding failed");
+    e = launch_tc_recon(djobs, tj, tc_dev, p, s);
+  } else {
+    e = launch_recon_compressed(djobs, p, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "reconstruct: compressed rows");
   stage_mark(s, ST_RECON_COMPRESSED);
   if ((e = launch_recon_exact(djobs, p, max_exact, s)) != cudaSuccess)
     return cuda_fail(e, "reconstruct: exact rows");

@@ -51,8 +51,6 @@ cudaError_t launch_fold_finalize(const FoldJob *jobs, const FoldParams &p, cudaS
 
 cudaError_t launch_core(const char *jobs, const CoreParams &p, cudaStream_t s);
 cudaError_t launch_rotate_basis(const char *jobs, const RotParams &p, cudaStream_t s);
-cudaError_t launch_rotate_coords(const char *jobs, const RotParams &p, int64_t n_cap_max,
-                                 cudaStream_t s);
 cudaError_t launch_rotate_coords_ffma(const char *jobs, const RotParams &p, int64_t n_cap_max,
                                       cudaStream_t s);
 

@@ -306,7 +306,10 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   q.bn = W.Bn;
   q.hs = r;
   q.pld = 1;
-  e = launch_rotate_coords(reinterpret_cast<const char *>(jobs), q, p.n_cap, s);
+  if (p.tc_host)
+    e = launch_tc_rotation(p.tc_host, p.count, p.tc_dev, r, p.n_cap, s);
+  else
+    e = launch_rotate_coords_ffma(reinterpret_cast<const char *>(jobs), q, p.n_cap, s);
   if (e != cudaSuccess) return e;
   stage_mark(s, ST_REORTH_COORDS);
   e = launch_rotate_basis(reinterpret_cast<const char *>(jobs), q, s);

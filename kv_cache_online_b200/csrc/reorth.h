@@ -2,6 +2,7 @@
 #pragma once
 
 #include "kernels.h"
+#include "tc.h"
 
 namespace iskv {
 
@@ -20,6 +21,8 @@ struct ReorthParams {
   int d, r, storage, count;
   int64_t n_cap;
   ReorthWsLayout ws;
+  const TcJob *tc_host;  // tensor-core coordinate rotation jobs (host copy) or null
+  TcJob *tc_dev;         // their device table
 };
 
 cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s);

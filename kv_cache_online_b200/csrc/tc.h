@@ -1,0 +1,48 @@
+// Tensor-core (tcgen05) path: job table and host launchers.
+#pragma once
+
+#include <cuda.h>
+
+#include <vector>
+
+#include "kernels.h"
+#include "recon.h"
+
+namespace iskv {
+
+// One tensor-core job: two TMA descriptors plus the pointers its epilogue needs. 64-byte aligned
+// (TMA descriptors must be); lives in the caller's workspace.
+struct alignas(64) TcJob {
+  CUtensorMap mapA;      // U [n_cap][r] bf16, box {64, 128}
+  CUtensorMap mapB;      // rotation: G^T [r][r] bf16, box {64, r}; reconstruction: sigma B [d][r]
+  void *U;               // rotation output (in place)
+  const int32_t *sc;     // rotation: the job's FS_* scalars
+  void *out;             // reconstruction output [n_total][d] bf16
+  const int32_t *pos;    // reconstruction: row positions
+  int64_t *meta;         // status word target
+  int64_t n_total;
+  int32_t rope;
+  int32_t pad_;
+};
+
+struct TcParams {
+  int r, d, n_heads, count, tiles_per_job;
+  double theta;
+};
+
+bool tc_rotation_supported(int r, int storage);
+bool tc_recon_supported(int r, int storage, int out_dtype, int head_dim);
+
+bool encode_rotation_job(TcJob &tj, void *U, int64_t n_cap, int r, const void *gtb,
+                         const int32_t *sc, int64_t *meta);
+bool encode_recon_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void *bsig, int d,
+                      void *out, const int32_t *pos, int64_t *meta, int64_t n_total, int rope);
+
+cudaError_t launch_tc_rotation(const TcJob *hjobs, int count, TcJob *djobs, int r,
+                               int64_t n_cap_max, cudaStream_t s);
+cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob> &hjobs,
+                            TcJob *djobs, const ReconParams &p, cudaStream_t s);
+
+inline size_t tc_table_bytes(int count) { return ((size_t)count * sizeof(TcJob) + 255) / 256 * 256; }
+
+}  // namespace iskv

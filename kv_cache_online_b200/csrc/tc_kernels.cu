@@ -1,0 +1,538 @@
+// Tensor-core (tcgen05) kernels for the two dense contractions that sweep every history row:
+//
+//  * coordinate rotation (iS-KV reading notes, Algorithm 2 step 7; Section 4.4):
+//      U[0:n] <- U[0:n] G,  in place, bf16 factors, fp32 accumulation in tensor memory;
+//  * reconstruction (Algorithm 3 steps 7-8):
+//      out[pos_i] = RoPE_pos_i( U_i (diag(sigma) B^T) ),  bf16 out, RoPE fused into the epilogue.
+//
+// Both are persistent kernels over 128-row tiles of U. Roles: warp 0 issues TMA loads (U tiles,
+// and the small right-hand operand), warp 1 owns tensor memory and issues tcgen05.mma from one
+// thread, warps 2-9 drain the fp32 accumulators from tensor memory (each warp reads the 32 TMEM
+// lanes it may access, i.e. 32 rows) and write the results. The U tile is held as r/64 K-slabs of
+// 16 KB; each slab is released to the producer as soon as the last MMA reading it completes, so the
+// next tile's loads overlap the current tile's MMAs. Two TMEM accumulator buffers let the epilogue
+// of one tile (or head) overlap the MMAs of the next.
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "profiling.h"
+#include "recon.h"
+#include "tc.h"
+#include "tc_sm100.cuh"
+
+namespace iskv {
+
+using namespace tc;
+
+constexpr int TC_THREADS = 320;        // 10 warps
+constexpr int TC_M = 128;              // rows per tile
+constexpr int SLAB_BYTES = 128 * 128;  // 128 rows x 64 bf16
+constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
+
+struct TcCtl {
+  uint64_t a_full[4], a_empty[4];
+  uint64_t b_full[2], b_empty[2];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t done;
+  uint32_t tmem;
+  int abort;
+};
+
+// ------------------------------------------------------------------------------------------------
+// Tile iteration shared by all roles: contiguous ranges of (job, 128-row tile) per CTA.
+struct TileRange {
+  int begin, end, tiles_per_job;
+};
+
+ISKV_DEV TileRange my_tiles(int count, int tiles_per_job) {
+  const int total = count * tiles_per_job;
+  const int per = (total + gridDim.x - 1) / gridDim.x;
+  TileRange t;
+  t.begin = blockIdx.x * per;
+  t.end = min(total, t.begin + per);
+  t.tiles_per_job = tiles_per_job;
+  return t;
+}
+
+ISKV_DEV void fail_timeout(TcCtl *c, int64_t *meta) {
+  c->abort = 1;
+  if (meta) record_status(meta, ISKV_ERR_TIMEOUT);
+}
+
+// ================================================================================================
+// Coordinate rotation. Job fields: mapA (U), mapB (G^T as bf16, r x r), U, sc (scalars).
+__global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int R = p.r, KS = R / 64, N = R;
+  uint8_t *sA = smem;                       // KS slabs x 16 KB
+  uint8_t *sB = smem + KS * SLAB_BYTES;     // KS slabs x (N x 128 B)
+  TcCtl *ctl = reinterpret_cast<TcCtl *>(sB + KS * N * 128);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = N <= 64 ? 128 : (N <= 128 ? 256 : 512);
+  const uint32_t idesc = idesc_bf16_f32(TC_M, N);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 4; ++s) { mbar_init(&ctl->a_full[s], 1); mbar_init(&ctl->a_empty[s], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->b_full[i], 1);
+      mbar_init(&ctl->b_empty[i], 1);
+      mbar_init(&ctl->acc_full[i], 1);
+      mbar_init(&ctl->acc_empty[i], 8);
+    }
+    mbar_init(&ctl->done, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&ctl->tmem, ncols);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int *abort = &ctl->abort;
+  const TileRange tr = my_tiles(p.count, p.tiles_per_job);
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer
+    int cur = -1, nb = 0, na = 0;
+    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
+      const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+      const TcJob &jb = jobs[j];
+      if (jb.sc[FS_SKIP] || row0 >= jb.sc[FS_N_OLD] || jb.sc[FS_K_OLD] == 0) continue;
+      if (j != cur) {
+        if (nb > 0 && !mbar_wait(&ctl->b_empty[0], (nb - 1) & 1, abort, WAIT_NS)) {
+          fail_timeout(ctl, jb.meta);
+          break;
+        }
+        tensormap_acquire(&jb.mapA);
+        tensormap_acquire(&jb.mapB);
+        mbar_arrive_expect_tx(&ctl->b_full[0], KS * N * 128);
+        for (int s = 0; s < KS; ++s) tma_load_2d(sB + s * N * 128, &jb.mapB, s * 64, 0, &ctl->b_full[0]);
+        cur = j;
+        ++nb;
+      }
+      for (int s = 0; s < KS; ++s) {
+        if (na > 0 && !mbar_wait(&ctl->a_empty[s], (na - 1) & 1, abort, WAIT_NS)) {
+          fail_timeout(ctl, jb.meta);
+          break;
+        }
+        mbar_arrive_expect_tx(&ctl->a_full[s], SLAB_BYTES);
+        tma_load_2d(sA + s * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[s]);
+      }
+      ++na;
+    }
+    // Let every load this thread issued land before the CTA can exit.
+    if (na > 0)
+      for (int s = 0; s < KS; ++s) mbar_wait(&ctl->a_full[s], (na - 1) & 1, abort, WAIT_NS / 4);
+    if (nb > 0) mbar_wait(&ctl->b_full[0], (nb - 1) & 1, abort, WAIT_NS / 4);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    int cur = -1, nb = 0, na = 0;
+    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
+      const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+      const TcJob &jb = jobs[j];
+      if (jb.sc[FS_SKIP] || row0 >= jb.sc[FS_N_OLD] || jb.sc[FS_K_OLD] == 0) continue;
+      if (j != cur) {
+        if (cur >= 0) mma_commit(&ctl->b_empty[0]);
+        if (!mbar_wait(&ctl->b_full[0], nb & 1, abort, WAIT_NS)) { fail_timeout(ctl, jb.meta); break; }
+        cur = j;
+        ++nb;
+      }
+      const int buf = na & 1, use = na >> 1;
+      if (use > 0 && !mbar_wait(&ctl->acc_empty[buf], (use - 1) & 1, abort, WAIT_NS)) {
+        fail_timeout(ctl, jb.meta);
+        break;
+      }
+      fence_after_sync();
+      const uint32_t d = tmem + buf * N;
+      bool ok = true;
+      for (int s = 0; s < KS && ok; ++s) {
+        if (!mbar_wait(&ctl->a_full[s], na & 1, abort, WAIT_NS)) { ok = false; break; }
+        fence_after_sync();
+        const uint32_t a0 = smem_u32(sA + s * SLAB_BYTES), b0 = smem_u32(sB + s * N * 128);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (s | kk) != 0);
+        mma_commit(&ctl->a_empty[s]);
+      }
+      if (!ok) { fail_timeout(ctl, jb.meta); break; }
+      mma_commit(&ctl->acc_full[buf]);
+      ++na;
+    }
+    mma_commit(&ctl->done);
+    mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: TMEM -> bf16 -> U rows (in place)
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    const int cols = N / 2, c0 = half * cols;
+    int na = 0;
+    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
+      const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+      const TcJob &jb = jobs[j];
+      const int n = jb.sc[FS_N_OLD];
+      if (jb.sc[FS_SKIP] || row0 >= n || jb.sc[FS_K_OLD] == 0) continue;
+      const int buf = na & 1, use = na >> 1;
+      if (!mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS)) {
+        fail_timeout(ctl, jb.meta);
+        break;
+      }
+      fence_after_sync();
+      const int row = row0 + q * 32 + lane;
+      __nv_bfloat16 *U = static_cast<__nv_bfloat16 *>(jb.U) + (size_t)row * R;
+      for (int cc = 0; cc < cols; cc += 16) {
+        float v[16];
+        tmem_ld16(tmem + buf * N + ((uint32_t)(q * 32) << 16) + c0 + cc, v);
+        tmem_ld_wait();
+        if (row < n) {
+          uint4 w0, w1;
+          w0.x = pack_bf16(v[0], v[1]);   w0.y = pack_bf16(v[2], v[3]);
+          w0.z = pack_bf16(v[4], v[5]);   w0.w = pack_bf16(v[6], v[7]);
+          w1.x = pack_bf16(v[8], v[9]);   w1.y = pack_bf16(v[10], v[11]);
+          w1.z = pack_bf16(v[12], v[13]); w1.w = pack_bf16(v[14], v[15]);
+          uint4 *dst = reinterpret_cast<uint4 *>(U + c0 + cc);
+          dst[0] = w0;
+          dst[1] = w1;
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+      ++na;
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+// ================================================================================================
+// Reconstruction. Job fields: mapA (U), mapB (sigma-scaled basis, d x r bf16), out, pos, meta.
+__global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int R = p.r, KS = R / 64, H = p.n_heads, D = p.d;
+  constexpr int N = 128;  // one head per MMA chunk
+  constexpr int CHUNK_BYTES_PER_SLAB = N * 128;
+  uint8_t *sA = smem;                                    // KS x 16 KB
+  uint8_t *sB = smem + KS * SLAB_BYTES;                  // 2 stages x KS x 16 KB
+  TcCtl *ctl = reinterpret_cast<TcCtl *>(sB + 2 * KS * CHUNK_BYTES_PER_SLAB);
+  double *invf = reinterpret_cast<double *>(ctl + 1);    // 64 doubles
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr uint32_t NCOLS = 256;
+  const uint32_t idesc = idesc_bf16_f32(TC_M, N);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 4; ++s) { mbar_init(&ctl->a_full[s], 1); mbar_init(&ctl->a_empty[s], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->b_full[i], 1);
+      mbar_init(&ctl->b_empty[i], 1);
+      mbar_init(&ctl->acc_full[i], 1);
+      mbar_init(&ctl->acc_empty[i], 8);
+    }
+    mbar_init(&ctl->done, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x < 64) invf[threadIdx.x] = exp(-2.0 * threadIdx.x / 128.0 * log(p.theta));
+  if (warp == 1) tmem_alloc(&ctl->tmem, NCOLS);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int *abort = &ctl->abort;
+  const TileRange tr = my_tiles(p.count, p.tiles_per_job);
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer
+    int na = 0, nc = 0, cur = -1;
+    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
+      const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+      const TcJob &jb = jobs[j];
+      if (row0 >= jb.meta[ISKV_META_N]) continue;
+      if (j != cur) {
+        tensormap_acquire(&jb.mapA);
+        tensormap_acquire(&jb.mapB);
+        cur = j;
+      }
+      bool ok = true;
+      for (int s = 0; s < KS; ++s) {
+        if (na > 0 && !mbar_wait(&ctl->a_empty[s], (na - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
+        mbar_arrive_expect_tx(&ctl->a_full[s], SLAB_BYTES);
+        tma_load_2d(sA + s * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[s]);
+      }
+      ++na;
+      for (int c = 0; c < H && ok; ++c) {
+        const int st = nc & 1, use = nc >> 1;
+        if (use > 0 && !mbar_wait(&ctl->b_empty[st], (use - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
+        mbar_arrive_expect_tx(&ctl->b_full[st], KS * CHUNK_BYTES_PER_SLAB);
+        for (int s = 0; s < KS; ++s)
+          tma_load_2d(sB + (st * KS + s) * CHUNK_BYTES_PER_SLAB, &jb.mapB, s * 64, c * N,
+                      &ctl->b_full[st]);
+        ++nc;
+      }
+      if (!ok) { fail_timeout(ctl, jb.meta); break; }
+    }
+    if (na > 0)
+      for (int s = 0; s < KS; ++s) mbar_wait(&ctl->a_full[s], (na - 1) & 1, abort, WAIT_NS / 4);
+    for (int k = 1; k <= 2 && nc - k >= 0; ++k)
+      mbar_wait(&ctl->b_full[(nc - k) & 1], ((nc - k) >> 1) & 1, abort, WAIT_NS / 4);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    int na = 0, nc = 0;
+    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
+      const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+      const TcJob &jb = jobs[j];
+      if (row0 >= jb.meta[ISKV_META_N]) continue;
+      bool ok = true;
+      for (int c = 0; c < H && ok; ++c) {
+        const int buf = nc & 1, use = nc >> 1;
+        if (use > 0 && !mbar_wait(&ctl->acc_empty[buf], (use - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
+        fence_after_sync();
+        if (!mbar_wait(&ctl->b_full[buf], use & 1, abort, WAIT_NS)) { ok = false; break; }
+        const uint32_t d = tmem + buf * N;
+        for (int s = 0; s < KS; ++s) {
+          if (c == 0 && !mbar_wait(&ctl->a_full[s], na & 1, abort, WAIT_NS)) { ok = false; break; }
+          fence_after_sync();
+          const uint32_t a0 = smem_u32(sA + s * SLAB_BYTES);
+          const uint32_t b0 = smem_u32(sB + (buf * KS + s) * CHUNK_BYTES_PER_SLAB);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (s | kk) != 0);
+          if (c == H - 1) mma_commit(&ctl->a_empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&ctl->b_empty[buf]);
+        mma_commit(&ctl->acc_full[buf]);
+        ++nc;
+      }
+      if (!ok) { fail_timeout(ctl, jb.meta); break; }
+      ++na;
+    }
+    mma_commit(&ctl->done);
+    mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: TMEM -> RoPE -> bf16 -> out[pos]
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    const int j0 = half * 32;  // this thread's head-local pairs j0 .. j0 + 31 (cols j and j + 64)
+    int nc = 0;
+    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
+      const int jj = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+      const TcJob &jb = jobs[jj];
+      const int64_t n = jb.meta[ISKV_META_N];
+      if (row0 >= n) continue;
+      const int64_t row = row0 + q * 32 + lane;
+      bool valid = row < n;
+      int64_t ps = valid ? (int64_t)jb.pos[row] : 0;
+      if (valid && (ps < 0 || ps >= jb.n_total)) {
+        record_status(jb.meta, ISKV_ERR_SHAPE);
+        valid = false;
+      }
+      float cs[32], sn[32];
+      const bool rope = jb.rope != 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        cs[i] = 1.f;
+        sn[i] = 0.f;
+      }
+      if (rope && valid) {
+        const double two_pi = 6.283185307179586476925286766559;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          double a = (double)ps * invf[j0 + i];
+          a -= two_pi * rint(a / two_pi);
+          sincosf((float)a, &sn[i], &cs[i]);
+        }
+      }
+      __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(jb.out) + (size_t)(valid ? ps : 0) * D;
+      bool ok = true;
+      for (int c = 0; c < H; ++c) {
+        const int buf = nc & 1, use = nc >> 1;
+        if (!mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS)) { ok = false; break; }
+        fence_after_sync();
+        const uint32_t base = tmem + buf * N + ((uint32_t)(q * 32) << 16);
+#pragma unroll
+        for (int jb16 = 0; jb16 < 32; jb16 += 16) {
+          float lo[16], hi[16];
+          tmem_ld16(base + j0 + jb16, lo);
+          tmem_ld16(base + 64 + j0 + jb16, hi);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t wl[8], wh[8];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              const float c0 = cs[jb16 + i], s0 = sn[jb16 + i];
+              const float c1 = cs[jb16 + i + 1], s1 = sn[jb16 + i + 1];
+              const float l0 = lo[i] * c0 - hi[i] * s0, h0 = hi[i] * c0 + lo[i] * s0;
+              const float l1 = lo[i + 1] * c1 - hi[i + 1] * s1, h1 = hi[i + 1] * c1 + lo[i + 1] * s1;
+              wl[i / 2] = pack_bf16(l0, l1);
+              wh[i / 2] = pack_bf16(h0, h1);
+            }
+            uint4 *dl = reinterpret_cast<uint4 *>(orow + c * N + j0 + jb16);
+            uint4 *dh = reinterpret_cast<uint4 *>(orow + c * N + 64 + j0 + jb16);
+            dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+            dh[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            dh[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+          }
+        }
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+        ++nc;
+      }
+      if (!ok) { fail_timeout(ctl, jb.meta); break; }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, NCOLS);
+}
+
+// Sigma-scaled basis for the reconstruction: bsig[c][l] = bf16(sigma_l * B[c][l]) for l < k, else 0.
+__global__ void k_bsig(const ReconJob *jobs, int d, int r) {
+  const ReconJob &jb = jobs[blockIdx.y];
+  const int k = (int)jb.meta[ISKV_META_K];
+  const __nv_bfloat16 *B = static_cast<const __nv_bfloat16 *>(jb.B);
+  __nv_bfloat16 *bs = static_cast<__nv_bfloat16 *>(jb.bsig);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < d * r; e += gridDim.x * blockDim.x) {
+    const int l = e % r;
+    bs[e] = __float2bfloat16_rn(l < k ? jb.sigma[l] * __bfloat162float(B[e]) : 0.f);
+  }
+}
+
+// ================================================================================================
+// Host side: tensor-map encoding through the driver entry point, job tables, launches.
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major matrix [rows][cols], box {64 cols, box_rows}, 128-byte swizzle.
+bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+bool tc_rotation_supported(int r, int storage) {
+  return storage == ISKV_BF16 && r % 64 == 0 && r >= 64 && r <= 256 && encode_fn() != nullptr;
+}
+
+bool tc_recon_supported(int r, int storage, int out_dtype, int head_dim) {
+  return storage == ISKV_BF16 && out_dtype == ISKV_BF16 && head_dim == 128 && r % 64 == 0 &&
+         r >= 64 && r <= 256 && encode_fn() != nullptr;
+}
+
+size_t tc_rot_smem(int r) { return 1024 + (size_t)(r / 64) * SLAB_BYTES + (size_t)(r / 64) * r * 128 + sizeof(TcCtl); }
+
+size_t tc_rec_smem(int r) {
+  return 1024 + (size_t)(r / 64) * SLAB_BYTES * 3 + sizeof(TcCtl) + 64 * sizeof(double);
+}
+
+cudaError_t launch_tc_rotation(const TcJob *hjobs, int count, TcJob *djobs, int r,
+                               int64_t n_cap_max, cudaStream_t s) {
+  TcParams tp;
+  tp.r = r;
+  tp.d = 0;
+  tp.n_heads = 0;
+  tp.count = count;
+  tp.tiles_per_job = (int)((n_cap_max + TC_M - 1) / TC_M);
+  tp.theta = 0.0;
+  cudaError_t e = upload_jobs(djobs, hjobs, sizeof(TcJob) * count, s);
+  if (e != cudaSuccess) return e;
+  const size_t smem = tc_rot_smem(r);
+  e = cudaFuncSetAttribute(k_rot_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int total = tp.count * tp.tiles_per_job;
+  const int grid = total < num_sms() ? total : num_sms();
+  k_rot_tc<<<grid, TC_THREADS, smem, s>>>(djobs, tp);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+bool encode_rotation_job(TcJob &tj, void *U, int64_t n_cap, int r, const void *gtb,
+                         const int32_t *sc, int64_t *meta) {
+  std::memset(&tj, 0, sizeof(tj));
+  if (!encode_2d(&tj.mapA, U, (uint64_t)n_cap, (uint64_t)r, 128)) return false;
+  if (!encode_2d(&tj.mapB, gtb, (uint64_t)r, (uint64_t)r, (uint32_t)r)) return false;
+  tj.U = U;
+  tj.sc = sc;
+  tj.meta = meta;
+  return true;
+}
+
+bool encode_recon_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void *bsig, int d,
+                      void *out, const int32_t *pos, int64_t *meta, int64_t n_total, int rope) {
+  std::memset(&tj, 0, sizeof(tj));
+  if (!encode_2d(&tj.mapA, U, (uint64_t)n_cap, (uint64_t)r, 128)) return false;
+  if (!encode_2d(&tj.mapB, bsig, (uint64_t)d, (uint64_t)r, 128)) return false;
+  tj.out = out;
+  tj.pos = pos;
+  tj.meta = meta;
+  tj.n_total = n_total;
+  tj.rope = rope;
+  return true;
+}
+
+cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob> &hjobs,
+                            TcJob *djobs, const ReconParams &p, cudaStream_t s) {
+  k_bsig<<<dim3(64, p.count), 256, 0, s>>>(djobs_recon, p.d, p.r);
+  count_launches(1);
+  TcParams tp;
+  tp.r = p.r;
+  tp.d = p.d;
+  tp.n_heads = p.n_heads;
+  tp.count = p.count;
+  tp.tiles_per_job = (int)((p.n_cap_max + TC_M - 1) / TC_M);
+  tp.theta = p.theta;
+  cudaError_t e = upload_jobs(djobs, hjobs.data(), sizeof(TcJob) * hjobs.size(), s);
+  if (e != cudaSuccess) return e;
+  const size_t smem = tc_rec_smem(p.r);
+  e = cudaFuncSetAttribute(k_rec_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int total = tp.count * tp.tiles_per_job;
+  const int grid = total < num_sms() ? total : num_sms();
+  k_rec_tc<<<grid, TC_THREADS, smem, s>>>(djobs, tp);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace iskv
