@@ -110,12 +110,34 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------
+# Multi-rank plumbing: one process per GPU, independent histories (weak scaling). The only
+# collectives are the start/stop barriers and this max over ranks of the device-timed duration.
+
+def max_over_ranks(value: float, device) -> float:
+    """Maximum of `value` over all ranks of the default process group (the value itself when
+    running alone)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's synthetic histories: every rank folds different data."""
+    return 1000 + 100 * int(rank)
+
+
+# ------------------------------------------------------------------------------------------------
 # The B200 arm.
 
 class Workload:
     """64 histories (32 layers x {K, V}) and every per-step input, resident on the device."""
 
-    def __init__(self, kv, torch, dev, warmup: int, timed: int, extra: int, seed: int = 1000):
+    def __init__(self, kv, torch, dev, warmup: int, timed: int, extra: int, seed: int = 1000,
+                 layers: int = LAYERS):
         import synth
         self.kv, self.torch, self.dev = kv, torch, dev
         # n after the fold of step t is n0 + 64 (t + 1); the timed steps are centred on N_MID.
@@ -123,7 +145,7 @@ class Workload:
         self.n_cap = self.n0 + BLK * (warmup + timed + extra + 1)
         self.hists, self.kinds = [], []
         gen = torch.Generator(device=dev)
-        for layer in range(LAYERS):
+        for layer in range(layers):
             for kind in ("K", "V"):
                 h = kv.LowRankHistory(D, R, self.n_cap, storage=torch.bfloat16, device=dev)
                 sd = seed + 2 * layer + (kind == "V")
@@ -210,9 +232,10 @@ class Workload:
                                                ws=self._aligned(self.ws_sel), out=self.sel_out)
 
 
-def stage_bytes(n_mean: float):
-    """Algorithmic bytes per call of each stage for one whole step (64 histories), bf16 factors."""
-    H = LAYERS * 2
+def stage_bytes(n_mean: float, layers: int = LAYERS):
+    """Algorithmic bytes per call of each stage for one whole step (2 histories per layer), bf16
+    factors."""
+    H = layers * 2
     n_tot = PROMPT + n_mean + WINDOW
     return {
         # U read + write over every history row (Algorithm 2 step 7).
@@ -248,7 +271,8 @@ def run_b200(args):
     kv._lib.load()
     steps_total = args.warmup + args.steps
     e2e_steps = 0 if args.no_e2e else args.steps
-    wl = Workload(kv, torch, dev, args.warmup, args.steps, e2e_steps, seed=1000 + 100 * rank)
+    wl = Workload(kv, torch, dev, args.warmup, args.steps, e2e_steps, seed=rank_seed(rank),
+                  layers=args.layers)
     pos = [wl.positions(t) for t in range(steps_total + e2e_steps)]
     stream = torch.cuda.current_stream(dev)
 
@@ -281,11 +305,7 @@ def run_b200(args):
     launches = kv.launch_count() - launches0
     kv.stage_timing(False)
     st = kv.stage_times(reset=True)
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_step = ms / args.steps
     folds_step = len(wl.hists)
     n_mean = sum(wl.n_after(t) for t in range(args.warmup, steps_total)) / args.steps
@@ -300,7 +320,7 @@ def run_b200(args):
 
     # Stage rooflines.
     hbm, tc, peak_kind = peaks()
-    sbytes, _ = stage_bytes(n_mean)
+    sbytes, _ = stage_bytes(n_mean, args.layers)
     stages = {}
     for name, (tot_ms, calls) in st.items():
         if calls == 0:
@@ -341,7 +361,7 @@ def run_b200(args):
             "config": {"workload": "decode step, 32 layers x {K,V} histories at n~16K "
                                    "(fold b=64 + reorth + reconstruct with RoPE + one 64K-token "
                                    "prompt selection)",
-                       "layers": LAYERS, "histories_per_gpu": folds_step, "d": D, "r": R,
+                       "layers": args.layers, "histories_per_gpu": folds_step, "d": D, "r": R,
                        "b": BLK, "n_mean": n_mean, "kv_heads": HEADS, "head_dim": HEAD_DIM,
                        "exact_rows": PROMPT + WINDOW, "rope_theta": THETA,
                        "select_prompt_tokens": SEL_L, "storage": "bf16",
@@ -439,11 +459,7 @@ def run_e2e(wl, kv, torch, dev, stream, pos, first_step, steps, world):
     ms = ev0.elapsed_time(ev1)
     wl.keys = keys_dev
     ok = bool(torch.all(res_meta[:, 3] == 0).item())
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, dev)
     return {"value": round(world * cnt * steps / (ms / 1e3), 2), "unit": "folds/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms / steps, 4),
@@ -559,6 +575,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="model layers (2 histories each); the headline workload is 32")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "b200":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
