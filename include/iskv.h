@@ -171,6 +171,31 @@ iskv_status iskv_select_prompt_blocks(const void *keys, int32_t k_dtype, int64_t
                                       int64_t *counts_out, void *ws, size_t ws_bytes,
                                       void *stream);
 
+/*
+ * Prompt-block selection that allocates nothing and takes no workspace. No counterpart on the
+ * pages: it exists for callers that cannot allocate device memory -- a plugin running inside a host
+ * framework that owns all device memory and passes it only inputs and outputs, or a
+ * latency-critical path where a cudaMalloc could synchronise the device. Same arguments, limits
+ * and results as iskv_select_prompt_blocks() without ws / ws_bytes.
+ *  - Scratch: a fixed device array of ISKV_NOALLOC_SCRATCH bytes inside the library, present on
+ *    every GPU that loads it until the process exits. A size whose workspace
+ *    (iskv_select_workspace_size) exceeds it is refused with ISKV_ERR_WORKSPACE; at 8 heads and
+ *    8-token blocks that allows prompts up to about 230K tokens.
+ *  - Calls no cudaMalloc, cudaFree or allocating library routine.
+ *  - The first call on a device looks up the array's device address with that device current;
+ *    make that first call before any stream capture on the device.
+ *  - All calls on a device share the array and it keeps the last call's contents (the parts that
+ *    must start at zero are cleared by each call): calls that overlap on the GPU race and corrupt
+ *    each other's results, so order them on one stream.
+ */
+#define ISKV_NOALLOC_SCRATCH (4u << 20)
+iskv_status iskv_select_prompt_blocks_noalloc(const void *keys, int32_t k_dtype, int64_t L,
+                                              int32_t n_heads, int32_t head_dim, int32_t block,
+                                              int32_t per_head, int32_t suffix_blocks,
+                                              int32_t v_radius, int32_t *pk_out, int32_t *pv_out,
+                                              int32_t *head_blocks_out, int64_t *counts_out,
+                                              void *stream);
+
 /* Zero a history's meta word and sigma (stream-ordered). U and B are not touched. */
 iskv_status iskv_reset(const iskv_lowrank *h, void *stream);
 

@@ -49,6 +49,8 @@ SIGNATURES = {
     "iskv_select_workspace_size": (c_sz, [c_i64, c_i32, c_i32]),
     "iskv_select_prompt_blocks": (c_i32, [c_vp, c_i32, c_i64, c_i32, c_i32, c_i32, c_i32, c_i32,
                                           c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "iskv_select_prompt_blocks_noalloc": (c_i32, [c_vp, c_i32, c_i64, c_i32, c_i32, c_i32, c_i32,
+                                                  c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "iskv_reset": (c_i32, [ctypes.POINTER(IskvLowRank), c_vp]),
     "iskv_get_status": (c_i32, [ctypes.POINTER(IskvLowRank), ctypes.POINTER(c_i64),
                                 ctypes.POINTER(c_i64), ctypes.POINTER(c_i64),
