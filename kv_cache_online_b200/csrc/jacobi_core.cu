@@ -28,23 +28,29 @@ namespace iskv {
 
 
 struct CoreSmem {
-  size_t buf, pairs, where, nrm_local, nrm_all, flags, total;
+  size_t buf, pairs, where, nP, nQ, nrm_local, nrm_all, flags, total;
 };
 
-__host__ __device__ inline CoreSmem core_smem(int cj, int w, int ne) {
+// Shared-memory plan (4-byte words). Column blocks are double-buffered when `dbuf` so a round's
+// block exchange needs a single cluster barrier.
+__host__ __device__ inline CoreSmem core_smem(int cj, int w, int ne, bool dbuf) {
   CoreSmem s;
   size_t o = 0;
   auto take = [&](size_t words) { size_t at = o; o += words; return at; };
   const int M = 2 * cj;
-  s.buf = take((size_t)2 * w * 32 * ne);
+  s.buf = take((size_t)(dbuf ? 2 : 1) * 2 * w * 32 * ne);
   s.pairs = take((size_t)(M - 1) * cj * 2);
   s.where = take((size_t)(M - 1) * M);
+  s.nP = take((size_t)w);
+  s.nQ = take((size_t)w);
   s.nrm_local = take((size_t)2 * w);
   s.nrm_all = take((size_t)M * w);
   s.flags = take(4);
   s.total = o * 4;
   return s;
 }
+
+constexpr size_t kCoreSmemCap = 200 * 1024;
 
 JacobiCfg jacobi_cfg(int ncols_max, int col_len_max) {
   JacobiCfg c;
@@ -64,46 +70,70 @@ JacobiCfg jacobi_cfg(int ncols_max, int col_len_max) {
   for (int v : choices)
     if (v >= ne) { ne = v; break; }
   c.ne = ne;
-  c.smem = core_smem(c.cj, c.w, c.ne).total;
+  c.dbuf = core_smem(c.cj, c.w, c.ne, true).total <= kCoreSmemCap;
+  c.smem = core_smem(c.cj, c.w, c.ne, c.dbuf).total;
   return c;
 }
 
-// Rotate the pair of columns x, y (length 32 * NE, this warp) if they are not yet orthogonal to
-// tolerance; the dot products cover the first m entries only.
-template <int NE>
-ISKV_DEV bool warp_rotate_pair(float *x, float *y, int m, double tol) {
+// Dot product of two register-resident columns over their first m entries (float32, the whole
+// warp receives the sum).
+template <int NE, bool DD>
+ISKV_DEV float warp_dot(const float (&x)[NE], const float (&y)[NE], int m) {
   const int lane = threadIdx.x & 31;
-  float xr[NE], yr[NE];
-  double al = 0.0, be = 0.0, ga = 0.0;
+  if (DD) {  // float64 accumulation of the exact float32 products
+    double acc = 0.0;
 #pragma unroll
-  for (int t = 0; t < NE; ++t) {
-    xr[t] = x[lane + 32 * t];
-    yr[t] = y[lane + 32 * t];
-    if (lane + 32 * t < m) {
-      const double xv = xr[t], yv = yr[t];
-      al = fma(xv, xv, al);
-      be = fma(yv, yv, be);
-      ga = fma(xv, yv, ga);
-    }
+    for (int t = 0; t < NE; ++t)
+      if (lane + 32 * t < m) acc = fma((double)x[t], (double)y[t], acc);
+    return (float)warp_sum(acc);
   }
-  al = warp_sum(al);
-  be = warp_sum(be);
-  ga = warp_sum(ga);
-  if (!(ga != 0.0 && fabs(ga) > tol * sqrt(al * be))) return false;
-  double c, s;
-  jacobi_rotation(al, be, ga, c, s);
-  const float cf = (float)c, sf = (float)s;
+  float acc = 0.f;
 #pragma unroll
-  for (int t = 0; t < NE; ++t) {
-    const float xv = xr[t], yv = yr[t];
-    x[lane + 32 * t] = cf * xv - sf * yv;
-    y[lane + 32 * t] = sf * xv + cf * yv;
+  for (int t = 0; t < NE; ++t)
+    if (lane + 32 * t < m) acc = fmaf(x[t], y[t], acc);
+  return warp_sum(acc);
+}
+
+// One Jacobi rotation of the pair (x, y) with squared norms ax, by and inner product g, when the
+// pair is not orthogonal to tolerance. Norms follow Rutishauser: ax -= t g, by += t g.
+template <int NE>
+ISKV_DEV bool rotate_regs(float (&x)[NE], float (&y)[NE], float &ax, float &by, float g, float tol) {
+  if (!(g != 0.f && fabsf(g) > tol * sqrtf(ax) * sqrtf(by))) return false;
+  // The 2 x 2 rotation itself is formed in float64 so that c^2 + s^2 = 1 to float32 rounding:
+  // a biased cosine would shrink or grow both norms on every one of the many rotations.
+  double cd, sd;
+  jacobi_rotation((double)ax, (double)by, (double)g, cd, sd);
+  const float c = (float)cd, s = (float)sd;
+  const float t = (float)(sd / cd);
+#pragma unroll
+  for (int q = 0; q < NE; ++q) {
+    const float xv = x[q], yv = y[q];
+    x[q] = c * xv - s * yv;
+    y[q] = s * xv + c * yv;
   }
+  ax -= t * g;
+  by += t * g;
+  if (ax < 0.f) ax = 0.f;
+  if (by < 0.f) by = 0.f;
   return true;
 }
 
 template <int NE>
-__global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, int w) {
+ISKV_DEV void col_load(float (&x)[NE], const float *src) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < NE; ++q) x[q] = src[lane + 32 * q];
+}
+
+template <int NE>
+ISKV_DEV void col_store(float *dst, const float (&x)[NE]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < NE; ++q) dst[lane + 32 * q] = x[q];
+}
+
+template <int NE, bool DD>
+__global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, int w, int dbuf) {
   cg::cluster_group cluster = cg::this_cluster();
   const int cj = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
   const JobHead &jh = job_head(jobs, p.job_stride, blockIdx.x / cj);
@@ -117,11 +147,13 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
   const int pp = dense ? k : sc[FS_P];          // explicit V rows stored after the A part
   const int m = k + b;                          // A rows
   const int ncol = dense ? k : k + pp, kn = min(r, ncol);
-  const CoreSmem S = core_smem(cj, w, NE);
+  const CoreSmem S = core_smem(cj, w, NE, dbuf != 0);
   extern __shared__ float smem[];
-  float *buf = smem + S.buf;
+  float *buf0 = smem + S.buf;
+  const int bufw = 2 * w * LP;                  // words per buffer
   int *pairs = reinterpret_cast<int *>(smem + S.pairs);   // [M-1][cj][2]
   int *where = reinterpret_cast<int *>(smem + S.where);   // [M-1][M] = cta * 2 + slot
+  float *nP = smem + S.nP, *nQ = smem + S.nQ;
   float *nrm_local = smem + S.nrm_local;
   float *nrm_all = smem + S.nrm_all;
   int *flags = reinterpret_cast<int *>(smem + S.flags);
@@ -146,7 +178,7 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
   const float *C = reinterpret_cast<const float *>(jh.ws + p.C);
   const float *FP = reinterpret_cast<const float *>(jh.ws + p.FP);
   const float *Md = reinterpret_cast<const float *>(jh.ws + p.M);
-  for (int e = tid; e < 2 * w * LP; e += blockDim.x) {
+  for (int e = tid; e < bufw; e += blockDim.x) {
     const int slot = e / (w * LP), lc = (e / LP) % w, el = e % LP;
     const int j = pairs[(0 * cj + rank) * 2 + slot] * w + lc;
     float v = 0.f;
@@ -163,56 +195,107 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
     } else if (el < m + pp) {
       v = (j >= k && j < ncol && el - m == j - k) ? 1.f : 0.f;
     }
-    buf[e] = v;
+    buf0[e] = v;
   }
   __syncthreads();
 
-  const double tol = 2.0 * sqrt((double)(m > 1 ? m : 1)) * 5.960464477539063e-08;
+  // Rotate unless |cos| <= tol. In float32 the inner product has relative error ~ sqrt(m) 2^-24 and
+  // the tolerance sits a few units above it; residual cosines of that size change singular values
+  // only at second order. The dense mode (re-orthogonalisation, whose purpose is orthonormal
+  // factors) accumulates inner products in float64 and uses a tighter tolerance.
+  const float tol = (DD ? 2.f : 4.f) * sqrtf((float)(m > 1 ? m : 1)) * 5.9604645e-08f;
   int sweeps_used = -1;
+  int cur = 0;  // which buffer holds the current blocks (double-buffered exchange)
   for (int sweep = 0; sweep < p.max_sweeps; ++sweep) {
     bool rot = false;
     for (int t = 0; t < M - 1; ++t) {
+      float *buf = buf0 + (dbuf ? cur * bufw : 0);
+      float *Pb = buf, *Qb = buf + w * LP;
+      // Exact squared norms at the start of the round; tracked through the round's rotations.
+      if (warp < w) {
+        float x[NE], y[NE];
+        col_load<NE>(x, Pb + warp * LP);
+        col_load<NE>(y, Qb + warp * LP);
+        const float a = warp_dot<NE, DD>(x, x, m), c = warp_dot<NE, DD>(y, y, m);
+        if (lane == 0) { nP[warp] = a; nQ[warp] = c; }
+      }
+      __syncthreads();
       if (t == 0) {
+        // Pairs inside each block (both columns from shared memory).
         for (int st = 0; st < w - 1; ++st) {
           if (warp < w) {
             const int slot = warp < w / 2 ? 0 : 1, q = warp % (w / 2);
             const int a = circle_player(q, st, w), bb = circle_player(w - 1 - q, st, w);
-            rot |= warp_rotate_pair<NE>(buf + (slot * w + a) * LP, buf + (slot * w + bb) * LP, m,
-                                        tol);
+            float *base = slot ? Qb : Pb;
+            float *nb = slot ? nQ : nP;
+            float x[NE], y[NE];
+            col_load<NE>(x, base + a * LP);
+            col_load<NE>(y, base + bb * LP);
+            float ax = nb[a], by = nb[bb];
+            const float g = warp_dot<NE, DD>(x, y, m);
+            if (rotate_regs<NE>(x, y, ax, by, g, tol)) {
+              col_store<NE>(base + a * LP, x);
+              col_store<NE>(base + bb * LP, y);
+              if (lane == 0) { nb[a] = ax; nb[bb] = by; }
+              rot = true;
+            }
           }
           __syncthreads();
         }
       }
+      // Cross pairs: warp i keeps P[i] in registers while the Q columns circulate.
+      float x[NE];
+      float ax = 0.f;
+      if (warp < w) {
+        col_load<NE>(x, Pb + warp * LP);
+        ax = nP[warp];
+      }
       for (int st = 0; st < w; ++st) {
         if (warp < w) {
-          const int bb = (warp + st) % w;
-          rot |= warp_rotate_pair<NE>(buf + warp * LP, buf + (w + bb) * LP, m, tol);
+          const int q = (warp + st) % w;
+          float y[NE];
+          col_load<NE>(y, Qb + q * LP);
+          float by = nQ[q];
+          const float g = warp_dot<NE, DD>(x, y, m);
+          if (rotate_regs<NE>(x, y, ax, by, g, tol)) {
+            col_store<NE>(Qb + q * LP, y);
+            if (lane == 0) nQ[q] = by;
+            rot = true;
+          }
         }
         __syncthreads();
       }
-      if (cj > 1) {
-        // Move both blocks to where round t+1 needs them (single buffer: read, barrier, write).
-        const int tn = (t + 1) % (M - 1);
-        float reg[2][NE];
-        int dst[2];
-#pragma unroll
-        for (int slot = 0; slot < 2; ++slot) {
-          const int X = pairs[(t * cj + rank) * 2 + slot];
-          dst[slot] = where[tn * M + X];
-          if (dst[slot] != rank * 2 + slot && warp < w) {
-#pragma unroll
-            for (int q = 0; q < NE; ++q) reg[slot][q] = buf[(slot * w + warp) * LP + lane + 32 * q];
-          }
+      if (cj == 1) {
+        if (warp < w) col_store<NE>(Pb + warp * LP, x);
+        __syncthreads();
+        continue;
+      }
+      // Move both blocks to where round t+1 needs them.
+      const int tn = (t + 1) % (M - 1);
+      const int X0 = pairs[(t * cj + rank) * 2 + 0], X1 = pairs[(t * cj + rank) * 2 + 1];
+      const int d0 = where[tn * M + X0], d1 = where[tn * M + X1];
+      if (dbuf) {
+        // Write straight into the destination's other buffer; nobody reads it this round.
+        if (warp < w) {
+          float y[NE];
+          col_load<NE>(y, Qb + warp * LP);
+          float *r0 = cluster.map_shared_rank(buf0, d0 >> 1) + (cur ^ 1) * bufw + ((d0 & 1) * w + warp) * LP;
+          float *r1 = cluster.map_shared_rank(buf0, d1 >> 1) + (cur ^ 1) * bufw + ((d1 & 1) * w + warp) * LP;
+          col_store<NE>(r0, x);
+          col_store<NE>(r1, y);
         }
         cluster.sync();
-#pragma unroll
-        for (int slot = 0; slot < 2; ++slot) {
-          if (dst[slot] != rank * 2 + slot && warp < w) {
-            const int dc = dst[slot] >> 1, ds = dst[slot] & 1;
-            float *rb = cluster.map_shared_rank(buf, dc) + (ds * w + warp) * LP;
-#pragma unroll
-            for (int q = 0; q < NE; ++q) rb[lane + 32 * q] = reg[slot][q];
-          }
+        cur ^= 1;
+      } else {
+        // Single buffer: read everything, barrier, then write.
+        float y[NE];
+        if (warp < w) col_load<NE>(y, Qb + warp * LP);
+        cluster.sync();
+        if (warp < w) {
+          float *r0 = cluster.map_shared_rank(buf0, d0 >> 1) + ((d0 & 1) * w + warp) * LP;
+          float *r1 = cluster.map_shared_rank(buf0, d1 >> 1) + ((d1 & 1) * w + warp) * LP;
+          col_store<NE>(r0, x);
+          col_store<NE>(r1, y);
         }
         cluster.sync();
       }
@@ -228,6 +311,7 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
       break;
     }
   }
+  float *buf = buf0 + (dbuf ? cur * bufw : 0);
 
   // Column norms of my columns (blocks are at their round-0 places again).
   for (int slot = 0; slot < 2; ++slot) {
@@ -316,7 +400,7 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
 template <int NE>
 static cudaError_t core_launch(const char *jobs, const CoreParams &p, const JacobiCfg &c,
                                cudaStream_t s) {
-  auto kern = k_core<NE>;
+  auto kern = p.mode == 1 ? k_core<NE, true> : k_core<NE, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)c.smem);
   if (e != cudaSuccess) return e;
@@ -337,7 +421,7 @@ static cudaError_t core_launch(const char *jobs, const CoreParams &p, const Jaco
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   count_launches(1);
-  return cudaLaunchKernelEx(&cfg, kern, jobs, p, c.w);
+  return cudaLaunchKernelEx(&cfg, kern, jobs, p, c.w, c.dbuf ? 1 : 0);
 }
 
 cudaError_t launch_core(const char *jobs, const CoreParams &p, cudaStream_t s) {

@@ -38,6 +38,7 @@ struct JacobiCfg {
   int cj;         // CTAs per cluster
   int w;          // columns per block (two blocks per CTA)
   int ne;         // column elements per lane (column buffer = 32 * ne floats)
+  bool dbuf;      // double-buffered block exchange (one cluster barrier per round)
   size_t smem;    // dynamic shared memory bytes
 };
 

@@ -172,6 +172,33 @@ __global__ void __launch_bounds__(256) k_ns_step(const ReorthJob *jobs, ReorthPa
   }
 }
 
+// Convergence check of the iteration: the last T = 1.5 I - 0.5 Z Y must be I to working accuracy
+// (quadratic convergence from a Gram matrix within ~10% of a multiple of I needs 4 iterations).
+__global__ void k_ns_check(const ReorthJob *jobs, ReorthParams p) {
+  const int job = blockIdx.x >> 1, which = blockIdx.x & 1;
+  const ReorthJob &jb = jobs[job];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], r = p.r;
+  const float *T = reinterpret_cast<const float *>(jb.h.ws + p.ws.T[which]);
+  float worst = 0.f;
+  for (int e = threadIdx.x; e < k * k; e += blockDim.x) {
+    const int i = e / k, j = e % k;
+    const float v = T[(size_t)i * r + j] - (i == j ? 1.f : 0.f);
+    worst = fmaxf(worst, fabsf(v));
+  }
+  __shared__ float wmax[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) worst = fmaxf(worst, __shfl_xor_sync(0xffffffffu, worst, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = worst;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
+    if (!(m <= 1e-3f)) record_status(jb.h.meta, ISKV_ERR_NOT_CONVERGED);
+  }
+}
+
 // M = sqrt(c_u c_b) Y_u diag(sigma) Y_b  (= R_U diag(sigma) R_B^T with symmetric R_B).
 __global__ void __launch_bounds__(256) k_reorth_M(const ReorthJob *jobs, ReorthParams p,
                                                   size_t yu, size_t yb) {
@@ -264,8 +291,9 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
       t = z0[w]; z0[w] = z1[w]; z1[w] = t;
     }
   }
+  k_ns_check<<<p.count * 2, 256, 0, s>>>(jobs, p);
   k_reorth_M<<<dim3(tn, tm, p.count), 256, 0, s>>>(jobs, p, y0[0], y0[1]);
-  count_launches(2 + 2 * NS_ITERS);
+  count_launches(3 + 2 * NS_ITERS);
   stage_mark(s, ST_REORTH_NS);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

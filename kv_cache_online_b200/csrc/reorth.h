@@ -7,7 +7,7 @@
 namespace iskv {
 
 constexpr int REORTH_SPLIT = 1024;  // rows per Gram partial
-constexpr int NS_ITERS = 8;         // coupled Newton-Schulz iterations
+constexpr int NS_ITERS = 5;         // coupled Newton-Schulz iterations
 
 struct ReorthWsLayout {
   size_t scal, gpart_u, gpart_b, G[2], Y[2], Z[2], T[2], Y2[2], Z2[2], M, Gt, Gtb, Ht, sig, TUt,
