@@ -51,7 +51,7 @@ enum { ISKV_META_K = 0, ISKV_META_N = 1, ISKV_META_FOLDS = 2, ISKV_META_STATUS =
  * One compressed history: one (sequence, layer, K|V) path, the factors U diag(sigma) B^T of
  * Section 2.2 ("iS-KV reading notes"), rank k <= r_max, n compressed rows.
  *   U      [n_cap][r_max]  storage dtype; row i = coordinates of compressed row i. Must be
- *                          zero-initialised (columns >= k are read as zero).
+ *                          zero-initialised: columns >= k and rows >= n are read as zero.
  *   sigma  [r_max]         float32, descending; entries >= k are zero.
  *   B      [d][r_max]      storage dtype; column j = basis vector j. Zero-initialised.
  *   pos    [n_cap]         int32 original token position of U row i (Section 3.2: K and V
@@ -196,7 +196,7 @@ iskv_status iskv_select_prompt_blocks_noalloc(const void *keys, int32_t k_dtype,
                                               int32_t *head_blocks_out, int64_t *counts_out,
                                               void *stream);
 
-/* Zero a history's meta word and sigma (stream-ordered). U and B are not touched. */
+/* Empty a history: zero its meta word, sigma, U and B (stream-ordered). */
 iskv_status iskv_reset(const iskv_lowrank *h, void *stream);
 
 /*

@@ -208,7 +208,7 @@ iskv_status iskv_fold_block(const iskv_lowrank *h, const void *F, int32_t f_dtyp
 size_t iskv_reorth_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap) {
   if (count < 1 || d < 1 || r_max < 1 || n_cap < 0) return 0;
   const ReorthWsLayout L = reorth_ws_layout(d, r_max, n_cap);
-  return jobs_bytes(count, sizeof(ReorthJob)) + tc_table_bytes(count) + (size_t)count * L.total;
+  return jobs_bytes(count, sizeof(ReorthJob)) + 2 * tc_table_bytes(count) + (size_t)count * L.total;
 }
 
 iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t ws_bytes,
@@ -238,7 +238,9 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   p.ws = reorth_ws_layout(d, r, ncap);
   char *base = static_cast<char *>(ws);
   TcJob *tc_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReorthJob)));
-  const size_t jb = jobs_bytes(count, sizeof(ReorthJob)) + tc_table_bytes(count);
+  TcJob *gram_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReorthJob)) +
+                                              tc_table_bytes(count));
+  const size_t jb = jobs_bytes(count, sizeof(ReorthJob)) + 2 * tc_table_bytes(count);
   std::vector<ReorthJob> jobs(count);
   for (int32_t i = 0; i < count; ++i) {
     ReorthJob &j = jobs[i];
@@ -251,9 +253,20 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
     j.n_cap = hs[i].n_cap;
     j.pad_ = 0;
   }
-  std::vector<TcJob> tj;
+  std::vector<TcJob> tj, gj;
   p.tc_host = nullptr;
   p.tc_dev = tc_dev;
+  p.gram_host = nullptr;
+  p.gram_dev = gram_dev;
+  if (tc_gram_supported(r, p.storage)) {
+    gj.resize(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_gram_job(gj[i], hs[i].U, hs[i].n_cap, hs[i].B, d, r,
+                           reinterpret_cast<const int32_t *>(jobs[i].h.ws + p.ws.scal), hs[i].meta,
+                           jobs[i].h.ws))
+        return fail(ISKV_ERR_CUDA, "reorth: tensor map encoding failed");
+    p.gram_host = gj.data();
+  }
   if (tc_rotation_supported(r, p.storage)) {
     tj.resize(count);
     for (int32_t i = 0; i < count; ++i)
@@ -444,8 +457,11 @@ iskv_status iskv_reset(const iskv_lowrank *h, void *stream) {
   iskv_status st = check_handle(h, "iskv_reset");
   if (st != ISKV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t es = h->storage == ISKV_BF16 ? 2 : 4;
   cudaError_t e = cudaMemsetAsync(h->meta, 0, 4 * sizeof(int64_t), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->sigma, 0, sizeof(float) * h->r_max, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->U, 0, es * (size_t)h->n_cap * h->r_max, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->B, 0, es * (size_t)h->d * h->r_max, s);
   if (e != cudaSuccess) return cuda_fail(e, "iskv_reset");
   return ISKV_OK;
 }

@@ -98,7 +98,9 @@ __global__ void k_gram_reduce(const ReorthJob *jobs, ReorthParams p) {
   const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
   if (sc[FS_SKIP]) return;
   const int k = sc[FS_K_OLD], r = p.r;
-  const int ns = which == 0 ? p.ws.nsplit_u : p.ws.nsplit_b;
+  const int rows = which == 0 ? sc[FS_N_OLD] : p.d;
+  const int ns = min(which == 0 ? p.ws.nsplit_u : p.ws.nsplit_b,
+                     (rows + REORTH_SPLIT - 1) / REORTH_SPLIT);  // splits that hold rows
   const float *part = reinterpret_cast<const float *>(jb.h.ws + (which == 0 ? p.ws.gpart_u : p.ws.gpart_b));
   float *G = reinterpret_cast<float *>(jb.h.ws + p.ws.G[which]);
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < k * k; e += gridDim.x * blockDim.x) {
@@ -268,15 +270,29 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   const ReorthWsLayout &W = p.ws;
   k_reorth_prepare<<<(p.count + 127) / 128, 128, 0, s>>>(jobs, p);
   const unsigned tn = (r + GBN - 1) / GBN, tm = (r + GBM - 1) / GBM;
-  if (p.storage == ISKV_BF16) {
+  if (p.gram_host) {
+    GramParams gp;
+    gp.r = r;
+    gp.d = p.d;
+    gp.count = p.count;
+    gp.nsu = W.nsplit_u;
+    gp.nsb = W.nsplit_b;
+    gp.split = REORTH_SPLIT;
+    gp.off_gu = W.gpart_u;
+    gp.off_gb = W.gpart_b;
+    cudaError_t e0 = launch_tc_gram(p.gram_host, p.gram_dev, gp, s);
+    if (e0 != cudaSuccess) return e0;
+  } else if (p.storage == ISKV_BF16) {
     k_gram_partial<__nv_bfloat16><<<dim3(tn, tm, p.count * W.nsplit_u), 256, 0, s>>>(jobs, p, 0, W.nsplit_u);
     k_gram_partial<__nv_bfloat16><<<dim3(tn, tm, p.count * W.nsplit_b), 256, 0, s>>>(jobs, p, 1, W.nsplit_b);
+    count_launches(2);
   } else {
     k_gram_partial<float><<<dim3(tn, tm, p.count * W.nsplit_u), 256, 0, s>>>(jobs, p, 0, W.nsplit_u);
     k_gram_partial<float><<<dim3(tn, tm, p.count * W.nsplit_b), 256, 0, s>>>(jobs, p, 1, W.nsplit_b);
+    count_launches(2);
   }
   k_gram_reduce<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
-  count_launches(4);
+  count_launches(2);
   stage_mark(s, ST_REORTH_GRAM);
   k_ns_init<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
   size_t y0[2] = {W.Y[0], W.Y[1]}, z0[2] = {W.Z[0], W.Z[1]};

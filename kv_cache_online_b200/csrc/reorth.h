@@ -6,7 +6,7 @@
 
 namespace iskv {
 
-constexpr int REORTH_SPLIT = 1024;  // rows per Gram partial
+constexpr int REORTH_SPLIT = 2048;  // rows per Gram partial
 constexpr int NS_ITERS = 5;         // coupled Newton-Schulz iterations
 
 struct ReorthWsLayout {
@@ -21,8 +21,10 @@ struct ReorthParams {
   int d, r, storage, count;
   int64_t n_cap;
   ReorthWsLayout ws;
-  const TcJob *tc_host;  // tensor-core coordinate rotation jobs (host copy) or null
-  TcJob *tc_dev;         // their device table
+  const TcJob *tc_host;    // tensor-core coordinate rotation jobs (host copy) or null
+  TcJob *tc_dev;           // their device table
+  const TcJob *gram_host;  // tensor-core Gram jobs (host copy) or null
+  TcJob *gram_dev;         // their device table
 };
 
 cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s);

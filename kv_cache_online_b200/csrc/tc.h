@@ -30,6 +30,19 @@ struct TcParams {
   double theta;
 };
 
+// Gram partials for the re-orthogonalisation: `count` jobs, each with nsu splits of U rows and nsb
+// splits of B rows (`split` rows each); outputs at byte offsets off_gu / off_gb of the job's
+// workspace (TcJob::out), one r x r float32 matrix per split.
+struct GramParams {
+  int r, d, count, nsu, nsb, split;
+  size_t off_gu, off_gb;
+};
+
+bool tc_gram_supported(int r, int storage);
+bool encode_gram_job(TcJob &tj, const void *U, int64_t n_cap, const void *B, int d, int r,
+                     const int32_t *sc, int64_t *meta, void *ws);
+cudaError_t launch_tc_gram(const TcJob *hjobs, TcJob *djobs, const GramParams &p, cudaStream_t s);
+
 bool tc_rotation_supported(int r, int storage);
 bool tc_recon_supported(int r, int storage, int out_dtype, int head_dim);
 

@@ -395,6 +395,119 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
   if (warp == 1) tmem_dealloc(tmem, NCOLS);
 }
 
+// ================================================================================================
+// Gram matrices for the re-orthogonalisation: G = X^T X over the rows of X = U (n rows) or B (d
+// rows). The contraction runs over rows, so both operands are read MN-major: a TMA box of 64 rows
+// x 64 columns is one MN-major stack of 128-byte rows, slabs of 64 columns sit 8 KB apart. Each
+// CTA reduces one split of up to GRAM_SPLIT rows into an r x r float32 partial (two M = 128,
+// N = r accumulators in tensor memory); a second kernel sums the partials.
+constexpr int GRAM_THREADS = 192;  // producer warp, MMA warp, 4 epilogue warps
+constexpr int GRAM_STAGES = 4;
+constexpr int GRAM_KT = 64;        // rows per pipeline stage
+
+__global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, GramParams p) {
+  const int per_job = p.nsu + p.nsb;
+  const int job = blockIdx.x / per_job, rem = blockIdx.x % per_job;
+  const int which = rem < p.nsu ? 0 : 1, split = which ? rem - p.nsu : rem;
+  const TcJob &jb = jobs[job];
+  const int32_t *sc = jb.sc;
+  const int R = p.r, SL = R / 64, MH = R / 128, N = R;
+  const int rows_total = which ? p.d : sc[FS_N_OLD];
+  const int r0 = split * p.split;
+  const int nrows = min(p.split, rows_total - r0);
+  if (sc[FS_SKIP] || nrows <= 0 || sc[FS_K_OLD] == 0) return;  // uniform over the CTA
+  const int nk = (nrows + GRAM_KT - 1) / GRAM_KT;
+  const CUtensorMap *map = which ? &jb.mapB : &jb.mapA;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int STAGE_BYTES = SL * GRAM_KT * 128;
+  TcCtl *ctl = reinterpret_cast<TcCtl *>(smem + GRAM_STAGES * STAGE_BYTES);
+  uint64_t *full = reinterpret_cast<uint64_t *>(ctl + 1);   // [GRAM_STAGES]
+  uint64_t *empty = full + GRAM_STAGES;                      // [GRAM_STAGES]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = MH * N <= 128 ? 128 : (MH * N <= 256 ? 256 : 512);
+  const uint32_t idesc = idesc_bf16_f32_mn(128, N);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < GRAM_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(&ctl->acc_full[0], 1);
+    mbar_init(&ctl->done, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&ctl->tmem, ncols);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int *abort = &ctl->abort;
+
+  if (warp == 0 && lane == 0) {
+    tensormap_acquire(map);
+    for (int kt = 0; kt < nk && !*abort; ++kt) {
+      const int st = kt % GRAM_STAGES, use = kt / GRAM_STAGES;
+      if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, abort, WAIT_NS)) {
+        fail_timeout(ctl, jb.meta);
+        break;
+      }
+      mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
+      for (int sl = 0; sl < SL; ++sl)
+        tma_load_2d(smem + st * STAGE_BYTES + sl * GRAM_KT * 128, map, sl * 64, r0 + kt * GRAM_KT,
+                    &full[st]);
+    }
+    for (int k = 1; k <= GRAM_STAGES && nk - k >= 0; ++k)
+      mbar_wait(&full[(nk - k) % GRAM_STAGES], ((nk - k) / GRAM_STAGES) & 1, abort, WAIT_NS / 4);
+  } else if (warp == 1 && lane == 0) {
+    bool ok = true;
+    for (int kt = 0; kt < nk && ok && !*abort; ++kt) {
+      const int st = kt % GRAM_STAGES, use = kt / GRAM_STAGES;
+      if (!mbar_wait(&full[st], use & 1, abort, WAIT_NS)) { ok = false; break; }
+      fence_after_sync();
+      const uint32_t base = smem_u32(smem + st * STAGE_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < GRAM_KT / 16; ++kk) {
+        const uint64_t bdesc = sw128_mn_desc(base + kk * 2048, GRAM_KT * 128);
+        for (int h = 0; h < MH; ++h) {
+          const uint64_t adesc = sw128_mn_desc(base + h * 2 * GRAM_KT * 128 + kk * 2048, GRAM_KT * 128);
+          mma_bf16(tmem + h * N, adesc, bdesc, idesc, (kt | kk) != 0);
+        }
+      }
+      mma_commit(&empty[st]);
+    }
+    if (!ok) fail_timeout(ctl, jb.meta);
+    mma_commit(&ctl->acc_full[0]);
+    mma_commit(&ctl->done);
+    mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
+  } else if (warp >= 2) {
+    const int q = warp & 3;
+    float *out = reinterpret_cast<float *>(jb.out) +
+                 (which ? p.off_gb : p.off_gu) / sizeof(float) + (size_t)split * R * R;
+    if (mbar_wait(&ctl->acc_full[0], 0, abort, WAIT_NS) && !*abort) {
+      fence_after_sync();
+      for (int h = 0; h < MH; ++h) {
+        const int row = h * 128 + q * 32 + lane;
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + h * N + ((uint32_t)(q * 32) << 16) + c0, v);
+          tmem_ld_wait();
+          float4 *dst = reinterpret_cast<float4 *>(out + (size_t)row * R + c0);
+          dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+          dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+          dst[2] = make_float4(v[8], v[9], v[10], v[11]);
+          dst[3] = make_float4(v[12], v[13], v[14], v[15]);
+        }
+      }
+    } else {
+      fail_timeout(ctl, jb.meta);
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
 // Sigma-scaled basis for the reconstruction: bsig[c][l] = bf16(sigma_l * B[c][l]) for l < k, else 0.
 __global__ void k_bsig(const ReconJob *jobs, int d, int r) {
   const ReconJob &jb = jobs[blockIdx.y];
@@ -531,6 +644,33 @@ cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob
   const int total = tp.count * tp.tiles_per_job;
   const int grid = total < num_sms() ? total : num_sms();
   k_rec_tc<<<grid, TC_THREADS, smem, s>>>(djobs, tp);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+bool tc_gram_supported(int r, int storage) {
+  return storage == ISKV_BF16 && (r == 128 || r == 256) && encode_fn() != nullptr;
+}
+
+bool encode_gram_job(TcJob &tj, const void *U, int64_t n_cap, const void *B, int d, int r,
+                     const int32_t *sc, int64_t *meta, void *ws) {
+  std::memset(&tj, 0, sizeof(tj));
+  if (!encode_2d(&tj.mapA, U, (uint64_t)n_cap, (uint64_t)r, GRAM_KT)) return false;
+  if (!encode_2d(&tj.mapB, B, (uint64_t)d, (uint64_t)r, GRAM_KT)) return false;
+  tj.sc = sc;
+  tj.meta = meta;
+  tj.out = ws;
+  return true;
+}
+
+cudaError_t launch_tc_gram(const TcJob *hjobs, TcJob *djobs, const GramParams &p, cudaStream_t s) {
+  cudaError_t e = upload_jobs(djobs, hjobs, sizeof(TcJob) * p.count, s);
+  if (e != cudaSuccess) return e;
+  const size_t smem = 1024 + (size_t)GRAM_STAGES * (p.r / 64) * GRAM_KT * 128 + sizeof(TcCtl) +
+                      2 * GRAM_STAGES * sizeof(uint64_t);
+  e = cudaFuncSetAttribute(k_gram_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_gram_tc<<<p.count * (p.nsu + p.nsb), GRAM_THREADS, smem, s>>>(djobs, p);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -120,6 +120,25 @@ ISKV_DEV uint64_t sw128_desc(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor: MN-major, 128-byte swizzle. The tile is stored as 64-element
+// (128-byte) MN slabs of consecutive K rows; 8-row atoms are 1024 bytes apart (stride byte offset)
+// and consecutive MN slabs `slab_bytes` apart (leading byte offset).
+ISKV_DEV uint64_t sw128_mn_desc(uint32_t smem_addr, uint32_t slab_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((slab_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next MN slab
+  d |= (uint64_t)(1024 >> 4) << 32;                     // stride byte offset: next 8 K rows
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, both operands MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
