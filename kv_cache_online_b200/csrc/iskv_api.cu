@@ -122,7 +122,7 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
     return fail(ISKV_ERR_SHAPE, "%s: d = %d with b = %d exceeds the residual QR cluster", who, d, b);
   {
     const JacobiCfg jc = jacobi_cfg(r + b, r + 2 * b);
-    if (jc.smem > 200 * 1024 || 32 * jc.w > 640)
+    if (jc.smem > 200 * 1024 || 16 * jc.w > 640)
       return fail(ISKV_ERR_SHAPE, "%s: r_max + b too large for the core SVD cluster", who);
   }
   const size_t need = iskv_fold_workspace_size(count, d, r, b);

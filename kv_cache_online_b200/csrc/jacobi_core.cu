@@ -51,16 +51,19 @@ __host__ __device__ inline CoreSmem core_smem(int cj, int w, int ne, bool dbuf) 
 }
 
 constexpr size_t kCoreSmemCap = 200 * 1024;
+constexpr int kMaxWarps = 20;  // register budget: 96 registers x 640 threads
 
+// Columns per block w (two blocks per CTA, two column pairs per warp, so w / 2 warps).
 JacobiCfg jacobi_cfg(int ncols_max, int col_len_max) {
   JacobiCfg c;
   int cj = 1;
   for (;;) {
     int w = (ncols_max + 2 * cj - 1) / (2 * cj);
     w += w & 1;
-    if (w <= 20 || cj == 16) {
+    if (w < 4) w = 4;
+    if (w <= 2 * kMaxWarps || cj == 16) {
       c.cj = cj;
-      c.w = w < 2 ? 2 : w;
+      c.w = w;
       break;
     }
     cj *= 2;
@@ -75,41 +78,62 @@ JacobiCfg jacobi_cfg(int ncols_max, int col_len_max) {
   return c;
 }
 
-// Dot product of two register-resident columns over their first m entries (float32, the whole
-// warp receives the sum).
+// Dot product of two register-resident columns over their first m entries, two accumulators
+// (shorter dependency chain); the whole warp receives the sum.
 template <int NE, bool DD>
 ISKV_DEV float warp_dot(const float (&x)[NE], const float (&y)[NE], int m) {
   const int lane = threadIdx.x & 31;
   if (DD) {  // float64 accumulation of the exact float32 products
-    double acc = 0.0;
+    double a0 = 0.0, a1 = 0.0;
 #pragma unroll
     for (int t = 0; t < NE; ++t)
-      if (lane + 32 * t < m) acc = fma((double)x[t], (double)y[t], acc);
-    return (float)warp_sum(acc);
+      if (lane + 32 * t < m) {
+        if (t & 1) a1 = fma((double)x[t], (double)y[t], a1);
+        else a0 = fma((double)x[t], (double)y[t], a0);
+      }
+    return (float)warp_sum(a0 + a1);
   }
-  float acc = 0.f;
+  float a0 = 0.f, a1 = 0.f;
 #pragma unroll
   for (int t = 0; t < NE; ++t)
-    if (lane + 32 * t < m) acc = fmaf(x[t], y[t], acc);
-  return warp_sum(acc);
+    if (lane + 32 * t < m) {
+      if (t & 1) a1 = fmaf(x[t], y[t], a1);
+      else a0 = fmaf(x[t], y[t], a0);
+    }
+  return warp_sum(a0 + a1);
 }
 
 // One Jacobi rotation of the pair (x, y) with squared norms ax, by and inner product g, when the
-// pair is not orthogonal to tolerance. Norms follow Rutishauser: ax -= t g, by += t g.
-template <int NE>
+// pair is not orthogonal to tolerance. Applied in the half-angle form
+//   x' = x - s (y + tau x),  y' = y + s (x - tau y),  tau = tan(theta / 2) = s / (1 + c),
+// which equals (c x - s y, s x + c y) but keeps the rotation orthogonal even when c rounds to 1 in
+// float32 (a plain c = 1, s = t would grow both norms by t^2 / 2 on every small rotation). Norms
+// follow Rutishauser: ax -= t g, by += t g.
+template <int NE, bool DD>
 ISKV_DEV bool rotate_regs(float (&x)[NE], float (&y)[NE], float &ax, float &by, float g, float tol) {
   if (!(g != 0.f && fabsf(g) > tol * sqrtf(ax) * sqrtf(by))) return false;
-  // The 2 x 2 rotation itself is formed in float64 so that c^2 + s^2 = 1 to float32 rounding:
-  // a biased cosine would shrink or grow both norms on every one of the many rotations.
-  double cd, sd;
-  jacobi_rotation((double)ax, (double)by, (double)g, cd, sd);
-  const float c = (float)cd, s = (float)sd;
-  const float t = (float)(sd / cd);
+  float t, s, tau;
+  if (DD) {
+    const double zeta = ((double)by - (double)ax) / (2.0 * (double)g);
+    const double td = fabs(zeta) > 1e100 ? 0.5 / zeta
+                                         : (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
+    const double sq = sqrt(1.0 + td * td);
+    t = (float)td;
+    s = (float)(td / sq);
+    tau = (float)(td / (1.0 + sq));
+  } else {
+    const float zeta = (by - ax) / (2.f * g);
+    t = fabsf(zeta) > 1e18f ? 0.5f / zeta
+                            : copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
+    const float sq = sqrtf(fmaf(t, t, 1.f));
+    s = t / sq;
+    tau = t / (1.f + sq);
+  }
 #pragma unroll
   for (int q = 0; q < NE; ++q) {
     const float xv = x[q], yv = y[q];
-    x[q] = c * xv - s * yv;
-    y[q] = s * xv + c * yv;
+    x[q] = fmaf(-s, fmaf(tau, xv, yv), xv);
+    y[q] = fmaf(s, fmaf(-tau, yv, xv), yv);
   }
   ax -= t * g;
   by += t * g;
@@ -158,6 +182,8 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
   float *nrm_all = smem + S.nrm_all;
   int *flags = reinterpret_cast<int *>(smem + S.flags);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = w / 2;                         // warps; warp i owns columns i and i + nw
+  const int c0 = warp, c1 = warp + nw;
 
   // Tournament: round t, CTA 0 plays block M-1 against block t; CTA i plays (t+i) vs (t-i).
   for (int e = tid; e < (M - 1) * cj; e += blockDim.x) {
@@ -212,19 +238,26 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
       float *buf = buf0 + (dbuf ? cur * bufw : 0);
       float *Pb = buf, *Qb = buf + w * LP;
       // Exact squared norms at the start of the round; tracked through the round's rotations.
-      if (warp < w) {
+      {
         float x[NE], y[NE];
-        col_load<NE>(x, Pb + warp * LP);
-        col_load<NE>(y, Qb + warp * LP);
-        const float a = warp_dot<NE, DD>(x, x, m), c = warp_dot<NE, DD>(y, y, m);
-        if (lane == 0) { nP[warp] = a; nQ[warp] = c; }
+        col_load<NE>(x, Pb + c0 * LP);
+        col_load<NE>(y, Qb + c0 * LP);
+        float a = warp_dot<NE, DD>(x, x, m), c = warp_dot<NE, DD>(y, y, m);
+        if (lane == 0) { nP[c0] = a; nQ[c0] = c; }
+        col_load<NE>(x, Pb + c1 * LP);
+        col_load<NE>(y, Qb + c1 * LP);
+        a = warp_dot<NE, DD>(x, x, m);
+        c = warp_dot<NE, DD>(y, y, m);
+        if (lane == 0) { nP[c1] = a; nQ[c1] = c; }
       }
       __syncthreads();
       if (t == 0) {
-        // Pairs inside each block (both columns from shared memory).
+        // Pairs inside each block (both columns from shared memory); pair indices c0 and c1.
         for (int st = 0; st < w - 1; ++st) {
-          if (warp < w) {
-            const int slot = warp < w / 2 ? 0 : 1, q = warp % (w / 2);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int pi = u ? c1 : c0;
+            const int slot = pi < w / 2 ? 0 : 1, q = pi % (w / 2);
             const int a = circle_player(q, st, w), bb = circle_player(w - 1 - q, st, w);
             float *base = slot ? Qb : Pb;
             float *nb = slot ? nQ : nP;
@@ -233,7 +266,7 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
             col_load<NE>(y, base + bb * LP);
             float ax = nb[a], by = nb[bb];
             const float g = warp_dot<NE, DD>(x, y, m);
-            if (rotate_regs<NE>(x, y, ax, by, g, tol)) {
+            if (rotate_regs<NE, DD>(x, y, ax, by, g, tol)) {
               col_store<NE>(base + a * LP, x);
               col_store<NE>(base + bb * LP, y);
               if (lane == 0) { nb[a] = ax; nb[bb] = by; }
@@ -243,30 +276,34 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
           __syncthreads();
         }
       }
-      // Cross pairs: warp i keeps P[i] in registers while the Q columns circulate.
-      float x[NE];
-      float ax = 0.f;
-      if (warp < w) {
-        col_load<NE>(x, Pb + warp * LP);
-        ax = nP[warp];
-      }
+      // Cross pairs: warp i keeps P[i] and P[i + w/2] in registers while the Q columns circulate.
+      float x0[NE], x1[NE];
+      col_load<NE>(x0, Pb + c0 * LP);
+      col_load<NE>(x1, Pb + c1 * LP);
+      float ax0 = nP[c0], ax1 = nP[c1];
       for (int st = 0; st < w; ++st) {
-        if (warp < w) {
-          const int q = (warp + st) % w;
-          float y[NE];
-          col_load<NE>(y, Qb + q * LP);
-          float by = nQ[q];
-          const float g = warp_dot<NE, DD>(x, y, m);
-          if (rotate_regs<NE>(x, y, ax, by, g, tol)) {
-            col_store<NE>(Qb + q * LP, y);
-            if (lane == 0) nQ[q] = by;
-            rot = true;
-          }
+        const int q0 = (c0 + st) % w, q1 = (c1 + st) % w;
+        float y0[NE], y1[NE];
+        col_load<NE>(y0, Qb + q0 * LP);
+        col_load<NE>(y1, Qb + q1 * LP);
+        float by0 = nQ[q0], by1 = nQ[q1];
+        const float g0 = warp_dot<NE, DD>(x0, y0, m);
+        const float g1 = warp_dot<NE, DD>(x1, y1, m);
+        if (rotate_regs<NE, DD>(x0, y0, ax0, by0, g0, tol)) {
+          col_store<NE>(Qb + q0 * LP, y0);
+          if (lane == 0) nQ[q0] = by0;
+          rot = true;
+        }
+        if (rotate_regs<NE, DD>(x1, y1, ax1, by1, g1, tol)) {
+          col_store<NE>(Qb + q1 * LP, y1);
+          if (lane == 0) nQ[q1] = by1;
+          rot = true;
         }
         __syncthreads();
       }
       if (cj == 1) {
-        if (warp < w) col_store<NE>(Pb + warp * LP, x);
+        col_store<NE>(Pb + c0 * LP, x0);
+        col_store<NE>(Pb + c1 * LP, x1);
         __syncthreads();
         continue;
       }
@@ -274,31 +311,21 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
       const int tn = (t + 1) % (M - 1);
       const int X0 = pairs[(t * cj + rank) * 2 + 0], X1 = pairs[(t * cj + rank) * 2 + 1];
       const int d0 = where[tn * M + X0], d1 = where[tn * M + X1];
-      if (dbuf) {
-        // Write straight into the destination's other buffer; nobody reads it this round.
-        if (warp < w) {
-          float y[NE];
-          col_load<NE>(y, Qb + warp * LP);
-          float *r0 = cluster.map_shared_rank(buf0, d0 >> 1) + (cur ^ 1) * bufw + ((d0 & 1) * w + warp) * LP;
-          float *r1 = cluster.map_shared_rank(buf0, d1 >> 1) + (cur ^ 1) * bufw + ((d1 & 1) * w + warp) * LP;
-          col_store<NE>(r0, x);
-          col_store<NE>(r1, y);
-        }
-        cluster.sync();
-        cur ^= 1;
-      } else {
-        // Single buffer: read everything, barrier, then write.
-        float y[NE];
-        if (warp < w) col_load<NE>(y, Qb + warp * LP);
-        cluster.sync();
-        if (warp < w) {
-          float *r0 = cluster.map_shared_rank(buf0, d0 >> 1) + ((d0 & 1) * w + warp) * LP;
-          float *r1 = cluster.map_shared_rank(buf0, d1 >> 1) + ((d1 & 1) * w + warp) * LP;
-          col_store<NE>(r0, x);
-          col_store<NE>(r1, y);
-        }
-        cluster.sync();
+      float y0[NE], y1[NE];
+      col_load<NE>(y0, Qb + c0 * LP);
+      col_load<NE>(y1, Qb + c1 * LP);
+      float *dst = dbuf ? buf0 + (cur ^ 1) * bufw : buf0;
+      if (!dbuf) cluster.sync();  // single buffer: everyone has read its blocks before writes
+      {
+        float *r0 = cluster.map_shared_rank(dst, d0 >> 1) + (d0 & 1) * w * LP;
+        float *r1 = cluster.map_shared_rank(dst, d1 >> 1) + (d1 & 1) * w * LP;
+        col_store<NE>(r0 + c0 * LP, x0);
+        col_store<NE>(r0 + c1 * LP, x1);
+        col_store<NE>(r1 + c0 * LP, y0);
+        col_store<NE>(r1 + c1 * LP, y1);
       }
+      cluster.sync();
+      if (dbuf) cur ^= 1;
     }
     // Cluster-wide "any rotation in this sweep".
     const int any_local = __syncthreads_or(rot ? 1 : 0);
@@ -314,20 +341,18 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
   float *buf = buf0 + (dbuf ? cur * bufw : 0);
 
   // Column norms of my columns (blocks are at their round-0 places again).
-  for (int slot = 0; slot < 2; ++slot) {
-    if (warp < w) {
-      const float *x = buf + (slot * w + warp) * LP;
-      double s = 0.0;
+  for (int e = warp; e < 2 * w; e += nw) {
+    const float *x = buf + e * LP;
+    double s = 0.0;
 #pragma unroll
-      for (int t = 0; t < NE; ++t) {
-        if (lane + 32 * t < m) {
-          const double v = x[lane + 32 * t];
-          s = fma(v, v, s);
-        }
+    for (int t = 0; t < NE; ++t) {
+      if (lane + 32 * t < m) {
+        const double v = x[lane + 32 * t];
+        s = fma(v, v, s);
       }
-      s = warp_sum(s);
-      if (lane == 0) nrm_local[slot * w + warp] = (float)sqrt(s);
     }
+    s = warp_sum(s);
+    if (lane == 0) nrm_local[e] = (float)sqrt(s);
   }
   cluster.sync();
   for (int e = tid; e < M * w; e += blockDim.x) {
@@ -344,9 +369,9 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
   float *Ht = reinterpret_cast<float *>(jh.ws + p.Ht);
   float *sig = reinterpret_cast<float *>(jh.ws + p.sig);
   const int npad = M * w;
-  for (int slot = 0; slot < 2; ++slot) {
-    if (warp >= w) continue;
-    const int j = pairs[(0 * cj + rank) * 2 + slot] * w + warp;
+  for (int e = warp; e < 2 * w; e += nw) {
+    const int slot = e / w, lc = e % w;
+    const int j = pairs[(0 * cj + rank) * 2 + slot] * w + lc;
     const float nj = nrm_all[j];
     // Rank by (norm desc, index asc) on a key where a non-finite norm sorts last, so the ranks
     // form a permutation even for NaN input.
@@ -362,7 +387,7 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
     const int q = cnt;
     if (j >= ncol || q >= kn) continue;
     if (!isfinite(nj) && lane == 0) record_status(jh.meta, ISKV_ERR_NONFINITE);
-    const float *x = buf + (slot * w + warp) * LP;
+    const float *x = buf + e * LP;
     const float inv = nj > 0.f ? 1.f / nj : 0.f;
     if (lane == 0) sig[q] = nj;
     for (int l = lane; l < r; l += 32) {
@@ -410,7 +435,7 @@ static cudaError_t core_launch(const char *jobs, const CoreParams &p, const Jaco
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.count * c.cj);
-  cfg.blockDim = dim3(32 * c.w);
+  cfg.blockDim = dim3(16 * c.w);  // w / 2 warps
   cfg.dynamicSmemBytes = c.smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
