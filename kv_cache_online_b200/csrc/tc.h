@@ -27,6 +27,7 @@ struct alignas(64) TcJob {
 
 struct TcParams {
   int r, d, n_heads, count, tiles_per_job;
+  int hp, stages;  // reconstruction: heads per CTA, U slab ring depth
   double theta;
 };
 

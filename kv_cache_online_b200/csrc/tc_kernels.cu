@@ -57,7 +57,8 @@ ISKV_DEV TileRange my_tiles(int count, int tiles_per_job) {
   return t;
 }
 
-ISKV_DEV void fail_timeout(TcCtl *c, int64_t *meta) {
+template <class Ctl>
+ISKV_DEV void fail_timeout(Ctl *c, int64_t *meta) {
   c->abort = 1;
   if (meta) record_status(meta, ISKV_ERR_TIMEOUT);
 }
@@ -170,13 +171,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
     const int q = warp & 3, half = (warp - 2) >> 2;
     const int cols = N / 2, c0 = half * cols;
     int na = 0;
-    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
+    // Lanes of a warp take every exit together: tcgen05.ld is a warp-wide instruction.
+    for (int t = tr.begin; t < tr.end && !__any_sync(~0u, *abort != 0); ++t) {
       const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
       const TcJob &jb = jobs[j];
       const int n = jb.sc[FS_N_OLD];
       if (jb.sc[FS_SKIP] || row0 >= n || jb.sc[FS_K_OLD] == 0) continue;
       const int buf = na & 1, use = na >> 1;
-      if (!mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS)) {
+      if (!__all_sync(~0u, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
         fail_timeout(ctl, jb.meta);
         break;
       }
@@ -212,26 +214,60 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
 
 // ================================================================================================
 // Reconstruction. Job fields: mapA (U), mapB (sigma-scaled basis, d x r bf16), out, pos, meta.
+//
+// Basis-stationary schedule. Each CTA owns `hp` heads (two when the head count is even) and keeps
+// their rows of sigma*B^T resident in shared memory while it streams U through a ring of 16 KB
+// K-slabs (128 rows x 64 coordinates). The n_heads/hp CTAs that own the other heads of the same
+// rows form a group and walk the same row tiles in step, so each U tile is read from HBM once and
+// served from L2 to the rest of the group. One MMA of N = hp x 128 covers all of the CTA's heads,
+// so the tensor core reads each A slab once per K step.
+//
+// Output rows are scattered (row i goes to position pos_i), so the epilogue stages each head's
+// 128 x 128 bf16 block in shared memory (rows padded by 16 bytes against bank conflicts) and
+// writes every row with one 256-byte bulk copy instead of 16-byte stores to 128 different lines.
+constexpr int REC_MAX_STAGES = 8;
+constexpr int REC_STG_PITCH = 256 + 16;  // bytes per staged row
+
+struct RecCtl {
+  uint64_t a_full[REC_MAX_STAGES], a_empty[REC_MAX_STAGES];
+  uint64_t b_full, b_empty;
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t done;
+  uint32_t tmem;
+  int abort;
+};
+
 __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  const int R = p.r, KS = R / 64, H = p.n_heads, D = p.d;
-  constexpr int N = 128;  // one head per MMA chunk
-  constexpr int CHUNK_BYTES_PER_SLAB = N * 128;
-  uint8_t *sA = smem;                                    // KS x 16 KB
-  uint8_t *sB = smem + KS * SLAB_BYTES;                  // 2 stages x KS x 16 KB
-  TcCtl *ctl = reinterpret_cast<TcCtl *>(sB + 2 * KS * CHUNK_BYTES_PER_SLAB);
-  double *invf = reinterpret_cast<double *>(ctl + 1);    // 64 doubles
+  const int R = p.r, KS = R / 64, D = p.d, HP = p.hp, NA = p.stages;
+  constexpr int HN = 128;                        // columns per head
+  uint8_t *sB = smem;                            // KS slabs x (HP x 128 rows) x 128 B, resident
+  uint8_t *sA = sB + KS * HP * SLAB_BYTES;       // NA slabs x 16 KB
+  uint8_t *sStg = sA + NA * SLAB_BYTES;          // 128 rows x REC_STG_PITCH
+  RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + TC_M * REC_STG_PITCH);
+  double *invf = reinterpret_cast<double *>(ctl + 1);  // 64 doubles
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr uint32_t NCOLS = 256;
-  const uint32_t idesc = idesc_bf16_f32(TC_M, N);
+  const int NN = HP * HN;                        // MMA N
+  const uint32_t ncols = HP == 2 ? 512 : 256;    // two accumulator buffers of NN columns
+  const uint32_t idesc = idesc_bf16_f32(TC_M, NN);
+  // Group and member: CTAs g*G .. g*G+G-1 cover the heads of the same row tiles.
+  const int G = p.n_heads / HP, group = blockIdx.x / G, member = blockIdx.x % G;
+  const int ngroups = gridDim.x / G;
+  const int total = p.count * p.tiles_per_job;
+  const int per = (total + ngroups - 1) / ngroups;
+  const int t_begin = group * per, t_end = min(total, t_begin + per);
+  const int tpj = p.tiles_per_job;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 4; ++s) { mbar_init(&ctl->a_full[s], 1); mbar_init(&ctl->a_empty[s], 1); }
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(&ctl->a_full[i], 1);
+      mbar_init(&ctl->a_empty[i], 1);
+    }
+    mbar_init(&ctl->b_full, 1);
+    mbar_init(&ctl->b_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&ctl->b_full[i], 1);
-      mbar_init(&ctl->b_empty[i], 1);
       mbar_init(&ctl->acc_full[i], 1);
       mbar_init(&ctl->acc_empty[i], 8);
     }
@@ -240,159 +276,184 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     fence_barrier_init();
   }
   if (threadIdx.x < 64) invf[threadIdx.x] = exp(-2.0 * threadIdx.x / 128.0 * log(p.theta));
-  if (warp == 1) tmem_alloc(&ctl->tmem, NCOLS);
+  if (warp == 1) tmem_alloc(&ctl->tmem, ncols);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = ctl->tmem;
   volatile int *abort = &ctl->abort;
-  const TileRange tr = my_tiles(p.count, p.tiles_per_job);
+  // First valid tile at or after t (rows below the history's current length), or -1. Every role
+  // walks the same sequence.
+  auto next_valid = [&](int t) {
+    for (; t < t_end; ++t)
+      if ((t % tpj) * TC_M < jobs[t / tpj].meta[ISKV_META_N]) return t;
+    return -1;
+  };
 
   if (warp == 0 && lane == 0) {
-    // ---------------- producer
-    int na = 0, nc = 0, cur = -1;
-    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
-      const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+    // ---------------- producer: basis rows of this CTA's heads once per history, U slabs per tile
+    int na = 0, nb = 0, cur = -1;
+    int64_t *fm = nullptr;  // meta of the history being loaded: where a timeout is recorded
+    bool ok = true;
+    for (int t = next_valid(t_begin); t >= 0 && ok && !*abort; t = next_valid(t + 1)) {
+      const int j = t / tpj, row0 = (t % tpj) * TC_M;
       const TcJob &jb = jobs[j];
-      if (row0 >= jb.meta[ISKV_META_N]) continue;
+      fm = jb.meta;
       if (j != cur) {
+        if (nb > 0 && !mbar_wait(&ctl->b_empty, (nb - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
         tensormap_acquire(&jb.mapA);
         tensormap_acquire(&jb.mapB);
-        cur = j;
-      }
-      bool ok = true;
-      for (int s = 0; s < KS; ++s) {
-        if (na > 0 && !mbar_wait(&ctl->a_empty[s], (na - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
-        mbar_arrive_expect_tx(&ctl->a_full[s], SLAB_BYTES);
-        tma_load_2d(sA + s * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[s]);
-      }
-      ++na;
-      for (int c = 0; c < H && ok; ++c) {
-        const int st = nc & 1, use = nc >> 1;
-        if (use > 0 && !mbar_wait(&ctl->b_empty[st], (use - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
-        mbar_arrive_expect_tx(&ctl->b_full[st], KS * CHUNK_BYTES_PER_SLAB);
+        mbar_arrive_expect_tx(&ctl->b_full, KS * HP * SLAB_BYTES);
         for (int s = 0; s < KS; ++s)
-          tma_load_2d(sB + (st * KS + s) * CHUNK_BYTES_PER_SLAB, &jb.mapB, s * 64, c * N,
-                      &ctl->b_full[st]);
-        ++nc;
+          for (int h = 0; h < HP; ++h)
+            tma_load_2d(sB + (s * HP + h) * SLAB_BYTES, &jb.mapB, s * 64, (member * HP + h) * HN,
+                        &ctl->b_full);
+        cur = j;
+        ++nb;
       }
-      if (!ok) { fail_timeout(ctl, jb.meta); break; }
+      for (int s = 0; s < KS; ++s) {
+        const int st = na % NA, use = na / NA;
+        if (use > 0 && !mbar_wait(&ctl->a_empty[st], (use - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
+        mbar_arrive_expect_tx(&ctl->a_full[st], SLAB_BYTES);
+        tma_load_2d(sA + st * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[st]);
+        ++na;
+      }
     }
-    if (na > 0)
-      for (int s = 0; s < KS; ++s) mbar_wait(&ctl->a_full[s], (na - 1) & 1, abort, WAIT_NS / 4);
-    for (int k = 1; k <= 2 && nc - k >= 0; ++k)
-      mbar_wait(&ctl->b_full[(nc - k) & 1], ((nc - k) >> 1) & 1, abort, WAIT_NS / 4);
+    if (!ok) fail_timeout(ctl, fm);
+    // Let every copy issued land before the CTA exits.
+    if (nb > 0) mbar_wait(&ctl->b_full, (nb - 1) & 1, abort, WAIT_NS / 4);
+    for (int k = 1; k <= NA && na - k >= 0; ++k)
+      mbar_wait(&ctl->a_full[(na - k) % NA], ((na - k) / NA) & 1, abort, WAIT_NS / 4);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    int na = 0, nc = 0;
-    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
-      const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
-      const TcJob &jb = jobs[j];
-      if (row0 >= jb.meta[ISKV_META_N]) continue;
-      bool ok = true;
-      for (int c = 0; c < H && ok; ++c) {
-        const int buf = nc & 1, use = nc >> 1;
-        if (use > 0 && !mbar_wait(&ctl->acc_empty[buf], (use - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
-        fence_after_sync();
-        if (!mbar_wait(&ctl->b_full[buf], use & 1, abort, WAIT_NS)) { ok = false; break; }
-        const uint32_t d = tmem + buf * N;
-        for (int s = 0; s < KS; ++s) {
-          if (c == 0 && !mbar_wait(&ctl->a_full[s], na & 1, abort, WAIT_NS)) { ok = false; break; }
-          fence_after_sync();
-          const uint32_t a0 = smem_u32(sA + s * SLAB_BYTES);
-          const uint32_t b0 = smem_u32(sB + (buf * KS + s) * CHUNK_BYTES_PER_SLAB);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (s | kk) != 0);
-          if (c == H - 1) mma_commit(&ctl->a_empty[s]);
-        }
-        if (!ok) break;
-        mma_commit(&ctl->b_empty[buf]);
-        mma_commit(&ctl->acc_full[buf]);
-        ++nc;
+    int na = 0, nb = 0, nc = 0, cur = -1;
+    int64_t *fm = nullptr;
+    bool ok = true;
+    for (int t = next_valid(t_begin); t >= 0 && ok && !*abort; t = next_valid(t + 1)) {
+      const int j = t / tpj;
+      fm = jobs[j].meta;
+      if (j != cur) {
+        // The resident basis may be replaced once every MMA reading it has completed.
+        if (nb > 0) mma_commit(&ctl->b_empty);
+        if (!mbar_wait(&ctl->b_full, nb & 1, abort, WAIT_NS)) { ok = false; break; }
+        cur = j;
+        ++nb;
       }
-      if (!ok) { fail_timeout(ctl, jb.meta); break; }
-      ++na;
+      const int buf = nc & 1, use = nc >> 1;
+      if (use > 0 && !mbar_wait(&ctl->acc_empty[buf], (use - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
+      fence_after_sync();
+      const uint32_t d0 = tmem + buf * NN;
+      for (int s = 0; s < KS; ++s) {
+        const int st = na % NA;
+        if (!mbar_wait(&ctl->a_full[st], (na / NA) & 1, abort, WAIT_NS)) { ok = false; break; }
+        fence_after_sync();
+        const uint32_t a0 = smem_u32(sA + st * SLAB_BYTES);
+        const uint32_t b0 = smem_u32(sB + s * HP * SLAB_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(d0, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (s | kk) != 0);
+        mma_commit(&ctl->a_empty[st]);
+        ++na;
+      }
+      if (!ok) break;
+      mma_commit(&ctl->acc_full[buf]);
+      ++nc;
     }
+    if (!ok) fail_timeout(ctl, fm);
     mma_commit(&ctl->done);
     mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
   } else if (warp >= 2) {
-    // ---------------- epilogue: TMEM -> RoPE -> bf16 -> out[pos]
+    // ---------------- epilogue: TMEM -> RoPE -> bf16 -> staged rows -> bulk copies to out[pos]
     const int q = warp & 3, half = (warp - 2) >> 2;
     const int j0 = half * 32;  // this thread's head-local pairs j0 .. j0 + 31 (cols j and j + 64)
+    const int srow = q * 32 + lane;
+    uint8_t *stg = sStg + srow * REC_STG_PITCH;
+    const double inv_two_pi = 0.15915494309189533576888376337251;
+    const double two_pi = 6.283185307179586476925286766559;
     int nc = 0;
-    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
-      const int jj = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+    // The two warps that share rows (q, half 0 and 1) take every decision together through an
+    // AND-reducing named barrier: they meet at named barriers below, and tcgen05.ld is warp-wide.
+    const int pair_bar = 1 + q;
+    for (int t = next_valid(t_begin);; t = next_valid(t + 1)) {
+      if (!named_and(pair_bar, 64, t >= 0 && !*abort)) break;
+      const int jj = t / tpj, row0 = (t % tpj) * TC_M;
       const TcJob &jb = jobs[jj];
       const int64_t n = jb.meta[ISKV_META_N];
-      if (row0 >= n) continue;
-      const int64_t row = row0 + q * 32 + lane;
+      const int64_t row = row0 + srow;
       bool valid = row < n;
-      int64_t ps = valid ? (int64_t)jb.pos[row] : 0;
+      const int64_t ps = valid ? (int64_t)jb.pos[row] : 0;
       if (valid && (ps < 0 || ps >= jb.n_total)) {
         record_status(jb.meta, ISKV_ERR_SHAPE);
         valid = false;
       }
+      // Rotation angles pos * theta^(-2j/128): reduced to [-pi, pi] in float64, then the fast
+      // hardware sine/cosine (absolute error ~1e-6 there, far below the bf16 output's rounding).
       float cs[32], sn[32];
-      const bool rope = jb.rope != 0;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         cs[i] = 1.f;
         sn[i] = 0.f;
       }
-      if (rope && valid) {
-        const double two_pi = 6.283185307179586476925286766559;
+      if (jb.rope != 0 && valid) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           double a = (double)ps * invf[j0 + i];
-          a -= two_pi * rint(a / two_pi);
-          sincosf((float)a, &sn[i], &cs[i]);
+          a = fma(-two_pi, rint(a * inv_two_pi), a);
+          __sincosf((float)a, &sn[i], &cs[i]);
         }
       }
-      __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(jb.out) + (size_t)(valid ? ps : 0) * D;
-      bool ok = true;
-      for (int c = 0; c < H; ++c) {
-        const int buf = nc & 1, use = nc >> 1;
-        if (!mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS)) { ok = false; break; }
-        fence_after_sync();
-        const uint32_t base = tmem + buf * N + ((uint32_t)(q * 32) << 16);
+      __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(jb.out) + (size_t)(valid ? ps : 0) * D +
+                            (size_t)member * HP * HN;
+      const int buf = nc & 1, use = nc >> 1;
+      if (!named_and(pair_bar, 64, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
+        fail_timeout(ctl, jb.meta);
+        break;
+      }
+      fence_after_sync();
+      const uint32_t base = tmem + buf * NN + ((uint32_t)(q * 32) << 16);
+      for (int h = 0; h < HP; ++h) {
+        // The staged row is free once the previous bulk copy out of it has been read.
+        if (half == 0) bulk_wait_read0();
+        named_sync(pair_bar, 64);
 #pragma unroll
         for (int jb16 = 0; jb16 < 32; jb16 += 16) {
           float lo[16], hi[16];
-          tmem_ld16(base + j0 + jb16, lo);
-          tmem_ld16(base + 64 + j0 + jb16, hi);
+          tmem_ld16(base + h * HN + j0 + jb16, lo);
+          tmem_ld16(base + h * HN + 64 + j0 + jb16, hi);
           tmem_ld_wait();
-          if (valid) {
-            uint32_t wl[8], wh[8];
+          uint32_t wl[8], wh[8];
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              const float c0 = cs[jb16 + i], s0 = sn[jb16 + i];
-              const float c1 = cs[jb16 + i + 1], s1 = sn[jb16 + i + 1];
-              const float l0 = lo[i] * c0 - hi[i] * s0, h0 = hi[i] * c0 + lo[i] * s0;
-              const float l1 = lo[i + 1] * c1 - hi[i + 1] * s1, h1 = hi[i + 1] * c1 + lo[i + 1] * s1;
-              wl[i / 2] = pack_bf16(l0, l1);
-              wh[i / 2] = pack_bf16(h0, h1);
-            }
-            uint4 *dl = reinterpret_cast<uint4 *>(orow + c * N + j0 + jb16);
-            uint4 *dh = reinterpret_cast<uint4 *>(orow + c * N + 64 + j0 + jb16);
-            dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-            dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
-            dh[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-            dh[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+          for (int i = 0; i < 16; i += 2) {
+            const float c0 = cs[jb16 + i], s0 = sn[jb16 + i];
+            const float c1 = cs[jb16 + i + 1], s1 = sn[jb16 + i + 1];
+            wl[i / 2] = pack_bf16(lo[i] * c0 - hi[i] * s0, lo[i + 1] * c1 - hi[i + 1] * s1);
+            wh[i / 2] = pack_bf16(hi[i] * c0 + lo[i] * s0, hi[i + 1] * c1 + lo[i + 1] * s1);
           }
+          uint4 *dl = reinterpret_cast<uint4 *>(stg + 2 * (j0 + jb16));
+          uint4 *dh = reinterpret_cast<uint4 *>(stg + 2 * (64 + j0 + jb16));
+          dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+          dh[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          dh[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
         }
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
-        ++nc;
+        fence_proxy_async_smem();
+        named_sync(pair_bar, 64);
+        if (half == 0 && valid) {
+          bulk_store(orow + h * HN, stg, 2 * HN);
+          bulk_commit();
+        }
       }
-      if (!ok) { fail_timeout(ctl, jb.meta); break; }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+      ++nc;
     }
+    if (half == 0) bulk_wait0();
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 1) tmem_dealloc(tmem, NCOLS);
+  if (warp == 1) tmem_dealloc(tmem, ncols);
 }
 
 // ================================================================================================
@@ -483,7 +544,8 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, 
     const int q = warp & 3;
     float *out = reinterpret_cast<float *>(jb.out) +
                  (which ? p.off_gb : p.off_gu) / sizeof(float) + (size_t)split * R * R;
-    if (mbar_wait(&ctl->acc_full[0], 0, abort, WAIT_NS) && !*abort) {
+    // One decision per warp: tcgen05.ld is a warp-wide instruction.
+    if (__all_sync(~0u, mbar_wait(&ctl->acc_full[0], 0, abort, WAIT_NS) && !*abort)) {
       fence_after_sync();
       for (int h = 0; h < MH; ++h) {
         const int row = h * 128 + q * 32 + lane;
@@ -576,8 +638,21 @@ bool tc_recon_supported(int r, int storage, int out_dtype, int head_dim) {
 
 size_t tc_rot_smem(int r) { return 1024 + (size_t)(r / 64) * SLAB_BYTES + (size_t)(r / 64) * r * 128 + sizeof(TcCtl); }
 
-size_t tc_rec_smem(int r) {
-  return 1024 + (size_t)(r / 64) * SLAB_BYTES * 3 + sizeof(TcCtl) + 64 * sizeof(double);
+// Resident basis rows for hp heads, the U slab ring, the output staging rows, the barriers and the
+// RoPE frequencies.
+size_t tc_rec_smem(int r, int hp, int stages) {
+  return 1024 + (size_t)hp * (r / 64) * SLAB_BYTES + (size_t)stages * SLAB_BYTES +
+         (size_t)TC_M * REC_STG_PITCH + sizeof(RecCtl) + 64 * sizeof(double);
+}
+
+constexpr size_t kRecSmemCap = 227 * 1024;
+
+// Heads per CTA and U ring depth for the reconstruction: two heads when the head count is even,
+// and as many 16 KB slabs (up to REC_MAX_STAGES) as the shared memory left over holds.
+void tc_rec_shape(int r, int n_heads, int &hp, int &stages) {
+  hp = (n_heads % 2 == 0 && tc_rec_smem(r, 2, 3) <= kRecSmemCap) ? 2 : 1;
+  stages = REC_MAX_STAGES;
+  while (stages > 2 && tc_rec_smem(r, hp, stages) > kRecSmemCap) --stages;
 }
 
 cudaError_t launch_tc_rotation(const TcJob *hjobs, int count, TcJob *djobs, int r,
@@ -586,6 +661,8 @@ cudaError_t launch_tc_rotation(const TcJob *hjobs, int count, TcJob *djobs, int 
   tp.r = r;
   tp.d = 0;
   tp.n_heads = 0;
+  tp.hp = 0;
+  tp.stages = 0;
   tp.count = count;
   tp.tiles_per_job = (int)((n_cap_max + TC_M - 1) / TC_M);
   tp.theta = 0.0;
@@ -636,14 +713,20 @@ cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob
   tp.count = p.count;
   tp.tiles_per_job = (int)((p.n_cap_max + TC_M - 1) / TC_M);
   tp.theta = p.theta;
+  tc_rec_shape(p.r, p.n_heads, tp.hp, tp.stages);
   cudaError_t e = upload_jobs(djobs, hjobs.data(), sizeof(TcJob) * hjobs.size(), s);
   if (e != cudaSuccess) return e;
-  const size_t smem = tc_rec_smem(p.r);
+  const size_t smem = tc_rec_smem(p.r, tp.hp, tp.stages);
   e = cudaFuncSetAttribute(k_rec_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // Whole groups of n_heads / hp CTAs, as many as fit one per SM (at least one group), and no
+  // more groups than row tiles.
+  const int G = p.n_heads / tp.hp;
   const int total = tp.count * tp.tiles_per_job;
-  const int grid = total < num_sms() ? total : num_sms();
-  k_rec_tc<<<grid, TC_THREADS, smem, s>>>(djobs, tp);
+  int groups = num_sms() / G;
+  if (groups < 1) groups = 1;
+  if (groups > total) groups = total;
+  k_rec_tc<<<groups * G, TC_THREADS, smem, s>>>(djobs, tp);
   count_launches(1);
   return cudaGetLastError();
 }

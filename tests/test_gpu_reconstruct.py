@@ -82,3 +82,36 @@ def test_full_size_sampled_rows():
     got = np64(out)
     sel = np.r_[pos[rows], epos[:16]]
     assert of.rel_fro(got[sel], ref[sel]) < 2e-2
+
+
+@pytest.mark.parametrize("d,r,H", [(1024, 256, 8), (384, 128, 3), (512, 64, 4), (256, 192, 2)])
+def test_batched_tensor_core_shapes(d, r, H):
+    """Several bf16 histories in one call (row counts with ragged last tiles, one of a single row,
+    one below full rank, keys and values mixed): every history's dense output against the oracle,
+    rows at no position left as they were."""
+    m = kv()
+    ns, ks = [700, 1, 129, 256], [r, r, r - 17, r]
+    hs, ref, outs, n_total = [], [], [], []
+    for i, (n, k) in enumerate(zip(ns, ks)):
+        k = min(k, n)  # a history's rank is at most its row count
+        U, s, B = synthetic_history(n, d, r, seed=40 + i, dtype=torch.bfloat16)
+        U, s, B = U[:, :k], s[:k], B[:, :k]
+        g = np.random.Generator(np.random.PCG64(50 + i))
+        nt = n + 37
+        pos = g.permutation(nt)[:n]
+        h = m.LowRankHistory(d, r, n + 5, storage=torch.bfloat16)
+        set_state(h, U, s, B, pos)
+        rope = i % 2 == 0
+        ref.append(orec.reconstruct(U, s, B, pos, np.zeros((0, d)), np.zeros(0, dtype=int), nt, H,
+                                    d // H, rope, 500000.0, fill=3.0))
+        outs.append(torch.full((nt, d), 3.0, dtype=torch.bfloat16, device="cuda"))
+        hs.append(h)
+        n_total.append(nt)
+    m.reconstruct_batched(hs, [None] * 4, [None] * 4, n_total, H, d // H,
+                          [i % 2 == 0 for i in range(4)], 500000.0, outs=outs)
+    for h, o, rf, n, nt in zip(hs, outs, ref, ns, n_total):
+        got = np64(o)
+        assert of.rel_fro(got, rf) < 2e-2
+        untouched = np.setdiff1d(np.arange(nt), h.pos[:n].cpu().numpy())
+        assert np.all(got[untouched] == 3.0)
+        assert h.status()[3] == 0
