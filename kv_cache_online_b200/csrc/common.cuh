@@ -50,7 +50,7 @@ enum FoldScalar {
   FS_SKIP = 4,    // 1 when the fold is skipped (capacity)
   FS_SWEEPS = 5,  // Jacobi sweeps used by the core SVD
   FS_RSWEEPS = 6, // Jacobi sweeps used by the residual SVD
-  FS_COUNT = 16
+  FS_COUNT = 32
 };
 
 // Fields every job descriptor starts with (fold and re-orthogonalisation jobs share them, so the

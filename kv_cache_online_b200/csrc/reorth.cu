@@ -17,7 +17,21 @@
 
 namespace iskv {
 
-enum { RS_CU = 8, RS_CB = 9 };  // scalar slots holding the Newton-Schulz scales (float bits)
+// Scalar slots: the Newton-Schulz scales (float bits), and from RS_DEV on, per iteration `it` and
+// factor `which`, the squared Frobenius norm of T - I accumulated by that iteration's first stage.
+enum { RS_CU = 8, RS_CB = 9, RS_DEV = 16 };
+static_assert(RS_DEV + 2 * NS_ITERS <= FS_COUNT, "scalar slots");
+
+// Early exit of the iteration. With D = Z Y - I, one step maps D to -(3/4) D^2 + (1/4) D^3, and
+// T - I = -D / 2. Once ||T - I||_F <= 5e-4 (so ||D||_2 <= 1e-3), the step that applies this T leaves
+// ||D||_2 below 1e-6: further steps would change Y and Z only at float32 rounding level. Those
+// steps are skipped (their outputs are copies). Rounding puts a floor near 2e-5 under ||T - I||_F
+// for r = 256 (the diagonal's sums of r products near 1), well below the threshold.
+constexpr float NS_STOP_SQ = 2.5e-7f;  // (5e-4)^2
+
+ISKV_DEV bool ns_converged(const int32_t *sc, int it, int which) {
+  return it > 0 && __int_as_float(sc[RS_DEV + 2 * (it - 1) + which]) <= NS_STOP_SQ;
+}
 
 ReorthWsLayout reorth_ws_layout(int d, int r, int64_t n_cap) {
   ReorthWsLayout L;
@@ -63,9 +77,10 @@ __global__ void k_reorth_prepare(const ReorthJob *jobs, ReorthParams p) {
   sc[FS_K_NEW] = (int32_t)k;
   sc[FS_SKIP] = (k <= 0 || k > p.r || n < 0 || n > jb.n_cap) ? 1 : 0;
   sc[FS_SWEEPS] = 0;
+  for (int i = 0; i < 2 * NS_ITERS; ++i) sc[RS_DEV + i] = 0;  // float 0
 }
 
-constexpr int GBM = 32, GBN = 64, GBK = 16, GTM = 2, GTN = 4;
+constexpr int GBM = 64, GBN = 64, GBK = 16, GTM = 4, GTN = 4;
 
 // Gram partial: Gpart[s] = X[rows of split s]^T X[rows of split s] (k x k), X = U (n rows) or B.
 template <typename TS>
@@ -137,15 +152,17 @@ __global__ void k_ns_init(const ReorthJob *jobs, ReorthParams p) {
   }
 }
 
-// Newton-Schulz stages. STAGE 0: T = 1.5 I - 0.5 Z Y. STAGE 1: Y2 = Y T (g = 0), Z2 = T Z (g = 1).
+// Newton-Schulz stages of iteration `it`. STAGE 0: T = 1.5 I - 0.5 Z Y, and ||T - I||_F^2 summed
+// into the iteration's slot. STAGE 1: Y2 = Y T (g = 0), Z2 = T Z (g = 1). Once an earlier
+// iteration's T met the stopping threshold, stage 0 does nothing and stage 1 copies Y, Z forward.
 template <int STAGE>
-__global__ void __launch_bounds__(256) k_ns_step(const ReorthJob *jobs, ReorthParams p,
+__global__ void __launch_bounds__(256) k_ns_step(const ReorthJob *jobs, ReorthParams p, int it,
                                                  size_t y0, size_t z0, size_t y1, size_t z1,
                                                  size_t yb0, size_t zb0, size_t yb1, size_t zb1) {
   const int per = STAGE == 0 ? 2 : 4;
   const int job = blockIdx.z / per, rem = blockIdx.z % per, which = rem & 1, g = rem >> 1;
   const ReorthJob &jb = jobs[job];
-  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  int32_t *sc = reinterpret_cast<int32_t *>(jb.h.ws);
   if (sc[FS_SKIP]) return;
   const int k = sc[FS_K_OLD], r = p.r;
   char *ws = jb.h.ws;
@@ -154,23 +171,47 @@ __global__ void __launch_bounds__(256) k_ns_step(const ReorthJob *jobs, ReorthPa
   float *T = reinterpret_cast<float *>(ws + p.ws.T[which]);
   const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
   if (m0 >= k || n0 >= k) return;
+  const bool done = ns_converged(sc, it, which);  // uniform over the block
   if (STAGE == 0) {
+    if (done) return;
+    float ss = 0.f;
     tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
         m0, n0, k, k, k, [&](int m, int kk) { return Z[(size_t)m * r + kk]; },
         [&](int kk, int n) { return Y[(size_t)kk * r + n]; },
-        [&](int m, int n, float acc) { T[(size_t)m * r + n] = (m == n ? 1.5f : 0.f) - 0.5f * acc; });
+        [&](int m, int n, float acc) {
+          const float t = (m == n ? 1.5f : 0.f) - 0.5f * acc;
+          const float dv = t - (m == n ? 1.f : 0.f);
+          ss = fmaf(dv, dv, ss);
+          T[(size_t)m * r + n] = t;
+        });
+    __shared__ float red[8];
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float tot = 0.f;
+      for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+      atomicAdd(reinterpret_cast<float *>(sc + RS_DEV + 2 * it + which), tot);
+    }
+    return;
+  }
+  const float *X = g == 0 ? Y : Z;
+  float *Xo = reinterpret_cast<float *>(ws + (g == 0 ? (which == 0 ? y1 : yb1) : (which == 0 ? z1 : zb1)));
+  if (done) {
+    for (int e = threadIdx.x; e < GBM * GBN; e += blockDim.x) {
+      const int m = m0 + e / GBN, n = n0 + e % GBN;
+      if (m < k && n < k) Xo[(size_t)m * r + n] = X[(size_t)m * r + n];
+    }
   } else if (g == 0) {
-    float *Yo = reinterpret_cast<float *>(ws + (which == 0 ? y1 : yb1));
     tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
         m0, n0, k, k, k, [&](int m, int kk) { return Y[(size_t)m * r + kk]; },
         [&](int kk, int n) { return T[(size_t)kk * r + n]; },
-        [&](int m, int n, float acc) { Yo[(size_t)m * r + n] = acc; });
+        [&](int m, int n, float acc) { Xo[(size_t)m * r + n] = acc; });
   } else {
-    float *Zo = reinterpret_cast<float *>(ws + (which == 0 ? z1 : zb1));
     tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
         m0, n0, k, k, k, [&](int m, int kk) { return T[(size_t)m * r + kk]; },
         [&](int kk, int n) { return Z[(size_t)kk * r + n]; },
-        [&](int m, int n, float acc) { Zo[(size_t)m * r + n] = acc; });
+        [&](int m, int n, float acc) { Xo[(size_t)m * r + n] = acc; });
   }
 }
 
@@ -298,10 +339,10 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   size_t y0[2] = {W.Y[0], W.Y[1]}, z0[2] = {W.Z[0], W.Z[1]};
   size_t y1[2] = {W.Y2[0], W.Y2[1]}, z1[2] = {W.Z2[0], W.Z2[1]};
   for (int it = 0; it < NS_ITERS; ++it) {
-    k_ns_step<0><<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p, y0[0], z0[0], y1[0], z1[0],
-                                                         y0[1], z0[1], y1[1], z1[1]);
-    k_ns_step<1><<<dim3(tn, tm, p.count * 4), 256, 0, s>>>(jobs, p, y0[0], z0[0], y1[0], z1[0],
-                                                         y0[1], z0[1], y1[1], z1[1]);
+    k_ns_step<0><<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p, it, y0[0], z0[0], y1[0],
+                                                         z1[0], y0[1], z0[1], y1[1], z1[1]);
+    k_ns_step<1><<<dim3(tn, tm, p.count * 4), 256, 0, s>>>(jobs, p, it, y0[0], z0[0], y1[0],
+                                                         z1[0], y0[1], z0[1], y1[1], z1[1]);
     for (int w = 0; w < 2; ++w) {
       size_t t = y0[w]; y0[w] = y1[w]; y1[w] = t;
       t = z0[w]; z0[w] = z1[w]; z1[w] = t;
