@@ -176,7 +176,9 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
       Rm[c * b + i] = i < c ? A[i * b + c] : (i == c ? alph[c] : 0.f);
     }
     __syncthreads();
-    const double tol = 2.0 * sqrt((double)b) * 5.960464477539063e-08;
+    // Float32 inner products carry relative error ~ sqrt(b) 2^-24; the tolerance sits a few units
+    // above it (a residual cosine of that size moves the rho only at second order).
+    const float tol = 4.f * sqrtf((float)b) * 5.9604645e-08f;
     const int sw = cta_jacobi_columns(Rm, b, b, b, tol, 60);
     __shared__ float nrm[128];
     __shared__ int order[128];

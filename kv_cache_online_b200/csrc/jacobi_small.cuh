@@ -1,39 +1,29 @@
 // One-sided (Hestenes) Jacobi on the columns of a small matrix held in one CTA's shared memory.
 // Used for the SVD of the b x b residual factor R_R of the fold (iS-KV reading notes, Section 4.1:
 // "QR + SVD of the small factor"). Written from the published method: Hestenes (1958), with the
-// stable rotation of Rutishauser and the convergence test of Demmel and Veselic (1992).
+// rotation angle of Rutishauser and the convergence test of Demmel and Veselic (1992).
 #pragma once
 
 #include "common.cuh"
 
 namespace iskv {
 
-// Rotation angle that makes columns with squared norms alpha, beta and inner product gamma
-// orthogonal: returns (c, s) with x' = c x - s y, y' = s x + c y.
-ISKV_DEV void jacobi_rotation(double alpha, double beta, double gamma, double &c, double &s) {
-  const double zeta = (beta - alpha) / (2.0 * gamma);
-  double t;
-  if (fabs(zeta) > 1e100) {
-    t = 0.5 / zeta;
-  } else {
-    t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-  }
-  c = 1.0 / sqrt(1.0 + t * t);
-  s = c * t;
-}
-
 // Round-robin ("circle") pairing: n even players, player 0 fixed, the rest rotate by `step`.
 ISKV_DEV int circle_player(int i, int step, int n) {
   return i == 0 ? 0 : ((i - 1 + step) % (n - 1)) + 1;
 }
 
-// Orthogonalise the `ncols` columns of M (column-major, leading dimension ld, `rows` rows) in
-// place. All threads of the CTA must call it. Returns the number of sweeps used, or -1 when the
-// sweep cap was reached without convergence. Rotations are skipped when
-// |gamma| <= tol * sqrt(alpha * beta).
-ISKV_DEV int cta_jacobi_columns(float *M, int rows, int ncols, int ld, double tol, int max_sweeps) {
+// Orthogonalise the `ncols` columns of M (column-major, leading dimension ld, `rows` <= 128 rows)
+// in place, in float32. All threads of the CTA must call it (blockDim a multiple of 32). Each
+// half-warp rotates one column pair at a time (16 lanes x up to 8 rows each), so a 256-thread CTA
+// handles 16 pairs of a round in parallel. Rotations use the half-angle form
+//   x' = x - s (y + tau x),  y' = y + s (x - tau y),  tau = t / (1 + sqrt(1 + t^2)),
+// which stays orthogonal when c = 1 / sqrt(1 + t^2) rounds to 1. A pair is skipped when
+// |gamma| <= tol * sqrt(alpha * beta). Returns the sweeps used, or -1 when the cap was reached.
+ISKV_DEV int cta_jacobi_columns(float *M, int rows, int ncols, int ld, float tol, int max_sweeps) {
   __shared__ int rotated;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int half = (threadIdx.x >> 4) & 1, l16 = threadIdx.x & 15;
   const int ne = ncols + (ncols & 1);
   const int npairs = ne / 2;
   if (ne < 2) return 0;
@@ -41,30 +31,51 @@ ISKV_DEV int cta_jacobi_columns(float *M, int rows, int ncols, int ld, double to
     if (threadIdx.x == 0) rotated = 0;
     __syncthreads();
     for (int step = 0; step < ne - 1; ++step) {
-      for (int pr = warp; pr < npairs; pr += nwarps) {
-        const int a = circle_player(pr, step, ne), b = circle_player(ne - 1 - pr, step, ne);
-        if (a >= ncols || b >= ncols) continue;
-        float *x = M + (size_t)a * ld, *y = M + (size_t)b * ld;
-        double al = 0.0, be = 0.0, ga = 0.0;
-        for (int i = lane; i < rows; i += 32) {
-          const double xv = x[i], yv = y[i];
-          al = fma(xv, xv, al);
-          be = fma(yv, yv, be);
-          ga = fma(xv, yv, ga);
+      // Both half-warps of a warp run the same number of iterations (they shuffle together).
+      for (int base = 2 * warp; base < npairs; base += 2 * nwarps) {
+        const int pr = base + half;
+        int a = 0, b = 0;
+        bool live = pr < npairs;
+        if (live) {
+          a = circle_player(pr, step, ne);
+          b = circle_player(ne - 1 - pr, step, ne);
+          live = a < ncols && b < ncols;
         }
-        al = warp_sum(al);
-        be = warp_sum(be);
-        ga = warp_sum(ga);
-        if (ga != 0.0 && fabs(ga) > tol * sqrt(al * be)) {
-          double c, s;
-          jacobi_rotation(al, be, ga, c, s);
-          const float cf = (float)c, sf = (float)s;
-          for (int i = lane; i < rows; i += 32) {
-            const float xv = x[i], yv = y[i];
-            x[i] = cf * xv - sf * yv;
-            y[i] = sf * xv + cf * yv;
+        float *x = M + (size_t)a * ld, *y = M + (size_t)b * ld;
+        float xv[8], yv[8];
+        float al = 0.f, be = 0.f, ga = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int i = l16 + 16 * q;
+          const bool in = live && i < rows;
+          xv[q] = in ? x[i] : 0.f;
+          yv[q] = in ? y[i] : 0.f;
+          al = fmaf(xv[q], xv[q], al);
+          be = fmaf(yv[q], yv[q], be);
+          ga = fmaf(xv[q], yv[q], ga);
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+          al += __shfl_xor_sync(0xffffffffu, al, o);
+          be += __shfl_xor_sync(0xffffffffu, be, o);
+          ga += __shfl_xor_sync(0xffffffffu, ga, o);
+        }
+        if (live && ga != 0.f && fabsf(ga) > tol * sqrtf(al) * sqrtf(be)) {
+          const float zeta = (be - al) / (2.f * ga);
+          const float t = fabsf(zeta) > 1e18f
+                              ? 0.5f / zeta
+                              : copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
+          const float sq = sqrtf(fmaf(t, t, 1.f));
+          const float sn = t / sq, tau = t / (1.f + sq);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int i = l16 + 16 * q;
+            if (i < rows) {
+              x[i] = fmaf(-sn, fmaf(tau, xv[q], yv[q]), xv[q]);
+              y[i] = fmaf(sn, fmaf(-tau, yv[q], xv[q]), yv[q]);
+            }
           }
-          if (lane == 0) rotated = 1;
+          if (l16 == 0) rotated = 1;
         }
       }
       __syncthreads();
