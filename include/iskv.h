@@ -116,7 +116,8 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
  * B = Q_B R_B, decompose R_U diag(sigma) R_B^T = X diag(sigma') Y^T and set U <- Q_U X,
  * sigma <- sigma', B <- Q_B Y. The product U diag(sigma) B^T is unchanged in exact arithmetic;
  * k and n are unchanged; meta[FOLDS] is reset to 0. hs is a HOST array of `count` handles sharing
- * d, r_max, storage and n_cap.
+ * d, r_max, storage and n_cap. r_max <= 384 (the dense r x r core SVD must fit one thread-block
+ * cluster); larger r_max returns ISKV_ERR_SHAPE.
  */
 size_t iskv_reorth_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap);
 iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t ws_bytes,

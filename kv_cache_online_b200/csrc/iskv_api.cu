@@ -121,8 +121,8 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   if (fold_residual_smem(d, b) > 200 * 1024)
     return fail(ISKV_ERR_SHAPE, "%s: d = %d with b = %d exceeds the residual QR cluster", who, d, b);
   {
-    const JacobiCfg jc = jacobi_cfg(r + b, r + 2 * b);
-    if (jc.smem > 200 * 1024 || 16 * jc.w > 640)
+    JacobiCfg jc;
+    if (!core_cfg(r, b, false, jc))
       return fail(ISKV_ERR_SHAPE, "%s: r_max + b too large for the core SVD cluster", who);
   }
   const size_t need = iskv_fold_workspace_size(count, d, r, b);
@@ -226,6 +226,12 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   }
   const int d = hs[0].d, r = hs[0].r_max;
   const int64_t ncap = hs[0].n_cap;
+  {
+    JacobiCfg jc;
+    if (!core_cfg(r, 0, true, jc))
+      return fail(ISKV_ERR_SHAPE, "%s: r_max = %d too large for the dense core SVD (r_max <= 384)",
+                  who, r);
+  }
   const size_t need = iskv_reorth_workspace_size(count, d, r, ncap);
   iskv_status st = check_ws(ws, ws_bytes, need, who);
   if (st != ISKV_OK) return st;

@@ -51,56 +51,87 @@ __host__ __device__ inline CoreSmem core_smem(int cj, int w, int ne, bool dbuf) 
 }
 
 constexpr size_t kCoreSmemCap = 200 * 1024;
-constexpr int kMaxWarps = 20;  // register budget: 96 registers x 640 threads
 
-// Columns per block w (two blocks per CTA, two column pairs per warp, so w / 2 warps).
+// Threads per CTA the register file allows for NE column entries per lane (four columns live in
+// registers): 640 x 96, 512 x 128 or 384 x 170 registers.
+__host__ __device__ constexpr int core_max_threads(int ne) {
+  return ne <= 12 ? 640 : (ne <= 16 ? 512 : 384);
+}
+
+// Columns per block w (two blocks per CTA, two column pairs per warp, so w / 2 warps): the
+// smallest cluster whose blocks fit the warp budget and the shared-memory cap; column blocks are
+// double-buffered when that fits too. `ne` = 0 when no register template covers the column.
 JacobiCfg jacobi_cfg(int ncols_max, int col_len_max) {
   JacobiCfg c;
-  int cj = 1;
-  for (;;) {
+  int ne = (col_len_max + 31) / 32;
+  const int choices[] = {2, 4, 8, 12, 16, 20, 24};
+  int pick = 0;
+  for (int v : choices)
+    if (v >= ne) { pick = v; break; }
+  c.ne = pick;
+  const int nes = pick ? pick : 24;
+  for (int cj = 1; cj <= 16; cj *= 2) {
     int w = (ncols_max + 2 * cj - 1) / (2 * cj);
     w += w & 1;
     if (w < 4) w = 4;
-    if (w <= 2 * kMaxWarps || cj == 16) {
-      c.cj = cj;
-      c.w = w;
-      break;
-    }
-    cj *= 2;
+    c.cj = cj;
+    c.w = w;
+    c.dbuf = core_smem(cj, w, nes, true).total <= kCoreSmemCap;
+    c.smem = core_smem(cj, w, nes, c.dbuf).total;
+    if (16 * w <= core_max_threads(nes) && c.smem <= kCoreSmemCap) break;
   }
-  int ne = (col_len_max + 31) / 32;
-  const int choices[] = {2, 4, 8, 12, 16, 20, 24};
-  for (int v : choices)
-    if (v >= ne) { ne = v; break; }
-  c.ne = ne;
-  c.dbuf = core_smem(c.cj, c.w, c.ne, true).total <= kCoreSmemCap;
-  c.smem = core_smem(c.cj, c.w, c.ne, c.dbuf).total;
   return c;
 }
 
-// Dot product of two register-resident columns over their first m entries, two accumulators
-// (shorter dependency chain); the whole warp receives the sum.
-template <int NE, bool DD>
-ISKV_DEV float warp_dot(const float (&x)[NE], const float (&y)[NE], int m) {
+bool core_cfg(int r, int b, bool dense, JacobiCfg &c) {
+  // Column length: the A part zero-padded to a multiple of 64, then the explicit V rows.
+  const int pad64 = dense ? (r + 63) / 64 * 64 : (r + b + 63) / 64 * 64;
+  const int len = dense ? pad64 + r : pad64 + b;
+  c = jacobi_cfg(dense ? r : r + b, len);
+  return c.ne > 0 && 16 * c.w <= core_max_threads(c.ne) && c.smem <= kCoreSmemCap;
+}
+
+// Register layout of a column: lane l holds the float2 pairs l + 32 q (elements 2 l + 64 q and
+// 2 l + 64 q + 1), q < NE / 2, so loads, stores and the arithmetic run on packed float2
+// (sm_100 issues one FFMA2 for two FMAs).
+template <int NE>
+ISKV_DEV void col_load(float2 (&x)[NE / 2], const float *src) {
+  const float2 *s2 = reinterpret_cast<const float2 *>(src);
   const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < NE / 2; ++q) x[q] = s2[lane + 32 * q];
+}
+
+template <int NE>
+ISKV_DEV void col_store(float *dst, const float2 (&x)[NE / 2]) {
+  float2 *d2 = reinterpret_cast<float2 *>(dst);
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < NE / 2; ++q) d2[lane + 32 * q] = x[q];
+}
+
+// Dot product of two register-resident columns over their first 64 nq entries (the A part,
+// zero-padded to a multiple of 64); the whole warp receives the sum.
+template <int NE, bool DD>
+ISKV_DEV float warp_dot(const float2 (&x)[NE / 2], const float2 (&y)[NE / 2], int nq) {
   if (DD) {  // float64 accumulation of the exact float32 products
     double a0 = 0.0, a1 = 0.0;
 #pragma unroll
-    for (int t = 0; t < NE; ++t)
-      if (lane + 32 * t < m) {
-        if (t & 1) a1 = fma((double)x[t], (double)y[t], a1);
-        else a0 = fma((double)x[t], (double)y[t], a0);
+    for (int q = 0; q < NE / 2; ++q)
+      if (q < nq) {
+        a0 = fma((double)x[q].x, (double)y[q].x, a0);
+        a1 = fma((double)x[q].y, (double)y[q].y, a1);
       }
     return (float)warp_sum(a0 + a1);
   }
-  float a0 = 0.f, a1 = 0.f;
+  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int t = 0; t < NE; ++t)
-    if (lane + 32 * t < m) {
-      if (t & 1) a1 = fmaf(x[t], y[t], a1);
-      else a0 = fmaf(x[t], y[t], a0);
+  for (int q = 0; q < NE / 2; ++q)
+    if (q < nq) {
+      if (q & 1) a1 = __ffma2_rn(x[q], y[q], a1);
+      else a0 = __ffma2_rn(x[q], y[q], a0);
     }
-  return warp_sum(a0 + a1);
+  return warp_sum((a0.x + a1.x) + (a0.y + a1.y));
 }
 
 // One Jacobi rotation of the pair (x, y) with squared norms ax, by and inner product g, when the
@@ -110,7 +141,8 @@ ISKV_DEV float warp_dot(const float (&x)[NE], const float (&y)[NE], int m) {
 // float32 (a plain c = 1, s = t would grow both norms by t^2 / 2 on every small rotation). Norms
 // follow Rutishauser: ax -= t g, by += t g.
 template <int NE, bool DD>
-ISKV_DEV bool rotate_regs(float (&x)[NE], float (&y)[NE], float &ax, float &by, float g, float tol) {
+ISKV_DEV bool rotate_regs(float2 (&x)[NE / 2], float2 (&y)[NE / 2], float &ax, float &by, float g,
+                          float tol) {
   if (!(g != 0.f && fabsf(g) > tol * sqrtf(ax) * sqrtf(by))) return false;
   float t, s, tau;
   if (DD) {
@@ -129,11 +161,13 @@ ISKV_DEV bool rotate_regs(float (&x)[NE], float (&y)[NE], float &ax, float &by, 
     s = t / sq;
     tau = t / (1.f + sq);
   }
+  const float2 s2 = make_float2(s, s), ms2 = make_float2(-s, -s);
+  const float2 t2 = make_float2(tau, tau), mt2 = make_float2(-tau, -tau);
 #pragma unroll
-  for (int q = 0; q < NE; ++q) {
-    const float xv = x[q], yv = y[q];
-    x[q] = fmaf(-s, fmaf(tau, xv, yv), xv);
-    y[q] = fmaf(s, fmaf(-tau, yv, xv), yv);
+  for (int q = 0; q < NE / 2; ++q) {
+    const float2 xv = x[q], yv = y[q];
+    x[q] = __ffma2_rn(ms2, __ffma2_rn(t2, xv, yv), xv);
+    y[q] = __ffma2_rn(s2, __ffma2_rn(mt2, yv, xv), yv);
   }
   ax -= t * g;
   by += t * g;
@@ -142,22 +176,8 @@ ISKV_DEV bool rotate_regs(float (&x)[NE], float (&y)[NE], float &ax, float &by, 
   return true;
 }
 
-template <int NE>
-ISKV_DEV void col_load(float (&x)[NE], const float *src) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int q = 0; q < NE; ++q) x[q] = src[lane + 32 * q];
-}
-
-template <int NE>
-ISKV_DEV void col_store(float *dst, const float (&x)[NE]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int q = 0; q < NE; ++q) dst[lane + 32 * q] = x[q];
-}
-
 template <int NE, bool DD>
-__global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, int w, int dbuf) {
+__global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs, CoreParams p, int w, int dbuf) {
   cg::cluster_group cluster = cg::this_cluster();
   const int cj = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
   const JobHead &jh = job_head(jobs, p.job_stride, blockIdx.x / cj);
@@ -170,6 +190,8 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
   const int k = sc[FS_K_OLD], b = dense ? 0 : p.b, r = p.r, hs = p.hs;
   const int pp = dense ? k : sc[FS_P];          // explicit V rows stored after the A part
   const int m = k + b;                          // A rows
+  const int mp = (m + 63) / 64 * 64;            // A part zero-padded to whole float2 lanes
+  const int nq = mp / 64;                       // float2 pairs per lane in the A part
   const int ncol = dense ? k : k + pp, kn = min(r, ncol);
   const CoreSmem S = core_smem(cj, w, NE, dbuf != 0);
   extern __shared__ float smem[];
@@ -207,19 +229,20 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
   for (int e = tid; e < bufw; e += blockDim.x) {
     const int slot = e / (w * LP), lc = (e / LP) % w, el = e % LP;
     const int j = pairs[(0 * cj + rank) * 2 + slot] * w + lc;
+    // Column layout: A rows [0, m), zeros [m, mp), explicit V rows [mp, mp + pp), zeros after.
     float v = 0.f;
     if (dense) {
       if (j < k) {
         if (el < k) v = Md[(size_t)el * p.ldm + j];
-        else if (el < m + pp) v = (el - m == j) ? 1.f : 0.f;
+        else if (el >= mp && el < mp + pp) v = (el - mp == j) ? 1.f : 0.f;
       }
     } else if (el < k) {
       v = (j < k && el == j) ? sig_old[j] : 0.f;
     } else if (el < m) {
       const int i = el - k;
       v = j < k ? C[(size_t)i * r + j] : (j < ncol ? FP[(size_t)i * b + (j - k)] : 0.f);
-    } else if (el < m + pp) {
-      v = (j >= k && j < ncol && el - m == j - k) ? 1.f : 0.f;
+    } else if (el >= mp && el < mp + pp) {
+      v = (j >= k && j < ncol && el - mp == j - k) ? 1.f : 0.f;
     }
     buf0[e] = v;
   }
@@ -239,15 +262,15 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
       float *Pb = buf, *Qb = buf + w * LP;
       // Exact squared norms at the start of the round; tracked through the round's rotations.
       {
-        float x[NE], y[NE];
+        float2 x[NE / 2], y[NE / 2];
         col_load<NE>(x, Pb + c0 * LP);
         col_load<NE>(y, Qb + c0 * LP);
-        float a = warp_dot<NE, DD>(x, x, m), c = warp_dot<NE, DD>(y, y, m);
+        float a = warp_dot<NE, DD>(x, x, nq), c = warp_dot<NE, DD>(y, y, nq);
         if (lane == 0) { nP[c0] = a; nQ[c0] = c; }
         col_load<NE>(x, Pb + c1 * LP);
         col_load<NE>(y, Qb + c1 * LP);
-        a = warp_dot<NE, DD>(x, x, m);
-        c = warp_dot<NE, DD>(y, y, m);
+        a = warp_dot<NE, DD>(x, x, nq);
+        c = warp_dot<NE, DD>(y, y, nq);
         if (lane == 0) { nP[c1] = a; nQ[c1] = c; }
       }
       __syncthreads();
@@ -261,11 +284,11 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
             const int a = circle_player(q, st, w), bb = circle_player(w - 1 - q, st, w);
             float *base = slot ? Qb : Pb;
             float *nb = slot ? nQ : nP;
-            float x[NE], y[NE];
+            float2 x[NE / 2], y[NE / 2];
             col_load<NE>(x, base + a * LP);
             col_load<NE>(y, base + bb * LP);
             float ax = nb[a], by = nb[bb];
-            const float g = warp_dot<NE, DD>(x, y, m);
+            const float g = warp_dot<NE, DD>(x, y, nq);
             if (rotate_regs<NE, DD>(x, y, ax, by, g, tol)) {
               col_store<NE>(base + a * LP, x);
               col_store<NE>(base + bb * LP, y);
@@ -277,18 +300,18 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
         }
       }
       // Cross pairs: warp i keeps P[i] and P[i + w/2] in registers while the Q columns circulate.
-      float x0[NE], x1[NE];
+      float2 x0[NE / 2], x1[NE / 2];
       col_load<NE>(x0, Pb + c0 * LP);
       col_load<NE>(x1, Pb + c1 * LP);
       float ax0 = nP[c0], ax1 = nP[c1];
       for (int st = 0; st < w; ++st) {
         const int q0 = (c0 + st) % w, q1 = (c1 + st) % w;
-        float y0[NE], y1[NE];
+        float2 y0[NE / 2], y1[NE / 2];
         col_load<NE>(y0, Qb + q0 * LP);
         col_load<NE>(y1, Qb + q1 * LP);
         float by0 = nQ[q0], by1 = nQ[q1];
-        const float g0 = warp_dot<NE, DD>(x0, y0, m);
-        const float g1 = warp_dot<NE, DD>(x1, y1, m);
+        const float g0 = warp_dot<NE, DD>(x0, y0, nq);
+        const float g1 = warp_dot<NE, DD>(x1, y1, nq);
         if (rotate_regs<NE, DD>(x0, y0, ax0, by0, g0, tol)) {
           col_store<NE>(Qb + q0 * LP, y0);
           if (lane == 0) nQ[q0] = by0;
@@ -311,7 +334,7 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
       const int tn = (t + 1) % (M - 1);
       const int X0 = pairs[(t * cj + rank) * 2 + 0], X1 = pairs[(t * cj + rank) * 2 + 1];
       const int d0 = where[tn * M + X0], d1 = where[tn * M + X1];
-      float y0[NE], y1[NE];
+      float2 y0[NE / 2], y1[NE / 2];
       col_load<NE>(y0, Qb + c0 * LP);
       col_load<NE>(y1, Qb + c1 * LP);
       float *dst = dbuf ? buf0 + (cur ^ 1) * bufw : buf0;
@@ -398,9 +421,9 @@ __global__ void __launch_bounds__(640) k_core(const char *jobs, CoreParams p, in
     for (int i = lane; i < b; i += 32) Gbot[(size_t)i * r + q] = x[k + i] * inv;
     for (int l = lane; l < hs; l += 32) {
       float h = 0.f;
-      if (dense) h = l < k ? x[m + l] : 0.f;
+      if (dense) h = l < k ? x[mp + l] : 0.f;
       else if (l < k) h = sig_old[l] > 0.f ? x[l] / sig_old[l] : 0.f;
-      else if (l < ncol) h = x[m + (l - k)];
+      else if (l < ncol) h = x[mp + (l - k)];
       Ht[(size_t)q * hs + l] = h;
     }
   }
@@ -450,7 +473,8 @@ static cudaError_t core_launch(const char *jobs, const CoreParams &p, const Jaco
 }
 
 cudaError_t launch_core(const char *jobs, const CoreParams &p, cudaStream_t s) {
-  const JacobiCfg c = p.mode == 1 ? jacobi_cfg(p.r, 2 * p.r) : jacobi_cfg(p.r + p.b, p.r + 2 * p.b);
+  JacobiCfg c;
+  if (!core_cfg(p.r, p.b, p.mode == 1, c)) return cudaErrorInvalidConfiguration;
   switch (c.ne) {
     case 2: return core_launch<2>(jobs, p, c, s);
     case 4: return core_launch<4>(jobs, p, c, s);

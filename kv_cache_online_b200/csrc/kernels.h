@@ -43,6 +43,9 @@ struct JacobiCfg {
 };
 
 JacobiCfg jacobi_cfg(int ncols_max, int col_len_max);
+// Configuration of the core SVD for r_max = r and block b (fold) or of the dense r x r core
+// (re-orthogonalisation); false when no cluster shape fits.
+bool core_cfg(int r, int b, bool dense, JacobiCfg &c);
 size_t fold_residual_smem(int d, int b);
 
 cudaError_t launch_fold_prepare(const FoldJob *jobs, const FoldParams &p, cudaStream_t s);
