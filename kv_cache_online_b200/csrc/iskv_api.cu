@@ -381,6 +381,7 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
         return fail(ISKV_ERR_CUDA, "reconstruct: tensor map encoding failed");
     e = launch_tc_recon(djobs, tj, tc_dev, p, s);
   } else {
+    stage_mark(s, ST_RECON_PREPARE);
     e = launch_recon_compressed(djobs, p, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "reconstruct: compressed rows");

@@ -135,32 +135,31 @@ ISKV_DEV float warp_dot(const float2 (&x)[NE / 2], const float2 (&y)[NE / 2], in
 }
 
 // One Jacobi rotation of the pair (x, y) with squared norms ax, by and inner product g, when the
-// pair is not orthogonal to tolerance. Applied in the half-angle form
-//   x' = x - s (y + tau x),  y' = y + s (x - tau y),  tau = tan(theta / 2) = s / (1 + c),
-// which equals (c x - s y, s x + c y) but keeps the rotation orthogonal even when c rounds to 1 in
-// float32 (a plain c = 1, s = t would grow both norms by t^2 / 2 on every small rotation). Norms
-// follow Rutishauser: ax -= t g, by += t g.
+// pair is not orthogonal to tolerance (g^2 > tol^2 ax by). Rutishauser's angle: zeta =
+// (by - ax) / 2g, t = tan(theta) = sign(zeta) / (|zeta| + sqrt(1 + zeta^2)); applied in the
+// half-angle form
+//   x' = x - s (y + tau x),  y' = y + s (x - tau y),  tau = tan(theta / 2),  s = 2 tau / (1 + tau^2),
+// which equals (c x - s y, s x + c y) and stays orthogonal to rounding because s is derived from
+// tau. The parameters only have to define some rotation that nearly orthogonalises the pair (a
+// residual cosine is removed by a later sweep), so they use the hardware reciprocal and
+// reciprocal square root. Norms follow Rutishauser: ax -= t g, by += t g. Both accumulation modes
+// (DD: the inner products were summed in float64) use these float32 parameters.
 template <int NE, bool DD>
 ISKV_DEV bool rotate_regs(float2 (&x)[NE / 2], float2 (&y)[NE / 2], float &ax, float &by, float g,
-                          float tol) {
-  if (!(g != 0.f && fabsf(g) > tol * sqrtf(ax) * sqrtf(by))) return false;
-  float t, s, tau;
-  if (DD) {
-    const double zeta = ((double)by - (double)ax) / (2.0 * (double)g);
-    const double td = fabs(zeta) > 1e100 ? 0.5 / zeta
-                                         : (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-    const double sq = sqrt(1.0 + td * td);
-    t = (float)td;
-    s = (float)(td / sq);
-    tau = (float)(td / (1.0 + sq));
+                          float tol2) {
+  if (!(g != 0.f && g * g > (tol2 * ax) * by)) return false;
+  const float zeta = 0.5f * (by - ax) * __fdividef(1.f, g);
+  const float az = fabsf(zeta);
+  float t;
+  if (az > 1e18f) {
+    t = __fdividef(0.5f, zeta);
   } else {
-    const float zeta = (by - ax) / (2.f * g);
-    t = fabsf(zeta) > 1e18f ? 0.5f / zeta
-                            : copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
-    const float sq = sqrtf(fmaf(t, t, 1.f));
-    s = t / sq;
-    tau = t / (1.f + sq);
+    const float q = fmaf(zeta, zeta, 1.f);
+    t = copysignf(__fdividef(1.f, az + q * rsqrtf(q)), zeta);
   }
+  const float q2 = fmaf(t, t, 1.f);
+  const float tau = __fdividef(t, 1.f + q2 * rsqrtf(q2));
+  const float s = __fdividef(2.f * tau, fmaf(tau, tau, 1.f));
   const float2 s2 = make_float2(s, s), ms2 = make_float2(-s, -s);
   const float2 t2 = make_float2(tau, tau), mt2 = make_float2(-tau, -tau);
 #pragma unroll
@@ -253,6 +252,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   // only at second order. The dense mode (re-orthogonalisation, whose purpose is orthonormal
   // factors) accumulates inner products in float64 and uses a tighter tolerance.
   const float tol = (DD ? 2.f : 4.f) * sqrtf((float)(m > 1 ? m : 1)) * 5.9604645e-08f;
+  const float tol2 = tol * tol;
   int sweeps_used = -1;
   int cur = 0;  // which buffer holds the current blocks (double-buffered exchange)
   for (int sweep = 0; sweep < p.max_sweeps; ++sweep) {
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
             col_load<NE>(y, base + bb * LP);
             float ax = nb[a], by = nb[bb];
             const float g = warp_dot<NE, DD>(x, y, nq);
-            if (rotate_regs<NE, DD>(x, y, ax, by, g, tol)) {
+            if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
               col_store<NE>(base + a * LP, x);
               col_store<NE>(base + bb * LP, y);
               if (lane == 0) { nb[a] = ax; nb[bb] = by; }
@@ -312,12 +312,12 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
         float by0 = nQ[q0], by1 = nQ[q1];
         const float g0 = warp_dot<NE, DD>(x0, y0, nq);
         const float g1 = warp_dot<NE, DD>(x1, y1, nq);
-        if (rotate_regs<NE, DD>(x0, y0, ax0, by0, g0, tol)) {
+        if (rotate_regs<NE, DD>(x0, y0, ax0, by0, g0, tol2)) {
           col_store<NE>(Qb + q0 * LP, y0);
           if (lane == 0) nQ[q0] = by0;
           rot = true;
         }
-        if (rotate_regs<NE, DD>(x1, y1, ax1, by1, g1, tol)) {
+        if (rotate_regs<NE, DD>(x1, y1, ax1, by1, g1, tol2)) {
           col_store<NE>(Qb + q1 * LP, y1);
           if (lane == 0) nQ[q1] = by1;
           rot = true;

@@ -19,7 +19,7 @@ ISKV_DEV int circle_player(int i, int step, int n) {
 // handles 16 pairs of a round in parallel. Rotations use the half-angle form
 //   x' = x - s (y + tau x),  y' = y + s (x - tau y),  tau = t / (1 + sqrt(1 + t^2)),
 // which stays orthogonal when c = 1 / sqrt(1 + t^2) rounds to 1. A pair is skipped when
-// |gamma| <= tol * sqrt(alpha * beta). Returns the sweeps used, or -1 when the cap was reached.
+// gamma^2 <= tol^2 alpha beta. Returns the sweeps used, or -1 when the cap was reached.
 ISKV_DEV int cta_jacobi_columns(float *M, int rows, int ncols, int ld, float tol, int max_sweeps) {
   __shared__ int rotated;
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -60,13 +60,21 @@ ISKV_DEV int cta_jacobi_columns(float *M, int rows, int ncols, int ld, float tol
           be += __shfl_xor_sync(0xffffffffu, be, o);
           ga += __shfl_xor_sync(0xffffffffu, ga, o);
         }
-        if (live && ga != 0.f && fabsf(ga) > tol * sqrtf(al) * sqrtf(be)) {
-          const float zeta = (be - al) / (2.f * ga);
-          const float t = fabsf(zeta) > 1e18f
-                              ? 0.5f / zeta
-                              : copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
-          const float sq = sqrtf(fmaf(t, t, 1.f));
-          const float sn = t / sq, tau = t / (1.f + sq);
+        if (live && ga != 0.f && ga * ga > (tol * tol * al) * be) {
+          // Rutishauser's angle; tau = tan(theta / 2) and sn = 2 tau / (1 + tau^2) keep the
+          // rotation orthogonal to rounding, so fast reciprocals suffice for the parameters.
+          const float zeta = 0.5f * (be - al) * __fdividef(1.f, ga);
+          const float az = fabsf(zeta);
+          float t;
+          if (az > 1e18f) {
+            t = __fdividef(0.5f, zeta);
+          } else {
+            const float q = fmaf(zeta, zeta, 1.f);
+            t = copysignf(__fdividef(1.f, az + q * rsqrtf(q)), zeta);
+          }
+          const float q2 = fmaf(t, t, 1.f);
+          const float tau = __fdividef(t, 1.f + q2 * rsqrtf(q2));
+          const float sn = __fdividef(2.f * tau, fmaf(tau, tau, 1.f));
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const int i = l16 + 16 * q;

@@ -27,7 +27,8 @@ std::atomic<long long> g_launches{0};
 const char *kNames[ST_COUNT] = {
     "fold.project",   "fold.residual_qr_svd", "fold.core_svd",      "fold.basis_rotate",
     "fold.coord_rotate", "fold.finalize",     "reorth.gram",        "reorth.newton_schulz",
-    "reorth.core_svd", "reorth.coord_rotate", "reorth.basis_rotate", "reconstruct.compressed",
+    "reorth.core_svd", "reorth.coord_rotate", "reorth.basis_rotate", "reconstruct.prepare",
+    "reconstruct.compressed",
     "reconstruct.exact", "select",            "job_upload"};
 
 cudaEvent_t take_event() {

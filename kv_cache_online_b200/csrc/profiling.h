@@ -21,6 +21,7 @@ enum Stage {
   ST_REORTH_CORE,
   ST_REORTH_COORDS,
   ST_REORTH_BASIS,
+  ST_RECON_PREPARE,
   ST_RECON_COMPRESSED,
   ST_RECON_EXACT,
   ST_SELECT,

@@ -16,8 +16,9 @@ ISKV_DEV double rope_inv_freq(int j, int hd, double log_theta) {
 
 ISKV_DEV void rope_sincos(int64_t pos, double inv_freq, float &c, float &s) {
   const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
   double a = (double)pos * inv_freq;
-  a -= two_pi * rint(a / two_pi);
+  a = fma(-two_pi, rint(a * inv_two_pi), a);
   sincosf((float)a, &s, &c);
 }
 
@@ -99,20 +100,27 @@ __global__ void __launch_bounds__(256) k_recon_ffma(const ReconJob *jobs, ReconP
   }
 }
 
-// Exact rows: copy (and rotate) exact_rows[e] to out[exact_pos[e]].
+// Exact rows: copy (and rotate) exact_rows[e] to out[exact_pos[e]]. Thread = (row, head, pair);
+// consecutive threads take consecutive pairs of a head, so loads and stores are contiguous.
 template <typename TE, typename TO>
-__global__ void k_recon_exact(const ReconJob *jobs, ReconParams p) {
+__global__ void __launch_bounds__(256) k_recon_exact(const ReconJob *jobs, ReconParams p) {
   const ReconJob &jb = jobs[blockIdx.y];
   const int hd = p.head_dim, half = hd / 2, d = p.d, H = p.n_heads;
-  const int64_t npairs = jb.n_exact * (int64_t)H * half;
-  const double lt = log(p.theta);
+  __shared__ double invf[128];
+  if (jb.apply_rope) {
+    const double lt = log(p.theta);
+    for (int j = threadIdx.x; j < half; j += blockDim.x) invf[j] = rope_inv_freq(j, hd, lt);
+  }
+  __syncthreads();
+  const int per_row = H * half;
+  const int64_t npairs = jb.n_exact * (int64_t)per_row;
   const TE *X = static_cast<const TE *>(jb.exact_rows);
   TO *out = static_cast<TO *>(jb.out);
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < npairs;
        t += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t e = t / (H * half);
-    const int rem = (int)(t % (H * half));
-    const int h = rem / half, c = rem % half;
+    const int64_t e = t / per_row;
+    const int rem = (int)(t - e * per_row);
+    const int h = rem / half, c = rem - h * half;
     const int64_t ps = jb.exact_pos[e];
     if (ps < 0 || ps >= jb.n_total) {
       record_status(jb.meta, ISKV_ERR_SHAPE);
@@ -122,7 +130,7 @@ __global__ void k_recon_exact(const ReconJob *jobs, ReconParams p) {
     float x2 = to_f<TE>(X[(size_t)e * d + h * hd + c + half]);
     if (jb.apply_rope) {
       float cs, sn;
-      rope_sincos(ps, rope_inv_freq(c, hd, lt), cs, sn);
+      rope_sincos(ps, invf[c], cs, sn);
       const float y1 = x1 * cs - x2 * sn, y2 = x2 * cs + x1 * sn;
       x1 = y1;
       x2 = y2;

@@ -14,6 +14,7 @@
 // of one tile (or head) overlap the MMAs of the next.
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -228,6 +229,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
 constexpr int REC_MAX_STAGES = 8;
 constexpr int REC_STG_PITCH = 256 + 16;  // bytes per staged row
 
+// RoPE tables (head_dim 128, 64 frequencies omega_j = theta^(-2j/128)). Angles are reduced in
+// exact integer arithmetic: W_j = omega_j / (2 pi) is held as a 0.64 fixed-point fraction
+// (wh, wl), and for a position p < 2^31 the top 32 bits of frac(p W_j) are
+// p * wh + umulhi(p, wl) (mod 2^32) -- the signed turn count in [-1/2, 1/2) at resolution
+// 2^-32, with error below 2^-22 turns from W_j's float64 rounding. The angle in [-pi, pi) then goes
+// to the hardware sine/cosine (absolute error ~1e-6 there, far below the bf16 output's rounding).
+struct RopeTab {
+  uint32_t wh[64], wl[64];
+};
+
+// Host-side table for rope_theta (float64 arithmetic; the kernel only copies it).
+RopeTab make_rope_tab(double theta) {
+  RopeTab t;
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int j = 0; j < 64; ++j) {
+    const double w = std::exp(-2.0 * j / 128.0 * std::log(theta)) / two_pi;  // turns per position
+    const double hi = std::floor(std::ldexp(w, 32));
+    t.wh[j] = (uint32_t)hi;
+    t.wl[j] = (uint32_t)std::floor(std::ldexp(std::ldexp(w, 32) - hi, 32));
+  }
+  return t;
+}
+
+ISKV_DEV void rope_angle(const RopeTab *t, int j, uint32_t p, float &c, float &s) {
+  const uint32_t top = p * t->wh[j] + __umulhi(p, t->wl[j]);
+  const float ang = (float)(int32_t)top * 1.46291807926715968e-09f;  // 2 pi / 2^32
+  __sincosf(ang, &s, &c);
+}
+
 struct RecCtl {
   uint64_t a_full[REC_MAX_STAGES], a_empty[REC_MAX_STAGES];
   uint64_t b_full, b_empty;
@@ -237,7 +267,8 @@ struct RecCtl {
   int abort;
 };
 
-__global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcParams p) {
+__global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcParams p,
+                                                           const __grid_constant__ RopeTab rt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -247,7 +278,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
   uint8_t *sA = sB + KS * HP * SLAB_BYTES;       // NA slabs x 16 KB
   uint8_t *sStg = sA + NA * SLAB_BYTES;          // 128 rows x REC_STG_PITCH
   RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + TC_M * REC_STG_PITCH);
-  double *invf = reinterpret_cast<double *>(ctl + 1);  // 64 doubles
+  RopeTab *rope_tab = reinterpret_cast<RopeTab *>(ctl + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NN = HP * HN;                        // MMA N
   const uint32_t ncols = HP == 2 ? 512 : 256;    // two accumulator buffers of NN columns
@@ -275,7 +306,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     ctl->abort = 0;
     fence_barrier_init();
   }
-  if (threadIdx.x < 64) invf[threadIdx.x] = exp(-2.0 * threadIdx.x / 128.0 * log(p.theta));
+  if (threadIdx.x < 64) {
+    rope_tab->wh[threadIdx.x] = rt.wh[threadIdx.x];
+    rope_tab->wl[threadIdx.x] = rt.wl[threadIdx.x];
+  }
   if (warp == 1) tmem_alloc(&ctl->tmem, ncols);
   fence_before_sync();
   __syncthreads();
@@ -368,38 +402,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     const int j0 = half * 32;  // this thread's head-local pairs j0 .. j0 + 31 (cols j and j + 64)
     const int srow = q * 32 + lane;
     uint8_t *stg = sStg + srow * REC_STG_PITCH;
-    const double inv_two_pi = 0.15915494309189533576888376337251;
-    const double two_pi = 6.283185307179586476925286766559;
     int nc = 0;
     // The two warps that share rows (q, half 0 and 1) take every decision together through an
     // AND-reducing named barrier: they meet at named barriers below, and tcgen05.ld is warp-wide.
     const int pair_bar = 1 + q;
-    for (int t = next_valid(t_begin);; t = next_valid(t + 1)) {
+    float cs[32], sn[32];
+    // Position of this thread's row in the next unit, loaded one unit ahead.
+    auto row_pos = [&](int t) -> int64_t {
+      if (t < 0) return 0;
+      const TcJob &jb = jobs[t / tpj];
+      const int64_t row = (t % tpj) * TC_M + srow;
+      return row < jb.meta[ISKV_META_N] ? (int64_t)jb.pos[row] : 0;
+    };
+    int t = next_valid(t_begin);
+    int64_t ps_next = row_pos(t);
+    for (;;) {
       if (!named_and(pair_bar, 64, t >= 0 && !*abort)) break;
-      const int jj = t / tpj, row0 = (t % tpj) * TC_M;
+      const int tn = next_valid(t + 1);
+      const int64_t ps_raw = ps_next;
+      ps_next = row_pos(tn);  // consumed by the next unit: its latency hides behind this one
+      const int jj = t / tpj;
       const TcJob &jb = jobs[jj];
-      const int64_t n = jb.meta[ISKV_META_N];
-      const int64_t row = row0 + srow;
-      bool valid = row < n;
-      const int64_t ps = valid ? (int64_t)jb.pos[row] : 0;
+      bool valid = (t % tpj) * TC_M + srow < jb.meta[ISKV_META_N];
+      const int64_t ps = valid ? ps_raw : 0;
       if (valid && (ps < 0 || ps >= jb.n_total)) {
         record_status(jb.meta, ISKV_ERR_SHAPE);
         valid = false;
       }
-      // Rotation angles pos * theta^(-2j/128): reduced to [-pi, pi] in float64, then the fast
-      // hardware sine/cosine (absolute error ~1e-6 there, far below the bf16 output's rounding).
-      float cs[32], sn[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        cs[i] = 1.f;
-        sn[i] = 0.f;
-      }
       if (jb.rope != 0 && valid) {
 #pragma unroll
+        for (int i = 0; i < 32; ++i) rope_angle(rope_tab, j0 + i, (uint32_t)ps, cs[i], sn[i]);
+      } else {
+#pragma unroll
         for (int i = 0; i < 32; ++i) {
-          double a = (double)ps * invf[j0 + i];
-          a = fma(-two_pi, rint(a * inv_two_pi), a);
-          __sincosf((float)a, &sn[i], &cs[i]);
+          cs[i] = 1.f;
+          sn[i] = 0.f;
         }
       }
       __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(jb.out) + (size_t)(valid ? ps : 0) * D +
@@ -447,6 +484,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
       ++nc;
+      t = tn;
     }
     if (half == 0) bulk_wait0();
   }
@@ -642,7 +680,7 @@ size_t tc_rot_smem(int r) { return 1024 + (size_t)(r / 64) * SLAB_BYTES + (size_
 // RoPE frequencies.
 size_t tc_rec_smem(int r, int hp, int stages) {
   return 1024 + (size_t)hp * (r / 64) * SLAB_BYTES + (size_t)stages * SLAB_BYTES +
-         (size_t)TC_M * REC_STG_PITCH + sizeof(RecCtl) + 64 * sizeof(double);
+         (size_t)TC_M * REC_STG_PITCH + sizeof(RecCtl) + sizeof(RopeTab);
 }
 
 constexpr size_t kRecSmemCap = 227 * 1024;
@@ -716,6 +754,7 @@ cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob
   tc_rec_shape(p.r, p.n_heads, tp.hp, tp.stages);
   cudaError_t e = upload_jobs(djobs, hjobs.data(), sizeof(TcJob) * hjobs.size(), s);
   if (e != cudaSuccess) return e;
+  stage_mark(s, ST_RECON_PREPARE);  // sigma-scaled basis and the descriptor table are in place
   const size_t smem = tc_rec_smem(p.r, tp.hp, tp.stages);
   e = cudaFuncSetAttribute(k_rec_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -726,7 +765,7 @@ cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob
   int groups = num_sms() / G;
   if (groups < 1) groups = 1;
   if (groups > total) groups = total;
-  k_rec_tc<<<groups * G, TC_THREADS, smem, s>>>(djobs, tp);
+  k_rec_tc<<<groups * G, TC_THREADS, smem, s>>>(djobs, tp, make_rope_tab(p.theta));
   count_launches(1);
   return cudaGetLastError();
 }
