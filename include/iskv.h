@@ -128,7 +128,8 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
  * compressed rows, out[exact_pos[e], :] = exact_rows[e] for the n_exact exact rows; when
  * apply_rope != 0 every written row is then rotated by its own position with rotate-half RoPE
  * (pairs (j, j + head_dim/2) inside each head, angle pos * rope_theta^(-2j/head_dim)).
- * out          [n_total][d] out_dtype; rows not named by either set are left untouched.
+ * out          [n_total][d] out_dtype; rows not named by either set are left untouched. bf16 outputs
+ *              that are 16-byte aligned take the tensor-core path; others a CUDA-core path.
  * exact_rows   [n_exact][d] exact_dtype (may be NULL when n_exact == 0); exact_pos [n_exact].
  * Positions must be distinct across both sets; a position outside [0, n_total) is not written and
  * ISKV_ERR_SHAPE is recorded in the history's status word.

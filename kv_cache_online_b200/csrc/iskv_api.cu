@@ -373,7 +373,10 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReconJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "reconstruct: upload");
   stage_mark(s, ST_UPLOAD);
-  if (tc_recon_supported(r, p.storage, out_dtype, head_dim)) {
+  // The tensor-core path writes 16-byte vectors and tiles: every output must be 16-byte aligned.
+  bool outs_aligned = true;
+  for (int32_t i = 0; i < count; ++i) outs_aligned = outs_aligned && aligned(out[i], 16);
+  if (outs_aligned && tc_recon_supported(r, p.storage, out_dtype, head_dim)) {
     std::vector<TcJob> tj(count);
     for (int32_t i = 0; i < count; ++i)
       if (!encode_recon_job(tj[i], hs[i].U, hs[i].n_cap, r, jobs[i].bsig, d, out[i], hs[i].pos,

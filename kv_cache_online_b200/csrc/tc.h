@@ -15,6 +15,7 @@ namespace iskv {
 struct alignas(64) TcJob {
   CUtensorMap mapA;      // U [n_cap][r] bf16, box {64, 128}
   CUtensorMap mapB;      // rotation: G^T [r][r] bf16, box {64, r}; reconstruction: sigma B [d][r]
+  CUtensorMap mapO;      // reconstruction: out [n_total][d] bf16, box {64, 32} (tile stores)
   void *U;               // rotation output (in place)
   const int32_t *sc;     // rotation: the job's FS_* scalars
   void *out;             // reconstruction output [n_total][d] bf16
@@ -22,7 +23,7 @@ struct alignas(64) TcJob {
   int64_t *meta;         // status word target
   int64_t n_total;
   int32_t rope;
-  int32_t pad_;
+  int32_t tiles_ok;      // reconstruction: mapO is encoded (n_total >= 32), tile stores allowed
 };
 
 struct TcParams {

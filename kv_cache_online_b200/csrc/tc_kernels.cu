@@ -223,11 +223,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
 // served from L2 to the rest of the group. One MMA of N = hp x 128 covers all of the CTA's heads,
 // so the tensor core reads each A slab once per K step.
 //
-// Output rows are scattered (row i goes to position pos_i), so the epilogue stages each head's
-// 128 x 128 bf16 block in shared memory (rows padded by 16 bytes against bank conflicts) and
-// writes every row with one 256-byte bulk copy instead of 16-byte stores to 128 different lines.
+// Output rows go to their positions pos_i. The epilogue stages each head's 128 x 128 bf16 block
+// in shared memory as two 64-column halves in the 128-byte swizzled layout (bank-conflict-free
+// writes); a group of 32 rows whose positions are consecutive -- rows stored in position order,
+// the usual case -- then leaves with two TMA tile stores (32 rows x 64 columns each). Groups with
+// gaps or invalid rows are written from registers.
 constexpr int REC_MAX_STAGES = 8;
-constexpr int REC_STG_PITCH = 256 + 16;  // bytes per staged row
+constexpr int REC_STG_BYTES = 2 * TC_M * 128;  // lo and hi column halves of one head
 
 // RoPE tables (head_dim 128, 64 frequencies omega_j = theta^(-2j/128)). Angles are reduced in
 // exact integer arithmetic: W_j = omega_j / (2 pi) is held as a 0.64 fixed-point fraction
@@ -276,8 +278,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
   constexpr int HN = 128;                        // columns per head
   uint8_t *sB = smem;                            // KS slabs x (HP x 128 rows) x 128 B, resident
   uint8_t *sA = sB + KS * HP * SLAB_BYTES;       // NA slabs x 16 KB
-  uint8_t *sStg = sA + NA * SLAB_BYTES;          // 128 rows x REC_STG_PITCH
-  RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + TC_M * REC_STG_PITCH);
+  uint8_t *sStg = sA + NA * SLAB_BYTES;          // 2 x (128 rows x 128 B), SW128
+  RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + REC_STG_BYTES);
   RopeTab *rope_tab = reinterpret_cast<RopeTab *>(ctl + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NN = HP * HN;                        // MMA N
@@ -401,7 +403,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     const int q = warp & 3, half = (warp - 2) >> 2;
     const int j0 = half * 32;  // this thread's head-local pairs j0 .. j0 + 31 (cols j and j + 64)
     const int srow = q * 32 + lane;
-    uint8_t *stg = sStg + srow * REC_STG_PITCH;
+    uint8_t *stg_lo = sStg + srow * 128, *stg_hi = sStg + TC_M * 128 + srow * 128;
+    const bool issuer = half == 0 && lane == 0;  // issues this lane quarter's tile stores
     int nc = 0;
     // The two warps that share rows (q, half 0 and 1) take every decision together through an
     // AND-reducing named barrier: they meet at named barriers below, and tcgen05.ld is warp-wide.
@@ -441,6 +444,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       }
       __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(jb.out) + (size_t)(valid ? ps : 0) * D +
                             (size_t)member * HP * HN;
+      // This lane quarter's 32 rows go out as tiles when their positions are consecutive (the
+      // same answer in both warps of the pair: they hold the same rows).
+      const int64_t first = __shfl_sync(~0u, ps, 0);
+      const bool tiles = jb.tiles_ok && __all_sync(~0u, valid && ps == first + lane);
+      if (tiles && issuer) tensormap_acquire(&jb.mapO);
       const int buf = nc & 1, use = nc >> 1;
       if (!named_and(pair_bar, 64, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
         fail_timeout(ctl, jb.meta);
@@ -449,8 +457,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       fence_after_sync();
       const uint32_t base = tmem + buf * NN + ((uint32_t)(q * 32) << 16);
       for (int h = 0; h < HP; ++h) {
-        // The staged row is free once the previous bulk copy out of it has been read.
-        if (half == 0) bulk_wait_read0();
+        // The staged rows are free once the previous tile stores out of them have been read.
+        if (issuer) bulk_wait_read0();
         named_sync(pair_bar, 64);
 #pragma unroll
         for (int jb16 = 0; jb16 < 32; jb16 += 16) {
@@ -466,17 +474,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
             wl[i / 2] = pack_bf16(lo[i] * c0 - hi[i] * s0, lo[i + 1] * c1 - hi[i + 1] * s1);
             wh[i / 2] = pack_bf16(hi[i] * c0 + lo[i] * s0, hi[i + 1] * c1 + lo[i + 1] * s1);
           }
-          uint4 *dl = reinterpret_cast<uint4 *>(stg + 2 * (j0 + jb16));
-          uint4 *dh = reinterpret_cast<uint4 *>(stg + 2 * (64 + j0 + jb16));
-          dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-          dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
-          dh[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          dh[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+          if (tiles) {
+            // 16-byte chunk c of a 128-byte staged row sits at chunk c ^ (row & 7).
+            const int ck = (j0 + jb16) / 8, sw = srow & 7;
+            *reinterpret_cast<uint4 *>(stg_lo + 16 * (ck ^ sw)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            *reinterpret_cast<uint4 *>(stg_lo + 16 * ((ck + 1) ^ sw)) = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+            *reinterpret_cast<uint4 *>(stg_hi + 16 * (ck ^ sw)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            *reinterpret_cast<uint4 *>(stg_hi + 16 * ((ck + 1) ^ sw)) = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+          } else if (valid) {
+            uint4 *dl = reinterpret_cast<uint4 *>(orow + h * HN + j0 + jb16);
+            uint4 *dh = reinterpret_cast<uint4 *>(orow + h * HN + 64 + j0 + jb16);
+            dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+            dh[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            dh[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+          }
         }
         fence_proxy_async_smem();
         named_sync(pair_bar, 64);
-        if (half == 0 && valid) {
-          bulk_store(orow + h * HN, stg, 2 * HN);
+        if (tiles && issuer) {
+          const int x = (member * HP + h) * HN;
+          tma_store_2d(&jb.mapO, x, (int)first, sStg + q * 32 * 128);
+          tma_store_2d(&jb.mapO, x + 64, (int)first, sStg + TC_M * 128 + q * 32 * 128);
           bulk_commit();
         }
       }
@@ -486,7 +505,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       ++nc;
       t = tn;
     }
-    if (half == 0) bulk_wait0();
+    if (issuer) bulk_wait0();
   }
   fence_before_sync();
   __syncthreads();
@@ -680,7 +699,7 @@ size_t tc_rot_smem(int r) { return 1024 + (size_t)(r / 64) * SLAB_BYTES + (size_
 // RoPE frequencies.
 size_t tc_rec_smem(int r, int hp, int stages) {
   return 1024 + (size_t)hp * (r / 64) * SLAB_BYTES + (size_t)stages * SLAB_BYTES +
-         (size_t)TC_M * REC_STG_PITCH + sizeof(RecCtl) + sizeof(RopeTab);
+         (size_t)REC_STG_BYTES + sizeof(RecCtl) + sizeof(RopeTab);
 }
 
 constexpr size_t kRecSmemCap = 227 * 1024;
@@ -732,6 +751,8 @@ bool encode_recon_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void
   std::memset(&tj, 0, sizeof(tj));
   if (!encode_2d(&tj.mapA, U, (uint64_t)n_cap, (uint64_t)r, 128)) return false;
   if (!encode_2d(&tj.mapB, bsig, (uint64_t)d, (uint64_t)r, 128)) return false;
+  tj.tiles_ok = n_total >= 32;
+  if (tj.tiles_ok && !encode_2d(&tj.mapO, out, (uint64_t)n_total, (uint64_t)d, 32)) return false;
   tj.out = out;
   tj.pos = pos;
   tj.meta = meta;

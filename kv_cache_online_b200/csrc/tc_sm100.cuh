@@ -103,6 +103,16 @@ ISKV_DEV void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// TMA tile store shared -> global (box of the tensor map at coordinates {x, y}), tracked in the
+// issuing thread's bulk group.
+ISKV_DEV void tma_store_2d(const CUtensorMap *map, int x, int y, const void *smem_src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(smem_u32(smem_src))
+      : "memory");
+}
+
 // Named barrier with an AND reduction: every participating thread gets the AND of all their `v`.
 ISKV_DEV bool named_and(int id, int count, bool v) {
   uint32_t r;
