@@ -224,6 +224,16 @@ iskv_status iskv_stage_read(double *ms, int64_t *calls);
 void iskv_stage_reset(void);
 int64_t iskv_launch_count(void);
 
+/*
+ * Failure-path self-test (no counterpart on the pages; it lets failure detection be tested without
+ * faulting a GPU). Launches one CTA that waits on a shared-memory barrier nothing ever arrives at,
+ * through the same bounded wait the tensor-core kernels use, with a limit of `limit_ns`
+ * nanoseconds (clamped to [1e5, 2e9]). When the wait gives up, the kernel records
+ * ISKV_ERR_TIMEOUT in meta[3] (bit 1 << ISKV_ERR_TIMEOUT) as those kernels do, and returns; the
+ * context stays usable. meta: device int64[4], 8-byte aligned. Stream-ordered.
+ */
+iskv_status iskv_selftest_wait_timeout(int64_t *meta, int64_t limit_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

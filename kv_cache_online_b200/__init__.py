@@ -267,3 +267,11 @@ def stage_times(reset: bool = False):
 def launch_count() -> int:
     """Number of kernels the library has launched in this process."""
     return int(_lib.load().iskv_launch_count())
+
+
+def selftest_wait_timeout(hist, limit_ns: int = 10_000_000, stream=None):
+    """Run the failure-path self-test on ``hist``'s status word: a bounded wait that nothing
+    satisfies gives up after ``limit_ns`` and records ISKV_ERR_TIMEOUT (no GPU fault)."""
+    _lib.check(_lib.load().iskv_selftest_wait_timeout(hist.meta.data_ptr(), int(limit_ns),
+                                                      _stream(stream)), "selftest_wait_timeout")
+

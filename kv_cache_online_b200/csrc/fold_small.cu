@@ -12,10 +12,10 @@
 namespace iskv {
 
 // ------------------------------------------------------------------------------------------------
-// Job upload: a host array travels as kernel parameters, so the copy is stream-ordered and needs
-// no host buffer to outlive the call.
+// Job upload: a host array travels as kernel parameters (up to 16 KB per launch), so the copy is
+// stream-ordered and needs no host buffer to outlive the call.
 struct UploadChunk {
-  unsigned char data[3072];
+  unsigned char data[16384];
 };
 
 __global__ void k_upload(unsigned char *dst, UploadChunk c, int nbytes) {

@@ -157,10 +157,21 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
     j.pad_ = 0;
     if (hs[i].n_cap > ncap_max) ncap_max = hs[i].n_cap;
   }
+  const bool tc_rot = tc_rotation_supported(r, p.storage);
+  std::vector<TcJob> tj;
+  if (tc_rot) {
+    tj.resize(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_rotation_job(tj[i], hs[i].U, hs[i].n_cap, r, jobs[i].h.ws + p.ws.Gtb,
+                               reinterpret_cast<const int32_t *>(jobs[i].h.ws + p.ws.scal),
+                               hs[i].meta))
+        return fail(ISKV_ERR_CUDA, "fold: tensor map encoding failed");
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   FoldJob *djobs = reinterpret_cast<FoldJob *>(base);
   stage_begin(s);
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(FoldJob) * count, s);
+  if (e == cudaSuccess && tc_rot) e = upload_jobs(tc_dev, tj.data(), sizeof(TcJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "fold: upload");
   if ((e = launch_fold_prepare(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: prepare");
   stage_mark(s, ST_UPLOAD);
@@ -176,14 +187,8 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   if ((e = launch_rotate_basis(cj, rp, s)) != cudaSuccess)
     return cuda_fail(e, "fold: basis rotation");
   stage_mark(s, ST_FOLD_BASIS);
-  if (tc_rotation_supported(r, p.storage)) {
-    std::vector<TcJob> tj(count);
-    for (int32_t i = 0; i < count; ++i)
-      if (!encode_rotation_job(tj[i], hs[i].U, hs[i].n_cap, r, jobs[i].h.ws + p.ws.Gtb,
-                               reinterpret_cast<const int32_t *>(jobs[i].h.ws + p.ws.scal),
-                               hs[i].meta))
-        return fail(ISKV_ERR_CUDA, "fold: tensor map encoding failed");
-    e = launch_tc_rotation(tj.data(), count, tc_dev, r, ncap_max, s);
+  if (tc_rot) {
+    e = launch_tc_rotation(tc_dev, count, r, ncap_max, s);
   } else {
     e = launch_rotate_coords_ffma(cj, rp, ncap_max, s);
   }
@@ -286,6 +291,8 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   ReorthJob *djobs = reinterpret_cast<ReorthJob *>(base);
   stage_begin(s);
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReorthJob) * count, s);
+  if (e == cudaSuccess && p.gram_host) e = upload_jobs(gram_dev, gj.data(), sizeof(TcJob) * count, s);
+  if (e == cudaSuccess && p.tc_host) e = upload_jobs(tc_dev, tj.data(), sizeof(TcJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "reorth: upload");
   stage_mark(s, ST_UPLOAD);
   if ((e = launch_reorth(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "reorth");
@@ -347,6 +354,10 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
   p.count = count;
   p.theta = rope_theta;
   p.n_cap_max = ncap_max;
+  // Exact rows move as 16-byte vectors when every row starts on a 16-byte boundary.
+  p.exact_vec = head_dim % 16 == 0;
+  for (int32_t i = 0; i < count; ++i)
+    if (n_exact[i] > 0 && (!aligned(exact_rows[i], 16) || !aligned(out[i], 16))) p.exact_vec = 0;
   char *base = static_cast<char *>(ws);
   TcJob *tc_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReconJob)));
   const size_t jb = jobs_bytes(count, sizeof(ReconJob)) + tc_table_bytes(count);
@@ -367,22 +378,30 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
     j.apply_rope = apply_rope[i];
     j.pad_ = 0;
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ReconJob *djobs = reinterpret_cast<ReconJob *>(base);
-  stage_begin(s);
-  cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReconJob) * count, s);
-  if (e != cudaSuccess) return cuda_fail(e, "reconstruct: upload");
-  stage_mark(s, ST_UPLOAD);
   // The tensor-core path writes 16-byte vectors and tiles: every output must be 16-byte aligned.
   bool outs_aligned = true;
   for (int32_t i = 0; i < count; ++i) outs_aligned = outs_aligned && aligned(out[i], 16);
-  if (outs_aligned && tc_recon_supported(r, p.storage, out_dtype, head_dim)) {
-    std::vector<TcJob> tj(count);
+  const bool tc = outs_aligned && tc_recon_supported(r, p.storage, out_dtype, head_dim);
+  std::vector<TcJob> tj;
+  if (tc) {
+    tj.resize(count);
     for (int32_t i = 0; i < count; ++i)
       if (!encode_recon_job(tj[i], hs[i].U, hs[i].n_cap, r, jobs[i].bsig, d, out[i], hs[i].pos,
                             hs[i].meta, n_total[i], apply_rope[i]))
         return fail(ISKV_ERR_CUDA, "reconstruct: tensor map encoding failed");
-    e = launch_tc_recon(djobs, tj, tc_dev, p, s);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ReconJob *djobs = reinterpret_cast<ReconJob *>(base);
+  stage_begin(s);
+  cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReconJob) * count, s);
+  if (e == cudaSuccess && tc) e = upload_jobs(tc_dev, tj.data(), sizeof(TcJob) * count, s);
+  if (e != cudaSuccess) return cuda_fail(e, "reconstruct: upload");
+  stage_mark(s, ST_UPLOAD);
+  if (tc) {
+    if ((e = launch_recon_bsig(djobs, p, s)) != cudaSuccess)
+      return cuda_fail(e, "reconstruct: scaled basis");
+    stage_mark(s, ST_RECON_PREPARE);
+    e = launch_tc_recon(tc_dev, p, s);
   } else {
     stage_mark(s, ST_RECON_PREPARE);
     e = launch_recon_compressed(djobs, p, s);
@@ -493,3 +512,12 @@ iskv_status iskv_get_status(const iskv_lowrank *h, int64_t *k, int64_t *n, int64
 }
 
 }  // extern "C"
+
+extern "C" iskv_status iskv_selftest_wait_timeout(int64_t *meta, int64_t limit_ns, void *stream) {
+  g_last_error.clear();
+  if (!meta || !aligned(meta, 8)) return fail(ISKV_ERR_ARG, "selftest: meta must be 8-byte aligned");
+  int64_t ns = limit_ns < 100000 ? 100000 : (limit_ns > 2000000000 ? 2000000000 : limit_ns);
+  cudaError_t e = launch_wait_timeout(meta, (uint64_t)ns, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest: launch");
+  return ISKV_OK;
+}

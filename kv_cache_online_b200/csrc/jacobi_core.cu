@@ -8,9 +8,9 @@
 // are cut into 2 CJ blocks of w columns; each CTA holds two blocks in shared memory and a
 // round-robin tournament over the blocks (2 CJ - 1 rounds per sweep) moves blocks between CTAs
 // through distributed shared memory. Inside a round a CTA rotates every cross pair of its two
-// blocks (w steps of w disjoint pairs, one warp per pair); in the first round of a sweep it also
-// rotates the pairs inside each block. Dot products accumulate in float64, rotations apply in
-// float32.
+// blocks (w steps of w disjoint pairs, one half-warp per pair); in the first round of a sweep it
+// also rotates the pairs inside each block. Rotations apply in float32; inner products accumulate
+// in float32 (fold) or float64 (re-orthogonalisation).
 //
 // Structure used: the top k rows of A equal diag(sigma) times the top k rows of V (they start as
 // diag(sigma) and I and see the same column rotations), so those k rows of V are not stored:
@@ -84,54 +84,63 @@ JacobiCfg jacobi_cfg(int ncols_max, int col_len_max) {
 }
 
 bool core_cfg(int r, int b, bool dense, JacobiCfg &c) {
-  // Column length: the A part zero-padded to a multiple of 64, then the explicit V rows.
-  const int pad64 = dense ? (r + 63) / 64 * 64 : (r + b + 63) / 64 * 64;
-  const int len = dense ? pad64 + r : pad64 + b;
+  // Column length: the A part zero-padded to a multiple of 32, then the explicit V rows.
+  const int pad32 = dense ? (r + 31) / 32 * 32 : (r + b + 31) / 32 * 32;
+  const int len = dense ? pad32 + r : pad32 + b;
   c = jacobi_cfg(dense ? r : r + b, len);
   return c.ne > 0 && 16 * c.w <= core_max_threads(c.ne) && c.smem <= kCoreSmemCap;
 }
 
-// Register layout of a column: lane l holds the float2 pairs l + 32 q (elements 2 l + 64 q and
-// 2 l + 64 q + 1), q < NE / 2, so loads, stores and the arithmetic run on packed float2
-// (sm_100 issues one FFMA2 for two FMAs).
+// Register layout of a column: each half-warp holds one column; lane l16 = lane % 16 holds the
+// float2 pairs l16 + 16 q (elements 2 l16 + 32 q and 2 l16 + 32 q + 1), q < NE, so loads, stores
+// and the arithmetic run on packed float2 (sm_100 issues one FFMA2 for two FMAs), and the two
+// half-warps of a warp work on two column pairs with one instruction stream: the per-pair
+// rotation parameters and the 4-step reduction serve both pairs at once.
 template <int NE>
-ISKV_DEV void col_load(float2 (&x)[NE / 2], const float *src) {
+ISKV_DEV void col_load(float2 (&x)[NE], const float *src) {
   const float2 *s2 = reinterpret_cast<const float2 *>(src);
-  const int lane = threadIdx.x & 31;
+  const int l16 = threadIdx.x & 15;
 #pragma unroll
-  for (int q = 0; q < NE / 2; ++q) x[q] = s2[lane + 32 * q];
+  for (int q = 0; q < NE; ++q) x[q] = s2[l16 + 16 * q];
 }
 
 template <int NE>
-ISKV_DEV void col_store(float *dst, const float2 (&x)[NE / 2]) {
+ISKV_DEV void col_store(float *dst, const float2 (&x)[NE]) {
   float2 *d2 = reinterpret_cast<float2 *>(dst);
-  const int lane = threadIdx.x & 31;
+  const int l16 = threadIdx.x & 15;
 #pragma unroll
-  for (int q = 0; q < NE / 2; ++q) d2[lane + 32 * q] = x[q];
+  for (int q = 0; q < NE; ++q) d2[l16 + 16 * q] = x[q];
 }
 
-// Dot product of two register-resident columns over their first 64 nq entries (the A part,
-// zero-padded to a multiple of 64); the whole warp receives the sum.
+// Dot product of two half-warp-resident columns over their first 32 nq entries (the A part,
+// zero-padded to a multiple of 32); every lane of the half-warp receives the sum. Both half-warps
+// of the warp must call it together (the reduction shuffles across the whole warp).
 template <int NE, bool DD>
-ISKV_DEV float warp_dot(const float2 (&x)[NE / 2], const float2 (&y)[NE / 2], int nq) {
+ISKV_DEV float half_dot(const float2 (&x)[NE], const float2 (&y)[NE], int nq) {
   if (DD) {  // float64 accumulation of the exact float32 products
     double a0 = 0.0, a1 = 0.0;
 #pragma unroll
-    for (int q = 0; q < NE / 2; ++q)
+    for (int q = 0; q < NE; ++q)
       if (q < nq) {
         a0 = fma((double)x[q].x, (double)y[q].x, a0);
         a1 = fma((double)x[q].y, (double)y[q].y, a1);
       }
-    return (float)warp_sum(a0 + a1);
+    double v = a0 + a1;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return (float)v;
   }
   float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int q = 0; q < NE / 2; ++q)
+  for (int q = 0; q < NE; ++q)
     if (q < nq) {
       if (q & 1) a1 = __ffma2_rn(x[q], y[q], a1);
       else a0 = __ffma2_rn(x[q], y[q], a0);
     }
-  return warp_sum((a0.x + a1.x) + (a0.y + a1.y));
+  float v = (a0.x + a1.x) + (a0.y + a1.y);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 // One Jacobi rotation of the pair (x, y) with squared norms ax, by and inner product g, when the
@@ -145,7 +154,7 @@ ISKV_DEV float warp_dot(const float2 (&x)[NE / 2], const float2 (&y)[NE / 2], in
 // reciprocal square root. Norms follow Rutishauser: ax -= t g, by += t g. Both accumulation modes
 // (DD: the inner products were summed in float64) use these float32 parameters.
 template <int NE, bool DD>
-ISKV_DEV bool rotate_regs(float2 (&x)[NE / 2], float2 (&y)[NE / 2], float &ax, float &by, float g,
+ISKV_DEV bool rotate_regs(float2 (&x)[NE], float2 (&y)[NE], float &ax, float &by, float g,
                           float tol2) {
   if (!(g != 0.f && g * g > (tol2 * ax) * by)) return false;
   const float zeta = 0.5f * (by - ax) * __fdividef(1.f, g);
@@ -163,7 +172,7 @@ ISKV_DEV bool rotate_regs(float2 (&x)[NE / 2], float2 (&y)[NE / 2], float &ax, f
   const float2 s2 = make_float2(s, s), ms2 = make_float2(-s, -s);
   const float2 t2 = make_float2(tau, tau), mt2 = make_float2(-tau, -tau);
 #pragma unroll
-  for (int q = 0; q < NE / 2; ++q) {
+  for (int q = 0; q < NE; ++q) {
     const float2 xv = x[q], yv = y[q];
     x[q] = __ffma2_rn(ms2, __ffma2_rn(t2, xv, yv), xv);
     y[q] = __ffma2_rn(s2, __ffma2_rn(mt2, yv, xv), yv);
@@ -189,8 +198,8 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   const int k = sc[FS_K_OLD], b = dense ? 0 : p.b, r = p.r, hs = p.hs;
   const int pp = dense ? k : sc[FS_P];          // explicit V rows stored after the A part
   const int m = k + b;                          // A rows
-  const int mp = (m + 63) / 64 * 64;            // A part zero-padded to whole float2 lanes
-  const int nq = mp / 64;                       // float2 pairs per lane in the A part
+  const int mp = (m + 31) / 32 * 32;            // A part zero-padded to whole half-warp rows
+  const int nq = mp / 32;                       // float2 pairs per lane in the A part
   const int ncol = dense ? k : k + pp, kn = min(r, ncol);
   const CoreSmem S = core_smem(cj, w, NE, dbuf != 0);
   extern __shared__ float smem[];
@@ -203,8 +212,9 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   float *nrm_all = smem + S.nrm_all;
   int *flags = reinterpret_cast<int *>(smem + S.flags);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nw = w / 2;                         // warps; warp i owns columns i and i + nw
-  const int c0 = warp, c1 = warp + nw;
+  const int nw = w / 2;                         // warps; half-warp h of warp i owns column i + h nw
+  const int l16 = lane & 15;
+  const int c = warp + (lane >> 4) * nw;
 
   // Tournament: round t, CTA 0 plays block M-1 against block t; CTA i plays (t+i) vs (t-i).
   for (int e = tid; e < (M - 1) * cj; e += blockDim.x) {
@@ -262,71 +272,55 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
       float *Pb = buf, *Qb = buf + w * LP;
       // Exact squared norms at the start of the round; tracked through the round's rotations.
       {
-        float2 x[NE / 2], y[NE / 2];
-        col_load<NE>(x, Pb + c0 * LP);
-        col_load<NE>(y, Qb + c0 * LP);
-        float a = warp_dot<NE, DD>(x, x, nq), c = warp_dot<NE, DD>(y, y, nq);
-        if (lane == 0) { nP[c0] = a; nQ[c0] = c; }
-        col_load<NE>(x, Pb + c1 * LP);
-        col_load<NE>(y, Qb + c1 * LP);
-        a = warp_dot<NE, DD>(x, x, nq);
-        c = warp_dot<NE, DD>(y, y, nq);
-        if (lane == 0) { nP[c1] = a; nQ[c1] = c; }
+        float2 x[NE], y[NE];
+        col_load<NE>(x, Pb + c * LP);
+        col_load<NE>(y, Qb + c * LP);
+        const float a = half_dot<NE, DD>(x, x, nq), cq = half_dot<NE, DD>(y, y, nq);
+        if (l16 == 0) { nP[c] = a; nQ[c] = cq; }
       }
       __syncthreads();
       if (t == 0) {
-        // Pairs inside each block (both columns from shared memory); pair indices c0 and c1.
+        // Pairs inside each block (both columns from shared memory): half-warp c takes pair
+        // c mod w/2 of block c / (w/2).
         for (int st = 0; st < w - 1; ++st) {
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int pi = u ? c1 : c0;
-            const int slot = pi < w / 2 ? 0 : 1, q = pi % (w / 2);
-            const int a = circle_player(q, st, w), bb = circle_player(w - 1 - q, st, w);
-            float *base = slot ? Qb : Pb;
-            float *nb = slot ? nQ : nP;
-            float2 x[NE / 2], y[NE / 2];
-            col_load<NE>(x, base + a * LP);
-            col_load<NE>(y, base + bb * LP);
-            float ax = nb[a], by = nb[bb];
-            const float g = warp_dot<NE, DD>(x, y, nq);
-            if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
-              col_store<NE>(base + a * LP, x);
-              col_store<NE>(base + bb * LP, y);
-              if (lane == 0) { nb[a] = ax; nb[bb] = by; }
-              rot = true;
-            }
+          const int slot = c < w / 2 ? 0 : 1, q = slot ? c - w / 2 : c;
+          const int a = circle_player(q, st, w), bb = circle_player(w - 1 - q, st, w);
+          float *base = slot ? Qb : Pb;
+          float *nb = slot ? nQ : nP;
+          float2 x[NE], y[NE];
+          col_load<NE>(x, base + a * LP);
+          col_load<NE>(y, base + bb * LP);
+          float ax = nb[a], by = nb[bb];
+          const float g = half_dot<NE, DD>(x, y, nq);
+          if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
+            col_store<NE>(base + a * LP, x);
+            col_store<NE>(base + bb * LP, y);
+            if (l16 == 0) { nb[a] = ax; nb[bb] = by; }
+            rot = true;
           }
           __syncthreads();
         }
       }
-      // Cross pairs: warp i keeps P[i] and P[i + w/2] in registers while the Q columns circulate.
-      float2 x0[NE / 2], x1[NE / 2];
-      col_load<NE>(x0, Pb + c0 * LP);
-      col_load<NE>(x1, Pb + c1 * LP);
-      float ax0 = nP[c0], ax1 = nP[c1];
+      // Cross pairs: half-warp c keeps P[c] in registers while the Q columns circulate.
+      float2 x[NE];
+      col_load<NE>(x, Pb + c * LP);
+      float ax = nP[c];
       for (int st = 0; st < w; ++st) {
-        const int q0 = (c0 + st) % w, q1 = (c1 + st) % w;
-        float2 y0[NE / 2], y1[NE / 2];
-        col_load<NE>(y0, Qb + q0 * LP);
-        col_load<NE>(y1, Qb + q1 * LP);
-        float by0 = nQ[q0], by1 = nQ[q1];
-        const float g0 = warp_dot<NE, DD>(x0, y0, nq);
-        const float g1 = warp_dot<NE, DD>(x1, y1, nq);
-        if (rotate_regs<NE, DD>(x0, y0, ax0, by0, g0, tol2)) {
-          col_store<NE>(Qb + q0 * LP, y0);
-          if (lane == 0) nQ[q0] = by0;
-          rot = true;
-        }
-        if (rotate_regs<NE, DD>(x1, y1, ax1, by1, g1, tol2)) {
-          col_store<NE>(Qb + q1 * LP, y1);
-          if (lane == 0) nQ[q1] = by1;
+        int qc = c + st;  // (c + st) mod w, with c, st < w
+        if (qc >= w) qc -= w;
+        float2 y[NE];
+        col_load<NE>(y, Qb + qc * LP);
+        float by = nQ[qc];
+        const float g = half_dot<NE, DD>(x, y, nq);
+        if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
+          col_store<NE>(Qb + qc * LP, y);
+          if (l16 == 0) nQ[qc] = by;
           rot = true;
         }
         __syncthreads();
       }
       if (cj == 1) {
-        col_store<NE>(Pb + c0 * LP, x0);
-        col_store<NE>(Pb + c1 * LP, x1);
+        col_store<NE>(Pb + c * LP, x);
         __syncthreads();
         continue;
       }
@@ -334,18 +328,15 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
       const int tn = (t + 1) % (M - 1);
       const int X0 = pairs[(t * cj + rank) * 2 + 0], X1 = pairs[(t * cj + rank) * 2 + 1];
       const int d0 = where[tn * M + X0], d1 = where[tn * M + X1];
-      float2 y0[NE / 2], y1[NE / 2];
-      col_load<NE>(y0, Qb + c0 * LP);
-      col_load<NE>(y1, Qb + c1 * LP);
+      float2 y[NE];
+      col_load<NE>(y, Qb + c * LP);
       float *dst = dbuf ? buf0 + (cur ^ 1) * bufw : buf0;
       if (!dbuf) cluster.sync();  // single buffer: everyone has read its blocks before writes
       {
         float *r0 = cluster.map_shared_rank(dst, d0 >> 1) + (d0 & 1) * w * LP;
         float *r1 = cluster.map_shared_rank(dst, d1 >> 1) + (d1 & 1) * w * LP;
-        col_store<NE>(r0 + c0 * LP, x0);
-        col_store<NE>(r0 + c1 * LP, x1);
-        col_store<NE>(r1 + c0 * LP, y0);
-        col_store<NE>(r1 + c1 * LP, y1);
+        col_store<NE>(r0 + c * LP, x);
+        col_store<NE>(r1 + c * LP, y);
       }
       cluster.sync();
       if (dbuf) cur ^= 1;

@@ -9,8 +9,12 @@
 namespace iskv {
 
 // Round-robin ("circle") pairing: n even players, player 0 fixed, the rest rotate by `step`.
+// Requires 0 <= i < n and 0 <= step < n - 1 (so one conditional subtraction reduces mod n - 1).
 ISKV_DEV int circle_player(int i, int step, int n) {
-  return i == 0 ? 0 : ((i - 1 + step) % (n - 1)) + 1;
+  if (i == 0) return 0;
+  int v = i - 1 + step;
+  if (v >= n - 1) v -= n - 1;
+  return v + 1;
 }
 
 // Orthogonalise the `ncols` columns of M (column-major, leading dimension ld, `rows` <= 128 rows)

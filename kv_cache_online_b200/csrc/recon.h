@@ -23,6 +23,7 @@ struct ReconJob {
 
 struct ReconParams {
   int d, r, storage, exact_dtype, out_dtype, n_heads, head_dim, count;
+  int exact_vec;  // exact rows move as 16-byte vectors (head_dim % 16 == 0, 16-byte aligned rows)
   double theta;
   int64_t n_cap_max;
 };

@@ -100,9 +100,39 @@ __global__ void __launch_bounds__(256) k_recon_ffma(const ReconJob *jobs, ReconP
   }
 }
 
-// Exact rows: copy (and rotate) exact_rows[e] to out[exact_pos[e]]. Thread = (row, head, pair);
-// consecutive threads take consecutive pairs of a head, so loads and stores are contiguous.
-template <typename TE, typename TO>
+// Eight consecutive elements as floats (16-byte aligned source / destination).
+ISKV_DEV void load8(const __nv_bfloat16 *p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+ISKV_DEV void load8(const float *p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+ISKV_DEV void store8(__nv_bfloat16 *p, const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+ISKV_DEV void store8(float *p, const float (&v)[8]) {
+  reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// Exact rows: copy (and rotate) exact_rows[e] to out[exact_pos[e]]. Thread = (row, head, group of
+// V consecutive pairs); consecutive threads take consecutive groups of a head, so loads and stores
+// are contiguous. V = 8 moves 16-byte vectors (head_dim a multiple of 16, rows 16-byte aligned).
+template <typename TE, typename TO, int V>
 __global__ void __launch_bounds__(256) k_recon_exact(const ReconJob *jobs, ReconParams p) {
   const ReconJob &jb = jobs[blockIdx.y];
   const int hd = p.head_dim, half = hd / 2, d = p.d, H = p.n_heads;
@@ -112,31 +142,47 @@ __global__ void __launch_bounds__(256) k_recon_exact(const ReconJob *jobs, Recon
     for (int j = threadIdx.x; j < half; j += blockDim.x) invf[j] = rope_inv_freq(j, hd, lt);
   }
   __syncthreads();
-  const int per_row = H * half;
-  const int64_t npairs = jb.n_exact * (int64_t)per_row;
+  const int groups = half / V, per_row = H * groups;
+  const int64_t nwork = jb.n_exact * (int64_t)per_row;
   const TE *X = static_cast<const TE *>(jb.exact_rows);
   TO *out = static_cast<TO *>(jb.out);
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < npairs;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < nwork;
        t += (int64_t)gridDim.x * blockDim.x) {
     const int64_t e = t / per_row;
     const int rem = (int)(t - e * per_row);
-    const int h = rem / half, c = rem - h * half;
+    const int h = rem / groups, c = (rem - h * groups) * V;
     const int64_t ps = jb.exact_pos[e];
     if (ps < 0 || ps >= jb.n_total) {
       record_status(jb.meta, ISKV_ERR_SHAPE);
       continue;
     }
-    float x1 = to_f<TE>(X[(size_t)e * d + h * hd + c]);
-    float x2 = to_f<TE>(X[(size_t)e * d + h * hd + c + half]);
-    if (jb.apply_rope) {
-      float cs, sn;
-      rope_sincos(ps, invf[c], cs, sn);
-      const float y1 = x1 * cs - x2 * sn, y2 = x2 * cs + x1 * sn;
-      x1 = y1;
-      x2 = y2;
+    const TE *src = X + (size_t)e * d + h * hd + c;
+    TO *dst = out + (size_t)ps * d + h * hd + c;
+    float x1[V], x2[V];
+    if constexpr (V == 8) {
+      load8(src, x1);
+      load8(src + half, x2);
+    } else {
+      x1[0] = to_f<TE>(src[0]);
+      x2[0] = to_f<TE>(src[half]);
     }
-    out[(size_t)ps * d + h * hd + c] = from_f<TO>(x1);
-    out[(size_t)ps * d + h * hd + c + half] = from_f<TO>(x2);
+    if (jb.apply_rope) {
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        float cs, sn;
+        rope_sincos(ps, invf[c + i], cs, sn);
+        const float y1 = x1[i] * cs - x2[i] * sn, y2 = x2[i] * cs + x1[i] * sn;
+        x1[i] = y1;
+        x2[i] = y2;
+      }
+    }
+    if constexpr (V == 8) {
+      store8(dst, x1);
+      store8(dst + half, x2);
+    } else {
+      dst[0] = from_f<TO>(x1[0]);
+      dst[half] = from_f<TO>(x2[0]);
+    }
   }
 }
 
@@ -164,14 +210,22 @@ cudaError_t launch_recon_compressed(const ReconJob *jobs, const ReconParams &p, 
 cudaError_t launch_recon_exact(const ReconJob *jobs, const ReconParams &p, int64_t max_exact,
                                cudaStream_t s) {
   if (max_exact <= 0) return cudaSuccess;
-  const int64_t work = max_exact * (int64_t)p.n_heads * (p.head_dim / 2);
+  const int V = p.exact_vec ? 8 : 1;
+  const int64_t work = max_exact * (int64_t)p.n_heads * (p.head_dim / 2 / V);
   const unsigned gx = (unsigned)((work + 255) / 256 < 4096 ? (work + 255) / 256 : 4096);
   const dim3 g(gx, p.count);
   const bool eb = p.exact_dtype == ISKV_BF16, ob = p.out_dtype == ISKV_BF16;
-  if (eb && ob) k_recon_exact<__nv_bfloat16, __nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
-  else if (eb) k_recon_exact<__nv_bfloat16, float><<<g, 256, 0, s>>>(jobs, p);
-  else if (ob) k_recon_exact<float, __nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
-  else k_recon_exact<float, float><<<g, 256, 0, s>>>(jobs, p);
+  if (V == 8) {
+    if (eb && ob) k_recon_exact<__nv_bfloat16, __nv_bfloat16, 8><<<g, 256, 0, s>>>(jobs, p);
+    else if (eb) k_recon_exact<__nv_bfloat16, float, 8><<<g, 256, 0, s>>>(jobs, p);
+    else if (ob) k_recon_exact<float, __nv_bfloat16, 8><<<g, 256, 0, s>>>(jobs, p);
+    else k_recon_exact<float, float, 8><<<g, 256, 0, s>>>(jobs, p);
+  } else {
+    if (eb && ob) k_recon_exact<__nv_bfloat16, __nv_bfloat16, 1><<<g, 256, 0, s>>>(jobs, p);
+    else if (eb) k_recon_exact<__nv_bfloat16, float, 1><<<g, 256, 0, s>>>(jobs, p);
+    else if (ob) k_recon_exact<float, __nv_bfloat16, 1><<<g, 256, 0, s>>>(jobs, p);
+    else k_recon_exact<float, float, 1><<<g, 256, 0, s>>>(jobs, p);
+  }
   count_launches(1);
   return cudaGetLastError();
 }

@@ -321,7 +321,7 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
     gp.split = REORTH_SPLIT;
     gp.off_gu = W.gpart_u;
     gp.off_gb = W.gpart_b;
-    cudaError_t e0 = launch_tc_gram(p.gram_host, p.gram_dev, gp, s);
+    cudaError_t e0 = launch_tc_gram(p.gram_dev, gp, s);
     if (e0 != cudaSuccess) return e0;
   } else if (p.storage == ISKV_BF16) {
     k_gram_partial<__nv_bfloat16><<<dim3(tn, tm, p.count * W.nsplit_u), 256, 0, s>>>(jobs, p, 0, W.nsplit_u);
@@ -392,7 +392,7 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   q.hs = r;
   q.pld = 1;
   if (p.tc_host)
-    e = launch_tc_rotation(p.tc_host, p.count, p.tc_dev, r, p.n_cap, s);
+    e = launch_tc_rotation(p.tc_dev, p.count, r, p.n_cap, s);
   else
     e = launch_rotate_coords_ffma(reinterpret_cast<const char *>(jobs), q, p.n_cap, s);
   if (e != cudaSuccess) return e;

@@ -43,7 +43,8 @@ struct GramParams {
 bool tc_gram_supported(int r, int storage);
 bool encode_gram_job(TcJob &tj, const void *U, int64_t n_cap, const void *B, int d, int r,
                      const int32_t *sc, int64_t *meta, void *ws);
-cudaError_t launch_tc_gram(const TcJob *hjobs, TcJob *djobs, const GramParams &p, cudaStream_t s);
+// The launchers take job tables already uploaded to the device (upload_jobs).
+cudaError_t launch_tc_gram(const TcJob *djobs, const GramParams &p, cudaStream_t s);
 
 bool tc_rotation_supported(int r, int storage);
 bool tc_recon_supported(int r, int storage, int out_dtype, int head_dim);
@@ -53,10 +54,14 @@ bool encode_rotation_job(TcJob &tj, void *U, int64_t n_cap, int r, const void *g
 bool encode_recon_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void *bsig, int d,
                       void *out, const int32_t *pos, int64_t *meta, int64_t n_total, int rope);
 
-cudaError_t launch_tc_rotation(const TcJob *hjobs, int count, TcJob *djobs, int r,
-                               int64_t n_cap_max, cudaStream_t s);
-cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob> &hjobs,
-                            TcJob *djobs, const ReconParams &p, cudaStream_t s);
+cudaError_t launch_tc_rotation(const TcJob *djobs, int count, int r, int64_t n_cap_max,
+                               cudaStream_t s);
+// Sigma-scaled basis for every job (the operand of launch_tc_recon); stage "reconstruct.prepare".
+cudaError_t launch_recon_bsig(const ReconJob *djobs_recon, const ReconParams &p, cudaStream_t s);
+cudaError_t launch_tc_recon(const TcJob *djobs, const ReconParams &p, cudaStream_t s);
+
+// One CTA waiting on a barrier nothing arrives at, bounded by limit_ns (failure-path self-test).
+cudaError_t launch_wait_timeout(int64_t *meta, uint64_t limit_ns, cudaStream_t s);
 
 inline size_t tc_table_bytes(int count) { return ((size_t)count * sizeof(TcJob) + 255) / 256 * 256; }
 

@@ -640,6 +640,26 @@ __global__ void k_bsig(const ReconJob *jobs, int d, int r) {
 }
 
 // ================================================================================================
+// Failure-path self-test: a bounded wait on a barrier that nothing arrives at.
+__global__ void k_wait_timeout(int64_t *meta, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort, limit_ns)) record_status(meta, ISKV_ERR_TIMEOUT);
+}
+
+cudaError_t launch_wait_timeout(int64_t *meta, uint64_t limit_ns, cudaStream_t s) {
+  k_wait_timeout<<<1, 32, 0, s>>>(meta, limit_ns);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ================================================================================================
 // Host side: tensor-map encoding through the driver entry point, job tables, launches.
 
 namespace {
@@ -693,7 +713,9 @@ bool tc_recon_supported(int r, int storage, int out_dtype, int head_dim) {
          r >= 64 && r <= 256 && encode_fn() != nullptr;
 }
 
-size_t tc_rot_smem(int r) { return 1024 + (size_t)(r / 64) * SLAB_BYTES + (size_t)(r / 64) * r * 128 + sizeof(TcCtl); }
+size_t tc_rot_smem(int r) {
+  return 1024 + (size_t)(r / 64) * SLAB_BYTES + (size_t)(r / 64) * r * 128 + sizeof(TcCtl);
+}
 
 // Resident basis rows for hp heads, the U slab ring, the output staging rows, the barriers and the
 // RoPE frequencies.
@@ -712,8 +734,8 @@ void tc_rec_shape(int r, int n_heads, int &hp, int &stages) {
   while (stages > 2 && tc_rec_smem(r, hp, stages) > kRecSmemCap) --stages;
 }
 
-cudaError_t launch_tc_rotation(const TcJob *hjobs, int count, TcJob *djobs, int r,
-                               int64_t n_cap_max, cudaStream_t s) {
+cudaError_t launch_tc_rotation(const TcJob *djobs, int count, int r, int64_t n_cap_max,
+                               cudaStream_t s) {
   TcParams tp;
   tp.r = r;
   tp.d = 0;
@@ -723,10 +745,8 @@ cudaError_t launch_tc_rotation(const TcJob *hjobs, int count, TcJob *djobs, int 
   tp.count = count;
   tp.tiles_per_job = (int)((n_cap_max + TC_M - 1) / TC_M);
   tp.theta = 0.0;
-  cudaError_t e = upload_jobs(djobs, hjobs, sizeof(TcJob) * count, s);
-  if (e != cudaSuccess) return e;
   const size_t smem = tc_rot_smem(r);
-  e = cudaFuncSetAttribute(k_rot_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(k_rot_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int total = tp.count * tp.tiles_per_job;
   const int grid = total < num_sms() ? total : num_sms();
@@ -761,10 +781,13 @@ bool encode_recon_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void
   return true;
 }
 
-cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob> &hjobs,
-                            TcJob *djobs, const ReconParams &p, cudaStream_t s) {
+cudaError_t launch_recon_bsig(const ReconJob *djobs_recon, const ReconParams &p, cudaStream_t s) {
   k_bsig<<<dim3(64, p.count), 256, 0, s>>>(djobs_recon, p.d, p.r);
   count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_recon(const TcJob *djobs, const ReconParams &p, cudaStream_t s) {
   TcParams tp;
   tp.r = p.r;
   tp.d = p.d;
@@ -773,11 +796,8 @@ cudaError_t launch_tc_recon(const ReconJob *djobs_recon, const std::vector<TcJob
   tp.tiles_per_job = (int)((p.n_cap_max + TC_M - 1) / TC_M);
   tp.theta = p.theta;
   tc_rec_shape(p.r, p.n_heads, tp.hp, tp.stages);
-  cudaError_t e = upload_jobs(djobs, hjobs.data(), sizeof(TcJob) * hjobs.size(), s);
-  if (e != cudaSuccess) return e;
-  stage_mark(s, ST_RECON_PREPARE);  // sigma-scaled basis and the descriptor table are in place
   const size_t smem = tc_rec_smem(p.r, tp.hp, tp.stages);
-  e = cudaFuncSetAttribute(k_rec_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(k_rec_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Whole groups of n_heads / hp CTAs, as many as fit one per SM (at least one group), and no
   // more groups than row tiles.
@@ -806,9 +826,8 @@ bool encode_gram_job(TcJob &tj, const void *U, int64_t n_cap, const void *B, int
   return true;
 }
 
-cudaError_t launch_tc_gram(const TcJob *hjobs, TcJob *djobs, const GramParams &p, cudaStream_t s) {
-  cudaError_t e = upload_jobs(djobs, hjobs, sizeof(TcJob) * p.count, s);
-  if (e != cudaSuccess) return e;
+cudaError_t launch_tc_gram(const TcJob *djobs, const GramParams &p, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
   const size_t smem = 1024 + (size_t)GRAM_STAGES * (p.r / 64) * GRAM_KT * 128 + sizeof(TcCtl) +
                       2 * GRAM_STAGES * sizeof(uint64_t);
   e = cudaFuncSetAttribute(k_gram_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
