@@ -81,7 +81,9 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
   float *vdiag = smem + L.vdiag, *alph = smem + L.alph, *tauv = smem + L.tauv;
   const int tid = threadIdx.x;
   const float *E = reinterpret_cast<const float *>(jb.h.ws + p.ws.E);
-  float *T = reinterpret_cast<float *>(jb.h.ws + p.ws.T);
+  // Compact-WY factor T (b x b, rank 0): kept in the F P partial buffer, which is idle until
+  // the end; each thread of rank 0 builds and re-reads only its own row.
+  float *T = fpp;
   float *W = reinterpret_cast<float *>(jb.h.ws + p.ws.W);
   float *Y2 = reinterpret_cast<float *>(jb.h.ws + p.ws.Y2);
   float *P = reinterpret_cast<float *>(jb.h.ws + p.ws.P);
@@ -221,7 +223,7 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
     }
     __syncthreads();
     // Y1 = V_top^T W_p (V_top = rows 0..b-1 of the reflectors, lower triangular), Y2 = T Y1.
-    float *Y1 = fpp;  // scratch, b x b
+    float *Y1 = Rm;  // scratch, b x b (R_R's columns are no longer needed once W is formed)
     for (int e = tid; e < b * pp; e += RES_NTH) {
       const int l = e / pp, q = e % pp;
       double s = (double)vdiag[l] * W[l * b + q];
@@ -242,28 +244,98 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
   // p broadcast: every CTA reads rank 0's s_p.
   const int pp = *cluster.map_shared_rank(&s_p, 0);
 
-  // ---- P rows: P = [W_p; 0] - V Y2 for my rows, then my partial of F P.
-  for (int e = tid; e < rpc * pp; e += RES_NTH) {
-    const int i = e / pp, q = e % pp;
-    const int gi = row0 + i;
-    double s = gi < b ? (double)W[gi * b + q] : 0.0;
-    const int lmax = min(gi, b - 1);
-    for (int l = 0; l <= lmax; ++l) {
-      const double v = gi == l ? (double)vdiag[l] : (double)A[i * b + l];
-      s = fma(-v, (double)Y2[l * b + q], s);
-    }
-    P[(size_t)gi * b + q] = (float)s;
+  // ---- P rows: P = [W_p; 0] - V Y2 for my rows, then my partial of F P. Both are small
+  // products done with 8 x 8 (P) and 4 x 4 (F P) register tiles in float32; Y2 and my P rows are
+  // staged in shared memory (R_R's buffer and the reflector buffer, both free by now).
+  float *Y2s = Rm;  // b x b, Y2[l][q] at l * b + q
+  for (int e = tid; e < b * b; e += RES_NTH) {
+    const int l = e / b, q = e % b;
+    Y2s[e] = q < pp ? Y2[l * b + q] : 0.f;
   }
   __syncthreads();
-  // F P partial over my rows (read P back from global: written by this CTA, visible after the
-  // barrier above for the same CTA).
+  {
+    // Thread (ti, tq) owns rows ti*8 .. ti*8+7 (strided by rpc/8 groups) and columns tq*8 .. tq*8+7.
+    constexpr int PT = 8;
+    const int ncg = (b + PT - 1) / PT;              // column groups
+    const int nrg = RES_NTH / ncg;                  // row groups
+    const int tq = tid % ncg, tig = tid / ncg;
+    const int niter = (rpc + nrg * PT - 1) / (nrg * PT);  // the same for every thread (barrier)
+    float acc[PT][PT];
+    for (int it = 0; it < niter; ++it) {
+      const int i0 = (it * nrg + tig) * PT;
+#pragma unroll
+      for (int u = 0; u < PT; ++u)
+#pragma unroll
+        for (int v = 0; v < PT; ++v) acc[u][v] = 0.f;
+      for (int l = 0; l < b; ++l) {
+        float yv[PT], vv[PT];
+#pragma unroll
+        for (int v = 0; v < PT; ++v) yv[v] = Y2s[l * b + tq * PT + v];
+#pragma unroll
+        for (int u = 0; u < PT; ++u) {
+          const int i = i0 + u, gi = row0 + i;
+          vv[u] = (i < rpc && gi >= l) ? (gi == l ? vdiag[l] : A[i * b + l]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < PT; ++u)
+#pragma unroll
+          for (int v = 0; v < PT; ++v) acc[u][v] = fmaf(vv[u], yv[v], acc[u][v]);
+      }
+      __syncthreads();  // every thread has read the reflectors of its rows before any is replaced
+#pragma unroll
+      for (int u = 0; u < PT; ++u) {
+        const int i = i0 + u, gi = row0 + i;
+        if (i >= rpc) continue;
+#pragma unroll
+        for (int v = 0; v < PT; ++v) {
+          const int q = tq * PT + v;
+          if (q >= b) continue;
+          const float wv = (gi < b && q < pp) ? W[gi * b + q] : 0.f;
+          const float pv = q < pp ? wv - acc[u][v] : 0.f;
+          A[i * b + q] = pv;                 // my P rows, for F P below
+          if (q < pp) P[(size_t)gi * b + q] = pv;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // F P partial over my rows: fpp[m][q] = sum_i F[m][row0 + i] P[row0 + i][q].
   const TF *F = static_cast<const TF *>(jb.F);
-  for (int e = tid; e < b * pp; e += RES_NTH) {
-    const int m = e / pp, q = e % pp;
-    double s = 0.0;
-    for (int i = 0; i < rpc; ++i)
-      s = fma((double)to_f<TF>(F[(size_t)m * d + row0 + i]), (double)P[(size_t)(row0 + i) * b + q], s);
-    fpp[m * b + q] = (float)s;
+  {
+    constexpr int FT = 4;
+    const int ncg = (b + FT - 1) / FT, nmg = (b + FT - 1) / FT;
+    for (int g = tid; g < ncg * nmg; g += RES_NTH) {
+      const int tq = g % ncg, tm = g / ncg;
+      float acc[FT][FT];
+#pragma unroll
+      for (int u = 0; u < FT; ++u)
+#pragma unroll
+        for (int v = 0; v < FT; ++v) acc[u][v] = 0.f;
+      for (int i = 0; i < rpc; ++i) {
+        float fv[FT], pv[FT];
+#pragma unroll
+        for (int u = 0; u < FT; ++u) {
+          const int m = tm * FT + u;
+          fv[u] = m < b ? to_f<TF>(F[(size_t)m * d + row0 + i]) : 0.f;
+        }
+#pragma unroll
+        for (int v = 0; v < FT; ++v) {
+          const int q = tq * FT + v;
+          pv[v] = q < b ? A[i * b + q] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < FT; ++u)
+#pragma unroll
+          for (int v = 0; v < FT; ++v) acc[u][v] = fmaf(fv[u], pv[v], acc[u][v]);
+      }
+#pragma unroll
+      for (int u = 0; u < FT; ++u)
+#pragma unroll
+        for (int v = 0; v < FT; ++v) {
+          const int m = tm * FT + u, q = tq * FT + v;
+          if (m < b && q < b) fpp[m * b + q] = acc[u][v];
+        }
+    }
   }
   cluster.sync();
   if (rank == 0) {
