@@ -97,6 +97,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
   const uint32_t tmem = ctl->tmem;
   volatile int *abort = &ctl->abort;
   const TileRange tr = my_tiles(p.count, p.tiles_per_job);
+  // Per-thread cache of the current history's scalars: every role tests every tile, and the
+  // scalars change only with the history, so they are read from global memory once per history.
+  int cache_j = -1, cache_n = 0;
+  auto rows_of = [&](int j) -> int {
+    if (j != cache_j) {
+      const int32_t *sc = jobs[j].sc;
+      cache_j = j;
+      cache_n = (sc[FS_SKIP] || sc[FS_K_OLD] == 0) ? 0 : sc[FS_N_OLD];
+    }
+    return cache_n;
+  };
 
   if (warp == 0 && lane == 0) {
     // ---------------- producer
@@ -104,7 +115,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
     for (int t = tr.begin; t < tr.end && !*abort; ++t) {
       const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
       const TcJob &jb = jobs[j];
-      if (jb.sc[FS_SKIP] || row0 >= jb.sc[FS_N_OLD] || jb.sc[FS_K_OLD] == 0) continue;
+      if (row0 >= rows_of(j)) continue;
       if (j != cur) {
         if (nb > 0 && !mbar_wait(&ctl->b_empty[0], (nb - 1) & 1, abort, WAIT_NS)) {
           fail_timeout(ctl, jb.meta);
@@ -137,7 +148,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
     for (int t = tr.begin; t < tr.end && !*abort; ++t) {
       const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
       const TcJob &jb = jobs[j];
-      if (jb.sc[FS_SKIP] || row0 >= jb.sc[FS_N_OLD] || jb.sc[FS_K_OLD] == 0) continue;
+      if (row0 >= rows_of(j)) continue;
       if (j != cur) {
         if (cur >= 0) mma_commit(&ctl->b_empty[0]);
         if (!mbar_wait(&ctl->b_full[0], nb & 1, abort, WAIT_NS)) { fail_timeout(ctl, jb.meta); break; }
@@ -176,8 +187,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
     for (int t = tr.begin; t < tr.end && !__any_sync(~0u, *abort != 0); ++t) {
       const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
       const TcJob &jb = jobs[j];
-      const int n = jb.sc[FS_N_OLD];
-      if (jb.sc[FS_SKIP] || row0 >= n || jb.sc[FS_K_OLD] == 0) continue;
+      const int n = rows_of(j);
+      if (row0 >= n) continue;
       const int buf = na & 1, use = na >> 1;
       if (!__all_sync(~0u, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
         fail_timeout(ctl, jb.meta);
@@ -318,11 +329,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
   fence_after_sync();
   const uint32_t tmem = ctl->tmem;
   volatile int *abort = &ctl->abort;
+  // Per-thread cache of the current history's row count: every role tests every tile, and the
+  // count changes only with the history, so it is read from global memory once per history.
+  int cache_j = -1;
+  int64_t cache_n = 0;
+  auto rows_of = [&](int j) -> int64_t {
+    if (j != cache_j) {
+      cache_j = j;
+      cache_n = jobs[j].meta[ISKV_META_N];
+    }
+    return cache_n;
+  };
   // First valid tile at or after t (rows below the history's current length), or -1. Every role
   // walks the same sequence.
   auto next_valid = [&](int t) {
     for (; t < t_end; ++t)
-      if ((t % tpj) * TC_M < jobs[t / tpj].meta[ISKV_META_N]) return t;
+      if ((t % tpj) * TC_M < rows_of(t / tpj)) return t;
     return -1;
   };
 
@@ -413,9 +435,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     // Position of this thread's row in the next unit, loaded one unit ahead.
     auto row_pos = [&](int t) -> int64_t {
       if (t < 0) return 0;
-      const TcJob &jb = jobs[t / tpj];
       const int64_t row = (t % tpj) * TC_M + srow;
-      return row < jb.meta[ISKV_META_N] ? (int64_t)jb.pos[row] : 0;
+      return row < rows_of(t / tpj) ? (int64_t)jobs[t / tpj].pos[row] : 0;
     };
     int t = next_valid(t_begin);
     int64_t ps_next = row_pos(t);
@@ -426,7 +447,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       ps_next = row_pos(tn);  // consumed by the next unit: its latency hides behind this one
       const int jj = t / tpj;
       const TcJob &jb = jobs[jj];
-      bool valid = (t % tpj) * TC_M + srow < jb.meta[ISKV_META_N];
+      bool valid = (t % tpj) * TC_M + srow < rows_of(jj);
       const int64_t ps = valid ? ps_raw : 0;
       if (valid && (ps < 0 || ps >= jb.n_total)) {
         record_status(jb.meta, ISKV_ERR_SHAPE);
