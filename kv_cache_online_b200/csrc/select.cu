@@ -79,6 +79,85 @@ __global__ void k_block_scores(const TK *keys, int64_t n_cand, int H, int hd, in
   if (lane == 0) scores[(size_t)h * n_cand + j] = best;
 }
 
+// Fast path for 8-token blocks of 128-dimensional heads: one warp per (head, block), lane l holds
+// dimensions 4l .. 4l+3 of all 8 tokens (one 8- or 16-byte load per token). The 16 per-token
+// sums (dot with the mean, squared norm) are reduced together by a transposed butterfly: at each
+// of 4 levels a lane keeps half of its values and adds the partner's other half, so after 4 + 1
+// shuffle levels lanes 4t, 4t+1 hold token t's dot and lanes 4t+2, 4t+3 its squared norm.
+ISKV_DEV void load4(const __nv_bfloat16 *p, double (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+ISKV_DEV void load4(const float *p, double (&v)[4]) {
+  const float4 f = *reinterpret_cast<const float4 *>(p);
+  v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
+
+template <typename TK>
+__global__ void __launch_bounds__(256) k_block_scores_8x128(const TK *keys, int64_t n_cand, int H,
+                                                            double *scores) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  if (gw >= n_cand * H) return;  // whole warps
+  const int h = (int)(gw % H);
+  const int64_t j = gw / H;
+  double x[8][4];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) load4(keys + ((size_t)(j * 8 + t) * H + h) * 128 + 4 * lane, x[t]);
+  double mean[4], mn2 = 0.0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    double m = 0.0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) m += x[t][u];
+    mean[u] = m / 8.0;
+    mn2 = fma(mean[u], mean[u], mn2);
+  }
+  const double mn = sqrt(warp_sum(mn2));
+  // v[2t] = partial dot of token t with the mean, v[2t+1] = partial squared norm of token t.
+  double v[16];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    double dt = 0.0, k2 = 0.0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      dt = fma(x[t][u], mean[u], dt);
+      k2 = fma(x[t][u], x[t][u], k2);
+    }
+    v[2 * t] = dt;
+    v[2 * t + 1] = k2;
+  }
+  // Transposed butterfly over lane bits 4, 3, 2, 1: value index bits 3, 2, 1, 0.
+#pragma unroll
+  for (int lev = 0; lev < 4; ++lev) {
+    const int half = 8 >> lev;                // values kept after this level
+    const int bit = 16 >> lev;                // lane bit deciding which half is kept
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i < half) {
+        const double send = upper ? v[i] : v[i + half];
+        const double keep = upper ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+      }
+    }
+  }
+  const double tot = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);  // lanes 2i, 2i+1: value i
+  // Lane 4t: dot of token t; lane 4t + 2: its squared norm.
+  const double k2t = __shfl_down_sync(0xffffffffu, tot, 2);
+  double cs = 0.0;
+  if ((lane & 3) == 0) cs = tot / fmax(sqrt(k2t) * mn, 1e-30);
+  // Minimum over the 8 tokens (lanes 0, 4, ..., 28).
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    const double other = __shfl_xor_sync(0xffffffffu, cs, o);
+    cs = fmin(cs, other);
+  }
+  if (lane == 0) scores[(size_t)h * n_cand + j] = cs;
+}
+
 // Order-preserving map from a finite double to uint64 (-0 is folded onto +0).
 ISKV_DEV unsigned long long order_key(double v) {
   if (v == 0.0) v = 0.0;
@@ -287,7 +366,15 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int64_t warps = n_cand * a.H;
     const unsigned g = (unsigned)((warps * 32 + 255) / 256);
-    if (a.k_dtype == ISKV_BF16)
+    const bool fast = a.block == 8 && a.hd == 128 &&
+                      reinterpret_cast<uintptr_t>(a.keys) % (a.k_dtype == ISKV_BF16 ? 8 : 16) == 0;
+    if (fast && a.k_dtype == ISKV_BF16)
+      k_block_scores_8x128<<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(a.keys), n_cand,
+                                             a.H, scores);
+    else if (fast)
+      k_block_scores_8x128<<<g, 256, 0, s>>>(static_cast<const float *>(a.keys), n_cand, a.H,
+                                             scores);
+    else if (a.k_dtype == ISKV_BF16)
       k_block_scores<<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(a.keys), n_cand, a.H,
                                        a.hd, a.block, scores);
     else
