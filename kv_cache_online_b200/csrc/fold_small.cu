@@ -139,8 +139,10 @@ cudaError_t launch_fold_project(const FoldJob *jobs, const FoldParams &p, cudaSt
 }
 
 // ------------------------------------------------------------------------------------------------
-// Basis rotation: Bn = [B, P] H  (d x k'), K = k + p. Written to workspace and copied into B
-// afterwards, so that no tile reads basis columns another tile is overwriting.
+// Basis rotation: Bn = [B, P] H  (d x k'), K = k + p, in 64 x 64 tiles (4 x 4 per thread). Written
+// to workspace and copied into B afterwards, so that no tile reads basis columns another tile is
+// overwriting.
+constexpr int RBM = 64, RTM = 4;
 template <typename TS>
 __global__ void __launch_bounds__(256) k_rotate_basis(const char *jobs, RotParams p) {
   const JobHead &jh = job_head(jobs, p.job_stride, blockIdx.z);
@@ -148,13 +150,13 @@ __global__ void __launch_bounds__(256) k_rotate_basis(const char *jobs, RotParam
   if (sc[FS_SKIP]) return;
   const int k = sc[FS_K_OLD], pp = sc[FS_P], kn = sc[FS_K_NEW];
   const int r = p.r, pld = p.pld, hs = p.hs;
-  const int m0 = blockIdx.y * PBM, n0 = blockIdx.x * PBN;
+  const int m0 = blockIdx.y * RBM, n0 = blockIdx.x * PBN;
   if (n0 >= kn) return;
   const TS *B = static_cast<const TS *>(jh.B);
   const float *P = reinterpret_cast<const float *>(jh.ws + p.pmat);
   const float *Ht = reinterpret_cast<const float *>(jh.ws + p.ht);
   float *Bn = reinterpret_cast<float *>(jh.ws + p.bn);
-  tile_gemm<PBM, PBN, PBK, PTM, PTN, true, false>(
+  tile_gemm<RBM, PBN, PBK, RTM, PTN, true, false>(
       m0, n0, p.d, kn, k + pp,
       [&](int m, int l) {
         return l < k ? to_f<TS>(B[(size_t)m * r + l]) : P[(size_t)m * pld + (l - k)];
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(256) k_rotate_basis(const char *jobs, RotParam
 }
 
 cudaError_t launch_rotate_basis(const char *jobs, const RotParams &p, cudaStream_t s) {
-  const dim3 g((p.r + PBN - 1) / PBN, (p.d + PBM - 1) / PBM, p.count);
+  const dim3 g((p.r + PBN - 1) / PBN, (p.d + RBM - 1) / RBM, p.count);
   if (p.storage == ISKV_BF16)
     k_rotate_basis<__nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
   else

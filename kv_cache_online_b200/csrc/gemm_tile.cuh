@@ -32,35 +32,70 @@ ISKV_DEV void tile_gemm(int m0, int n0, int M, int N, int K, const LA &la, const
                         const EP &ep) {
   static_assert(TN % 2 == 0 && (TM == 2 || TM == 4) && (TN == 2 || TN == 4), "thread tile");
   constexpr int TR = BM / TM, TC = BN / TN, NT = TR * TC;
-  __shared__ __align__(16) float As[BK][BM + 4];
-  __shared__ __align__(16) float Bs[BK][BN + 4];
+  constexpr int AE = (BM * BK + NT - 1) / NT, BE = (BK * BN + NT - 1) / NT;  // loads per thread
+  // Two shared buffers: the next K block is fetched into registers while the current one is
+  // multiplied, then stored into the other buffer (one barrier per K block).
+  __shared__ __align__(16) float As[2][BK][BM + 4];
+  __shared__ __align__(16) float Bs[2][BK][BN + 4];
   const int tid = threadIdx.x;
   const int tr = tid / TC, tc = tid % TC;
+  float ra[AE], rb[BE];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < AE; ++u) {
+      const int e = tid + u * NT;
+      int mm, kk;
+      if (A_KFAST) { mm = e / BK; kk = e % BK; } else { kk = e / BM; mm = e % BM; }
+      const int gm = m0 + mm, gk = k0 + kk;
+      ra[u] = (e < BM * BK && gm < M && gk < K) ? la(gm, gk) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < BE; ++u) {
+      const int e = tid + u * NT;
+      int kk, nn;
+      if (B_NFAST) { kk = e / BN; nn = e % BN; } else { nn = e / BK; kk = e % BK; }
+      const int gk = k0 + kk, gn = n0 + nn;
+      rb[u] = (e < BK * BN && gk < K && gn < N) ? lb(gk, gn) : 0.f;
+    }
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int u = 0; u < AE; ++u) {
+      const int e = tid + u * NT;
+      if (e >= BM * BK) continue;
+      int mm, kk;
+      if (A_KFAST) { mm = e / BK; kk = e % BK; } else { kk = e / BM; mm = e % BM; }
+      As[buf][kk][mm] = ra[u];
+    }
+#pragma unroll
+    for (int u = 0; u < BE; ++u) {
+      const int e = tid + u * NT;
+      if (e >= BK * BN) continue;
+      int kk, nn;
+      if (B_NFAST) { kk = e / BN; nn = e % BN; } else { nn = e / BK; kk = e % BK; }
+      Bs[buf][kk][nn] = rb[u];
+    }
+  };
   float2 acc[TM][TN / 2];
 #pragma unroll
   for (int i = 0; i < TM; ++i)
 #pragma unroll
     for (int j = 0; j < TN / 2; ++j) acc[i][j] = make_float2(0.f, 0.f);
 
-  for (int k0 = 0; k0 < K; k0 += BK) {
-    for (int e = tid; e < BM * BK; e += NT) {
-      int mm, kk;
-      if (A_KFAST) { mm = e / BK; kk = e % BK; } else { kk = e / BM; mm = e % BM; }
-      const int gm = m0 + mm, gk = k0 + kk;
-      As[kk][mm] = (gm < M && gk < K) ? la(gm, gk) : 0.f;
-    }
-    for (int e = tid; e < BK * BN; e += NT) {
-      int kk, nn;
-      if (B_NFAST) { kk = e / BN; nn = e % BN; } else { nn = e / BK; kk = e % BK; }
-      const int gk = k0 + kk, gn = n0 + nn;
-      Bs[kk][nn] = (gk < K && gn < N) ? lb(gk, gn) : 0.f;
-    }
-    __syncthreads();
+  const int nk = (K + BK - 1) / BK;
+  if (nk > 0) {
+    fetch(0);
+    stash(0);
+  }
+  __syncthreads();
+  for (int kb = 0; kb < nk; ++kb) {
+    const int cur = kb & 1;
+    if (kb + 1 < nk) fetch((kb + 1) * BK);  // in flight during the multiply below
 #pragma unroll 4
     for (int kk = 0; kk < BK; ++kk) {
       float a[TM], bb[TN];
-      lds_vec<TM>(a, &As[kk][tr * TM]);
-      lds_vec<TN>(bb, &Bs[kk][tc * TN]);
+      lds_vec<TM>(a, &As[cur][kk][tr * TM]);
+      lds_vec<TN>(bb, &Bs[cur][kk][tc * TN]);
 #pragma unroll
       for (int i = 0; i < TM; ++i) {
         const float2 ai = make_float2(a[i], a[i]);
@@ -69,6 +104,7 @@ ISKV_DEV void tile_gemm(int m0, int n0, int M, int N, int K, const LA &la, const
           acc[i][j] = __ffma2_rn(ai, make_float2(bb[2 * j], bb[2 * j + 1]), acc[i][j]);
       }
     }
+    if (kb + 1 < nk) stash(cur ^ 1);
     __syncthreads();
   }
 #pragma unroll
