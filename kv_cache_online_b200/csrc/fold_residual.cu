@@ -102,14 +102,20 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
   const bool active = my_g < G;
 
   for (int j = 0; j < b; ++j) {
-    // Partial dots of column j with every column over my rows with global index >= j.
+    // Partial dots of column j with every column over my rows with global index >= j: four
+    // independent float32 accumulators (short dependency chains), combined in float64.
     if (active) {
-      double acc = 0.0;
-      for (int i = my_g; i < rpc; i += G) {
-        if (row0 + i < j) continue;
-        acc = fma((double)A[i * b + j], (double)A[i * b + my_c], acc);
+      int i = my_g;
+      if (row0 + i < j) i += ((j - row0 - i) + G - 1) / G * G;  // first of my rows at or past j
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      for (; i + 3 * G < rpc; i += 4 * G) {
+        a0 = fmaf(A[i * b + j], A[i * b + my_c], a0);
+        a1 = fmaf(A[(i + G) * b + j], A[(i + G) * b + my_c], a1);
+        a2 = fmaf(A[(i + 2 * G) * b + j], A[(i + 2 * G) * b + my_c], a2);
+        a3 = fmaf(A[(i + 3 * G) * b + j], A[(i + 3 * G) * b + my_c], a3);
       }
-      part[my_g * b + my_c] = acc;
+      for (; i < rpc; i += G) a0 = fmaf(A[i * b + j], A[i * b + my_c], a0);
+      part[my_g * b + my_c] = ((double)a0 + (double)a1) + ((double)a2 + (double)a3);
     }
     __syncthreads();
     float *slot = pay + (j & 1) * 2 * b;
@@ -159,12 +165,14 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
     if (active && my_c > j && tau != 0.0) {
       const double wc = (double)tot[my_c] - alpha * tot[b + my_c];
       const float tw = (float)(tau * wc);
-      for (int i = my_g; i < rpc; i += G) {
-        const int gi = row0 + i;
-        if (gi < j) continue;
-        const float vi = gi == j ? (float)vj : A[i * b + j];
-        A[i * b + my_c] -= tw * vi;
+      int i = my_g;
+      if (row0 + i < j) i += ((j - row0 - i) + G - 1) / G * G;  // first of my rows at or past j
+      if (i < rpc && row0 + i == j) {  // the reflector's leading entry is vj, not A[j][j]
+        A[i * b + my_c] -= tw * (float)vj;
+        i += G;
       }
+#pragma unroll 4
+      for (; i < rpc; i += G) A[i * b + my_c] = fmaf(-tw, A[i * b + j], A[i * b + my_c]);
     }
     __syncthreads();
   }
