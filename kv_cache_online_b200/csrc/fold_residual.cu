@@ -189,7 +189,10 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
     // Float32 inner products carry relative error ~ sqrt(b) 2^-24; the tolerance sits a few units
     // above it (a residual cosine of that size moves the rho only at second order).
     const float tol = 4.f * sqrtf((float)b) * 5.9604645e-08f;
-    const int sw = cta_jacobi_columns(Rm, b, b, b, tol, 60);
+    const int sw = b <= 16   ? cta_jacobi_columns<1>(Rm, b, b, b, tol, 60)
+                   : b <= 32 ? cta_jacobi_columns<2>(Rm, b, b, b, tol, 60)
+                   : b <= 64 ? cta_jacobi_columns<4>(Rm, b, b, b, tol, 60)
+                             : cta_jacobi_columns<8>(Rm, b, b, b, tol, 60);
     __shared__ float nrm[128];
     __shared__ int order[128];
     if (tid < b) {
