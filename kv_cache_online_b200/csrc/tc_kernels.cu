@@ -432,28 +432,52 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     // AND-reducing named barrier: they meet at named barriers below, and tcgen05.ld is warp-wide.
     const int pair_bar = 1 + q;
     float cs[32], sn[32];
-    // Position of this thread's row in the next unit, loaded one unit ahead.
-    auto row_pos = [&](int t) -> int64_t {
+    // Fields of the history being written, read from global memory once per history rather than
+    // once per unit (each read is a dependent global load on the unit's critical path).
+    int hj = -1;
+    const int32_t *h_pos = nullptr;
+    __nv_bfloat16 *h_out = nullptr;
+    int64_t h_rows = 0, h_total = 0;
+    bool h_rope = false, h_tiles = false;
+    auto hist = [&](int j) {
+      if (j != hj) {
+        hj = j;
+        const TcJob &jb = jobs[j];
+        h_pos = jb.pos;
+        h_out = static_cast<__nv_bfloat16 *>(jb.out);
+        h_rows = rows_of(j);
+        h_total = jb.n_total;
+        h_rope = jb.rope != 0;
+        h_tiles = jb.tiles_ok != 0;
+      }
+    };
+    // Position of this thread's row in a unit, loaded one unit ahead. The raw 32-bit value is
+    // carried to the next unit unconverted, so nothing waits on the load until then.
+    auto row_pos = [&](int t) -> int32_t {
       if (t < 0) return 0;
+      hist(t / tpj);
       const int64_t row = (t % tpj) * TC_M + srow;
-      return row < rows_of(t / tpj) ? (int64_t)jobs[t / tpj].pos[row] : 0;
+      return row < h_rows ? __ldg(h_pos + row) : 0;
     };
     int t = next_valid(t_begin);
-    int64_t ps_next = row_pos(t);
+    int32_t ps_next = row_pos(t);
     for (;;) {
       if (!named_and(pair_bar, 64, t >= 0 && !*abort)) break;
-      const int tn = next_valid(t + 1);
-      const int64_t ps_raw = ps_next;
-      ps_next = row_pos(tn);  // consumed by the next unit: its latency hides behind this one
       const int jj = t / tpj;
-      const TcJob &jb = jobs[jj];
-      bool valid = (t % tpj) * TC_M + srow < rows_of(jj);
-      const int64_t ps = valid ? ps_raw : 0;
-      if (valid && (ps < 0 || ps >= jb.n_total)) {
-        record_status(jb.meta, ISKV_ERR_SHAPE);
+      const int32_t ps_raw = ps_next;
+      hist(jj);
+      bool valid = (t % tpj) * TC_M + srow < h_rows;
+      const bool rope = h_rope, tiles_ok = h_tiles;
+      __nv_bfloat16 *const out = h_out;
+      const int64_t n_total = h_total;
+      const int tn = next_valid(t + 1);
+      ps_next = row_pos(tn);  // consumed by the next unit: its latency hides behind this one
+      const int64_t ps = valid ? (int64_t)ps_raw : 0;
+      if (valid && (ps < 0 || ps >= n_total)) {
+        record_status(jobs[jj].meta, ISKV_ERR_SHAPE);
         valid = false;
       }
-      if (jb.rope != 0 && valid) {
+      if (rope && valid) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) rope_angle(rope_tab, j0 + i, (uint32_t)ps, cs[i], sn[i]);
       } else {
@@ -463,12 +487,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
           sn[i] = 0.f;
         }
       }
-      __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(jb.out) + (size_t)(valid ? ps : 0) * D +
-                            (size_t)member * HP * HN;
+      __nv_bfloat16 *orow = out + (size_t)(valid ? ps : 0) * D + (size_t)member * HP * HN;
       // This lane quarter's 32 rows go out as tiles when their positions are consecutive (the
       // same answer in both warps of the pair: they hold the same rows).
       const int64_t first = __shfl_sync(~0u, ps, 0);
-      const bool tiles = jb.tiles_ok && __all_sync(~0u, valid && ps == first + lane);
+      const bool tiles = tiles_ok && __all_sync(~0u, valid && ps == first + lane);
+      const TcJob &jb = jobs[jj];
       if (tiles && issuer) tensormap_acquire(&jb.mapO);
       const int buf = nc & 1, use = nc >> 1;
       if (!named_and(pair_bar, 64, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
