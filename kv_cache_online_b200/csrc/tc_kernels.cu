@@ -340,21 +340,43 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     }
     return cache_n;
   };
-  // First valid tile at or after t (rows below the history's current length), or -1. Every role
-  // walks the same sequence.
-  auto next_valid = [&](int t) {
-    for (; t < t_end; ++t)
-      if ((t % tpj) * TC_M < rows_of(t / tpj)) return t;
-    return -1;
+  // Tile cursor: linear tile t = j * tpj + k (history j, row tile k). Every role walks the same
+  // sequence of valid tiles (rows below the history's current length, a prefix of its tiles),
+  // advancing incrementally so that no division sits on a unit's critical path.
+  struct Cur {
+    int t, j, k;
   };
+  auto seek = [&](Cur c) -> Cur {  // first valid tile at or after c; t = -1 when none is left
+    while (c.t < t_end) {
+      if (c.k * TC_M < rows_of(c.j)) return c;
+      c.t += tpj - c.k;  // the rest of this history is past its length
+      ++c.j;
+      c.k = 0;
+    }
+    c.t = -1;
+    return c;
+  };
+  auto advance = [&](Cur c) -> Cur {
+    ++c.t;
+    if (++c.k == tpj) {
+      c.k = 0;
+      ++c.j;
+    }
+    return seek(c);
+  };
+  Cur c_first;
+  c_first.t = t_begin;
+  c_first.j = t_begin / tpj;
+  c_first.k = t_begin - c_first.j * tpj;
+  c_first = seek(c_first);
 
   if (warp == 0 && lane == 0) {
     // ---------------- producer: basis rows of this CTA's heads once per history, U slabs per tile
     int na = 0, nb = 0, cur = -1;
     int64_t *fm = nullptr;  // meta of the history being loaded: where a timeout is recorded
     bool ok = true;
-    for (int t = next_valid(t_begin); t >= 0 && ok && !*abort; t = next_valid(t + 1)) {
-      const int j = t / tpj, row0 = (t % tpj) * TC_M;
+    for (Cur c = c_first; c.t >= 0 && ok && !*abort; c = advance(c)) {
+      const int j = c.j, row0 = c.k * TC_M;
       const TcJob &jb = jobs[j];
       fm = jb.meta;
       if (j != cur) {
@@ -387,8 +409,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     int na = 0, nb = 0, nc = 0, cur = -1;
     int64_t *fm = nullptr;
     bool ok = true;
-    for (int t = next_valid(t_begin); t >= 0 && ok && !*abort; t = next_valid(t + 1)) {
-      const int j = t / tpj;
+    for (Cur c = c_first; c.t >= 0 && ok && !*abort; c = advance(c)) {
+      const int j = c.j;
       fm = jobs[j].meta;
       if (j != cur) {
         // The resident basis may be replaced once every MMA reading it has completed.
@@ -453,25 +475,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     };
     // Position of this thread's row in a unit, loaded one unit ahead. The raw 32-bit value is
     // carried to the next unit unconverted, so nothing waits on the load until then.
-    auto row_pos = [&](int t) -> int32_t {
-      if (t < 0) return 0;
-      hist(t / tpj);
-      const int64_t row = (t % tpj) * TC_M + srow;
+    auto row_pos = [&](const Cur &c) -> int32_t {
+      if (c.t < 0) return 0;
+      hist(c.j);
+      const int64_t row = (int64_t)c.k * TC_M + srow;
       return row < h_rows ? __ldg(h_pos + row) : 0;
     };
-    int t = next_valid(t_begin);
-    int32_t ps_next = row_pos(t);
+    int acq_j = -1;  // history whose output tensor map this thread last acquired
+    Cur c = c_first;
+    int32_t ps_next = row_pos(c);
     for (;;) {
-      if (!named_and(pair_bar, 64, t >= 0 && !*abort)) break;
-      const int jj = t / tpj;
+      if (!named_and(pair_bar, 64, c.t >= 0 && !*abort)) break;
+      const int jj = c.j;
       const int32_t ps_raw = ps_next;
       hist(jj);
-      bool valid = (t % tpj) * TC_M + srow < h_rows;
+      bool valid = c.k * TC_M + srow < h_rows;
       const bool rope = h_rope, tiles_ok = h_tiles;
       __nv_bfloat16 *const out = h_out;
       const int64_t n_total = h_total;
-      const int tn = next_valid(t + 1);
-      ps_next = row_pos(tn);  // consumed by the next unit: its latency hides behind this one
+      const Cur cn = advance(c);
+      ps_next = row_pos(cn);  // consumed by the next unit: its latency hides behind this one
       const int64_t ps = valid ? (int64_t)ps_raw : 0;
       if (valid && (ps < 0 || ps >= n_total)) {
         record_status(jobs[jj].meta, ISKV_ERR_SHAPE);
@@ -493,7 +516,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       const int64_t first = __shfl_sync(~0u, ps, 0);
       const bool tiles = tiles_ok && __all_sync(~0u, valid && ps == first + lane);
       const TcJob &jb = jobs[jj];
-      if (tiles && issuer) tensormap_acquire(&jb.mapO);
+      if (tiles && issuer && acq_j != jj) {
+        tensormap_acquire(&jb.mapO);
+        acq_j = jj;
+      }
       const int buf = nc & 1, use = nc >> 1;
       if (!named_and(pair_bar, 64, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
         fail_timeout(ctl, jb.meta);
@@ -502,53 +528,59 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       fence_after_sync();
       const uint32_t base = tmem + buf * NN + ((uint32_t)(q * 32) << 16);
       for (int h = 0; h < HP; ++h) {
-        // The staged rows are free once the previous tile stores out of them have been read.
-        if (issuer) bulk_wait_read0();
-        named_sync(pair_bar, 64);
+        // The head's 32 RoPE pairs go to packed registers first, so the TMEM loads and the math
+        // overlap the previous tile stores still reading the staged rows.
+        uint32_t wl[16], wh[16];
 #pragma unroll
         for (int jb16 = 0; jb16 < 32; jb16 += 16) {
           float lo[16], hi[16];
           tmem_ld16(base + h * HN + j0 + jb16, lo);
           tmem_ld16(base + h * HN + 64 + j0 + jb16, hi);
           tmem_ld_wait();
-          uint32_t wl[8], wh[8];
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
             const float c0 = cs[jb16 + i], s0 = sn[jb16 + i];
             const float c1 = cs[jb16 + i + 1], s1 = sn[jb16 + i + 1];
-            wl[i / 2] = pack_bf16(lo[i] * c0 - hi[i] * s0, lo[i + 1] * c1 - hi[i + 1] * s1);
-            wh[i / 2] = pack_bf16(hi[i] * c0 + lo[i] * s0, hi[i + 1] * c1 + lo[i + 1] * s1);
-          }
-          if (tiles) {
-            // 16-byte chunk c of a 128-byte staged row sits at chunk c ^ (row & 7).
-            const int ck = (j0 + jb16) / 8, sw = srow & 7;
-            *reinterpret_cast<uint4 *>(stg_lo + 16 * (ck ^ sw)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-            *reinterpret_cast<uint4 *>(stg_lo + 16 * ((ck + 1) ^ sw)) = make_uint4(wl[4], wl[5], wl[6], wl[7]);
-            *reinterpret_cast<uint4 *>(stg_hi + 16 * (ck ^ sw)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-            *reinterpret_cast<uint4 *>(stg_hi + 16 * ((ck + 1) ^ sw)) = make_uint4(wh[4], wh[5], wh[6], wh[7]);
-          } else if (valid) {
-            uint4 *dl = reinterpret_cast<uint4 *>(orow + h * HN + j0 + jb16);
-            uint4 *dh = reinterpret_cast<uint4 *>(orow + h * HN + 64 + j0 + jb16);
-            dl[0] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-            dl[1] = make_uint4(wl[4], wl[5], wl[6], wl[7]);
-            dh[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-            dh[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+            wl[(jb16 + i) / 2] = pack_bf16(lo[i] * c0 - hi[i] * s0, lo[i + 1] * c1 - hi[i + 1] * s1);
+            wh[(jb16 + i) / 2] = pack_bf16(hi[i] * c0 + lo[i] * s0, hi[i + 1] * c1 + lo[i + 1] * s1);
           }
         }
-        fence_proxy_async_smem();
-        named_sync(pair_bar, 64);
-        if (tiles && issuer) {
-          const int x = (member * HP + h) * HN;
-          tma_store_2d(&jb.mapO, x, (int)first, sStg + q * 32 * 128);
-          tma_store_2d(&jb.mapO, x + 64, (int)first, sStg + TC_M * 128 + q * 32 * 128);
-          bulk_commit();
+        if (tiles) {
+          // The staged rows are free once the previous tile stores out of them have been read.
+          if (issuer) bulk_wait_read0();
+          named_sync(pair_bar, 64);
+          // 16-byte chunk c of a 128-byte staged row sits at chunk c ^ (row & 7).
+          const int ck = j0 / 8, sw = srow & 7;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            *reinterpret_cast<uint4 *>(stg_lo + 16 * ((ck + u) ^ sw)) =
+                make_uint4(wl[4 * u], wl[4 * u + 1], wl[4 * u + 2], wl[4 * u + 3]);
+            *reinterpret_cast<uint4 *>(stg_hi + 16 * ((ck + u) ^ sw)) =
+                make_uint4(wh[4 * u], wh[4 * u + 1], wh[4 * u + 2], wh[4 * u + 3]);
+          }
+          fence_proxy_async_smem();
+          named_sync(pair_bar, 64);
+          if (issuer) {
+            const int x = (member * HP + h) * HN;
+            tma_store_2d(&jb.mapO, x, (int)first, sStg + q * 32 * 128);
+            tma_store_2d(&jb.mapO, x + 64, (int)first, sStg + TC_M * 128 + q * 32 * 128);
+            bulk_commit();
+          }
+        } else if (valid) {
+          uint4 *dl = reinterpret_cast<uint4 *>(orow + h * HN + j0);
+          uint4 *dh = reinterpret_cast<uint4 *>(orow + h * HN + 64 + j0);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            dl[u] = make_uint4(wl[4 * u], wl[4 * u + 1], wl[4 * u + 2], wl[4 * u + 3]);
+            dh[u] = make_uint4(wh[4 * u], wh[4 * u + 1], wh[4 * u + 2], wh[4 * u + 3]);
+          }
         }
       }
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
       ++nc;
-      t = tn;
+      c = cn;
     }
     if (issuer) bulk_wait0();
   }
