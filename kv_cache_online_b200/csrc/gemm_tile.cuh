@@ -7,11 +7,16 @@
 
 namespace iskv {
 
-// Vector load of N consecutive floats from shared memory (N = 2 or 4, 8- or 16-byte aligned).
+// Vector load of N consecutive floats from shared memory (N = 2, 4 or 8; 8- or 16-byte aligned).
 template <int N>
 ISKV_DEV void lds_vec(float (&v)[N], const float *p) {
-  static_assert(N == 2 || N == 4, "vector width");
-  if constexpr (N == 4) {
+  static_assert(N == 2 || N == 4 || N == 8, "vector width");
+  if constexpr (N == 8) {
+    const float4 t = *reinterpret_cast<const float4 *>(p);
+    const float4 u = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    v[4] = u.x; v[5] = u.y; v[6] = u.z; v[7] = u.w;
+  } else if constexpr (N == 4) {
     const float4 t = *reinterpret_cast<const float4 *>(p);
     v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
   } else {
@@ -30,7 +35,8 @@ template <int BM, int BN, int BK, int TM, int TN, bool A_KFAST, bool B_NFAST, cl
           class EP>
 ISKV_DEV void tile_gemm(int m0, int n0, int M, int N, int K, const LA &la, const LB &lb,
                         const EP &ep) {
-  static_assert(TN % 2 == 0 && (TM == 2 || TM == 4) && (TN == 2 || TN == 4), "thread tile");
+  static_assert(TN % 2 == 0 && (TM == 2 || TM == 4 || TM == 8) && (TN == 2 || TN == 4 || TN == 8),
+                "thread tile");
   constexpr int TR = BM / TM, TC = BN / TN, NT = TR * TC;
   constexpr int AE = (BM * BK + NT - 1) / NT, BE = (BK * BN + NT - 1) / NT;  // loads per thread
   // Two shared buffers: the next K block is fetched into registers while the current one is

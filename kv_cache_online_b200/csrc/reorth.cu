@@ -33,6 +33,15 @@ ISKV_DEV bool ns_converged(const int32_t *sc, int it, int which) {
   return it > 0 && __int_as_float(sc[RS_DEV + 2 * (it - 1) + which]) <= NS_STOP_SQ;
 }
 
+// Iterations actually computed for factor `which` (a skipped iteration leaves Y, Z where they
+// are). Iteration it reads the first buffer of its pair when it is even and writes the second, so
+// the result sits in the first buffer after an even count and in the second after an odd count.
+ISKV_DEV bool ns_result_in_second(const int32_t *sc, int which) {
+  int done = 0;
+  while (done < NS_ITERS && !ns_converged(sc, done, which)) ++done;
+  return done & 1;
+}
+
 ReorthWsLayout reorth_ws_layout(int d, int r, int64_t n_cap) {
   ReorthWsLayout L;
   size_t o = 0;
@@ -80,7 +89,9 @@ __global__ void k_reorth_prepare(const ReorthJob *jobs, ReorthParams p) {
   for (int i = 0; i < 2 * NS_ITERS; ++i) sc[RS_DEV + i] = 0;  // float 0
 }
 
-constexpr int GBM = 64, GBN = 64, GBK = 16, GTM = 4, GTN = 4;
+// Register tiles of the r x r products: 128 x 64 blocks, 8 x 4 outputs per thread (each k step
+// reads 12 floats from shared memory per 32 FMAs), two blocks resident per SM.
+constexpr int GBM = 128, GBN = 64, GBK = 16, GTM = 8, GTN = 4;
 
 // Gram partial: Gpart[s] = X[rows of split s]^T X[rows of split s] (k x k), X = U (n rows) or B.
 template <typename TS>
@@ -157,9 +168,10 @@ __global__ void __launch_bounds__(256) k_ns_init(const ReorthJob *jobs, ReorthPa
 
 // Newton-Schulz stages of iteration `it`. STAGE 0: T = 1.5 I - 0.5 Z Y, and ||T - I||_F^2 summed
 // into the iteration's slot. STAGE 1: Y2 = Y T (g = 0), Z2 = T Z (g = 1). Once an earlier
-// iteration's T met the stopping threshold, stage 0 does nothing and stage 1 copies Y, Z forward.
+// iteration's T met the stopping threshold, both stages do nothing: Y, Z stay in the buffers the
+// last computed iteration wrote, which the consumers locate with ns_result_in_second.
 template <int STAGE>
-__global__ void __launch_bounds__(256) k_ns_step(const ReorthJob *jobs, ReorthParams p, int it,
+__global__ void __launch_bounds__(256, 2) k_ns_step(const ReorthJob *jobs, ReorthParams p, int it,
                                                  size_t y0, size_t z0, size_t y1, size_t z1,
                                                  size_t yb0, size_t zb0, size_t yb1, size_t zb1) {
   const int per = STAGE == 0 ? 2 : 4;
@@ -198,24 +210,14 @@ __global__ void __launch_bounds__(256) k_ns_step(const ReorthJob *jobs, ReorthPa
     }
     return;
   }
-  const float *X = g == 0 ? Y : Z;
   float *Xo = reinterpret_cast<float *>(ws + (g == 0 ? (which == 0 ? y1 : yb1) : (which == 0 ? z1 : zb1)));
-  if (done) {
-    for (int e = threadIdx.x; e < GBM * GBN; e += blockDim.x) {
-      const int m = m0 + e / GBN, n = n0 + e % GBN;
-      if (m < k && n < k) Xo[(size_t)m * r + n] = X[(size_t)m * r + n];
-    }
-  } else if (g == 0) {
-    tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
-        m0, n0, k, k, k, [&](int m, int kk) { return Y[(size_t)m * r + kk]; },
-        [&](int kk, int n) { return T[(size_t)kk * r + n]; },
-        [&](int m, int n, float acc) { Xo[(size_t)m * r + n] = acc; });
-  } else {
-    tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
-        m0, n0, k, k, k, [&](int m, int kk) { return T[(size_t)m * r + kk]; },
-        [&](int kk, int n) { return Z[(size_t)kk * r + n]; },
-        [&](int m, int n, float acc) { Xo[(size_t)m * r + n] = acc; });
-  }
+  if (done) return;
+  // Y2 = Y T (g = 0) or Z2 = T Z (g = 1): one tile routine with the operands chosen per block.
+  const float *A = g == 0 ? Y : T, *Bm = g == 0 ? T : Z;
+  tile_gemm<GBM, GBN, GBK, GTM, GTN, true, true>(
+      m0, n0, k, k, k, [&](int m, int kk) { return A[(size_t)m * r + kk]; },
+      [&](int kk, int n) { return Bm[(size_t)kk * r + n]; },
+      [&](int m, int n, float acc) { Xo[(size_t)m * r + n] = acc; });
 }
 
 // Convergence check of the iteration: the last computed T = 1.5 I - 0.5 Z Y must be I to working
@@ -234,12 +236,13 @@ __global__ void k_ns_check(const ReorthJob *jobs, ReorthParams p) {
 }
 
 // M = sqrt(c_u c_b) Y_u diag(sigma) Y_b  (= R_U diag(sigma) R_B^T with symmetric R_B).
-__global__ void __launch_bounds__(256) k_reorth_M(const ReorthJob *jobs, ReorthParams p,
-                                                  size_t yu, size_t yb) {
+__global__ void __launch_bounds__(256, 2) k_reorth_M(const ReorthJob *jobs, ReorthParams p) {
   const ReorthJob &jb = jobs[blockIdx.z];
   const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
   if (sc[FS_SKIP]) return;
   const int k = sc[FS_K_OLD], r = p.r;
+  const size_t yu = ns_result_in_second(sc, 0) ? p.ws.Y2[0] : p.ws.Y[0];
+  const size_t yb = ns_result_in_second(sc, 1) ? p.ws.Y2[1] : p.ws.Y[1];
   const float scale = sqrtf(__int_as_float(sc[RS_CU]) * __int_as_float(sc[RS_CB]));
   const float *Yu = reinterpret_cast<const float *>(jb.h.ws + yu);
   const float *Yb = reinterpret_cast<const float *>(jb.h.ws + yb);
@@ -255,15 +258,15 @@ __global__ void __launch_bounds__(256) k_reorth_M(const ReorthJob *jobs, ReorthP
 
 // Rotations: TUt[q][l] = (Z_u X)[l][q] / sqrt(c_u) with X[j][q] = Gt[q][j];
 //            TBt[q][l] = (Z_b Y)[l][q] / sqrt(c_b) with Y[j][q] = Ht[q][j].
-__global__ void __launch_bounds__(256) k_reorth_T(const ReorthJob *jobs, ReorthParams p, size_t zu,
-                                                  size_t zb) {
+__global__ void __launch_bounds__(256, 2) k_reorth_T(const ReorthJob *jobs, ReorthParams p) {
   const int job = blockIdx.z >> 1, which = blockIdx.z & 1;
   const ReorthJob &jb = jobs[job];
   const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
   if (sc[FS_SKIP]) return;
   const int k = sc[FS_K_OLD], r = p.r;
   const float inv = rsqrtf(__int_as_float(sc[which == 0 ? RS_CU : RS_CB]));
-  const float *Z = reinterpret_cast<const float *>(jb.h.ws + (which == 0 ? zu : zb));
+  const size_t zo = ns_result_in_second(sc, which) ? p.ws.Z2[which] : p.ws.Z[which];
+  const float *Z = reinterpret_cast<const float *>(jb.h.ws + zo);
   const float *V = reinterpret_cast<const float *>(jb.h.ws + (which == 0 ? p.ws.Gt : p.ws.Ht));
   float *out = reinterpret_cast<float *>(jb.h.ws + (which == 0 ? p.ws.TUt : p.ws.TBt));
   __nv_bfloat16 *outb = reinterpret_cast<__nv_bfloat16 *>(jb.h.ws + p.ws.TUtb);
@@ -340,7 +343,7 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
     }
   }
   k_ns_check<<<(p.count * 2 + 127) / 128, 128, 0, s>>>(jobs, p);
-  k_reorth_M<<<dim3(tn, tm, p.count), 256, 0, s>>>(jobs, p, y0[0], y0[1]);
+  k_reorth_M<<<dim3(tn, tm, p.count), 256, 0, s>>>(jobs, p);
   count_launches(3 + 2 * NS_ITERS);
   stage_mark(s, ST_REORTH_NS);
   cudaError_t e = cudaGetLastError();
@@ -365,7 +368,7 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   c.max_sweeps = 40;
   e = launch_core(reinterpret_cast<const char *>(jobs), c, s);
   if (e != cudaSuccess) return e;
-  k_reorth_T<<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p, z0[0], z0[1]);
+  k_reorth_T<<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p);
   count_launches(1);
   stage_mark(s, ST_REORTH_CORE);
 
