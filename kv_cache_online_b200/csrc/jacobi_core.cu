@@ -10,7 +10,7 @@
 // through distributed shared memory. Inside a round a CTA rotates every cross pair of its two
 // blocks (w steps of w disjoint pairs, one half-warp per pair); in the first round of a sweep it
 // also rotates the pairs inside each block. Rotations apply in float32; inner products accumulate
-// in float32 (fold) or float64 (re-orthogonalisation).
+// in float32, or in float64 for the re-orthogonalisation of float32-stored factors.
 //
 // Structure used: the top k rows of A equal diag(sigma) times the top k rows of V (they start as
 // diag(sigma) and I and see the same column rotations), so those k rows of V are not stored:
@@ -259,8 +259,9 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
 
   // Rotate unless |cos| <= tol. In float32 the inner product has relative error ~ sqrt(m) 2^-24 and
   // the tolerance sits a few units above it; residual cosines of that size change singular values
-  // only at second order. The dense mode (re-orthogonalisation, whose purpose is orthonormal
-  // factors) accumulates inner products in float64 and uses a tighter tolerance.
+  // only at second order. The re-orthogonalisation of float32 factors (whose purpose is
+  // orthonormal factors to float32 accuracy) accumulates inner products in float64 and uses a
+  // tighter tolerance.
   const float tol = (DD ? 2.f : 4.f) * sqrtf((float)(m > 1 ? m : 1)) * 5.9604645e-08f;
   const float tol2 = tol * tol;
   int sweeps_used = -1;
@@ -439,7 +440,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
 template <int NE>
 static cudaError_t core_launch(const char *jobs, const CoreParams &p, const JacobiCfg &c,
                                cudaStream_t s) {
-  auto kern = p.mode == 1 ? k_core<NE, true> : k_core<NE, false>;
+  auto kern = p.dd ? k_core<NE, true> : k_core<NE, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)c.smem);
   if (e != cudaSuccess) return e;
@@ -495,6 +496,7 @@ CoreParams fold_core_params(const FoldParams &p) {
   c.hs = p.ws.hs;
   c.ldm = 0;
   c.max_sweeps = 40;
+  c.dd = 0;
   return c;
 }
 

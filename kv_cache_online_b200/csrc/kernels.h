@@ -32,6 +32,7 @@ struct CoreParams {
   size_t C, FP, M;  // inputs (mode 0: C [b][r], FP [b][b]; mode 1: M [k][ldm])
   size_t Gt, Gtb, Gbot, Ht, sig;  // outputs
   int hs, ldm, max_sweeps;
+  int dd;           // 1: inner products accumulated in float64 (tighter tolerance), 0: float32
 };
 
 struct JacobiCfg {

@@ -32,6 +32,40 @@ def test_reorth_parity(storage, tol):
     if storage == torch.float32:
         assert oreo.orthogonality_error(U2) < 1e-4
         assert oreo.orthogonality_error(B2) < 1e-4
+    else:
+        # bf16 factors are orthonormal up to bf16 rounding: the floor is the oracle's orthonormal
+        # result rounded to bf16. The tensor-core rotation applies a bf16 rotation matrix, which
+        # adds about as much again, hence the factor 1.5.
+        for got, ref in ((U2, Ur), (B2, Br)):
+            assert oreo.orthogonality_error(got) < 1.5 * oreo.orthogonality_error(
+                stored(ref, torch.bfloat16))
+
+
+def test_reorth_bf16_removes_drift():
+    """Factors drifted ten times further than in the parity test come back near orthonormal."""
+    m = kv()
+    n, d, r, k = 4096, 1024, 256, 256
+    g = np.random.Generator(np.random.PCG64(37))
+    U = stored(np.linalg.qr(g.standard_normal((n, k)))[0] + 2e-2 * g.standard_normal((n, k)) /
+               np.sqrt(n), torch.bfloat16)
+    B = stored(np.linalg.qr(g.standard_normal((d, k)))[0] + 2e-2 * g.standard_normal((d, k)) /
+               np.sqrt(d), torch.bfloat16)
+    s = stored(np.sqrt(n) * np.arange(1, k + 1) ** -1.0, torch.float32)
+    h = m.LowRankHistory(d, r, n, storage=torch.bfloat16)
+    set_state(h, U, s, B, np.arange(n), folds=16)
+    m.reorth(h)
+    U2, s2, B2, _, (_, _, _, st) = state(h)
+    assert st == 0
+    Ur, sr, Br = oreo.reorth(U, s, B)
+    np.testing.assert_allclose(s2, sr, rtol=1e-4)
+    assert of.rel_fro(of.low_rank_product(U2, s2, B2), of.low_rank_product(U, s, B)) < 2e-2
+    # The rotation matrices are bf16 tensor-core operands, so the result is orthonormal to about
+    # 2^-9 ||T||_F (~0.04 here, per-pair cosines ~1e-4) rather than to the floor of bf16 rounding
+    # of the factors alone (~0.01).
+    for got, ref, before in ((U2, Ur, U), (B2, Br, B)):
+        err = oreo.orthogonality_error(got)
+        assert err < 5.0 * oreo.orthogonality_error(stored(ref, torch.bfloat16))
+        assert err < 0.4 * oreo.orthogonality_error(before)
 
 
 def test_reorth_partial_rank_after_folds():
