@@ -152,6 +152,50 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
                                      size_t ws_bytes, void *stream);
 
 /*
+ * Decode attention over the compressed cache -- Algorithm 3 steps 7-9 without the dense cache
+ * (Section 5.2 names this factor-aware form as the route to a speed-up). For one (sequence,
+ * layer): the keys at every cached position are the compressed rows (U_k[i] sigma_k) B_k^T at
+ * hk.pos[i] and the exact keys k_exact[e] at k_exact_pos[e], each rotated by its own position with
+ * rotate-half RoPE (as iskv_reconstruct); the values are the compressed rows of hv at hv.pos and
+ * the exact values at v_exact_pos (no rotation). For each query head j (KV head
+ * h = j / (n_q_heads / n_kv_heads)):
+ *   s_j(p) = scale * q[j] . key_p[h],  P_j = softmax over the key positions,
+ *   out[j] = sum_p P_j(p) value_p[h],
+ * where the compressed values are mixed in their r-dimensional coordinates and projected once:
+ * sum_i P_j(pos_v[i]) (U_v[i] sigma_v) B_v,h^T. Scores are float32 from the stored factors (bf16
+ * factors: the tensor-core kernel, keys never leave the SM); the softmax and mixing are float32.
+ * q            [n_q_heads][head_dim] float32 device, already rotated for the query position.
+ * out          [n_q_heads][head_dim] float32 device.
+ * k_exact, v_exact  [n][d] exact_dtype device (NULL when n == 0); positions int32 device.
+ * Positions must lie in [0, n_total); the K and V caches must cover the same positions: a key
+ * position without a value leaves probability mass unaccounted (checked to 1e-3) and, like an
+ * out-of-range position or a cache with no key at all, records ISKV_ERR_SHAPE in the status word
+ * (hk for key-side conditions, hv for value-side ones). hk and hv share d, r_max, storage and
+ * n_cap; d == n_kv_heads * head_dim, head_dim even <= 256, n_q_heads a multiple of n_kv_heads
+ * and <= 64.
+ * ws           iskv_attention_workspace_size(count, d, r_max, n_cap, max n_total, n_q_heads) bytes,
+ *              256-byte aligned (scores by position, softmax statistics, partial value sums).
+ * hk, hv and the per-job arrays of the batched form are HOST arrays of `count` entries.
+ */
+size_t iskv_attention_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap,
+                                     int64_t n_total_max, int32_t n_q_heads);
+iskv_status iskv_decode_attention(const iskv_lowrank *hk, const iskv_lowrank *hv,
+                                  const void *k_exact, const int32_t *k_exact_pos,
+                                  int64_t n_k_exact, const void *v_exact,
+                                  const int32_t *v_exact_pos, int64_t n_v_exact,
+                                  int32_t exact_dtype, int64_t n_total, int32_t n_q_heads,
+                                  int32_t n_kv_heads, int32_t head_dim, double rope_theta,
+                                  float scale, const float *q, float *out, void *ws,
+                                  size_t ws_bytes, void *stream);
+iskv_status iskv_decode_attention_batched(
+    const iskv_lowrank *hk, const iskv_lowrank *hv, int32_t count, const void *const *k_exact,
+    const int32_t *const *k_exact_pos, const int64_t *n_k_exact, const void *const *v_exact,
+    const int32_t *const *v_exact_pos, const int64_t *n_v_exact, int32_t exact_dtype,
+    const int64_t *n_total, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+    double rope_theta, float scale, const float *const *q, float *const *out, void *ws,
+    size_t ws_bytes, void *stream);
+
+/*
  * Prompt-block protection -- Section 3.1 and Algorithm 1 steps 2-4: blocks of `block` prompt
  * tokens; the last `suffix_blocks` full blocks and the partial tail are the local suffix; for each
  * KV head, score(block) = min over its tokens of cos(post-RoPE key, block-mean key) (float64,

@@ -11,6 +11,7 @@ Sources: "iS-KV reading notes" (zhongzhuzhou.org), Sections 3-5 and Algorithms 1
 from __future__ import annotations
 
 import ctypes
+import math
 
 import torch
 
@@ -212,6 +213,77 @@ def reconstruct(hist, exact_rows, exact_pos, n_total, n_heads, head_dim, rope, t
     return reconstruct_batched([hist], [exact_rows], [exact_pos], [n_total], n_heads, head_dim,
                                [rope], theta, None if out is None else [out], out_dtype, ws,
                                stream)[0]
+
+
+def attention_workspace_size(count, d, r_max, n_cap, n_total_max, n_q_heads) -> int:
+    return int(_lib.load().iskv_attention_workspace_size(count, d, r_max, n_cap, n_total_max,
+                                                         n_q_heads))
+
+
+def _exact_arrays(rows, pos, d):
+    ptr_r, ptr_p, cnt, dt = [], [], [], ISKV_F32
+    for x, p in zip(rows, pos):
+        if x is None or p is None or p.numel() == 0:
+            ptr_r.append(None)
+            ptr_p.append(None)
+            cnt.append(0)
+            continue
+        _need_cuda(x, p)
+        dt = _dt(x)
+        if p.dtype != torch.int32 or x.shape != (p.numel(), d) or not x.is_contiguous():
+            raise ValueError("exact rows must be (n_exact, d) contiguous with int32 positions")
+        ptr_r.append(x.data_ptr())
+        ptr_p.append(p.data_ptr())
+        cnt.append(p.numel())
+    return ptr_r, ptr_p, cnt, dt
+
+
+def decode_attention_batched(k_hists, v_hists, k_exact, k_exact_pos, v_exact, v_exact_pos,
+                             n_total, q, n_kv_heads, head_dim, theta=500000.0, scale=None,
+                             outs=None, ws=None, stream=None):
+    """Algorithm 3 steps 7-9 without the dense cache: one decode query ``q[i]`` (float32,
+    ``(n_q_heads, head_dim)``, already rotated) per (K, V) history pair. Returns float32
+    ``(n_q_heads, head_dim)`` outputs."""
+    lib = _lib.load()
+    n = len(k_hists)
+    if len(v_hists) != n or len(q) != n:
+        raise ValueError("one V history and one query per K history")
+    d = k_hists[0].d
+    if isinstance(n_total, int):
+        n_total = [n_total] * n
+    for x in q:
+        _need_cuda(x)
+        if x.dtype != torch.float32 or x.dim() != 2 or x.shape[1] != head_dim or not x.is_contiguous():
+            raise ValueError("queries must be contiguous float32 (n_q_heads, head_dim)")
+    nq = q[0].shape[0]
+    if outs is None:
+        outs = [torch.empty(nq, head_dim, dtype=torch.float32, device=x.device) for x in q]
+    scale = 1.0 / math.sqrt(head_dim) if scale is None else float(scale)
+    kr, kp, kn, kdt = _exact_arrays(k_exact, k_exact_pos, d)
+    vr, vp, vn, vdt = _exact_arrays(v_exact, v_exact_pos, d)
+    edt = kdt if any(kn) else vdt
+    if any(kn) and any(vn) and kdt != vdt:
+        raise ValueError("exact keys and values must share a dtype")
+    need = lib.iskv_attention_workspace_size(n, d, k_hists[0].r_max, k_hists[0].n_cap,
+                                             max(n_total), nq)
+    w = ws if ws is not None else _ws(k_hists[0].device, need)
+    P = ctypes.c_void_p * n
+    _lib.check(lib.iskv_decode_attention_batched(
+        _handles(k_hists), _handles(v_hists), n, P(*kr), P(*kp), (ctypes.c_int64 * n)(*kn),
+        P(*vr), P(*vp), (ctypes.c_int64 * n)(*vn), edt, (ctypes.c_int64 * n)(*n_total), nq,
+        n_kv_heads, head_dim, float(theta), scale, P(*[x.data_ptr() for x in q]),
+        P(*[o.data_ptr() for o in outs]), w.data_ptr(), w.numel(), _stream(stream)),
+        "decode_attention")
+    return outs
+
+
+def decode_attention(k_hist, v_hist, k_exact, k_exact_pos, v_exact, v_exact_pos, n_total, q,
+                     n_kv_heads, head_dim, theta=500000.0, scale=None, out=None, ws=None,
+                     stream=None):
+    """Single-pair form of :func:`decode_attention_batched`."""
+    return decode_attention_batched([k_hist], [v_hist], [k_exact], [k_exact_pos], [v_exact],
+                                    [v_exact_pos], [n_total], [q], n_kv_heads, head_dim, theta,
+                                    scale, None if out is None else [out], ws, stream)[0]
 
 
 def select_workspace_size(L, n_heads, block=8) -> int:

@@ -1,0 +1,53 @@
+// Decode attention over the compressed cache: job table and launchers.
+#pragma once
+
+#include "kernels.h"
+
+namespace iskv {
+
+// One (sequence, layer) job: the K and V histories, the exact rows of both caches, the decode
+// query and the output, plus this job's workspace slices.
+struct AttnJob {
+  const void *Uk;            // K history: U [n_cap][r], sigma [r], B [d][r], pos [n_cap], meta
+  const float *sk;
+  const void *Bk;
+  const int32_t *posk;
+  int64_t *metak;
+  const void *Uv;            // V history
+  const float *sv;
+  const void *Bv;
+  const int32_t *posv;
+  int64_t *metav;
+  const void *kex;           // exact keys [n_kex][d] (pre-RoPE) at kexpos
+  const int32_t *kexpos;
+  const void *vex;           // exact values [n_vex][d] at vexpos
+  const int32_t *vexpos;
+  const float *q;            // [n_q][head_dim] float32, already rotated for the query position
+  float *out;                // [n_q][head_dim] float32
+  float *S;                  // workspace [n_q][n_total]: scores by position (-inf where no key)
+  float *stats;              // workspace [n_q][2]: max score, sum of exp(score - max)
+  float *wpart;              // workspace [nchunk][n_q][r]: partial sums of p * U_v rows
+  float *mpart;              // workspace [nchunk][n_q]: partial probability mass on V rows
+  void *bsig;                // workspace: sigma-scaled K basis (tensor-core scores)
+  int64_t n_kex, n_vex, n_total;
+};
+
+struct AttnParams {
+  int d, r, storage, exact_dtype, n_kv, n_q, head_dim, count, nchunk;
+  double theta;
+  float scale;
+  int64_t n_cap_max, n_total_max;
+};
+
+constexpr int ATTN_CHUNK = 512;  // V rows per value-mixing block
+constexpr int ATTN_MAX_Q = 64;   // query heads
+
+cudaError_t launch_attn_init(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
+cudaError_t launch_attn_scores_ffma(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
+cudaError_t launch_attn_scores_exact(const AttnJob *jobs, const AttnParams &p, int64_t max_kex,
+                                     cudaStream_t s);
+cudaError_t launch_attn_stats(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
+cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
+cudaError_t launch_attn_out(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
+
+}  // namespace iskv

@@ -68,6 +68,35 @@ size_t jobs_bytes(int32_t count, size_t each) { return align_up((size_t)count * 
 
 }  // namespace
 
+namespace {
+
+struct AttnWsLayout {
+  size_t tc, recon, slices, bsig, S, stats, wpart, mpart, per_job, total;
+  int nchunk;
+};
+
+AttnWsLayout attn_ws_layout(int32_t count, int32_t d, int32_t r, int64_t n_cap, int64_t n_total_max,
+                            int32_t n_q) {
+  AttnWsLayout L;
+  L.nchunk = (int)((n_cap + ATTN_CHUNK - 1) / ATTN_CHUNK);
+  if (L.nchunk < 1) L.nchunk = 1;
+  L.tc = jobs_bytes(count, sizeof(AttnJob));
+  L.recon = L.tc + tc_table_bytes(count);
+  L.slices = L.recon + jobs_bytes(count, sizeof(ReconJob));
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  L.bsig = take((size_t)d * r * 2);
+  L.S = take((size_t)n_q * (size_t)n_total_max * 4);
+  L.stats = take((size_t)n_q * 2 * 4);
+  L.wpart = take((size_t)L.nchunk * n_q * r * 4);
+  L.mpart = take((size_t)L.nchunk * n_q * 4);
+  L.per_job = o;
+  L.total = L.slices + (size_t)count * L.per_job;
+  return L;
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t iskv_abi_version(void) { return ISKV_ABI_VERSION; }
@@ -428,6 +457,187 @@ iskv_status iskv_reconstruct(const iskv_lowrank *h, const void *exact_rows, int3
   void *o[1] = {out};
   return iskv_reconstruct_batched(h, 1, er, exact_dtype, ep, ne, nt, n_heads, head_dim, ar,
                                   rope_theta, o, out_dtype, ws, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Decode attention over the compressed cache
+size_t iskv_attention_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap,
+                                     int64_t n_total_max, int32_t n_q_heads) {
+  if (count < 1 || d < 1 || r_max < 1 || n_cap < 0 || n_total_max < 0 || n_q_heads < 1) return 0;
+  return attn_ws_layout(count, d, r_max, n_cap, n_total_max, n_q_heads).total;
+}
+
+iskv_status iskv_decode_attention_batched(
+    const iskv_lowrank *hk, const iskv_lowrank *hv, int32_t count, const void *const *k_exact,
+    const int32_t *const *k_exact_pos, const int64_t *n_k_exact, const void *const *v_exact,
+    const int32_t *const *v_exact_pos, const int64_t *n_v_exact, int32_t exact_dtype,
+    const int64_t *n_total, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+    double rope_theta, float scale, const float *const *q, float *const *out, void *ws,
+    size_t ws_bytes, void *stream) {
+  const char *who = "iskv_decode_attention";
+  g_last_error.clear();
+  if (!hk || !hv || !k_exact || !k_exact_pos || !n_k_exact || !v_exact || !v_exact_pos ||
+      !n_v_exact || !n_total || !q || !out)
+    return fail(ISKV_ERR_ARG, "%s: null host array", who);
+  if (count < 1 || count > 4096) return fail(ISKV_ERR_SHAPE, "%s: count must be in [1, 4096]", who);
+  if (!valid_dtype(exact_dtype)) return fail(ISKV_ERR_ARG, "%s: bad dtype", who);
+  if (head_dim < 2 || head_dim % 2 || head_dim > 256)
+    return fail(ISKV_ERR_SHAPE, "%s: need even head_dim <= 256", who);
+  if (n_kv_heads < 1 || n_q_heads < 1 || n_q_heads > ATTN_MAX_Q || n_q_heads % n_kv_heads)
+    return fail(ISKV_ERR_SHAPE, "%s: need n_q_heads a multiple of n_kv_heads, <= %d", who,
+                ATTN_MAX_Q);
+  if (!(rope_theta > 0.0)) return fail(ISKV_ERR_ARG, "%s: rope_theta must be > 0", who);
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
+    return fail(ISKV_ERR_ARG, "%s: scale must be finite", who);
+  int64_t max_kex = 0, ntot_max = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_status st = check_handle(&hk[i], who);
+    if (st == ISKV_OK) st = check_handle(&hv[i], who);
+    if (st != ISKV_OK) return st;
+    for (const iskv_lowrank *h : {&hk[i], &hv[i]})
+      if (h->d != hk[0].d || h->r_max != hk[0].r_max || h->storage != hk[0].storage ||
+          h->n_cap != hk[0].n_cap)
+        return fail(ISKV_ERR_SHAPE, "%s: K and V histories must share d, r_max, storage, n_cap",
+                    who);
+    if (hk[i].d != n_kv_heads * head_dim)
+      return fail(ISKV_ERR_SHAPE, "%s: d must equal n_kv_heads * head_dim", who);
+    if (!q[i] || !out[i]) return fail(ISKV_ERR_ARG, "%s: null query or output", who);
+    if (n_k_exact[i] < 0 || n_v_exact[i] < 0 || n_total[i] < 1)
+      return fail(ISKV_ERR_SHAPE, "%s: bad sizes", who);
+    if ((n_k_exact[i] > 0 && (!k_exact[i] || !k_exact_pos[i])) ||
+        (n_v_exact[i] > 0 && (!v_exact[i] || !v_exact_pos[i])))
+      return fail(ISKV_ERR_ARG, "%s: null exact rows", who);
+    if (n_k_exact[i] > max_kex) max_kex = n_k_exact[i];
+    if (n_total[i] > ntot_max) ntot_max = n_total[i];
+  }
+  const int d = hk[0].d, r = hk[0].r_max;
+  const int64_t ncap = hk[0].n_cap;
+  const AttnWsLayout L = attn_ws_layout(count, d, r, ncap, ntot_max, n_q_heads);
+  iskv_status st = check_ws(ws, ws_bytes, L.total, who);
+  if (st != ISKV_OK) return st;
+  AttnParams p;
+  p.d = d;
+  p.r = r;
+  p.storage = hk[0].storage;
+  p.exact_dtype = exact_dtype;
+  p.n_kv = n_kv_heads;
+  p.n_q = n_q_heads;
+  p.head_dim = head_dim;
+  p.count = count;
+  p.nchunk = L.nchunk;
+  p.theta = rope_theta;
+  p.scale = scale;
+  p.n_cap_max = ncap;
+  p.n_total_max = ntot_max;
+  char *base = static_cast<char *>(ws);
+  std::vector<AttnJob> jobs(count);
+  for (int32_t i = 0; i < count; ++i) {
+    AttnJob &j = jobs[i];
+    char *slice = base + L.slices + (size_t)i * L.per_job;
+    j.Uk = hk[i].U;
+    j.sk = hk[i].sigma;
+    j.Bk = hk[i].B;
+    j.posk = hk[i].pos;
+    j.metak = hk[i].meta;
+    j.Uv = hv[i].U;
+    j.sv = hv[i].sigma;
+    j.Bv = hv[i].B;
+    j.posv = hv[i].pos;
+    j.metav = hv[i].meta;
+    j.kex = k_exact[i];
+    j.kexpos = k_exact_pos[i];
+    j.vex = v_exact[i];
+    j.vexpos = v_exact_pos[i];
+    j.q = q[i];
+    j.out = out[i];
+    j.S = reinterpret_cast<float *>(slice + L.S);
+    j.stats = reinterpret_cast<float *>(slice + L.stats);
+    j.wpart = reinterpret_cast<float *>(slice + L.wpart);
+    j.mpart = reinterpret_cast<float *>(slice + L.mpart);
+    j.bsig = slice + L.bsig;
+    j.n_kex = n_k_exact[i];
+    j.n_vex = n_v_exact[i];
+    j.n_total = n_total[i];
+  }
+  const bool tc = tc_attn_supported(r, p.storage, head_dim, n_q_heads, n_kv_heads);
+  std::vector<TcJob> tj;
+  std::vector<ReconJob> rj;
+  ReconParams rp;
+  if (tc) {
+    tj.resize(count);
+    rj.resize(count);
+    for (int32_t i = 0; i < count; ++i) {
+      std::memset(&rj[i], 0, sizeof(ReconJob));
+      rj[i].U = hk[i].U;
+      rj[i].sigma = hk[i].sigma;
+      rj[i].B = hk[i].B;
+      rj[i].pos = hk[i].pos;
+      rj[i].meta = hk[i].meta;
+      rj[i].bsig = jobs[i].bsig;
+      if (!encode_attn_job(tj[i], hk[i].U, ncap, r, jobs[i].bsig, d, jobs[i].S, q[i], hk[i].pos,
+                           hk[i].meta, n_total[i], scale))
+        return fail(ISKV_ERR_CUDA, "%s: tensor map encoding failed", who);
+    }
+    rp.d = d;
+    rp.r = r;
+    rp.storage = p.storage;
+    rp.exact_dtype = exact_dtype;
+    rp.out_dtype = ISKV_BF16;
+    rp.n_heads = n_kv_heads;
+    rp.head_dim = head_dim;
+    rp.count = count;
+    rp.exact_vec = 0;
+    rp.theta = rope_theta;
+    rp.n_cap_max = ncap;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  AttnJob *djobs = reinterpret_cast<AttnJob *>(base);
+  TcJob *tc_dev = reinterpret_cast<TcJob *>(base + L.tc);
+  ReconJob *recon_dev = reinterpret_cast<ReconJob *>(base + L.recon);
+  stage_begin(s);
+  cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(AttnJob) * count, s);
+  if (e == cudaSuccess && tc) e = upload_jobs(tc_dev, tj.data(), sizeof(TcJob) * count, s);
+  if (e == cudaSuccess && tc) e = upload_jobs(recon_dev, rj.data(), sizeof(ReconJob) * count, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention: upload");
+  stage_mark(s, ST_UPLOAD);
+  if ((e = launch_attn_init(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "attention: init");
+  if (tc && (e = launch_recon_bsig(recon_dev, rp, s)) != cudaSuccess)
+    return cuda_fail(e, "attention: scaled basis");
+  stage_mark(s, ST_ATTN_PREPARE);
+  e = tc ? launch_tc_attn_scores(tc_dev, p, s) : launch_attn_scores_ffma(djobs, p, s);
+  if (e == cudaSuccess) e = launch_attn_scores_exact(djobs, p, max_kex, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention: scores");
+  stage_mark(s, ST_ATTN_SCORES);
+  if ((e = launch_attn_stats(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "attention: softmax");
+  stage_mark(s, ST_ATTN_SOFTMAX);
+  e = launch_attn_values(djobs, p, s);
+  if (e == cudaSuccess) e = launch_attn_out(djobs, p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention: values");
+  stage_mark(s, ST_ATTN_VALUES);
+  return ISKV_OK;
+}
+
+iskv_status iskv_decode_attention(const iskv_lowrank *hk, const iskv_lowrank *hv,
+                                  const void *k_exact, const int32_t *k_exact_pos,
+                                  int64_t n_k_exact, const void *v_exact,
+                                  const int32_t *v_exact_pos, int64_t n_v_exact,
+                                  int32_t exact_dtype, int64_t n_total, int32_t n_q_heads,
+                                  int32_t n_kv_heads, int32_t head_dim, double rope_theta,
+                                  float scale, const float *q, float *out, void *ws,
+                                  size_t ws_bytes, void *stream) {
+  if (!hk || !hv) return fail(ISKV_ERR_ARG, "iskv_decode_attention: null history handle");
+  const void *ke[1] = {k_exact};
+  const int32_t *kp[1] = {k_exact_pos};
+  const int64_t nk[1] = {n_k_exact};
+  const void *ve[1] = {v_exact};
+  const int32_t *vp[1] = {v_exact_pos};
+  const int64_t nv[1] = {n_v_exact};
+  const int64_t nt[1] = {n_total};
+  const float *qq[1] = {q};
+  float *oo[1] = {out};
+  return iskv_decode_attention_batched(hk, hv, 1, ke, kp, nk, ve, vp, nv, exact_dtype, nt,
+                                       n_q_heads, n_kv_heads, head_dim, rope_theta, scale, qq, oo,
+                                       ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------------------------------------

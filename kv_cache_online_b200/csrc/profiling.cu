@@ -29,7 +29,8 @@ const char *kNames[ST_COUNT] = {
     "fold.coord_rotate", "fold.finalize",     "reorth.gram",        "reorth.newton_schulz",
     "reorth.core_svd", "reorth.coord_rotate", "reorth.basis_rotate", "reconstruct.prepare",
     "reconstruct.compressed",
-    "reconstruct.exact", "select",            "job_upload"};
+    "reconstruct.exact", "select",            "job_upload",        "attention.prepare",
+    "attention.scores", "attention.softmax",  "attention.values"};
 
 cudaEvent_t take_event() {
   if (!g_free.empty()) {

@@ -26,6 +26,10 @@ enum Stage {
   ST_RECON_EXACT,
   ST_SELECT,
   ST_UPLOAD,
+  ST_ATTN_PREPARE,
+  ST_ATTN_SCORES,
+  ST_ATTN_SOFTMAX,
+  ST_ATTN_VALUES,
   ST_COUNT
 };
 

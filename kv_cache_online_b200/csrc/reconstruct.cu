@@ -1,26 +1,12 @@
 // Per-step reconstruction (iS-KV reading notes, Algorithm 3 steps 7-8): compressed row i of a
 // history is (U[i] * sigma) B^T, written to its original position pos[i]; exact rows are copied to
-// their own positions; keys are rotated by their own position with rotate-half RoPE.
-//
-// RoPE angles: pos * theta^(-2j/hd) reaches tens of thousands of radians, where one float32 ulp is
-// ~4e-3 rad. The angle is therefore formed and reduced modulo 2 pi in float64 and only the reduced
-// angle (|a| <= pi) goes to sincosf.
+// their own positions; keys are rotated by their own position with rotate-half RoPE (angles
+// reduced in float64, rope.cuh).
 #include "profiling.h"
 #include "recon.h"
+#include "rope.cuh"
 
 namespace iskv {
-
-ISKV_DEV double rope_inv_freq(int j, int hd, double log_theta) {
-  return exp(-2.0 * (double)j / (double)hd * log_theta);
-}
-
-ISKV_DEV void rope_sincos(int64_t pos, double inv_freq, float &c, float &s) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_two_pi = 0.15915494309189533576888376337251;
-  double a = (double)pos * inv_freq;
-  a = fma(-two_pi, rint(a * inv_two_pi), a);
-  sincosf((float)a, &s, &c);
-}
 
 // ------------------------------------------------------------------------------------------------
 // CUDA-core path (float32 storage, and any storage when the tensor-core path is not selected).

@@ -5,6 +5,7 @@
 
 #include <vector>
 
+#include "attention.h"
 #include "kernels.h"
 #include "recon.h"
 
@@ -24,6 +25,9 @@ struct alignas(64) TcJob {
   int64_t n_total;
   int32_t rope;
   int32_t tiles_ok;      // reconstruction: mapO is encoded (n_total >= 32), tile stores allowed
+  float *S;              // attention scores: [n_q][n_total] float32 by position
+  const float *q;        // attention scores: queries [n_q][128] float32
+  float scale;           // attention scores: score scale
 };
 
 struct TcParams {
@@ -59,6 +63,14 @@ cudaError_t launch_tc_rotation(const TcJob *djobs, int count, int r, int64_t n_c
 // Sigma-scaled basis for every job (the operand of launch_tc_recon); stage "reconstruct.prepare".
 cudaError_t launch_recon_bsig(const ReconJob *djobs_recon, const ReconParams &p, cudaStream_t s);
 cudaError_t launch_tc_recon(const TcJob *djobs, const ReconParams &p, cudaStream_t s);
+
+// Decode-attention scores of compressed keys (the reconstruction kernel with a scores epilogue):
+// bf16 factors, head_dim 128, r a multiple of 64 up to 256, 1, 2, 4 or 8 query heads per KV head.
+bool tc_attn_supported(int r, int storage, int head_dim, int n_q, int n_kv);
+bool encode_attn_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void *bsig, int d,
+                     float *S, const float *q, const int32_t *pos, int64_t *meta, int64_t n_total,
+                     float scale);
+cudaError_t launch_tc_attn_scores(const TcJob *djobs, const AttnParams &p, cudaStream_t s);
 
 // One CTA waiting on a barrier nothing arrives at, bounded by limit_ns (failure-path self-test).
 cudaError_t launch_wait_timeout(int64_t *meta, uint64_t limit_ns, cudaStream_t s);

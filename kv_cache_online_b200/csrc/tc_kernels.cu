@@ -241,6 +241,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
 // gaps or invalid rows are written from registers.
 constexpr int REC_MAX_STAGES = 8;
 constexpr int REC_STG_BYTES = 2 * TC_M * 128;  // lo and hi column halves of one head
+// Attention scores (qpk query heads per KV head): the staging region holds, per warp pair, the
+// query groups of the CTA's (at most two) heads and a 32-row exchange of partial scores.
+__host__ __device__ constexpr int attn_pair_floats(int qpk) { return 2 * 64 * 2 * qpk + 32 * 2 * qpk; }
+__host__ __device__ constexpr int rec_stg_bytes(int qpk) { return qpk ? 4 * attn_pair_floats(qpk) * 4 : REC_STG_BYTES; }
 
 // RoPE tables (head_dim 128, 64 frequencies omega_j = theta^(-2j/128)). Angles are reduced in
 // exact integer arithmetic: W_j = omega_j / (2 pi) is held as a 0.64 fixed-point fraction
@@ -280,6 +284,10 @@ struct RecCtl {
   int abort;
 };
 
+// QPK = 0: reconstruction (rows written to out[pos]). QPK > 0: decode-attention scores -- each
+// RoPE'd key row is dotted with the QPK query heads of its KV head and only the scores
+// S[query head][pos] are written; the dense keys never leave the SM.
+template <int QPK>
 __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcParams p,
                                                            const __grid_constant__ RopeTab rt) {
   extern __shared__ uint8_t smem_raw[];
@@ -290,7 +298,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
   uint8_t *sB = smem;                            // KS slabs x (HP x 128 rows) x 128 B, resident
   uint8_t *sA = sB + KS * HP * SLAB_BYTES;       // NA slabs x 16 KB
   uint8_t *sStg = sA + NA * SLAB_BYTES;          // 2 x (128 rows x 128 B), SW128
-  RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + REC_STG_BYTES);
+  RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + rec_stg_bytes(QPK));
   RopeTab *rope_tab = reinterpret_cast<RopeTab *>(ctl + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NN = HP * HN;                        // MMA N
@@ -461,12 +469,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     __nv_bfloat16 *h_out = nullptr;
     int64_t h_rows = 0, h_total = 0;
     bool h_rope = false, h_tiles = false;
+    float *h_S = nullptr;
+    float h_scale = 0.f;
     auto hist = [&](int j) {
       if (j != hj) {
         hj = j;
         const TcJob &jb = jobs[j];
         h_pos = jb.pos;
         h_out = static_cast<__nv_bfloat16 *>(jb.out);
+        h_S = jb.S;
+        h_scale = jb.scale;
         h_rows = rows_of(j);
         h_total = jb.n_total;
         h_rope = jb.rope != 0;
@@ -482,6 +494,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       return row < h_rows ? __ldg(h_pos + row) : 0;
     };
     int acq_j = -1;  // history whose output tensor map this thread last acquired
+    int q_job = -1;  // history whose query groups this pair holds (scores mode)
     Cur c = c_first;
     int32_t ps_next = row_pos(c);
     for (;;) {
@@ -509,6 +522,77 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
           cs[i] = 1.f;
           sn[i] = 0.f;
         }
+      }
+      if constexpr (QPK > 0) {
+        // Scores: the pair keeps the query groups of the CTA's heads in shared memory, laid out
+        // [head][pair j][lo, hi][query] so that each key pair reads its 2 QPK weights contiguously.
+        float *qv = reinterpret_cast<float *>(sStg) + q * attn_pair_floats(QPK);
+        float *xch = qv + 2 * 64 * 2 * QPK;  // [32 rows][2 heads][QPK] partial scores of half 1
+        if (jj != q_job) {  // the same in both warps of the pair; both are past the last reads
+          const float *qg = jobs[jj].q;
+          for (int e = half * 32 + lane; e < HP * QPK * HN; e += 64) {
+            const int hh = e / (QPK * HN), g = (e / HN) % QPK, f = e % HN;
+            qv[((hh * 64 + (f & 63)) * 2 + (f >> 6)) * QPK + g] =
+                qg[(size_t)((member * HP + hh) * QPK + g) * HN + f];
+          }
+          named_sync(pair_bar, 64);
+          q_job = jj;
+        }
+        const int buf = nc & 1, use = nc >> 1;
+        if (!named_and(pair_bar, 64, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
+          fail_timeout(ctl, jobs[jj].meta);
+          break;
+        }
+        fence_after_sync();
+        const uint32_t base = tmem + buf * NN + ((uint32_t)(q * 32) << 16);
+        float acc[2][QPK];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int g = 0; g < QPK; ++g) acc[h][g] = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h >= HP) break;
+#pragma unroll
+          for (int jb16 = 0; jb16 < 32; jb16 += 16) {
+            float lo[16], hi[16];
+            tmem_ld16(base + h * HN + j0 + jb16, lo);
+            tmem_ld16(base + h * HN + 64 + j0 + jb16, hi);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float c0 = cs[jb16 + i], s0 = sn[jb16 + i];
+              const float olo = lo[i] * c0 - hi[i] * s0, ohi = hi[i] * c0 + lo[i] * s0;
+              const float *qj = qv + ((h * 64 + j0 + jb16 + i) * 2) * QPK;
+#pragma unroll
+              for (int g = 0; g < QPK; ++g)
+                acc[h][g] = fmaf(qj[g], olo, fmaf(qj[QPK + g], ohi, acc[h][g]));
+            }
+          }
+        }
+        // The accumulators are in registers: tensor memory can take the next unit.
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+        if (half == 1)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int g = 0; g < QPK; ++g) xch[(lane * 2 + h) * QPK + g] = acc[h][g];
+        named_sync(pair_bar, 64);
+        if (half == 0 && valid) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int g = 0; g < QPK; ++g) {
+              if (h >= HP) break;
+              const int qh = (member * HP + h) * QPK + g;
+              h_S[(size_t)qh * n_total + ps] = h_scale * (acc[h][g] + xch[(lane * 2 + h) * QPK + g]);
+            }
+        }
+        ++nc;
+        c = cn;
+        continue;
       }
       __nv_bfloat16 *orow = out + (size_t)(valid ? ps : 0) * D + (size_t)member * HP * HN;
       // This lane quarter's 32 rows go out as tiles when their positions are consecutive (the
@@ -796,19 +880,19 @@ size_t tc_rot_smem(int r) {
 
 // Resident basis rows for hp heads, the U slab ring, the output staging rows, the barriers and the
 // RoPE frequencies.
-size_t tc_rec_smem(int r, int hp, int stages) {
+size_t tc_rec_smem(int r, int hp, int stages, int stg_bytes) {
   return 1024 + (size_t)hp * (r / 64) * SLAB_BYTES + (size_t)stages * SLAB_BYTES +
-         (size_t)REC_STG_BYTES + sizeof(RecCtl) + sizeof(RopeTab);
+         (size_t)stg_bytes + sizeof(RecCtl) + sizeof(RopeTab);
 }
 
 constexpr size_t kRecSmemCap = 227 * 1024;
 
 // Heads per CTA and U ring depth for the reconstruction: two heads when the head count is even,
 // and as many 16 KB slabs (up to REC_MAX_STAGES) as the shared memory left over holds.
-void tc_rec_shape(int r, int n_heads, int &hp, int &stages) {
-  hp = (n_heads % 2 == 0 && tc_rec_smem(r, 2, 3) <= kRecSmemCap) ? 2 : 1;
+void tc_rec_shape(int r, int n_heads, int stg_bytes, int &hp, int &stages) {
+  hp = (n_heads % 2 == 0 && tc_rec_smem(r, 2, 3, stg_bytes) <= kRecSmemCap) ? 2 : 1;
   stages = REC_MAX_STAGES;
-  while (stages > 2 && tc_rec_smem(r, hp, stages) > kRecSmemCap) --stages;
+  while (stages > 2 && tc_rec_smem(r, hp, stages, stg_bytes) > kRecSmemCap) --stages;
 }
 
 cudaError_t launch_tc_rotation(const TcJob *djobs, int count, int r, int64_t n_cap_max,
@@ -872,9 +956,9 @@ cudaError_t launch_tc_recon(const TcJob *djobs, const ReconParams &p, cudaStream
   tp.count = p.count;
   tp.tiles_per_job = (int)((p.n_cap_max + TC_M - 1) / TC_M);
   tp.theta = p.theta;
-  tc_rec_shape(p.r, p.n_heads, tp.hp, tp.stages);
-  const size_t smem = tc_rec_smem(p.r, tp.hp, tp.stages);
-  cudaError_t e = cudaFuncSetAttribute(k_rec_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  tc_rec_shape(p.r, p.n_heads, REC_STG_BYTES, tp.hp, tp.stages);
+  const size_t smem = tc_rec_smem(p.r, tp.hp, tp.stages, REC_STG_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(k_rec_tc<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Whole groups of n_heads / hp CTAs, as many as fit one per SM (at least one group), and no
   // more groups than row tiles.
@@ -883,9 +967,68 @@ cudaError_t launch_tc_recon(const TcJob *djobs, const ReconParams &p, cudaStream
   int groups = num_sms() / G;
   if (groups < 1) groups = 1;
   if (groups > total) groups = total;
-  k_rec_tc<<<groups * G, TC_THREADS, smem, s>>>(djobs, tp, make_rope_tab(p.theta));
+  k_rec_tc<0><<<groups * G, TC_THREADS, smem, s>>>(djobs, tp, make_rope_tab(p.theta));
   count_launches(1);
   return cudaGetLastError();
+}
+
+bool tc_attn_supported(int r, int storage, int head_dim, int n_q, int n_kv) {
+  if (n_kv < 1 || n_q % n_kv) return false;
+  const int qpk = n_q / n_kv;
+  return storage == ISKV_BF16 && head_dim == 128 && r % 64 == 0 && r >= 64 && r <= 256 &&
+         (qpk == 1 || qpk == 2 || qpk == 4 || qpk == 8) && encode_fn() != nullptr;
+}
+
+bool encode_attn_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void *bsig, int d,
+                     float *S, const float *q, const int32_t *pos, int64_t *meta, int64_t n_total,
+                     float scale) {
+  std::memset(&tj, 0, sizeof(tj));
+  if (!encode_2d(&tj.mapA, U, (uint64_t)n_cap, (uint64_t)r, 128)) return false;
+  if (!encode_2d(&tj.mapB, bsig, (uint64_t)d, (uint64_t)r, 128)) return false;
+  tj.pos = pos;
+  tj.meta = meta;
+  tj.n_total = n_total;
+  tj.rope = 1;
+  tj.tiles_ok = 0;
+  tj.S = S;
+  tj.q = q;
+  tj.scale = scale;
+  return true;
+}
+
+template <int QPK>
+static cudaError_t attn_scores_qpk(const TcJob *djobs, const TcParams &tp, int G, cudaStream_t s) {
+  const size_t smem = tc_rec_smem(tp.r, tp.hp, tp.stages, rec_stg_bytes(QPK));
+  cudaError_t e = cudaFuncSetAttribute(k_rec_tc<QPK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int total = tp.count * tp.tiles_per_job;
+  int groups = num_sms() / G;
+  if (groups < 1) groups = 1;
+  if (groups > total) groups = total;
+  k_rec_tc<QPK><<<groups * G, TC_THREADS, smem, s>>>(djobs, tp, make_rope_tab(tp.theta));
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_attn_scores(const TcJob *djobs, const AttnParams &p, cudaStream_t s) {
+  TcParams tp;
+  tp.r = p.r;
+  tp.d = p.d;
+  tp.n_heads = p.n_kv;
+  tp.count = p.count;
+  tp.tiles_per_job = (int)((p.n_cap_max + TC_M - 1) / TC_M);
+  tp.theta = p.theta;
+  const int qpk = p.n_q / p.n_kv;
+  tc_rec_shape(p.r, p.n_kv, rec_stg_bytes(qpk), tp.hp, tp.stages);
+  const int G = p.n_kv / tp.hp;
+  switch (qpk) {
+    case 1: return attn_scores_qpk<1>(djobs, tp, G, s);
+    case 2: return attn_scores_qpk<2>(djobs, tp, G, s);
+    case 4: return attn_scores_qpk<4>(djobs, tp, G, s);
+    case 8: return attn_scores_qpk<8>(djobs, tp, G, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 bool tc_gram_supported(int r, int storage) {
