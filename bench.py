@@ -44,6 +44,7 @@ N_MID = 16384
 PROMPT, WINDOW = 512, 128
 THETA = 500000.0
 SEL_L = 65536
+Q_HEADS = 32  # decode-attention query heads (grouped: 4 per KV head)
 SPEC = {"K": 1.2, "V": 0.6}
 NOISE = 0.02
 
@@ -255,6 +256,59 @@ def stage_bytes(n_mean: float, layers: int = LAYERS):
     }, H * n_tot
 
 
+def time_attention(wl, kv, torch, dev, stream, reps: int = 10, warm: int = 3):
+    """Decode attention over the compressed cache of every layer (K and V histories of the
+    benchmark state, the same 640 exact rows per history, one float32 query of 32 heads per
+    layer), timed on its own: it is the next row after the hot path, not part of the step."""
+    layers = len(wl.hists) // 2
+    n = int(wl.hists[0].status()[1])
+    epos = torch.cat([torch.arange(0, PROMPT, dtype=torch.int32, device=dev),
+                      torch.arange(PROMPT + n, PROMPT + n + WINDOW, dtype=torch.int32,
+                                   device=dev)])
+    n_total = PROMPT + n + WINDOW
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(777)
+    qs = [torch.randn(Q_HEADS, HEAD_DIM, generator=gen, device=dev) for _ in range(layers)]
+    outs = [torch.empty(Q_HEADS, HEAD_DIM, dtype=torch.float32, device=dev) for _ in range(layers)]
+    kh, vh = wl.hists[0::2], wl.hists[1::2]
+    kex, vex = wl.exact[0::2], wl.exact[1::2]
+    ws = torch.empty(kv.attention_workspace_size(layers, D, R, wl.n_cap, n_total, Q_HEADS) + 256,
+                     dtype=torch.uint8, device=dev)
+    wsa = Workload._aligned(ws)
+
+    def call():
+        kv.decode_attention_batched(kh, vh, kex, [epos] * layers, vex, [epos] * layers, n_total,
+                                    qs, HEADS, HEAD_DIM, THETA, outs=outs, ws=wsa, stream=stream)
+
+    for _ in range(warm):
+        call()
+    torch.cuda.synchronize(dev)
+    kv.stage_times(reset=True)
+    kv.stage_timing(True)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(reps):
+        call()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    kv.stage_timing(False)
+    st = kv.stage_times(reset=True)
+    ms = ev0.elapsed_time(ev1) / reps
+    status = [h.status()[3] for h in wl.hists]
+    # Algorithmic bytes per call: both coordinate tables, both bases, the exact rows of both
+    # caches and the positions (scores and partial sums are the kernels' own intermediates).
+    byt = layers * (2 * n * R * 2 + 2 * D * R * 2 + 2 * (PROMPT + WINDOW) * D * 2 + 2 * n * 4)
+    hbm, _, _ = peaks()
+    gbs = byt / (ms / 1e3) / 1e9
+    return {"ms_per_call": round(ms, 4), "layers": layers, "n": n, "n_total": n_total,
+            "q_heads": Q_HEADS, "kv_heads": HEADS, "bytes_per_call": int(byt),
+            "achieved_gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+            "stages": {k: round(v[0] / max(v[1], 1), 4) for k, v in st.items()
+                       if k.startswith("attention") and v[1]},
+            "status_clean": all(x == 0 for x in status)}
+
+
 def run_b200(args):
     import torch
     import torch.distributed as dist
@@ -348,6 +402,11 @@ def run_b200(args):
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
                 "traffic": traffic, "dominant_stage": dom}
 
+    # Decode attention over the compressed cache (the next row after the hot path), timed apart.
+    attn = None
+    if not args.no_attention:
+        attn = time_attention(wl, kv, torch, dev, stream)
+
     # End-to-end through the C ABI with host buffers.
     e2e = None
     if not args.no_e2e:
@@ -380,6 +439,7 @@ def run_b200(args):
             "clocks": clocks,
             "cpu_baseline": cpu,
             "parity_spot_check": check,
+            "decode_attention": attn,
         }
         print(json.dumps(line))
     if world > 1:
@@ -579,6 +639,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-check", action="store_true")
+    ap.add_argument("--no-attention", action="store_true",
+                    help="skip the separately timed decode attention over the compressed cache")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="model layers (2 histories each); the headline workload is 32")

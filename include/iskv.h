@@ -171,8 +171,8 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
  * position without a value leaves probability mass unaccounted (checked to 1e-3) and, like an
  * out-of-range position or a cache with no key at all, records ISKV_ERR_SHAPE in the status word
  * (hk for key-side conditions, hv for value-side ones). hk and hv share d, r_max, storage and
- * n_cap; d == n_kv_heads * head_dim, head_dim even <= 256, n_q_heads a multiple of n_kv_heads
- * and <= 64.
+ * n_cap; d == n_kv_heads * head_dim, head_dim even <= 256, n_q_heads a multiple of n_kv_heads,
+ * <= 64 and at most 8 per KV head.
  * ws           iskv_attention_workspace_size(count, d, r_max, n_cap, max n_total, n_q_heads) bytes,
  *              256-byte aligned (scores by position, softmax statistics, partial value sums).
  * hk, hv and the per-job arrays of the batched form are HOST arrays of `count` entries.

@@ -12,6 +12,7 @@
 // The probability mass that lands on value rows is summed as well: a key position without a value
 // row leaves it short of 1 and records ISKV_ERR_SHAPE.
 #include "attention.h"
+#include "gemm_tile.cuh"
 #include "profiling.h"
 #include "rope.cuh"
 
@@ -215,155 +216,191 @@ cudaError_t launch_attn_stats(const AttnJob *jobs, const AttnParams &p, cudaStre
 }
 
 // ------------------------------------------------------------------------------------------------
-// Compressed values, mixed in coordinate space: block c of a job sums P_j(pos_v[i]) U_v[i] over its
-// ATTN_CHUNK rows for every query head j (one column of U per thread, one accumulator per head),
-// 64 rows at a time with the probabilities staged in shared memory.
-constexpr int AV_SUB = 64;
-
-template <typename TS>
-__global__ void __launch_bounds__(256) k_attn_values(const AttnJob *jobs, AttnParams p) {
+// Probabilities at the compressed value rows, P[j][i] = P_j(pos_v[i]), laid out densely by row so
+// that the value-mixing GEMM streams them (0 for a row outside the cache, which is flagged).
+__global__ void __launch_bounds__(256) k_attn_probs(const AttnJob *jobs, AttnParams p) {
   const AttnJob &jb = jobs[blockIdx.y];
-  const int c = blockIdx.x, nq = p.n_q, r = p.r;
   const int64_t n = jb.metav[ISKV_META_N];
-  const int k = (int)jb.metav[ISKV_META_K];
-  __shared__ float P[AV_SUB][ATTN_MAX_Q];
-  __shared__ float mass[ATTN_MAX_Q];
-  const TS *U = static_cast<const TS *>(jb.Uv);
-  const int64_t i0 = (int64_t)c * ATTN_CHUNK, i1 = min64(n, i0 + ATTN_CHUNK);
-  if (threadIdx.x < ATTN_MAX_Q) mass[threadIdx.x] = 0.f;
-  for (int l0 = 0; l0 < r; l0 += blockDim.x) {
-    const int l = l0 + threadIdx.x;
-    float acc[ATTN_MAX_Q];
-#pragma unroll
-    for (int j = 0; j < ATTN_MAX_Q; ++j) acc[j] = 0.f;
-    for (int64_t s0 = i0; s0 < i1; s0 += AV_SUB) {
-      const int rows = (int)min64(AV_SUB, i1 - s0);
-      __syncthreads();
-      for (int e = threadIdx.x; e < AV_SUB * nq; e += blockDim.x) {
-        const int ii = e / nq, j = e % nq;
-        float pv = 0.f;
-        if (ii < rows) {
-          const int64_t pos = jb.posv[s0 + ii];
-          if (pos >= 0 && pos < jb.n_total) {
-            pv = __expf(jb.S[(size_t)j * jb.n_total + pos] - jb.stats[2 * j]) * jb.stats[2 * j + 1];
-          } else if (j == 0) {
-            record_status(jb.metav, ISKV_ERR_SHAPE);
-          }
-        }
-        P[ii][j] = pv;
-      }
-      __syncthreads();
-      if (l0 == 0 && threadIdx.x < nq) {
-        float m = 0.f;
-        for (int ii = 0; ii < rows; ++ii) m += P[ii][threadIdx.x];
-        mass[threadIdx.x] += m;
-      }
-      if (l < k) {
-        for (int ii = 0; ii < rows; ++ii) {
-          const float u = to_f<TS>(U[(size_t)(s0 + ii) * r + l]);
-#pragma unroll
-          for (int j = 0; j < ATTN_MAX_Q; j += 4) {
-            if (j >= nq) break;
-            const float4 pv = *reinterpret_cast<const float4 *>(&P[ii][j]);
-            acc[j] = fmaf(pv.x, u, acc[j]);
-            acc[j + 1] = fmaf(pv.y, u, acc[j + 1]);
-            acc[j + 2] = fmaf(pv.z, u, acc[j + 2]);
-            acc[j + 3] = fmaf(pv.w, u, acc[j + 3]);
-          }
-        }
-      }
-    }
-    if (l < r) {
-      float *wp = jb.wpart + (size_t)c * nq * r;
-#pragma unroll
-      for (int j = 0; j < ATTN_MAX_Q; ++j)
-        if (j < nq) wp[(size_t)j * r + l] = acc[j];
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x < nq) jb.mpart[(size_t)c * nq + threadIdx.x] = mass[threadIdx.x];
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int64_t pos = jb.posv[i], nt = jb.n_total;
+  const bool ok = pos >= 0 && pos < nt;
+  if (!ok) record_status(jb.metav, ISKV_ERR_SHAPE);
+  for (int j = 0; j < p.n_q; ++j)
+    jb.P[(size_t)j * p.n_cap_max + i] =
+        ok ? __expf(jb.S[(size_t)j * nt + pos] - jb.stats[2 * j]) * jb.stats[2 * j + 1] : 0.f;
 }
 
-cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
-  if (p.storage == ISKV_BF16)
-    k_attn_values<__nv_bfloat16><<<dim3(p.nchunk, p.count), 256, 0, s>>>(jobs, p);
-  else
-    k_attn_values<float><<<dim3(p.nchunk, p.count), 256, 0, s>>>(jobs, p);
+cudaError_t launch_attn_probs(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
+  const unsigned gx = (unsigned)((p.n_cap_max + 255) / 256);
+  if (gx == 0) return cudaSuccess;
+  k_attn_probs<<<dim3(gx, p.count), 256, 0, s>>>(jobs, p);
   count_launches(1);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------------------------------
-// Output of one query head: o = B_v,h (sigma_v * sum_c wpart[c]) + sum_e P(pos_e) v_e[h], and the
-// probability-mass check.
+// Compressed values, mixed in coordinate space: W_c = P_c^T [U_v | 1] over the ATTN_CHUNK rows of
+// chunk c -- a register-tiled GEMM (M = query heads, N = r + 1, K = rows). The appended column of
+// ones yields the probability mass the chunk's value rows carry.
+constexpr int AV_BM = 32, AV_BN = 64, AV_BK = 16, AV_TM = 4, AV_TN = 4;
+constexpr int AV_THREADS = (AV_BM / AV_TM) * (AV_BN / AV_TN);
+
+template <typename TS>
+__global__ void __launch_bounds__(AV_THREADS) k_attn_values(const AttnJob *jobs, AttnParams p) {
+  const AttnJob &jb = jobs[blockIdx.z];
+  const int mt = (p.n_q + AV_BM - 1) / AV_BM;
+  const int c = blockIdx.y / mt, m0 = (blockIdx.y % mt) * AV_BM, n0 = blockIdx.x * AV_BN;
+  const int nq = p.n_q, r = p.r;
+  const int64_t n = jb.metav[ISKV_META_N];
+  const int k = (int)jb.metav[ISKV_META_K];
+  const int64_t i0 = (int64_t)c * ATTN_CHUNK;
+  const int rows = (int)min64(ATTN_CHUNK, n > i0 ? n - i0 : 0);
+  const TS *U = static_cast<const TS *>(jb.Uv);
+  const float *P = jb.P + i0;
+  const size_t ldp = (size_t)p.n_cap_max;
+  float *wp = jb.wpart + (size_t)c * nq * r;
+  float *mp = jb.mpart + (size_t)c * nq;
+  tile_gemm<AV_BM, AV_BN, AV_BK, AV_TM, AV_TN, true, true>(
+      m0, n0, nq, r + 1, rows,
+      [&](int j, int i) { return P[(size_t)j * ldp + i]; },
+      [&](int i, int l) {
+        return l < k ? to_f<TS>(U[(size_t)(i0 + i) * r + l]) : (l == r ? 1.f : 0.f);
+      },
+      [&](int j, int l, float acc) {
+        if (l < r) wp[(size_t)j * r + l] = acc;
+        else mp[j] = acc;
+      });
+}
+
+cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
+  const int mt = (p.n_q + AV_BM - 1) / AV_BM;
+  const dim3 g((p.r + 1 + AV_BN - 1) / AV_BN, mt * p.nchunk, p.count);
+  if (p.storage == ISKV_BF16)
+    k_attn_values<__nv_bfloat16><<<g, AV_THREADS, 0, s>>>(jobs, p);
+  else
+    k_attn_values<float><<<g, AV_THREADS, 0, s>>>(jobs, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------------
+// Outputs of the query group of one KV head h: o_j = B_v,h (sigma_v * sum_c wpart[c][j]) +
+// sum_e P_j(pos_e) v_e[h], and the probability-mass check. One block per (KV head, job): the
+// group's coordinate vectors and exact-row probabilities sit in shared memory, each value row of
+// the head is read once for the whole group, and the row loops keep several loads in flight.
+constexpr int AO_ROWS = 512;  // exact rows per staged batch
+
 template <typename TS, typename TE>
 __global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParams p) {
   const AttnJob &jb = jobs[blockIdx.y];
-  const int qh = blockIdx.x, nq = p.n_q, r = p.r, hd = p.head_dim;
-  const int h = qh / (nq / p.n_kv);
+  const int h = blockIdx.x, nq = p.n_q, r = p.r, hd = p.head_dim;
+  const int qpk = nq / p.n_kv, q0 = h * qpk;
   const int k = (int)jb.metav[ISKV_META_K];
   extern __shared__ float sm[];
-  float *w = sm;            // [r]
-  float *pe = sm + r;       // [256] exact-row probabilities of the current batch
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const float mx = jb.stats[2 * qh], inv = jb.stats[2 * qh + 1];
-  for (int l = threadIdx.x; l < r; l += blockDim.x) {
+  float *w = sm;                        // [qpk][r]
+  float *pe = w + (size_t)qpk * r;      // [qpk][AO_ROWS]
+  float *part = pe + qpk * AO_ROWS;     // [2][qpk][hd] partial outputs of the two thread halves
+  __shared__ float mass[8];
+  const int tid = threadIdx.x, f = tid % hd, half = tid / hd;  // blockDim = 2 hd
+  for (int e = tid; e < qpk * r; e += blockDim.x) {
+    const int g = e / r, l = e % r;
     float acc = 0.f;
     if (l < k) {
-      for (int c = 0; c < p.nchunk; ++c) acc += jb.wpart[((size_t)c * nq + qh) * r + l];
+      for (int c = 0; c < p.nchunk; ++c) acc += jb.wpart[((size_t)c * nq + q0 + g) * r + l];
       acc *= jb.sv[l];
     }
-    w[l] = acc;
+    w[e] = acc;
   }
-  float mass = 0.f;
-  if (threadIdx.x == 0)
-    for (int c = 0; c < p.nchunk; ++c) mass += jb.mpart[(size_t)c * nq + qh];
+  if (tid < qpk) {
+    float m = 0.f;
+    for (int c = 0; c < p.nchunk; ++c) m += jb.mpart[(size_t)c * nq + q0 + tid];
+    mass[tid] = m;
+  }
   __syncthreads();
-  // Compressed part: o[f] = sum_l B[h hd + f][l] w[l], one warp per output feature at a time.
-  const TS *B = static_cast<const TS *>(jb.Bv);
-  float *o = jb.out + (size_t)qh * hd;
-  float ofeat = 0.f;  // thread f < hd accumulates the exact part of feature f
-  for (int f = warp; f < hd; f += nw) {
-    float acc = 0.f;
-    for (int l = lane; l < k; l += 32) acc = fmaf(to_f<TS>(B[(size_t)(h * hd + f) * r + l]), w[l], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) o[f] = acc;
+  float acc[8];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) acc[g] = 0.f;
+  // Compressed part: feature f of the head, half of the coordinates per thread half.
+  const TS *B = static_cast<const TS *>(jb.Bv) + (size_t)(h * hd + f) * r;
+  const int lh = (k + 1) / 2, la = half * lh, lb = min(k, la + lh);
+#pragma unroll 8
+  for (int l = la; l < lb; ++l) {
+    const float b = to_f<TS>(B[l]);
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+      if (g < qpk) acc[g] = fmaf(b, w[g * r + l], acc[g]);
   }
-  // Exact values.
-  const TE *V = static_cast<const TE *>(jb.vex);
-  for (int64_t e0 = 0; e0 < jb.n_vex; e0 += blockDim.x) {
+  // Exact values, in staged batches of rows; the two halves take alternate rows.
+  const TE *V = static_cast<const TE *>(jb.vex) + h * hd + f;
+  const float *S = jb.S;
+  const int64_t nt = jb.n_total;
+  for (int64_t e0 = 0; e0 < jb.n_vex; e0 += AO_ROWS) {
+    const int ne = (int)min64(AO_ROWS, jb.n_vex - e0);
     __syncthreads();
-    const int64_t e = e0 + threadIdx.x;
-    float pv = 0.f;
-    if (e < jb.n_vex) {
-      const int64_t pos = jb.vexpos[e];
-      if (pos >= 0 && pos < jb.n_total)
-        pv = __expf(jb.S[(size_t)qh * jb.n_total + pos] - mx) * inv;
-      else
+    for (int e = tid; e < qpk * ne; e += blockDim.x) {
+      const int g = e / ne, i = e % ne;
+      const int64_t pos = jb.vexpos[e0 + i];
+      float pv = 0.f;
+      if (pos >= 0 && pos < nt)
+        pv = __expf(S[(size_t)(q0 + g) * nt + pos] - jb.stats[2 * (q0 + g)]) *
+             jb.stats[2 * (q0 + g) + 1];
+      else if (g == 0)
         record_status(jb.metav, ISKV_ERR_SHAPE);
+      pe[g * AO_ROWS + i] = pv;
     }
-    pe[threadIdx.x] = pv;
     __syncthreads();
-    const int ne = (int)min64(blockDim.x, jb.n_vex - e0);
-    if (threadIdx.x < hd)
-      for (int i = 0; i < ne; ++i)
-        ofeat = fmaf(pe[i], to_f<TE>(V[(size_t)(e0 + i) * p.d + h * hd + threadIdx.x]), ofeat);
-    if (threadIdx.x == 0)
-      for (int i = 0; i < ne; ++i) mass += pe[i];
+    if (tid < qpk) {
+      float m = 0.f;
+      for (int i = 0; i < ne; ++i) m += pe[tid * AO_ROWS + i];
+      mass[tid] += m;
+    }
+#pragma unroll 8
+    for (int i = half; i < ne; i += 2) {
+      const float v = to_f<TE>(V[(size_t)(e0 + i) * p.d]);
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        if (g < qpk) acc[g] = fmaf(pe[g * AO_ROWS + i], v, acc[g]);
+    }
   }
-  __syncthreads();  // the compressed part of o is written
-  if (threadIdx.x < hd) o[threadIdx.x] += ofeat;
-  if (threadIdx.x == 0 && !(fabsf(mass - 1.f) <= 1e-3f)) record_status(jb.metav, ISKV_ERR_SHAPE);
+#pragma unroll
+  for (int g = 0; g < 8; ++g)
+    if (g < qpk) part[(half * qpk + g) * hd + f] = acc[g];
+  __syncthreads();
+  for (int e = tid; e < qpk * hd; e += blockDim.x) {
+    const int g = e / hd, ff = e % hd;
+    jb.out[(size_t)(q0 + g) * hd + ff] = part[g * hd + ff] + part[(qpk + g) * hd + ff];
+  }
+  if (tid < qpk && !(fabsf(mass[tid] - 1.f) <= 1e-3f)) record_status(jb.metav, ISKV_ERR_SHAPE);
 }
 
 cudaError_t launch_attn_out(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (size_t)(p.r + 256);
+  const int qpk = p.n_q / p.n_kv;
+  if (qpk > 8) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(float) * ((size_t)qpk * p.r + (size_t)qpk * AO_ROWS +
+                                       2 * (size_t)qpk * p.head_dim);
   const bool sb = p.storage == ISKV_BF16, eb = p.exact_dtype == ISKV_BF16;
-  const dim3 g(p.n_q, p.count);
-  if (sb && eb) k_attn_out<__nv_bfloat16, __nv_bfloat16><<<g, 256, smem, s>>>(jobs, p);
-  else if (sb) k_attn_out<__nv_bfloat16, float><<<g, 256, smem, s>>>(jobs, p);
-  else if (eb) k_attn_out<float, __nv_bfloat16><<<g, 256, smem, s>>>(jobs, p);
-  else k_attn_out<float, float><<<g, 256, smem, s>>>(jobs, p);
+  const dim3 g(p.n_kv, p.count);
+  const int nth = 2 * p.head_dim;
+  cudaError_t e = cudaSuccess;
+  if (sb && eb) {
+    e = cudaFuncSetAttribute(k_attn_out<__nv_bfloat16, __nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) k_attn_out<__nv_bfloat16, __nv_bfloat16><<<g, nth, smem, s>>>(jobs, p);
+  } else if (sb) {
+    e = cudaFuncSetAttribute(k_attn_out<__nv_bfloat16, float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) k_attn_out<__nv_bfloat16, float><<<g, nth, smem, s>>>(jobs, p);
+  } else if (eb) {
+    e = cudaFuncSetAttribute(k_attn_out<float, __nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) k_attn_out<float, __nv_bfloat16><<<g, nth, smem, s>>>(jobs, p);
+  } else {
+    e = cudaFuncSetAttribute(k_attn_out<float, float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e == cudaSuccess) k_attn_out<float, float><<<g, nth, smem, s>>>(jobs, p);
+  }
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }

@@ -28,6 +28,7 @@ struct AttnJob {
   float *stats;              // workspace [n_q][2]: max score, sum of exp(score - max)
   float *wpart;              // workspace [nchunk][n_q][r]: partial sums of p * U_v rows
   float *mpart;              // workspace [nchunk][n_q]: partial probability mass on V rows
+  float *P;                  // workspace [n_q][n_cap]: probabilities at the compressed V rows
   void *bsig;                // workspace: sigma-scaled K basis (tensor-core scores)
   int64_t n_kex, n_vex, n_total;
 };
@@ -39,7 +40,7 @@ struct AttnParams {
   int64_t n_cap_max, n_total_max;
 };
 
-constexpr int ATTN_CHUNK = 512;  // V rows per value-mixing block
+constexpr int ATTN_CHUNK = 2048;  // V rows per value-mixing block
 constexpr int ATTN_MAX_Q = 64;   // query heads
 
 cudaError_t launch_attn_init(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
@@ -47,6 +48,7 @@ cudaError_t launch_attn_scores_ffma(const AttnJob *jobs, const AttnParams &p, cu
 cudaError_t launch_attn_scores_exact(const AttnJob *jobs, const AttnParams &p, int64_t max_kex,
                                      cudaStream_t s);
 cudaError_t launch_attn_stats(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
+cudaError_t launch_attn_probs(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
 cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
 cudaError_t launch_attn_out(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
 

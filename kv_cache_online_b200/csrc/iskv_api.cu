@@ -71,7 +71,7 @@ size_t jobs_bytes(int32_t count, size_t each) { return align_up((size_t)count * 
 namespace {
 
 struct AttnWsLayout {
-  size_t tc, recon, slices, bsig, S, stats, wpart, mpart, per_job, total;
+  size_t tc, recon, slices, bsig, S, stats, wpart, mpart, P, per_job, total;
   int nchunk;
 };
 
@@ -90,6 +90,7 @@ AttnWsLayout attn_ws_layout(int32_t count, int32_t d, int32_t r, int64_t n_cap, 
   L.stats = take((size_t)n_q * 2 * 4);
   L.wpart = take((size_t)L.nchunk * n_q * r * 4);
   L.mpart = take((size_t)L.nchunk * n_q * 4);
+  L.P = take((size_t)n_q * (size_t)n_cap * 4);
   L.per_job = o;
   L.total = L.slices + (size_t)count * L.per_job;
   return L;
@@ -483,8 +484,10 @@ iskv_status iskv_decode_attention_batched(
   if (!valid_dtype(exact_dtype)) return fail(ISKV_ERR_ARG, "%s: bad dtype", who);
   if (head_dim < 2 || head_dim % 2 || head_dim > 256)
     return fail(ISKV_ERR_SHAPE, "%s: need even head_dim <= 256", who);
-  if (n_kv_heads < 1 || n_q_heads < 1 || n_q_heads > ATTN_MAX_Q || n_q_heads % n_kv_heads)
-    return fail(ISKV_ERR_SHAPE, "%s: need n_q_heads a multiple of n_kv_heads, <= %d", who,
+  if (n_kv_heads < 1 || n_q_heads < 1 || n_q_heads > ATTN_MAX_Q || n_q_heads % n_kv_heads ||
+      n_q_heads / n_kv_heads > 8)
+    return fail(ISKV_ERR_SHAPE,
+                "%s: need n_q_heads a multiple of n_kv_heads, <= %d, at most 8 per KV head", who,
                 ATTN_MAX_Q);
   if (!(rope_theta > 0.0)) return fail(ISKV_ERR_ARG, "%s: rope_theta must be > 0", who);
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
@@ -554,6 +557,7 @@ iskv_status iskv_decode_attention_batched(
     j.stats = reinterpret_cast<float *>(slice + L.stats);
     j.wpart = reinterpret_cast<float *>(slice + L.wpart);
     j.mpart = reinterpret_cast<float *>(slice + L.mpart);
+    j.P = reinterpret_cast<float *>(slice + L.P);
     j.bsig = slice + L.bsig;
     j.n_kex = n_k_exact[i];
     j.n_vex = n_v_exact[i];
@@ -610,7 +614,8 @@ iskv_status iskv_decode_attention_batched(
   stage_mark(s, ST_ATTN_SCORES);
   if ((e = launch_attn_stats(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "attention: softmax");
   stage_mark(s, ST_ATTN_SOFTMAX);
-  e = launch_attn_values(djobs, p, s);
+  e = launch_attn_probs(djobs, p, s);
+  if (e == cudaSuccess) e = launch_attn_values(djobs, p, s);
   if (e == cudaSuccess) e = launch_attn_out(djobs, p, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention: values");
   stage_mark(s, ST_ATTN_VALUES);
