@@ -39,23 +39,31 @@ cudaError_t launch_attn_init(const AttnJob *jobs, const AttnParams &p, cudaStrea
   return cudaGetLastError();
 }
 
+// RoPE cosines and sines of position pos for the pairs j = lane + 32 t of this lane.
+template <int T>
+ISKV_DEV void key_angles(int64_t pos, int half, const double *invf, float (&c)[T], float (&s)[T]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const int j = lane + 32 * t;
+    c[t] = 1.f;
+    s[t] = 0.f;
+    if (j < half) rope_sincos(pos, invf[j], c[t], s[t]);
+  }
+}
+
 // Scale, rotate and dot one key of KV head h, held as pairs (lo = k[j], hi = k[j + hd/2]) for
 // j = lane + 32 t, with every query head of its group; lane 0 writes the scores.
 template <int T>
 ISKV_DEV void score_key(const AttnJob &jb, const AttnParams &p, int h, int64_t pos,
-                        const float (&lo)[T], const float (&hi)[T], const double *invf) {
+                        const float (&lo)[T], const float (&hi)[T], const float (&c)[T],
+                        const float (&s)[T]) {
   const int lane = threadIdx.x & 31, half = p.head_dim / 2, qpk = p.n_q / p.n_kv;
   float rl[T], rh[T];
 #pragma unroll
   for (int t = 0; t < T; ++t) {
-    const int j = lane + 32 * t;
-    rl[t] = rh[t] = 0.f;
-    if (j < half) {
-      float c, s;
-      rope_sincos(pos, invf[j], c, s);
-      rl[t] = lo[t] * c - hi[t] * s;
-      rh[t] = hi[t] * c + lo[t] * s;
-    }
+    rl[t] = lo[t] * c[t] - hi[t] * s[t];
+    rh[t] = hi[t] * c[t] + lo[t] * s[t];
   }
   for (int g = 0; g < qpk; ++g) {
     const int qh = h * qpk + g;
@@ -106,6 +114,8 @@ __global__ void __launch_bounds__(256) k_attn_scores_ffma(const AttnJob *jobs, A
       if (threadIdx.x == 0) record_status(jb.metak, ISKV_ERR_SHAPE);
       continue;
     }
+    float cs[4], sn[4];
+    key_angles<4>(pos, half, invf, cs, sn);
     for (int h = warp; h < p.n_kv; h += blockDim.x >> 5) {
       float lo[4], hi[4];
 #pragma unroll
@@ -114,7 +124,7 @@ __global__ void __launch_bounds__(256) k_attn_scores_ffma(const AttnJob *jobs, A
         lo[t] = j < half ? krow[h * hd + j] : 0.f;
         hi[t] = j < half ? krow[h * hd + j + half] : 0.f;
       }
-      score_key<4>(jb, p, h, pos, lo, hi, invf);
+      score_key<4>(jb, p, h, pos, lo, hi, cs, sn);
     }
   }
 }
@@ -148,6 +158,8 @@ __global__ void __launch_bounds__(256) k_attn_scores_exact(const AttnJob *jobs, 
     return;
   }
   const TE *x = static_cast<const TE *>(jb.kex) + (size_t)e * p.d;
+  float cs[4], sn[4];
+  key_angles<4>(pos, half, invf, cs, sn);  // the same angles for every head of the row
   for (int h = 0; h < p.n_kv; ++h) {
     float lo[4], hi[4];
 #pragma unroll
@@ -156,7 +168,7 @@ __global__ void __launch_bounds__(256) k_attn_scores_exact(const AttnJob *jobs, 
       lo[t] = j < half ? to_f<TE>(x[h * hd + j]) : 0.f;
       hi[t] = j < half ? to_f<TE>(x[h * hd + j + half]) : 0.f;
     }
-    score_key<4>(jb, p, h, pos, lo, hi, invf);
+    score_key<4>(jb, p, h, pos, lo, hi, cs, sn);
   }
 }
 
@@ -292,7 +304,7 @@ cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStr
 constexpr int AO_ROWS = 512;  // exact rows per staged batch
 
 template <typename TS, typename TE>
-__global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParams p) {
+__global__ void __launch_bounds__(1024) k_attn_out(const AttnJob *jobs, AttnParams p) {
   const AttnJob &jb = jobs[blockIdx.y];
   const int h = blockIdx.x, nq = p.n_q, r = p.r, hd = p.head_dim;
   const int qpk = nq / p.n_kv, q0 = h * qpk;
@@ -300,9 +312,10 @@ __global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParam
   extern __shared__ float sm[];
   float *w = sm;                        // [qpk][r]
   float *pe = w + (size_t)qpk * r;      // [qpk][AO_ROWS]
-  float *part = pe + qpk * AO_ROWS;     // [2][qpk][hd] partial outputs of the two thread halves
+  float *part = pe + qpk * AO_ROWS;     // [NS][qpk][hd] partial outputs of the thread groups
   __shared__ float mass[8];
-  const int tid = threadIdx.x, f = tid % hd, half = tid / hd;  // blockDim = 2 hd
+  const int tid = threadIdx.x, f = tid % hd, half = tid / hd;  // blockDim = NS hd
+  const int NS = blockDim.x / hd;  // thread groups splitting the coordinates and the rows
   for (int e = tid; e < qpk * r; e += blockDim.x) {
     const int g = e / r, l = e % r;
     float acc = 0.f;
@@ -321,9 +334,9 @@ __global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParam
   float acc[8];
 #pragma unroll
   for (int g = 0; g < 8; ++g) acc[g] = 0.f;
-  // Compressed part: feature f of the head, half of the coordinates per thread half.
+  // Compressed part: feature f of the head, a slice of the coordinates per thread group.
   const TS *B = static_cast<const TS *>(jb.Bv) + (size_t)(h * hd + f) * r;
-  const int lh = (k + 1) / 2, la = half * lh, lb = min(k, la + lh);
+  const int lh = (k + NS - 1) / NS, la = half * lh, lb = min(k, la + lh);
 #pragma unroll 8
   for (int l = la; l < lb; ++l) {
     const float b = to_f<TS>(B[l]);
@@ -331,7 +344,7 @@ __global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParam
     for (int g = 0; g < 8; ++g)
       if (g < qpk) acc[g] = fmaf(b, w[g * r + l], acc[g]);
   }
-  // Exact values, in staged batches of rows; the two halves take alternate rows.
+  // Exact values, in staged batches of rows; the thread groups take rows in turn.
   const TE *V = static_cast<const TE *>(jb.vex) + h * hd + f;
   const float *S = jb.S;
   const int64_t nt = jb.n_total;
@@ -355,8 +368,8 @@ __global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParam
       for (int i = 0; i < ne; ++i) m += pe[tid * AO_ROWS + i];
       mass[tid] += m;
     }
-#pragma unroll 8
-    for (int i = half; i < ne; i += 2) {
+#pragma unroll 4
+    for (int i = half; i < ne; i += NS) {
       const float v = to_f<TE>(V[(size_t)(e0 + i) * p.d]);
 #pragma unroll
       for (int g = 0; g < 8; ++g)
@@ -369,7 +382,9 @@ __global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParam
   __syncthreads();
   for (int e = tid; e < qpk * hd; e += blockDim.x) {
     const int g = e / hd, ff = e % hd;
-    jb.out[(size_t)(q0 + g) * hd + ff] = part[g * hd + ff] + part[(qpk + g) * hd + ff];
+    float o = 0.f;
+    for (int t = 0; t < NS; ++t) o += part[(t * qpk + g) * hd + ff];
+    jb.out[(size_t)(q0 + g) * hd + ff] = o;
   }
   if (tid < qpk && !(fabsf(mass[tid] - 1.f) <= 1e-3f)) record_status(jb.metav, ISKV_ERR_SHAPE);
 }
@@ -377,11 +392,12 @@ __global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParam
 cudaError_t launch_attn_out(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
   const int qpk = p.n_q / p.n_kv;
   if (qpk > 8) return cudaErrorInvalidValue;
+  const int ns = 2;  // thread groups splitting the coordinates and the exact rows
   const size_t smem = sizeof(float) * ((size_t)qpk * p.r + (size_t)qpk * AO_ROWS +
-                                       2 * (size_t)qpk * p.head_dim);
+                                       (size_t)ns * qpk * p.head_dim);
   const bool sb = p.storage == ISKV_BF16, eb = p.exact_dtype == ISKV_BF16;
   const dim3 g(p.n_kv, p.count);
-  const int nth = 2 * p.head_dim;
+  const int nth = ns * p.head_dim;
   cudaError_t e = cudaSuccess;
   if (sb && eb) {
     e = cudaFuncSetAttribute(k_attn_out<__nv_bfloat16, __nv_bfloat16>,
