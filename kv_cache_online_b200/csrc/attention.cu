@@ -228,23 +228,56 @@ cudaError_t launch_attn_stats(const AttnJob *jobs, const AttnParams &p, cudaStre
 }
 
 // ------------------------------------------------------------------------------------------------
-// Probabilities at the compressed value rows, P[j][i] = P_j(pos_v[i]), laid out densely by row so
-// that the value-mixing GEMM streams them (0 for a row outside the cache, which is flagged).
+// Probabilities at the compressed value rows, P_j(pos_v[i]), laid out densely by row so that the
+// value mixing streams them: float32 [n_q][n_cap] for the CUDA-core GEMM, or bf16 [n_cap][64]
+// (queries padded to 64 columns) for the tensor cores. Rows past the history, and rows outside
+// the cache (flagged), get 0. Each block also sums its rows' probabilities per query head.
 __global__ void __launch_bounds__(256) k_attn_probs(const AttnJob *jobs, AttnParams p) {
   const AttnJob &jb = jobs[blockIdx.y];
-  const int64_t n = jb.metav[ISKV_META_N];
+  const int64_t n = jb.metav[ISKV_META_N], nt = jb.n_total;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const int64_t pos = jb.posv[i], nt = jb.n_total;
-  const bool ok = pos >= 0 && pos < nt;
-  if (!ok) record_status(jb.metav, ISKV_ERR_SHAPE);
-  for (int j = 0; j < p.n_q; ++j)
-    jb.P[(size_t)j * p.n_cap_max + i] =
-        ok ? __expf(jb.S[(size_t)j * nt + pos] - jb.stats[2 * j]) * jb.stats[2 * j + 1] : 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float red[8][ATTN_MAX_Q];
+  bool ok = false;
+  int64_t pos = 0;
+  if (i < n) {
+    pos = jb.posv[i];
+    ok = pos >= 0 && pos < nt;
+    if (!ok) record_status(jb.metav, ISKV_ERR_SHAPE);
+  }
+  __nv_bfloat16 *pb = static_cast<__nv_bfloat16 *>(jb.Pb) + (size_t)i * 64;
+  for (int j0 = 0; j0 < 64; j0 += 2) {
+    float v[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = j0 + u;
+      v[u] = (ok && j < p.n_q)
+                 ? __expf(jb.S[(size_t)j * nt + pos] - jb.stats[2 * j]) * jb.stats[2 * j + 1]
+                 : 0.f;
+      if (j < p.n_q) {
+        const float m = warp_sum(v[u]);
+        if (lane == 0) red[warp][j] = m;
+      }
+    }
+    if (i < p.n_cap_max) {
+      if (p.tc_values)
+        *reinterpret_cast<__nv_bfloat162 *>(pb + j0) = __floats2bfloat162_rn(v[0], v[1]);
+      else
+        for (int u = 0; u < 2; ++u)
+          if (j0 + u < p.n_q) jb.P[(size_t)(j0 + u) * p.n_cap_max + i] = v[u];
+    }
+    if (j0 + 2 >= p.n_q && !p.tc_values) break;
+  }
+  __syncthreads();
+  if (threadIdx.x < p.n_q) {
+    float m = 0.f;
+    for (int w = 0; w < 8; ++w) m += red[w][threadIdx.x];
+    jb.mpart[(size_t)blockIdx.x * p.n_q + threadIdx.x] = m;
+  }
 }
 
 cudaError_t launch_attn_probs(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
-  const unsigned gx = (unsigned)((p.n_cap_max + 255) / 256);
+  const unsigned gx = (unsigned)p.nblk;
   if (gx == 0) return cudaSuccess;
   k_attn_probs<<<dim3(gx, p.count), 256, 0, s>>>(jobs, p);
   count_launches(1);
@@ -252,9 +285,8 @@ cudaError_t launch_attn_probs(const AttnJob *jobs, const AttnParams &p, cudaStre
 }
 
 // ------------------------------------------------------------------------------------------------
-// Compressed values, mixed in coordinate space: W_c = P_c^T [U_v | 1] over the ATTN_CHUNK rows of
-// chunk c -- a register-tiled GEMM (M = query heads, N = r + 1, K = rows). The appended column of
-// ones yields the probability mass the chunk's value rows carry.
+// Compressed values, mixed in coordinate space on CUDA cores: W_c = P_c^T U_v over the ATTN_CHUNK
+// rows of chunk c -- a register-tiled GEMM (M = query heads, N = r, K = rows).
 constexpr int AV_BM = 32, AV_BN = 64, AV_BK = 16, AV_TM = 4, AV_TN = 4;
 constexpr int AV_THREADS = (AV_BM / AV_TM) * (AV_BN / AV_TN);
 
@@ -272,22 +304,16 @@ __global__ void __launch_bounds__(AV_THREADS) k_attn_values(const AttnJob *jobs,
   const float *P = jb.P + i0;
   const size_t ldp = (size_t)p.n_cap_max;
   float *wp = jb.wpart + (size_t)c * nq * r;
-  float *mp = jb.mpart + (size_t)c * nq;
   tile_gemm<AV_BM, AV_BN, AV_BK, AV_TM, AV_TN, true, true>(
-      m0, n0, nq, r + 1, rows,
+      m0, n0, nq, r, rows,
       [&](int j, int i) { return P[(size_t)j * ldp + i]; },
-      [&](int i, int l) {
-        return l < k ? to_f<TS>(U[(size_t)(i0 + i) * r + l]) : (l == r ? 1.f : 0.f);
-      },
-      [&](int j, int l, float acc) {
-        if (l < r) wp[(size_t)j * r + l] = acc;
-        else mp[j] = acc;
-      });
+      [&](int i, int l) { return l < k ? to_f<TS>(U[(size_t)(i0 + i) * r + l]) : 0.f; },
+      [&](int j, int l, float acc) { wp[(size_t)j * r + l] = acc; });
 }
 
 cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
   const int mt = (p.n_q + AV_BM - 1) / AV_BM;
-  const dim3 g((p.r + 1 + AV_BN - 1) / AV_BN, mt * p.nchunk, p.count);
+  const dim3 g((p.r + AV_BN - 1) / AV_BN, mt * p.nchunk, p.count);
   if (p.storage == ISKV_BF16)
     k_attn_values<__nv_bfloat16><<<g, AV_THREADS, 0, s>>>(jobs, p);
   else
@@ -320,14 +346,16 @@ __global__ void __launch_bounds__(1024) k_attn_out(const AttnJob *jobs, AttnPara
     const int g = e / r, l = e % r;
     float acc = 0.f;
     if (l < k) {
-      for (int c = 0; c < p.nchunk; ++c) acc += jb.wpart[((size_t)c * nq + q0 + g) * r + l];
+      for (int c = 0; c < p.nchunk; ++c)
+        acc += p.tc_values ? jb.wpart[((size_t)c * r + l) * 64 + q0 + g]
+                           : jb.wpart[((size_t)c * nq + q0 + g) * r + l];
       acc *= jb.sv[l];
     }
     w[e] = acc;
   }
   if (tid < qpk) {
     float m = 0.f;
-    for (int c = 0; c < p.nchunk; ++c) m += jb.mpart[(size_t)c * nq + q0 + tid];
+    for (int c = 0; c < p.nblk; ++c) m += jb.mpart[(size_t)c * nq + q0 + tid];
     mass[tid] = m;
   }
   __syncthreads();

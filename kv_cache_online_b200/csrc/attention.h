@@ -29,12 +29,15 @@ struct AttnJob {
   float *wpart;              // workspace [nchunk][n_q][r]: partial sums of p * U_v rows
   float *mpart;              // workspace [nchunk][n_q]: partial probability mass on V rows
   float *P;                  // workspace [n_q][n_cap]: probabilities at the compressed V rows
+  void *Pb;                  // the same workspace as bf16 [n_cap][64] (tensor-core value mixing)
   void *bsig;                // workspace: sigma-scaled K basis (tensor-core scores)
   int64_t n_kex, n_vex, n_total;
 };
 
 struct AttnParams {
   int d, r, storage, exact_dtype, n_kv, n_q, head_dim, count, nchunk;
+  int nblk;        // probability-mass partials: blocks of 256 value rows
+  int tc_values;   // value mixing on the tensor cores (partials [chunk][r][64])
   double theta;
   float scale;
   int64_t n_cap_max, n_total_max;

@@ -71,8 +71,8 @@ size_t jobs_bytes(int32_t count, size_t each) { return align_up((size_t)count * 
 namespace {
 
 struct AttnWsLayout {
-  size_t tc, recon, slices, bsig, S, stats, wpart, mpart, P, per_job, total;
-  int nchunk;
+  size_t tc, tcpv, recon, slices, bsig, S, stats, wpart, mpart, P, per_job, total;
+  int nchunk, nblk;
 };
 
 AttnWsLayout attn_ws_layout(int32_t count, int32_t d, int32_t r, int64_t n_cap, int64_t n_total_max,
@@ -80,17 +80,22 @@ AttnWsLayout attn_ws_layout(int32_t count, int32_t d, int32_t r, int64_t n_cap, 
   AttnWsLayout L;
   L.nchunk = (int)((n_cap + ATTN_CHUNK - 1) / ATTN_CHUNK);
   if (L.nchunk < 1) L.nchunk = 1;
+  L.nblk = (int)((n_cap + 255) / 256);
+  if (L.nblk < 1) L.nblk = 1;
   L.tc = jobs_bytes(count, sizeof(AttnJob));
-  L.recon = L.tc + tc_table_bytes(count);
+  L.tcpv = L.tc + tc_table_bytes(count);
+  L.recon = L.tcpv + tc_table_bytes(count);
   L.slices = L.recon + jobs_bytes(count, sizeof(ReconJob));
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
   L.bsig = take((size_t)d * r * 2);
   L.S = take((size_t)n_q * (size_t)n_total_max * 4);
   L.stats = take((size_t)n_q * 2 * 4);
-  L.wpart = take((size_t)L.nchunk * n_q * r * 4);
-  L.mpart = take((size_t)L.nchunk * n_q * 4);
-  L.P = take((size_t)n_q * (size_t)n_cap * 4);
+  // Value-mixing partials and probabilities: the CUDA-core layouts ([chunk][n_q][r] and
+  // [n_q][n_cap] float32) or the tensor-core ones ([chunk][r][64] float32, [n_cap][64] bf16).
+  L.wpart = take((size_t)L.nchunk * r * (n_q > 64 ? n_q : 64) * 4);
+  L.mpart = take((size_t)L.nblk * n_q * 4);
+  L.P = take((size_t)(L.nblk * 256) * (4 * n_q > 128 ? 4 * n_q : 128));
   L.per_job = o;
   L.total = L.slices + (size_t)count * L.per_job;
   return L;
@@ -528,6 +533,8 @@ iskv_status iskv_decode_attention_batched(
   p.head_dim = head_dim;
   p.count = count;
   p.nchunk = L.nchunk;
+  p.nblk = L.nblk;
+  p.tc_values = tc_pv_supported(r, p.storage, n_q_heads) ? 1 : 0;
   p.theta = rope_theta;
   p.scale = scale;
   p.n_cap_max = ncap;
@@ -558,6 +565,7 @@ iskv_status iskv_decode_attention_batched(
     j.wpart = reinterpret_cast<float *>(slice + L.wpart);
     j.mpart = reinterpret_cast<float *>(slice + L.mpart);
     j.P = reinterpret_cast<float *>(slice + L.P);
+    j.Pb = slice + L.P;
     j.bsig = slice + L.bsig;
     j.n_kex = n_k_exact[i];
     j.n_vex = n_v_exact[i];
@@ -594,14 +602,23 @@ iskv_status iskv_decode_attention_batched(
     rp.theta = rope_theta;
     rp.n_cap_max = ncap;
   }
+  std::vector<TcJob> pj;
+  if (p.tc_values) {
+    pj.resize(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_pv_job(pj[i], hv[i].U, ncap, r, jobs[i].Pb, jobs[i].wpart, hv[i].meta))
+        return fail(ISKV_ERR_CUDA, "%s: tensor map encoding failed", who);
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   AttnJob *djobs = reinterpret_cast<AttnJob *>(base);
+  TcJob *pv_dev = reinterpret_cast<TcJob *>(base + L.tcpv);
   TcJob *tc_dev = reinterpret_cast<TcJob *>(base + L.tc);
   ReconJob *recon_dev = reinterpret_cast<ReconJob *>(base + L.recon);
   stage_begin(s);
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(AttnJob) * count, s);
   if (e == cudaSuccess && tc) e = upload_jobs(tc_dev, tj.data(), sizeof(TcJob) * count, s);
   if (e == cudaSuccess && tc) e = upload_jobs(recon_dev, rj.data(), sizeof(ReconJob) * count, s);
+  if (e == cudaSuccess && p.tc_values) e = upload_jobs(pv_dev, pj.data(), sizeof(TcJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention: upload");
   stage_mark(s, ST_UPLOAD);
   if ((e = launch_attn_init(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "attention: init");
@@ -615,7 +632,17 @@ iskv_status iskv_decode_attention_batched(
   if ((e = launch_attn_stats(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "attention: softmax");
   stage_mark(s, ST_ATTN_SOFTMAX);
   e = launch_attn_probs(djobs, p, s);
-  if (e == cudaSuccess) e = launch_attn_values(djobs, p, s);
+  if (e == cudaSuccess) {
+    if (p.tc_values) {
+      PvParams pv;
+      pv.r = r;
+      pv.count = count;
+      pv.nsplit = L.nchunk;
+      e = launch_tc_pv(pv_dev, pv, s);
+    } else {
+      e = launch_attn_values(djobs, p, s);
+    }
+  }
   if (e == cudaSuccess) e = launch_attn_out(djobs, p, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention: values");
   stage_mark(s, ST_ATTN_VALUES);

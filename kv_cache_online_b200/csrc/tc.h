@@ -72,6 +72,15 @@ bool encode_attn_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void 
                      float scale);
 cudaError_t launch_tc_attn_scores(const TcJob *djobs, const AttnParams &p, cudaStream_t s);
 
+// Decode-attention value mixing: per split of ATTN_CHUNK rows, U^T P -> [split][r][64] float32.
+struct PvParams {
+  int r, count, nsplit;
+};
+bool tc_pv_supported(int r, int storage, int n_q);
+bool encode_pv_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void *Pb, float *wpart,
+                   int64_t *meta);
+cudaError_t launch_tc_pv(const TcJob *djobs, const PvParams &p, cudaStream_t s);
+
 // One CTA waiting on a barrier nothing arrives at, bounded by limit_ns (failure-path self-test).
 cudaError_t launch_wait_timeout(int64_t *meta, uint64_t limit_ns, cudaStream_t s);
 

@@ -1035,6 +1035,141 @@ bool tc_gram_supported(int r, int storage) {
   return storage == ISKV_BF16 && (r == 128 || r == 256) && encode_fn() != nullptr;
 }
 
+// ================================================================================================
+// Decode-attention value mixing on the tensor cores: for each split of ATTN_CHUNK value rows,
+// D = U_split^T P_split (r x 64), the coordinates of the history rows weighted by the query
+// heads' probabilities (P: [n_cap][64] bf16, queries padded to 64 columns). The structure is the
+// Gram kernel's: both operands MN-major, 64-row stages of r/64 U slabs plus one P slab, two
+// M = 128 halves, N = 64; the epilogue writes the float32 partial [split][r][64].
+__global__ void __launch_bounds__(GRAM_THREADS, 1) k_pv_tc(const TcJob *jobs, PvParams p) {
+  const int job = blockIdx.x / p.nsplit, split = blockIdx.x % p.nsplit;
+  const TcJob &jb = jobs[job];
+  const int R = p.r, SL = R / 64, MH = R / 128, N = 64;
+  const int64_t n = jb.meta[ISKV_META_N];
+  const int r0 = split * ATTN_CHUNK;
+  const int nrows = (int)(n - r0 < ATTN_CHUNK ? n - r0 : ATTN_CHUNK);
+  float *out = reinterpret_cast<float *>(jb.out) + (size_t)split * R * N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (nrows <= 0) {  // an empty split contributes zeros (uniform over the CTA)
+    for (int e = threadIdx.x; e < R * N; e += blockDim.x) out[e] = 0.f;
+    return;
+  }
+  const int nk = (nrows + GRAM_KT - 1) / GRAM_KT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int SLAB = GRAM_KT * 128;  // 64 rows x 64 columns bf16
+  const int STAGE_BYTES = (SL + 1) * SLAB;
+  TcCtl *ctl = reinterpret_cast<TcCtl *>(smem + GRAM_STAGES * STAGE_BYTES);
+  uint64_t *full = reinterpret_cast<uint64_t *>(ctl + 1);   // [GRAM_STAGES]
+  uint64_t *empty = full + GRAM_STAGES;                      // [GRAM_STAGES]
+  const uint32_t ncols = MH * N <= 128 ? 128 : 256;
+  const uint32_t idesc = idesc_bf16_f32_mn(128, N);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < GRAM_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(&ctl->acc_full[0], 1);
+    mbar_init(&ctl->done, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&ctl->tmem, ncols);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int *abort = &ctl->abort;
+
+  if (warp == 0 && lane == 0) {
+    tensormap_acquire(&jb.mapA);
+    tensormap_acquire(&jb.mapB);
+    for (int kt = 0; kt < nk && !*abort; ++kt) {
+      const int st = kt % GRAM_STAGES, use = kt / GRAM_STAGES;
+      if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, abort, WAIT_NS)) {
+        fail_timeout(ctl, jb.meta);
+        break;
+      }
+      mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
+      uint8_t *stage = smem + st * STAGE_BYTES;
+      for (int sl = 0; sl < SL; ++sl)
+        tma_load_2d(stage + sl * SLAB, &jb.mapA, sl * 64, r0 + kt * GRAM_KT, &full[st]);
+      tma_load_2d(stage + SL * SLAB, &jb.mapB, 0, r0 + kt * GRAM_KT, &full[st]);
+    }
+    for (int k = 1; k <= GRAM_STAGES && nk - k >= 0; ++k)
+      mbar_wait(&full[(nk - k) % GRAM_STAGES], ((nk - k) / GRAM_STAGES) & 1, abort, WAIT_NS / 4);
+  } else if (warp == 1 && lane == 0) {
+    bool ok = true;
+    for (int kt = 0; kt < nk && ok && !*abort; ++kt) {
+      const int st = kt % GRAM_STAGES, use = kt / GRAM_STAGES;
+      if (!mbar_wait(&full[st], use & 1, abort, WAIT_NS)) { ok = false; break; }
+      fence_after_sync();
+      const uint32_t base = smem_u32(smem + st * STAGE_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < GRAM_KT / 16; ++kk) {
+        const uint64_t bdesc = sw128_mn_desc(base + SL * SLAB + kk * 2048, SLAB);
+        for (int h = 0; h < MH; ++h) {
+          const uint64_t adesc = sw128_mn_desc(base + h * 2 * SLAB + kk * 2048, SLAB);
+          mma_bf16(tmem + h * N, adesc, bdesc, idesc, (kt | kk) != 0);
+        }
+      }
+      mma_commit(&empty[st]);
+    }
+    if (!ok) fail_timeout(ctl, jb.meta);
+    mma_commit(&ctl->acc_full[0]);
+    mma_commit(&ctl->done);
+    mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
+  } else if (warp >= 2) {
+    const int q = warp & 3;
+    if (__all_sync(~0u, mbar_wait(&ctl->acc_full[0], 0, abort, WAIT_NS) && !*abort)) {
+      fence_after_sync();
+      for (int h = 0; h < MH; ++h) {
+        const int row = h * 128 + q * 32 + lane;
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + h * N + ((uint32_t)(q * 32) << 16) + c0, v);
+          tmem_ld_wait();
+          float4 *dst = reinterpret_cast<float4 *>(out + (size_t)row * N + c0);
+          dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+          dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+          dst[2] = make_float4(v[8], v[9], v[10], v[11]);
+          dst[3] = make_float4(v[12], v[13], v[14], v[15]);
+        }
+      }
+    } else {
+      fail_timeout(ctl, jb.meta);
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+bool tc_pv_supported(int r, int storage, int n_q) {
+  return storage == ISKV_BF16 && r % 128 == 0 && r >= 128 && r <= 256 && n_q <= 64 &&
+         encode_fn() != nullptr;
+}
+
+bool encode_pv_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void *Pb, float *wpart,
+                   int64_t *meta) {
+  std::memset(&tj, 0, sizeof(tj));
+  if (!encode_2d(&tj.mapA, U, (uint64_t)n_cap, (uint64_t)r, GRAM_KT)) return false;
+  if (!encode_2d(&tj.mapB, Pb, (uint64_t)n_cap, 64, GRAM_KT)) return false;
+  tj.meta = meta;
+  tj.out = wpart;
+  return true;
+}
+
+cudaError_t launch_tc_pv(const TcJob *djobs, const PvParams &p, cudaStream_t s) {
+  const size_t smem = 1024 + (size_t)GRAM_STAGES * (p.r / 64 + 1) * GRAM_KT * 128 + sizeof(TcCtl) +
+                      2 * GRAM_STAGES * sizeof(uint64_t);
+  cudaError_t e = cudaFuncSetAttribute(k_pv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  k_pv_tc<<<p.count * p.nsplit, GRAM_THREADS, smem, s>>>(djobs, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 bool encode_gram_job(TcJob &tj, const void *U, int64_t n_cap, const void *B, int d, int r,
                      const int32_t *sc, int64_t *meta, void *ws) {
   std::memset(&tj, 0, sizeof(tj));
