@@ -235,38 +235,48 @@ cudaError_t launch_attn_stats(const AttnJob *jobs, const AttnParams &p, cudaStre
 __global__ void __launch_bounds__(256) k_attn_probs(const AttnJob *jobs, AttnParams p) {
   const AttnJob &jb = jobs[blockIdx.y];
   const int64_t n = jb.metav[ISKV_META_N], nt = jb.n_total;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int jend = p.tc_values ? 64 : p.n_q;  // columns written per row
   __shared__ float red[8][ATTN_MAX_Q];
-  bool ok = false;
-  int64_t pos = 0;
-  if (i < n) {
-    pos = jb.posv[i];
-    ok = pos >= 0 && pos < nt;
-    if (!ok) record_status(jb.metav, ISKV_ERR_SHAPE);
-  }
-  __nv_bfloat16 *pb = static_cast<__nv_bfloat16 *>(jb.Pb) + (size_t)i * 64;
-  for (int j0 = 0; j0 < 64; j0 += 2) {
-    float v[2];
+  float mass[ATTN_MAX_Q];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int j = j0 + u;
-      v[u] = (ok && j < p.n_q)
-                 ? __expf(jb.S[(size_t)j * nt + pos] - jb.stats[2 * j]) * jb.stats[2 * j + 1]
-                 : 0.f;
-      if (j < p.n_q) {
-        const float m = warp_sum(v[u]);
-        if (lane == 0) red[warp][j] = m;
-      }
+  for (int j = 0; j < ATTN_MAX_Q; ++j) mass[j] = 0.f;
+  for (int u = 0; u < ATTN_PROB_ROWS; ++u) {
+    // Rows of this block, strided by the block so that a warp's accesses stay contiguous.
+    const int64_t i = ((int64_t)blockIdx.x * ATTN_PROB_ROWS + u) * blockDim.x + threadIdx.x;
+    if (i >= p.n_cap_max) break;
+    bool ok = false;
+    int64_t pos = 0;
+    if (i < n) {
+      pos = jb.posv[i];
+      ok = pos >= 0 && pos < nt;
+      if (!ok) record_status(jb.metav, ISKV_ERR_SHAPE);
     }
-    if (i < p.n_cap_max) {
+    __nv_bfloat16 *pb = static_cast<__nv_bfloat16 *>(jb.Pb) + (size_t)i * 64;
+#pragma unroll
+    for (int j0 = 0; j0 < ATTN_MAX_Q; j0 += 2) {
+      if (j0 >= jend) break;
+      float v[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int j = j0 + t;
+        v[t] = (ok && j < p.n_q)
+                   ? __expf(jb.S[(size_t)j * nt + pos] - jb.stats[2 * j]) * jb.stats[2 * j + 1]
+                   : 0.f;
+        mass[j] += v[t];
+      }
       if (p.tc_values)
         *reinterpret_cast<__nv_bfloat162 *>(pb + j0) = __floats2bfloat162_rn(v[0], v[1]);
       else
-        for (int u = 0; u < 2; ++u)
-          if (j0 + u < p.n_q) jb.P[(size_t)(j0 + u) * p.n_cap_max + i] = v[u];
+        for (int t = 0; t < 2; ++t)
+          if (j0 + t < p.n_q) jb.P[(size_t)(j0 + t) * p.n_cap_max + i] = v[t];
     }
-    if (j0 + 2 >= p.n_q && !p.tc_values) break;
+  }
+#pragma unroll
+  for (int j = 0; j < ATTN_MAX_Q; ++j) {
+    if (j >= p.n_q) break;
+    const float m = warp_sum(mass[j]);
+    if (lane == 0) red[warp][j] = m;
   }
   __syncthreads();
   if (threadIdx.x < p.n_q) {
@@ -323,61 +333,65 @@ cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStr
 }
 
 // ------------------------------------------------------------------------------------------------
-// Outputs of the query group of one KV head h: o_j = B_v,h (sigma_v * sum_c wpart[c][j]) +
-// sum_e P_j(pos_e) v_e[h], and the probability-mass check. One block per (KV head, job): the
-// group's coordinate vectors and exact-row probabilities sit in shared memory, each value row of
-// the head is read once for the whole group, and the row loops keep several loads in flight.
+// Outputs of the query group of one KV head h, in AO_SPLIT parts per (head, job): part s takes
+// a slice of the coordinates, o_j += B_v,h[:, slice] (sigma_v * sum_c wpart[c][j])[slice], and a
+// slice of the exact rows, o_j += sum_e P_j(pos_e) v_e[h], and writes its partial outputs and
+// probability mass; k_attn_final adds the parts in order and checks the mass. Each value row of
+// the head is read once for the whole query group.
 constexpr int AO_ROWS = 512;  // exact rows per staged batch
 
 template <typename TS, typename TE>
-__global__ void __launch_bounds__(1024) k_attn_out(const AttnJob *jobs, AttnParams p) {
+__global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParams p) {
   const AttnJob &jb = jobs[blockIdx.y];
-  const int h = blockIdx.x, nq = p.n_q, r = p.r, hd = p.head_dim;
+  const int h = blockIdx.x, part_id = blockIdx.z, nq = p.n_q, r = p.r, hd = p.head_dim;
   const int qpk = nq / p.n_kv, q0 = h * qpk;
   const int k = (int)jb.metav[ISKV_META_K];
   extern __shared__ float sm[];
-  float *w = sm;                        // [qpk][r]
+  float *w = sm;                        // [qpk][lslice]
   float *pe = w + (size_t)qpk * r;      // [qpk][AO_ROWS]
   float *part = pe + qpk * AO_ROWS;     // [NS][qpk][hd] partial outputs of the thread groups
   __shared__ float mass[8];
-  const int tid = threadIdx.x, f = tid % hd, half = tid / hd;  // blockDim = NS hd
-  const int NS = blockDim.x / hd;  // thread groups splitting the coordinates and the rows
-  for (int e = tid; e < qpk * r; e += blockDim.x) {
-    const int g = e / r, l = e % r;
+  const int tid = threadIdx.x, f = tid % hd, grp = tid / hd;
+  const int NS = blockDim.x / hd;
+  // This part's coordinates [la, lb) and exact rows [ea, eb).
+  const int lsz = (k + AO_SPLIT - 1) / AO_SPLIT, la = min(k, part_id * lsz), lb = min(k, la + lsz);
+  const int64_t esz = (jb.n_vex + AO_SPLIT - 1) / AO_SPLIT;
+  const int64_t ea = min64(jb.n_vex, part_id * esz), eb = min64(jb.n_vex, ea + esz);
+  const int nl = lb - la;
+  for (int e = tid; e < qpk * nl; e += blockDim.x) {
+    const int g = p.tc_values ? e % qpk : e / nl, li = p.tc_values ? e / qpk : e % nl;
+    const int l = la + li;
     float acc = 0.f;
-    if (l < k) {
-      for (int c = 0; c < p.nchunk; ++c)
-        acc += p.tc_values ? jb.wpart[((size_t)c * r + l) * 64 + q0 + g]
-                           : jb.wpart[((size_t)c * nq + q0 + g) * r + l];
-      acc *= jb.sv[l];
-    }
-    w[e] = acc;
+    for (int c = 0; c < p.nchunk; ++c)
+      acc += p.tc_values ? jb.wpart[((size_t)c * r + l) * 64 + q0 + g]
+                         : jb.wpart[((size_t)c * nq + q0 + g) * r + l];
+    w[g * r + li] = acc * jb.sv[l];
   }
   if (tid < qpk) {
     float m = 0.f;
-    for (int c = 0; c < p.nblk; ++c) m += jb.mpart[(size_t)c * nq + q0 + tid];
+    if (part_id == 0)
+      for (int c = 0; c < p.nblk; ++c) m += jb.mpart[(size_t)c * nq + q0 + tid];
     mass[tid] = m;
   }
   __syncthreads();
   float acc[8];
 #pragma unroll
   for (int g = 0; g < 8; ++g) acc[g] = 0.f;
-  // Compressed part: feature f of the head, a slice of the coordinates per thread group.
-  const TS *B = static_cast<const TS *>(jb.Bv) + (size_t)(h * hd + f) * r;
-  const int lh = (k + NS - 1) / NS, la = half * lh, lb = min(k, la + lh);
-#pragma unroll 8
-  for (int l = la; l < lb; ++l) {
-    const float b = to_f<TS>(B[l]);
+  // Compressed part: feature f of the head over this part's coordinates, split by thread group.
+  const TS *B = static_cast<const TS *>(jb.Bv) + (size_t)(h * hd + f) * r + la;
+#pragma unroll 4
+  for (int li = grp; li < nl; li += NS) {
+    const float b = to_f<TS>(B[li]);
 #pragma unroll
     for (int g = 0; g < 8; ++g)
-      if (g < qpk) acc[g] = fmaf(b, w[g * r + l], acc[g]);
+      if (g < qpk) acc[g] = fmaf(b, w[g * r + li], acc[g]);
   }
-  // Exact values, in staged batches of rows; the thread groups take rows in turn.
+  // Exact values of this part, in staged batches; the thread groups take rows in turn.
   const TE *V = static_cast<const TE *>(jb.vex) + h * hd + f;
   const float *S = jb.S;
   const int64_t nt = jb.n_total;
-  for (int64_t e0 = 0; e0 < jb.n_vex; e0 += AO_ROWS) {
-    const int ne = (int)min64(AO_ROWS, jb.n_vex - e0);
+  for (int64_t e0 = ea; e0 < eb; e0 += AO_ROWS) {
+    const int ne = (int)min64(AO_ROWS, eb - e0);
     __syncthreads();
     for (int e = tid; e < qpk * ne; e += blockDim.x) {
       const int g = e / ne, i = e % ne;
@@ -397,7 +411,7 @@ __global__ void __launch_bounds__(1024) k_attn_out(const AttnJob *jobs, AttnPara
       mass[tid] += m;
     }
 #pragma unroll 4
-    for (int i = half; i < ne; i += NS) {
+    for (int i = grp; i < ne; i += NS) {
       const float v = to_f<TE>(V[(size_t)(e0 + i) * p.d]);
 #pragma unroll
       for (int g = 0; g < 8; ++g)
@@ -406,25 +420,43 @@ __global__ void __launch_bounds__(1024) k_attn_out(const AttnJob *jobs, AttnPara
   }
 #pragma unroll
   for (int g = 0; g < 8; ++g)
-    if (g < qpk) part[(half * qpk + g) * hd + f] = acc[g];
+    if (g < qpk) part[(grp * qpk + g) * hd + f] = acc[g];
   __syncthreads();
+  float *op = jb.opart + (size_t)part_id * nq * hd;
   for (int e = tid; e < qpk * hd; e += blockDim.x) {
     const int g = e / hd, ff = e % hd;
     float o = 0.f;
     for (int t = 0; t < NS; ++t) o += part[(t * qpk + g) * hd + ff];
-    jb.out[(size_t)(q0 + g) * hd + ff] = o;
+    op[(size_t)(q0 + g) * hd + ff] = o;
   }
-  if (tid < qpk && !(fabsf(mass[tid] - 1.f) <= 1e-3f)) record_status(jb.metav, ISKV_ERR_SHAPE);
+  if (tid < qpk) jb.omass[(size_t)part_id * nq + q0 + tid] = mass[tid];
+}
+
+// Sum of the AO_SPLIT parts in order, and the probability-mass check per query head.
+__global__ void __launch_bounds__(256) k_attn_final(const AttnJob *jobs, AttnParams p) {
+  const AttnJob &jb = jobs[blockIdx.y];
+  const int nq = p.n_q, hd = p.head_dim;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < nq * hd; e += gridDim.x * blockDim.x) {
+    float o = 0.f;
+    for (int s = 0; s < AO_SPLIT; ++s) o += jb.opart[(size_t)s * nq * hd + e];
+    jb.out[e] = o;
+    if (e % hd == 0) {
+      const int j = e / hd;
+      float m = 0.f;
+      for (int s = 0; s < AO_SPLIT; ++s) m += jb.omass[(size_t)s * nq + j];
+      if (!(fabsf(m - 1.f) <= 1e-3f)) record_status(jb.metav, ISKV_ERR_SHAPE);
+    }
+  }
 }
 
 cudaError_t launch_attn_out(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
   const int qpk = p.n_q / p.n_kv;
   if (qpk > 8) return cudaErrorInvalidValue;
-  const int ns = 2;  // thread groups splitting the coordinates and the exact rows
+  const int ns = 256 / p.head_dim > 0 ? 256 / p.head_dim : 1;  // thread groups
   const size_t smem = sizeof(float) * ((size_t)qpk * p.r + (size_t)qpk * AO_ROWS +
                                        (size_t)ns * qpk * p.head_dim);
   const bool sb = p.storage == ISKV_BF16, eb = p.exact_dtype == ISKV_BF16;
-  const dim3 g(p.n_kv, p.count);
+  const dim3 g(p.n_kv, p.count, AO_SPLIT);
   const int nth = ns * p.head_dim;
   cudaError_t e = cudaSuccess;
   if (sb && eb) {
@@ -445,7 +477,8 @@ cudaError_t launch_attn_out(const AttnJob *jobs, const AttnParams &p, cudaStream
     if (e == cudaSuccess) k_attn_out<float, float><<<g, nth, smem, s>>>(jobs, p);
   }
   if (e != cudaSuccess) return e;
-  count_launches(1);
+  k_attn_final<<<dim3(4, p.count), 256, 0, s>>>(jobs, p);
+  count_launches(2);
   return cudaGetLastError();
 }
 

@@ -30,13 +30,15 @@ struct AttnJob {
   float *mpart;              // workspace [nchunk][n_q]: partial probability mass on V rows
   float *P;                  // workspace [n_q][n_cap]: probabilities at the compressed V rows
   void *Pb;                  // the same workspace as bf16 [n_cap][64] (tensor-core value mixing)
+  float *opart;              // workspace [AO_SPLIT][n_q][head_dim]: partial outputs
+  float *omass;              // workspace [AO_SPLIT][n_q]: partial probability mass
   void *bsig;                // workspace: sigma-scaled K basis (tensor-core scores)
   int64_t n_kex, n_vex, n_total;
 };
 
 struct AttnParams {
   int d, r, storage, exact_dtype, n_kv, n_q, head_dim, count, nchunk;
-  int nblk;        // probability-mass partials: blocks of 256 value rows
+  int nblk;        // probability-mass partials: blocks of 256 * ATTN_PROB_ROWS value rows
   int tc_values;   // value mixing on the tensor cores (partials [chunk][r][64])
   double theta;
   float scale;
@@ -45,6 +47,8 @@ struct AttnParams {
 
 constexpr int ATTN_CHUNK = 2048;  // V rows per value-mixing block
 constexpr int ATTN_MAX_Q = 64;   // query heads
+constexpr int ATTN_PROB_ROWS = 8;  // value rows per thread in the probability kernel
+constexpr int AO_SPLIT = 8;        // output parts per (KV head, job)
 
 cudaError_t launch_attn_init(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);
 cudaError_t launch_attn_scores_ffma(const AttnJob *jobs, const AttnParams &p, cudaStream_t s);

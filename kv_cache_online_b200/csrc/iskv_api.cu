@@ -71,7 +71,7 @@ size_t jobs_bytes(int32_t count, size_t each) { return align_up((size_t)count * 
 namespace {
 
 struct AttnWsLayout {
-  size_t tc, tcpv, recon, slices, bsig, S, stats, wpart, mpart, P, per_job, total;
+  size_t tc, tcpv, recon, slices, bsig, S, stats, wpart, mpart, P, opart, omass, per_job, total;
   int nchunk, nblk;
 };
 
@@ -80,7 +80,7 @@ AttnWsLayout attn_ws_layout(int32_t count, int32_t d, int32_t r, int64_t n_cap, 
   AttnWsLayout L;
   L.nchunk = (int)((n_cap + ATTN_CHUNK - 1) / ATTN_CHUNK);
   if (L.nchunk < 1) L.nchunk = 1;
-  L.nblk = (int)((n_cap + 255) / 256);
+  L.nblk = (int)((n_cap + 256 * ATTN_PROB_ROWS - 1) / (256 * ATTN_PROB_ROWS));
   if (L.nblk < 1) L.nblk = 1;
   L.tc = jobs_bytes(count, sizeof(AttnJob));
   L.tcpv = L.tc + tc_table_bytes(count);
@@ -95,7 +95,9 @@ AttnWsLayout attn_ws_layout(int32_t count, int32_t d, int32_t r, int64_t n_cap, 
   // [n_q][n_cap] float32) or the tensor-core ones ([chunk][r][64] float32, [n_cap][64] bf16).
   L.wpart = take((size_t)L.nchunk * r * (n_q > 64 ? n_q : 64) * 4);
   L.mpart = take((size_t)L.nblk * n_q * 4);
-  L.P = take((size_t)(L.nblk * 256) * (4 * n_q > 128 ? 4 * n_q : 128));
+  L.P = take((size_t)n_cap * (4 * n_q > 128 ? 4 * n_q : 128));
+  L.opart = take((size_t)AO_SPLIT * n_q * d * 4);  // head_dim <= d
+  L.omass = take((size_t)AO_SPLIT * n_q * 4);
   L.per_job = o;
   L.total = L.slices + (size_t)count * L.per_job;
   return L;
@@ -566,6 +568,8 @@ iskv_status iskv_decode_attention_batched(
     j.mpart = reinterpret_cast<float *>(slice + L.mpart);
     j.P = reinterpret_cast<float *>(slice + L.P);
     j.Pb = slice + L.P;
+    j.opart = reinterpret_cast<float *>(slice + L.opart);
+    j.omass = reinterpret_cast<float *>(slice + L.omass);
     j.bsig = slice + L.bsig;
     j.n_kex = n_k_exact[i];
     j.n_vex = n_v_exact[i];
