@@ -309,6 +309,26 @@ def time_attention(wl, kv, torch, dev, stream, reps: int = 10, warm: int = 3):
             "status_clean": all(x == 0 for x in status)}
 
 
+def run_diagnostics(wl, kv, torch, dev, stream):
+    """Section 5.1 eq. (12) and factor orthogonality of every history after the timed steps:
+    ||U^T U - I||_F, ||B^T B - I||_F, persistent bytes against the dense cache."""
+    n = [int(h.status()[1]) for h in wl.hists]
+    ne = [PROMPT + WINDOW] * len(wl.hists)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    kv.diagnostics(wl.hists, n_exact=ne, exact_bytes=2, stream=stream)  # warm-up
+    ev0.record(stream)
+    ou, ob, pb = kv.diagnostics(wl.hists, n_exact=ne, exact_bytes=2, stream=stream)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    dense = sum(2 * (x + PROMPT + WINDOW) * D for x in n)
+    tot = int(pb.sum().item())
+    return {"ms_per_call": round(ev0.elapsed_time(ev1), 4),
+            "orth_u_max": float(ou.max().item()), "orth_b_max": float(ob.max().item()),
+            "persistent_bytes": tot, "dense_bytes": int(dense),
+            "compression": round(dense / max(tot, 1), 3)}
+
+
 def run_b200(args):
     import torch
     import torch.distributed as dist
@@ -402,6 +422,11 @@ def run_b200(args):
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
                 "traffic": traffic, "dominant_stage": dom}
 
+    # Diagnostics of the benchmark state (eq. 12 bytes, factor orthogonality).
+    diag = None
+    if not args.no_attention:
+        diag = run_diagnostics(wl, kv, torch, dev, stream)
+
     # Decode attention over the compressed cache (the next row after the hot path), timed apart.
     attn = None
     if not args.no_attention:
@@ -440,6 +465,7 @@ def run_b200(args):
             "cpu_baseline": cpu,
             "parity_spot_check": check,
             "decode_attention": attn,
+            "diagnostics": diag,
         }
         print(json.dumps(line))
     if world > 1:

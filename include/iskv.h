@@ -152,6 +152,24 @@ iskv_status iskv_reconstruct_batched(const iskv_lowrank *hs, int32_t count,
                                      size_t ws_bytes, void *stream);
 
 /*
+ * Diagnostics -- Section 5.1 eq. (12) and the orthogonality Section 4.4 restores. For each history:
+ *   orth_u[i] = ||U^T U - I||_F and orth_b[i] = ||B^T B - I||_F over the current rank k (float64
+ *   from the Gram matrices the re-orthogonalisation computes, float32 accumulation; 0 for an empty
+ *   history, NaN for an inconsistent one),
+ *   persistent_bytes[i] = s_f (n k + d k + k) + exact_elem_bytes * n_exact[i] * d, s_f the factor
+ *   element size (U, the shared basis and the diagonal of Sigma; the exact rows -- protected,
+ *   recent, pending -- held beside the history; positions, reserved capacity, workspaces and any
+ *   reconstructed cache are not counted).
+ * orth_u, orth_b [count] float64 and persistent_bytes [count] int64 are DEVICE arrays; n_exact is a
+ * HOST array of count entries or NULL (no exact rows). hs share d, r_max, storage and n_cap.
+ * ws           iskv_diagnostics_workspace_size(count, d, r_max, n_cap) bytes, 256-byte aligned.
+ */
+size_t iskv_diagnostics_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap);
+iskv_status iskv_diagnostics(const iskv_lowrank *hs, int32_t count, const int64_t *n_exact,
+                             int32_t exact_elem_bytes, double *orth_u, double *orth_b,
+                             int64_t *persistent_bytes, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Decode attention over the compressed cache -- Algorithm 3 steps 7-9 without the dense cache
  * (Section 5.2 names this factor-aware form as the route to a speed-up). For one (sequence,
  * layer): the keys at every cached position are the compressed rows (U_k[i] sigma_k) B_k^T at

@@ -215,6 +215,25 @@ def reconstruct(hist, exact_rows, exact_pos, n_total, n_heads, head_dim, rope, t
                                stream)[0]
 
 
+def diagnostics(hists, n_exact=None, exact_bytes=2, ws=None, stream=None):
+    """Section 5.1 eq. (12) and factor orthogonality for each history: device tensors
+    ``(orth_u, orth_b)`` float64 (``||U^T U - I||_F``, ``||B^T B - I||_F`` over the current rank)
+    and ``persistent_bytes`` int64."""
+    lib = _lib.load()
+    n = len(hists)
+    dev = hists[0].device
+    orth_u = torch.empty(n, dtype=torch.float64, device=dev)
+    orth_b = torch.empty(n, dtype=torch.float64, device=dev)
+    pbytes = torch.empty(n, dtype=torch.int64, device=dev)
+    need = lib.iskv_diagnostics_workspace_size(n, hists[0].d, hists[0].r_max, hists[0].n_cap)
+    w = ws if ws is not None else _ws(dev, need)
+    ne = None if n_exact is None else (ctypes.c_int64 * n)(*[int(x) for x in n_exact])
+    _lib.check(lib.iskv_diagnostics(_handles(hists), n, ne, int(exact_bytes), orth_u.data_ptr(),
+                                    orth_b.data_ptr(), pbytes.data_ptr(), w.data_ptr(), w.numel(),
+                                    _stream(stream)), "diagnostics")
+    return orth_u, orth_b, pbytes
+
+
 def attention_workspace_size(count, d, r_max, n_cap, n_total_max, n_q_heads) -> int:
     return int(_lib.load().iskv_attention_workspace_size(count, d, r_max, n_cap, n_total_max,
                                                          n_q_heads))

@@ -46,6 +46,9 @@ SIGNATURES = {
                                          ctypes.POINTER(c_i64), c_i32, c_i32,
                                          ctypes.POINTER(c_i32), c_f64, ctypes.POINTER(c_vp), c_i32,
                                          c_vp, c_sz, c_vp]),
+    "iskv_diagnostics_workspace_size": (c_sz, [c_i32, c_i32, c_i32, c_i64]),
+    "iskv_diagnostics": (c_i32, [ctypes.POINTER(IskvLowRank), c_i32, ctypes.POINTER(c_i64), c_i32,
+                                 c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "iskv_attention_workspace_size": (c_sz, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32]),
     "iskv_decode_attention": (c_i32, [ctypes.POINTER(IskvLowRank), ctypes.POINTER(IskvLowRank),
                                       c_vp, c_vp, c_i64, c_vp, c_vp, c_i64, c_i32, c_i64, c_i32,

@@ -77,7 +77,7 @@ struct FoldJob {
 struct ReorthJob {
   JobHead h;
   int64_t n_cap;
-  int64_t pad_;
+  int64_t n_exact;  // diagnostics: exact rows held beside the history (persistent bytes)
 };
 
 ISKV_DEV const JobHead &job_head(const char *jobs, int stride, int i) {

@@ -299,7 +299,7 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
     j.h.meta = hs[i].meta;
     j.h.ws = base + jb + (size_t)i * p.ws.total;
     j.n_cap = hs[i].n_cap;
-    j.pad_ = 0;
+    j.n_exact = 0;
   }
   std::vector<TcJob> tj, gj;
   p.tc_host = nullptr;
@@ -465,6 +465,83 @@ iskv_status iskv_reconstruct(const iskv_lowrank *h, const void *exact_rows, int3
   void *o[1] = {out};
   return iskv_reconstruct_batched(h, 1, er, exact_dtype, ep, ne, nt, n_heads, head_dim, ar,
                                   rope_theta, o, out_dtype, ws, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Diagnostics: orthogonality of the factors and persistent bytes (eq. 12)
+size_t iskv_diagnostics_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap) {
+  return iskv_reorth_workspace_size(count, d, r_max, n_cap);
+}
+
+iskv_status iskv_diagnostics(const iskv_lowrank *hs, int32_t count, const int64_t *n_exact,
+                             int32_t exact_elem_bytes, double *orth_u, double *orth_b,
+                             int64_t *persistent_bytes, void *ws, size_t ws_bytes, void *stream) {
+  const char *who = "iskv_diagnostics";
+  g_last_error.clear();
+  if (!hs || !orth_u || !orth_b || !persistent_bytes)
+    return fail(ISKV_ERR_ARG, "%s: null argument", who);
+  if (count < 1 || count > 4096) return fail(ISKV_ERR_SHAPE, "%s: count must be in [1, 4096]", who);
+  if (exact_elem_bytes < 0 || exact_elem_bytes > 8)
+    return fail(ISKV_ERR_ARG, "%s: exact_elem_bytes must be in [0, 8]", who);
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_status st = check_handle(&hs[i], who);
+    if (st != ISKV_OK) return st;
+    if (hs[i].d != hs[0].d || hs[i].r_max != hs[0].r_max || hs[i].storage != hs[0].storage ||
+        hs[i].n_cap != hs[0].n_cap)
+      return fail(ISKV_ERR_SHAPE, "%s: batched histories must share d, r_max, storage, n_cap", who);
+    if (n_exact && n_exact[i] < 0) return fail(ISKV_ERR_SHAPE, "%s: negative n_exact", who);
+  }
+  const int d = hs[0].d, r = hs[0].r_max;
+  const int64_t ncap = hs[0].n_cap;
+  const size_t need = iskv_diagnostics_workspace_size(count, d, r, ncap);
+  iskv_status st = check_ws(ws, ws_bytes, need, who);
+  if (st != ISKV_OK) return st;
+  ReorthParams p;
+  p.d = d;
+  p.r = r;
+  p.storage = hs[0].storage;
+  p.count = count;
+  p.n_cap = ncap;
+  p.ws = reorth_ws_layout(d, r, ncap);
+  char *base = static_cast<char *>(ws);
+  TcJob *gram_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReorthJob)) +
+                                              tc_table_bytes(count));
+  const size_t jb = jobs_bytes(count, sizeof(ReorthJob)) + 2 * tc_table_bytes(count);
+  std::vector<ReorthJob> jobs(count);
+  for (int32_t i = 0; i < count; ++i) {
+    ReorthJob &j = jobs[i];
+    j.h.U = hs[i].U;
+    j.h.sigma = hs[i].sigma;
+    j.h.B = hs[i].B;
+    j.h.pos = hs[i].pos;
+    j.h.meta = hs[i].meta;
+    j.h.ws = base + jb + (size_t)i * p.ws.total;
+    j.n_cap = hs[i].n_cap;
+    j.n_exact = n_exact ? n_exact[i] : 0;
+  }
+  std::vector<TcJob> gj;
+  p.tc_host = nullptr;
+  p.tc_dev = nullptr;
+  p.gram_host = nullptr;
+  p.gram_dev = gram_dev;
+  if (tc_gram_supported(r, p.storage)) {
+    gj.resize(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_gram_job(gj[i], hs[i].U, hs[i].n_cap, hs[i].B, d, r,
+                           reinterpret_cast<const int32_t *>(jobs[i].h.ws + p.ws.scal), hs[i].meta,
+                           jobs[i].h.ws))
+        return fail(ISKV_ERR_CUDA, "%s: tensor map encoding failed", who);
+    p.gram_host = gj.data();
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ReorthJob *djobs = reinterpret_cast<ReorthJob *>(base);
+  cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReorthJob) * count, s);
+  if (e == cudaSuccess && p.gram_host) e = upload_jobs(gram_dev, gj.data(), sizeof(TcJob) * count, s);
+  if (e != cudaSuccess) return cuda_fail(e, "diagnostics: upload");
+  if ((e = launch_diagnostics(djobs, p, exact_elem_bytes, orth_u, orth_b, persistent_bytes, s)) !=
+      cudaSuccess)
+    return cuda_fail(e, "diagnostics");
+  return ISKV_OK;
 }
 
 // ------------------------------------------------------------------------------------------------

@@ -300,7 +300,8 @@ __global__ void k_reorth_finalize(const ReorthJob *jobs, ReorthParams p) {
   if (tid == 0) jb.h.meta[ISKV_META_FOLDS] = 0;
 }
 
-cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s) {
+// Gram matrices U^T U and B^T B of every job into the workspace (G[0], G[1]), after the scalars.
+static cudaError_t reorth_gram(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s) {
   const int r = p.r;
   const ReorthWsLayout &W = p.ws;
   k_reorth_prepare<<<(p.count + 127) / 128, 128, 0, s>>>(jobs, p);
@@ -328,6 +329,65 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   }
   k_gram_reduce<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
   count_launches(2);
+  return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256) k_diag_finish(const ReorthJob *jobs, ReorthParams p,
+                                                     int exact_bytes, double *orth_u,
+                                                     double *orth_b, int64_t *pbytes) {
+  const ReorthJob &jb = jobs[blockIdx.x];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
+  const int64_t k = jb.h.meta[ISKV_META_K], n = jb.h.meta[ISKV_META_N];
+  const int r = p.r;
+  __shared__ double red[2][8];
+  double acc[2] = {0.0, 0.0};
+  const bool skip = sc[FS_SKIP] != 0;
+  if (!skip)
+    for (int w = 0; w < 2; ++w) {
+      const float *G = reinterpret_cast<const float *>(jb.h.ws + p.ws.G[w]);
+      for (int64_t e = threadIdx.x; e < k * k; e += blockDim.x) {
+        const int64_t i = e / k, j = e % k;
+        const double v = (double)G[i * r + j] - (i == j ? 1.0 : 0.0);
+        acc[w] = fma(v, v, acc[w]);
+      }
+    }
+  for (int w = 0; w < 2; ++w) {
+    const double t = warp_sum(acc[w]);
+    if ((threadIdx.x & 31) == 0) red[w][threadIdx.x >> 5] = t;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tu = 0.0, tb = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+      tu += red[0][i];
+      tb += red[1][i];
+    }
+    // An empty history is orthonormal by convention; an inconsistent one reports NaN.
+    const bool bad = skip && k != 0;
+    orth_u[blockIdx.x] = bad ? nan("") : sqrt(tu);
+    orth_b[blockIdx.x] = bad ? nan("") : sqrt(tb);
+    const int64_t sf = p.storage == ISKV_BF16 ? 2 : 4;
+    pbytes[blockIdx.x] = sf * (n * k + (int64_t)p.d * k + k) + (int64_t)exact_bytes * jb.n_exact * p.d;
+  }
+}
+
+cudaError_t launch_diagnostics(const ReorthJob *jobs, const ReorthParams &p, int exact_bytes,
+                               double *orth_u, double *orth_b, int64_t *pbytes, cudaStream_t s) {
+  cudaError_t e = reorth_gram(jobs, p, s);
+  if (e != cudaSuccess) return e;
+  k_diag_finish<<<p.count, 256, 0, s>>>(jobs, p, exact_bytes, orth_u, orth_b, pbytes);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s) {
+  const int r = p.r;
+  const ReorthWsLayout &W = p.ws;
+  const unsigned tn = (r + GBN - 1) / GBN, tm = (r + GBM - 1) / GBM;
+  {
+    cudaError_t e0 = reorth_gram(jobs, p, s);
+    if (e0 != cudaSuccess) return e0;
+  }
   stage_mark(s, ST_REORTH_GRAM);
   k_ns_init<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
   size_t y0[2] = {W.Y[0], W.Y[1]}, z0[2] = {W.Z[0], W.Z[1]};

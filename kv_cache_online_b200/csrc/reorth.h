@@ -29,4 +29,10 @@ struct ReorthParams {
 
 cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s);
 
+// Diagnostics (iS-KV reading notes, Section 5.1 eq. 12 and the orthogonality the re-
+// orthogonalisation restores): ||U^T U - I||_F and ||B^T B - I||_F over the current rank from the
+// same Gram kernels, and the persistent bytes s_f (n k + d k + k) + s_e n_exact d of each history.
+cudaError_t launch_diagnostics(const ReorthJob *jobs, const ReorthParams &p, int exact_bytes,
+                               double *orth_u, double *orth_b, int64_t *pbytes, cudaStream_t s);
+
 }  // namespace iskv
