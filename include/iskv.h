@@ -42,7 +42,7 @@ typedef enum {
   ISKV_ERR_WORKSPACE = 8       /* workspace pointer null, misaligned or too small             */
 } iskv_status;
 
-typedef enum { ISKV_F32 = 0, ISKV_BF16 = 1 } iskv_dtype;
+typedef enum { ISKV_F32 = 0, ISKV_BF16 = 1, ISKV_F16 = 2 } iskv_dtype;
 
 /* Indices into the device meta word of a history. */
 enum { ISKV_META_K = 0, ISKV_META_N = 1, ISKV_META_FOLDS = 2, ISKV_META_STATUS = 3 };

@@ -16,17 +16,17 @@ import math
 import torch
 
 from . import _lib
-from ._lib import ISKV_BF16, ISKV_F32, IskvError, IskvLowRank  # noqa: F401
+from ._lib import ISKV_BF16, ISKV_F16, ISKV_F32, IskvError, IskvLowRank  # noqa: F401
 
-_DT = {torch.float32: ISKV_F32, torch.bfloat16: ISKV_BF16}
-_TD = {ISKV_F32: torch.float32, ISKV_BF16: torch.bfloat16}
+_DT = {torch.float32: ISKV_F32, torch.bfloat16: ISKV_BF16, torch.float16: ISKV_F16}
+_TD = {ISKV_F32: torch.float32, ISKV_BF16: torch.bfloat16, ISKV_F16: torch.float16}
 
 
 def _dt(t: torch.Tensor) -> int:
     try:
         return _DT[t.dtype]
     except KeyError:
-        raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16") from None
+        raise TypeError(f"unsupported dtype {t.dtype}; use float32, bfloat16 or float16") from None
 
 
 def _stream(stream) -> int:

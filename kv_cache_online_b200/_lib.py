@@ -11,7 +11,7 @@ LIB_PATH = os.path.join(_PKG, "libiskv.so")
 c_i32, c_i64, c_sz, c_vp, c_f32, c_f64 = (ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
                                           ctypes.c_void_p, ctypes.c_float, ctypes.c_double)
 
-ISKV_F32, ISKV_BF16 = 0, 1
+ISKV_F32, ISKV_BF16, ISKV_F16 = 0, 1, 2
 META_K, META_N, META_FOLDS, META_STATUS = 0, 1, 2, 3
 STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_CUDA", 4: "ERR_CAPACITY",
           5: "ERR_NONFINITE", 6: "ERR_NOT_CONVERGED", 7: "ERR_TIMEOUT", 8: "ERR_WORKSPACE"}

@@ -133,10 +133,9 @@ cudaError_t launch_attn_scores_ffma(const AttnJob *jobs, const AttnParams &p, cu
   const int gx = (int)((p.n_cap_max + 7) / 8);
   const size_t smem = sizeof(float) * (size_t)(p.r + p.d);
   if (gx < 1) return cudaSuccess;
-  if (p.storage == ISKV_BF16)
-    k_attn_scores_ffma<__nv_bfloat16><<<dim3(gx, p.count), 256, smem, s>>>(jobs, p);
-  else
-    k_attn_scores_ffma<float><<<dim3(gx, p.count), 256, smem, s>>>(jobs, p);
+  with_dtype(p.storage, [&](auto ts) {
+    k_attn_scores_ffma<decltype(ts)><<<dim3(gx, p.count), 256, smem, s>>>(jobs, p);
+  });
   count_launches(1);
   return cudaGetLastError();
 }
@@ -176,10 +175,9 @@ cudaError_t launch_attn_scores_exact(const AttnJob *jobs, const AttnParams &p, i
                                      cudaStream_t s) {
   if (max_kex <= 0) return cudaSuccess;
   const dim3 g((unsigned)((max_kex + 7) / 8), p.count);
-  if (p.exact_dtype == ISKV_BF16)
-    k_attn_scores_exact<__nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
-  else
-    k_attn_scores_exact<float><<<g, 256, 0, s>>>(jobs, p);
+  with_dtype(p.exact_dtype, [&](auto te) {
+    k_attn_scores_exact<decltype(te)><<<g, 256, 0, s>>>(jobs, p);
+  });
   count_launches(1);
   return cudaGetLastError();
 }
@@ -324,10 +322,9 @@ __global__ void __launch_bounds__(AV_THREADS) k_attn_values(const AttnJob *jobs,
 cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
   const int mt = (p.n_q + AV_BM - 1) / AV_BM;
   const dim3 g((p.r + AV_BN - 1) / AV_BN, mt * p.nchunk, p.count);
-  if (p.storage == ISKV_BF16)
-    k_attn_values<__nv_bfloat16><<<g, AV_THREADS, 0, s>>>(jobs, p);
-  else
-    k_attn_values<float><<<g, AV_THREADS, 0, s>>>(jobs, p);
+  with_dtype(p.storage, [&](auto ts) {
+    k_attn_values<decltype(ts)><<<g, AV_THREADS, 0, s>>>(jobs, p);
+  });
   count_launches(1);
   return cudaGetLastError();
 }
@@ -455,27 +452,16 @@ cudaError_t launch_attn_out(const AttnJob *jobs, const AttnParams &p, cudaStream
   const int ns = 256 / p.head_dim > 0 ? 256 / p.head_dim : 1;  // thread groups
   const size_t smem = sizeof(float) * ((size_t)qpk * p.r + (size_t)qpk * AO_ROWS +
                                        (size_t)ns * qpk * p.head_dim);
-  const bool sb = p.storage == ISKV_BF16, eb = p.exact_dtype == ISKV_BF16;
   const dim3 g(p.n_kv, p.count, AO_SPLIT);
   const int nth = ns * p.head_dim;
   cudaError_t e = cudaSuccess;
-  if (sb && eb) {
-    e = cudaFuncSetAttribute(k_attn_out<__nv_bfloat16, __nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) k_attn_out<__nv_bfloat16, __nv_bfloat16><<<g, nth, smem, s>>>(jobs, p);
-  } else if (sb) {
-    e = cudaFuncSetAttribute(k_attn_out<__nv_bfloat16, float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) k_attn_out<__nv_bfloat16, float><<<g, nth, smem, s>>>(jobs, p);
-  } else if (eb) {
-    e = cudaFuncSetAttribute(k_attn_out<float, __nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) k_attn_out<float, __nv_bfloat16><<<g, nth, smem, s>>>(jobs, p);
-  } else {
-    e = cudaFuncSetAttribute(k_attn_out<float, float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e == cudaSuccess) k_attn_out<float, float><<<g, nth, smem, s>>>(jobs, p);
-  }
+  with_dtype(p.storage, [&](auto ts) {
+    with_dtype(p.exact_dtype, [&](auto te) {
+      auto kern = k_attn_out<decltype(ts), decltype(te)>;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) kern<<<g, nth, smem, s>>>(jobs, p);
+    });
+  });
   if (e != cudaSuccess) return e;
   k_attn_final<<<dim3(4, p.count), 256, 0, s>>>(jobs, p);
   count_launches(2);

@@ -2,8 +2,11 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "iskv.h"
 
@@ -12,14 +15,24 @@
 namespace iskv {
 
 // ---------------------------------------------------------------------------------------------
-// Element access for the two storage types.
+// Element access for the storage types (float32, bf16, fp16).
 template <typename T> ISKV_DEV float to_f(T v);
 template <> ISKV_DEV float to_f<float>(float v) { return v; }
 template <> ISKV_DEV float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <> ISKV_DEV float to_f<__half>(__half v) { return __half2float(v); }
 
 template <typename T> ISKV_DEV T from_f(float v);
 template <> ISKV_DEV float from_f<float>(float v) { return v; }
 template <> ISKV_DEV __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <> ISKV_DEV __half from_f<__half>(float v) { return __float2half_rn(v); }
+
+// Host dispatch over an iskv_dtype: f(tag) with tag a value of the element type.
+template <class F>
+inline void with_dtype(int dtype, F &&f) {
+  if (dtype == ISKV_BF16) f(__nv_bfloat16{});
+  else if (dtype == ISKV_F16) f(__half{});
+  else f(float{});
+}
 
 // ---------------------------------------------------------------------------------------------
 // Warp reductions.
@@ -38,6 +51,17 @@ ISKV_DEV double warp_sum(double v) {
 ISKV_DEV void record_status(int64_t *meta, int code) {
   atomicOr(reinterpret_cast<unsigned long long *>(meta + ISKV_META_STATUS),
            (unsigned long long)(1ull << code));
+}
+
+// Store v as T. fp16 reaches only 65504: a finite value that overflows it (the failure the pages
+// report for fp16 factors, Section 7.3) records ISKV_ERR_NONFINITE in meta.
+template <typename T>
+ISKV_DEV void store_checked(T *p, float v, int64_t *meta) {
+  const T t = from_f<T>(v);
+  if constexpr (sizeof(T) == 2 && !std::is_same<T, __nv_bfloat16>::value) {
+    if (__hisinf(t) && isfinite(v)) record_status(meta, ISKV_ERR_NONFINITE);
+  }
+  *p = t;
 }
 
 // ---------------------------------------------------------------------------------------------

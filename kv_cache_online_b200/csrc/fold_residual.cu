@@ -380,18 +380,14 @@ cudaError_t launch_fold_residual(const FoldJob *jobs, const FoldParams &p, cudaS
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e;
-  if (p.f_dtype == ISKV_BF16) {
-    e = cudaFuncSetAttribute(k_fold_residual<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
-    if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, k_fold_residual<__nv_bfloat16>, jobs, p);
-  } else {
-    e = cudaFuncSetAttribute(k_fold_residual<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaSuccess;
+  with_dtype(p.f_dtype, [&](auto tf) {
+    using TF = decltype(tf);
+    e = cudaFuncSetAttribute(k_fold_residual<TF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)L.total);
-    if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, k_fold_residual<float>, jobs, p);
-  }
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k_fold_residual<TF>, jobs, p);
+  });
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return e;
 }

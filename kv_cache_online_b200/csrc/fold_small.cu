@@ -131,11 +131,13 @@ static cudaError_t project_t(const FoldJob *jobs, const FoldParams &p, cudaStrea
 }
 
 cudaError_t launch_fold_project(const FoldJob *jobs, const FoldParams &p, cudaStream_t s) {
-  const bool fb = p.f_dtype == ISKV_BF16, sb = p.storage == ISKV_BF16;
-  if (fb && sb) return project_t<__nv_bfloat16, __nv_bfloat16>(jobs, p, s);
-  if (fb) return project_t<__nv_bfloat16, float>(jobs, p, s);
-  if (sb) return project_t<float, __nv_bfloat16>(jobs, p, s);
-  return project_t<float, float>(jobs, p, s);
+  cudaError_t e = cudaSuccess;
+  with_dtype(p.f_dtype, [&](auto tf) {
+    with_dtype(p.storage, [&](auto ts) {
+      e = project_t<decltype(tf), decltype(ts)>(jobs, p, s);
+    });
+  });
+  return e;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -167,10 +169,7 @@ __global__ void __launch_bounds__(256) k_rotate_basis(const char *jobs, RotParam
 
 cudaError_t launch_rotate_basis(const char *jobs, const RotParams &p, cudaStream_t s) {
   const dim3 g((p.r + PBN - 1) / PBN, (p.d + RBM - 1) / RBM, p.count);
-  if (p.storage == ISKV_BF16)
-    k_rotate_basis<__nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
-  else
-    k_rotate_basis<float><<<g, 256, 0, s>>>(jobs, p);
+  with_dtype(p.storage, [&](auto ts) { k_rotate_basis<decltype(ts)><<<g, 256, 0, s>>>(jobs, p); });
   count_launches(1);
   return cudaGetLastError();
 }
@@ -228,7 +227,7 @@ __global__ void __launch_bounds__(256) k_rotate_coords_ffma(const char *jobs, Ro
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int row = i0 + tr + 16 * i, q = q0 + tc + 16 * j;
-        if (row < n && q < kn) U[(size_t)row * r + q] = from_f<TS>(acc[i][j]);
+        if (row < n && q < kn) store_checked(&U[(size_t)row * r + q], acc[i][j], jh.meta);
       }
   }
 }
@@ -237,18 +236,14 @@ cudaError_t launch_rotate_coords_ffma(const char *jobs, const RotParams &p, int6
                                       cudaStream_t s) {
   const dim3 g((unsigned)((n_cap_max + CRM - 1) / CRM), p.count);
   const size_t smem = sizeof(float) * CRM * (p.r + 1);
-  cudaError_t e;
-  if (p.storage == ISKV_BF16) {
-    e = cudaFuncSetAttribute(k_rotate_coords_ffma<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k_rotate_coords_ffma<__nv_bfloat16><<<g, 256, smem, s>>>(jobs, p);
-  } else {
-    e = cudaFuncSetAttribute(k_rotate_coords_ffma<float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k_rotate_coords_ffma<float><<<g, 256, smem, s>>>(jobs, p);
-  }
+  cudaError_t e = cudaSuccess;
+  with_dtype(p.storage, [&](auto ts) {
+    using TS = decltype(ts);
+    e = cudaFuncSetAttribute(k_rotate_coords_ffma<TS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e == cudaSuccess) k_rotate_coords_ffma<TS><<<g, 256, smem, s>>>(jobs, p);
+  });
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }
@@ -274,11 +269,11 @@ __global__ void k_fold_finalize(const FoldJob *jobs, FoldParams p) {
   const float *sig = reinterpret_cast<const float *>(jb.h.ws + p.ws.sig);
   for (int e = tid; e < d * r; e += nth) {
     const int q = e % r;
-    B[e] = from_f<TS>(q < kn ? Bn[e] : 0.f);
+    store_checked(&B[e], q < kn ? Bn[e] : 0.f, jb.h.meta);
   }
   for (int e = tid; e < b * r; e += nth) {
     const int i = e / r, q = e % r;
-    U[(size_t)(n + i) * r + q] = from_f<TS>(q < kn ? Gbot[e] : 0.f);
+    store_checked(&U[(size_t)(n + i) * r + q], q < kn ? Gbot[e] : 0.f, jb.h.meta);
   }
   for (int e = tid; e < b; e += nth) jb.h.pos[n + e] = jb.f_pos[e];
   for (int e = tid; e < r; e += nth) jb.h.sigma[e] = e < kn ? sig[e] : 0.f;
@@ -291,10 +286,7 @@ __global__ void k_fold_finalize(const FoldJob *jobs, FoldParams p) {
 
 cudaError_t launch_fold_finalize(const FoldJob *jobs, const FoldParams &p, cudaStream_t s) {
   const dim3 g(32, p.count);
-  if (p.storage == ISKV_BF16)
-    k_fold_finalize<__nv_bfloat16><<<g, 256, 0, s>>>(jobs, p);
-  else
-    k_fold_finalize<float><<<g, 256, 0, s>>>(jobs, p);
+  with_dtype(p.storage, [&](auto ts) { k_fold_finalize<decltype(ts)><<<g, 256, 0, s>>>(jobs, p); });
   count_launches(1);
   return cudaGetLastError();
 }

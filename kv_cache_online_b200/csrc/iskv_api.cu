@@ -36,7 +36,7 @@ iskv_status cuda_fail(cudaError_t e, const char *where) {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-bool valid_dtype(int32_t t) { return t == ISKV_F32 || t == ISKV_BF16; }
+bool valid_dtype(int32_t t) { return t == ISKV_F32 || t == ISKV_BF16 || t == ISKV_F16; }
 
 iskv_status check_handle(const iskv_lowrank *h, const char *who) {
   if (!h) return fail(ISKV_ERR_ARG, "%s: null history handle", who);
@@ -770,7 +770,8 @@ iskv_status iskv_select_prompt_blocks(const void *keys, int32_t k_dtype, int64_t
   g_last_error.clear();
   if (!keys || !pk_out || !pv_out || !head_blocks_out || !counts_out)
     return fail(ISKV_ERR_ARG, "%s: null pointer", who);
-  if (!valid_dtype(k_dtype)) return fail(ISKV_ERR_ARG, "%s: bad key dtype", who);
+  if (k_dtype != ISKV_F32 && k_dtype != ISKV_BF16)
+    return fail(ISKV_ERR_ARG, "%s: keys must be float32 or bf16", who);
   if (L < 1 || L > ((int64_t)1 << 24)) return fail(ISKV_ERR_SHAPE, "%s: need 1 <= L <= 2^24", who);
   if (n_heads < 1 || n_heads > 64 || head_dim < 2 || head_dim > 256 || head_dim % 2)
     return fail(ISKV_ERR_SHAPE, "%s: need n_heads <= 64, even head_dim <= 256", who);
@@ -809,7 +810,7 @@ iskv_status iskv_reset(const iskv_lowrank *h, void *stream) {
   iskv_status st = check_handle(h, "iskv_reset");
   if (st != ISKV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t es = h->storage == ISKV_BF16 ? 2 : 4;
+  const size_t es = h->storage == ISKV_F32 ? 4 : 2;
   cudaError_t e = cudaMemsetAsync(h->meta, 0, 4 * sizeof(int64_t), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->sigma, 0, sizeof(float) * h->r_max, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->U, 0, es * (size_t)h->n_cap * h->r_max, s);

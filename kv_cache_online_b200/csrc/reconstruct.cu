@@ -81,8 +81,8 @@ __global__ void __launch_bounds__(256) k_recon_ffma(const ReconJob *jobs, ReconP
       x1 = y1;
       x2 = y2;
     }
-    out[c] = from_f<TO>(x1);
-    out[c + half] = from_f<TO>(x2);
+    store_checked(&out[c], x1, jb.meta);
+    store_checked(&out[c + half], x2, jb.meta);
   }
 }
 
@@ -93,6 +93,16 @@ ISKV_DEV void load8(const __nv_bfloat16 *p, float (&v)[8]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+ISKV_DEV void load8(const __half *p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
     v[2 * i] = f.x;
     v[2 * i + 1] = f.y;
   }
@@ -114,6 +124,21 @@ ISKV_DEV void store8(float *p, const float (&v)[8]) {
   reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
   reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
+// fp16: finite values beyond 65504 become infinities; that is recorded as ISKV_ERR_NONFINITE.
+ISKV_DEV void store8(__half *p, const float (&v)[8], int64_t *meta) {
+  uint32_t w[4];
+  bool over = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+    over |= (__hisinf(h.x) && isfinite(v[2 * i])) || (__hisinf(h.y) && isfinite(v[2 * i + 1]));
+    w[i] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  if (over) record_status(meta, ISKV_ERR_NONFINITE);
+  *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <typename T>
+ISKV_DEV void store8(T *p, const float (&v)[8], int64_t *) { store8(p, v); }
 
 // Exact rows: copy (and rotate) exact_rows[e] to out[exact_pos[e]]. Thread = (row, head, group of
 // V consecutive pairs); consecutive threads take consecutive groups of a head, so loads and stores
@@ -163,11 +188,11 @@ __global__ void __launch_bounds__(256) k_recon_exact(const ReconJob *jobs, Recon
       }
     }
     if constexpr (V == 8) {
-      store8(dst, x1);
-      store8(dst + half, x2);
+      store8(dst, x1, jb.meta);
+      store8(dst + half, x2, jb.meta);
     } else {
-      dst[0] = from_f<TO>(x1[0]);
-      dst[half] = from_f<TO>(x2[0]);
+      store_checked(&dst[0], x1[0], jb.meta);
+      store_checked(&dst[half], x2[0], jb.meta);
     }
   }
 }
@@ -182,11 +207,13 @@ static cudaError_t recon_ffma_t(const ReconJob *jobs, const ReconParams &p, cuda
 
 cudaError_t launch_recon_compressed_ffma(const ReconJob *jobs, const ReconParams &p,
                                          cudaStream_t s) {
-  const bool sb = p.storage == ISKV_BF16, ob = p.out_dtype == ISKV_BF16;
-  if (sb && ob) return recon_ffma_t<__nv_bfloat16, __nv_bfloat16>(jobs, p, s);
-  if (sb) return recon_ffma_t<__nv_bfloat16, float>(jobs, p, s);
-  if (ob) return recon_ffma_t<float, __nv_bfloat16>(jobs, p, s);
-  return recon_ffma_t<float, float>(jobs, p, s);
+  cudaError_t e = cudaSuccess;
+  with_dtype(p.storage, [&](auto ts) {
+    with_dtype(p.out_dtype, [&](auto to) {
+      e = recon_ffma_t<decltype(ts), decltype(to)>(jobs, p, s);
+    });
+  });
+  return e;
 }
 
 cudaError_t launch_recon_compressed(const ReconJob *jobs, const ReconParams &p, cudaStream_t s) {
@@ -200,18 +227,14 @@ cudaError_t launch_recon_exact(const ReconJob *jobs, const ReconParams &p, int64
   const int64_t work = max_exact * (int64_t)p.n_heads * (p.head_dim / 2 / V);
   const unsigned gx = (unsigned)((work + 255) / 256 < 4096 ? (work + 255) / 256 : 4096);
   const dim3 g(gx, p.count);
-  const bool eb = p.exact_dtype == ISKV_BF16, ob = p.out_dtype == ISKV_BF16;
-  if (V == 8) {
-    if (eb && ob) k_recon_exact<__nv_bfloat16, __nv_bfloat16, 8><<<g, 256, 0, s>>>(jobs, p);
-    else if (eb) k_recon_exact<__nv_bfloat16, float, 8><<<g, 256, 0, s>>>(jobs, p);
-    else if (ob) k_recon_exact<float, __nv_bfloat16, 8><<<g, 256, 0, s>>>(jobs, p);
-    else k_recon_exact<float, float, 8><<<g, 256, 0, s>>>(jobs, p);
-  } else {
-    if (eb && ob) k_recon_exact<__nv_bfloat16, __nv_bfloat16, 1><<<g, 256, 0, s>>>(jobs, p);
-    else if (eb) k_recon_exact<__nv_bfloat16, float, 1><<<g, 256, 0, s>>>(jobs, p);
-    else if (ob) k_recon_exact<float, __nv_bfloat16, 1><<<g, 256, 0, s>>>(jobs, p);
-    else k_recon_exact<float, float, 1><<<g, 256, 0, s>>>(jobs, p);
-  }
+  with_dtype(p.exact_dtype, [&](auto te) {
+    with_dtype(p.out_dtype, [&](auto to) {
+      using TE = decltype(te);
+      using TO = decltype(to);
+      if (V == 8) k_recon_exact<TE, TO, 8><<<g, 256, 0, s>>>(jobs, p);
+      else k_recon_exact<TE, TO, 1><<<g, 256, 0, s>>>(jobs, p);
+    });
+  });
   count_launches(1);
   return cudaGetLastError();
 }

@@ -294,7 +294,7 @@ __global__ void k_reorth_finalize(const ReorthJob *jobs, ReorthParams p) {
   const float *sig = reinterpret_cast<const float *>(jb.h.ws + p.ws.sig);
   for (int e = tid; e < d * r; e += nth) {
     const int q = e % r;
-    B[e] = from_f<TS>(q < k ? Bn[e] : 0.f);
+    store_checked(&B[e], q < k ? Bn[e] : 0.f, jb.h.meta);
   }
   for (int e = tid; e < r; e += nth) jb.h.sigma[e] = e < k ? sig[e] : 0.f;
   if (tid == 0) jb.h.meta[ISKV_META_FOLDS] = 0;
@@ -318,13 +318,12 @@ static cudaError_t reorth_gram(const ReorthJob *jobs, const ReorthParams &p, cud
     gp.off_gb = W.gpart_b;
     cudaError_t e0 = launch_tc_gram(p.gram_dev, gp, s);
     if (e0 != cudaSuccess) return e0;
-  } else if (p.storage == ISKV_BF16) {
-    k_gram_partial<__nv_bfloat16><<<dim3(tn, tm, p.count * W.nsplit_u), 256, 0, s>>>(jobs, p, 0, W.nsplit_u);
-    k_gram_partial<__nv_bfloat16><<<dim3(tn, tm, p.count * W.nsplit_b), 256, 0, s>>>(jobs, p, 1, W.nsplit_b);
-    count_launches(2);
   } else {
-    k_gram_partial<float><<<dim3(tn, tm, p.count * W.nsplit_u), 256, 0, s>>>(jobs, p, 0, W.nsplit_u);
-    k_gram_partial<float><<<dim3(tn, tm, p.count * W.nsplit_b), 256, 0, s>>>(jobs, p, 1, W.nsplit_b);
+    with_dtype(p.storage, [&](auto ts) {
+      using TS = decltype(ts);
+      k_gram_partial<TS><<<dim3(tn, tm, p.count * W.nsplit_u), 256, 0, s>>>(jobs, p, 0, W.nsplit_u);
+      k_gram_partial<TS><<<dim3(tn, tm, p.count * W.nsplit_b), 256, 0, s>>>(jobs, p, 1, W.nsplit_b);
+    });
     count_launches(2);
   }
   k_gram_reduce<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
@@ -366,7 +365,7 @@ __global__ void __launch_bounds__(256) k_diag_finish(const ReorthJob *jobs, Reor
     const bool bad = skip && k != 0;
     orth_u[blockIdx.x] = bad ? nan("") : sqrt(tu);
     orth_b[blockIdx.x] = bad ? nan("") : sqrt(tb);
-    const int64_t sf = p.storage == ISKV_BF16 ? 2 : 4;
+    const int64_t sf = p.storage == ISKV_F32 ? 4 : 2;
     pbytes[blockIdx.x] = sf * (n * k + (int64_t)p.d * k + k) + (int64_t)exact_bytes * jb.n_exact * p.d;
   }
 }
@@ -456,10 +455,9 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   stage_mark(s, ST_REORTH_COORDS);
   e = launch_rotate_basis(reinterpret_cast<const char *>(jobs), q, s);
   if (e != cudaSuccess) return e;
-  if (p.storage == ISKV_BF16)
-    k_reorth_finalize<__nv_bfloat16><<<dim3(32, p.count), 256, 0, s>>>(jobs, p);
-  else
-    k_reorth_finalize<float><<<dim3(32, p.count), 256, 0, s>>>(jobs, p);
+  with_dtype(p.storage, [&](auto ts) {
+    k_reorth_finalize<decltype(ts)><<<dim3(32, p.count), 256, 0, s>>>(jobs, p);
+  });
   count_launches(1);
   stage_mark(s, ST_REORTH_BASIS);
   return cudaGetLastError();
