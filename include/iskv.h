@@ -42,6 +42,15 @@ typedef enum {
   ISKV_ERR_WORKSPACE = 8       /* workspace pointer null, misaligned or too small             */
 } iskv_status;
 
+/*
+ * Element types of factors, blocks, exact rows and reconstruction outputs. The tensor-core kernels
+ * take bf16 factors (and bf16 reconstruction outputs); float32 and fp16 run on CUDA cores. fp16 has
+ * a maximum finite value of 65504 (Section 7.3: fp16 factors overflowed on long generations): U and
+ * B have orthonormal columns and sigma stays float32 here, so stored factors stay below 1, but a
+ * reconstructed cache can exceed it -- every store of a finite value that overflows fp16 records
+ * ISKV_ERR_NONFINITE in the history's status word. Prompt keys for the selection are float32 or
+ * bf16.
+ */
 typedef enum { ISKV_F32 = 0, ISKV_BF16 = 1, ISKV_F16 = 2 } iskv_dtype;
 
 /* Indices into the device meta word of a history. */
