@@ -688,7 +688,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-attention", action="store_true",
-                    help="skip the separately timed decode attention over the compressed cache")
+                    help="skip the rows timed apart from the step: decode attention over the "
+                         "compressed cache and the diagnostics")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="model layers (2 histories each); the headline workload is 32")

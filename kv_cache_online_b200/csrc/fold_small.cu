@@ -12,14 +12,20 @@
 namespace iskv {
 
 // ------------------------------------------------------------------------------------------------
-// Job upload: a host array travels as kernel parameters (up to 16 KB per launch), so the copy is
-// stream-ordered and needs no host buffer to outlive the call.
-struct UploadChunk {
-  unsigned char data[16384];
+// Job upload: a host array travels as kernel parameters (up to 32736 bytes per launch, inside the
+// 32764-byte parameter limit), so the copy is stream-ordered and needs no host buffer to outlive
+// the call. Parameters live in a constant bank, where a warp's distinct addresses are served one
+// at a time: the copy moves 16-byte words to keep that count low.
+struct alignas(16) UploadChunk {
+  unsigned char data[32736];
 };
 
 __global__ void k_upload(unsigned char *dst, UploadChunk c, int nbytes) {
-  for (int i = threadIdx.x; i < nbytes; i += blockDim.x) dst[i] = c.data[i];
+  const int words = nbytes / 16;  // dst is 16-byte aligned (workspace tables, chunk offsets)
+  const uint4 *src4 = reinterpret_cast<const uint4 *>(c.data);
+  uint4 *dst4 = reinterpret_cast<uint4 *>(dst);
+  for (int i = threadIdx.x; i < words; i += blockDim.x) dst4[i] = src4[i];
+  for (int i = words * 16 + threadIdx.x; i < nbytes; i += blockDim.x) dst[i] = c.data[i];
 }
 
 cudaError_t upload_jobs(void *dst, const void *src, size_t bytes, cudaStream_t s) {
