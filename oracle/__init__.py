@@ -27,8 +27,12 @@ reconstruct per-step reconstruction (Algorithm 3 steps 7-8).
 select      Algorithm 1 steps 2-4 (block outlier score, lowest-128 per head, union, value radius).
 accounting  Section 5.1 persistent-storage arithmetic (eq. 12 and its consequences).
 drift       Section 2.3 coordinate drift and the appendix factor-drift measure (eq. 14).
+attention   decode attention over the compressed cache (Algorithm 3 steps 7-9).
+policy      the cache policy: protected rows, recent window, pending FIFO and the fold schedule
+            (Algorithm 1 steps 5-8, Algorithm 3 steps 1-6).
 """
 
-from . import accounting, drift, fold, reconstruct, reorth, rope, select  # noqa: F401
+from . import accounting, attention, drift, fold, policy, reconstruct, reorth, rope, select  # noqa: F401
 
-__all__ = ["accounting", "drift", "fold", "reconstruct", "reorth", "rope", "select"]
+__all__ = ["accounting", "attention", "drift", "fold", "policy", "reconstruct", "reorth", "rope",
+           "select"]

@@ -1,0 +1,130 @@
+"""Pins for the cache-policy oracle (Section 3.1, Section 3.2, Algorithm 1 steps 5-8, Algorithm 3
+steps 1-6): a schedule worked by hand, a closed form, a reduction to the pinned block stream, the
+partition invariants, and exact recovery of rank-deficient data."""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from conftest import GOLDEN
+from oracle import fold as of
+from oracle import policy as op
+from oracle import reconstruct as orec
+import synth
+
+
+def _golden():
+    with open(os.path.join(GOLDEN, "policy_small.json")) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden(), ids=lambda c: c["name"][:6])
+def test_hand_worked_schedule(case):
+    side, comp = op.new_side(case["L"], case["protected"], case["init_window"], case["window"],
+                             case["block"], case["reorth_rows"])
+    assert side.prot == case["prefill"]["prot"]
+    assert side.live == case["prefill"]["live"]
+    assert comp == case["prefill"]["comp"]
+    for i in range(case["decode_steps"]):
+        t = case["L"] + i
+        acts = op.append(side, t)
+        assert [list(a[:1]) + [list(a[1])] if a[0] == "fold" else list(a) for a in acts] == \
+            case["steps"][str(t)], t
+    assert op.exact_positions(side) == case["final"]["exact"]
+    assert comp + side.compressed == case["final"]["history"]
+
+
+@pytest.mark.parametrize("L,W,b", [(10, 4, 2), (1000, 128, 64), (37, 16, 8), (5, 0, 8)])
+def test_empty_window_closed_form(L, W, b):
+    """Keys (empty window at prefill, protected rows inside the prompt only): the j-th fold comes
+    with position L - 1 + W + j b and merges positions L + (j-1) b .. L + j b - 1."""
+    side, _ = op.new_side(L, [L - 1], 0, W, b, 0)
+    folds = []
+    for t in range(L, L + W + 6 * b - 1):    # just before the sixth fold
+        for a in op.append(side, t):
+            folds.append((t, a[1]))
+    assert len(folds) == 5
+    for j, (t, blk) in enumerate(folds, start=1):
+        assert t == L - 1 + W + j * b
+        assert blk == list(range(L + (j - 1) * b, L + j * b))
+
+
+def test_no_prompt_no_window_reduces_to_block_stream():
+    """Empty prompt and W = 0: every b decode rows are folded as they arrive, which is the pinned
+    block stream ``fold_stream``; the rows after the last full block stay exact."""
+    d, b, r = 24, 4, 6
+    X = synth.lowrank_rows(30, d, 1.0, 0.05, seed=3)
+    out = op.run_decode(np.zeros((0, d)), X, [], 0, 0, b, r, 0)
+    U, s, B, pos = out["history"]
+    Us, ss, Bs, _ = of.fold_stream(X, b, r)
+    np.testing.assert_array_equal(U, Us)
+    np.testing.assert_array_equal(s, ss)
+    np.testing.assert_array_equal(B, Bs)
+    np.testing.assert_array_equal(pos, np.arange(28))
+    np.testing.assert_array_equal(out["exact"][1], [28, 29])
+    np.testing.assert_array_equal(out["exact"][0], X[28:])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_partition_invariants(seed):
+    g = synth.rng(100 + seed)
+    L = int(g.integers(0, 300))
+    W = int(g.integers(0, 40))
+    b = int(g.choice([1, 2, 8, 16]))
+    w0 = int(g.integers(0, W + 1))
+    R = int(g.choice([0, b, 3 * b, 5 * b + 1]))
+    P = np.flatnonzero(g.random(L) < 0.2).tolist()
+    side, comp = op.new_side(L, P, w0, W, b, R)
+    n_folds = n_reorth = 0
+    for t in range(L, L + 400):
+        acts = op.append(side, t)
+        for a in acts:
+            if a[0] == "fold":
+                n_folds += 1
+                blk = a[1]
+                assert len(blk) == b and blk == sorted(blk)
+                assert all(p not in P and p <= t - W for p in blk)
+            else:
+                n_reorth += 1
+        assert len(side.pending()) < b
+        exact = set(op.exact_positions(side))
+        everything = sorted(list(exact) + comp + side.compressed)
+        assert everything == list(range(t + 1))                          # a partition of 0..t
+        # the window is exact, except prompt rows compressed at prefill (outside the initial window)
+        assert all(p in exact for p in range(max(0, t - W + 1, L - w0), t + 1))
+        assert set(side.prot) == set(P)
+    if R:
+        assert n_reorth == n_folds // math.ceil(R / b)
+    else:
+        assert n_reorth == 0
+
+
+def test_rank_deficient_rows_are_recovered():
+    """Rows of rank below the budget: the history represents every compressed row exactly, the exact
+    table holds the stored rows, and reconstruction returns the whole sequence."""
+    d, r, b, W, L, T = 32, 10, 4, 6, 40, 50
+    g = synth.rng(9)
+    X = g.standard_normal((L + T, 5)) @ g.standard_normal((5, d))
+    P = [0, 3, 4, 20, 38, 39]
+    out = op.run_decode(X[:L], X[L:], P, 6, W, b, r, 8)
+    U, s, B, pos = out["history"]
+    np.testing.assert_allclose(of.low_rank_product(U, s, B), X[pos], atol=1e-9)
+    rows, epos = out["exact"]
+    np.testing.assert_array_equal(rows, X[epos])
+    full = orec.reconstruct(U, s, B, pos, rows, epos, L + T, 1, d, False, 500000.0)
+    np.testing.assert_allclose(full, X, atol=1e-9)
+
+
+def test_argument_errors():
+    with pytest.raises(ValueError):
+        op.new_side(10, [1], 5, 4, 2, 0)          # init window longer than the window
+    with pytest.raises(ValueError):
+        op.prefill_partition(10, [3, 3], 0)       # repeated protected position
+    with pytest.raises(ValueError):
+        op.prefill_partition(10, [10], 0)         # outside the prompt
+    side, _ = op.new_side(10, [], 0, 4, 2, 0)
+    with pytest.raises(ValueError):
+        op.append(side, 12)                        # positions arrive one at a time
