@@ -329,6 +329,58 @@ def run_diagnostics(wl, kv, torch, dev, stream):
             "compression": round(dense / max(tot, 1), 3)}
 
 
+def time_cache_policy(wl, kv, torch, dev, stream):
+    """The cache policy's decode step (Algorithm 3 steps 1-2 and 4-6) on the benchmark's 64 histories:
+    each side's exact-row table holds its 512 protected prompt rows and its 128 window rows (W = 128,
+    b = 64); 63 steps only store the new rows, the 64th folds the oldest 64 rows of every table and
+    removes them from the tables. Run last: it folds one more block into every history."""
+    cnt = len(wl.hists)
+    tabs = []
+    for i, h in enumerate(wl.hists):
+        n = int(h.status()[1])
+        t = kv.ExactTable(D, PROMPT + WINDOW + BLK, window=WINDOW, block=BLK, reorth_rows=0,
+                          dtype=torch.bfloat16, device=dev)
+        t.rows[:PROMPT + WINDOW].copy_(wl.exact[i])
+        win = torch.arange(PROMPT + n, PROMPT + n + WINDOW, dtype=torch.int32, device=dev)
+        t.pos[:PROMPT + WINDOW].copy_(torch.cat([torch.arange(PROMPT, dtype=torch.int32,
+                                                              device=dev), win]))
+        for j in range(WINDOW):
+            t.live[j] = PROMPT + n + j
+        t.t.n_prot, t.t.n_live, t.t.last, t.t.hist_rows = PROMPT, WINDOW, PROMPT + n + WINDOW - 1, n
+        tabs.append(t)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4242)
+    rows = torch.randn(BLK, cnt, D, generator=gen, device=dev).to(torch.bfloat16)
+    ws = kv.Workspace(dev).get(kv.cache_step_workspace_size(cnt, D, R, BLK, wl.hists[0].n_cap))
+    torch.cuda.synchronize(dev)
+    kv.stage_times(reset=True)
+    kv.stage_timing(True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record(stream)
+    for j in range(BLK - 1):
+        folded, _ = kv.cache_step(tabs, wl.hists, rows[j], ws=ws, stream=stream)
+        assert not any(folded)
+    ev[1].record(stream)
+    folded, _ = kv.cache_step(tabs, wl.hists, rows[BLK - 1], ws=ws, stream=stream)
+    ev[2].record(stream)
+    torch.cuda.synchronize(dev)
+    kv.stage_timing(False)
+    st = kv.stage_times(reset=True)
+    a_ms = ev[0].elapsed_time(ev[1]) / (BLK - 1)
+    f_ms = ev[1].elapsed_time(ev[2])
+    per = {k: round(v[0] / max(v[1], 1), 4) for k, v in st.items()
+           if v[1] and (k.startswith("cache") or k.startswith("fold"))}
+    ok = all(folded) and all(t.t.n_live == WINDOW for t in tabs) and \
+        all(h.status()[3] == 0 for h in wl.hists)
+    return {"tables": cnt, "window": WINDOW, "block": BLK,
+            "store_step_ms": round(a_ms, 4), "fold_step_ms": round(f_ms, 4),
+            "ms_per_token_amortised": round(((BLK - 1) * a_ms + f_ms) / BLK, 4),
+            "kernel_ms": per, "status_ok": bool(ok),
+            "note": "step times are CUDA events on the stream around each call, so a store-only "
+                    "step includes the host's per-call overhead; kernel_ms are the library's "
+                    "stage events"}
+
+
 def run_b200(args):
     import torch
     import torch.distributed as dist
@@ -437,6 +489,11 @@ def run_b200(args):
     if not args.no_e2e:
         e2e = run_e2e(wl, kv, torch, dev, stream, pos, steps_total, e2e_steps, world)
 
+    # The cache policy's decode step on the same histories (folds one more block into each).
+    policy = None
+    if not args.no_attention:
+        policy = time_cache_policy(wl, kv, torch, dev, stream)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(args.cpu_budget)
@@ -466,6 +523,7 @@ def run_b200(args):
             "parity_spot_check": check,
             "decode_attention": attn,
             "diagnostics": diag,
+            "cache_policy": policy,
         }
         print(json.dumps(line))
     if world > 1:
@@ -689,7 +747,7 @@ def main(argv=None):
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-attention", action="store_true",
                     help="skip the rows timed apart from the step: decode attention over the "
-                         "compressed cache and the diagnostics")
+                         "compressed cache, the diagnostics and the cache-policy step")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="model layers (2 histories each); the headline workload is 32")

@@ -35,7 +35,8 @@ typedef enum {
   ISKV_ERR_ARG = 1,            /* null pointer, bad enum, misaligned pointer                  */
   ISKV_ERR_SHAPE = 2,          /* inconsistent or unsupported sizes                           */
   ISKV_ERR_CUDA = 3,           /* a CUDA runtime call or kernel launch failed                 */
-  ISKV_ERR_CAPACITY = 4,       /* device: n + b > n_cap, the fold was skipped                 */
+  ISKV_ERR_CAPACITY = 4,       /* device: n + b > n_cap, the fold was skipped; host: a cache
+                                  table or history has no room for the step                    */
   ISKV_ERR_NONFINITE = 5,      /* device: a non-finite singular value came out of a fold      */
   ISKV_ERR_NOT_CONVERGED = 6,  /* device: Jacobi / Newton-Schulz hit its iteration cap        */
   ISKV_ERR_TIMEOUT = 7,        /* device: a bounded cluster wait gave up                      */
@@ -269,6 +270,104 @@ iskv_status iskv_select_prompt_blocks_noalloc(const void *keys, int32_t k_dtype,
                                               int32_t *head_blocks_out, int64_t *counts_out,
                                               void *stream);
 
+/*
+ * Cache policy: the exact rows of one side (K or V) of one (sequence, layer), and when its pending
+ * rows are folded (Section 3.1, Section 3.2; Algorithm 1 steps 5-8, Algorithm 3 steps 1-6).
+ *
+ * A side keeps exact: its protected rows P_X (fixed at prefill), the rows at the `window` most recent
+ * positions, and the pending FIFO (unprotected rows that have left the window and wait for a full
+ * block of `block` rows). Readings: the window is the set of the W most recent positions; a
+ * protected position inside it is stored once, as protected, and stays exact when it leaves; decode
+ * rows are never protected; the window at prefill is no longer than W (empty for keys by
+ * Algorithm 1 step 5, the last min(W, L) prompt positions for values), so at most one row joins
+ * the FIFO per decode step. The value side's first refit (Algorithm 3 step 3) is not implemented:
+ * both sides fold regular blocks from the first full one.
+ *
+ * Exact-row table (device, caller-owned):
+ *   rows [cap_e][d]  dtype; rows 0 .. n_prot-1 are the protected rows in ascending position, rows
+ *                    n_prot .. n_prot+n_live-1 the live rows (FIFO, then the unprotected window
+ *                    rows) in ascending position. 16-byte aligned; d * element size a multiple of
+ *                    16 bytes.
+ *   pos  [cap_e]     int32 positions of those rows. rows/pos are directly the exact_rows /
+ *                    exact_pos arguments of iskv_reconstruct() and iskv_decode_attention(), with
+ *                    n_exact = n_prot + n_live.
+ * Host mirror (maintained by the library; the caller sets the first block of fields and live_host /
+ * live_cap, then lets iskv_cache_prefill() fill the rest):
+ *   live_host [live_cap]  HOST int32: positions of the live rows, ascending; live_cap >=
+ *                         window + block.
+ *   n_prot, n_live, last  counts and the last stored position (prompt length - 1 after prefill).
+ *   fold_rows             rows merged by folds since the last re-orthogonalisation.
+ *   hist_rows             rows of the side's history (prefill sets it to the compressed prompt
+ *                         rows; each fold adds `block`); a fold that would pass the history's n_cap
+ *                         is refused on the host before anything is launched.
+ * The mirror lets the host decide, without reading the device, which tables fold in a step.
+ */
+typedef struct {
+  int32_t d;
+  int32_t window;      /* W: the most recent W positions stay exact                         */
+  int32_t block;       /* b: rows per fold, as iskv_fold_block() accepts                    */
+  int32_t reorth_rows; /* re-orthogonalise after this many folded rows; 0 = never           */
+  int32_t dtype;       /* iskv_dtype of rows                                                */
+  int32_t reserved;
+  int64_t cap_e;       /* row capacity of rows / pos                                        */
+  void *rows;
+  int32_t *pos;
+  int32_t *live_host;  /* host */
+  int64_t live_cap;
+  int64_t n_prot;
+  int64_t n_live;
+  int64_t last;
+  int64_t fold_rows;
+  int64_t hist_rows;
+} iskv_exact_table;
+
+/*
+ * Prefill partition (Algorithm 1 steps 5-7): split the L prompt rows X [L][d] (x_dtype) of one side.
+ *   protected_pos [n_protected]  int32, strictly ascending, inside [0, L): P_X (for keys the
+ *                                selection's P_K, for values its P_V).
+ *   init_window                  0 for keys, min(W, L) for values; 0 <= init_window <= t->window.
+ * Writes the protected rows, then the unprotected rows among the last init_window positions, into
+ * the exact-row table (converted to t->dtype), and every other row, in ascending position, into
+ * comp_rows [L][d] (x_dtype) with comp_pos [L]: the rows the prompt's truncated SVD compresses
+ * (Algorithm 1 step 7; that SVD itself is not part of the library). Sets the host mirror
+ * (n_prot = n_protected, n_live, live_host, last = L - 1, fold_rows = 0, hist_rows = *n_comp) and
+ * *n_comp (host). The caller then puts the compressed rows' factors in the side's history, with
+ * their positions comp_pos in its position table.
+ * SYNCHRONOUS: waits for the stream, because the mirror needs the live positions. Errors:
+ * ISKV_ERR_ARG for null / misaligned pointers, bad dtypes, init_window out of range, or
+ * protected_pos not strictly ascending inside [0, L) (found on the device, reported after the
+ * wait; the table is then undefined); ISKV_ERR_CAPACITY when n_protected + init_window > cap_e;
+ * ISKV_ERR_NONFINITE when a finite row value overflows an fp16 table.
+ */
+size_t iskv_cache_prefill_workspace_size(int32_t init_window);
+iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dtype, int64_t L,
+                               const int32_t *protected_pos, int64_t n_protected,
+                               int32_t init_window, void *comp_rows, int32_t *comp_pos,
+                               int64_t *n_comp, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * One decode step for `count` tables (Algorithm 3 steps 1-2 and 4-6): tables[i] (host pointer to a
+ * host struct, updated in place) with its history hists[i] (host pointer) stores new_rows[i] (device
+ * [count][d], row_dtype, converted to the table dtype) at position tables[i]->last + 1; when that
+ * makes `block` rows pending, the oldest `block` of them are folded into hists[i]
+ * (iskv_fold_block_batched over every table that folds, with tau_rel), their positions join the
+ * history's position table and their exact copies leave the table; when a table's folded rows
+ * reach reorth_rows, its history is re-orthogonalised (iskv_reorth) in the same step and the count
+ * restarts. All tables share d, window, block and dtype; the histories share d, r_max, storage
+ * and n_cap, as the batched fold and re-orthogonalisation require. folded / reorthed (host
+ * [count], may be NULL) receive 1 where a table folded / re-orthogonalised. Stream-ordered; the host
+ * mirror is updated at once. Errors (nothing launched, no table changed): ISKV_ERR_ARG,
+ * ISKV_ERR_SHAPE (mixed table shapes, a history whose d differs, a block the fold does not take),
+ * ISKV_ERR_CAPACITY (a table without room for the new row, or a history without room for the
+ * block: hist_rows + block > n_cap), ISKV_ERR_WORKSPACE; ISKV_ERR_CUDA when a launch fails.
+ */
+size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block,
+                                      int64_t n_cap);
+iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank *const *hists,
+                            int32_t count, const void *new_rows, int32_t row_dtype, float tau_rel,
+                            int32_t *folded, int32_t *reorthed, void *ws, size_t ws_bytes,
+                            void *stream);
+
 /* Empty a history: zero its meta word, sigma, U and B (stream-ordered). */
 iskv_status iskv_reset(const iskv_lowrank *h, void *stream);
 
@@ -283,7 +382,8 @@ iskv_status iskv_get_status(const iskv_lowrank *h, int64_t *k, int64_t *n, int64
  * Instrumentation (no counterpart on the pages; measurement support). When stage timing is on,
  * every entry point records CUDA events on its own stream around each internal stage (fold:
  * projection, residual QR + SVD, core SVD, basis rotation, coordinate rotation, write-back;
- * reorth; reconstruction; selection). iskv_stage_read() waits for those events and returns the
+ * reorth; reconstruction; selection; decode attention; cache step: append and eviction).
+ * iskv_stage_read() waits for those events and returns the
  * accumulated milliseconds and call counts per stage (arrays of iskv_stage_count() entries, host
  * memory). iskv_stage_timing() returns the previous setting. iskv_launch_count() is the number of
  * kernels the library has launched in this process (always counted).

@@ -16,7 +16,7 @@ import math
 import torch
 
 from . import _lib
-from ._lib import ISKV_BF16, ISKV_F16, ISKV_F32, IskvError, IskvLowRank  # noqa: F401
+from ._lib import ISKV_BF16, ISKV_F16, ISKV_F32, IskvError, IskvExactTable, IskvLowRank  # noqa: F401
 
 _DT = {torch.float32: ISKV_F32, torch.bfloat16: ISKV_BF16, torch.float16: ISKV_F16}
 _TD = {ISKV_F32: torch.float32, ISKV_BF16: torch.bfloat16, ISKV_F16: torch.float16}
@@ -332,6 +332,90 @@ def select_prompt_blocks(keys, block=8, per_head=128, suffix_blocks=4, v_radius=
         out["P_K"].data_ptr(), out["P_V"].data_ptr(), out["head_blocks"].data_ptr(),
         out["counts"].data_ptr(), w.data_ptr(), w.numel(), _stream(stream)), "select_prompt_blocks")
     return out
+
+
+# ------------------------------------------------------------------------------------------------
+# Cache policy (Section 3.1, Section 3.2, Algorithm 1 steps 5-8, Algorithm 3 steps 1-6).
+
+class ExactTable:
+    """The exact rows of one side (K or V) of one (sequence, layer): protected rows, then the live
+    rows (pending FIFO and unprotected window rows), ascending by position, in device tensors
+    ``rows`` (cap_e, d) and ``pos`` (cap_e,) int32, with the host mirror the library keeps in
+    ``self.t`` (an ``IskvExactTable``)."""
+
+    def __init__(self, d: int, cap_e: int, window: int = 128, block: int = 64,
+                 reorth_rows: int = 256, dtype=torch.bfloat16, device="cuda"):
+        self.rows = torch.zeros(max(int(cap_e), 1), int(d), dtype=dtype, device=device)
+        self.pos = torch.full((max(int(cap_e), 1),), -1, dtype=torch.int32, device=device)
+        self.live = (ctypes.c_int32 * (int(window) + int(block)))()
+        self.t = IskvExactTable(int(d), int(window), int(block), int(reorth_rows), _DT[dtype], 0,
+                                int(cap_e), _ptr(self.rows), _ptr(self.pos),
+                                ctypes.cast(self.live, ctypes.POINTER(ctypes.c_int32)),
+                                int(window) + int(block), 0, 0, -1, 0, 0)
+
+    @property
+    def n_exact(self) -> int:
+        return int(self.t.n_prot + self.t.n_live)
+
+    def exact(self):
+        """``(rows, pos)`` views of the exact rows: the exact_rows / exact_pos of a reconstruction or
+        a decode attention."""
+        n = self.n_exact
+        return self.rows[:n], self.pos[:n]
+
+    def live_positions(self):
+        return [self.live[i] for i in range(self.t.n_live)]
+
+
+def cache_prefill(table: ExactTable, X, protected_pos, init_window: int, ws=None, stream=None):
+    """Algorithm 1 steps 5-7 for one side: protected rows and the unprotected rows of the initial
+    window go to ``table``; returns ``(comp_rows, comp_pos)``, the rows the prompt SVD compresses
+    (device tensors, ascending positions). Synchronises the stream."""
+    lib = _lib.load()
+    _need_cuda(X, protected_pos)
+    if X.dim() != 2 or not X.is_contiguous() or X.shape[1] != table.t.d:
+        raise ValueError("X must be a contiguous (L, d) tensor")
+    if protected_pos.dtype != torch.int32 or not protected_pos.is_contiguous():
+        raise ValueError("protected_pos must be a contiguous int32 tensor")
+    L = int(X.shape[0])
+    comp = torch.empty(max(L, 1), table.t.d, dtype=X.dtype, device=X.device)
+    comp_pos = torch.empty(max(L, 1), dtype=torch.int32, device=X.device)
+    n_comp = ctypes.c_int64()
+    need = lib.iskv_cache_prefill_workspace_size(init_window)
+    w = ws if ws is not None else _ws(X.device, need)
+    _lib.check(lib.iskv_cache_prefill(
+        ctypes.byref(table.t), X.data_ptr(), _dt(X), L, protected_pos.data_ptr(),
+        protected_pos.numel(), int(init_window), comp.data_ptr(), comp_pos.data_ptr(),
+        ctypes.byref(n_comp), w.data_ptr(), w.numel(), _stream(stream)), "cache_prefill")
+    return comp[:n_comp.value], comp_pos[:n_comp.value]
+
+
+def cache_step_workspace_size(count, d, r_max, block, n_cap) -> int:
+    return int(_lib.load().iskv_cache_step_workspace_size(count, d, r_max, block, n_cap))
+
+
+def cache_step(tables, hists, new_rows, tau_rel: float = 0.0, ws=None, stream=None):
+    """Algorithm 3 steps 1-2 and 4-6 for every (table, history) pair: ``new_rows`` (count, d) holds
+    each table's row for its next position. Returns ``(folded, reorthed)`` lists of bools."""
+    lib = _lib.load()
+    n = len(tables)
+    if n == 0 or len(hists) != n:
+        raise ValueError("one history per table")
+    _need_cuda(new_rows)
+    if new_rows.dim() != 2 or new_rows.shape[0] != n or not new_rows.is_contiguous():
+        raise ValueError("new_rows must be a contiguous (count, d) tensor")
+    h0 = hists[0]
+    need = lib.iskv_cache_step_workspace_size(n, h0.d, h0.r_max, tables[0].t.block, h0.n_cap)
+    w = ws if ws is not None else _ws(new_rows.device, need)
+    handles = [h.handle() for h in hists]
+    tp = (ctypes.POINTER(IskvExactTable) * n)(*[ctypes.pointer(t.t) for t in tables])
+    hp = (ctypes.POINTER(IskvLowRank) * n)(*[ctypes.pointer(h) for h in handles])
+    folded = (ctypes.c_int32 * n)()
+    reorthed = (ctypes.c_int32 * n)()
+    _lib.check(lib.iskv_cache_step(tp, hp, n, new_rows.data_ptr(), _dt(new_rows), float(tau_rel),
+                                   folded, reorthed, w.data_ptr(), w.numel(), _stream(stream)),
+               "cache_step")
+    return [bool(x) for x in folded], [bool(x) for x in reorthed]
 
 
 # ------------------------------------------------------------------------------------------------

@@ -25,6 +25,16 @@ class IskvLowRank(ctypes.Structure):
                 ("meta", c_vp)]
 
 
+class IskvExactTable(ctypes.Structure):
+    """Mirror of ``iskv_exact_table``."""
+
+    _fields_ = [("d", c_i32), ("window", c_i32), ("block", c_i32), ("reorth_rows", c_i32),
+                ("dtype", c_i32), ("reserved", c_i32), ("cap_e", c_i64), ("rows", c_vp),
+                ("pos", c_vp), ("live_host", ctypes.POINTER(c_i32)), ("live_cap", c_i64),
+                ("n_prot", c_i64), ("n_live", c_i64), ("last", c_i64), ("fold_rows", c_i64),
+                ("hist_rows", c_i64)]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
     "iskv_abi_version": (c_i32, []),
@@ -66,6 +76,14 @@ SIGNATURES = {
                                           c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "iskv_select_prompt_blocks_noalloc": (c_i32, [c_vp, c_i32, c_i64, c_i32, c_i32, c_i32, c_i32,
                                                   c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "iskv_cache_prefill_workspace_size": (c_sz, [c_i32]),
+    "iskv_cache_prefill": (c_i32, [ctypes.POINTER(IskvExactTable), c_vp, c_i32, c_i64, c_vp, c_i64,
+                                   c_i32, c_vp, c_vp, ctypes.POINTER(c_i64), c_vp, c_sz, c_vp]),
+    "iskv_cache_step_workspace_size": (c_sz, [c_i32, c_i32, c_i32, c_i32, c_i64]),
+    "iskv_cache_step": (c_i32, [ctypes.POINTER(ctypes.POINTER(IskvExactTable)),
+                                ctypes.POINTER(ctypes.POINTER(IskvLowRank)), c_i32, c_vp, c_i32,
+                                c_f32, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32), c_vp, c_sz,
+                                c_vp]),
     "iskv_reset": (c_i32, [ctypes.POINTER(IskvLowRank), c_vp]),
     "iskv_get_status": (c_i32, [ctypes.POINTER(IskvLowRank), ctypes.POINTER(c_i64),
                                 ctypes.POINTER(c_i64), ctypes.POINTER(c_i64),

@@ -8,6 +8,7 @@
 
 #include "iskv.h"
 #include "kernels.h"
+#include "policy.h"
 #include "profiling.h"
 #include "recon.h"
 #include "reorth.h"
@@ -102,6 +103,45 @@ AttnWsLayout attn_ws_layout(int32_t count, int32_t d, int32_t r, int64_t n_cap, 
   L.total = L.slices + (size_t)count * L.per_job;
   return L;
 }
+
+}  // namespace
+
+namespace {
+
+size_t elem_size(int32_t dtype) { return dtype == ISKV_F32 ? 4 : 2; }
+
+iskv_status check_table(const iskv_exact_table *t, const char *who) {
+  if (!t) return fail(ISKV_ERR_ARG, "%s: null table", who);
+  if (!t->rows || !t->pos || !t->live_host)
+    return fail(ISKV_ERR_ARG, "%s: null pointer in exact-row table", who);
+  if (!valid_dtype(t->dtype)) return fail(ISKV_ERR_ARG, "%s: bad table dtype", who);
+  if (!aligned(t->rows, 16) || !aligned(t->pos, 4))
+    return fail(ISKV_ERR_ARG, "%s: table rows must be 16-byte aligned", who);
+  if (t->d <= 0 || ((size_t)t->d * elem_size(t->dtype)) % 16)
+    return fail(ISKV_ERR_SHAPE, "%s: d * element size must be a multiple of 16 bytes", who);
+  if (t->window < 0 || t->block < 1 || t->reorth_rows < 0)
+    return fail(ISKV_ERR_SHAPE, "%s: need window >= 0, block >= 1, reorth_rows >= 0", who);
+  if (t->cap_e < 0 || t->cap_e >= (int64_t)1 << 31)
+    return fail(ISKV_ERR_SHAPE, "%s: cap_e out of range", who);
+  if (t->live_cap < (int64_t)t->window + t->block)
+    return fail(ISKV_ERR_SHAPE, "%s: live_cap must be >= window + block", who);
+  return ISKV_OK;
+}
+
+// Rows of the FIFO once position t is stored: live rows at or before t - window (the live rows are
+// ascending, so they are a prefix), counting t itself when the window is empty.
+int64_t pending_after(const iskv_exact_table *t, int64_t pos) {
+  const int64_t edge = pos - t->window;
+  int64_t lo = 0, hi = t->n_live;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi) >> 1;
+    if (t->live_host[mid] <= edge) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo + (pos <= edge ? 1 : 0);
+}
+
+static_assert(sizeof(AppendJob) <= 64 && sizeof(EvictJob) <= 64, "policy job sizes");
 
 }  // namespace
 
@@ -801,6 +841,232 @@ iskv_status iskv_select_prompt_blocks(const void *keys, int32_t k_dtype, int64_t
   cudaError_t e = launch_select(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "select");
   stage_mark(s, ST_SELECT);
+  return ISKV_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Cache policy
+size_t iskv_cache_prefill_workspace_size(int32_t init_window) {
+  (void)init_window;
+  return 256;  // an int64[4] scratch word: live-row count and error bits
+}
+
+iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dtype, int64_t L,
+                               const int32_t *protected_pos, int64_t n_protected,
+                               int32_t init_window, void *comp_rows, int32_t *comp_pos,
+                               int64_t *n_comp, void *ws, size_t ws_bytes, void *stream) {
+  const char *who = "iskv_cache_prefill";
+  g_last_error.clear();
+  iskv_status st = check_table(t, who);
+  if (st != ISKV_OK) return st;
+  if (!valid_dtype(x_dtype)) return fail(ISKV_ERR_ARG, "%s: bad X dtype", who);
+  if (!n_comp) return fail(ISKV_ERR_ARG, "%s: null n_comp", who);
+  if (L < 0 || L >= (int64_t)1 << 31) return fail(ISKV_ERR_SHAPE, "%s: L out of range", who);
+  if (L > 0 && (!X || !comp_rows || !comp_pos))
+    return fail(ISKV_ERR_ARG, "%s: null X / comp_rows / comp_pos", who);
+  if (!aligned(X, elem_size(x_dtype)) || !aligned(comp_rows, elem_size(x_dtype)) ||
+      !aligned(comp_pos, 4) || !aligned(protected_pos, 4))
+    return fail(ISKV_ERR_ARG, "%s: misaligned X / comp_rows / positions", who);
+  if (n_protected < 0 || n_protected > L)
+    return fail(ISKV_ERR_SHAPE, "%s: need 0 <= n_protected <= L", who);
+  if (n_protected > 0 && !protected_pos) return fail(ISKV_ERR_ARG, "%s: null protected_pos", who);
+  if (init_window < 0 || init_window > t->window)
+    return fail(ISKV_ERR_ARG, "%s: need 0 <= init_window <= window", who);
+  const int64_t w = init_window < L ? init_window : L;
+  if (n_protected + w > t->cap_e)
+    return fail(ISKV_ERR_CAPACITY, "%s: %lld protected + %lld window rows exceed cap_e = %lld", who,
+                (long long)n_protected, (long long)w, (long long)t->cap_e);
+  st = check_ws(ws, ws_bytes, iskv_cache_prefill_workspace_size(init_window), who);
+  if (st != ISKV_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int64_t *scal = static_cast<int64_t *>(ws);
+  PrefillArgs a;
+  a.X = X;
+  a.P = protected_pos;
+  a.rows = t->rows;
+  a.pos = t->pos;
+  a.comp = comp_rows;
+  a.comp_pos = comp_pos;
+  a.st = scal;
+  a.L = L;
+  a.n_p = n_protected;
+  a.w = w;
+  a.d = t->d;
+  a.x_dtype = x_dtype;
+  a.t_dtype = t->dtype;
+  int64_t hst[4] = {0, 0, 0, 0};
+  cudaError_t e = cudaMemsetAsync(scal, 0, sizeof hst, s);
+  if (e == cudaSuccess) e = launch_prefill_partition(a, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(hst, scal, sizeof hst, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && w > 0)
+    e = cudaMemcpyAsync(t->live_host, t->pos + n_protected, sizeof(int32_t) * (size_t)w,
+                        cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cache prefill");
+  const int64_t n_live = hst[0];
+  if ((hst[ISKV_META_STATUS] >> ISKV_ERR_ARG) & 1 || n_live < 0 || n_live > w)
+    return fail(ISKV_ERR_ARG, "%s: protected positions must be strictly ascending inside [0, L)",
+                who);
+  t->n_prot = n_protected;
+  t->n_live = n_live;
+  t->last = L - 1;
+  t->fold_rows = 0;
+  t->hist_rows = L - n_protected - n_live;
+  *n_comp = t->hist_rows;
+  if ((hst[ISKV_META_STATUS] >> ISKV_ERR_NONFINITE) & 1)
+    return fail(ISKV_ERR_NONFINITE, "%s: a finite row value overflows the fp16 table", who);
+  return ISKV_OK;
+}
+
+size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block,
+                                      int64_t n_cap) {
+  if (count < 1 || d < 1 || r_max < 1 || block < 1 || n_cap < 0) return 0;
+  size_t need = jobs_bytes(count, sizeof(AppendJob));
+  const size_t ev = jobs_bytes(count, sizeof(EvictJob));
+  const size_t fw = iskv_fold_workspace_size(count, d, r_max, block);
+  const size_t rw = iskv_reorth_workspace_size(count, d, r_max, n_cap);
+  if (ev > need) need = ev;
+  if (fw > need) need = fw;
+  if (rw > need) need = rw;
+  return need;
+}
+
+iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank *const *hists,
+                            int32_t count, const void *new_rows, int32_t row_dtype, float tau_rel,
+                            int32_t *folded, int32_t *reorthed, void *ws, size_t ws_bytes,
+                            void *stream) {
+  const char *who = "iskv_cache_step";
+  g_last_error.clear();
+  if (!tables || !hists || !new_rows) return fail(ISKV_ERR_ARG, "%s: null argument", who);
+  if (count < 1 || count > 4096) return fail(ISKV_ERR_SHAPE, "%s: count must be in [1, 4096]", who);
+  if (!valid_dtype(row_dtype)) return fail(ISKV_ERR_ARG, "%s: bad row dtype", who);
+  if (!(tau_rel >= 0.f)) return fail(ISKV_ERR_ARG, "%s: tau_rel must be >= 0", who);
+  if (!aligned(new_rows, elem_size(row_dtype))) return fail(ISKV_ERR_ARG, "%s: misaligned rows", who);
+  bool any_reorth = false;
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_status st = check_table(tables[i], who);
+    if (st != ISKV_OK) return st;
+    if ((st = check_handle(hists[i], who)) != ISKV_OK) return st;
+    const iskv_exact_table *T = tables[i], *T0 = tables[0];
+    if (T->d != T0->d || T->window != T0->window || T->block != T0->block || T->dtype != T0->dtype)
+      return fail(ISKV_ERR_SHAPE, "%s: tables must share d, window, block and dtype", who);
+    const iskv_lowrank *H = hists[i], *H0 = hists[0];
+    if (H->d != T0->d || H->r_max != H0->r_max || H->storage != H0->storage || H->n_cap != H0->n_cap)
+      return fail(ISKV_ERR_SHAPE, "%s: histories must have the tables' d and share r_max, storage, "
+                  "n_cap", who);
+    if (T->n_prot < 0 || T->n_live < 0 || T->hist_rows < 0 || T->last + 1 >= (int64_t)1 << 31)
+      return fail(ISKV_ERR_SHAPE, "%s: table %d: inconsistent host mirror", who, i);
+    if (T->n_prot + T->n_live + 1 > T->cap_e || T->n_live + 1 > T->live_cap)
+      return fail(ISKV_ERR_CAPACITY, "%s: table %d has no room for the new row", who, i);
+    if (T->reorth_rows > 0) any_reorth = true;
+  }
+  const iskv_exact_table *T0 = tables[0];
+  const int d = T0->d, b = T0->block, r = hists[0]->r_max;
+  const int64_t ncap = hists[0]->n_cap;
+  // The fold's and re-orthogonalisation's own argument checks, made before anything is launched.
+  if (b < 8 || b % 8 || b > 128 || b > d)
+    return fail(ISKV_ERR_SHAPE, "%s: need 8 <= block <= min(d, 128), block %% 8 == 0", who);
+  if (fold_residual_smem(d, b) > 200 * 1024)
+    return fail(ISKV_ERR_SHAPE, "%s: d = %d with block = %d exceeds the residual QR cluster", who,
+                d, b);
+  {
+    JacobiCfg jc;
+    if (!core_cfg(r, b, false, jc))
+      return fail(ISKV_ERR_SHAPE, "%s: r_max + block too large for the core SVD cluster", who);
+    if (any_reorth && !core_cfg(r, 0, true, jc))
+      return fail(ISKV_ERR_SHAPE, "%s: r_max too large for the dense core SVD", who);
+  }
+  const size_t need = iskv_cache_step_workspace_size(count, d, r, b, ncap);
+  iskv_status st = check_ws(ws, ws_bytes, need, who);
+  if (st != ISKV_OK) return st;
+
+  // The plan of the step, from the host mirror alone.
+  const size_t esz = elem_size(T0->dtype), rsz = elem_size(row_dtype);
+  std::vector<AppendJob> aj(count);
+  std::vector<int32_t> fold_idx, reorth_idx;
+  for (int32_t i = 0; i < count; ++i) {
+    const iskv_exact_table *T = tables[i];
+    const int64_t t = T->last + 1, slot = T->n_prot + T->n_live;
+    AppendJob &j = aj[i];
+    j.src = static_cast<const char *>(new_rows) + (size_t)i * d * rsz;
+    j.dst = static_cast<char *>(T->rows) + (size_t)slot * d * esz;
+    j.dst_pos = T->pos + slot;
+    j.meta = hists[i]->meta;
+    j.position = (int32_t)t;
+    j.pad_ = 0;
+    if (pending_after(T, t) >= b) {
+      if (T->hist_rows + b > ncap)
+        return fail(ISKV_ERR_CAPACITY, "%s: table %d: history has no room for a block (%lld + %d > "
+                    "%lld)", who, i, (long long)T->hist_rows, b, (long long)ncap);
+      fold_idx.push_back(i);
+      if (T->reorth_rows > 0 && T->fold_rows + b >= T->reorth_rows) reorth_idx.push_back(i);
+    }
+  }
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char *base = static_cast<char *>(ws);
+  AppendJob *daj = reinterpret_cast<AppendJob *>(base);
+  stage_begin(s);
+  cudaError_t e = upload_jobs(daj, aj.data(), sizeof(AppendJob) * count, s);
+  if (e == cudaSuccess) e = launch_cache_append(daj, count, d, row_dtype, T0->dtype, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cache step: append");
+  stage_mark(s, ST_CACHE_APPEND);
+  const int nf = (int)fold_idx.size();
+  if (nf > 0) {
+    std::vector<iskv_lowrank> fh(nf);
+    std::vector<const void *> F(nf);
+    std::vector<const int32_t *> fp(nf);
+    std::vector<EvictJob> ej(nf);
+    for (int k = 0; k < nf; ++k) {
+      const iskv_exact_table *T = tables[fold_idx[k]];
+      fh[k] = *hists[fold_idx[k]];
+      F[k] = static_cast<const char *>(T->rows) + (size_t)T->n_prot * d * esz;
+      fp[k] = T->pos + T->n_prot;
+      ej[k].rows = const_cast<void *>(F[k]);
+      ej[k].pos = T->pos + T->n_prot;
+      ej[k].keep = T->n_live + 1 - b;
+      ej[k].row_bytes = (int64_t)d * esz;
+      ej[k].shift = b;
+      ej[k].pad_ = 0;
+    }
+    st = iskv_fold_block_batched(fh.data(), nf, F.data(), T0->dtype, b, fp.data(), tau_rel, ws,
+                                 ws_bytes, stream);
+    if (st != ISKV_OK) return st;
+    EvictJob *dej = reinterpret_cast<EvictJob *>(base);
+    stage_begin(s);
+    e = upload_jobs(dej, ej.data(), sizeof(EvictJob) * nf, s);
+    if (e == cudaSuccess) e = launch_cache_evict(dej, nf, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cache step: evict");
+    stage_mark(s, ST_CACHE_EVICT);
+  }
+  const int nr = (int)reorth_idx.size();
+  if (nr > 0) {
+    std::vector<iskv_lowrank> rh(nr);
+    for (int k = 0; k < nr; ++k) rh[k] = *hists[reorth_idx[k]];
+    st = iskv_reorth(rh.data(), nr, ws, ws_bytes, stream);
+    if (st != ISKV_OK) return st;
+  }
+
+  // Host mirror.
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_exact_table *T = tables[i];
+    T->last += 1;
+    T->live_host[T->n_live++] = (int32_t)T->last;
+    if (folded) folded[i] = 0;
+    if (reorthed) reorthed[i] = 0;
+  }
+  for (int32_t i : fold_idx) {
+    iskv_exact_table *T = tables[i];
+    std::memmove(T->live_host, T->live_host + b, sizeof(int32_t) * (size_t)(T->n_live - b));
+    T->n_live -= b;
+    T->fold_rows += b;
+    T->hist_rows += b;
+    if (folded) folded[i] = 1;
+  }
+  for (int32_t i : reorth_idx) {
+    tables[i]->fold_rows = 0;
+    if (reorthed) reorthed[i] = 1;
+  }
   return ISKV_OK;
 }
 

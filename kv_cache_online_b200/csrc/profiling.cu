@@ -30,7 +30,8 @@ const char *kNames[ST_COUNT] = {
     "reorth.core_svd", "reorth.coord_rotate", "reorth.basis_rotate", "reconstruct.prepare",
     "reconstruct.compressed",
     "reconstruct.exact", "select",            "job_upload",        "attention.prepare",
-    "attention.scores", "attention.softmax",  "attention.values"};
+    "attention.scores", "attention.softmax",  "attention.values", "cache.append",
+    "cache.evict"};
 
 cudaEvent_t take_event() {
   if (!g_free.empty()) {

@@ -30,6 +30,8 @@ enum Stage {
   ST_ATTN_SCORES,
   ST_ATTN_SOFTMAX,
   ST_ATTN_VALUES,
+  ST_CACHE_APPEND,
+  ST_CACHE_EVICT,
   ST_COUNT
 };
 

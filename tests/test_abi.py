@@ -114,3 +114,58 @@ def test_python_binding_fails_loudly_without_library(tmp_path):
     from kv_cache_online_b200 import _lib as L
     with pytest.raises(RuntimeError, match="not found"):
         L.load(str(tmp_path / "missing.so"))
+
+
+def _fake_table(L, live, d=1024, window=128, block=64, cap_e=1024, dtype=1, base=0x80000):
+    return L.IskvExactTable(d, window, block, 256, dtype, 0, cap_e, base, base + 0x100000,
+                            ctypes.cast(live, ctypes.POINTER(ctypes.c_int32)), window + block,
+                            0, 0, -1, 0, 0)
+
+
+def test_cache_policy_host_side_errors():
+    """The cache-policy entry points refuse bad tables on the host and leave the mirror unchanged."""
+    L, lib = _lib()
+    live = (ctypes.c_int32 * 256)()
+    ws = ctypes.c_void_p(0x40000)
+    big = 1 << 40
+    X = ctypes.c_void_p(0x20000)
+    P = ctypes.c_void_p(0x30000)
+    n = ctypes.c_int64()
+    t = _fake_table(L, live)
+    # initial window longer than the window; protected + window rows beyond the capacity
+    assert lib.iskv_cache_prefill(ctypes.byref(t), X, 1, 1000, P, 10, 129, X, P, ctypes.byref(n),
+                                  ws, big, None) == 1
+    small = _fake_table(L, live, cap_e=100)
+    assert lib.iskv_cache_prefill(ctypes.byref(small), X, 1, 1000, P, 10, 128, X, P,
+                                  ctypes.byref(n), ws, big, None) == 4
+    # live_cap below window + block
+    bad = _fake_table(L, live)
+    bad.live_cap = 100
+    assert lib.iskv_cache_prefill(ctypes.byref(bad), X, 1, 1000, P, 10, 0, X, P, ctypes.byref(n),
+                                  ws, big, None) == 2
+
+    h = _fake_handle(L)
+    tp = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t))
+    hp = (ctypes.POINTER(L.IskvLowRank) * 1)(ctypes.pointer(h))
+    rows = ctypes.c_void_p(0x90000)
+    assert lib.iskv_cache_step(tp, hp, 0, rows, 1, 0.0, None, None, ws, big, None) == 2
+    # a full table
+    t.n_prot, t.n_live = 1000, 24
+    assert lib.iskv_cache_step(tp, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 4
+    # a fold is due (window 0: the new row makes 8 pending) but the history has no room
+    t2 = _fake_table(L, live, window=0, block=8)
+    for i in range(7):
+        live[i] = i
+    t2.n_live, t2.last, t2.hist_rows = 7, 6, 4090
+    tp2 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t2))
+    assert lib.iskv_cache_step(tp2, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 4
+    assert b"no room" in lib.iskv_last_error()
+    assert (t2.n_live, t2.last, t2.hist_rows) == (7, 6, 4090)
+    # a block the fold does not take; tables that disagree on d
+    t3 = _fake_table(L, live, block=12)
+    tp3 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t3))
+    assert lib.iskv_cache_step(tp3, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
+    ta, tb = _fake_table(L, live), _fake_table(L, live, d=512)
+    tp4 = (ctypes.POINTER(L.IskvExactTable) * 2)(ctypes.pointer(ta), ctypes.pointer(tb))
+    hp4 = (ctypes.POINTER(L.IskvLowRank) * 2)(ctypes.pointer(h), ctypes.pointer(h))
+    assert lib.iskv_cache_step(tp4, hp4, 2, rows, 1, 0.0, None, None, ws, big, None) == 2

@@ -1,0 +1,156 @@
+"""GPU parity of the cache policy (Section 3.1, Section 3.2, Algorithm 1 steps 5-8, Algorithm 3
+steps 1-6) against the oracle: the prefill partition bit for bit, then decode steps whose schedule
+(which tables fold or re-orthogonalise in which step), exact-row tables and history positions match
+exactly and whose factors, reconstruction and decode attention match within the fp32 / bf16
+tolerances."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import kv, np64, set_state, state, stored
+from oracle import attention as oatt
+from oracle import fold as of
+from oracle import policy as op
+from oracle import reconstruct as orec
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _protected(L, seed, frac=0.08, suffix=36):
+    g = np.random.Generator(np.random.PCG64(seed))
+    mask = g.random(L) < frac
+    mask[max(0, L - suffix):] = True
+    return np.flatnonzero(mask)
+
+
+def _widen(P, L, radius):
+    near = np.zeros(L, dtype=bool)
+    for p in P:
+        near[max(0, p - radius):min(L, p + radius + 1)] = True
+    return np.flatnonzero(near)
+
+
+@pytest.mark.parametrize("L,frac,init_window,xdt,tdt", [
+    (5000, 0.1, 128, torch.float32, torch.float32),
+    (5000, 0.1, 0, torch.bfloat16, torch.bfloat16),
+    (3000, 0.3, 100, torch.float32, torch.bfloat16),
+    (50, 0.2, 128, torch.bfloat16, torch.bfloat16),     # prompt shorter than the window
+    (700, 0.0, 64, torch.float32, torch.float32),       # nothing protected
+    (400, 1.0, 128, torch.float32, torch.float32),      # everything protected
+    (0, 0.0, 0, torch.float32, torch.float32),          # empty prompt
+])
+def test_prefill_partition(L, frac, init_window, xdt, tdt):
+    m = kv()
+    d = 256
+    g = np.random.Generator(np.random.PCG64(L + init_window))
+    X = torch.as_tensor(g.standard_normal((max(L, 1), d)), dtype=xdt, device="cuda")[:L].contiguous()
+    P = np.flatnonzero(g.random(L) < frac) if frac < 1 else np.arange(L)
+    t = m.ExactTable(d, L + 128, window=128, block=64, dtype=tdt)
+    comp_rows, comp_pos = m.cache_prefill(t, X, torch.as_tensor(P, dtype=torch.int32,
+                                                                 device="cuda"), init_window)
+    prot, live, comp = op.prefill_partition(L, P.tolist(), init_window)
+    assert (t.t.n_prot, t.t.n_live, t.t.last, t.t.hist_rows) == (len(prot), len(live), L - 1,
+                                                                  len(comp))
+    assert t.live_positions() == live
+    rows, pos = t.exact()
+    assert pos.cpu().tolist() == prot + live
+    assert torch.equal(rows, X[pos.long()].to(tdt))
+    assert comp_pos.cpu().tolist() == comp
+    assert torch.equal(comp_rows, X[comp_pos.long()])
+
+
+def test_prefill_rejects_unordered_protected_positions():
+    m = kv()
+    X = torch.zeros(100, 256, device="cuda")
+    t = m.ExactTable(256, 512, window=32, block=16, dtype=torch.float32)
+    with pytest.raises(m.IskvError, match="ascending"):
+        m.cache_prefill(t, X, torch.tensor([5, 3, 90], dtype=torch.int32, device="cuda"), 32)
+    with pytest.raises(m.IskvError, match="ascending"):
+        m.cache_prefill(t, X, torch.tensor([5, 100], dtype=torch.int32, device="cuda"), 32)
+
+
+def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36):
+    """Two sequences x (K, V) = four tables stepped together through T decode steps, against four
+    oracle runs started from the same stored prompt factors."""
+    sides = []
+    for s, L in enumerate(Ls):
+        PK = _protected(L, seed + s, suffix=suffix)
+        PV = _widen(PK, L, 4)
+        for kind, P, w0, ex in (("K", PK, 0, 1.1), ("V", PV, min(W, L), 0.7)):
+            X = stored(synth.lowrank_rows(L + T, d, ex, 0.02, seed=seed + 10 * s + len(sides)),
+                       storage)
+            sides.append(dict(kind=kind, L=L, P=P, w0=w0, X=X))
+    n_cap = max(L for L in Ls) + T
+    tabs, hists, refs = [], [], []
+    for sd in sides:
+        L = sd["L"]
+        Xd = torch.as_tensor(sd["X"], dtype=storage, device="cuda")
+        t = m.ExactTable(d, 1024, window=W, block=b, reorth_rows=R, dtype=storage)
+        comp_rows, comp_pos = m.cache_prefill(t, Xd[:L].contiguous(),
+                                              torch.as_tensor(sd["P"], dtype=torch.int32,
+                                                              device="cuda"), sd["w0"])
+        U0, s0, B0 = of.truncated_svd(sd["X"][comp_pos.cpu().numpy()], r)
+        U0, s0, B0 = stored(U0, storage), stored(s0, torch.float32), stored(B0, storage)
+        h = m.LowRankHistory(d, r, n_cap, storage=storage)
+        set_state(h, U0, s0, B0, comp_pos.cpu().numpy())
+        ref = op.run_decode(sd["X"][:L], sd["X"][L:], sd["P"], sd["w0"], W, b, r, R,
+                            init_history=(U0, s0, B0))
+        sd["Xd"] = Xd
+        tabs.append(t)
+        hists.append(h)
+        refs.append(ref)
+    for i in range(T):
+        rows = torch.stack([sd["Xd"][sd["L"] + i] for sd in sides]).contiguous()
+        folded, reorthed = m.cache_step(tabs, hists, rows)
+        for k, ref in enumerate(refs):
+            acts = ref["steps"][i]
+            assert folded[k] == any(a[0] == "fold" for a in acts), (i, k)
+            assert reorthed[k] == any(a[0] == "reorth" for a in acts), (i, k)
+    for sd, t, h, ref in zip(sides, tabs, hists, refs):
+        U, s, B, pos, (k, n, _, st) = state(h)
+        Uo, so, Bo, poso = ref["history"]
+        assert st == 0
+        assert (k, n) == (so.shape[0], poso.shape[0])
+        np.testing.assert_array_equal(pos, poso)
+        assert of.rel_fro(of.low_rank_product(U, s, B), of.low_rank_product(Uo, so, Bo)) < tol
+        rows, epos = t.exact()
+        assert epos.cpu().tolist() == ref["exact"][1].tolist()
+        np.testing.assert_array_equal(np64(rows), ref["exact"][0])
+        assert t.live_positions() == ref["side"].live
+        n_total = sd["L"] + T
+        out = m.reconstruct(h, rows, epos, n_total, d // 128, 128, sd["kind"] == "K", 500000.0,
+                            out_dtype=torch.float32)
+        want = orec.reconstruct(Uo, so, Bo, poso, ref["exact"][0], ref["exact"][1], n_total,
+                                d // 128, 128, sd["kind"] == "K", 500000.0)
+        assert of.rel_fro(np64(out), want) < tol
+    return sides, tabs, hists, refs
+
+
+def test_decode_policy_fp32():
+    m = kv()
+    d, T = 256, 130
+    # An 8-token suffix leaves unprotected rows in the value window at prefill.
+    sides, tabs, hists, refs = _run(m, d=d, r=32, b=16, W=24, R=32, Ls=(300, 180), T=T,
+                                    storage=torch.float32, seed=70, tol=1e-4, suffix=8)
+    assert tabs[1].t.n_prot > 0 and refs[1]["side"].compressed
+    # Decode attention of sequence 0 straight from its K and V tables (Algorithm 3 steps 7-9).
+    g = np.random.Generator(np.random.PCG64(71))
+    q = stored(40 * g.standard_normal((8, 128)) / np.sqrt(128), torch.float32)
+    n_total = sides[0]["L"] + T
+    kr, kp = tabs[0].exact()
+    vr, vp = tabs[1].exact()
+    out = m.decode_attention(hists[0], hists[1], kr, kp, vr, vp, n_total,
+                             torch.as_tensor(q, dtype=torch.float32, device="cuda"), 2, 128)
+    rk, rv = refs[0], refs[1]
+    want = oatt.decode_attention(rk["history"], rv["history"], rk["exact"][0], rk["exact"][1],
+                                 rv["exact"][0], rv["exact"][1], n_total, q, 2, 128)
+    assert float(np.linalg.norm(np64(out) - want) / np.linalg.norm(want)) < 1e-4
+
+
+def test_decode_policy_bf16_model_width():
+    """d = 1024 (8 KV heads x 128), r = 64, b = 64, W = 128, re-orthogonalisation every 128 rows."""
+    m = kv()
+    _run(m, d=1024, r=64, b=64, W=128, R=128, Ls=(600, 450), T=300, storage=torch.bfloat16,
+         seed=90, tol=2e-2)
