@@ -1,5 +1,5 @@
 """Oracle: the cache policy -- which rows stay exact and when pending rows are folded (iS-KV reading
-notes, Section 3.1, Section 3.2, Algorithm 1 steps 5-8 and Algorithm 3 steps 1-6).
+notes, Section 3.1, Section 3.2, Algorithm 1 steps 5-9 and Algorithm 3 steps 1-6).
 
 TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
 
@@ -21,11 +21,13 @@ Readings where the pages leave a step open:
   once (as protected) and stays exact when it leaves; an unprotected one moves to the FIFO;
 * a decode row is never protected (the protected set is fixed at prefill);
 * the initial window is no longer than ``W`` (``init_window <= W``), so at most one row joins the FIFO
-  per decode step and a fold always takes exactly the ``b`` rows that are pending;
+  per decode step and a fold (a refit) takes exactly the ``b`` (``r_V``) rows that are pending;
 * re-orthogonalisation runs in the step whose fold brings the count to ``reorth_rows``; the count
   then restarts from zero;
-* the value side's first refit (Algorithm 3 step 3) is not part of this module: it is written for a
-  policy without it (regular block folds from the first full block).
+* the value side's first refit (Algorithm 3 step 3, ``refit_rows`` = r_V > 0): the FIFO grows until
+  ``refit_rows`` rows are pending; those rows, appended to the rows the history represents, are
+  re-factored by a rank-r truncated SVD; regular ``block`` folds follow. The refit's rows do not
+  count toward ``reorth_rows`` (Section 4.4 excludes the value side's first refactorisation).
 """
 
 from __future__ import annotations
@@ -68,6 +70,8 @@ class Side:
     last: int                  # last stored position
     fold_rows: int = 0
     compressed: list = field(default_factory=list)   # positions merged by decode-time folds
+    refit_rows: int = 0        # r_V for the value side's first refit; 0 = none
+    refit_done: bool = True
 
     def pending(self):
         """The FIFO: live rows whose position has left the window ``(last - W, last]``."""
@@ -75,19 +79,23 @@ class Side:
         return [p for p in self.live if p <= edge]
 
 
-def new_side(L: int, protected, init_window: int, window: int, block: int, reorth_rows: int):
-    """State after Algorithm 1 (steps 5-8) and the positions the prompt SVD compresses."""
+def new_side(L: int, protected, init_window: int, window: int, block: int, reorth_rows: int,
+             refit_rows: int = 0):
+    """State after Algorithm 1 (steps 5-9) and the positions the prompt SVD compresses."""
     if not 0 <= int(init_window) <= int(window):
         raise ValueError("need 0 <= init_window <= window")
     prot, live, comp = prefill_partition(L, protected, init_window)
-    return Side(int(window), int(block), int(reorth_rows), prot, live, int(L) - 1), comp
+    side = Side(int(window), int(block), int(reorth_rows), prot, live, int(L) - 1,
+                refit_rows=int(refit_rows), refit_done=int(refit_rows) == 0)
+    return side, comp
 
 
 def append(side: Side, position: int):
-    """Algorithm 3 steps 1-2 and the scheduling of steps 4-5 for one new row at ``position``.
+    """Algorithm 3 steps 1-2 and the scheduling of steps 3-5 for one new row at ``position``.
 
-    Returns the actions of this step: ``("fold", positions)`` for the block to merge and
-    ``("reorth",)`` when the merged-row count reaches ``reorth_rows``.
+    Returns the actions of this step: ``("refit", positions)`` for the value side's first refit,
+    ``("fold", positions)`` for the block to merge and ``("reorth",)`` when the merged-row count
+    reaches ``reorth_rows``.
     """
     if position != side.last + 1:
         raise ValueError("decode rows arrive one position at a time")
@@ -95,6 +103,14 @@ def append(side: Side, position: int):
     side.live.append(position)
     actions = []
     pend = side.pending()
+    if not side.refit_done:
+        if len(pend) >= side.refit_rows:
+            blk = pend[: side.refit_rows]
+            side.live = side.live[side.refit_rows:]
+            side.compressed.extend(blk)
+            side.refit_done = True
+            actions.append(("refit", blk))
+        return actions
     if len(pend) >= side.block:
         blk = pend[: side.block]
         side.live = side.live[side.block:]
@@ -113,8 +129,17 @@ def exact_positions(side: Side):
     return list(side.prot) + list(side.live)
 
 
+def refit(U, sigma, B, F, r: int):
+    """Algorithm 3 step 3: the rank-``r`` truncated SVD of the rows the history represents followed
+    by the rows ``F``. Returns ``(U, sigma, B)``."""
+    F = np.asarray(F, dtype=np.float64)
+    X = np.concatenate([_fold.low_rank_product(U, sigma, B), F]) if np.size(U) else F
+    return _fold.truncated_svd(X, r)
+
+
 def run_decode(prompt_rows, decode_rows, protected, init_window: int, window: int, block: int,
-               r: int, reorth_rows: int, tau_rel: float = 0.0, init_history=None):
+               r: int, reorth_rows: int, tau_rel: float = 0.0, init_history=None,
+               refit_rows: int = 0):
     """Algorithm 1 then Algorithm 3 steps 1-6 for one side, with the row data.
 
     ``init_history`` = ``(U, sigma, B)`` for the compressed prompt rows (in ``comp`` order); when
@@ -125,7 +150,7 @@ def run_decode(prompt_rows, decode_rows, protected, init_window: int, window: in
     Xp = np.asarray(prompt_rows, dtype=np.float64)
     Xd = np.asarray(decode_rows, dtype=np.float64)
     L, d = Xp.shape
-    side, comp = new_side(L, protected, init_window, window, block, reorth_rows)
+    side, comp = new_side(L, protected, init_window, window, block, reorth_rows, refit_rows)
     if init_history is None:
         if comp:
             U, sigma, B = _fold.truncated_svd(Xp[comp], r)
@@ -141,10 +166,13 @@ def run_decode(prompt_rows, decode_rows, protected, init_window: int, window: in
         rows[t] = Xd[i]
         acts = append(side, t)
         for a in acts:
-            if a[0] == "fold":
+            if a[0] in ("fold", "refit"):
                 F = np.stack([rows[p] for p in a[1]])
-                res = _fold.fold_block(U, sigma, B, F, r, tau_rel)
-                U, sigma, B = res.U, res.sigma, res.B
+                if a[0] == "fold":
+                    res = _fold.fold_block(U, sigma, B, F, r, tau_rel)
+                    U, sigma, B = res.U, res.sigma, res.B
+                else:
+                    U, sigma, B = refit(U, sigma, B, F, r)
                 hpos.extend(a[1])
                 for p in a[1]:
                     del rows[p]

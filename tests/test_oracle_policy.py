@@ -24,14 +24,14 @@ def _golden():
 @pytest.mark.parametrize("case", _golden(), ids=lambda c: c["name"][:6])
 def test_hand_worked_schedule(case):
     side, comp = op.new_side(case["L"], case["protected"], case["init_window"], case["window"],
-                             case["block"], case["reorth_rows"])
+                             case["block"], case["reorth_rows"], case.get("refit_rows", 0))
     assert side.prot == case["prefill"]["prot"]
     assert side.live == case["prefill"]["live"]
     assert comp == case["prefill"]["comp"]
     for i in range(case["decode_steps"]):
         t = case["L"] + i
         acts = op.append(side, t)
-        assert [list(a[:1]) + [list(a[1])] if a[0] == "fold" else list(a) for a in acts] == \
+        assert [list(a[:1]) + [list(a[1])] if len(a) > 1 else list(a) for a in acts] == \
             case["steps"][str(t)], t
     assert op.exact_positions(side) == case["final"]["exact"]
     assert comp + side.compressed == case["final"]["history"]
@@ -76,20 +76,26 @@ def test_partition_invariants(seed):
     b = int(g.choice([1, 2, 8, 16]))
     w0 = int(g.integers(0, W + 1))
     R = int(g.choice([0, b, 3 * b, 5 * b + 1]))
+    F = int(g.choice([0, b, 2 * b, 3]))
     P = np.flatnonzero(g.random(L) < 0.2).tolist()
-    side, comp = op.new_side(L, P, w0, W, b, R)
+    side, comp = op.new_side(L, P, w0, W, b, R, F)
+    n_refit = 0
     n_folds = n_reorth = 0
     for t in range(L, L + 400):
         acts = op.append(side, t)
         for a in acts:
-            if a[0] == "fold":
-                n_folds += 1
+            if a[0] in ("fold", "refit"):
                 blk = a[1]
-                assert len(blk) == b and blk == sorted(blk)
+                assert len(blk) == (b if a[0] == "fold" else F) and blk == sorted(blk)
                 assert all(p not in P and p <= t - W for p in blk)
+                if a[0] == "fold":
+                    assert n_refit == (1 if F else 0)        # the refit comes first
+                    n_folds += 1
+                else:
+                    n_refit += 1
             else:
                 n_reorth += 1
-        assert len(side.pending()) < b
+        assert len(side.pending()) < (b if side.refit_done else F)
         exact = set(op.exact_positions(side))
         everything = sorted(list(exact) + comp + side.compressed)
         assert everything == list(range(t + 1))                          # a partition of 0..t
@@ -116,6 +122,37 @@ def test_rank_deficient_rows_are_recovered():
     np.testing.assert_array_equal(rows, X[epos])
     full = orec.reconstruct(U, s, B, pos, rows, epos, L + T, 1, d, False, 500000.0)
     np.testing.assert_allclose(full, X, atol=1e-9)
+
+
+def test_refit_of_an_empty_history_is_the_untruncated_block_stream():
+    """Algorithm 3 step 3 with nothing compressed yet (a short prompt, fully protected): the rank-r
+    SVD of the first r_V pending rows equals folding them in blocks with rank budget r >= r_V, since
+    no fold then truncates. This is how the device carries out the refit."""
+    d, b, r, rv = 40, 4, 16, 12
+    X = synth.lowrank_rows(rv, d, 0.7, 0.05, seed=21)
+    U, s, B = op.refit(*of.empty_history(d), X, r)
+    Uf, sf, Bf, _ = of.fold_stream(X, b, r)
+    np.testing.assert_allclose(s, sf, rtol=1e-12)
+    np.testing.assert_allclose(of.low_rank_product(U, s, B), of.low_rank_product(Uf, sf, Bf),
+                               atol=1e-12)
+    np.testing.assert_allclose(of.low_rank_product(U, s, B), X, atol=1e-12)
+
+
+def test_refit_keeps_history_rows_then_new_rows():
+    """The refit factors the history's rows followed by the new rows: with enough rank both come
+    back exactly, in that order."""
+    d = 30
+    g = synth.rng(22)
+    basis = g.standard_normal((4, d))
+    Xh = g.standard_normal((20, 4)) @ basis
+    F = g.standard_normal((6, 4)) @ basis
+    Uh, sh, Bh = of.truncated_svd(Xh, 4)
+    U, s, B = op.refit(Uh, sh, Bh, F, 8)
+    np.testing.assert_allclose(of.low_rank_product(U, s, B), np.concatenate([Xh, F]), atol=1e-10)
+    # rank 1: the best rank-1 approximation of the stacked rows (Eckart-Young)
+    U1, s1, B1 = op.refit(Uh, sh, Bh, F, 1)
+    sv = np.linalg.svd(np.concatenate([Xh, F]), compute_uv=False)
+    assert s1[0] == pytest.approx(sv[0], rel=1e-12)
 
 
 def test_argument_errors():
