@@ -280,8 +280,12 @@ iskv_status iskv_select_prompt_blocks_noalloc(const void *keys, int32_t k_dtype,
  * protected position inside it is stored once, as protected, and stays exact when it leaves; decode
  * rows are never protected; the window at prefill is no longer than W (empty for keys by
  * Algorithm 1 step 5, the last min(W, L) prompt positions for values), so at most one row joins
- * the FIFO per decode step. The value side's first refit (Algorithm 3 step 3) is not implemented:
- * both sides fold regular blocks from the first full one.
+ * the FIFO per decode step. The value side's first refit (Algorithm 3 step 3; refit_rows = r_V > 0)
+ * waits until refit_rows rows are pending and re-factors them, after the rows the history holds, by
+ * a rank-r_V SVD; its rows do not count toward reorth_rows (Section 4.4). The device carries out the
+ * refit of an EMPTY history (the prompt's values all protected, as with short prompts): there the
+ * rank-r_V SVD of the pending rows equals folding them block by block with no truncation
+ * (refit_rows <= r_max, a multiple of block). The refit of a non-empty history is not implemented.
  *
  * Exact-row table (device, caller-owned):
  *   rows [cap_e][d]  dtype; rows 0 .. n_prot-1 are the protected rows in ascending position, rows
@@ -294,7 +298,7 @@ iskv_status iskv_select_prompt_blocks_noalloc(const void *keys, int32_t k_dtype,
  * Host mirror (maintained by the library; the caller sets the first block of fields and live_host /
  * live_cap, then lets iskv_cache_prefill() fill the rest):
  *   live_host [live_cap]  HOST int32: positions of the live rows, ascending; live_cap >=
- *                         window + block.
+ *                         window + max(block, refit_rows).
  *   n_prot, n_live, last  counts and the last stored position (prompt length - 1 after prefill).
  *   fold_rows             rows merged by folds since the last re-orthogonalisation.
  *   hist_rows             rows of the side's history (prefill sets it to the compressed prompt
@@ -308,7 +312,7 @@ typedef struct {
   int32_t block;       /* b: rows per fold, as iskv_fold_block() accepts                    */
   int32_t reorth_rows; /* re-orthogonalise after this many folded rows; 0 = never           */
   int32_t dtype;       /* iskv_dtype of rows                                                */
-  int32_t reserved;
+  int32_t refit_rows;  /* r_V: rows of the value side's first refit; 0 = no refit           */
   int64_t cap_e;       /* row capacity of rows / pos                                        */
   void *rows;
   int32_t *pos;
@@ -319,6 +323,7 @@ typedef struct {
   int64_t last;
   int64_t fold_rows;
   int64_t hist_rows;
+  int64_t refit_done;  /* 1 once the first refit has run (or when refit_rows == 0)           */
 } iskv_exact_table;
 
 /*
@@ -330,7 +335,8 @@ typedef struct {
  * the exact-row table (converted to t->dtype), and every other row, in ascending position, into
  * comp_rows [L][d] (x_dtype) with comp_pos [L]: the rows the prompt's truncated SVD compresses
  * (Algorithm 1 step 7; that SVD itself is not part of the library). Sets the host mirror
- * (n_prot = n_protected, n_live, live_host, last = L - 1, fold_rows = 0, hist_rows = *n_comp) and
+ * (n_prot = n_protected, n_live, live_host, last = L - 1, fold_rows = 0, hist_rows = *n_comp,
+ * refit_done = (refit_rows == 0)) and
  * *n_comp (host). The caller then puts the compressed rows' factors in the side's history, with
  * their positions comp_pos in its position table.
  * SYNCHRONOUS: waits for the stream, because the mirror needs the live positions. Errors:
@@ -353,13 +359,16 @@ iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dty
  * (iskv_fold_block_batched over every table that folds, with tau_rel), their positions join the
  * history's position table and their exact copies leave the table; when a table's folded rows
  * reach reorth_rows, its history is re-orthogonalised (iskv_reorth) in the same step and the count
- * restarts. All tables share d, window, block and dtype; the histories share d, r_max, storage
- * and n_cap, as the batched fold and re-orthogonalisation require. folded / reorthed (host
- * [count], may be NULL) receive 1 where a table folded / re-orthogonalised. Stream-ordered; the host
- * mirror is updated at once. Errors (nothing launched, no table changed): ISKV_ERR_ARG,
- * ISKV_ERR_SHAPE (mixed table shapes, a history whose d differs, a block the fold does not take),
+ * restarts. A table whose first refit is still to come waits for refit_rows pending rows instead,
+ * then folds all of them, block by block, into its (empty) history. All tables share d, window,
+ * block and dtype; the histories share d, r_max, storage and n_cap, as the batched fold and
+ * re-orthogonalisation require. folded / reorthed (host [count], may be NULL) receive 1 where a
+ * table folded a block (2 where it ran its first refit) / re-orthogonalised. Stream-ordered; the
+ * host mirror is updated at once. Errors (nothing launched, no table changed): ISKV_ERR_ARG,
+ * ISKV_ERR_SHAPE (mixed table shapes, a history whose d differs, a block the fold does not take, a
+ * refit that comes due on a non-empty history or with refit_rows > r_max),
  * ISKV_ERR_CAPACITY (a table without room for the new row, or a history without room for the
- * block: hist_rows + block > n_cap), ISKV_ERR_WORKSPACE; ISKV_ERR_CUDA when a launch fails.
+ * block or the refit: hist_rows + block > n_cap), ISKV_ERR_WORKSPACE; ISKV_ERR_CUDA when a launch fails.
  */
 size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block,
                                       int64_t n_cap);

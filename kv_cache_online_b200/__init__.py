@@ -344,14 +344,15 @@ class ExactTable:
     ``self.t`` (an ``IskvExactTable``)."""
 
     def __init__(self, d: int, cap_e: int, window: int = 128, block: int = 64,
-                 reorth_rows: int = 256, dtype=torch.bfloat16, device="cuda"):
+                 reorth_rows: int = 256, dtype=torch.bfloat16, device="cuda", refit_rows: int = 0):
         self.rows = torch.zeros(max(int(cap_e), 1), int(d), dtype=dtype, device=device)
         self.pos = torch.full((max(int(cap_e), 1),), -1, dtype=torch.int32, device=device)
-        self.live = (ctypes.c_int32 * (int(window) + int(block)))()
-        self.t = IskvExactTable(int(d), int(window), int(block), int(reorth_rows), _DT[dtype], 0,
-                                int(cap_e), _ptr(self.rows), _ptr(self.pos),
+        live_cap = int(window) + max(int(block), int(refit_rows))
+        self.live = (ctypes.c_int32 * live_cap)()
+        self.t = IskvExactTable(int(d), int(window), int(block), int(reorth_rows), _DT[dtype],
+                                int(refit_rows), int(cap_e), _ptr(self.rows), _ptr(self.pos),
                                 ctypes.cast(self.live, ctypes.POINTER(ctypes.c_int32)),
-                                int(window) + int(block), 0, 0, -1, 0, 0)
+                                live_cap, 0, 0, -1, 0, 0, int(refit_rows) == 0)
 
     @property
     def n_exact(self) -> int:
@@ -395,8 +396,9 @@ def cache_step_workspace_size(count, d, r_max, block, n_cap) -> int:
 
 
 def cache_step(tables, hists, new_rows, tau_rel: float = 0.0, ws=None, stream=None):
-    """Algorithm 3 steps 1-2 and 4-6 for every (table, history) pair: ``new_rows`` (count, d) holds
-    each table's row for its next position. Returns ``(folded, reorthed)`` lists of bools."""
+    """Algorithm 3 steps 1-6 for every (table, history) pair: ``new_rows`` (count, d) holds each
+    table's row for its next position. Returns ``(folded, reorthed)``: per table 0, 1 (a block
+    fold) or 2 (the first refit), and a bool."""
     lib = _lib.load()
     n = len(tables)
     if n == 0 or len(hists) != n:
@@ -415,7 +417,7 @@ def cache_step(tables, hists, new_rows, tau_rel: float = 0.0, ws=None, stream=No
     _lib.check(lib.iskv_cache_step(tp, hp, n, new_rows.data_ptr(), _dt(new_rows), float(tau_rel),
                                    folded, reorthed, w.data_ptr(), w.numel(), _stream(stream)),
                "cache_step")
-    return [bool(x) for x in folded], [bool(x) for x in reorthed]
+    return [int(x) for x in folded], [bool(x) for x in reorthed]
 
 
 # ------------------------------------------------------------------------------------------------

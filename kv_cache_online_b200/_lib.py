@@ -29,10 +29,10 @@ class IskvExactTable(ctypes.Structure):
     """Mirror of ``iskv_exact_table``."""
 
     _fields_ = [("d", c_i32), ("window", c_i32), ("block", c_i32), ("reorth_rows", c_i32),
-                ("dtype", c_i32), ("reserved", c_i32), ("cap_e", c_i64), ("rows", c_vp),
+                ("dtype", c_i32), ("refit_rows", c_i32), ("cap_e", c_i64), ("rows", c_vp),
                 ("pos", c_vp), ("live_host", ctypes.POINTER(c_i32)), ("live_cap", c_i64),
                 ("n_prot", c_i64), ("n_live", c_i64), ("last", c_i64), ("fold_rows", c_i64),
-                ("hist_rows", c_i64)]
+                ("hist_rows", c_i64), ("refit_done", c_i64)]
 
 
 # name -> (restype, argtypes)

@@ -119,12 +119,16 @@ iskv_status check_table(const iskv_exact_table *t, const char *who) {
     return fail(ISKV_ERR_ARG, "%s: table rows must be 16-byte aligned", who);
   if (t->d <= 0 || ((size_t)t->d * elem_size(t->dtype)) % 16)
     return fail(ISKV_ERR_SHAPE, "%s: d * element size must be a multiple of 16 bytes", who);
-  if (t->window < 0 || t->block < 1 || t->reorth_rows < 0)
-    return fail(ISKV_ERR_SHAPE, "%s: need window >= 0, block >= 1, reorth_rows >= 0", who);
+  if (t->window < 0 || t->block < 1 || t->reorth_rows < 0 || t->refit_rows < 0)
+    return fail(ISKV_ERR_SHAPE, "%s: need window >= 0, block >= 1, reorth_rows >= 0, "
+                "refit_rows >= 0", who);
+  if (t->refit_rows % t->block)
+    return fail(ISKV_ERR_SHAPE, "%s: refit_rows must be a multiple of block", who);
   if (t->cap_e < 0 || t->cap_e >= (int64_t)1 << 31)
     return fail(ISKV_ERR_SHAPE, "%s: cap_e out of range", who);
-  if (t->live_cap < (int64_t)t->window + t->block)
-    return fail(ISKV_ERR_SHAPE, "%s: live_cap must be >= window + block", who);
+  const int64_t fifo = t->block > t->refit_rows ? t->block : t->refit_rows;
+  if (t->live_cap < (int64_t)t->window + fifo)
+    return fail(ISKV_ERR_SHAPE, "%s: live_cap must be >= window + max(block, refit_rows)", who);
   return ISKV_OK;
 }
 
@@ -912,6 +916,7 @@ iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dty
   t->last = L - 1;
   t->fold_rows = 0;
   t->hist_rows = L - n_protected - n_live;
+  t->refit_done = t->refit_rows > 0 ? 0 : 1;
   *n_comp = t->hist_rows;
   if ((hst[ISKV_META_STATUS] >> ISKV_ERR_NONFINITE) & 1)
     return fail(ISKV_ERR_NONFINITE, "%s: a finite row value overflows the fp16 table", who);
@@ -984,6 +989,8 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
   const size_t esz = elem_size(T0->dtype), rsz = elem_size(row_dtype);
   std::vector<AppendJob> aj(count);
   std::vector<int32_t> fold_idx, reorth_idx;
+  std::vector<int32_t> fold_rows(count, 0);  // rows this step folds per table (b, or refit_rows)
+  int32_t passes = 0;                        // block folds in this step: the longest refit / b
   for (int32_t i = 0; i < count; ++i) {
     const iskv_exact_table *T = tables[i];
     const int64_t t = T->last + 1, slot = T->n_prot + T->n_live;
@@ -994,12 +1001,21 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
     j.meta = hists[i]->meta;
     j.position = (int32_t)t;
     j.pad_ = 0;
-    if (pending_after(T, t) >= b) {
-      if (T->hist_rows + b > ncap)
+    const bool refit = !T->refit_done;
+    const int32_t rows = refit ? T->refit_rows : b;
+    if (pending_after(T, t) >= rows) {
+      if (T->hist_rows + rows > ncap)
         return fail(ISKV_ERR_CAPACITY, "%s: table %d: history has no room for a block (%lld + %d > "
-                    "%lld)", who, i, (long long)T->hist_rows, b, (long long)ncap);
+                    "%lld)", who, i, (long long)T->hist_rows, rows, (long long)ncap);
+      if (refit && (T->hist_rows != 0 || rows > r))
+        return fail(ISKV_ERR_SHAPE, "%s: table %d: the first refit is carried out for an empty "
+                    "history and refit_rows <= r_max only (history rows %lld, refit_rows %d)", who,
+                    i, (long long)T->hist_rows, rows);
       fold_idx.push_back(i);
-      if (T->reorth_rows > 0 && T->fold_rows + b >= T->reorth_rows) reorth_idx.push_back(i);
+      fold_rows[i] = rows;
+      if (rows / b > passes) passes = rows / b;
+      if (!refit && T->reorth_rows > 0 && T->fold_rows + b >= T->reorth_rows)
+        reorth_idx.push_back(i);
     }
   }
 
@@ -1013,25 +1029,34 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
   stage_mark(s, ST_CACHE_APPEND);
   const int nf = (int)fold_idx.size();
   if (nf > 0) {
-    std::vector<iskv_lowrank> fh(nf);
-    std::vector<const void *> F(nf);
-    std::vector<const int32_t *> fp(nf);
     std::vector<EvictJob> ej(nf);
     for (int k = 0; k < nf; ++k) {
       const iskv_exact_table *T = tables[fold_idx[k]];
-      fh[k] = *hists[fold_idx[k]];
-      F[k] = static_cast<const char *>(T->rows) + (size_t)T->n_prot * d * esz;
-      fp[k] = T->pos + T->n_prot;
-      ej[k].rows = const_cast<void *>(F[k]);
+      ej[k].rows = static_cast<char *>(T->rows) + (size_t)T->n_prot * d * esz;
       ej[k].pos = T->pos + T->n_prot;
-      ej[k].keep = T->n_live + 1 - b;
+      ej[k].keep = T->n_live + 1 - fold_rows[fold_idx[k]];
       ej[k].row_bytes = (int64_t)d * esz;
-      ej[k].shift = b;
+      ej[k].shift = fold_rows[fold_idx[k]];
       ej[k].pad_ = 0;
     }
-    st = iskv_fold_block_batched(fh.data(), nf, F.data(), T0->dtype, b, fp.data(), tau_rel, ws,
-                                 ws_bytes, stream);
-    if (st != ISKV_OK) return st;
+    // Pass j folds the j-th block of the FIFO of every table that folds that many rows: regular
+    // folds take pass 0 only, a refit of refit_rows rows takes passes 0 .. refit_rows / b - 1.
+    for (int32_t j = 0; j < passes; ++j) {
+      std::vector<iskv_lowrank> fh;
+      std::vector<const void *> F;
+      std::vector<const int32_t *> fp;
+      for (int32_t i : fold_idx) {
+        if (fold_rows[i] / b <= j) continue;
+        const iskv_exact_table *T = tables[i];
+        const int64_t row0 = T->n_prot + (int64_t)j * b;
+        fh.push_back(*hists[i]);
+        F.push_back(static_cast<const char *>(T->rows) + (size_t)row0 * d * esz);
+        fp.push_back(T->pos + row0);
+      }
+      st = iskv_fold_block_batched(fh.data(), (int32_t)fh.size(), F.data(), T0->dtype, b,
+                                   fp.data(), tau_rel, ws, ws_bytes, stream);
+      if (st != ISKV_OK) return st;
+    }
     EvictJob *dej = reinterpret_cast<EvictJob *>(base);
     stage_begin(s);
     e = upload_jobs(dej, ej.data(), sizeof(EvictJob) * nf, s);
@@ -1057,11 +1082,17 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
   }
   for (int32_t i : fold_idx) {
     iskv_exact_table *T = tables[i];
-    std::memmove(T->live_host, T->live_host + b, sizeof(int32_t) * (size_t)(T->n_live - b));
-    T->n_live -= b;
-    T->fold_rows += b;
-    T->hist_rows += b;
-    if (folded) folded[i] = 1;
+    const int32_t rows = fold_rows[i];
+    std::memmove(T->live_host, T->live_host + rows, sizeof(int32_t) * (size_t)(T->n_live - rows));
+    T->n_live -= rows;
+    T->hist_rows += rows;
+    if (T->refit_done) {
+      T->fold_rows += rows;
+      if (folded) folded[i] = 1;
+    } else {
+      T->refit_done = 1;  // the refit does not count toward reorth_rows
+      if (folded) folded[i] = 2;
+    }
   }
   for (int32_t i : reorth_idx) {
     tables[i]->fold_rows = 0;

@@ -119,7 +119,7 @@ def test_python_binding_fails_loudly_without_library(tmp_path):
 def _fake_table(L, live, d=1024, window=128, block=64, cap_e=1024, dtype=1, base=0x80000):
     return L.IskvExactTable(d, window, block, 256, dtype, 0, cap_e, base, base + 0x100000,
                             ctypes.cast(live, ctypes.POINTER(ctypes.c_int32)), window + block,
-                            0, 0, -1, 0, 0)
+                            0, 0, -1, 0, 0, 1)
 
 
 def test_cache_policy_host_side_errors():
@@ -165,6 +165,19 @@ def test_cache_policy_host_side_errors():
     t3 = _fake_table(L, live, block=12)
     tp3 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t3))
     assert lib.iskv_cache_step(tp3, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
+    # a refit that is not a multiple of the block; a refit due on a non-empty history
+    t5 = _fake_table(L, live, window=0, block=8)
+    t5.refit_rows, t5.refit_done, t5.live_cap = 12, 0, 12
+    tp5 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t5))
+    assert lib.iskv_cache_step(tp5, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
+    t6 = _fake_table(L, live, window=0, block=8)
+    t6.refit_rows, t6.refit_done, t6.live_cap = 16, 0, 16
+    for i in range(15):
+        live[i] = i
+    t6.n_live, t6.last, t6.hist_rows = 15, 14, 100
+    tp6 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t6))
+    assert lib.iskv_cache_step(tp6, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
+    assert b"empty" in lib.iskv_last_error()
     ta, tb = _fake_table(L, live), _fake_table(L, live, d=512)
     tp4 = (ctypes.POINTER(L.IskvExactTable) * 2)(ctypes.pointer(ta), ctypes.pointer(tb))
     hp4 = (ctypes.POINTER(L.IskvLowRank) * 2)(ctypes.pointer(h), ctypes.pointer(h))

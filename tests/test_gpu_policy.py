@@ -71,32 +71,37 @@ def test_prefill_rejects_unordered_protected_positions():
         m.cache_prefill(t, X, torch.tensor([5, 100], dtype=torch.int32, device="cuda"), 32)
 
 
-def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36):
+def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36, refit=0):
     """Two sequences x (K, V) = four tables stepped together through T decode steps, against four
-    oracle runs started from the same stored prompt factors."""
+    oracle runs started from the same stored prompt factors. With ``refit`` > 0 the value sides
+    protect their whole prompt (a short prompt) and run the first refit of ``refit`` rows."""
     sides = []
     for s, L in enumerate(Ls):
         PK = _protected(L, seed + s, suffix=suffix)
-        PV = _widen(PK, L, 4)
+        PV = np.arange(L) if refit else _widen(PK, L, 4)
         for kind, P, w0, ex in (("K", PK, 0, 1.1), ("V", PV, min(W, L), 0.7)):
             X = stored(synth.lowrank_rows(L + T, d, ex, 0.02, seed=seed + 10 * s + len(sides)),
                        storage)
-            sides.append(dict(kind=kind, L=L, P=P, w0=w0, X=X))
+            sides.append(dict(kind=kind, L=L, P=P, w0=w0, X=X, F=refit if kind == "V" else 0))
     n_cap = max(L for L in Ls) + T
     tabs, hists, refs = [], [], []
     for sd in sides:
         L = sd["L"]
         Xd = torch.as_tensor(sd["X"], dtype=storage, device="cuda")
-        t = m.ExactTable(d, 1024, window=W, block=b, reorth_rows=R, dtype=storage)
+        t = m.ExactTable(d, 1024, window=W, block=b, reorth_rows=R, dtype=storage,
+                         refit_rows=sd["F"])
         comp_rows, comp_pos = m.cache_prefill(t, Xd[:L].contiguous(),
                                               torch.as_tensor(sd["P"], dtype=torch.int32,
                                                               device="cuda"), sd["w0"])
-        U0, s0, B0 = of.truncated_svd(sd["X"][comp_pos.cpu().numpy()], r)
+        if comp_pos.numel():
+            U0, s0, B0 = of.truncated_svd(sd["X"][comp_pos.cpu().numpy()], r)
+        else:
+            U0, s0, B0 = of.empty_history(d)
         U0, s0, B0 = stored(U0, storage), stored(s0, torch.float32), stored(B0, storage)
         h = m.LowRankHistory(d, r, n_cap, storage=storage)
         set_state(h, U0, s0, B0, comp_pos.cpu().numpy())
         ref = op.run_decode(sd["X"][:L], sd["X"][L:], sd["P"], sd["w0"], W, b, r, R,
-                            init_history=(U0, s0, B0))
+                            init_history=(U0, s0, B0), refit_rows=sd["F"])
         sd["Xd"] = Xd
         tabs.append(t)
         hists.append(h)
@@ -105,9 +110,9 @@ def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36):
         rows = torch.stack([sd["Xd"][sd["L"] + i] for sd in sides]).contiguous()
         folded, reorthed = m.cache_step(tabs, hists, rows)
         for k, ref in enumerate(refs):
-            acts = ref["steps"][i]
-            assert folded[k] == any(a[0] == "fold" for a in acts), (i, k)
-            assert reorthed[k] == any(a[0] == "reorth" for a in acts), (i, k)
+            acts = [a[0] for a in ref["steps"][i]]
+            assert folded[k] == (2 if "refit" in acts else 1 if "fold" in acts else 0), (i, k)
+            assert reorthed[k] == ("reorth" in acts), (i, k)
     for sd, t, h, ref in zip(sides, tabs, hists, refs):
         U, s, B, pos, (k, n, _, st) = state(h)
         Uo, so, Bo, poso = ref["history"]
@@ -147,6 +152,34 @@ def test_decode_policy_fp32():
     want = oatt.decode_attention(rk["history"], rv["history"], rk["exact"][0], rk["exact"][1],
                                  rv["exact"][0], rv["exact"][1], n_total, q, 2, 128)
     assert float(np.linalg.norm(np64(out) - want) / np.linalg.norm(want)) < 1e-4
+
+
+def test_decode_policy_value_first_refit():
+    """Short prompts whose values are all protected: the value sides wait for 32 pending rows, refit
+    them into their empty histories (two untruncated 16-row folds at r = 32), then fold 16-row
+    blocks; the key sides fold from the start."""
+    m = kv()
+    sides, tabs, hists, refs = _run(m, d=256, r=32, b=16, W=24, R=32, Ls=(120, 90), T=150,
+                                    storage=torch.float32, seed=80, tol=1e-4, refit=32)
+    for k in (1, 3):
+        assert any(a[0] == "refit" for acts in refs[k]["steps"] for a in acts)
+        assert tabs[k].t.refit_done == 1
+
+
+def test_refit_of_a_nonempty_history_is_refused():
+    m = kv()
+    d, b = 256, 16
+    X = torch.randn(200, d, device="cuda")
+    t = m.ExactTable(d, 512, window=8, block=b, reorth_rows=0, dtype=torch.float32, refit_rows=32)
+    comp, comp_pos = m.cache_prefill(t, X[:100].contiguous(),
+                                     torch.arange(90, 100, dtype=torch.int32, device="cuda"), 8)
+    assert t.t.hist_rows == 90 and t.t.refit_done == 0
+    h = m.LowRankHistory(d, 32, 400, storage=torch.float32)
+    for i in range(100, 100 + 8 + 31):
+        m.cache_step([t], [h], X[i:i + 1].contiguous())
+    with pytest.raises(m.IskvError, match="empty history"):
+        m.cache_step([t], [h], X[139:140].contiguous())
+    assert t.t.last == 138                           # the refused step changed nothing
 
 
 def test_decode_policy_bf16_model_width():
