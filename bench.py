@@ -351,17 +351,17 @@ def time_cache_policy(wl, kv, torch, dev, stream):
     gen = torch.Generator(device=dev)
     gen.manual_seed(4242)
     rows = torch.randn(BLK, cnt, D, generator=gen, device=dev).to(torch.bfloat16)
-    ws = kv.Workspace(dev).get(kv.cache_step_workspace_size(cnt, D, R, BLK, wl.hists[0].n_cap))
+    batch = kv.CacheBatch(tabs, wl.hists)
     torch.cuda.synchronize(dev)
     kv.stage_times(reset=True)
     kv.stage_timing(True)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     ev[0].record(stream)
     for j in range(BLK - 1):
-        folded, _ = kv.cache_step(tabs, wl.hists, rows[j], ws=ws, stream=stream)
+        folded, _ = batch.step(rows[j], stream=stream)
         assert not any(folded)
     ev[1].record(stream)
-    folded, _ = kv.cache_step(tabs, wl.hists, rows[BLK - 1], ws=ws, stream=stream)
+    folded, _ = batch.step(rows[BLK - 1], stream=stream)
     ev[2].record(stream)
     torch.cuda.synchronize(dev)
     kv.stage_timing(False)

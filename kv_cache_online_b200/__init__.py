@@ -395,29 +395,51 @@ def cache_step_workspace_size(count, d, r_max, block, n_cap) -> int:
     return int(_lib.load().iskv_cache_step_workspace_size(count, d, r_max, block, n_cap))
 
 
+class CacheBatch:
+    """A fixed set of (table, history) pairs stepped together: the C arrays of table and history
+    pointers, the result buffers and the workspace are built once, so that a decode step costs one
+    library call."""
+
+    def __init__(self, tables, hists, ws=None):
+        n = len(tables)
+        if n == 0 or len(hists) != n:
+            raise ValueError("one history per table")
+        self.n = n
+        self.tables, self.hists = list(tables), list(hists)
+        self._handles = [h.handle() for h in hists]
+        self._tp = (ctypes.POINTER(IskvExactTable) * n)(*[ctypes.pointer(t.t) for t in tables])
+        self._hp = (ctypes.POINTER(IskvLowRank) * n)(*[ctypes.pointer(h) for h in self._handles])
+        self._folded = (ctypes.c_int32 * n)()
+        self._reorthed = (ctypes.c_int32 * n)()
+        h0 = hists[0]
+        need = _lib.load().iskv_cache_step_workspace_size(n, h0.d, h0.r_max, tables[0].t.block,
+                                                          h0.n_cap)
+        self.ws = ws if ws is not None else Workspace(h0.device).get(need)
+
+    def step(self, new_rows, tau_rel: float = 0.0, stream=None):
+        """One decode step; ``new_rows`` (count, d) holds each table's row for its next position.
+        Returns ``(folded, reorthed)``: per table 0, 1 (a block fold) or 2 (the first refit), and
+        a bool."""
+        if new_rows.dim() != 2 or new_rows.shape[0] != self.n or not new_rows.is_contiguous() \
+                or not new_rows.is_cuda:
+            raise ValueError("new_rows must be a contiguous (count, d) CUDA tensor")
+        _lib.check(_lib.load().iskv_cache_step(
+            self._tp, self._hp, self.n, new_rows.data_ptr(), _dt(new_rows), float(tau_rel),
+            self._folded, self._reorthed, self.ws.data_ptr(), self.ws.numel(), _stream(stream)),
+            "cache_step")
+        return list(self._folded), [bool(x) for x in self._reorthed]
+
+
 def cache_step(tables, hists, new_rows, tau_rel: float = 0.0, ws=None, stream=None):
     """Algorithm 3 steps 1-6 for every (table, history) pair: ``new_rows`` (count, d) holds each
     table's row for its next position. Returns ``(folded, reorthed)``: per table 0, 1 (a block
-    fold) or 2 (the first refit), and a bool."""
-    lib = _lib.load()
-    n = len(tables)
-    if n == 0 or len(hists) != n:
-        raise ValueError("one history per table")
+    fold) or 2 (the first refit), and a bool. For a fixed set of tables use :class:`CacheBatch`."""
     _need_cuda(new_rows)
-    if new_rows.dim() != 2 or new_rows.shape[0] != n or not new_rows.is_contiguous():
-        raise ValueError("new_rows must be a contiguous (count, d) tensor")
-    h0 = hists[0]
-    need = lib.iskv_cache_step_workspace_size(n, h0.d, h0.r_max, tables[0].t.block, h0.n_cap)
-    w = ws if ws is not None else _ws(new_rows.device, need)
-    handles = [h.handle() for h in hists]
-    tp = (ctypes.POINTER(IskvExactTable) * n)(*[ctypes.pointer(t.t) for t in tables])
-    hp = (ctypes.POINTER(IskvLowRank) * n)(*[ctypes.pointer(h) for h in handles])
-    folded = (ctypes.c_int32 * n)()
-    reorthed = (ctypes.c_int32 * n)()
-    _lib.check(lib.iskv_cache_step(tp, hp, n, new_rows.data_ptr(), _dt(new_rows), float(tau_rel),
-                                   folded, reorthed, w.data_ptr(), w.numel(), _stream(stream)),
-               "cache_step")
-    return [int(x) for x in folded], [bool(x) for x in reorthed]
+    if ws is None:
+        h0 = hists[0]
+        ws = _ws(new_rows.device, _lib.load().iskv_cache_step_workspace_size(
+            len(tables), h0.d, h0.r_max, tables[0].t.block, h0.n_cap))
+    return CacheBatch(tables, hists, ws=ws).step(new_rows, tau_rel, stream)
 
 
 # ------------------------------------------------------------------------------------------------

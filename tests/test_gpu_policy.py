@@ -106,9 +106,10 @@ def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36, refit=0):
         tabs.append(t)
         hists.append(h)
         refs.append(ref)
+    batch = m.CacheBatch(tabs, hists)
     for i in range(T):
         rows = torch.stack([sd["Xd"][sd["L"] + i] for sd in sides]).contiguous()
-        folded, reorthed = m.cache_step(tabs, hists, rows)
+        folded, reorthed = batch.step(rows)
         for k, ref in enumerate(refs):
             acts = [a[0] for a in ref["steps"][i]]
             assert folded[k] == (2 if "refit" in acts else 1 if "fold" in acts else 0), (i, k)
