@@ -282,10 +282,12 @@ iskv_status iskv_select_prompt_blocks_noalloc(const void *keys, int32_t k_dtype,
  * Algorithm 1 step 5, the last min(W, L) prompt positions for values), so at most one row joins
  * the FIFO per decode step. The value side's first refit (Algorithm 3 step 3; refit_rows = r_V > 0)
  * waits until refit_rows rows are pending and re-factors them, after the rows the history holds, by
- * a rank-r_V SVD; its rows do not count toward reorth_rows (Section 4.4). The device carries out the
- * refit of an EMPTY history (the prompt's values all protected, as with short prompts): there the
- * rank-r_V SVD of the pending rows equals folding them block by block with no truncation
- * (refit_rows <= r_max, a multiple of block). The refit of a non-empty history is not implemented.
+ * a rank-r_V SVD; its rows do not count toward reorth_rows (Section 4.4). The device runs the refit
+ * as ONE fold whose block is all refit_rows rows (Algorithm 2 on the history's rows followed by
+ * them, truncated to r_max: exactly the refit) when the fold takes such a block (refit_rows <= 128,
+ * r_max + refit_rows inside the core SVD cluster); otherwise, for an EMPTY history (the prompt's
+ * values all protected, as with short prompts) and refit_rows <= r_max, as consecutive block folds
+ * that never truncate, which is the same SVD. Other refits are refused.
  *
  * Exact-row table (device, caller-owned):
  *   rows [cap_e][d]  dtype; rows 0 .. n_prot-1 are the protected rows in ascending position, rows
@@ -360,18 +362,19 @@ iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dty
  * history's position table and their exact copies leave the table; when a table's folded rows
  * reach reorth_rows, its history is re-orthogonalised (iskv_reorth) in the same step and the count
  * restarts. A table whose first refit is still to come waits for refit_rows pending rows instead,
- * then folds all of them, block by block, into its (empty) history. All tables share d, window,
+ * then folds all of them (in one fold or in untruncated block folds, as above). All tables share d, window,
  * block and dtype; the histories share d, r_max, storage and n_cap, as the batched fold and
  * re-orthogonalisation require. folded / reorthed (host [count], may be NULL) receive 1 where a
  * table folded a block (2 where it ran its first refit) / re-orthogonalised. Stream-ordered; the
- * host mirror is updated at once. Errors (nothing launched, no table changed): ISKV_ERR_ARG,
+ * host mirror is updated at once. The workspace query takes the largest refit_rows of the tables
+ * (0 when none refits). Errors (nothing launched, no table changed): ISKV_ERR_ARG,
  * ISKV_ERR_SHAPE (mixed table shapes, a history whose d differs, a block the fold does not take, a
- * refit that comes due on a non-empty history or with refit_rows > r_max),
+ * refit that can be run neither way),
  * ISKV_ERR_CAPACITY (a table without room for the new row, or a history without room for the
  * block or the refit: hist_rows + block > n_cap), ISKV_ERR_WORKSPACE; ISKV_ERR_CUDA when a launch fails.
  */
 size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block,
-                                      int64_t n_cap);
+                                      int64_t n_cap, int32_t refit_rows);
 iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank *const *hists,
                             int32_t count, const void *new_rows, int32_t row_dtype, float tau_rel,
                             int32_t *folded, int32_t *reorthed, void *ws, size_t ws_bytes,

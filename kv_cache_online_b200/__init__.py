@@ -391,8 +391,9 @@ def cache_prefill(table: ExactTable, X, protected_pos, init_window: int, ws=None
     return comp[:n_comp.value], comp_pos[:n_comp.value]
 
 
-def cache_step_workspace_size(count, d, r_max, block, n_cap) -> int:
-    return int(_lib.load().iskv_cache_step_workspace_size(count, d, r_max, block, n_cap))
+def cache_step_workspace_size(count, d, r_max, block, n_cap, refit_rows=0) -> int:
+    return int(_lib.load().iskv_cache_step_workspace_size(count, d, r_max, block, n_cap,
+                                                          refit_rows))
 
 
 class CacheBatch:
@@ -412,8 +413,9 @@ class CacheBatch:
         self._folded = (ctypes.c_int32 * n)()
         self._reorthed = (ctypes.c_int32 * n)()
         h0 = hists[0]
+        refit = max(int(t.t.refit_rows) for t in tables)
         need = _lib.load().iskv_cache_step_workspace_size(n, h0.d, h0.r_max, tables[0].t.block,
-                                                          h0.n_cap)
+                                                          h0.n_cap, refit)
         self.ws = ws if ws is not None else Workspace(h0.device).get(need)
 
     def step(self, new_rows, tau_rel: float = 0.0, stream=None):
@@ -438,7 +440,8 @@ def cache_step(tables, hists, new_rows, tau_rel: float = 0.0, ws=None, stream=No
     if ws is None:
         h0 = hists[0]
         ws = _ws(new_rows.device, _lib.load().iskv_cache_step_workspace_size(
-            len(tables), h0.d, h0.r_max, tables[0].t.block, h0.n_cap))
+            len(tables), h0.d, h0.r_max, tables[0].t.block, h0.n_cap,
+            max(int(t.t.refit_rows) for t in tables)))
     return CacheBatch(tables, hists, ws=ws).step(new_rows, tau_rel, stream)
 
 

@@ -79,7 +79,7 @@ SIGNATURES = {
     "iskv_cache_prefill_workspace_size": (c_sz, [c_i32]),
     "iskv_cache_prefill": (c_i32, [ctypes.POINTER(IskvExactTable), c_vp, c_i32, c_i64, c_vp, c_i64,
                                    c_i32, c_vp, c_vp, ctypes.POINTER(c_i64), c_vp, c_sz, c_vp]),
-    "iskv_cache_step_workspace_size": (c_sz, [c_i32, c_i32, c_i32, c_i32, c_i64]),
+    "iskv_cache_step_workspace_size": (c_sz, [c_i32, c_i32, c_i32, c_i32, c_i64, c_i32]),
     "iskv_cache_step": (c_i32, [ctypes.POINTER(ctypes.POINTER(IskvExactTable)),
                                 ctypes.POINTER(ctypes.POINTER(IskvLowRank)), c_i32, c_vp, c_i32,
                                 c_f32, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32), c_vp, c_sz,

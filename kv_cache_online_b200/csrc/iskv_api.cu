@@ -1,5 +1,6 @@
 // C ABI of libiskv: argument validation on the host, workspace carving and the launch sequence of
 // each entry point. Every numerical step runs in the kernels of the other translation units.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -146,6 +147,14 @@ int64_t pending_after(const iskv_exact_table *t, int64_t pos) {
 }
 
 static_assert(sizeof(AppendJob) <= 64 && sizeof(EvictJob) <= 64, "policy job sizes");
+
+// A refit of `rows` rows can be one fold with a block of that many rows (any history: Algorithm 2
+// on the history's rows followed by the block, truncated to r_max) when the fold takes the block.
+bool refit_in_one_fold(int d, int r, int rows) {
+  JacobiCfg jc;
+  return rows >= 8 && rows % 8 == 0 && rows <= 128 && rows <= d &&
+         fold_residual_smem(d, rows) <= 200 * 1024 && core_cfg(r, rows, false, jc);
+}
 
 }  // namespace
 
@@ -924,8 +933,8 @@ iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dty
 }
 
 size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block,
-                                      int64_t n_cap) {
-  if (count < 1 || d < 1 || r_max < 1 || block < 1 || n_cap < 0) return 0;
+                                      int64_t n_cap, int32_t refit_rows) {
+  if (count < 1 || d < 1 || r_max < 1 || block < 1 || n_cap < 0 || refit_rows < 0) return 0;
   size_t need = jobs_bytes(count, sizeof(AppendJob));
   const size_t ev = jobs_bytes(count, sizeof(EvictJob));
   const size_t fw = iskv_fold_workspace_size(count, d, r_max, block);
@@ -933,6 +942,10 @@ size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, i
   if (ev > need) need = ev;
   if (fw > need) need = fw;
   if (rw > need) need = rw;
+  if (refit_rows > 0 && refit_in_one_fold(d, r_max, refit_rows)) {
+    const size_t fr = iskv_fold_workspace_size(count, d, r_max, refit_rows);
+    if (fr > need) need = fr;
+  }
   return need;
 }
 
@@ -948,6 +961,7 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
   if (!(tau_rel >= 0.f)) return fail(ISKV_ERR_ARG, "%s: tau_rel must be >= 0", who);
   if (!aligned(new_rows, elem_size(row_dtype))) return fail(ISKV_ERR_ARG, "%s: misaligned rows", who);
   bool any_reorth = false;
+  int32_t refit_max = 0;
   for (int32_t i = 0; i < count; ++i) {
     iskv_status st = check_table(tables[i], who);
     if (st != ISKV_OK) return st;
@@ -964,6 +978,7 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
     if (T->n_prot + T->n_live + 1 > T->cap_e || T->n_live + 1 > T->live_cap)
       return fail(ISKV_ERR_CAPACITY, "%s: table %d has no room for the new row", who, i);
     if (T->reorth_rows > 0) any_reorth = true;
+    if (!T->refit_done && T->refit_rows > refit_max) refit_max = T->refit_rows;
   }
   const iskv_exact_table *T0 = tables[0];
   const int d = T0->d, b = T0->block, r = hists[0]->r_max;
@@ -981,7 +996,7 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
     if (any_reorth && !core_cfg(r, 0, true, jc))
       return fail(ISKV_ERR_SHAPE, "%s: r_max too large for the dense core SVD", who);
   }
-  const size_t need = iskv_cache_step_workspace_size(count, d, r, b, ncap);
+  const size_t need = iskv_cache_step_workspace_size(count, d, r, b, ncap, refit_max);
   iskv_status st = check_ws(ws, ws_bytes, need, who);
   if (st != ISKV_OK) return st;
 
@@ -990,7 +1005,7 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
   std::vector<AppendJob> aj(count);
   std::vector<int32_t> fold_idx, reorth_idx;
   std::vector<int32_t> fold_rows(count, 0);  // rows this step folds per table (b, or refit_rows)
-  int32_t passes = 0;                        // block folds in this step: the longest refit / b
+  std::vector<int32_t> fold_blk(count, 0);   // block size of those folds (b, or refit_rows)
   for (int32_t i = 0; i < count; ++i) {
     const iskv_exact_table *T = tables[i];
     const int64_t t = T->last + 1, slot = T->n_prot + T->n_live;
@@ -1007,13 +1022,21 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
       if (T->hist_rows + rows > ncap)
         return fail(ISKV_ERR_CAPACITY, "%s: table %d: history has no room for a block (%lld + %d > "
                     "%lld)", who, i, (long long)T->hist_rows, rows, (long long)ncap);
-      if (refit && (T->hist_rows != 0 || rows > r))
-        return fail(ISKV_ERR_SHAPE, "%s: table %d: the first refit is carried out for an empty "
-                    "history and refit_rows <= r_max only (history rows %lld, refit_rows %d)", who,
-                    i, (long long)T->hist_rows, rows);
+      // A refit is one fold of all its rows when the fold takes such a block; otherwise, for an
+      // empty history and refit_rows <= r_max, consecutive b-row folds that never truncate.
+      int32_t blk = b;
+      if (refit) {
+        if (refit_in_one_fold(d, r, rows)) blk = rows;
+        else if (T->hist_rows != 0 || rows > r)
+          return fail(ISKV_ERR_SHAPE, "%s: table %d: a first refit of %d rows is carried out as one "
+                      "fold (refit_rows <= 128 with r_max + refit_rows inside the core SVD "
+                      "cluster) or, for an empty history, as untruncated block folds "
+                      "(refit_rows <= r_max); history rows %lld", who, i, rows,
+                      (long long)T->hist_rows);
+      }
       fold_idx.push_back(i);
       fold_rows[i] = rows;
-      if (rows / b > passes) passes = rows / b;
+      fold_blk[i] = blk;
       if (!refit && T->reorth_rows > 0 && T->fold_rows + b >= T->reorth_rows)
         reorth_idx.push_back(i);
     }
@@ -1039,23 +1062,34 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
       ej[k].shift = fold_rows[fold_idx[k]];
       ej[k].pad_ = 0;
     }
-    // Pass j folds the j-th block of the FIFO of every table that folds that many rows: regular
-    // folds take pass 0 only, a refit of refit_rows rows takes passes 0 .. refit_rows / b - 1.
-    for (int32_t j = 0; j < passes; ++j) {
-      std::vector<iskv_lowrank> fh;
-      std::vector<const void *> F;
-      std::vector<const int32_t *> fp;
-      for (int32_t i : fold_idx) {
-        if (fold_rows[i] / b <= j) continue;
-        const iskv_exact_table *T = tables[i];
-        const int64_t row0 = T->n_prot + (int64_t)j * b;
-        fh.push_back(*hists[i]);
-        F.push_back(static_cast<const char *>(T->rows) + (size_t)row0 * d * esz);
-        fp.push_back(T->pos + row0);
+    // Batched folds per block size; pass j of a block size folds the j-th block of the FIFO of
+    // every table with that block size that folds more than j blocks (regular folds and one-fold
+    // refits take pass 0 only, a refit by b-row folds passes 0 .. refit_rows / b - 1).
+    std::vector<int32_t> sizes;
+    for (int32_t i : fold_idx)
+      if (std::find(sizes.begin(), sizes.end(), fold_blk[i]) == sizes.end())
+        sizes.push_back(fold_blk[i]);
+    std::sort(sizes.begin(), sizes.end());
+    for (int32_t fb : sizes) {
+      int32_t passes = 0;
+      for (int32_t i : fold_idx)
+        if (fold_blk[i] == fb && fold_rows[i] / fb > passes) passes = fold_rows[i] / fb;
+      for (int32_t j = 0; j < passes; ++j) {
+        std::vector<iskv_lowrank> fh;
+        std::vector<const void *> F;
+        std::vector<const int32_t *> fp;
+        for (int32_t i : fold_idx) {
+          if (fold_blk[i] != fb || fold_rows[i] / fb <= j) continue;
+          const iskv_exact_table *T = tables[i];
+          const int64_t row0 = T->n_prot + (int64_t)j * fb;
+          fh.push_back(*hists[i]);
+          F.push_back(static_cast<const char *>(T->rows) + (size_t)row0 * d * esz);
+          fp.push_back(T->pos + row0);
+        }
+        st = iskv_fold_block_batched(fh.data(), (int32_t)fh.size(), F.data(), T0->dtype, fb,
+                                     fp.data(), tau_rel, ws, ws_bytes, stream);
+        if (st != ISKV_OK) return st;
       }
-      st = iskv_fold_block_batched(fh.data(), (int32_t)fh.size(), F.data(), T0->dtype, b,
-                                   fp.data(), tau_rel, ws, ws_bytes, stream);
-      if (st != ISKV_OK) return st;
     }
     EvictJob *dej = reinterpret_cast<EvictJob *>(base);
     stage_begin(s);

@@ -165,16 +165,17 @@ def test_cache_policy_host_side_errors():
     t3 = _fake_table(L, live, block=12)
     tp3 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t3))
     assert lib.iskv_cache_step(tp3, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
-    # a refit that is not a multiple of the block; a refit due on a non-empty history
+    # a refit that is not a multiple of the block; a refit due on a non-empty history that one
+    # fold cannot take
     t5 = _fake_table(L, live, window=0, block=8)
     t5.refit_rows, t5.refit_done, t5.live_cap = 12, 0, 12
     tp5 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t5))
     assert lib.iskv_cache_step(tp5, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
     t6 = _fake_table(L, live, window=0, block=8)
-    t6.refit_rows, t6.refit_done, t6.live_cap = 16, 0, 16
-    for i in range(15):
+    t6.refit_rows, t6.refit_done, t6.live_cap = 136, 0, 136   # more rows than one fold takes
+    for i in range(135):
         live[i] = i
-    t6.n_live, t6.last, t6.hist_rows = 15, 14, 100
+    t6.n_live, t6.last, t6.hist_rows = 135, 134, 100
     tp6 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t6))
     assert lib.iskv_cache_step(tp6, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
     assert b"empty" in lib.iskv_last_error()

@@ -71,14 +71,16 @@ def test_prefill_rejects_unordered_protected_positions():
         m.cache_prefill(t, X, torch.tensor([5, 100], dtype=torch.int32, device="cuda"), 32)
 
 
-def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36, refit=0):
+def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36, refit=0, v_all=None):
     """Two sequences x (K, V) = four tables stepped together through T decode steps, against four
-    oracle runs started from the same stored prompt factors. With ``refit`` > 0 the value sides
-    protect their whole prompt (a short prompt) and run the first refit of ``refit`` rows."""
+    oracle runs started from the same stored prompt factors. With ``refit`` > 0 the value sides run
+    the first refit of ``refit`` rows; ``v_all`` (default: when refitting) protects their whole
+    prompt (a short prompt), so that their history is empty at the refit."""
+    v_all = bool(refit) if v_all is None else v_all
     sides = []
     for s, L in enumerate(Ls):
         PK = _protected(L, seed + s, suffix=suffix)
-        PV = np.arange(L) if refit else _widen(PK, L, 4)
+        PV = np.arange(L) if v_all else _widen(PK, L, 4)
         for kind, P, w0, ex in (("K", PK, 0, 1.1), ("V", PV, min(W, L), 0.7)):
             X = stored(synth.lowrank_rows(L + T, d, ex, 0.02, seed=seed + 10 * s + len(sides)),
                        storage)
@@ -155,32 +157,58 @@ def test_decode_policy_fp32():
     assert float(np.linalg.norm(np64(out) - want) / np.linalg.norm(want)) < 1e-4
 
 
-def test_decode_policy_value_first_refit():
-    """Short prompts whose values are all protected: the value sides wait for 32 pending rows, refit
-    them into their empty histories (two untruncated 16-row folds at r = 32), then fold 16-row
-    blocks; the key sides fold from the start."""
-    m = kv()
-    sides, tabs, hists, refs = _run(m, d=256, r=32, b=16, W=24, R=32, Ls=(120, 90), T=150,
-                                    storage=torch.float32, seed=80, tol=1e-4, refit=32)
+def _refits(refs, tabs):
     for k in (1, 3):
         assert any(a[0] == "refit" for acts in refs[k]["steps"] for a in acts)
         assert tabs[k].t.refit_done == 1
 
 
-def test_refit_of_a_nonempty_history_is_refused():
+def test_decode_policy_value_first_refit():
+    """Short prompts whose values are all protected: the value sides wait for 32 pending rows, refit
+    them into their empty histories (one 32-row fold at r = 32), then fold 16-row blocks; the key
+    sides fold from the start."""
     m = kv()
-    d, b = 256, 16
-    X = torch.randn(200, d, device="cuda")
-    t = m.ExactTable(d, 512, window=8, block=b, reorth_rows=0, dtype=torch.float32, refit_rows=32)
+    sides, tabs, hists, refs = _run(m, d=256, r=32, b=16, W=24, R=32, Ls=(120, 90), T=150,
+                                    storage=torch.float32, seed=80, tol=1e-4, refit=32)
+    _refits(refs, tabs)
+
+
+def test_refit_of_a_compressed_history_in_one_fold():
+    """Prompts with compressed values: the refit factors the history's rows followed by the 32
+    pending rows, truncated to r = 32 -- one 32-row fold on the device."""
+    m = kv()
+    sides, tabs, hists, refs = _run(m, d=256, r=32, b=16, W=24, R=32, Ls=(300, 180), T=150,
+                                    storage=torch.float32, seed=83, tol=1e-4, suffix=8, refit=32,
+                                    v_all=False)
+    _refits(refs, tabs)
+    assert all(len(refs[k]["comp"]) > 0 for k in (1, 3))
+
+
+def test_refit_by_untruncated_block_folds():
+    """A 144-row refit (more than one fold takes) of empty histories at r = 160: nine 16-row folds
+    in one step, none of which truncates."""
+    m = kv()
+    sides, tabs, hists, refs = _run(m, d=256, r=160, b=16, W=24, R=64, Ls=(60, 50), T=200,
+                                    storage=torch.float32, seed=86, tol=1e-4, refit=144)
+    _refits(refs, tabs)
+
+
+def test_refit_that_runs_neither_way_is_refused():
+    """144 rows (more than one fold takes) into a history that already holds compressed rows."""
+    m = kv()
+    d, b, rv = 256, 16, 144
+    X = torch.randn(300, d, device="cuda")
+    t = m.ExactTable(d, 512, window=8, block=b, reorth_rows=0, dtype=torch.float32, refit_rows=rv)
     comp, comp_pos = m.cache_prefill(t, X[:100].contiguous(),
                                      torch.arange(90, 100, dtype=torch.int32, device="cuda"), 8)
     assert t.t.hist_rows == 90 and t.t.refit_done == 0
-    h = m.LowRankHistory(d, 32, 400, storage=torch.float32)
-    for i in range(100, 100 + 8 + 31):
+    h = m.LowRankHistory(d, 160, 400, storage=torch.float32)
+    for i in range(100, 100 + 8 + rv - 1):
         m.cache_step([t], [h], X[i:i + 1].contiguous())
+    last = t.t.last
     with pytest.raises(m.IskvError, match="empty history"):
-        m.cache_step([t], [h], X[139:140].contiguous())
-    assert t.t.last == 138                           # the refused step changed nothing
+        m.cache_step([t], [h], X[last + 1:last + 2].contiguous())
+    assert t.t.last == last                          # the refused step changed nothing
 
 
 def test_decode_policy_bf16_model_width():
