@@ -380,6 +380,19 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
                             int32_t *folded, int32_t *reorthed, void *ws, size_t ws_bytes,
                             void *stream);
 
+/*
+ * Host-only dry run of iskv_cache_step()'s schedule (touches no device memory and launches
+ * nothing): folded[i] / reorthed[i] (host [count], may be NULL) receive what the next
+ * iskv_cache_step() would do to tables[i] -- 0, 1 (a block fold) or 2 (the first refit), and
+ * whether a re-orthogonalisation follows -- for histories of the given r_max and n_cap. With
+ * advance != 0 the host mirrors are then advanced exactly as that step would advance them. Lets a
+ * caller see which tables fold before a step (to plan workspaces or overlap other work). Errors as
+ * iskv_cache_step()'s host-side ones (ISKV_ERR_ARG, ISKV_ERR_SHAPE, ISKV_ERR_CAPACITY); on an error
+ * no mirror is changed.
+ */
+iskv_status iskv_cache_plan(iskv_exact_table *const *tables, int32_t count, int32_t r_max,
+                            int64_t n_cap, int32_t advance, int32_t *folded, int32_t *reorthed);
+
 /* Empty a history: zero its meta word, sigma, U and B (stream-ordered). */
 iskv_status iskv_reset(const iskv_lowrank *h, void *stream);
 

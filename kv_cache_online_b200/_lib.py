@@ -84,6 +84,8 @@ SIGNATURES = {
                                 ctypes.POINTER(ctypes.POINTER(IskvLowRank)), c_i32, c_vp, c_i32,
                                 c_f32, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32), c_vp, c_sz,
                                 c_vp]),
+    "iskv_cache_plan": (c_i32, [ctypes.POINTER(ctypes.POINTER(IskvExactTable)), c_i32, c_i32,
+                                c_i64, c_i32, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32)]),
     "iskv_reset": (c_i32, [ctypes.POINTER(IskvLowRank), c_vp]),
     "iskv_get_status": (c_i32, [ctypes.POINTER(IskvLowRank), ctypes.POINTER(c_i64),
                                 ctypes.POINTER(c_i64), ctypes.POINTER(c_i64),

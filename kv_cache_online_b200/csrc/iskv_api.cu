@@ -156,6 +156,67 @@ bool refit_in_one_fold(int d, int r, int rows) {
          fold_residual_smem(d, rows) <= 200 * 1024 && core_cfg(r, rows, false, jc);
 }
 
+// What the next decode step does to one table, decided from its host mirror alone: the rows it
+// folds (0: none; `block`, or refit_rows for the first refit), the block size of those folds, and
+// whether a re-orthogonalisation follows.
+struct TablePlan {
+  int32_t rows = 0, blk = 0;
+  bool refit = false, reorth = false;
+};
+
+iskv_status plan_table(const iskv_exact_table *T, int d, int r, int64_t ncap, int i,
+                       const char *who, TablePlan &p) {
+  p = TablePlan{};
+  const int b = T->block;
+  const bool refit = !T->refit_done;
+  const int32_t rows = refit ? T->refit_rows : b;
+  if (pending_after(T, T->last + 1) < rows) return ISKV_OK;
+  if (T->hist_rows + rows > ncap)
+    return fail(ISKV_ERR_CAPACITY, "%s: table %d: history has no room for a block (%lld + %d > "
+                "%lld)", who, i, (long long)T->hist_rows, rows, (long long)ncap);
+  // A refit is one fold of all its rows when the fold takes such a block; otherwise, for an empty
+  // history and refit_rows <= r_max, consecutive b-row folds that never truncate.
+  int32_t blk = b;
+  if (refit) {
+    if (refit_in_one_fold(d, r, rows)) blk = rows;
+    else if (T->hist_rows != 0 || rows > r)
+      return fail(ISKV_ERR_SHAPE, "%s: table %d: a first refit of %d rows is carried out as one "
+                  "fold (refit_rows <= 128 with r_max + refit_rows inside the core SVD cluster) "
+                  "or, for an empty history, as untruncated block folds (refit_rows <= r_max); "
+                  "history rows %lld", who, i, rows, (long long)T->hist_rows);
+  }
+  p.rows = rows;
+  p.blk = blk;
+  p.refit = refit;
+  p.reorth = !refit && T->reorth_rows > 0 && T->fold_rows + b >= T->reorth_rows;
+  return ISKV_OK;
+}
+
+// The host mirror after the step `p` describes: the new position is stored, the folded rows leave
+// the live rows and join the history, and the counters move (the refit is outside reorth_rows).
+void advance_table(iskv_exact_table *T, const TablePlan &p) {
+  T->last += 1;
+  T->live_host[T->n_live++] = (int32_t)T->last;
+  if (p.rows > 0) {
+    std::memmove(T->live_host, T->live_host + p.rows,
+                 sizeof(int32_t) * (size_t)(T->n_live - p.rows));
+    T->n_live -= p.rows;
+    T->hist_rows += p.rows;
+    if (p.refit) T->refit_done = 1;
+    else T->fold_rows += p.rows;
+  }
+  if (p.reorth) T->fold_rows = 0;
+}
+
+// Mirror checks shared by the step and its dry run: the table has room for the new row.
+iskv_status check_room(const iskv_exact_table *T, int i, const char *who) {
+  if (T->n_prot < 0 || T->n_live < 0 || T->hist_rows < 0 || T->last + 1 >= (int64_t)1 << 31)
+    return fail(ISKV_ERR_SHAPE, "%s: table %d: inconsistent host mirror", who, i);
+  if (T->n_prot + T->n_live + 1 > T->cap_e || T->n_live + 1 > T->live_cap)
+    return fail(ISKV_ERR_CAPACITY, "%s: table %d has no room for the new row", who, i);
+  return ISKV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -973,10 +1034,7 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
     if (H->d != T0->d || H->r_max != H0->r_max || H->storage != H0->storage || H->n_cap != H0->n_cap)
       return fail(ISKV_ERR_SHAPE, "%s: histories must have the tables' d and share r_max, storage, "
                   "n_cap", who);
-    if (T->n_prot < 0 || T->n_live < 0 || T->hist_rows < 0 || T->last + 1 >= (int64_t)1 << 31)
-      return fail(ISKV_ERR_SHAPE, "%s: table %d: inconsistent host mirror", who, i);
-    if (T->n_prot + T->n_live + 1 > T->cap_e || T->n_live + 1 > T->live_cap)
-      return fail(ISKV_ERR_CAPACITY, "%s: table %d has no room for the new row", who, i);
+    if ((st = check_room(T, i, who)) != ISKV_OK) return st;
     if (T->reorth_rows > 0) any_reorth = true;
     if (!T->refit_done && T->refit_rows > refit_max) refit_max = T->refit_rows;
   }
@@ -1004,6 +1062,7 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
   const size_t esz = elem_size(T0->dtype), rsz = elem_size(row_dtype);
   std::vector<AppendJob> aj(count);
   std::vector<int32_t> fold_idx, reorth_idx;
+  std::vector<TablePlan> plan(count);
   std::vector<int32_t> fold_rows(count, 0);  // rows this step folds per table (b, or refit_rows)
   std::vector<int32_t> fold_blk(count, 0);   // block size of those folds (b, or refit_rows)
   for (int32_t i = 0; i < count; ++i) {
@@ -1016,30 +1075,13 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
     j.meta = hists[i]->meta;
     j.position = (int32_t)t;
     j.pad_ = 0;
-    const bool refit = !T->refit_done;
-    const int32_t rows = refit ? T->refit_rows : b;
-    if (pending_after(T, t) >= rows) {
-      if (T->hist_rows + rows > ncap)
-        return fail(ISKV_ERR_CAPACITY, "%s: table %d: history has no room for a block (%lld + %d > "
-                    "%lld)", who, i, (long long)T->hist_rows, rows, (long long)ncap);
-      // A refit is one fold of all its rows when the fold takes such a block; otherwise, for an
-      // empty history and refit_rows <= r_max, consecutive b-row folds that never truncate.
-      int32_t blk = b;
-      if (refit) {
-        if (refit_in_one_fold(d, r, rows)) blk = rows;
-        else if (T->hist_rows != 0 || rows > r)
-          return fail(ISKV_ERR_SHAPE, "%s: table %d: a first refit of %d rows is carried out as one "
-                      "fold (refit_rows <= 128 with r_max + refit_rows inside the core SVD "
-                      "cluster) or, for an empty history, as untruncated block folds "
-                      "(refit_rows <= r_max); history rows %lld", who, i, rows,
-                      (long long)T->hist_rows);
-      }
+    if ((st = plan_table(T, d, r, ncap, i, who, plan[i])) != ISKV_OK) return st;
+    if (plan[i].rows > 0) {
       fold_idx.push_back(i);
-      fold_rows[i] = rows;
-      fold_blk[i] = blk;
-      if (!refit && T->reorth_rows > 0 && T->fold_rows + b >= T->reorth_rows)
-        reorth_idx.push_back(i);
+      fold_rows[i] = plan[i].rows;
+      fold_blk[i] = plan[i].blk;
     }
+    if (plan[i].reorth) reorth_idx.push_back(i);
   }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1108,29 +1150,32 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
 
   // Host mirror.
   for (int32_t i = 0; i < count; ++i) {
-    iskv_exact_table *T = tables[i];
-    T->last += 1;
-    T->live_host[T->n_live++] = (int32_t)T->last;
-    if (folded) folded[i] = 0;
-    if (reorthed) reorthed[i] = 0;
+    advance_table(tables[i], plan[i]);
+    if (folded) folded[i] = plan[i].rows > 0 ? (plan[i].refit ? 2 : 1) : 0;
+    if (reorthed) reorthed[i] = plan[i].reorth ? 1 : 0;
   }
-  for (int32_t i : fold_idx) {
-    iskv_exact_table *T = tables[i];
-    const int32_t rows = fold_rows[i];
-    std::memmove(T->live_host, T->live_host + rows, sizeof(int32_t) * (size_t)(T->n_live - rows));
-    T->n_live -= rows;
-    T->hist_rows += rows;
-    if (T->refit_done) {
-      T->fold_rows += rows;
-      if (folded) folded[i] = 1;
-    } else {
-      T->refit_done = 1;  // the refit does not count toward reorth_rows
-      if (folded) folded[i] = 2;
-    }
+  return ISKV_OK;
+}
+
+iskv_status iskv_cache_plan(iskv_exact_table *const *tables, int32_t count, int32_t r_max,
+                            int64_t n_cap, int32_t advance, int32_t *folded, int32_t *reorthed) {
+  const char *who = "iskv_cache_plan";
+  g_last_error.clear();
+  if (!tables) return fail(ISKV_ERR_ARG, "%s: null tables", who);
+  if (count < 1 || count > 4096) return fail(ISKV_ERR_SHAPE, "%s: count must be in [1, 4096]", who);
+  if (r_max < 1 || n_cap < 0) return fail(ISKV_ERR_SHAPE, "%s: bad r_max / n_cap", who);
+  std::vector<TablePlan> plan(count);
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_status st = check_table(tables[i], who);
+    if (st != ISKV_OK) return st;
+    if ((st = check_room(tables[i], i, who)) != ISKV_OK) return st;
+    if ((st = plan_table(tables[i], tables[i]->d, r_max, n_cap, i, who, plan[i])) != ISKV_OK)
+      return st;
   }
-  for (int32_t i : reorth_idx) {
-    tables[i]->fold_rows = 0;
-    if (reorthed) reorthed[i] = 1;
+  for (int32_t i = 0; i < count; ++i) {
+    if (folded) folded[i] = plan[i].rows > 0 ? (plan[i].refit ? 2 : 1) : 0;
+    if (reorthed) reorthed[i] = plan[i].reorth ? 1 : 0;
+    if (advance) advance_table(tables[i], plan[i]);
   }
   return ISKV_OK;
 }
