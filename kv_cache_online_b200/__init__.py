@@ -418,6 +418,15 @@ class CacheBatch:
                                                           h0.n_cap, refit)
         self.ws = ws if ws is not None else Workspace(h0.device).get(need)
 
+    def plan(self, advance: bool = False):
+        """What the next :meth:`step` will do to each table, decided on the host alone (no device
+        work): ``(folded, reorthed)`` as :meth:`step` returns them. With ``advance`` the host
+        mirrors move on as that step would move them (a dry run of the schedule)."""
+        h0 = self.hists[0]
+        _lib.check(_lib.load().iskv_cache_plan(self._tp, self.n, h0.r_max, h0.n_cap, int(advance),
+                                               self._folded, self._reorthed), "cache_plan")
+        return list(self._folded), [bool(x) for x in self._reorthed]
+
     def step(self, new_rows, tau_rel: float = 0.0, stream=None):
         """One decode step; ``new_rows`` (count, d) holds each table's row for its next position.
         Returns ``(folded, reorthed)``: per table 0, 1 (a block fold) or 2 (the first refit), and

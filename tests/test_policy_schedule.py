@@ -135,3 +135,26 @@ def test_history_capacity_is_checked_before_the_fold():
     before = tab.mirror()
     assert lib.iskv_cache_plan(arr, 1, R, 12, 1, None, None) == 4      # 16 > 12
     assert tab.mirror() == before
+
+
+def test_cache_batch_plan_through_the_binding():
+    """``CacheBatch.plan`` (host memory only, so CPU tensors serve): keys with an empty prompt,
+    W = 4, b = 8 -- the first fold comes with position W + b - 1 = 11, then every 8 positions."""
+    _lib()
+    import torch
+
+    import kv_cache_online_b200 as m
+    tabs = [m.ExactTable(64, 64, window=4, block=8, reorth_rows=16, dtype=torch.bfloat16,
+                         device="cpu") for _ in range(2)]
+    for t in tabs:
+        t.t.last = -1
+    hists = [m.LowRankHistory(64, 16, 64, storage=torch.bfloat16, device="cpu") for _ in range(2)]
+    batch = m.CacheBatch(tabs, hists)
+    seen = []
+    for pos in range(30):
+        folded, reorthed = batch.plan(advance=True)
+        if folded[0]:
+            seen.append((pos, folded[0], reorthed[0]))
+        assert folded == [folded[0]] * 2
+    assert seen == [(11, 1, False), (19, 1, True), (27, 1, False)]
+    assert tabs[0].live_positions() == list(range(24, 30)) and tabs[0].t.hist_rows == 24
