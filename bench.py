@@ -32,6 +32,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -66,10 +67,10 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, log_dir=None):
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = os.path.join(log_dir or tempfile.gettempdir(), f"clocks_rank{gpu_index}.csv")
 
     def start(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
@@ -416,7 +417,7 @@ def run_b200(args):
     barrier()
 
     # Timed region (device events on the launching stream, stage events inside the library).
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local, args.clock_log_dir)
     kv.stage_times(reset=True)
     kv.stage_timing(True)
     launches0 = kv.launch_count()
@@ -749,6 +750,9 @@ def main(argv=None):
                     help="skip the rows timed apart from the step: decode attention over the "
                          "compressed cache, the diagnostics and the cache-policy step")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--clock-log-dir", default=None,
+                    help="folder for the nvidia-smi clock samples of the timed region "
+                         "(default: the system's temporary folder)")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="model layers (2 histories each); the headline workload is 32")
     args = ap.parse_args(argv)
