@@ -168,7 +168,7 @@ iskv_status plan_table(const iskv_exact_table *T, int d, int r, int64_t ncap, in
                        const char *who, TablePlan &p) {
   p = TablePlan{};
   const int b = T->block;
-  const bool refit = !T->refit_done;
+  const bool refit = !T->refit_done && T->refit_rows > 0;  // a 0-row refit counts as done
   const int32_t rows = refit ? T->refit_rows : b;
   if (pending_after(T, T->last + 1) < rows) return ISKV_OK;
   if (T->hist_rows + rows > ncap)
@@ -204,6 +204,7 @@ void advance_table(iskv_exact_table *T, const TablePlan &p) {
     T->hist_rows += p.rows;
     if (p.refit) T->refit_done = 1;
     else T->fold_rows += p.rows;
+    if (T->refit_rows == 0) T->refit_done = 1;
   }
   if (p.reorth) T->fold_rows = 0;
 }

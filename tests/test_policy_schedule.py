@@ -158,3 +158,19 @@ def test_cache_batch_plan_through_the_binding():
         assert folded == [folded[0]] * 2
     assert seen == [(11, 1, False), (19, 1, True), (27, 1, False)]
     assert tabs[0].live_positions() == list(range(24, 30)) and tabs[0].t.hist_rows == 24
+
+
+def test_zero_row_refit_counts_as_done():
+    """A table without a refit (refit_rows = 0) folds regular blocks even if its mirror says the
+    refit is still to come."""
+    L_, lib = _lib()
+    side, comp = op.new_side(0, [], 0, 0, 8, 0, 0)
+    tab = _Table(L_, side, comp, 0, 8, 0, 0)
+    tab.t.refit_done = 0
+    arr = (ctypes.POINTER(L_.IskvExactTable) * 1)(ctypes.pointer(tab.t))
+    folded = (ctypes.c_int32 * 1)()
+    got = []
+    for _ in range(16):
+        assert lib.iskv_cache_plan(arr, 1, R, NCAP, 1, folded, None) == 0
+        got.append(folded[0])
+    assert got == [0] * 7 + [1] + [0] * 7 + [1] and tab.t.refit_done == 1
