@@ -469,11 +469,13 @@ def run_b200(args):
     rl_name = ROOFLINE_STAGE if ROOFLINE_STAGE in stages else max(
         (k for k in stages if k in sbytes), key=lambda k: stages[k]["ms_per_call"])
     rl = stages[rl_name]
-    traffic = load_traffic(rl_name)
+    traffic, earlier = load_traffic(rl_name)
     roofline = {"kernel": rl_name, "bound": "hbm", "achieved": rl["achieved_gbs"],
                 "peak": hbm, "unit": "GB/s", "frac": rl["frac_hbm"],
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
                 "traffic": traffic, "dominant_stage": dom}
+    if earlier is not None:
+        roofline["traffic_earlier_capture"] = earlier
 
     # Diagnostics of the benchmark state (eq. 12 bytes, factor orthogonality).
     diag = None
@@ -533,15 +535,21 @@ def run_b200(args):
 
 
 def load_traffic(stage: str):
-    """DRAM bytes per launch of `stage` from the committed ncu summary, if one was taken for the
-    current kernel (profiles/*.json with {"stage": ..., "dram_bytes_per_launch": ...})."""
+    """(DRAM bytes per launch of `stage`, context) from the committed ncu summary
+    (profiles/traffic.json). The bytes are None unless the capture was taken on the current kernel
+    ("current": true); an older capture is returned only as context."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
-        return None
+        return None, None
     with open(p) as f:
         j = json.load(f)
     ent = j.get(stage)
-    return None if ent is None else ent.get("dram_bytes_per_launch")
+    if ent is None:
+        return None, None
+    if ent.get("current", False):
+        return ent.get("dram_bytes_per_launch"), None
+    return None, {"dram_bytes_per_launch": ent.get("dram_bytes_per_launch"),
+                  "note": ent.get("note", "")}
 
 
 def spot_check(wl, torch):
