@@ -56,6 +56,16 @@ def test_workspace_queries_are_consistent():
     assert lib.iskv_reorth_workspace_size(1, 1024, 256, 16384) > 16 * 256 * 256 * 4
     assert lib.iskv_reconstruct_workspace_size(1, 1024, 256) >= 1024 * 256 * 2
     assert lib.iskv_select_workspace_size(65536, 8, 8) > 65536 * 8
+    # the cache step reuses one workspace for its append, folds, eviction and reorth in turn
+    step = lib.iskv_cache_step_workspace_size(64, 1024, 256, 64, 17000, 0)
+    assert step == max(lib.iskv_fold_workspace_size(64, 1024, 256, 64),
+                       lib.iskv_reorth_workspace_size(64, 1024, 256, 17000))
+    refit = lib.iskv_cache_step_workspace_size(64, 1024, 128, 64, 17000, 128)
+    assert refit >= lib.iskv_fold_workspace_size(64, 1024, 128, 128) > \
+        lib.iskv_fold_workspace_size(64, 1024, 128, 64)
+    # a refit larger than one fold takes runs as b-row folds: no extra workspace
+    assert lib.iskv_cache_step_workspace_size(64, 1024, 256, 64, 17000, 192) == step
+    assert lib.iskv_cache_step_workspace_size(0, 1024, 256, 64, 17000, 0) == 0
 
 
 def _fake_handle(L, d=1024, r=256, storage=1, base=0x10000):
