@@ -193,3 +193,47 @@ def test_cache_policy_host_side_errors():
     tp4 = (ctypes.POINTER(L.IskvExactTable) * 2)(ctypes.pointer(ta), ctypes.pointer(tb))
     hp4 = (ctypes.POINTER(L.IskvLowRank) * 2)(ctypes.pointer(h), ctypes.pointer(h))
     assert lib.iskv_cache_step(tp4, hp4, 2, rows, 1, 0.0, None, None, ws, big, None) == 2
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "iskv.h"
+
+/* A plain C caller: the ABI version, a status string, a workspace query, and the cache step's
+   schedule dry run on a host-only table (keys, empty prompt, W = 4, b = 8). */
+int main(void) {
+  int32_t live[12];
+  iskv_exact_table t;
+  iskv_exact_table *tabs[1];
+  int32_t folded = 0, first = -1, pos;
+  memset(&t, 0, sizeof t);
+  t.d = 64; t.window = 4; t.block = 8; t.dtype = ISKV_BF16; t.cap_e = 64;
+  t.rows = (void *)0x100000; t.pos = (int32_t *)0x200000;   /* never dereferenced by the dry run */
+  t.live_host = live; t.live_cap = 12; t.last = -1; t.refit_done = 1;
+  tabs[0] = &t;
+  for (pos = 0; pos < 16; ++pos) {
+    if (iskv_cache_plan(tabs, 1, 16, 64, 1, &folded, NULL) != ISKV_OK) return 2;
+    if (folded && first < 0) first = pos;
+  }
+  printf("%d %s %d %lld %lld\n", (int)iskv_abi_version(), iskv_status_string(ISKV_ERR_CAPACITY),
+         first, (long long)t.n_live, (long long)t.hist_rows);
+  return iskv_fold_workspace_size(1, 1024, 256, 64) > 0 ? 0 : 3;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/iskv.h compiles as strict C99 and a C program linked against libiskv.so runs the
+    host-side entry points (no GPU needed)."""
+    L, lib = _lib()
+    src = tmp_path / "caller.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(L.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir,
+                    "-liskv", f"-Wl,-rpath,{libdir}"], check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    # first fold with position W + b - 1 = 11; after 16 positions: 8 folded, 8 live
+    assert out == ["1", "history", "capacity", "exceeded", "11", "8", "8"]
