@@ -165,3 +165,33 @@ def test_argument_errors():
     side, _ = op.new_side(10, [], 0, 4, 2, 0)
     with pytest.raises(ValueError):
         op.append(side, 12)                        # positions arrive one at a time
+
+
+def test_policy_then_attention_equals_dense_attention():
+    """Algorithm 3 steps 1-9 compose: with K and V rows of rank below the budget, attention over the
+    policy's K and V (different protected sets, so row i of the two histories is not the same
+    token) equals attention over the dense sequence."""
+    from oracle import attention as oatt
+    from oracle import rope
+
+    d, hd, n_kv, r, b, W, L, T = 64, 32, 2, 8, 4, 6, 30, 40
+    g = synth.rng(31)
+    K = g.standard_normal((L + T, 4)) @ g.standard_normal((4, d))
+    V = g.standard_normal((L + T, 3)) @ g.standard_normal((3, d))
+    PK = [0, 1, 27, 28, 29]
+    PV = [0, 1, 2, 5, 26, 27, 28, 29]
+    ok = op.run_decode(K[:L], K[L:], PK, 0, W, b, r, 8)
+    ov = op.run_decode(V[:L], V[L:], PV, W, W, b, r, 8, refit_rows=8)
+    assert ok["history"][3].tolist() != ov["history"][3].tolist()
+    q = g.standard_normal((4, hd))
+    n = L + T
+    got = oatt.decode_attention(ok["history"], ov["history"], ok["exact"][0], ok["exact"][1],
+                                ov["exact"][0], ov["exact"][1], n, q, n_kv, hd)
+    Kr = rope.apply_rope(K, np.arange(n), n_kv, hd, 500000.0)
+    want = np.zeros((4, hd))
+    for j in range(4):
+        h = j // 2
+        s = Kr[:, h * hd:(h + 1) * hd] @ q[j] / np.sqrt(hd)
+        p = np.exp(s - s.max())
+        want[j] = (p / p.sum()) @ V[:, h * hd:(h + 1) * hd]
+    np.testing.assert_allclose(got, want, atol=1e-9)
