@@ -272,7 +272,7 @@ iskv_status iskv_select_prompt_blocks_noalloc(const void *keys, int32_t k_dtype,
 
 /*
  * Cache policy: the exact rows of one side (K or V) of one (sequence, layer), and when its pending
- * rows are folded (Section 3.1, Section 3.2; Algorithm 1 steps 5-8, Algorithm 3 steps 1-6).
+ * rows are folded (Section 3.1, Section 3.2; Algorithm 1 steps 5-9, Algorithm 3 steps 1-6).
  *
  * A side keeps exact: its protected rows P_X (fixed at prefill), the rows at the `window` most recent
  * positions, and the pending FIFO (unprotected rows that have left the window and wait for a full
@@ -329,7 +329,8 @@ typedef struct {
 } iskv_exact_table;
 
 /*
- * Prefill partition (Algorithm 1 steps 5-7): split the L prompt rows X [L][d] (x_dtype) of one side.
+ * Prefill partition (Algorithm 1 steps 5-9): split the L prompt rows X [L][d] (x_dtype) of one
+ * side.
  *   protected_pos [n_protected]  int32, strictly ascending, inside [0, L): P_X (for keys the
  *                                selection's P_K, for values its P_V).
  *   init_window                  0 for keys, min(W, L) for values; 0 <= init_window <= t->window.
@@ -338,9 +339,8 @@ typedef struct {
  * comp_rows [L][d] (x_dtype) with comp_pos [L]: the rows the prompt's truncated SVD compresses
  * (Algorithm 1 step 7; that SVD itself is not part of the library). Sets the host mirror
  * (n_prot = n_protected, n_live, live_host, last = L - 1, fold_rows = 0, hist_rows = *n_comp,
- * refit_done = (refit_rows == 0)) and
- * *n_comp (host). The caller then puts the compressed rows' factors in the side's history, with
- * their positions comp_pos in its position table.
+ * refit_done = (refit_rows == 0)) and *n_comp (host). The caller then puts the compressed rows'
+ * factors in the side's history, with their positions comp_pos in its position table.
  * SYNCHRONOUS: waits for the stream, because the mirror needs the live positions. Errors:
  * ISKV_ERR_ARG for null / misaligned pointers, bad dtypes, init_window out of range, or
  * protected_pos not strictly ascending inside [0, L) (found on the device, reported after the
@@ -354,7 +354,7 @@ iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dty
                                int64_t *n_comp, void *ws, size_t ws_bytes, void *stream);
 
 /*
- * One decode step for `count` tables (Algorithm 3 steps 1-2 and 4-6): tables[i] (host pointer to a
+ * One decode step for `count` tables (Algorithm 3 steps 1-6): tables[i] (host pointer to a
  * host struct, updated in place) with its history hists[i] (host pointer) stores new_rows[i] (device
  * [count][d], row_dtype, converted to the table dtype) at position tables[i]->last + 1; when that
  * makes `block` rows pending, the oldest `block` of them are folded into hists[i]
@@ -362,16 +362,16 @@ iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dty
  * history's position table and their exact copies leave the table; when a table's folded rows
  * reach reorth_rows, its history is re-orthogonalised (iskv_reorth) in the same step and the count
  * restarts. A table whose first refit is still to come waits for refit_rows pending rows instead,
- * then folds all of them (in one fold or in untruncated block folds, as above). All tables share d, window,
- * block and dtype; the histories share d, r_max, storage and n_cap, as the batched fold and
- * re-orthogonalisation require. folded / reorthed (host [count], may be NULL) receive 1 where a
+ * then folds all of them (in one fold or in untruncated block folds, as above). All tables share
+ * d, window, block and dtype; the histories share d, r_max, storage and n_cap, as the batched fold
+ * and re-orthogonalisation require. folded / reorthed (host [count], may be NULL) receive 1 where a
  * table folded a block (2 where it ran its first refit) / re-orthogonalised. Stream-ordered; the
  * host mirror is updated at once. The workspace query takes the largest refit_rows of the tables
  * (0 when none refits). Errors (nothing launched, no table changed): ISKV_ERR_ARG,
  * ISKV_ERR_SHAPE (mixed table shapes, a history whose d differs, a block the fold does not take, a
- * refit that can be run neither way),
- * ISKV_ERR_CAPACITY (a table without room for the new row, or a history without room for the
- * block or the refit: hist_rows + block > n_cap), ISKV_ERR_WORKSPACE; ISKV_ERR_CUDA when a launch fails.
+ * refit that can be run neither way), ISKV_ERR_CAPACITY (a table without room for the new row, or
+ * a history without room for the block or the refit: hist_rows + rows > n_cap),
+ * ISKV_ERR_WORKSPACE; ISKV_ERR_CUDA when a launch fails.
  */
 size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block,
                                       int64_t n_cap, int32_t refit_rows);
