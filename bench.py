@@ -1,27 +1,33 @@
 #!/usr/bin/env python
 """Benchmark of the iS-KV hot path on B200.
 
-Workload (one GPU): the decode step of a 32-layer GQA model (8 KV heads x head_dim 128, so
+Workload (one GPU): the decode steps of a 32-layer GQA model (8 KV heads x head_dim 128, so
 d = 1024) at which every layer's K and V pending queue fills at once -- 64 compressed histories at
 n ~ 16384 rows, rank r = 256, fold block b = 64, bf16 factors. One timed step runs every row of the
-hot path once:
+hot path:
 
   1. fold (Algorithm 2): one 64-row block into each of the 64 histories (one batched call);
-  2. re-orthogonalisation (Section 4.4) of all 64 histories (one batched call);
+  2. re-orthogonalisation (Section 4.4) of all 64 histories, every 4th step: the pages' cadence of
+     one re-orthogonalisation per 256 folded rows;
   3. reconstruction (Algorithm 3 steps 7-8) of all 64 caches -- compressed rows plus 640 exact rows
      (512-token prompt kept exact, 128-row recent window), RoPE theta = 500000 on K;
   4. prompt-block selection (Algorithm 1 steps 2-4) on one layer's 65536-token post-RoPE prompt.
 
-n grows by 64 rows per step; it starts so that the timed steps are centred on n = 16384. Inputs are
-seeded synthetic low-rank-plus-noise rows (K spectrum i^-1.2, V i^-0.6, noise 0.02) standing in for
-model traces. Everything a step reads is resident in HBM before timing starts; a step touches
-~4 GB, far more than the 126 MB L2, so no flush is needed.
+Inputs: every history is built on the device by folding seeded synthetic rows from the start, and
+the timed steps fold the rows that follow: per history, G diag(s) H(t)^T + 0.02 N(0, 1) with
+s_j = j^-1.2 (keys) or j^-0.6 (values) and a dominant subspace H(t) that turns by 0.05 rad per
+1024 rows (the decode-simulation workload), standing in for model traces. n starts so that the
+timed steps are centred on n = 16384. Everything a step reads is resident in HBM before timing
+starts; a step touches ~4 GB, far more than the 126 MB L2, so no flush is needed.
 
-metric: block folds/s (64 folds per step); the line also reports reconstructed KV rows/s and, per
-stage, device time and the achieved fraction of the measured HBM roofline.
+metric: block folds/s (64 folds per step); the line also reports reconstructed KV rows/s, per-stage
+device time with its roofline fraction (HBM for the streaming kernels, the float32 CUDA-core peak
+for the Jacobi core SVD), the core's sweep counts, rates at the sweep workload's cadence (one
+re-orthogonalisation per 16 folds), and the eq. (14) factor drift of one K and one V history.
 
---impl reference times the float64 CPU oracle on a bounded sample of the same step (one fold,
-one reorth and one reconstruction at n = 16384, one selection) and extrapolates to a whole step.
+--impl reference times the float64 CPU oracle, one history's share of a step per timed step.
+--gpus N runs N ranks (one process per GPU, launched through torch.distributed.run when the
+caller did not); --dry-run exercises that plumbing on CPU processes without a GPU.
 """
 
 from __future__ import annotations
@@ -48,6 +54,10 @@ SEL_L = 65536
 Q_HEADS = 32  # decode-attention query heads (grouped: 4 per KV head)
 SPEC = {"K": 1.2, "V": 0.6}
 NOISE = 0.02
+DRIFT_RAD_PER_1K = 0.05  # rotation of the rows' dominant subspace per 1024 rows
+REORTH_EVERY = 4         # folds per re-orthogonalisation: 256 rows at b = 64, as on the pages
+SWEEP_REORTH_EVERY = 16  # the cadence of the sweep workload
+SMS, FP32_LANES = 148, 128  # B200: SMs, float32 FMA lanes per SM
 
 
 def peaks():
@@ -136,7 +146,8 @@ def rank_seed(rank: int) -> int:
 # The B200 arm.
 
 class Workload:
-    """64 histories (32 layers x {K, V}) and every per-step input, resident on the device."""
+    """64 histories (32 layers x {K, V}) built on the device from drifting synthetic rows, and
+    every per-step input, resident on the device."""
 
     def __init__(self, kv, torch, dev, warmup: int, timed: int, extra: int, seed: int = 1000,
                  layers: int = LAYERS):
@@ -144,40 +155,39 @@ class Workload:
         self.kv, self.torch, self.dev = kv, torch, dev
         # n after the fold of step t is n0 + 64 (t + 1); the timed steps are centred on N_MID.
         self.n0 = N_MID - BLK * (warmup + (timed + 1) // 2)
-        self.n_cap = self.n0 + BLK * (warmup + timed + extra + 1)
-        self.hists, self.kinds = [], []
-        gen = torch.Generator(device=dev)
-        for layer in range(layers):
-            for kind in ("K", "V"):
-                h = kv.LowRankHistory(D, R, self.n_cap, storage=torch.bfloat16, device=dev)
-                sd = seed + 2 * layer + (kind == "V")
-                U = synth.torch_orthonormal(self.n0, R, sd, device=dev)
-                B = synth.torch_orthonormal(D, R, sd + 50000, device=dev)
-                s = (self.n0 ** 0.5) * torch.arange(1, R + 1, device=dev,
-                                                    dtype=torch.float32) ** (-SPEC[kind])
-                h.U[:self.n0] = U.to(torch.bfloat16)
-                h.B.copy_(B.to(torch.bfloat16))
-                h.sigma.copy_(s)
-                h.pos[:self.n0] = torch.arange(PROMPT, PROMPT + self.n0, dtype=torch.int32,
-                                               device=dev)
-                h.meta.copy_(torch.tensor([R, self.n0, 0, 0], dtype=torch.int64))
-                self.hists.append(h)
-                self.kinds.append(kind)
-        # Pending blocks: rows in the history's subspace plus noise (4 rotating sets).
-        self.F = []
-        for sset in range(4):
-            blocks = []
-            for i, h in enumerate(self.hists):
-                gen.manual_seed(seed + 7919 * sset + i)
-                a = SPEC[self.kinds[i]]
-                coef = torch.randn(BLK, R, generator=gen, device=dev) * (
-                    torch.arange(1, R + 1, device=dev, dtype=torch.float32) ** (-a))
-                rows = coef @ h.B.float().T + NOISE * torch.randn(BLK, D, generator=gen, device=dev)
-                blocks.append(rows.to(torch.bfloat16).contiguous())
-            self.F.append(blocks)
+        self.n_cap = self.n0 + BLK * (warmup + timed + extra + 2)
+        self.kinds = [kind for _ in range(layers) for kind in ("K", "V")]
+        cnt = len(self.kinds)
+        self.hists = [kv.LowRankHistory(D, R, self.n_cap, storage=torch.bfloat16, device=dev)
+                      for _ in range(cnt)]
+        # Workspaces (sized once).
+        self.ws_fold = torch.empty(kv.fold_workspace_size(cnt, D, R, BLK) + 256,
+                                   dtype=torch.uint8, device=dev)
+        self.ws_reorth = torch.empty(kv.reorth_workspace_size(cnt, D, R, self.n_cap) + 256,
+                                     dtype=torch.uint8, device=dev)
+        self.ws_recon = torch.empty(kv.reconstruct_workspace_size(cnt, D, R) + 256,
+                                    dtype=torch.uint8, device=dev)
+        self.ws_sel = torch.empty(kv.select_workspace_size(SEL_L, HEADS, 8) + 256,
+                                  dtype=torch.uint8, device=dev)
+        # Build: fold the first n0 rows of every stream, re-orthogonalising on the step's cadence.
+        # The rows of layer 0's K and V histories are kept for the factor-drift measurement.
+        self.drift = synth.DriftingRows(cnt, D, [SPEC[k] for k in self.kinds], NOISE, seed, BLK,
+                                        angle_per_1k=DRIFT_RAD_PER_1K, device=dev)
+        self.kept = [torch.empty(self.n_cap, D, dtype=torch.bfloat16, device=dev)
+                     for _ in range(2)]
+        for g in range(self.n0 // BLK):
+            F = self.drift.next_blocks().to(torch.bfloat16)
+            for i in range(2):
+                self.kept[i][g * BLK:(g + 1) * BLK].copy_(F[i])
+            self._fold(g, F)
+        # Pending blocks of every later step (warm-up, timed, end-to-end, one spare).
+        self.F = [self.drift.next_blocks().to(torch.bfloat16)
+                  for _ in range(warmup + timed + extra + 1)]
+        self.drift = None  # release the generator's d x d matrices
         # Exact rows per history: 512 prompt rows + 128 window rows.
+        gen = torch.Generator(device=dev)
         self.exact = []
-        for i in range(len(self.hists)):
+        for i in range(cnt):
             gen.manual_seed(seed + 31337 + i)
             self.exact.append((torch.randn(PROMPT + WINDOW, D, generator=gen, device=dev)
                                ).to(torch.bfloat16).contiguous())
@@ -189,49 +199,57 @@ class Workload:
         keys, _ = synth.outlier_prompt_keys(SEL_L, HEADS, HEAD_DIM, seed=4)
         self.keys = torch.as_tensor(keys, dtype=torch.float32).to(dev).to(torch.bfloat16)
         self.sel_out = None
-        # Workspaces (sized once).
-        cnt = len(self.hists)
-        self.ws_fold = torch.empty(kv.fold_workspace_size(cnt, D, R, BLK) + 256,
-                                   dtype=torch.uint8, device=dev)
-        self.ws_reorth = torch.empty(kv.reorth_workspace_size(cnt, D, R, self.n_cap) + 256,
-                                     dtype=torch.uint8, device=dev)
-        self.ws_recon = torch.empty(kv.reconstruct_workspace_size(cnt, D, R) + 256,
-                                    dtype=torch.uint8, device=dev)
-        self.ws_sel = torch.empty(kv.select_workspace_size(SEL_L, HEADS, 8) + 256,
-                                  dtype=torch.uint8, device=dev)
-        # Per-step positions.
-        self.step_idx = 0
         torch.cuda.synchronize(dev)
+
+    def _fold(self, g, F, stream=None):
+        """Fold block g (global block index; rows g*64 .. g*64+63 of every stream) and, when the
+        cadence says so, re-orthogonalise."""
+        torch, kv = self.torch, self.kv
+        fpos = torch.arange(PROMPT + g * BLK, PROMPT + (g + 1) * BLK, dtype=torch.int32,
+                            device=self.dev)
+        kv.fold_block_batched(self.hists, list(F), [fpos] * len(self.hists),
+                              ws=self._aligned(self.ws_fold), stream=stream)
+        if (g + 1) % REORTH_EVERY == 0:
+            kv.reorth(self.hists, ws=self._aligned(self.ws_reorth), stream=stream)
 
     @staticmethod
     def _aligned(buf):
         off = (-buf.data_ptr()) % 256
         return buf[off:]
 
+    def folded_rows(self, i, steps):
+        """Every row history i (0: layer 0's K, 1: its V) has folded after `steps` steps."""
+        for t in range(steps):
+            g = self.n0 // BLK + t
+            self.kept[i][g * BLK:(g + 1) * BLK].copy_(self.F[t][i])
+        return self.kept[i][:self.n0 + BLK * steps]
+
     def n_after(self, t):
         return self.n0 + BLK * (t + 1)
 
+    def reorths_in(self, t0, t1):
+        """Re-orthogonalisations run by steps t0 .. t1-1."""
+        g0 = self.n0 // BLK
+        return sum(1 for t in range(t0, t1) if (g0 + t + 1) % REORTH_EVERY == 0)
+
     def positions(self, t):
         torch = self.torch
-        n_before = self.n0 + BLK * t
-        fpos = torch.arange(PROMPT + n_before, PROMPT + n_before + BLK, dtype=torch.int32,
-                            device=self.dev)
-        n = n_before + BLK
+        n = self.n_after(t)
         epos = torch.cat([torch.arange(0, PROMPT, dtype=torch.int32, device=self.dev),
                           torch.arange(PROMPT + n, PROMPT + n + WINDOW, dtype=torch.int32,
                                        device=self.dev)])
-        return fpos, epos, PROMPT + n + WINDOW
+        return epos, PROMPT + n + WINDOW
 
-    def step(self, t, fpos, epos, n_total, F=None):
+    def step(self, t, epos, n_total, F=None, stream=None):
         kv = self.kv
-        F = F if F is not None else self.F[t % 4]
-        cnt = len(self.hists)
-        kv.fold_block_batched(self.hists, F, [fpos] * cnt, ws=self._aligned(self.ws_fold))
-        kv.reorth(self.hists, ws=self._aligned(self.ws_reorth))
-        kv.reconstruct_batched(self.hists, self.exact, [epos] * cnt, n_total, HEADS, HEAD_DIM,
-                               self.rope, THETA, outs=self.outs, ws=self._aligned(self.ws_recon))
+        F = F if F is not None else self.F[t]
+        self._fold(self.n0 // BLK + t, F, stream=stream)
+        kv.reconstruct_batched(self.hists, self.exact, [epos] * len(self.hists), n_total, HEADS,
+                               HEAD_DIM, self.rope, THETA, outs=self.outs,
+                               ws=self._aligned(self.ws_recon), stream=stream)
         self.sel_out = kv.select_prompt_blocks(self.keys, 8, 128, 4, 32,
-                                               ws=self._aligned(self.ws_sel), out=self.sel_out)
+                                               ws=self._aligned(self.ws_sel), out=self.sel_out,
+                                               stream=stream)
 
 
 ROOFLINE_STAGE = "reconstruct.compressed"
@@ -382,6 +400,60 @@ def time_cache_policy(wl, kv, torch, dev, stream):
                     "stage events"}
 
 
+def workload_config(layers: int, world: int):
+    """The workload's description, shared by both arms' JSON lines."""
+    return {"workload": "decode steps, 32 layers x {K,V} histories at n~16K (fold b=64 every step, "
+                        "reorth every 4 folds, reconstruct with RoPE + one 64K-token prompt "
+                        "selection per step)",
+            "layers": layers, "histories_per_gpu": 2 * layers, "d": D, "r": R, "b": BLK,
+            "n_center": N_MID, "kv_heads": HEADS, "head_dim": HEAD_DIM,
+            "exact_rows": PROMPT + WINDOW, "rope_theta": THETA, "select_prompt_tokens": SEL_L,
+            "storage": "bf16", "reorth_every_folds": REORTH_EVERY,
+            "inputs": f"rows G diag(s) H(t)^T + {NOISE} N(0,1), s_j = j^-1.2 (K) / j^-0.6 (V), "
+                      f"subspace drift {DRIFT_RAD_PER_1K} rad per 1024 rows; histories built by "
+                      f"folding the same streams from n = 0",
+            "parallelism": f"replicas x{world} (independent histories per GPU)",
+            "l2": "inputs > L2 (~4 GB touched per step), no flush"}
+
+
+def fp32_peak_tflops(sm_mhz):
+    """Float32 CUDA-core peak at the sampled SM clock: 148 SMs x 128 FMA lanes x 2 flop."""
+    mhz = sm_mhz or 1965.0
+    return SMS * FP32_LANES * 2 * mhz * 1e6 / 1e12
+
+
+def core_roofline(stats, stage, peak_tflops):
+    """Achieved float32 rate of the core SVD stage: the flops the kernel executed (counted on the
+    device: pair inner products and applied rotations) over its measured time, and the survey's
+    algorithmic count 7 (k + b)^3 flops per sweep per core for comparison."""
+    if not stats["cores"] or stage is None:
+        return None
+    ms = stage["ms_per_call"] * stage["calls"]
+    tflops = stats["flops"] / (ms / 1e3) / 1e12
+    return {"cores": stats["cores"], "sweeps_mean": round(stats["sweeps"] / stats["cores"], 3),
+            "sweeps_max": stats["max_sweeps"],
+            "rotations_per_core": round(stats["rotations"] / stats["cores"], 1),
+            "flops_per_core": round(stats["flops"] / stats["cores"], 1),
+            "achieved_tflops": round(tflops, 3), "peak_tflops": round(peak_tflops, 2),
+            "frac_fp32": round(tflops / peak_tflops, 4),
+            "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x median sampled SM clock"}
+
+
+def factor_drift(torch, X, h):
+    """Eq. (14) of the pages' appendix: the relative error of the history's factors against the
+    rows it folded, minus that of a fresh rank-r SVD of the same rows (float64, torch on the
+    device; a measurement, not part of the path)."""
+    k, n, _, _ = h.status()
+    Xd = X[:n].double()
+    inc = (h.U[:n, :k].double() * h.sigma[:k].double()) @ h.B[:, :k].double().T
+    nx = torch.linalg.matrix_norm(Xd)
+    e_inc = float(torch.linalg.matrix_norm(Xd - inc) / nx)
+    S = torch.linalg.svdvals(Xd)
+    e_svd = float(torch.sqrt(torch.sum(S[k:] ** 2)) / nx)
+    return {"n": int(n), "k": int(k), "rel_err_incremental": round(e_inc, 6),
+            "rel_err_fresh_svd": round(e_svd, 6), "factor_drift": round(e_inc - e_svd, 6)}
+
+
 def run_b200(args):
     import torch
     import torch.distributed as dist
@@ -401,8 +473,10 @@ def run_b200(args):
     kv._lib.load()
     steps_total = args.warmup + args.steps
     e2e_steps = 0 if args.no_e2e else args.steps
+    t_setup = time.perf_counter()
     wl = Workload(kv, torch, dev, args.warmup, args.steps, e2e_steps, seed=rank_seed(rank),
                   layers=args.layers)
+    setup_s = time.perf_counter() - t_setup
     pos = [wl.positions(t) for t in range(steps_total + e2e_steps)]
     stream = torch.cuda.current_stream(dev)
 
@@ -419,6 +493,7 @@ def run_b200(args):
     # Timed region (device events on the launching stream, stage events inside the library).
     sampler = ClockSampler(local, args.clock_log_dir)
     kv.stage_times(reset=True)
+    kv.core_stats(reset=True)
     kv.stage_timing(True)
     launches0 = kv.launch_count()
     sampler.start()
@@ -435,6 +510,8 @@ def run_b200(args):
     launches = kv.launch_count() - launches0
     kv.stage_timing(False)
     st = kv.stage_times(reset=True)
+    cstats = kv.core_stats(reset=True)
+    status_ok = all(h.status()[3] == 0 for h in wl.hists)
     ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_step = ms / args.steps
     folds_step = len(wl.hists)
@@ -442,14 +519,11 @@ def run_b200(args):
     value = world * folds_step * args.steps / (ms / 1e3)
     rows_step = len(wl.hists) * (PROMPT + n_mean + WINDOW)
     rows_per_s = world * rows_step * args.steps / (ms / 1e3)
+    n_reorth = wl.reorths_in(args.warmup, steps_total)
 
-    # Parity spot check of the benchmark state (one history, sampled rows) against the oracle.
-    check = None
-    if rank == 0 and not args.no_check:
-        check = spot_check(wl, torch)
-
-    # Stage rooflines.
+    # Stage rooflines: HBM for the streaming stages, float32 CUDA cores for the core SVDs.
     hbm, tc, peak_kind = peaks()
+    fp32 = fp32_peak_tflops(clocks.get("sm_mhz"))
     sbytes, _ = stage_bytes(n_mean, args.layers)
     stages = {}
     for name, (tot_ms, calls) in st.items():
@@ -463,19 +537,58 @@ def run_b200(args):
             ent.update({"bytes_per_call": int(sbytes[name]), "achieved_gbs": round(gbs, 1),
                         "frac_hbm": round(gbs / hbm, 4)})
         stages[name] = ent
+    core = {"fold": core_roofline(cstats["fold"], stages.get("fold.core_svd"), fp32),
+            "reorth": core_roofline(cstats["reorth"], stages.get("reorth.core_svd"), fp32)}
     dom = max(stages, key=lambda k: stages[k]["ms_per_call"] * stages[k]["calls"])
-    # The roofline line reports the reconstruction kernel: the step's largest HBM-bound kernel
-    # with an algorithmic byte count (the Jacobi stages have none independent of their sweeps).
-    rl_name = ROOFLINE_STAGE if ROOFLINE_STAGE in stages else max(
-        (k for k in stages if k in sbytes), key=lambda k: stages[k]["ms_per_call"])
-    rl = stages[rl_name]
-    traffic, earlier = load_traffic(rl_name)
-    roofline = {"kernel": rl_name, "bound": "hbm", "achieved": rl["achieved_gbs"],
-                "peak": hbm, "unit": "GB/s", "frac": rl["frac_hbm"],
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
-                "traffic": traffic, "dominant_stage": dom}
+    traffic, earlier = load_traffic(ROOFLINE_STAGE)
+    rl_hbm = {"kernel": ROOFLINE_STAGE, "bound": "hbm",
+              "achieved": stages[ROOFLINE_STAGE]["achieved_gbs"], "peak": hbm, "unit": "GB/s",
+              "frac": stages[ROOFLINE_STAGE]["frac_hbm"],
+              "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+              "traffic": traffic}
     if earlier is not None:
-        roofline["traffic_earlier_capture"] = earlier
+        rl_hbm["traffic_earlier_capture"] = earlier
+    rl_rot = None
+    if "fold.coord_rotate" in stages:
+        rr = stages["fold.coord_rotate"]
+        rl_rot = {"kernel": "fold.coord_rotate", "bound": "hbm", "achieved": rr["achieved_gbs"],
+                  "peak": hbm, "unit": "GB/s", "frac": rr["frac_hbm"],
+                  "traffic": load_traffic("fold.coord_rotate")[0]}
+    # The roofline line reports the dominant stage: the fold's core SVD (float32 ALU-bound) when
+    # it dominates, else the largest HBM-bound stage.
+    if dom in ("fold.core_svd", "reorth.core_svd") and core[dom.split(".")[0]] is not None:
+        c = core[dom.split(".")[0]]
+        roofline = {"kernel": f"{dom} (k_core)", "bound": "alu", "achieved": c["achieved_tflops"],
+                    "peak": c["peak_tflops"], "unit": "TFLOP/s", "frac": c["frac_fp32"],
+                    "peak_source": c["peak_source"], "traffic": load_traffic(dom)[0],
+                    "dominant_stage": dom}
+    else:
+        roofline = dict(rl_hbm, dominant_stage=dom)
+
+    # Rates at the sweep workload's cadence (one re-orthogonalisation per 16 folds), from the
+    # measured stage times of this run.
+    fold_ms = sum(v["ms_per_call"] * v["calls"] for k, v in stages.items()
+                  if k.startswith("fold.")) / args.steps
+    reorth_ms = (sum(v["ms_per_call"] * v["calls"] for k, v in stages.items()
+                     if k.startswith("reorth.")) / max(n_reorth, 1))
+    recon_ms = sum(v["ms_per_call"] for k, v in stages.items() if k.startswith("reconstruct."))
+    cadence = {
+        "fold_ms_per_call": round(fold_ms, 4), "reorth_ms_per_call": round(reorth_ms, 4),
+        "reconstruct_ms_per_call": round(recon_ms, 4),
+        "folds_per_s_fold_only": round(folds_step / (fold_ms / 1e3), 1),
+        f"folds_per_s_reorth_every_{REORTH_EVERY}": round(
+            folds_step / ((fold_ms + reorth_ms / REORTH_EVERY) / 1e3), 1),
+        f"folds_per_s_reorth_every_{SWEEP_REORTH_EVERY}": round(
+            folds_step / ((fold_ms + reorth_ms / SWEEP_REORTH_EVERY) / 1e3), 1),
+        "reorths_per_s": round(folds_step / (reorth_ms / 1e3), 1),
+        "note": "fold-only and cadence rates are sums of this run's stage times (CUDA events)"}
+
+    # Eq. (14) factor drift of layer 0's K and V histories against the rows they folded.
+    drift = None
+    if not args.no_check:
+        drift = {kind: factor_drift(torch, wl.folded_rows(i, steps_total), wl.hists[i])
+                 for i, kind in enumerate(("K", "V"))}
+        drift["pages_table5_fp16_factors"] = {"K": [0.0016, 0.0071], "V": [0.0160, 0.0207]}
 
     # Diagnostics of the benchmark state (eq. 12 bytes, factor orthogonality).
     diag = None
@@ -507,26 +620,23 @@ def run_b200(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "decode step, 32 layers x {K,V} histories at n~16K "
-                                   "(fold b=64 + reorth + reconstruct with RoPE + one 64K-token "
-                                   "prompt selection)",
-                       "layers": args.layers, "histories_per_gpu": folds_step, "d": D, "r": R,
-                       "b": BLK, "n_mean": n_mean, "kv_heads": HEADS, "head_dim": HEAD_DIM,
-                       "exact_rows": PROMPT + WINDOW, "rope_theta": THETA,
-                       "select_prompt_tokens": SEL_L, "storage": "bf16",
-                       "parallelism": f"replicas x{world} (independent histories per GPU)",
-                       "l2": "inputs > L2 (~4 GB touched per step), no flush"},
+            "config": dict(workload_config(args.layers, world), n_mean=n_mean),
             "reconstructed_rows_per_s": round(rows_per_s, 1),
             "roofline": roofline,
+            "roofline_kernels": {"reconstruct.compressed": rl_hbm, "fold.coord_rotate": rl_rot},
+            "core_svd": core,
             "stages": stages,
+            "cadence_rates": cadence,
+            "factor_drift_eq14": drift,
+            "status_ok": status_ok,
             "e2e": e2e,
             "gpu_launches": int(launches),
             "clocks": clocks,
             "cpu_baseline": cpu,
-            "parity_spot_check": check,
             "decode_attention": attn,
             "diagnostics": diag,
             "cache_policy": policy,
+            "setup_s": round(setup_s, 2),
         }
         print(json.dumps(line))
     if world > 1:
@@ -552,46 +662,23 @@ def load_traffic(stage: str):
                   "note": ent.get("note", "")}
 
 
-def spot_check(wl, torch):
-    """Oracle check of the benchmark's own state: the reconstruction of one K history (sampled
-    rows, RoPE) against the float64 definition."""
-    import numpy as np
-
-    from oracle import fold as of
-    from oracle import reconstruct as orec
-    h = wl.hists[0]
-    k, n, _, st = h.status()
-    U = h.U[:n, :k].double().cpu().numpy()
-    s = h.sigma[:k].double().cpu().numpy()
-    B = h.B[:, :k].double().cpu().numpy()
-    pos = h.pos[:n].cpu().numpy()
-    rows = np.random.Generator(np.random.PCG64(0)).choice(n, 256, replace=False)
-    out = wl.outs[0]
-    ref = orec.reconstruct(U[rows], s, B, pos[rows], np.zeros((0, D)), np.zeros(0, dtype=int),
-                           int(pos.max()) + 1, HEADS, HEAD_DIM, True, THETA)
-    got = out[torch.as_tensor(pos[rows], dtype=torch.long, device=out.device)].double().cpu().numpy()
-    err = of.rel_fro(got, ref[pos[rows]])
-    return {"history": "layer0.K", "k": k, "n": n, "status_bits": st,
-            "recon_rel_fro_sampled": float(err), "tol": 2e-2, "ok": bool(err < 2e-2 and st == 0)}
-
-
 def run_e2e(wl, kv, torch, dev, stream, pos, first_step, steps, world):
-    """Same step through the C ABI, with the step's inputs copied from pinned host memory and the
-    step's result (every history's sigma and meta word, and the selection outputs) copied back.
-    As a serving loop would, the inputs of step t+1 are copied on a second stream while step t
-    computes (two device input buffers, ordered by events); every copy of every step, and the
-    result read-back, lie inside the timed region."""
+    """Same steps through the C ABI, with each step's inputs (its 64 pending blocks and the prompt
+    keys) copied from pinned host memory and the step's result (every history's sigma and meta
+    word, and the selection outputs) copied back. As a serving loop would, the inputs of step t+1
+    are copied on a second stream while step t computes (two device input buffers, ordered by
+    events); every copy of every step, and the result read-back, lie inside the timed region."""
     cnt = len(wl.hists)
-    hostF = [[f.cpu().pin_memory() for f in s] for s in wl.F]
+    hostF = [wl.F[first_step + i].cpu().pin_memory() for i in range(steps)]
     hostK = wl.keys.cpu().pin_memory()
-    devF = [[torch.empty_like(f) for f in wl.F[0]] for _ in range(2)]
+    devF = [torch.empty_like(wl.F[0]) for _ in range(2)]
     devK = [torch.empty_like(wl.keys) for _ in range(2)]
     res_sig = torch.empty(cnt, R, dtype=torch.float32).pin_memory()
     res_meta = torch.empty(cnt, 4, dtype=torch.int64).pin_memory()
     res_cnt = torch.empty(2 + HEADS, dtype=torch.int64).pin_memory()
     res_pk = torch.empty(SEL_L, dtype=torch.int32).pin_memory()
     res_pv = torch.empty(SEL_L, dtype=torch.int32).pin_memory()
-    h2d = sum(f.numel() * f.element_size() for f in hostF[0]) + hostK.numel() * hostK.element_size()
+    h2d = hostF[0].numel() * hostF[0].element_size() + hostK.numel() * hostK.element_size()
     d2h = (res_sig.numel() * 4 + res_meta.numel() * 8 + res_cnt.numel() * 8 + res_pk.numel() * 4
            + res_pv.numel() * 4)
     keys_dev = wl.keys
@@ -604,9 +691,7 @@ def run_e2e(wl, kv, torch, dev, stream, pos, first_step, steps, world):
         with torch.cuda.stream(copy_stream):
             if i >= 2:
                 copy_stream.wait_event(free[b])
-            hf = hostF[(first_step + i) % 4]
-            for j in range(cnt):
-                devF[b][j].copy_(hf[j], non_blocking=True)
+            devF[b].copy_(hostF[i], non_blocking=True)
             devK[b].copy_(hostK, non_blocking=True)
             ready[b].record(copy_stream)
 
@@ -650,71 +735,92 @@ def run_e2e(wl, kv, torch, dev, stream, pos, first_step, steps, world):
 # CPU oracle legs (the baseline the task asks for; never a target).
 
 _KEYS = {}
+SEL_SLICE = SEL_L // (2 * LAYERS)  # one history's share of the step's prompt selection
 
 
-def _oracle_sample(seed=7):
-    """Float64 oracle on one history of the step: fold, reorth and reconstruction at n = 16384,
-    plus one prompt selection. Returns the seconds of each part."""
+def _oracle_inputs(seed):
     import numpy as np
-
-    import synth
-    from oracle import fold as of
-    from oracle import reconstruct as orec
-    from oracle import reorth as oreo
-    from oracle import select as osel
     g = np.random.Generator(np.random.PCG64(seed))
     n = N_MID
     U = np.linalg.qr(g.standard_normal((n, R)))[0]
     B = np.linalg.qr(g.standard_normal((D, R)))[0]
     s = np.sqrt(n) * np.arange(1, R + 1) ** -1.2
-    F = (g.standard_normal((BLK, R)) * np.arange(1, R + 1) ** -1.2) @ B.T + NOISE * g.standard_normal((BLK, D))
+    F = ((g.standard_normal((BLK, R)) * np.arange(1, R + 1) ** -1.2) @ B.T
+         + NOISE * g.standard_normal((BLK, D)))
+    ex = g.standard_normal((PROMPT + WINDOW, D))
+    return U, s, B, F, ex
+
+
+def _oracle_sample(seed, reorth: bool):
+    """One history's share of a step, on the float64 oracle: a fold at n = 16384, d = 1024,
+    r = 256, b = 64, a re-orthogonalisation when the cadence has one, the reconstruction of the
+    history's cache with RoPE, and the selection of a 1024-token prompt slice (1/64 of the step's
+    65536-token selection). Returns the seconds of each part (inputs are drawn untimed)."""
+    import synth
+    from oracle import fold as of
+    from oracle import reconstruct as orec
+    from oracle import reorth as oreo
+    from oracle import select as osel
+    import numpy as np
+    U, s, B, F, ex = _oracle_inputs(seed)
+    if "k" not in _KEYS:
+        _KEYS["k"] = synth.outlier_prompt_keys(SEL_SLICE, HEADS, HEAD_DIM, seed=4)[0]
     t = {}
     a = time.perf_counter()
     res = of.fold_block(U, s, B, F, R)
     t["fold"] = time.perf_counter() - a
+    U2, s2, B2 = res.U, res.sigma, res.B
+    t["reorth"] = 0.0
+    if reorth:
+        a = time.perf_counter()
+        U2, s2, B2 = oreo.reorth(U2, s2, B2)
+        t["reorth"] = time.perf_counter() - a
+    n = U2.shape[0]
     a = time.perf_counter()
-    U2, s2, B2 = oreo.reorth(res.U, res.sigma, res.B)
-    t["reorth"] = time.perf_counter() - a
-    a = time.perf_counter()
-    pos = np.arange(PROMPT, PROMPT + U2.shape[0])
-    ex = g.standard_normal((PROMPT + WINDOW, D))
-    epos = np.r_[np.arange(PROMPT), np.arange(PROMPT + U2.shape[0], PROMPT + U2.shape[0] + WINDOW)]
-    orec.reconstruct(U2, s2, B2, pos, ex, epos, PROMPT + U2.shape[0] + WINDOW, HEADS, HEAD_DIM,
-                     True, THETA)
+    pos = np.arange(PROMPT, PROMPT + n)
+    epos = np.r_[np.arange(PROMPT), np.arange(PROMPT + n, PROMPT + n + WINDOW)]
+    orec.reconstruct(U2, s2, B2, pos, ex, epos, PROMPT + n + WINDOW, HEADS, HEAD_DIM, True, THETA)
     t["reconstruct"] = time.perf_counter() - a
-    if "k" not in _KEYS:
-        _KEYS["k"] = synth.outlier_prompt_keys(SEL_L, HEADS, HEAD_DIM, seed=4)[0]
     a = time.perf_counter()
     osel.select_prompt_blocks(_KEYS["k"], 8, 128, 4, 32)
-    t["select"] = time.perf_counter() - a
+    t["select_slice"] = time.perf_counter() - a
     return t
 
 
-def _cpu_threads():
+def _host_cores():
+    """Cores this process may run on, and the BLAS thread count."""
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    blas = None
     try:
         from threadpoolctl import threadpool_info
-        info = threadpool_info()
-        return max((i.get("num_threads", 1) for i in info), default=1)
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=None)
     except Exception:
-        return os.cpu_count() or 1
+        pass
+    return int(cores or 1), blas
+
+
+ORACLE_SAMPLE = ("each step = one history's share of a B200 step on the float64 NumPy oracle: 1 "
+                 "fold at n=16384, d=1024, r=256, b=64 + 1 reorth on every 4th step + 1 "
+                 "reconstruction of 640 exact + ~16K compressed rows with RoPE + the selection of a "
+                 "1024-token prompt slice (1/64 of the 65536-token selection)")
 
 
 def cpu_baseline(budget_s: float):
-    reps, total, parts = 0, 0.0, None
-    while reps == 0 or (total < budget_s and reps < 3):
-        t = _oracle_sample(seed=7 + reps)
-        parts = t if parts is None else {k: parts[k] + t[k] for k in t}
+    """The oracle timed on this host's cores on a bounded sample of the workload (about
+    `budget_s` seconds of CPU work); folds/s = samples / their total time."""
+    _oracle_sample(99, False)  # untimed: imports, BLAS start-up, the prompt keys
+    reps, total, parts = 0, 0.0, {}
+    while reps < REORTH_EVERY or (total < budget_s and reps < 4 * REORTH_EVERY):
+        t = _oracle_sample(7 + reps, (reps + 1) % REORTH_EVERY == 0)
+        for k, v in t.items():
+            parts[k] = parts.get(k, 0.0) + v
         total += sum(t.values())
         reps += 1
-    parts = {k: v / reps for k, v in parts.items()}
-    hist = LAYERS * 2
-    step_s = hist * (parts["fold"] + parts["reorth"] + parts["reconstruct"]) + parts["select"]
-    return {"value": round(hist / step_s, 4), "unit": "folds/s", "cores": _cpu_threads(),
-            "kind": "oracle",
-            "sample": (f"{reps} x (1 fold + 1 reorth + 1 reconstruction at n=16384, d=1024, r=256, "
-                       f"+ 1 selection of a 65536-token prompt), float64 NumPy; a step = 64 x "
-                       f"(fold+reorth+reconstruct) + 1 selection"),
-            "seconds_per_part": {k: round(v, 4) for k, v in parts.items()}}
+    cores, blas = _host_cores()
+    return {"value": round(reps / total, 4), "unit": "folds/s", "cores": cores,
+            "blas_threads": blas, "kind": "oracle",
+            "sample": f"{reps} steps, {round(total, 2)} s; " + ORACLE_SAMPLE,
+            "seconds_per_part": {k: round(v / reps, 4) for k, v in parts.items()}}
 
 
 def run_reference(args):
@@ -722,38 +828,89 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    _oracle_sample(seed=99)  # one untimed pass: imports, BLAS start-up, the prompt keys
+    for i in range(args.warmup):   # untimed: imports, BLAS start-up, the prompt keys
+        _oracle_sample(99 + i, False)
     steps_s = []
     for i in range(args.steps):
-        t = _oracle_sample(seed=100 + i)
-        steps_s.append(LAYERS * 2 * (t["fold"] + t["reorth"] + t["reconstruct"]) + t["select"])
+        t = _oracle_sample(100 + i, (i + 1) % REORTH_EVERY == 0)
+        steps_s.append(sum(t.values()))
     step = sum(steps_s) / len(steps_s)
-    value = LAYERS * 2 / step
+    value = 1.0 / step
+    cores, blas = _host_cores()
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "folds/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(step * 1e3, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "decode step, 32 layers x {K,V} histories at n~16K (fold b=64 + "
-                                   "reorth + reconstruct with RoPE + one 64K-token prompt selection)",
-                       "d": D, "r": R, "b": BLK, "n": N_MID},
-            "cpu_baseline": {"value": round(value, 4), "unit": "folds/s", "cores": _cpu_threads(),
-                             "kind": "oracle",
-                             "sample": "per step: 1 fold + 1 reorth + 1 reconstruction at n=16384 "
-                                       "and 1 selection, extrapolated to 64 histories"},
+            "config": workload_config(args.layers, world),
+            "cpu_baseline": {"value": round(value, 4), "unit": "folds/s", "cores": cores,
+                             "blas_threads": blas, "kind": "oracle",
+                             "sample": ORACLE_SAMPLE, "extrapolated": False},
             "e2e": {"value": round(value, 4), "unit": "folds/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
 
+# ------------------------------------------------------------------------------------------------
+# Launch: N ranks (torch.distributed.run) and a CPU dry run of the multi-rank plumbing.
+
+def launch_ranks(argv, n):
+    """Re-run this script as `n` ranks through torch.distributed.run on this node."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def run_dry(args):
+    """The multi-rank plumbing without a GPU: gloo process group, a barrier-bracketed timed
+    region of host work per rank, the max over ranks, and rank 0's JSON line."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    for _ in range(args.warmup):
+        torch.ones(64, 64) @ torch.ones(64, 64)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        torch.ones(64, 64) @ torch.ones(64, 64)
+    ms = (time.perf_counter() - t0) * 1e3
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "dry_run": True, "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": round(ms / max(args.steps, 1), 6),
+                          "ranks_timed": world}))
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="exercise the multi-rank launch and timing plumbing on CPU (no GPU)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--no-check", action="store_true")
+    ap.add_argument("--no-check", action="store_true",
+                    help="skip the factor-drift measurement")
     ap.add_argument("--no-attention", action="store_true",
                     help="skip the rows timed apart from the step: decode attention over the "
                          "compressed cache, the diagnostics and the cache-policy step")
@@ -764,13 +921,22 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="model layers (2 histories each); the headline workload is 32")
     args = ap.parse_args(argv)
-    if args.warmup < 3 and args.impl == "b200":
+    if args.warmup < 3 and args.impl == "b200" and not args.dry_run:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
-    if args.impl == "reference":
+    world = int(os.environ.get("WORLD_SIZE", "0"))
+    if args.gpus > 1 and world == 0:
+        return launch_ranks(argv, args.gpus)
+    if world and world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but {world} ranks were launched; reporting {world}",
+              file=sys.stderr)
+    if args.dry_run:
+        run_dry(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_b200(args)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

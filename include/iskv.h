@@ -236,6 +236,9 @@ iskv_status iskv_decode_attention_batched(
  * counts_out      [2 + n_heads] int64: {n_pk, n_pv, n_picked[h]...}.
  * Limits: 1 <= L <= 2^24, n_heads <= 64, head_dim <= 256 and even, block in [1, 64],
  * per_head <= 4096.
+ * Scores: once the call has run, the first n_heads * n_cand float64 values of ws hold the block
+ * scores, head-major ([h][j], n_cand = max(L / block - suffix_blocks, 0) candidate blocks), for
+ * callers that want to inspect them; the rest of ws is scratch.
  */
 size_t iskv_select_workspace_size(int64_t L, int32_t n_heads, int32_t block);
 iskv_status iskv_select_prompt_blocks(const void *keys, int32_t k_dtype, int64_t L,
@@ -256,8 +259,11 @@ iskv_status iskv_select_prompt_blocks(const void *keys, int32_t k_dtype, int64_t
  *    (iskv_select_workspace_size) exceeds it is refused with ISKV_ERR_WORKSPACE; at 8 heads and
  *    8-token blocks that allows prompts up to about 230K tokens.
  *  - Calls no cudaMalloc, cudaFree or allocating library routine.
- *  - The first call on a device looks up the array's device address with that device current;
+ *  - Every call looks up the array's device address (a host-side query) with the caller's
+ *    device current, so the address stays right after the context is torn down and re-created
+ *    (cudaDeviceReset). The first call on a device may load the library's device code there:
  *    make that first call before any stream capture on the device.
+ *  - A refusal leaves its reason in iskv_last_error(), as for the other entry points.
  *  - All calls on a device share the array and it keeps the last call's contents (the parts that
  *    must start at zero are cleared by each call): calls that overlap on the GPU race and corrupt
  *    each other's results, so order them on one stream.
@@ -419,6 +425,19 @@ const char *iskv_stage_name(int32_t i);
 iskv_status iskv_stage_read(double *ms, int64_t *calls);
 void iskv_stage_reset(void);
 int64_t iskv_launch_count(void);
+
+/*
+ * Work counters of the one-sided Jacobi core SVD (no counterpart on the pages; measurement
+ * support for the fold's Algorithm 2 step 6 and the Section 4.4 re-orthogonalisation), always
+ * counted on the device and accumulated over every call since the last reset. out: host int64[12],
+ * six values for the fold's cores, then six for the re-orthogonalisation's: {cores solved, sweeps
+ * summed over cores, largest sweep count of one core, column-pair inner products, rotations
+ * applied, float32 flops}. Flops charge 2 m per inner product over the m rows of a column and
+ * 8 (m + v) per rotation of two columns holding m rows of A and v explicit rows of V (per-round
+ * column norms are not counted). Synchronous: waits for the device. reset != 0 zeroes the
+ * counters after reading them.
+ */
+iskv_status iskv_core_stats(int64_t *out, int32_t reset);
 
 /*
  * Failure-path self-test (no counterpart on the pages; it lets failure detection be tested without

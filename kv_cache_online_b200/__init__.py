@@ -475,6 +475,16 @@ def stage_times(reset: bool = False):
     return out
 
 
+def core_stats(reset: bool = False):
+    """Work counters of the core SVD (see ``iskv_core_stats``): a dict per mode ("fold",
+    "reorth") with cores, sweeps, max_sweeps, pair_checks, rotations and flops."""
+    buf = (ctypes.c_int64 * 12)()
+    _lib.check(_lib.load().iskv_core_stats(buf, 1 if reset else 0), "core_stats")
+    keys = ("cores", "sweeps", "max_sweeps", "pair_checks", "rotations", "flops")
+    return {mode: {k: int(buf[6 * i + j]) for j, k in enumerate(keys)}
+            for i, mode in enumerate(("fold", "reorth"))}
+
+
 def launch_count() -> int:
     """Number of kernels the library has launched in this process."""
     return int(_lib.load().iskv_launch_count())

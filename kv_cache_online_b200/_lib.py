@@ -96,6 +96,7 @@ SIGNATURES = {
     "iskv_stage_read": (c_i32, [ctypes.POINTER(c_f64), ctypes.POINTER(c_i64)]),
     "iskv_stage_reset": (None, []),
     "iskv_launch_count": (c_i64, []),
+    "iskv_core_stats": (c_i32, [c_vp, c_i32]),
     "iskv_selftest_wait_timeout": (c_i32, [c_vp, c_i64, c_vp]),
 }
 

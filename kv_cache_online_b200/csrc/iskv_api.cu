@@ -15,12 +15,15 @@
 #include "reorth.h"
 #include "select.h"
 #include "tc.h"
+#include "api_error.h"
 
 using namespace iskv;
 
-namespace {
+namespace iskv {
 
 thread_local std::string g_last_error;
+
+void clear_last_error() { g_last_error.clear(); }
 
 iskv_status fail(iskv_status st, const char *fmt, ...) {
   char buf[512];
@@ -35,6 +38,10 @@ iskv_status fail(iskv_status st, const char *fmt, ...) {
 iskv_status cuda_fail(cudaError_t e, const char *where) {
   return fail(ISKV_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
+
+}  // namespace iskv
+
+namespace {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -240,6 +247,16 @@ const char *iskv_status_string(int32_t st) {
 }
 
 const char *iskv_last_error(void) { return g_last_error.c_str(); }
+
+iskv_status iskv_core_stats(int64_t *out, int32_t reset) {
+  g_last_error.clear();
+  if (!out) return fail(ISKV_ERR_ARG, "iskv_core_stats: null output");
+  long long v[2 * CORE_STATS];
+  cudaError_t e = core_stats(v, reset != 0);
+  if (e != cudaSuccess) return cuda_fail(e, "iskv_core_stats");
+  for (int i = 0; i < 2 * CORE_STATS; ++i) out[i] = v[i];
+  return ISKV_OK;
+}
 
 // ------------------------------------------------------------------------------------------------
 // Fold

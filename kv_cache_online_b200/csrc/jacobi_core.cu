@@ -26,6 +26,13 @@ namespace cg = cooperative_groups;
 
 namespace iskv {
 
+// Work counters of the core SVD, per mode (0: fold, 1: re-orthogonalisation), accumulated over
+// every launch until reset: {cores solved, sweeps summed over cores, largest sweep count, pair
+// checks (inner products of a column pair), rotations applied, float32 flops}. The flop count
+// charges 2 m per pair check (one inner product over the m rows of A) and 8 (m + pp) per rotation
+// (two FMAs per element of each of the two columns, V rows included); the per-round norm
+// recomputations are not counted.
+static __device__ unsigned long long g_core_stats[2][CORE_STATS];
 
 struct CoreSmem {
   size_t buf, pairs, where, nP, nQ, nrm_local, nrm_all, flags, total;
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   int sweeps_used = -1;
   int cur = 0;  // which buffer holds the current blocks (double-buffered exchange)
   for (int sweep = 0; sweep < p.max_sweeps; ++sweep) {
-    bool rot = false;
+    unsigned rot = 0;  // rotations this half-warp applied in this sweep
     for (int t = 0; t < M - 1; ++t) {
       float *buf = buf0 + (dbuf ? cur * bufw : 0);
       float *Pb = buf, *Qb = buf + w * LP;
@@ -297,7 +304,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
             col_store<NE>(base + a * LP, x);
             col_store<NE>(base + bb * LP, y);
             if (l16 == 0) { nb[a] = ax; nb[bb] = by; }
-            rot = true;
+            ++rot;
           }
           __syncthreads();
         }
@@ -316,7 +323,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
         if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
           col_store<NE>(Qb + qc * LP, y);
           if (l16 == 0) nQ[qc] = by;
-          rot = true;
+          ++rot;
         }
         __syncthreads();
       }
@@ -343,6 +350,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
       if (dbuf) cur ^= 1;
     }
     // Cluster-wide "any rotation in this sweep".
+    if (l16 == 0 && rot) atomicAdd(reinterpret_cast<unsigned *>(flags + 2), rot);
     const int any_local = __syncthreads_or(rot ? 1 : 0);
     if (tid == 0) flags[sweep & 1] = any_local;
     cluster.sync();
@@ -434,6 +442,27 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
     sc[FS_SWEEPS] = sweeps_used;
     if (sweeps_used < 0) record_status(jh.meta, ISKV_ERR_NOT_CONVERGED);
   }
+  {
+    // Work counters. Every sweep checks each pair of the M w (padded) columns once; the CTA's
+    // rotations were summed in shared memory at the end of each sweep.
+    unsigned long long *st = g_core_stats[dense ? 1 : 0];
+    const unsigned long long rsum = *reinterpret_cast<const unsigned *>(flags + 2);
+    if (tid == 0 && rsum) {
+      atomicAdd(&st[4], rsum);
+      atomicAdd(&st[5], rsum * (8ull * (unsigned)(m + pp)));
+    }
+    if (rank == 0 && tid == 0) {
+      const unsigned long long sw = sweeps_used < 0 ? (unsigned long long)p.max_sweeps
+                                                    : (unsigned long long)sweeps_used;
+      const unsigned long long np = (unsigned long long)(M * w);
+      const unsigned long long chk = sw * (np * (np - 1) / 2);
+      atomicAdd(&st[0], 1ull);
+      atomicAdd(&st[1], sw);
+      atomicMax(&st[2], sw);
+      atomicAdd(&st[3], chk);
+      atomicAdd(&st[5], chk * (2ull * (unsigned)m));
+    }
+  }
   cluster.sync();  // my shared memory stays valid until every CTA has read nrm_local
 }
 
@@ -476,6 +505,19 @@ cudaError_t launch_core(const char *jobs, const CoreParams &p, cudaStream_t s) {
     case 20: return core_launch<20>(jobs, p, c, s);
     default: return core_launch<24>(jobs, p, c, s);
   }
+}
+
+cudaError_t core_stats(long long *out, bool reset) {
+  unsigned long long h[2][CORE_STATS];
+  cudaError_t e = cudaMemcpyFromSymbol(h, g_core_stats, sizeof h);
+  if (e != cudaSuccess) return e;
+  for (int m = 0; m < 2; ++m)
+    for (int i = 0; i < CORE_STATS; ++i) out[m * CORE_STATS + i] = (long long)h[m][i];
+  if (reset) {
+    unsigned long long z[2][CORE_STATS] = {};
+    e = cudaMemcpyToSymbol(g_core_stats, z, sizeof z);
+  }
+  return e;
 }
 
 CoreParams fold_core_params(const FoldParams &p) {

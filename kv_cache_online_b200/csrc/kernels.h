@@ -55,6 +55,9 @@ cudaError_t launch_fold_residual(const FoldJob *jobs, const FoldParams &p, cudaS
 cudaError_t launch_fold_finalize(const FoldJob *jobs, const FoldParams &p, cudaStream_t s);
 
 cudaError_t launch_core(const char *jobs, const CoreParams &p, cudaStream_t s);
+// Core SVD work counters: CORE_STATS values per mode (see jacobi_core.cu), synchronous read.
+constexpr int CORE_STATS = 6;
+cudaError_t core_stats(long long *out, bool reset);
 cudaError_t launch_rotate_basis(const char *jobs, const RotParams &p, cudaStream_t s);
 cudaError_t launch_rotate_coords_ffma(const char *jobs, const RotParams &p, int64_t n_cap_max,
                                       cudaStream_t s);

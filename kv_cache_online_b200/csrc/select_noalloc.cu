@@ -12,10 +12,12 @@
 //
 // In host code the array's name is only a host-side stand-in: a kernel given it would fault or,
 // where the GPU can reach host memory, silently use the wrong memory. Its device address is
-// therefore looked up with cudaGetSymbolAddress, once per device, with that device current, the
-// first time this entry point runs on that device.
-#include <mutex>
-
+// therefore looked up with cudaGetSymbolAddress, with the caller's device current, on every call:
+// the lookup is a host-side query, and an address is never carried over from an earlier call, so
+// a context that the host framework tore down and re-created (cudaDeviceReset) gets the array's
+// new address. The first call on a device may load the library's device code there; make it
+// before any stream capture on that device.
+#include "api_error.h"
 #include "iskv.h"
 #include "profiling.h"
 #include "select.h"
@@ -24,30 +26,6 @@ namespace iskv {
 
 static __device__ __align__(256) unsigned char g_select_scratch[ISKV_NOALLOC_SCRATCH];
 
-namespace {
-
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch array on the current device (looked up on first use).
-cudaError_t scratch_address(void **out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_select_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
-  return cudaSuccess;
-}
-
-}  // namespace
 }  // namespace iskv
 
 using namespace iskv;
@@ -56,17 +34,27 @@ extern "C" iskv_status iskv_select_prompt_blocks_noalloc(
     const void *keys, int32_t k_dtype, int64_t L, int32_t n_heads, int32_t head_dim, int32_t block,
     int32_t per_head, int32_t suffix_blocks, int32_t v_radius, int32_t *pk_out, int32_t *pv_out,
     int32_t *head_blocks_out, int64_t *counts_out, void *stream) {
-  if (!keys || !pk_out || !pv_out || !head_blocks_out || !counts_out) return ISKV_ERR_ARG;
-  if (k_dtype != ISKV_F32 && k_dtype != ISKV_BF16) return ISKV_ERR_ARG;
-  if (L < 1 || L > ((int64_t)1 << 24) || n_heads < 1 || n_heads > 64 || head_dim < 2 ||
-      head_dim > 256 || head_dim % 2 || block < 1 || block > 64 || per_head < 0 ||
-      per_head > 4096 || suffix_blocks < 0 || v_radius < 0)
-    return ISKV_ERR_SHAPE;
+  const char *who = "iskv_select_prompt_blocks_noalloc";
+  clear_last_error();
+  if (!keys || !pk_out || !pv_out || !head_blocks_out || !counts_out)
+    return fail(ISKV_ERR_ARG, "%s: null pointer", who);
+  if (k_dtype != ISKV_F32 && k_dtype != ISKV_BF16)
+    return fail(ISKV_ERR_ARG, "%s: keys must be float32 or bf16", who);
+  if (L < 1 || L > ((int64_t)1 << 24)) return fail(ISKV_ERR_SHAPE, "%s: need 1 <= L <= 2^24", who);
+  if (n_heads < 1 || n_heads > 64 || head_dim < 2 || head_dim > 256 || head_dim % 2)
+    return fail(ISKV_ERR_SHAPE, "%s: need n_heads <= 64, even head_dim <= 256", who);
+  if (block < 1 || block > 64 || per_head < 0 || per_head > 4096 || suffix_blocks < 0 ||
+      v_radius < 0)
+    return fail(ISKV_ERR_SHAPE, "%s: bad block / per_head / suffix / radius", who);
   // The scratch has a fixed size: larger problems are refused, never truncated.
-  if (select_ws_layout(L, n_heads, block).total > (size_t)ISKV_NOALLOC_SCRATCH)
-    return ISKV_ERR_WORKSPACE;
+  const size_t need = select_ws_layout(L, n_heads, block).total;
+  if (need > (size_t)ISKV_NOALLOC_SCRATCH)
+    return fail(ISKV_ERR_WORKSPACE,
+                "%s: this prompt needs %zu bytes of scratch, more than the %u-byte fixed array", who,
+                need, (unsigned)ISKV_NOALLOC_SCRATCH);
   void *scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return ISKV_ERR_CUDA;
+  cudaError_t e = cudaGetSymbolAddress(&scratch, g_select_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "iskv_select_prompt_blocks_noalloc: scratch address");
   SelectArgs a;
   a.keys = keys;
   a.k_dtype = k_dtype;
@@ -84,7 +72,8 @@ extern "C" iskv_status iskv_select_prompt_blocks_noalloc(
   a.ws = scratch;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   stage_begin(s);
-  if (launch_select(a, s) != cudaSuccess) return ISKV_ERR_CUDA;
+  e = launch_select(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "iskv_select_prompt_blocks_noalloc: launch");
   stage_mark(s, ST_SELECT);
   return ISKV_OK;
 }

@@ -105,3 +105,50 @@ def torch_lowrank_rows(n: int, d: int, exponent: float, noise: float, basis, see
     if noise:
         X = X + float(noise) * torch.randn(n, d, generator=gen, device=device, dtype=torch.float32)
     return X
+
+
+class DriftingRows:
+    """Rows of ``count`` independent streams whose dominant subspace drifts, drawn on ``device``
+    with a seeded torch generator, one block of ``block`` rows per stream at a time.
+
+    Stream i emits ``G diag(s_i) H_i(t)^T + noise * N(0, 1)`` with ``G`` standard normal,
+    ``s_i[j] = (j + 1) ** -exponents[i]`` and ``H_i(t) = H_i(0) exp((t / 1024) angle_per_1k S_i)``,
+    where ``H_i(0)`` is a random d x d orthogonal matrix and ``S_i`` a random skew-symmetric matrix
+    scaled to spectral norm 1 (estimated by power iteration): the subspace turns by about
+    ``angle_per_1k`` radians per 1024 rows. ``H`` advances by one block after each call of
+    :meth:`next_blocks`. Float32 throughout; returns (count, block, d) tensors."""
+
+    def __init__(self, count: int, d: int, exponents, noise: float, seed: int, block: int,
+                 angle_per_1k: float = 0.05, device="cuda"):
+        import torch
+
+        self.torch = torch
+        self.count, self.d, self.block, self.noise = int(count), int(d), int(block), float(noise)
+        self.gen = torch.Generator(device=device)
+        self.gen.manual_seed(int(seed))
+        self.device = device
+        A = torch.randn(self.count, d, d, generator=self.gen, device=device)
+        Q, R = torch.linalg.qr(A)
+        self.H = Q * torch.sign(torch.diagonal(R, dim1=-2, dim2=-1))[:, None, :]
+        A = torch.randn(self.count, d, d, generator=self.gen, device=device)
+        S = A - A.transpose(1, 2)
+        v = torch.randn(self.count, d, 1, generator=self.gen, device=device)
+        for _ in range(30):                       # power iteration on S^T S
+            v = S.transpose(1, 2) @ (S @ v)
+            v = v / torch.linalg.vector_norm(v, dim=1, keepdim=True)
+        snorm = torch.linalg.vector_norm(S @ v, dim=1, keepdim=True)
+        S = S / snorm
+        self.E = torch.linalg.matrix_exp(S * (float(angle_per_1k) * self.block / 1024.0))
+        ex = torch.as_tensor([float(e) for e in exponents], device=device)[:, None]
+        j = torch.arange(1, d + 1, device=device, dtype=torch.float32)[None, :]
+        self.s = j ** (-ex)                       # (count, d)
+
+    def next_blocks(self):
+        torch = self.torch
+        G = torch.randn(self.count, self.block, self.d, generator=self.gen, device=self.device)
+        X = (G * self.s[:, None, :]) @ self.H.transpose(1, 2)
+        if self.noise:
+            X = X + self.noise * torch.randn(self.count, self.block, self.d, generator=self.gen,
+                                             device=self.device)
+        self.H = self.H @ self.E
+        return X

@@ -115,6 +115,16 @@ def test_host_side_argument_errors():
                                          None) == 2
     assert lib.iskv_select_prompt_blocks(k, 1, 100, 8, 128, 8, 128, 4, 32, None, o, o, o, ws, big,
                                          None) == 1
+    # allocation-free selection: each refusal leaves its own reason, a later one replaces it
+    assert lib.iskv_select_prompt_blocks_noalloc(k, 1, 1 << 20, 8, 128, 8, 128, 4, 32, o, o, o, o,
+                                                 None) == 8
+    assert b"scratch" in lib.iskv_last_error()
+    assert lib.iskv_select_prompt_blocks_noalloc(k, 1, 100, 8, 127, 8, 128, 4, 32, o, o, o, o,
+                                                 None) == 2
+    assert b"head_dim" in lib.iskv_last_error()
+    assert lib.iskv_select_prompt_blocks_noalloc(k, 1, 100, 8, 128, 8, 128, 4, 32, None, o, o, o,
+                                                 None) == 1
+    assert b"null" in lib.iskv_last_error()
     # reorth: batched histories must agree
     arr = (L.IskvLowRank * 2)(_fake_handle(L), _fake_handle(L, r=128))
     assert lib.iskv_reorth(arr, 2, ws, big, None) == 2

@@ -78,3 +78,23 @@ def test_edge_cases():
     assert list(out["head_blocks"][0][:10]) == list(range(10))
     ref, out = _run(m, k403, torch.float32, per_head=0, radius=0)
     _check(ref, out, 2, 0)
+
+
+@pytest.mark.parametrize("L,dtype,seed", [(4096 + 5, torch.bfloat16, 7), (2000, torch.float32, 8)])
+def test_block_scores_match_oracle(L, dtype, seed):
+    """The float64 block scores themselves (left at the start of the workspace), not only the
+    blocks they select, against the oracle's scores to 1e-12 relative."""
+    m = kv()
+    H, hd = 8, 128
+    keys, _ = synth.outlier_prompt_keys(L, H, hd, seed)
+    keys[:8, 3, :] = 0.0                                   # a zero block scores 0
+    kt = torch.as_tensor(keys, dtype=dtype, device="cuda").contiguous()
+    seen = kt.to(torch.float64).cpu().numpy()
+    ref = osel.select_prompt_blocks(seen, 8, 128, 4, 32)
+    ws = torch.zeros(m.select_workspace_size(L, H, 8), dtype=torch.uint8, device="cuda")
+    m.select_prompt_blocks(kt, 8, 128, 4, 32, ws=ws)
+    torch.cuda.synchronize()
+    n_cand = ref["n_cand"]
+    got = ws[:8 * H * n_cand].view(torch.float64).view(H, n_cand).cpu().numpy()
+    assert ref["scores"][3, 0] == 0.0 and got[3, 0] == 0.0
+    np.testing.assert_allclose(got, ref["scores"], rtol=1e-12, atol=1e-15)

@@ -52,3 +52,24 @@ def test_single_process_is_identity():
 
     import bench
     assert bench.max_over_ranks(3.25, torch.device("cpu")) == 3.25
+
+
+@pytest.mark.timeout(300)
+def test_bench_gpus_two_launches_two_ranks():
+    """`bench.py --gpus 2` (no torchrun around it) launches two ranks itself; the CPU dry run
+    exercises the same launch, barriers and max-over-ranks timing, and rank 0 alone prints one
+    line that reports the two ranks it ran."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                          "--dry-run", "--steps", "2", "--warmup", "3"], cwd=root, env=env,
+                         capture_output=True, text=True, timeout=280)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["ranks_timed"] == 2 and line["dry_run"] is True

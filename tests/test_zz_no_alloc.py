@@ -64,6 +64,23 @@ def test_noalloc_selection_matches_workspace_form_on_two_calls():
         _same(out, ref, 8)
 
 
+def test_noalloc_small_call_then_larger_calls():
+    """A small prompt first, then a 16 times longer one with the same per-head budget, then a
+    prompt whose tail is not a whole block: each later call runs on scratch that the earlier,
+    smaller calls left partly written, and each must still equal the workspace form bit for bit."""
+    m = kv()
+    cases = [synth.outlier_prompt_keys(4101, 8, 128, seed=23)[0],
+             synth.outlier_prompt_keys(65536, 8, 128, seed=24)[0],
+             synth.outlier_prompt_keys(30000 + 3, 8, 128, seed=25)[0]]
+    for k in cases:
+        kt = torch.as_tensor(k, dtype=torch.float32).cuda().to(torch.bfloat16)
+        st, out = _noalloc(m, kt)
+        assert st == 0
+        ref = m.select_prompt_blocks(kt, 8, 128, 4, 32)
+        torch.cuda.synchronize()
+        _same(out, ref, 8)
+
+
 def test_noalloc_refuses_sizes_beyond_its_scratch():
     m = kv()
     lib = m._lib.load()
@@ -73,3 +90,8 @@ def test_noalloc_refuses_sizes_beyond_its_scratch():
     st = lib.iskv_select_prompt_blocks_noalloc(dummy, 1, 1 << 20, 8, 128, 8, 128, 4, 32, dummy,
                                                dummy, dummy, dummy, None)
     assert st == 8   # ISKV_ERR_WORKSPACE, nothing launched
+    assert b"scratch" in lib.iskv_last_error()
+    st = lib.iskv_select_prompt_blocks_noalloc(dummy, 7, 4096, 8, 128, 8, 128, 4, 32, dummy,
+                                               dummy, dummy, dummy, None)
+    assert st == 1   # ISKV_ERR_ARG: bad key dtype
+    assert b"float32 or bf16" in lib.iskv_last_error()
