@@ -35,7 +35,7 @@ namespace iskv {
 static __device__ unsigned long long g_core_stats[2][CORE_STATS];
 
 struct CoreSmem {
-  size_t buf, pairs, where, nP, nQ, nrm_local, nrm_all, flags, total;
+  size_t buf, pairs, where, nP, nQ, nrm_local, anrm, vnrm, nrm_all, flags, total;
 };
 
 // Shared-memory plan (4-byte words). Column blocks are double-buffered when `dbuf` so a round's
@@ -51,6 +51,8 @@ __host__ __device__ inline CoreSmem core_smem(int cj, int w, int ne, bool dbuf) 
   s.nP = take((size_t)w);
   s.nQ = take((size_t)w);
   s.nrm_local = take((size_t)2 * w);
+  s.anrm = take((size_t)2 * w);
+  s.vnrm = take((size_t)2 * w);
   s.nrm_all = take((size_t)M * w);
   s.flags = take(4);
   s.total = o * 4;
@@ -216,6 +218,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   int *where = reinterpret_cast<int *>(smem + S.where);   // [M-1][M] = cta * 2 + slot
   float *nP = smem + S.nP, *nQ = smem + S.nQ;
   float *nrm_local = smem + S.nrm_local;
+  float *anrm = smem + S.anrm, *vnrm = smem + S.vnrm;
   float *nrm_all = smem + S.nrm_all;
   int *flags = reinterpret_cast<int *>(smem + S.flags);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -363,19 +366,40 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   }
   float *buf = buf0 + (dbuf ? cur * bufw : 0);
 
-  // Column norms of my columns (blocks are at their round-0 places again).
+  // Singular values of my columns (blocks are at their round-0 places again). A column of A is
+  // Z times the matching column of V, and both come out of the float32 rotations a little too
+  // long: a rotation by a small angle theta should shorten a column's dominant entry (near +-1 in
+  // V, near sigma in A) by theta^2 / 2 of itself, which float32 cannot represent below half an
+  // ulp, while the first-order growth of the small entries is kept. Over a fold's few hundred
+  // rotations per column this lengthens both by ~1e-6 relative, the same for A and V. So
+  // sigma' = |A_q| / |V_q|, G_q = A_q / |A_q| and H_q = V_q / |V_q|: then Z H_q = G_q sigma'_q, and
+  // the kept product is Z times a projector instead of growing by |V_q|^2 at every fold.
+  const int nv = dense ? k : pp;  // explicit V rows after the A part
   for (int e = warp; e < 2 * w; e += nw) {
     const float *x = buf + e * LP;
-    double s = 0.0;
+    double sa = 0.0, sv = 0.0;
 #pragma unroll
     for (int t = 0; t < NE; ++t) {
-      if (lane + 32 * t < m) {
-        const double v = x[lane + 32 * t];
-        s = fma(v, v, s);
+      const int idx = lane + 32 * t;
+      const double v = x[idx];
+      if (idx < m) {
+        sa = fma(v, v, sa);
+        if (!dense && idx < k && sig_old[idx] > 0.f) {
+          const double hv = v / (double)sig_old[idx];
+          sv = fma(hv, hv, sv);
+        }
+      } else if (idx >= mp && idx < mp + nv) {
+        sv = fma(v, v, sv);
       }
     }
-    s = warp_sum(s);
-    if (lane == 0) nrm_local[e] = (float)sqrt(s);
+    sa = warp_sum(sa);
+    sv = warp_sum(sv);
+    if (lane == 0) {
+      const double vn = sv > 0.0 ? sqrt(sv) : 1.0;
+      anrm[e] = (float)sqrt(sa);
+      vnrm[e] = (float)vn;
+      nrm_local[e] = (float)(sqrt(sa) / vn);
+    }
   }
   cluster.sync();
   for (int e = tid; e < M * w; e += blockDim.x) {
@@ -411,7 +435,8 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
     if (j >= ncol || q >= kn) continue;
     if (!isfinite(nj) && lane == 0) record_status(jh.meta, ISKV_ERR_NONFINITE);
     const float *x = buf + e * LP;
-    const float inv = nj > 0.f ? 1.f / nj : 0.f;
+    const float inv = anrm[e] > 0.f ? 1.f / anrm[e] : 0.f;
+    const float vinv = 1.f / vnrm[e];
     if (lane == 0) sig[q] = nj;
     for (int l = lane; l < r; l += 32) {
       const float g = l < k ? x[l] * inv : 0.f;
@@ -424,7 +449,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
       if (dense) h = l < k ? x[mp + l] : 0.f;
       else if (l < k) h = sig_old[l] > 0.f ? x[l] / sig_old[l] : 0.f;
       else if (l < ncol) h = x[mp + (l - k)];
-      Ht[(size_t)q * hs + l] = h;
+      Ht[(size_t)q * hs + l] = h * vinv;
     }
   }
   // Zero the rows / columns beyond k'.
@@ -538,7 +563,11 @@ CoreParams fold_core_params(const FoldParams &p) {
   c.hs = p.ws.hs;
   c.ldm = 0;
   c.max_sweeps = 40;
-  c.dd = 0;
+  // Float32 factors (the parity-grade storage) take float64 inner products and the tighter
+  // tolerance: the kept subspace is then decided to float32 accuracy at the truncation boundary,
+  // where a nearly flat spectrum magnifies any residual cosine over a long trajectory. Two-byte
+  // factors round far above that, and keep the float32 sweep.
+  c.dd = p.storage == ISKV_F32 ? 1 : 0;
   return c;
 }
 
