@@ -198,11 +198,14 @@ iskv_status iskv_diagnostics(const iskv_lowrank *hs, int32_t count, const int64_
  * Positions must lie in [0, n_total); the K and V caches must cover the same positions: a key
  * position without a value leaves probability mass unaccounted (checked to 1e-3) and, like an
  * out-of-range position or a cache with no key at all, records ISKV_ERR_SHAPE in the status word
- * (hk for key-side conditions, hv for value-side ones). hk and hv share d, r_max, storage and
- * n_cap; d == n_kv_heads * head_dim, head_dim even <= 256, n_q_heads a multiple of n_kv_heads,
+ * (hk for key-side conditions, hv for value-side ones). hk and hv share d, storage and n_cap;
+ * their rank budgets may differ (the keys and values of a layer compressed at different ranks,
+ * the separate K / V ranks of Section 8), but all hk of a batched call share one r_max and all hv
+ * another. d == n_kv_heads * head_dim, head_dim even <= 256, n_q_heads a multiple of n_kv_heads,
  * <= 64 and at most 8 per KV head.
- * ws           iskv_attention_workspace_size(count, d, r_max, n_cap, max n_total, n_q_heads) bytes,
- *              256-byte aligned (scores by position, softmax statistics, partial value sums).
+ * ws           iskv_attention_workspace_size(count, d, r_max, n_cap, max n_total, n_q_heads) bytes
+ *              with r_max the larger of the K and V rank budgets, 256-byte aligned (scores by
+ *              position, softmax statistics, partial value sums).
  * hk, hv and the per-job arrays of the batched form are HOST arrays of `count` entries.
  */
 size_t iskv_attention_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap,

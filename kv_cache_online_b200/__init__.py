@@ -283,7 +283,8 @@ def decode_attention_batched(k_hists, v_hists, k_exact, k_exact_pos, v_exact, v_
     edt = kdt if any(kn) else vdt
     if any(kn) and any(vn) and kdt != vdt:
         raise ValueError("exact keys and values must share a dtype")
-    need = lib.iskv_attention_workspace_size(n, d, k_hists[0].r_max, k_hists[0].n_cap,
+    need = lib.iskv_attention_workspace_size(n, d, max(k_hists[0].r_max, v_hists[0].r_max),
+                                             k_hists[0].n_cap,
                                              max(n_total), nq)
     w = ws if ws is not None else _ws(k_hists[0].device, need)
     P = ctypes.c_void_p * n

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(256) k_attn_scores_ffma(const AttnJob *jobs, A
   const AttnJob &jb = jobs[blockIdx.y];
   const int64_t n = jb.metak[ISKV_META_N];
   const int k = (int)jb.metak[ISKV_META_K];
-  const int d = p.d, r = p.r, hd = p.head_dim, half = hd / 2;
+  const int d = p.d, r = p.rk, hd = p.head_dim, half = hd / 2;
   extern __shared__ float sm[];
   float *us = sm;                 // [r] sigma-scaled coordinates
   float *krow = sm + r;           // [d] rebuilt key
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(256) k_attn_scores_ffma(const AttnJob *jobs, A
 
 cudaError_t launch_attn_scores_ffma(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
   const int gx = (int)((p.n_cap_max + 7) / 8);
-  const size_t smem = sizeof(float) * (size_t)(p.r + p.d);
+  const size_t smem = sizeof(float) * (size_t)(p.rk + p.d);
   if (gx < 1) return cudaSuccess;
   with_dtype(p.storage, [&](auto ts) {
     k_attn_scores_ffma<decltype(ts)><<<dim3(gx, p.count), 256, smem, s>>>(jobs, p);
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(AV_THREADS) k_attn_values(const AttnJob *jobs,
   const AttnJob &jb = jobs[blockIdx.z];
   const int mt = (p.n_q + AV_BM - 1) / AV_BM;
   const int c = blockIdx.y / mt, m0 = (blockIdx.y % mt) * AV_BM, n0 = blockIdx.x * AV_BN;
-  const int nq = p.n_q, r = p.r;
+  const int nq = p.n_q, r = p.rv;
   const int64_t n = jb.metav[ISKV_META_N];
   const int k = (int)jb.metav[ISKV_META_K];
   const int64_t i0 = (int64_t)c * ATTN_CHUNK;
@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(AV_THREADS) k_attn_values(const AttnJob *jobs,
 
 cudaError_t launch_attn_values(const AttnJob *jobs, const AttnParams &p, cudaStream_t s) {
   const int mt = (p.n_q + AV_BM - 1) / AV_BM;
-  const dim3 g((p.r + AV_BN - 1) / AV_BN, mt * p.nchunk, p.count);
+  const dim3 g((p.rv + AV_BN - 1) / AV_BN, mt * p.nchunk, p.count);
   with_dtype(p.storage, [&](auto ts) {
     k_attn_values<decltype(ts)><<<g, AV_THREADS, 0, s>>>(jobs, p);
   });
@@ -340,7 +340,7 @@ constexpr int AO_ROWS = 512;  // exact rows per staged batch
 template <typename TS, typename TE>
 __global__ void __launch_bounds__(256) k_attn_out(const AttnJob *jobs, AttnParams p) {
   const AttnJob &jb = jobs[blockIdx.y];
-  const int h = blockIdx.x, part_id = blockIdx.z, nq = p.n_q, r = p.r, hd = p.head_dim;
+  const int h = blockIdx.x, part_id = blockIdx.z, nq = p.n_q, r = p.rv, hd = p.head_dim;
   const int qpk = nq / p.n_kv, q0 = h * qpk;
   const int k = (int)jb.metav[ISKV_META_K];
   extern __shared__ float sm[];
@@ -450,7 +450,7 @@ cudaError_t launch_attn_out(const AttnJob *jobs, const AttnParams &p, cudaStream
   const int qpk = p.n_q / p.n_kv;
   if (qpk > 8) return cudaErrorInvalidValue;
   const int ns = 256 / p.head_dim > 0 ? 256 / p.head_dim : 1;  // thread groups
-  const size_t smem = sizeof(float) * ((size_t)qpk * p.r + (size_t)qpk * AO_ROWS +
+  const size_t smem = sizeof(float) * ((size_t)qpk * p.rv + (size_t)qpk * AO_ROWS +
                                        (size_t)ns * qpk * p.head_dim);
   const dim3 g(p.n_kv, p.count, AO_SPLIT);
   const int nth = ns * p.head_dim;

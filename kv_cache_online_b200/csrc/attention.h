@@ -8,12 +8,12 @@ namespace iskv {
 // One (sequence, layer) job: the K and V histories, the exact rows of both caches, the decode
 // query and the output, plus this job's workspace slices.
 struct AttnJob {
-  const void *Uk;            // K history: U [n_cap][r], sigma [r], B [d][r], pos [n_cap], meta
+  const void *Uk;            // K history: U [n_cap][rk], sigma [rk], B [d][rk], pos [n_cap], meta
   const float *sk;
   const void *Bk;
   const int32_t *posk;
   int64_t *metak;
-  const void *Uv;            // V history
+  const void *Uv;            // V history: U [n_cap][rv], sigma [rv], B [d][rv], pos, meta
   const float *sv;
   const void *Bv;
   const int32_t *posv;
@@ -26,7 +26,7 @@ struct AttnJob {
   float *out;                // [n_q][head_dim] float32
   float *S;                  // workspace [n_q][n_total]: scores by position (-inf where no key)
   float *stats;              // workspace [n_q][2]: max score, sum of exp(score - max)
-  float *wpart;              // workspace [nchunk][n_q][r]: partial sums of p * U_v rows
+  float *wpart;              // workspace [nchunk][n_q][rv]: partial sums of p * U_v rows
   float *mpart;              // workspace [nchunk][n_q]: partial probability mass on V rows
   float *P;                  // workspace [n_q][n_cap]: probabilities at the compressed V rows
   void *Pb;                  // the same workspace as bf16 [n_cap][64] (tensor-core value mixing)
@@ -37,9 +37,10 @@ struct AttnJob {
 };
 
 struct AttnParams {
-  int d, r, storage, exact_dtype, n_kv, n_q, head_dim, count, nchunk;
+  int d, storage, exact_dtype, n_kv, n_q, head_dim, count, nchunk;
+  int rk, rv;      // rank budgets (row strides of U and B) of the K and of the V histories
   int nblk;        // probability-mass partials: blocks of 256 * ATTN_PROB_ROWS value rows
-  int tc_values;   // value mixing on the tensor cores (partials [chunk][r][64])
+  int tc_values;   // value mixing on the tensor cores (partials [chunk][rv][64])
   double theta;
   float scale;
   int64_t n_cap_max, n_total_max;

@@ -163,11 +163,44 @@ bool refit_in_one_fold(int d, int r, int rows) {
          fold_residual_smem(d, rows) <= 200 * 1024 && core_cfg(r, rows, false, jc);
 }
 
+// Rank budget of the wide history through which a refit of `rows` rows (b-row blocks) reaches an
+// exact truncated SVD: r + rows - b (rounded up to a multiple of 16) holds every direction of the
+// first rows / b - 1 folds, so only the last fold truncates, and its top r are the rank-r SVD of
+// the history's rows followed by the refit rows (Eckart-Young). 0 when no such fold fits.
+int32_t wide_refit_rank(int d, int r, int b, int rows) {
+  int32_t rw = (r + rows - b + 15) / 16 * 16;
+  if (rw < r) rw = r;
+  JacobiCfg jc;
+  if (rw > 512 || rw > d || !core_cfg(rw, b, false, jc) || fold_residual_smem(d, b) > 200 * 1024)
+    return 0;
+  return rw;
+}
+
+// Workspace of a wide refit: the fold workspace of the wide history, then its U, B, sigma,
+// positions and meta word (U and B sized for float32 elements, the widest storage).
+struct WideWs {
+  size_t fold, U, B, sig, pos, meta, total;
+};
+
+WideWs wide_ws(int d, int rw, int b, int64_t n_cap) {
+  WideWs w;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  w.fold = take(iskv_fold_workspace_size(1, d, rw, b));
+  w.U = take(sizeof(float) * (size_t)(n_cap > 0 ? n_cap : 1) * rw);
+  w.B = take(sizeof(float) * (size_t)d * rw);
+  w.sig = take(sizeof(float) * (size_t)rw);
+  w.pos = take(sizeof(int32_t) * (size_t)(n_cap > 0 ? n_cap : 1));
+  w.meta = take(4 * sizeof(int64_t));
+  w.total = o;
+  return w;
+}
+
 // What the next decode step does to one table, decided from its host mirror alone: the rows it
-// folds (0: none; `block`, or refit_rows for the first refit), the block size of those folds, and
-// whether a re-orthogonalisation follows.
+// folds (0: none; `block`, or refit_rows for the first refit), the block size of those folds,
+// whether they run through a wide history (rank rw), and whether a re-orthogonalisation follows.
 struct TablePlan {
-  int32_t rows = 0, blk = 0;
+  int32_t rows = 0, blk = 0, rw = 0;
   bool refit = false, reorth = false;
 };
 
@@ -182,18 +215,24 @@ iskv_status plan_table(const iskv_exact_table *T, int d, int r, int64_t ncap, in
     return fail(ISKV_ERR_CAPACITY, "%s: table %d: history has no room for a block (%lld + %d > "
                 "%lld)", who, i, (long long)T->hist_rows, rows, (long long)ncap);
   // A refit is one fold of all its rows when the fold takes such a block; otherwise, for an empty
-  // history and refit_rows <= r_max, consecutive b-row folds that never truncate.
-  int32_t blk = b;
+  // history and refit_rows <= r_max, consecutive b-row folds that never truncate; otherwise
+  // b-row folds into a wide history of rank r + refit_rows - b, of which the top r are kept.
+  int32_t blk = b, rw = 0;
   if (refit) {
     if (refit_in_one_fold(d, r, rows)) blk = rows;
-    else if (T->hist_rows != 0 || rows > r)
-      return fail(ISKV_ERR_SHAPE, "%s: table %d: a first refit of %d rows is carried out as one "
-                  "fold (refit_rows <= 128 with r_max + refit_rows inside the core SVD cluster) "
-                  "or, for an empty history, as untruncated block folds (refit_rows <= r_max); "
-                  "history rows %lld", who, i, rows, (long long)T->hist_rows);
+    else if (T->hist_rows != 0 || rows > r) {
+      rw = wide_refit_rank(d, r, b, rows);
+      if (rw == 0)
+        return fail(ISKV_ERR_SHAPE, "%s: table %d: a first refit of %d rows is carried out as one "
+                    "fold (refit_rows <= 128 with r_max + refit_rows inside the core SVD cluster), "
+                    "for an empty history as untruncated block folds (refit_rows <= r_max), or "
+                    "through a wide history of rank r_max + refit_rows - block (at most 512 and "
+                    "d); history rows %lld", who, i, rows, (long long)T->hist_rows);
+    }
   }
   p.rows = rows;
   p.blk = blk;
+  p.rw = rw;
   p.refit = refit;
   p.reorth = !refit && T->reorth_rows > 0 && T->fold_rows + b >= T->reorth_rows;
   return ISKV_OK;
@@ -714,10 +753,11 @@ iskv_status iskv_decode_attention_batched(
     if (st == ISKV_OK) st = check_handle(&hv[i], who);
     if (st != ISKV_OK) return st;
     for (const iskv_lowrank *h : {&hk[i], &hv[i]})
-      if (h->d != hk[0].d || h->r_max != hk[0].r_max || h->storage != hk[0].storage ||
-          h->n_cap != hk[0].n_cap)
-        return fail(ISKV_ERR_SHAPE, "%s: K and V histories must share d, r_max, storage, n_cap",
-                    who);
+      if (h->d != hk[0].d || h->storage != hk[0].storage || h->n_cap != hk[0].n_cap)
+        return fail(ISKV_ERR_SHAPE, "%s: K and V histories must share d, storage, n_cap", who);
+    if (hk[i].r_max != hk[0].r_max || hv[i].r_max != hv[0].r_max)
+      return fail(ISKV_ERR_SHAPE, "%s: batched K histories must share r_max, and so must the V "
+                  "histories", who);
     if (hk[i].d != n_kv_heads * head_dim)
       return fail(ISKV_ERR_SHAPE, "%s: d must equal n_kv_heads * head_dim", who);
     if (!q[i] || !out[i]) return fail(ISKV_ERR_ARG, "%s: null query or output", who);
@@ -729,14 +769,15 @@ iskv_status iskv_decode_attention_batched(
     if (n_k_exact[i] > max_kex) max_kex = n_k_exact[i];
     if (n_total[i] > ntot_max) ntot_max = n_total[i];
   }
-  const int d = hk[0].d, r = hk[0].r_max;
+  const int d = hk[0].d, rk = hk[0].r_max, rv = hv[0].r_max, r = rk > rv ? rk : rv;
   const int64_t ncap = hk[0].n_cap;
   const AttnWsLayout L = attn_ws_layout(count, d, r, ncap, ntot_max, n_q_heads);
   iskv_status st = check_ws(ws, ws_bytes, L.total, who);
   if (st != ISKV_OK) return st;
   AttnParams p;
   p.d = d;
-  p.r = r;
+  p.rk = rk;
+  p.rv = rv;
   p.storage = hk[0].storage;
   p.exact_dtype = exact_dtype;
   p.n_kv = n_kv_heads;
@@ -745,7 +786,7 @@ iskv_status iskv_decode_attention_batched(
   p.count = count;
   p.nchunk = L.nchunk;
   p.nblk = L.nblk;
-  p.tc_values = tc_pv_supported(r, p.storage, n_q_heads) ? 1 : 0;
+  p.tc_values = tc_pv_supported(rv, p.storage, n_q_heads) ? 1 : 0;
   p.theta = rope_theta;
   p.scale = scale;
   p.n_cap_max = ncap;
@@ -784,7 +825,7 @@ iskv_status iskv_decode_attention_batched(
     j.n_vex = n_v_exact[i];
     j.n_total = n_total[i];
   }
-  const bool tc = tc_attn_supported(r, p.storage, head_dim, n_q_heads, n_kv_heads);
+  const bool tc = tc_attn_supported(rk, p.storage, head_dim, n_q_heads, n_kv_heads);
   std::vector<TcJob> tj;
   std::vector<ReconJob> rj;
   ReconParams rp;
@@ -799,12 +840,12 @@ iskv_status iskv_decode_attention_batched(
       rj[i].pos = hk[i].pos;
       rj[i].meta = hk[i].meta;
       rj[i].bsig = jobs[i].bsig;
-      if (!encode_attn_job(tj[i], hk[i].U, ncap, r, jobs[i].bsig, d, jobs[i].S, q[i], hk[i].pos,
+      if (!encode_attn_job(tj[i], hk[i].U, ncap, rk, jobs[i].bsig, d, jobs[i].S, q[i], hk[i].pos,
                            hk[i].meta, n_total[i], scale))
         return fail(ISKV_ERR_CUDA, "%s: tensor map encoding failed", who);
     }
     rp.d = d;
-    rp.r = r;
+    rp.r = rk;
     rp.storage = p.storage;
     rp.exact_dtype = exact_dtype;
     rp.out_dtype = ISKV_BF16;
@@ -819,7 +860,7 @@ iskv_status iskv_decode_attention_batched(
   if (p.tc_values) {
     pj.resize(count);
     for (int32_t i = 0; i < count; ++i)
-      if (!encode_pv_job(pj[i], hv[i].U, ncap, r, jobs[i].Pb, jobs[i].wpart, hv[i].meta))
+      if (!encode_pv_job(pj[i], hv[i].U, ncap, rv, jobs[i].Pb, jobs[i].wpart, hv[i].meta))
         return fail(ISKV_ERR_CUDA, "%s: tensor map encoding failed", who);
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -848,7 +889,7 @@ iskv_status iskv_decode_attention_batched(
   if (e == cudaSuccess) {
     if (p.tc_values) {
       PvParams pv;
-      pv.r = r;
+      pv.r = rv;
       pv.count = count;
       pv.nsplit = L.nchunk;
       e = launch_tc_pv(pv_dev, pv, s);
@@ -1024,6 +1065,12 @@ size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, i
   if (refit_rows > 0 && refit_in_one_fold(d, r_max, refit_rows)) {
     const size_t fr = iskv_fold_workspace_size(count, d, r_max, refit_rows);
     if (fr > need) need = fr;
+  } else if (refit_rows > 0) {
+    const int32_t rw = wide_refit_rank(d, r_max, block, refit_rows);
+    if (rw > 0) {
+      const size_t wr = wide_ws(d, rw, block, n_cap).total;
+      if (wr > need) need = wr;
+    }
   }
   return need;
 }
@@ -1097,7 +1144,7 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
     if (plan[i].rows > 0) {
       fold_idx.push_back(i);
       fold_rows[i] = plan[i].rows;
-      fold_blk[i] = plan[i].blk;
+      fold_blk[i] = plan[i].rw > 0 ? 0 : plan[i].blk;  // wide refits fold on their own below
     }
     if (plan[i].reorth) reorth_idx.push_back(i);
   }
@@ -1127,7 +1174,7 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
     // refits take pass 0 only, a refit by b-row folds passes 0 .. refit_rows / b - 1).
     std::vector<int32_t> sizes;
     for (int32_t i : fold_idx)
-      if (std::find(sizes.begin(), sizes.end(), fold_blk[i]) == sizes.end())
+      if (fold_blk[i] > 0 && std::find(sizes.begin(), sizes.end(), fold_blk[i]) == sizes.end())
         sizes.push_back(fold_blk[i]);
     std::sort(sizes.begin(), sizes.end());
     for (int32_t fb : sizes) {
@@ -1150,6 +1197,49 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
                                      fp.data(), tau_rel, ws, ws_bytes, stream);
         if (st != ISKV_OK) return st;
       }
+    }
+    // Wide refits, one table at a time (a first refit happens once per side): the history is
+    // copied into a wide one of rank rw inside the workspace, the refit rows are folded into it
+    // in b-row blocks (none truncates before the last), and its top r components come back.
+    for (int32_t i : fold_idx) {
+      if (plan[i].rw == 0) continue;
+      const iskv_exact_table *T = tables[i];
+      const iskv_lowrank *H = hists[i];
+      const int32_t rw = plan[i].rw;
+      const WideWs W = wide_ws(d, rw, b, ncap);
+      WidenArgs wa;
+      wa.U = H->U;
+      wa.B = H->B;
+      wa.sigma = H->sigma;
+      wa.pos = H->pos;
+      wa.meta = H->meta;
+      wa.Uw = base + W.U;
+      wa.Bw = base + W.B;
+      wa.sigw = reinterpret_cast<float *>(base + W.sig);
+      wa.posw = reinterpret_cast<int32_t *>(base + W.pos);
+      wa.metaw = reinterpret_cast<int64_t *>(base + W.meta);
+      wa.n_cap = ncap;
+      wa.d = d;
+      wa.r = r;
+      wa.rw = rw;
+      wa.esz = (int)elem_size(H->storage);
+      if ((e = launch_history_widen(wa, s)) != cudaSuccess) return cuda_fail(e, "refit: widen");
+      iskv_lowrank hw = *H;
+      hw.r_max = rw;
+      hw.U = wa.Uw;
+      hw.B = wa.Bw;
+      hw.sigma = wa.sigw;
+      hw.pos = wa.posw;
+      hw.meta = wa.metaw;
+      for (int32_t j = 0; j < plan[i].rows / b; ++j) {
+        const int64_t row0 = T->n_prot + (int64_t)j * b;
+        const void *Fj = static_cast<const char *>(T->rows) + (size_t)row0 * d * esz;
+        const int32_t *pj = T->pos + row0;
+        st = iskv_fold_block_batched(&hw, 1, &Fj, T0->dtype, b, &pj, tau_rel, base + W.fold,
+                                     iskv_fold_workspace_size(1, d, rw, b), stream);
+        if (st != ISKV_OK) return st;
+      }
+      if ((e = launch_history_narrow(wa, s)) != cudaSuccess) return cuda_fail(e, "refit: narrow");
     }
     EvictJob *dej = reinterpret_cast<EvictJob *>(base);
     stage_begin(s);

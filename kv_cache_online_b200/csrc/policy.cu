@@ -168,4 +168,66 @@ cudaError_t launch_cache_evict(const EvictJob *jobs, int count, cudaStream_t s) 
   return cudaGetLastError();
 }
 
+
+// ------------------------------------------------------------------------------------------------
+// Widening and narrowing of a history (the value side's first refit of a history that already
+// holds compressed rows; Section 3.2 and Algorithm 3 step 3). Rows 0 .. n_cap - 1 are U's rows,
+// rows n_cap .. n_cap + d - 1 are B's; one CTA per row walks it in 16-byte words.
+__global__ void k_history_widen(WidenArgs a) {
+  const int64_t row = blockIdx.x;
+  const int64_t n = a.meta[ISKV_META_N];
+  const bool is_u = row < a.n_cap;
+  const int64_t i = is_u ? row : row - a.n_cap;
+  const bool live = !is_u || row < n;  // U rows past n are zeroed (the workspace holds anything)
+  const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const char *>(is_u ? a.U : a.B) +
+                                                     (size_t)i * a.r * a.esz);
+  uint4 *dst = reinterpret_cast<uint4 *>(static_cast<char *>(is_u ? a.Uw : a.Bw) +
+                                         (size_t)i * a.rw * a.esz);
+  const int wr = live ? a.r * a.esz / 16 : 0, ww = a.rw * a.esz / 16;
+  for (int w = threadIdx.x; w < ww; w += blockDim.x) dst[w] = w < wr ? src[w] : make_uint4(0, 0, 0, 0);
+  if (!live) return;
+  if (is_u && threadIdx.x == 0) a.posw[i] = a.pos[i];
+  if (row == 0) {
+    for (int l = threadIdx.x; l < a.rw; l += blockDim.x) a.sigw[l] = l < a.r ? a.sigma[l] : 0.f;
+    if (threadIdx.x < 4) a.metaw[threadIdx.x] = a.meta[threadIdx.x];
+  }
+}
+
+__global__ void k_history_narrow(WidenArgs a) {
+  const int64_t row = blockIdx.x;
+  const int64_t n = a.metaw[ISKV_META_N];
+  const bool is_u = row < a.n_cap;
+  if (is_u && row >= n) return;
+  const int64_t i = is_u ? row : row - a.n_cap;
+  const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const char *>(is_u ? a.Uw : a.Bw) +
+                                                     (size_t)i * a.rw * a.esz);
+  uint4 *dst = reinterpret_cast<uint4 *>(static_cast<char *>(is_u ? a.U : a.B) +
+                                         (size_t)i * a.r * a.esz);
+  const int wr = a.r * a.esz / 16;
+  for (int w = threadIdx.x; w < wr; w += blockDim.x) dst[w] = src[w];
+  if (is_u && threadIdx.x == 0) a.pos[i] = a.posw[i];
+  if (row == 0) {
+    for (int l = threadIdx.x; l < a.r; l += blockDim.x) a.sigma[l] = a.sigw[l];
+    if (threadIdx.x == 0) {
+      const int64_t kw = a.metaw[ISKV_META_K];
+      a.meta[ISKV_META_K] = kw < a.r ? kw : a.r;
+      a.meta[ISKV_META_N] = n;
+      a.meta[2] = a.metaw[2];
+      a.meta[ISKV_META_STATUS] |= a.metaw[ISKV_META_STATUS];
+    }
+  }
+}
+
+cudaError_t launch_history_widen(const WidenArgs &a, cudaStream_t s) {
+  k_history_widen<<<(unsigned)(a.n_cap + a.d), 128, 0, s>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_history_narrow(const WidenArgs &a, cudaStream_t s) {
+  k_history_narrow<<<(unsigned)(a.n_cap + a.d), 128, 0, s>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace iskv

@@ -42,6 +42,27 @@ struct EvictJob {
   int32_t pad_;
 };
 
+// A history copied into a wider one (rank budget rw >= r, the same n_cap) and back. Widening
+// copies U's n rows (n from the device meta word) and B into rows of rw entries with zeros after
+// the first r, and sigma, positions and meta; narrowing keeps the first r columns of the wide
+// history (its components are sorted by singular value, so these are its top r), sets k to
+// min(r, k') and n to n', and ORs the wide history's status bits into the history's.
+struct WidenArgs {
+  void *U, *B;            // [n_cap][r], [d][r] (storage dtype)
+  float *sigma;           // [r]
+  int32_t *pos;           // [n_cap]
+  int64_t *meta;          // [4]
+  void *Uw, *Bw;          // [n_cap][rw], [d][rw]
+  float *sigw;            // [rw]
+  int32_t *posw;          // [n_cap]
+  int64_t *metaw;         // [4]
+  int64_t n_cap;
+  int d, r, rw, esz;      // esz: element bytes of U and B (r * esz and rw * esz multiples of 16)
+};
+
+cudaError_t launch_history_widen(const WidenArgs &a, cudaStream_t s);
+cudaError_t launch_history_narrow(const WidenArgs &a, cudaStream_t s);
+
 cudaError_t launch_prefill_partition(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_cache_append(const AppendJob *jobs, int count, int d, int src_dtype,
                                 int dst_dtype, cudaStream_t s);

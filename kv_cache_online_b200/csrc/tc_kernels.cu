@@ -1013,14 +1013,14 @@ static cudaError_t attn_scores_qpk(const TcJob *djobs, const TcParams &tp, int G
 
 cudaError_t launch_tc_attn_scores(const TcJob *djobs, const AttnParams &p, cudaStream_t s) {
   TcParams tp;
-  tp.r = p.r;
+  tp.r = p.rk;
   tp.d = p.d;
   tp.n_heads = p.n_kv;
   tp.count = p.count;
   tp.tiles_per_job = (int)((p.n_cap_max + TC_M - 1) / TC_M);
   tp.theta = p.theta;
   const int qpk = p.n_q / p.n_kv;
-  tc_rec_shape(p.r, p.n_kv, rec_stg_bytes(qpk), tp.hp, tp.stages);
+  tc_rec_shape(p.rk, p.n_kv, rec_stg_bytes(qpk), tp.hp, tp.stages);
   const int G = p.n_kv / tp.hp;
   switch (qpk) {
     case 1: return attn_scores_qpk<1>(djobs, tp, G, s);

@@ -145,7 +145,7 @@ def _fake_table(L, live, d=1024, window=128, block=64, cap_e=1024, dtype=1, base
 def test_cache_policy_host_side_errors():
     """The cache-policy entry points refuse bad tables on the host and leave the mirror unchanged."""
     L, lib = _lib()
-    live = (ctypes.c_int32 * 256)()
+    live = (ctypes.c_int32 * 512)()
     ws = ctypes.c_void_p(0x40000)
     big = 1 << 40
     X = ctypes.c_void_p(0x20000)
@@ -185,20 +185,20 @@ def test_cache_policy_host_side_errors():
     t3 = _fake_table(L, live, block=12)
     tp3 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t3))
     assert lib.iskv_cache_step(tp3, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
-    # a refit that is not a multiple of the block; a refit due on a non-empty history that one
-    # fold cannot take
+    # a refit that is not a multiple of the block; a refit due on a non-empty history that neither
+    # one fold nor a wide history of rank r_max + refit_rows - block <= 512 takes
     t5 = _fake_table(L, live, window=0, block=8)
     t5.refit_rows, t5.refit_done, t5.live_cap = 12, 0, 12
     tp5 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t5))
     assert lib.iskv_cache_step(tp5, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
     t6 = _fake_table(L, live, window=0, block=8)
-    t6.refit_rows, t6.refit_done, t6.live_cap = 136, 0, 136   # more rows than one fold takes
-    for i in range(135):
+    t6.refit_rows, t6.refit_done, t6.live_cap = 280, 0, 280   # 256 + 280 - 8 > 512
+    for i in range(279):
         live[i] = i
-    t6.n_live, t6.last, t6.hist_rows = 135, 134, 100
+    t6.n_live, t6.last, t6.hist_rows = 279, 278, 100
     tp6 = (ctypes.POINTER(L.IskvExactTable) * 1)(ctypes.pointer(t6))
     assert lib.iskv_cache_step(tp6, hp, 1, rows, 1, 0.0, None, None, ws, big, None) == 2
-    assert b"empty" in lib.iskv_last_error()
+    assert b"wide history" in lib.iskv_last_error()
     ta, tb = _fake_table(L, live), _fake_table(L, live, d=512)
     tp4 = (ctypes.POINTER(L.IskvExactTable) * 2)(ctypes.pointer(ta), ctypes.pointer(tb))
     hp4 = (ctypes.POINTER(L.IskvLowRank) * 2)(ctypes.pointer(h), ctypes.pointer(h))

@@ -105,3 +105,34 @@ def test_key_without_value_is_flagged():
     m.decode_attention(hk, hv, a["k_exact"], a["k_exact_pos"], a["v_exact"][:keep].contiguous(),
                        a["v_exact_pos"][:keep].contiguous(), a["n_total"], a["q"], 2, 128)
     assert hv.status()[3] & bit(2)
+
+
+@pytest.mark.parametrize("storage,rk,rv,tol", [(torch.float32, 32, 48, 1e-4),
+                                               (torch.bfloat16, 256, 128, 2e-2),
+                                               (torch.bfloat16, 128, 256, 2e-2)])
+def test_keys_and_values_of_different_rank(storage, rk, rv, tol):
+    """A K history and a V history with their own rank budgets (Section 8's separate K / V
+    ranks), both full to their budget."""
+    m = kv()
+    d, n_kv, n = (256, 2, 700) if storage == torch.float32 else (1024, 8, 1200)
+    g = np.random.Generator(np.random.PCG64(rk + rv))
+    Uk, sk, Bk = synthetic_history(n, d, rk, 61, 1.2, storage)
+    Uv, sv, Bv = synthetic_history(n, d, rv, 62, 0.6, storage)
+    prompt, window = 64, 32
+    n_total = prompt + n + window
+    comp = prompt + np.arange(n)
+    exact = np.setdiff1d(np.arange(n_total), comp)
+    hk = m.LowRankHistory(d, rk, n + 8, storage=storage)
+    hv = m.LowRankHistory(d, rv, n + 8, storage=storage)
+    set_state(hk, Uk, sk, Bk, comp)
+    set_state(hv, Uv, sv, Bv, comp)
+    Kex = stored(0.3 * g.standard_normal((exact.size, d)), storage)
+    Vex = stored(0.3 * g.standard_normal((exact.size, d)), storage)
+    q = stored(48 * g.standard_normal((4 * n_kv, 128)) / np.sqrt(128), torch.float32)
+    t = lambda a, dt: torch.as_tensor(a, dtype=dt, device="cuda").contiguous()
+    out = m.decode_attention(hk, hv, t(Kex, storage), t(exact, torch.int32), t(Vex, storage),
+                             t(exact, torch.int32), n_total, t(q, torch.float32), n_kv, 128)
+    ref = oatt.decode_attention((Uk, sk, Bk, comp), (Uv, sv, Bv, comp), Kex, exact, Vex, exact,
+                                n_total, q, n_kv, 128, 500000.0)
+    assert hk.status()[3] == 0 and hv.status()[3] == 0
+    assert _rel(out.double().cpu().numpy(), ref) < tol

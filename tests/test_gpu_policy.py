@@ -71,12 +71,16 @@ def test_prefill_rejects_unordered_protected_positions():
         m.cache_prefill(t, X, torch.tensor([5, 100], dtype=torch.int32, device="cuda"), 32)
 
 
-def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36, refit=0, v_all=None):
+def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36, refit=0, v_all=None,
+         rv=None):
     """Two sequences x (K, V) = four tables stepped together through T decode steps, against four
     oracle runs started from the same stored prompt factors. With ``refit`` > 0 the value sides run
     the first refit of ``refit`` rows; ``v_all`` (default: when refitting) protects their whole
-    prompt (a short prompt), so that their history is empty at the refit."""
+    prompt (a short prompt), so that their history is empty at the refit. ``rv`` gives the value
+    sides their own rank budget; the key and value tables then step as two batches (a batched
+    step takes histories of one rank)."""
     v_all = bool(refit) if v_all is None else v_all
+    rv = r if rv is None else rv
     sides = []
     for s, L in enumerate(Ls):
         PK = _protected(L, seed + s, suffix=suffix)
@@ -84,7 +88,8 @@ def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36, refit=0, v_a
         for kind, P, w0, ex in (("K", PK, 0, 1.1), ("V", PV, min(W, L), 0.7)):
             X = stored(synth.lowrank_rows(L + T, d, ex, 0.02, seed=seed + 10 * s + len(sides)),
                        storage)
-            sides.append(dict(kind=kind, L=L, P=P, w0=w0, X=X, F=refit if kind == "V" else 0))
+            sides.append(dict(kind=kind, L=L, P=P, w0=w0, X=X, F=refit if kind == "V" else 0,
+                              r=rv if kind == "V" else r))
     n_cap = max(L for L in Ls) + T
     tabs, hists, refs = [], [], []
     for sd in sides:
@@ -96,22 +101,28 @@ def _run(m, *, d, r, b, W, R, Ls, T, storage, seed, tol, suffix=36, refit=0, v_a
                                               torch.as_tensor(sd["P"], dtype=torch.int32,
                                                               device="cuda"), sd["w0"])
         if comp_pos.numel():
-            U0, s0, B0 = of.truncated_svd(sd["X"][comp_pos.cpu().numpy()], r)
+            U0, s0, B0 = of.truncated_svd(sd["X"][comp_pos.cpu().numpy()], sd["r"])
         else:
             U0, s0, B0 = of.empty_history(d)
         U0, s0, B0 = stored(U0, storage), stored(s0, torch.float32), stored(B0, storage)
-        h = m.LowRankHistory(d, r, n_cap, storage=storage)
+        h = m.LowRankHistory(d, sd["r"], n_cap, storage=storage)
         set_state(h, U0, s0, B0, comp_pos.cpu().numpy())
-        ref = op.run_decode(sd["X"][:L], sd["X"][L:], sd["P"], sd["w0"], W, b, r, R,
+        ref = op.run_decode(sd["X"][:L], sd["X"][L:], sd["P"], sd["w0"], W, b, sd["r"], R,
                             init_history=(U0, s0, B0), refit_rows=sd["F"])
         sd["Xd"] = Xd
         tabs.append(t)
         hists.append(h)
         refs.append(ref)
-    batch = m.CacheBatch(tabs, hists)
+    groups = [list(range(len(sides)))] if rv == r else [
+        [k for k, sd in enumerate(sides) if sd["kind"] == kind] for kind in ("K", "V")]
+    batches = [m.CacheBatch([tabs[k] for k in g], [hists[k] for k in g]) for g in groups]
     for i in range(T):
-        rows = torch.stack([sd["Xd"][sd["L"] + i] for sd in sides]).contiguous()
-        folded, reorthed = batch.step(rows)
+        folded, reorthed = [0] * len(sides), [False] * len(sides)
+        for g, batch in zip(groups, batches):
+            rows = torch.stack([sides[k]["Xd"][sides[k]["L"] + i] for k in g]).contiguous()
+            fo, re = batch.step(rows)
+            for j, k in enumerate(g):
+                folded[k], reorthed[k] = fo[j], re[j]
         for k, ref in enumerate(refs):
             acts = [a[0] for a in ref["steps"][i]]
             assert folded[k] == (2 if "refit" in acts else 1 if "fold" in acts else 0), (i, k)
@@ -193,8 +204,22 @@ def test_refit_by_untruncated_block_folds():
     _refits(refs, tabs)
 
 
+def test_refit_of_a_compressed_history_through_a_wide_history():
+    """The pages' value refit (Section 3.2, Algorithm 3 step 3): r_V = 256 pending rows into a
+    history that already holds compressed prompt rows, at d = 1024, r = 256, b = 64 -- four 64-row
+    folds into a wide history of rank 448 (none truncates before the last), whose top 256
+    components come back: the rank-256 SVD of the history's rows followed by the refit rows."""
+    m = kv()
+    sides, tabs, hists, refs = _run(m, d=1024, r=256, b=64, W=128, R=256, Ls=(600, 450), T=450,
+                                    storage=torch.float32, seed=88, tol=1e-4, suffix=8,
+                                    refit=256, v_all=False)
+    _refits(refs, tabs)
+    assert all(len(refs[k]["comp"]) > 0 for k in (1, 3))
+
+
 def test_refit_that_runs_neither_way_is_refused():
-    """144 rows (more than one fold takes) into a history that already holds compressed rows."""
+    """144 rows (more than one fold takes) into a history that already holds compressed rows, where
+    the wide history would need rank 160 + 144 - 16 = 288 > d = 256."""
     m = kv()
     d, b, rv = 256, 16, 144
     X = torch.randn(300, d, device="cuda")
@@ -216,3 +241,41 @@ def test_decode_policy_bf16_model_width():
     m = kv()
     _run(m, d=1024, r=64, b=64, W=128, R=128, Ls=(600, 450), T=300, storage=torch.bfloat16,
          seed=90, tol=2e-2)
+
+
+def _attention_check(m, sides, tabs, hists, refs, T, n_kv, tol, seed):
+    """Decode attention of sequence 0 straight from its K and V tables (Algorithm 3 steps 7-9)."""
+    g = np.random.Generator(np.random.PCG64(seed))
+    q = stored(40 * g.standard_normal((4 * n_kv, 128)) / np.sqrt(128), torch.float32)
+    n_total = sides[0]["L"] + T
+    kr, kp = tabs[0].exact()
+    vr, vp = tabs[1].exact()
+    out = m.decode_attention(hists[0], hists[1], kr, kp, vr, vp, n_total,
+                             torch.as_tensor(q, dtype=torch.float32, device="cuda"), n_kv, 128)
+    assert hists[0].status()[3] == 0 and hists[1].status()[3] == 0
+    rk, rv = refs[0], refs[1]
+    want = oatt.decode_attention(rk["history"], rv["history"], rk["exact"][0], rk["exact"][1],
+                                 rv["exact"][0], rv["exact"][1], n_total, q, n_kv, 128)
+    assert float(np.linalg.norm(np64(out) - want) / np.linalg.norm(want)) < tol
+
+
+def test_decode_policy_different_key_and_value_ranks_fp32():
+    """Keys at r = 32 and values at r = 48 (Section 8's separate K / V ranks): the key and value
+    tables step as two batches, then decode attention reads a K history and a V history of
+    different rank."""
+    m = kv()
+    T = 130
+    sides, tabs, hists, refs = _run(m, d=256, r=32, rv=48, b=16, W=24, R=32, Ls=(300, 180), T=T,
+                                    storage=torch.float32, seed=75, tol=1e-4, suffix=8)
+    assert hists[0].r_max == 32 and hists[1].r_max == 48
+    _attention_check(m, sides, tabs, hists, refs, T, 2, 1e-4, 76)
+
+
+def test_decode_policy_different_key_and_value_ranks_bf16_model_width():
+    """d = 1024 (8 KV heads x 128), keys at r = 256 and values at r = 128, b = 64, W = 128, bf16:
+    the tensor-core score and value kernels each at their own rank."""
+    m = kv()
+    T = 200
+    sides, tabs, hists, refs = _run(m, d=1024, r=256, rv=128, b=64, W=128, R=256, Ls=(600, 450),
+                                    T=T, storage=torch.bfloat16, seed=95, tol=2e-2)
+    _attention_check(m, sides, tabs, hists, refs, T, 8, 2e-2, 96)

@@ -102,24 +102,26 @@ def test_schedule_on_hand_worked_cases(name):
 
 
 def test_refused_step_changes_nothing():
-    """A 136-row refit (more than one fold takes) due on a history that holds compressed rows is
-    refused, and the mirror stays as it was; an empty history takes it as untruncated folds."""
+    """A first refit due on a history that already holds compressed rows runs through a wide
+    history of rank r + refit_rows - block when that rank is at most 512 (136 rows at r = 256,
+    b = 8: rank 384); 280 rows would need rank 528 and are refused, leaving the mirror as it was.
+    An empty history takes 136 rows as untruncated folds."""
     L_, lib = _lib()
-    for hist_rows, want in ((100, 2), (0, 0)):
-        side, comp = op.new_side(0, [], 0, 0, 8, 0, 136)
-        tab = _Table(L_, side, comp, 0, 8, 0, 136)
+    for rows, hist_rows, want in ((280, 100, 2), (136, 100, 0), (136, 0, 0)):
+        side, comp = op.new_side(0, [], 0, 0, 8, 0, rows)
+        tab = _Table(L_, side, comp, 0, 8, 0, rows)
         tab.t.hist_rows = hist_rows
         arr = (ctypes.POINTER(L_.IskvExactTable) * 1)(ctypes.pointer(tab.t))
         folded = (ctypes.c_int32 * 1)()
-        for _ in range(135):
+        for _ in range(rows - 1):
             assert lib.iskv_cache_plan(arr, 1, R, NCAP, 1, folded, None) == 0
         before = tab.mirror()
         assert lib.iskv_cache_plan(arr, 1, R, NCAP, 1, folded, None) == want
         if want:
-            assert b"empty history" in lib.iskv_last_error()
+            assert b"wide history" in lib.iskv_last_error()
             assert tab.mirror() == before
         else:
-            assert folded[0] == 2 and tab.t.n_live == 0 and tab.t.hist_rows == 136
+            assert folded[0] == 2 and tab.t.n_live == 0 and tab.t.hist_rows == hist_rows + rows
 
 
 def test_history_capacity_is_checked_before_the_fold():
