@@ -126,8 +126,8 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
  * B = Q_B R_B, decompose R_U diag(sigma) R_B^T = X diag(sigma') Y^T and set U <- Q_U X,
  * sigma <- sigma', B <- Q_B Y. The product U diag(sigma) B^T is unchanged in exact arithmetic;
  * k and n are unchanged; meta[FOLDS] is reset to 0. hs is a HOST array of `count` handles sharing
- * d, r_max, storage and n_cap. r_max <= 384 (the dense r x r core SVD must fit one thread-block
- * cluster); larger r_max returns ISKV_ERR_SHAPE.
+ * d, r_max, storage and n_cap. Any r_max a history may have (<= 512) fits the dense r x r core
+ * SVD's thread-block cluster.
  */
 size_t iskv_reorth_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap);
 iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t ws_bytes,
@@ -346,7 +346,8 @@ typedef struct {
  * Writes the protected rows, then the unprotected rows among the last init_window positions, into
  * the exact-row table (converted to t->dtype), and every other row, in ascending position, into
  * comp_rows [L][d] (x_dtype) with comp_pos [L]: the rows the prompt's truncated SVD compresses
- * (Algorithm 1 step 7; that SVD itself is not part of the library). Sets the host mirror
+ * (Algorithm 1 step 7; iskv_compress_prompt() folds them into the side's history). Sets the host
+ * mirror
  * (n_prot = n_protected, n_live, live_host, last = L - 1, fold_rows = 0, hist_rows = *n_comp,
  * refit_done = (refit_rows == 0)) and *n_comp (host). The caller then puts the compressed rows'
  * factors in the side's history, with their positions comp_pos in its position table.
@@ -371,17 +372,44 @@ iskv_status iskv_cache_prefill(iskv_exact_table *t, const void *X, int32_t x_dty
  * history's position table and their exact copies leave the table; when a table's folded rows
  * reach reorth_rows, its history is re-orthogonalised (iskv_reorth) in the same step and the count
  * restarts. A table whose first refit is still to come waits for refit_rows pending rows instead,
- * then folds all of them (in one fold or in untruncated block folds, as above). All tables share
+ * then factors the history's rows followed by those rows at rank r_max (Section 3.2, Algorithm 3
+ * step 3): as one fold of all of them when the fold takes such a block; for an empty history with
+ * refit_rows <= r_max, as untruncated block folds; otherwise as block folds into a wide history of
+ * rank r_max + refit_rows - block (rounded up to a multiple of 16, at most 512 and d) held in the
+ * workspace, none of which truncates before the last, whose top r_max components come back -- in
+ * every case the rank-r_max truncated SVD of those rows (Eckart-Young). All tables share
  * d, window, block and dtype; the histories share d, r_max, storage and n_cap, as the batched fold
  * and re-orthogonalisation require. folded / reorthed (host [count], may be NULL) receive 1 where a
  * table folded a block (2 where it ran its first refit) / re-orthogonalised. Stream-ordered; the
  * host mirror is updated at once. The workspace query takes the largest refit_rows of the tables
  * (0 when none refits). Errors (nothing launched, no table changed): ISKV_ERR_ARG,
  * ISKV_ERR_SHAPE (mixed table shapes, a history whose d differs, a block the fold does not take, a
- * refit that can be run neither way), ISKV_ERR_CAPACITY (a table without room for the new row, or
+ * refit that can be run none of these ways), ISKV_ERR_CAPACITY (a table without room for the new row, or
  * a history without room for the block or the refit: hist_rows + rows > n_cap),
  * ISKV_ERR_WORKSPACE; ISKV_ERR_CUDA when a launch fails.
  */
+/*
+ * Compression of the prompt rows on the device (Algorithm 1 step 7): for each history hs[i], the
+ * n_rows[i] rows rows[i] ([n_rows[i]][d] dtype, device, ascending positions pos[i] [n_rows[i]]
+ * int32 device -- the comp_rows / comp_pos of iskv_cache_prefill) are folded (Algorithm 2) in
+ * blocks of `block` rows; a last block of t < block rows is folded as ceil(t / 8) * 8 rows, the
+ * real ones followed by zero rows, whose coordinate rows (zero) are then dropped again, so the
+ * history ends with exactly n_rows[i] more rows. Reading of the pages' "truncated SVD of the
+ * compressed prompt rows": the block fold reaches that SVD exactly when no fold truncates before
+ * the last, i.e. when the history's rank plus n_rows[i] - (last block) stays within r_max; a longer
+ * prompt is compressed incrementally, as the long-prompt workload compresses its prompt (rank 512
+ * by folds of 128 rows). Histories usually start empty; the batched fold's rules apply (shared d,
+ * r_max, storage; 8 <= block <= 128, a multiple of 8). Stream-ordered, no host synchronisation.
+ * ws: iskv_compress_prompt_workspace_size(count, d, r_max, block) bytes, 256-byte aligned.
+ * Errors: as iskv_fold_block_batched (ISKV_ERR_CAPACITY in a status word when a history has no
+ * room for its rows).
+ */
+size_t iskv_compress_prompt_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block);
+iskv_status iskv_compress_prompt(const iskv_lowrank *hs, int32_t count, const void *const *rows,
+                                 const int32_t *const *pos, const int64_t *n_rows, int32_t dtype,
+                                 int32_t block, float tau_rel, void *ws, size_t ws_bytes,
+                                 void *stream);
+
 size_t iskv_cache_step_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block,
                                       int64_t n_cap, int32_t refit_rows);
 iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank *const *hists,

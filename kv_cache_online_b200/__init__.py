@@ -392,6 +392,43 @@ def cache_prefill(table: ExactTable, X, protected_pos, init_window: int, ws=None
     return comp[:n_comp.value], comp_pos[:n_comp.value]
 
 
+def compress_prompt_workspace_size(count, d, r_max, block) -> int:
+    return int(_lib.load().iskv_compress_prompt_workspace_size(count, d, r_max, block))
+
+
+def compress_prompt(hists, rows, positions, block: int = 64, tau_rel: float = 0.0, ws=None,
+                    stream=None):
+    """Algorithm 1 step 7 on the device: fold each history's compressed prompt rows
+    (``rows[i]`` (n_i, d), ``positions[i]`` int32 -- what :func:`cache_prefill` returns) in blocks
+    of ``block`` rows (a short last block padded with zero rows that are dropped again)."""
+    if isinstance(hists, LowRankHistory):
+        hists, rows, positions = [hists], [rows], [positions]
+    lib = _lib.load()
+    n = len(hists)
+    d = hists[0].d
+    rp, pp, nr = [], [], []
+    dt = ISKV_F32
+    for x, p in zip(rows, positions):
+        if x is None or p is None or p.numel() == 0:
+            rp.append(None)
+            pp.append(None)
+            nr.append(0)
+            continue
+        _need_cuda(x, p)
+        if p.dtype != torch.int32 or x.shape != (p.numel(), d) or not x.is_contiguous():
+            raise ValueError("rows must be (n, d) contiguous with int32 positions")
+        dt = _dt(x)
+        rp.append(x.data_ptr())
+        pp.append(p.data_ptr())
+        nr.append(p.numel())
+    need = lib.iskv_compress_prompt_workspace_size(n, d, hists[0].r_max, block)
+    w = ws if ws is not None else _ws(hists[0].device, need)
+    P = ctypes.c_void_p * n
+    _lib.check(lib.iskv_compress_prompt(_handles(hists), n, P(*rp), P(*pp),
+                                        (ctypes.c_int64 * n)(*nr), dt, int(block), float(tau_rel),
+                                        w.data_ptr(), w.numel(), _stream(stream)), "compress_prompt")
+
+
 def cache_step_workspace_size(count, d, r_max, block, n_cap, refit_rows=0) -> int:
     return int(_lib.load().iskv_cache_step_workspace_size(count, d, r_max, block, n_cap,
                                                           refit_rows))

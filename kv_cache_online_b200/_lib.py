@@ -97,6 +97,10 @@ SIGNATURES = {
     "iskv_stage_reset": (None, []),
     "iskv_launch_count": (c_i64, []),
     "iskv_core_stats": (c_i32, [c_vp, c_i32]),
+    "iskv_compress_prompt_workspace_size": (c_sz, [c_i32, c_i32, c_i32, c_i32]),
+    "iskv_compress_prompt": (c_i32, [ctypes.POINTER(IskvLowRank), c_i32, ctypes.POINTER(c_vp),
+                                     ctypes.POINTER(c_vp), ctypes.POINTER(c_i64), c_i32, c_i32,
+                                     c_f32, c_vp, c_sz, c_vp]),
     "iskv_selftest_wait_timeout": (c_i32, [c_vp, c_i64, c_vp]),
 }
 

@@ -442,7 +442,7 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   {
     JacobiCfg jc;
     if (!core_cfg(r, 0, true, jc))
-      return fail(ISKV_ERR_SHAPE, "%s: r_max = %d too large for the dense core SVD (r_max <= 384)",
+      return fail(ISKV_ERR_SHAPE, "%s: r_max = %d too large for the dense core SVD",
                   who, r);
   }
   const size_t need = iskv_reorth_workspace_size(count, d, r, ncap);
@@ -1261,6 +1261,109 @@ iskv_status iskv_cache_step(iskv_exact_table *const *tables, const iskv_lowrank 
     advance_table(tables[i], plan[i]);
     if (folded) folded[i] = plan[i].rows > 0 ? (plan[i].refit ? 2 : 1) : 0;
     if (reorthed) reorthed[i] = plan[i].reorth ? 1 : 0;
+  }
+  return ISKV_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Prompt compression (Algorithm 1 step 7) by block folds.
+size_t iskv_compress_prompt_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t block) {
+  if (count < 1 || d < 1 || r_max < 1 || block < 1) return 0;
+  size_t need = align_up(iskv_fold_workspace_size(count, d, r_max, block), 256);
+  need += jobs_bytes(count, sizeof(TailJob));
+  need += (size_t)count * align_up((size_t)block * d * sizeof(float), 256);
+  need += (size_t)count * align_up((size_t)block * sizeof(int32_t), 256);
+  return need;
+}
+
+iskv_status iskv_compress_prompt(const iskv_lowrank *hs, int32_t count, const void *const *rows,
+                                 const int32_t *const *pos, const int64_t *n_rows, int32_t dtype,
+                                 int32_t block, float tau_rel, void *ws, size_t ws_bytes,
+                                 void *stream) {
+  const char *who = "iskv_compress_prompt";
+  g_last_error.clear();
+  if (!hs || !rows || !pos || !n_rows) return fail(ISKV_ERR_ARG, "%s: null host array", who);
+  if (count < 1 || count > 4096) return fail(ISKV_ERR_SHAPE, "%s: count must be in [1, 4096]", who);
+  if (!valid_dtype(dtype)) return fail(ISKV_ERR_ARG, "%s: bad dtype", who);
+  if (!(tau_rel >= 0.f)) return fail(ISKV_ERR_ARG, "%s: tau_rel must be >= 0", who);
+  int64_t nb_max = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    iskv_status st = check_handle(&hs[i], who);
+    if (st != ISKV_OK) return st;
+    if (hs[i].d != hs[0].d || hs[i].r_max != hs[0].r_max || hs[i].storage != hs[0].storage)
+      return fail(ISKV_ERR_SHAPE, "%s: histories must share d, r_max, storage", who);
+    if (n_rows[i] < 0) return fail(ISKV_ERR_SHAPE, "%s: negative row count", who);
+    if (n_rows[i] > 0 && (!rows[i] || !pos[i]))
+      return fail(ISKV_ERR_ARG, "%s: null rows or positions", who);
+    if (n_rows[i] > 0 && (!aligned(rows[i], 16) || !aligned(pos[i], 4)))
+      return fail(ISKV_ERR_ARG, "%s: rows must be 16-byte aligned", who);
+    if (n_rows[i] / block > nb_max) nb_max = n_rows[i] / block;
+  }
+  const int d = hs[0].d, r = hs[0].r_max;
+  if (block < 8 || block % 8 || block > 128 || block > d)
+    return fail(ISKV_ERR_SHAPE, "%s: need 8 <= block <= min(d, 128), block %% 8 == 0", who);
+  const size_t need = iskv_compress_prompt_workspace_size(count, d, r, block);
+  iskv_status st = check_ws(ws, ws_bytes, need, who);
+  if (st != ISKV_OK) return st;
+  const size_t esz = elem_size(dtype), fw = align_up(iskv_fold_workspace_size(count, d, r, block), 256);
+  char *base = static_cast<char *>(ws);
+  TailJob *tjobs = reinterpret_cast<TailJob *>(base + fw);
+  char *tbuf = base + fw + jobs_bytes(count, sizeof(TailJob));
+  const size_t rowbuf = align_up((size_t)block * d * sizeof(float), 256);
+  char *pbuf = tbuf + (size_t)count * rowbuf;
+  const size_t posbuf = align_up((size_t)block * sizeof(int32_t), 256);
+  // Full blocks: pass j folds block j of every history that has more than j of them.
+  for (int64_t j = 0; j < nb_max; ++j) {
+    std::vector<iskv_lowrank> fh;
+    std::vector<const void *> F;
+    std::vector<const int32_t *> fp;
+    for (int32_t i = 0; i < count; ++i) {
+      if (n_rows[i] / block <= j) continue;
+      fh.push_back(hs[i]);
+      F.push_back(static_cast<const char *>(rows[i]) + (size_t)j * block * d * esz);
+      fp.push_back(pos[i] + j * block);
+    }
+    st = iskv_fold_block_batched(fh.data(), (int32_t)fh.size(), F.data(), dtype, block, fp.data(),
+                                 tau_rel, ws, fw, stream);
+    if (st != ISKV_OK) return st;
+  }
+  // Short last blocks, one batched fold per padded size.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int32_t t8 = 8; t8 <= block; t8 += 8) {
+    std::vector<TailJob> tj;
+    std::vector<iskv_lowrank> fh;
+    std::vector<const void *> F;
+    std::vector<const int32_t *> fp;
+    for (int32_t i = 0; i < count; ++i) {
+      const int32_t t = (int32_t)(n_rows[i] % block);
+      if (t == 0 || (t + 7) / 8 * 8 != t8) continue;
+      const int64_t row0 = n_rows[i] - t;
+      const int k = (int)tj.size();
+      TailJob j;
+      j.src = static_cast<const char *>(rows[i]) + (size_t)row0 * d * esz;
+      j.src_pos = pos[i] + row0;
+      j.dst = tbuf + (size_t)k * rowbuf;
+      j.dst_pos = reinterpret_cast<int32_t *>(pbuf + (size_t)k * posbuf);
+      j.meta = hs[i].meta;
+      j.row_bytes = (int64_t)d * (int64_t)esz;
+      j.n0 = 0;
+      j.t = t;
+      j.t8 = t8;
+      tj.push_back(j);
+      fh.push_back(hs[i]);
+      F.push_back(j.dst);
+      fp.push_back(j.dst_pos);
+    }
+    if (tj.empty()) continue;
+    const int nt = (int)tj.size();
+    cudaError_t e = upload_jobs(tjobs, tj.data(), sizeof(TailJob) * nt, s);
+    if (e == cudaSuccess) e = launch_tail_pad(tjobs, nt, s);
+    if (e != cudaSuccess) return cuda_fail(e, "compress prompt: pad");
+    st = iskv_fold_block_batched(fh.data(), nt, F.data(), dtype, t8, fp.data(), tau_rel, ws, fw,
+                                 stream);
+    if (st != ISKV_OK) return st;
+    if ((e = launch_tail_drop(tjobs, nt, s)) != cudaSuccess)
+      return cuda_fail(e, "compress prompt: drop");
   }
   return ISKV_OK;
 }

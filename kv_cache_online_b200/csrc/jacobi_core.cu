@@ -62,9 +62,9 @@ __host__ __device__ inline CoreSmem core_smem(int cj, int w, int ne, bool dbuf) 
 constexpr size_t kCoreSmemCap = 200 * 1024;
 
 // Threads per CTA the register file allows for NE column entries per lane (four columns live in
-// registers): 640 x 96, 512 x 128 or 384 x 170 registers.
+// registers): 640 x 96, 512 x 128, 384 x 170 or 256 x 255 registers.
 __host__ __device__ constexpr int core_max_threads(int ne) {
-  return ne <= 12 ? 640 : (ne <= 16 ? 512 : 384);
+  return ne <= 12 ? 640 : (ne <= 16 ? 512 : (ne <= 24 ? 384 : 256));
 }
 
 // Columns per block w (two blocks per CTA, two column pairs per warp, so w / 2 warps): the
@@ -73,12 +73,12 @@ __host__ __device__ constexpr int core_max_threads(int ne) {
 JacobiCfg jacobi_cfg(int ncols_max, int col_len_max) {
   JacobiCfg c;
   int ne = (col_len_max + 31) / 32;
-  const int choices[] = {2, 4, 8, 12, 16, 20, 24};
+  const int choices[] = {2, 4, 8, 12, 16, 20, 24, 32};
   int pick = 0;
   for (int v : choices)
     if (v >= ne) { pick = v; break; }
   c.ne = pick;
-  const int nes = pick ? pick : 24;
+  const int nes = pick ? pick : 32;
   for (int cj = 1; cj <= 16; cj *= 2) {
     int w = (ncols_max + 2 * cj - 1) / (2 * cj);
     w += w & 1;
@@ -528,7 +528,8 @@ cudaError_t launch_core(const char *jobs, const CoreParams &p, cudaStream_t s) {
     case 12: return core_launch<12>(jobs, p, c, s);
     case 16: return core_launch<16>(jobs, p, c, s);
     case 20: return core_launch<20>(jobs, p, c, s);
-    default: return core_launch<24>(jobs, p, c, s);
+    case 24: return core_launch<24>(jobs, p, c, s);
+    default: return core_launch<32>(jobs, p, c, s);
   }
 }
 

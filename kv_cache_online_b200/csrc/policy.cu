@@ -230,4 +230,39 @@ cudaError_t launch_history_narrow(const WidenArgs &a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------------------------------
+// Short last block of a prompt compression (Algorithm 1 step 7): padding before the fold, and the
+// removal of the zero coordinate rows the padding appended.
+__global__ void k_tail_pad(TailJob *jobs) {
+  TailJob &j = jobs[blockIdx.x];
+  if (threadIdx.x == 0) j.n0 = j.meta[ISKV_META_N];
+  const int64_t words = j.row_bytes / 16;
+  const uint4 *src = static_cast<const uint4 *>(j.src);
+  uint4 *dst = static_cast<uint4 *>(j.dst);
+  for (int64_t e = threadIdx.x; e < (int64_t)j.t8 * words; e += blockDim.x)
+    dst[e] = e < (int64_t)j.t * words ? src[e] : make_uint4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < j.t8; i += blockDim.x)
+    j.dst_pos[i] = j.src_pos[i < j.t ? i : j.t - 1];
+}
+
+__global__ void k_tail_drop(const TailJob *jobs, int count) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  const TailJob &j = jobs[i];
+  // A fold skipped for capacity appended nothing: only a fold that ran leaves rows to drop.
+  if (j.meta[ISKV_META_N] == j.n0 + j.t8) j.meta[ISKV_META_N] -= j.t8 - j.t;
+}
+
+cudaError_t launch_tail_pad(TailJob *jobs, int count, cudaStream_t s) {
+  k_tail_pad<<<count, 256, 0, s>>>(jobs);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tail_drop(const TailJob *jobs, int count, cudaStream_t s) {
+  k_tail_drop<<<(count + 127) / 128, 128, 0, s>>>(jobs, count);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace iskv

@@ -60,6 +60,23 @@ struct WidenArgs {
   int d, r, rw, esz;      // esz: element bytes of U and B (r * esz and rw * esz multiples of 16)
 };
 
+// The last, short block of a prompt compression: t rows copied into a t8-row buffer (t8 = t
+// rounded up to a multiple of 8) followed by zero rows, positions padded with the last real one;
+// after the fold, the t8 - t zero coordinate rows it appended are dropped from the history.
+struct TailJob {
+  const void *src;         // [t][d] rows
+  const int32_t *src_pos;  // [t]
+  void *dst;               // [t8][d] buffer
+  int32_t *dst_pos;        // [t8]
+  int64_t *meta;           // the history's meta word
+  int64_t row_bytes;       // d * element size (a multiple of 16)
+  int64_t n0;              // device-written: the history's n before the fold
+  int32_t t, t8;
+};
+
+cudaError_t launch_tail_pad(TailJob *jobs, int count, cudaStream_t s);
+cudaError_t launch_tail_drop(const TailJob *jobs, int count, cudaStream_t s);
+
 cudaError_t launch_history_widen(const WidenArgs &a, cudaStream_t s);
 cudaError_t launch_history_narrow(const WidenArgs &a, cudaStream_t s);
 
