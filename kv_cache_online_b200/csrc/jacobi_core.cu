@@ -272,7 +272,8 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   // only at second order. The re-orthogonalisation of float32 factors (whose purpose is
   // orthonormal factors to float32 accuracy) accumulates inner products in float64 and uses a
   // tighter tolerance.
-  const float tol = (DD ? 2.f : 4.f) * sqrtf((float)(m > 1 ? m : 1)) * 5.9604645e-08f;
+  const float tol = fmaxf((DD ? 2.f : 4.f) * sqrtf((float)(m > 1 ? m : 1)) * 5.9604645e-08f,
+                          p.tol_floor);
   const float tol2 = tol * tol;
   int sweeps_used = -1;
   int cur = 0;  // which buffer holds the current blocks (double-buffered exchange)
@@ -569,6 +570,7 @@ CoreParams fold_core_params(const FoldParams &p) {
   // where a nearly flat spectrum magnifies any residual cosine over a long trajectory. Two-byte
   // factors round far above that, and keep the float32 sweep.
   c.dd = p.storage == ISKV_F32 ? 1 : 0;
+  c.tol_floor = core_tol_floor(p.storage, false);
   return c;
 }
 

@@ -33,7 +33,21 @@ struct CoreParams {
   size_t Gt, Gtb, Gbot, Ht, sig;  // outputs
   int hs, ldm, max_sweeps;
   int dd;           // 1: inner products accumulated in float64 (tighter tolerance), 0: float32
+  float tol_floor;  // smallest cosine tolerance (see core_tol_floor)
 };
+
+// Floor of the core SVD's cosine tolerance for factors stored as `storage`. The rotations G and H
+// a fold's core returns reach the two-byte factors through that storage's rounding (relative
+// 2^-9 for bf16, 2^-11 for fp16; the tensor-core rotation also takes G as bf16), so column pairs
+// whose cosine is already a sixteenth of it are left alone: the kept singular values move by the
+// square of such a cosine (below 1e-8), the represented rows by less than the storage rounding.
+// The re-orthogonalisation's core exists to make the factors orthonormal again, so its floor is
+// a sixty-fourth of the bf16 rounding and none for fp16 (whose rounding is four times finer).
+// float32 factors keep the float32 tolerance (no floor).
+inline float core_tol_floor(int storage, bool reorth) {
+  if (reorth) return storage == ISKV_BF16 ? 0x1p-15f : 0.f;
+  return storage == ISKV_BF16 ? 0x1p-13f : (storage == ISKV_F16 ? 0x1p-15f : 0.f);
+}
 
 struct JacobiCfg {
   int cj;         // CTAs per cluster

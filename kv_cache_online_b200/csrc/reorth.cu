@@ -428,6 +428,7 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   // Float64 inner products only pay for float32 factors: the bf16 rounding of stored factors
   // (2^-9) is far above the float32 orthogonality the float32-accumulating sweep reaches.
   c.dd = p.storage == ISKV_F32 ? 1 : 0;
+  c.tol_floor = core_tol_floor(p.storage, true);
   e = launch_core(reinterpret_cast<const char *>(jobs), c, s);
   if (e != cudaSuccess) return e;
   k_reorth_T<<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p);
