@@ -187,8 +187,10 @@ __global__ void __launch_bounds__(RES_NTH) k_fold_residual(const FoldJob *jobs, 
     }
     __syncthreads();
     // Float32 inner products carry relative error ~ sqrt(b) 2^-24; the tolerance sits a few units
-    // above it (a residual cosine of that size moves the rho only at second order).
-    const float tol = 4.f * sqrtf((float)b) * 5.9604645e-08f;
+    // above it (a residual cosine of that size moves the rho only at second order). W_R reaches
+    // the stored basis through P, so two-byte factors take the fold core's floor (see
+    // core_tol_floor).
+    const float tol = fmaxf(4.f * sqrtf((float)b) * 5.9604645e-08f, core_tol_floor(p.storage, false));
     const int sw = b <= 16   ? cta_jacobi_columns<1>(Rm, b, b, b, tol, 60)
                    : b <= 32 ? cta_jacobi_columns<2>(Rm, b, b, b, tol, 60)
                    : b <= 64 ? cta_jacobi_columns<4>(Rm, b, b, b, tol, 60)

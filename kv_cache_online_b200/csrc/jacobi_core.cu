@@ -28,14 +28,14 @@ namespace iskv {
 
 // Work counters of the core SVD, per mode (0: fold, 1: re-orthogonalisation), accumulated over
 // every launch until reset: {cores solved, sweeps summed over cores, largest sweep count, pair
-// checks (inner products of a column pair), rotations applied, float32 flops}. The flop count
-// charges 2 m per pair check (one inner product over the m rows of A) and 8 (m + pp) per rotation
-// (two FMAs per element of each of the two columns, V rows included); the per-round norm
+// checks taken (inner products of a column pair), rotations applied, float32 flops}. The flop
+// count charges 2 m per pair check (one inner product over the m rows of A) and 8 (m + pp) per
+// rotation (two FMAs per element of each of the two columns, V rows included); the per-round norm
 // recomputations are not counted.
 static __device__ unsigned long long g_core_stats[2][CORE_STATS];
 
 struct CoreSmem {
-  size_t buf, pairs, where, nP, nQ, nrm_local, anrm, vnrm, nrm_all, flags, total;
+  size_t buf, stamp, pairs, where, nP, nQ, nrm_local, anrm, vnrm, nrm_all, flags, total;
 };
 
 // Shared-memory plan (4-byte words). Column blocks are double-buffered when `dbuf` so a round's
@@ -46,6 +46,7 @@ __host__ __device__ inline CoreSmem core_smem(int cj, int w, int ne, bool dbuf) 
   auto take = [&](size_t words) { size_t at = o; o += words; return at; };
   const int M = 2 * cj;
   s.buf = take((size_t)(dbuf ? 2 : 1) * 2 * w * 32 * ne);
+  s.stamp = take((size_t)(dbuf ? 2 : 1) * 2 * w);
   s.pairs = take((size_t)(M - 1) * cj * 2);
   s.where = take((size_t)(M - 1) * M);
   s.nP = take((size_t)w);
@@ -214,6 +215,8 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   extern __shared__ float smem[];
   float *buf0 = smem + S.buf;
   const int bufw = 2 * w * LP;                  // words per buffer
+  // Per column: 1 + the step at which it was last rotated (0: never), moved with the column.
+  int *stamp0 = reinterpret_cast<int *>(smem + S.stamp);
   int *pairs = reinterpret_cast<int *>(smem + S.pairs);   // [M-1][cj][2]
   int *where = reinterpret_cast<int *>(smem + S.where);   // [M-1][M] = cta * 2 + slot
   float *nP = smem + S.nP, *nQ = smem + S.nQ;
@@ -238,6 +241,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
     where[t * M + bb] = i * 2 + 1;
   }
   if (tid < 4) flags[tid] = 0;
+  for (int e = tid; e < (dbuf ? 2 : 1) * 2 * w; e += blockDim.x) stamp0[e] = 0;
   __syncthreads();
 
   // Build my two blocks for round 0.
@@ -277,11 +281,19 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   const float tol2 = tol * tol;
   int sweeps_used = -1;
   int cur = 0;  // which buffer holds the current blocks (double-buffered exchange)
+  // Every sweep takes the same pairs at the same steps, steps_per_sweep apart. A pair whose two
+  // columns have not been rotated since it was checked one sweep ago would give the same inner
+  // product and again no rotation, so its check is skipped -- when both pairs of a warp are such
+  // pairs (the warp's shuffle reductions stay warp-uniform). The result is unchanged bit for bit;
+  // the late sweeps, where most columns have stopped moving, shrink to their barriers.
+  const int steps_per_sweep = (w - 1) + (M - 1) * w;
+  int gs = 0;  // steps taken so far
   for (int sweep = 0; sweep < p.max_sweeps; ++sweep) {
     unsigned rot = 0;  // rotations this half-warp applied in this sweep
     for (int t = 0; t < M - 1; ++t) {
       float *buf = buf0 + (dbuf ? cur * bufw : 0);
       float *Pb = buf, *Qb = buf + w * LP;
+      int *stP = stamp0 + (dbuf ? cur * 2 * w : 0), *stQ = stP + w;
       // Exact squared norms at the start of the round; tracked through the round's rotations.
       {
         float2 x[NE], y[NE];
@@ -294,21 +306,28 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
       if (t == 0) {
         // Pairs inside each block (both columns from shared memory): half-warp c takes pair
         // c mod w/2 of block c / (w/2).
-        for (int st = 0; st < w - 1; ++st) {
+        for (int st = 0; st < w - 1; ++st, ++gs) {
           const int slot = c < w / 2 ? 0 : 1, q = slot ? c - w / 2 : c;
           const int a = circle_player(q, st, w), bb = circle_player(w - 1 - q, st, w);
           float *base = slot ? Qb : Pb;
           float *nb = slot ? nQ : nP;
-          float2 x[NE], y[NE];
-          col_load<NE>(x, base + a * LP);
-          col_load<NE>(y, base + bb * LP);
-          float ax = nb[a], by = nb[bb];
-          const float g = half_dot<NE, DD>(x, y, nq);
-          if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
-            col_store<NE>(base + a * LP, x);
-            col_store<NE>(base + bb * LP, y);
-            if (l16 == 0) { nb[a] = ax; nb[bb] = by; }
-            ++rot;
+          int *sb = slot ? stQ : stP;
+          const int seen = gs - steps_per_sweep;  // the step that last checked this pair
+          const bool idle = sweep > 0 && sb[a] <= seen && sb[bb] <= seen;
+          if (__all_sync(0xffffffffu, idle)) {
+            if (lane == 0) atomicAdd(reinterpret_cast<unsigned *>(flags + 3), 2u);
+          } else {
+            float2 x[NE], y[NE];
+            col_load<NE>(x, base + a * LP);
+            col_load<NE>(y, base + bb * LP);
+            float ax = nb[a], by = nb[bb];
+            const float g = half_dot<NE, DD>(x, y, nq);
+            if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
+              col_store<NE>(base + a * LP, x);
+              col_store<NE>(base + bb * LP, y);
+              if (l16 == 0) { nb[a] = ax; nb[bb] = by; sb[a] = gs + 1; sb[bb] = gs + 1; }
+              ++rot;
+            }
           }
           __syncthreads();
         }
@@ -317,22 +336,31 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
       float2 x[NE];
       col_load<NE>(x, Pb + c * LP);
       float ax = nP[c];
-      for (int st = 0; st < w; ++st) {
+      int sx = stP[c];
+      for (int st = 0; st < w; ++st, ++gs) {
         int qc = c + st;  // (c + st) mod w, with c, st < w
         if (qc >= w) qc -= w;
-        float2 y[NE];
-        col_load<NE>(y, Qb + qc * LP);
-        float by = nQ[qc];
-        const float g = half_dot<NE, DD>(x, y, nq);
-        if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
-          col_store<NE>(Qb + qc * LP, y);
-          if (l16 == 0) nQ[qc] = by;
-          ++rot;
+        const int seen = gs - steps_per_sweep;
+        const bool idle = sweep > 0 && sx <= seen && stQ[qc] <= seen;
+        if (__all_sync(0xffffffffu, idle)) {
+          if (lane == 0) atomicAdd(reinterpret_cast<unsigned *>(flags + 3), 2u);
+        } else {
+          float2 y[NE];
+          col_load<NE>(y, Qb + qc * LP);
+          float by = nQ[qc];
+          const float g = half_dot<NE, DD>(x, y, nq);
+          if (rotate_regs<NE, DD>(x, y, ax, by, g, tol2)) {
+            col_store<NE>(Qb + qc * LP, y);
+            if (l16 == 0) { nQ[qc] = by; stQ[qc] = gs + 1; }
+            sx = gs + 1;
+            ++rot;
+          }
         }
         __syncthreads();
       }
       if (cj == 1) {
         col_store<NE>(Pb + c * LP, x);
+        if (l16 == 0) stP[c] = sx;
         __syncthreads();
         continue;
       }
@@ -342,13 +370,19 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
       const int d0 = where[tn * M + X0], d1 = where[tn * M + X1];
       float2 y[NE];
       col_load<NE>(y, Qb + c * LP);
+      const int sy = stQ[c];
       float *dst = dbuf ? buf0 + (cur ^ 1) * bufw : buf0;
+      int *sdst = stamp0 + (dbuf ? (cur ^ 1) * 2 * w : 0);
       if (!dbuf) cluster.sync();  // single buffer: everyone has read its blocks before writes
       {
         float *r0 = cluster.map_shared_rank(dst, d0 >> 1) + (d0 & 1) * w * LP;
         float *r1 = cluster.map_shared_rank(dst, d1 >> 1) + (d1 & 1) * w * LP;
         col_store<NE>(r0 + c * LP, x);
         col_store<NE>(r1 + c * LP, y);
+        if (l16 == 0) {
+          cluster.map_shared_rank(sdst, d0 >> 1)[(d0 & 1) * w + c] = sx;
+          cluster.map_shared_rank(sdst, d1 >> 1)[(d1 & 1) * w + c] = sy;
+        }
       }
       cluster.sync();
       if (dbuf) cur ^= 1;
@@ -469,13 +503,19 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
     if (sweeps_used < 0) record_status(jh.meta, ISKV_ERR_NOT_CONVERGED);
   }
   {
-    // Work counters. Every sweep checks each pair of the M w (padded) columns once; the CTA's
-    // rotations were summed in shared memory at the end of each sweep.
+    // Work counters. Every sweep takes each pair of the M w (padded) columns once, less the pair
+    // checks skipped as unchanged (counted per CTA); the CTA's rotations were summed in shared
+    // memory at the end of each sweep. Subtractions go in as two's-complement additions.
     unsigned long long *st = g_core_stats[dense ? 1 : 0];
     const unsigned long long rsum = *reinterpret_cast<const unsigned *>(flags + 2);
+    const unsigned long long skipped = *reinterpret_cast<const unsigned *>(flags + 3);
     if (tid == 0 && rsum) {
       atomicAdd(&st[4], rsum);
       atomicAdd(&st[5], rsum * (8ull * (unsigned)(m + pp)));
+    }
+    if (tid == 0 && skipped) {
+      atomicAdd(&st[3], 0ull - skipped);
+      atomicAdd(&st[5], 0ull - skipped * (2ull * (unsigned)m));
     }
     if (rank == 0 && tid == 0) {
       const unsigned long long sw = sweeps_used < 0 ? (unsigned long long)p.max_sweeps

@@ -44,7 +44,7 @@ struct CoreParams {
 // The re-orthogonalisation's core exists to make the factors orthonormal again, so its floor is
 // a sixty-fourth of the bf16 rounding and none for fp16 (whose rounding is four times finer).
 // float32 factors keep the float32 tolerance (no floor).
-inline float core_tol_floor(int storage, bool reorth) {
+__host__ __device__ inline float core_tol_floor(int storage, bool reorth) {
   if (reorth) return storage == ISKV_BF16 ? 0x1p-15f : 0.f;
   return storage == ISKV_BF16 ? 0x1p-13f : (storage == ISKV_F16 ? 0x1p-15f : 0.f);
 }
