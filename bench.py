@@ -155,7 +155,7 @@ class Workload:
         self.kv, self.torch, self.dev = kv, torch, dev
         # n after the fold of step t is n0 + 64 (t + 1); the timed steps are centred on N_MID.
         self.n0 = N_MID - BLK * (warmup + (timed + 1) // 2)
-        self.n_cap = self.n0 + BLK * (warmup + timed + extra + 2)
+        self.n_cap = self.n0 + BLK * (warmup + timed + extra + 4)
         self.kinds = [kind for _ in range(layers) for kind in ("K", "V")]
         cnt = len(self.kinds)
         self.hists = [kv.LowRankHistory(D, R, self.n_cap, storage=torch.bfloat16, device=dev)
@@ -175,14 +175,16 @@ class Workload:
                                         angle_per_1k=DRIFT_RAD_PER_1K, device=dev)
         self.kept = [torch.empty(self.n_cap, D, dtype=torch.bfloat16, device=dev)
                      for _ in range(2)]
+        self.fpos = torch.arange(PROMPT, PROMPT + self.n_cap + BLK, dtype=torch.int32, device=dev)
         for g in range(self.n0 // BLK):
             F = self.drift.next_blocks().to(torch.bfloat16)
             for i in range(2):
                 self.kept[i][g * BLK:(g + 1) * BLK].copy_(F[i])
             self._fold(g, F)
-        # Pending blocks of every later step (warm-up, timed, end-to-end, one spare).
+        # Pending blocks of every later step (warm-up, timed, end-to-end) and three more for the
+        # cache policy's step (its window rows and its new rows), made before any timing.
         self.F = [self.drift.next_blocks().to(torch.bfloat16)
-                  for _ in range(warmup + timed + extra + 1)]
+                  for _ in range(warmup + timed + extra + 3)]
         self.drift = None  # release the generator's d x d matrices
         # Exact rows per history: 512 prompt rows + 128 window rows.
         gen = torch.Generator(device=dev)
@@ -204,9 +206,8 @@ class Workload:
     def _fold(self, g, F, stream=None):
         """Fold block g (global block index; rows g*64 .. g*64+63 of every stream) and, when the
         cadence says so, re-orthogonalise."""
-        torch, kv = self.torch, self.kv
-        fpos = torch.arange(PROMPT + g * BLK, PROMPT + (g + 1) * BLK, dtype=torch.int32,
-                            device=self.dev)
+        kv = self.kv
+        fpos = self.fpos[g * BLK:(g + 1) * BLK]
         kv.fold_block_batched(self.hists, list(F), [fpos] * len(self.hists),
                               ws=self._aligned(self.ws_fold), stream=stream)
         if (g + 1) % REORTH_EVERY == 0:
@@ -350,16 +351,18 @@ def run_diagnostics(wl, kv, torch, dev, stream):
 
 def time_cache_policy(wl, kv, torch, dev, stream):
     """The cache policy's decode step (Algorithm 3 steps 1-2 and 4-6) on the benchmark's 64 histories:
-    each side's exact-row table holds its 512 protected prompt rows and its 128 window rows (W = 128,
-    b = 64); 63 steps only store the new rows, the 64th folds the oldest 64 rows of every table and
-    removes them from the tables. Run last: it folds one more block into every history."""
+    each side's exact-row table holds its 512 protected prompt rows and its 128 window rows (the next
+    rows of the history's stream; W = 128, b = 64); 63 steps only store the stream's following rows,
+    the 64th folds the oldest 64 rows of every table and removes them from the tables. Run last: it
+    folds one more block into every history."""
     cnt = len(wl.hists)
     tabs = []
     for i, h in enumerate(wl.hists):
         n = int(h.status()[1])
         t = kv.ExactTable(D, PROMPT + WINDOW + BLK, window=WINDOW, block=BLK, reorth_rows=0,
                           dtype=torch.bfloat16, device=dev)
-        t.rows[:PROMPT + WINDOW].copy_(wl.exact[i])
+        t.rows[:PROMPT].copy_(wl.exact[i][:PROMPT])
+        t.rows[PROMPT:PROMPT + WINDOW].copy_(torch.cat([wl.F[-3][i], wl.F[-2][i]]))
         win = torch.arange(PROMPT + n, PROMPT + n + WINDOW, dtype=torch.int32, device=dev)
         t.pos[:PROMPT + WINDOW].copy_(torch.cat([torch.arange(PROMPT, dtype=torch.int32,
                                                               device=dev), win]))
@@ -367,9 +370,8 @@ def time_cache_policy(wl, kv, torch, dev, stream):
             t.live[j] = PROMPT + n + j
         t.t.n_prot, t.t.n_live, t.t.last, t.t.hist_rows = PROMPT, WINDOW, PROMPT + n + WINDOW - 1, n
         tabs.append(t)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(4242)
-    rows = torch.randn(BLK, cnt, D, generator=gen, device=dev).to(torch.bfloat16)
+    # The window holds the next 128 rows of each history's stream; the decode rows follow them.
+    rows = wl.F[-1].transpose(0, 1).contiguous()
     batch = kv.CacheBatch(tabs, wl.hists)
     torch.cuda.synchronize(dev)
     kv.stage_times(reset=True)
