@@ -110,8 +110,10 @@ ISKV_DEV const JobHead &job_head(const char *jobs, int stride, int i) {
 
 // Byte offsets inside one job's fold workspace.
 struct FoldWsLayout {
-  size_t scal, C, E, C2, P, FP, rho, T, W, Y2, Gt, Gtb, Gbot, Ht, sig, Bn, total;
-  int hs;  // row stride (elements) of Ht: r_max + b
+  size_t scal, C, E, C2, P, FP, rho, T, W, Y2, Gt, Gtb, Gbot, Ht, sig, Bn, Pb, Htb, total;
+  int hs;    // row stride (elements) of Ht: r_max + b
+  int bpad;  // P's columns as fp16 (Pb), padded to a multiple of 64
+  int kpad;  // K extent of the tensor-core basis rotation: r_max + bpad (row stride of Htb, fp16)
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -132,11 +134,15 @@ __host__ __device__ inline FoldWsLayout fold_ws_layout(int d, int r, int b) {
   L.W = take(sizeof(float) * (size_t)b * b);
   L.Y2 = take(sizeof(float) * (size_t)b * b);
   L.Gt = take(sizeof(float) * (size_t)r * r);
-  L.Gtb = take(sizeof(__nv_bfloat16) * (size_t)r * r);
+  L.Gtb = take(sizeof(__half) * (size_t)r * r);
   L.Gbot = take(sizeof(float) * (size_t)b * r);
   L.Ht = take(sizeof(float) * (size_t)r * (r + b));
   L.sig = take(sizeof(float) * (size_t)r);
   L.Bn = take(sizeof(float) * (size_t)d * r);
+  L.bpad = (b + 63) / 64 * 64;
+  L.kpad = r + L.bpad;
+  L.Pb = take(sizeof(__half) * (size_t)d * L.bpad);
+  L.Htb = take(sizeof(__half) * (size_t)r * L.kpad);
   L.total = o;
   return L;
 }

@@ -181,6 +181,49 @@ cudaError_t launch_rotate_basis(const char *jobs, const RotParams &p, cudaStream
 }
 
 // ------------------------------------------------------------------------------------------------
+// Operands of the tensor-core basis rotation (bf16 factors): P as fp16 with zero columns from p to
+// bpad, and H^T as fp16 laid out against the K order [B columns 0 .. r-1 | P columns 0 .. bpad-1]: row q
+// (an output column) holds H's entries for B columns l < k at l and for P columns c < p at r + c,
+// zeros elsewhere and in every row q >= k'. B's columns k .. r-1 are cleared (they are zero after
+// every fold and re-orthogonalisation; clearing them keeps a stray non-finite value there from
+// reaching the products through a zero weight).
+__global__ void __launch_bounds__(256) k_basis_prep(const FoldJob *jobs, FoldParams p) {
+  const FoldJob &jb = jobs[blockIdx.y];
+  const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws + p.ws.scal);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], pp = sc[FS_P], kn = sc[FS_K_NEW];
+  const int r = p.r, d = p.d, bpad = p.ws.bpad, kpad = p.ws.kpad, hs = p.ws.hs, pld = p.b;
+  const float *P = reinterpret_cast<const float *>(jb.h.ws + p.ws.P);
+  const float *Ht = reinterpret_cast<const float *>(jb.h.ws + p.ws.Ht);
+  __half *Pb = reinterpret_cast<__half *>(jb.h.ws + p.ws.Pb);
+  __half *Htb = reinterpret_cast<__half *>(jb.h.ws + p.ws.Htb);
+  __nv_bfloat16 *B = static_cast<__nv_bfloat16 *>(jb.h.B);
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x, nth = gridDim.x * blockDim.x;
+  for (int e = tid; e < d * bpad; e += nth) {
+    const int i = e / bpad, c = e % bpad;
+    Pb[e] = __float2half_rn(c < pp ? P[(size_t)i * pld + c] : 0.f);
+  }
+  for (int e = tid; e < r * kpad; e += nth) {
+    const int q = e / kpad, l = e % kpad;
+    float v = 0.f;
+    if (q < kn) {
+      if (l < k) v = Ht[(size_t)q * hs + l];
+      else if (l >= r && l - r < pp) v = Ht[(size_t)q * hs + k + (l - r)];
+    }
+    Htb[e] = __float2half_rn(v);
+  }
+  const int w = r - k;
+  if (w > 0)
+    for (int e = tid; e < d * w; e += nth) B[(size_t)(e / w) * r + k + e % w] = __float2bfloat16_rn(0.f);
+}
+
+cudaError_t launch_basis_prep(const FoldJob *jobs, const FoldParams &p, cudaStream_t s) {
+  k_basis_prep<<<dim3(64, p.count), 256, 0, s>>>(jobs, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------------
 // Coordinate rotation with CUDA cores: U[0:n] <- U[0:n] G[0:k] in place. A CTA owns 32 whole rows:
 // it stages them in shared memory before writing any of them, so no other CTA reads what it
 // overwrites.
@@ -255,7 +298,7 @@ cudaError_t launch_rotate_coords_ffma(const char *jobs, const RotParams &p, int6
 }
 
 // ------------------------------------------------------------------------------------------------
-// Steps 8-9 write-back: B <- Bn, U[n:n+b] <- G[k:], pos[n:n+b] <- f_pos, sigma <- sigma+, meta.
+// Steps 8-9 write-back: B <- Bn (unless B was rotated in place), U[n:n+b] <- G[k:], pos[n:n+b] <- f_pos, sigma <- sigma+, meta.
 template <typename TS>
 __global__ void k_fold_finalize(const FoldJob *jobs, FoldParams p) {
   const FoldJob &jb = jobs[blockIdx.y];
@@ -273,10 +316,11 @@ __global__ void k_fold_finalize(const FoldJob *jobs, FoldParams p) {
   const float *Bn = reinterpret_cast<const float *>(jb.h.ws + p.ws.Bn);
   const float *Gbot = reinterpret_cast<const float *>(jb.h.ws + p.ws.Gbot);
   const float *sig = reinterpret_cast<const float *>(jb.h.ws + p.ws.sig);
-  for (int e = tid; e < d * r; e += nth) {
-    const int q = e % r;
-    store_checked(&B[e], q < kn ? Bn[e] : 0.f, jb.h.meta);
-  }
+  if (!p.tc_basis)  // the tensor-core basis rotation wrote B in place
+    for (int e = tid; e < d * r; e += nth) {
+      const int q = e % r;
+      store_checked(&B[e], q < kn ? Bn[e] : 0.f, jb.h.meta);
+    }
   for (int e = tid; e < b * r; e += nth) {
     const int i = e / r, q = e % r;
     store_checked(&U[(size_t)(n + i) * r + q], q < kn ? Gbot[e] : 0.f, jb.h.meta);

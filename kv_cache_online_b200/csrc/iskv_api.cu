@@ -302,7 +302,7 @@ iskv_status iskv_core_stats(int64_t *out, int32_t reset) {
 size_t iskv_fold_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t b) {
   if (count < 1 || d < 1 || r_max < 1 || b < 1) return 0;
   const FoldWsLayout L = fold_ws_layout(d, r_max, b);
-  return jobs_bytes(count, sizeof(FoldJob)) + tc_table_bytes(count) + (size_t)count * L.total;
+  return jobs_bytes(count, sizeof(FoldJob)) + 2 * tc_table_bytes(count) + (size_t)count * L.total;
 }
 
 iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const void *const *F,
@@ -346,9 +346,12 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   p.count = count;
   p.tau_rel = tau_rel;
   p.ws = fold_ws_layout(d, r, b);
+  p.tc_basis = tc_basis_supported(r, p.ws.bpad, p.storage) ? 1 : 0;
   char *base = static_cast<char *>(ws);
   TcJob *tc_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(FoldJob)));
-  const size_t jb = jobs_bytes(count, sizeof(FoldJob)) + tc_table_bytes(count);
+  TcJob *basis_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(FoldJob)) +
+                                               tc_table_bytes(count));
+  const size_t jb = jobs_bytes(count, sizeof(FoldJob)) + 2 * tc_table_bytes(count);
   std::vector<FoldJob> jobs(count);
   int64_t ncap_max = 0;
   for (int32_t i = 0; i < count; ++i) {
@@ -375,11 +378,23 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
                                hs[i].meta))
         return fail(ISKV_ERR_CUDA, "fold: tensor map encoding failed");
   }
+  std::vector<TcJob> bj;
+  if (p.tc_basis) {
+    bj.resize(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_basis_job(bj[i], hs[i].B, d, r, jobs[i].h.ws + p.ws.Pb, p.ws.bpad,
+                            jobs[i].h.ws + p.ws.Htb,
+                            reinterpret_cast<const int32_t *>(jobs[i].h.ws + p.ws.scal),
+                            hs[i].meta))
+        return fail(ISKV_ERR_CUDA, "fold: tensor map encoding failed");
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   FoldJob *djobs = reinterpret_cast<FoldJob *>(base);
   stage_begin(s);
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(FoldJob) * count, s);
   if (e == cudaSuccess && tc_rot) e = upload_jobs(tc_dev, tj.data(), sizeof(TcJob) * count, s);
+  if (e == cudaSuccess && p.tc_basis)
+    e = upload_jobs(basis_dev, bj.data(), sizeof(TcJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "fold: upload");
   if ((e = launch_fold_prepare(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: prepare");
   stage_mark(s, ST_UPLOAD);
@@ -392,8 +407,13 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
     return cuda_fail(e, "fold: core svd");
   stage_mark(s, ST_FOLD_CORE);
   const RotParams rp = fold_rot_params(p);
-  if ((e = launch_rotate_basis(cj, rp, s)) != cudaSuccess)
-    return cuda_fail(e, "fold: basis rotation");
+  if (p.tc_basis) {
+    e = launch_basis_prep(djobs, p, s);
+    if (e == cudaSuccess) e = launch_tc_basis(basis_dev, count, d, r, p.ws.kpad, s);
+  } else {
+    e = launch_rotate_basis(cj, rp, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "fold: basis rotation");
   stage_mark(s, ST_FOLD_BASIS);
   if (tc_rot) {
     e = launch_tc_rotation(tc_dev, count, r, ncap_max, s);
@@ -421,7 +441,7 @@ iskv_status iskv_fold_block(const iskv_lowrank *h, const void *F, int32_t f_dtyp
 size_t iskv_reorth_workspace_size(int32_t count, int32_t d, int32_t r_max, int64_t n_cap) {
   if (count < 1 || d < 1 || r_max < 1 || n_cap < 0) return 0;
   const ReorthWsLayout L = reorth_ws_layout(d, r_max, n_cap);
-  return jobs_bytes(count, sizeof(ReorthJob)) + 2 * tc_table_bytes(count) + (size_t)count * L.total;
+  return jobs_bytes(count, sizeof(ReorthJob)) + 3 * tc_table_bytes(count) + (size_t)count * L.total;
 }
 
 iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t ws_bytes,
@@ -459,7 +479,9 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   TcJob *tc_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReorthJob)));
   TcJob *gram_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReorthJob)) +
                                               tc_table_bytes(count));
-  const size_t jb = jobs_bytes(count, sizeof(ReorthJob)) + 2 * tc_table_bytes(count);
+  TcJob *basis_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(ReorthJob)) +
+                                               2 * tc_table_bytes(count));
+  const size_t jb = jobs_bytes(count, sizeof(ReorthJob)) + 3 * tc_table_bytes(count);
   std::vector<ReorthJob> jobs(count);
   for (int32_t i = 0; i < count; ++i) {
     ReorthJob &j = jobs[i];
@@ -472,11 +494,21 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
     j.n_cap = hs[i].n_cap;
     j.n_exact = 0;
   }
-  std::vector<TcJob> tj, gj;
+  std::vector<TcJob> tj, gj, bj;
   p.tc_host = nullptr;
   p.tc_dev = tc_dev;
   p.gram_host = nullptr;
   p.gram_dev = gram_dev;
+  p.tc_basis = tc_basis_supported(r, 0, p.storage) ? 1 : 0;
+  p.basis_dev = basis_dev;
+  if (p.tc_basis) {
+    bj.resize(count);
+    for (int32_t i = 0; i < count; ++i)
+      if (!encode_basis_job(bj[i], hs[i].B, d, r, nullptr, 0, jobs[i].h.ws + p.ws.TBtb,
+                            reinterpret_cast<const int32_t *>(jobs[i].h.ws + p.ws.scal),
+                            hs[i].meta))
+        return fail(ISKV_ERR_CUDA, "reorth: tensor map encoding failed");
+  }
   if (tc_gram_supported(r, p.storage)) {
     gj.resize(count);
     for (int32_t i = 0; i < count; ++i)
@@ -501,6 +533,8 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   cudaError_t e = upload_jobs(djobs, jobs.data(), sizeof(ReorthJob) * count, s);
   if (e == cudaSuccess && p.gram_host) e = upload_jobs(gram_dev, gj.data(), sizeof(TcJob) * count, s);
   if (e == cudaSuccess && p.tc_host) e = upload_jobs(tc_dev, tj.data(), sizeof(TcJob) * count, s);
+  if (e == cudaSuccess && p.tc_basis)
+    e = upload_jobs(basis_dev, bj.data(), sizeof(TcJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "reorth: upload");
   stage_mark(s, ST_UPLOAD);
   if ((e = launch_reorth(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "reorth");
@@ -695,6 +729,8 @@ iskv_status iskv_diagnostics(const iskv_lowrank *hs, int32_t count, const int64_
   p.tc_dev = nullptr;
   p.gram_host = nullptr;
   p.gram_dev = gram_dev;
+  p.tc_basis = 0;
+  p.basis_dev = nullptr;
   if (tc_gram_supported(r, p.storage)) {
     gj.resize(count);
     for (int32_t i = 0; i < count; ++i)

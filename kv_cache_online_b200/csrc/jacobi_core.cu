@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
 
   // Outputs for my kept columns: rank q of column j by (norm desc, index asc).
   float *Gt = reinterpret_cast<float *>(jh.ws + p.Gt);
-  __nv_bfloat16 *Gtb = reinterpret_cast<__nv_bfloat16 *>(jh.ws + p.Gtb);
+  __half *Gtb = reinterpret_cast<__half *>(jh.ws + p.Gtb);  // fp16: the tensor-core rotation's type
   float *Gbot = reinterpret_cast<float *>(jh.ws + p.Gbot);
   float *Ht = reinterpret_cast<float *>(jh.ws + p.Ht);
   float *sig = reinterpret_cast<float *>(jh.ws + p.sig);
@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
     for (int l = lane; l < r; l += 32) {
       const float g = l < k ? x[l] * inv : 0.f;
       Gt[(size_t)q * r + l] = g;
-      Gtb[(size_t)q * r + l] = __float2bfloat16_rn(g);
+      Gtb[(size_t)q * r + l] = __float2half_rn(g);
     }
     for (int i = lane; i < b; i += 32) Gbot[(size_t)i * r + q] = x[k + i] * inv;
     for (int l = lane; l < hs; l += 32) {
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(core_max_threads(NE)) k_core(const char *jobs,
   for (int q = kn + rank; q < r; q += cj) {
     for (int l = tid; l < r; l += blockDim.x) {
       Gt[(size_t)q * r + l] = 0.f;
-      Gtb[(size_t)q * r + l] = __float2bfloat16_rn(0.f);
+      Gtb[(size_t)q * r + l] = __float2half_rn(0.f);
     }
     for (int l = tid; l < hs; l += blockDim.x) Ht[(size_t)q * hs + l] = 0.f;
     for (int i = tid; i < b; i += blockDim.x) Gbot[(size_t)i * r + q] = 0.f;

@@ -12,13 +12,14 @@ struct FoldParams {
   int count;            // number of jobs
   float tau_rel;        // residual threshold floor (relative)
   FoldWsLayout ws;      // per-job workspace layout
+  int tc_basis;         // 1: the basis rotation ran on the tensor cores and wrote B in place
 };
 
 // Operands of the two rotations, as byte offsets into each job's workspace. The job's scalars
 // (FS_*) give n, k before, k after, and the residual count p.
 struct RotParams {
   int d, r, storage, count, job_stride;
-  size_t gt, gtb;   // coordinate rotation: row q holds G[0:k, q] (float32 / bf16), row stride r
+  size_t gt, gtb;   // coordinate rotation: row q holds G[0:k, q] (float32 / fp16), row stride r
   size_t ht;        // basis rotation: row q holds H[0:k+p, q], row stride hs
   size_t pmat;      // residual basis P (d x p), row stride pld (unused when p = 0)
   size_t bn;        // basis rotation output (d x r float32)
@@ -67,6 +68,9 @@ cudaError_t launch_fold_prepare(const FoldJob *jobs, const FoldParams &p, cudaSt
 cudaError_t launch_fold_project(const FoldJob *jobs, const FoldParams &p, cudaStream_t s);
 cudaError_t launch_fold_residual(const FoldJob *jobs, const FoldParams &p, cudaStream_t s);
 cudaError_t launch_fold_finalize(const FoldJob *jobs, const FoldParams &p, cudaStream_t s);
+// Operands of the tensor-core basis rotation: P and H as bf16 in the padded layout of
+// FoldWsLayout (Pb, Htb), and B's columns from k on zeroed.
+cudaError_t launch_basis_prep(const FoldJob *jobs, const FoldParams &p, cudaStream_t s);
 
 cudaError_t launch_core(const char *jobs, const CoreParams &p, cudaStream_t s);
 // Core SVD work counters: CORE_STATS values per mode (see jacobi_core.cu), synchronous read.

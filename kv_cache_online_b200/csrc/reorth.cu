@@ -67,8 +67,9 @@ ReorthWsLayout reorth_ws_layout(int d, int r, int64_t n_cap) {
   L.Ht = take(rr);
   L.sig = take(sizeof(float) * r);
   L.TUt = take(rr);
-  L.TUtb = take(sizeof(__nv_bfloat16) * (size_t)r * r);
+  L.TUtb = take(sizeof(__half) * (size_t)r * r);
   L.TBt = take(rr);
+  L.TBtb = take(sizeof(__half) * (size_t)r * r);
   L.Bn = take(sizeof(float) * (size_t)d * r);
   L.total = o;
   return L;
@@ -269,8 +270,28 @@ __global__ void __launch_bounds__(256, 2) k_reorth_T(const ReorthJob *jobs, Reor
   const float *Z = reinterpret_cast<const float *>(jb.h.ws + zo);
   const float *V = reinterpret_cast<const float *>(jb.h.ws + (which == 0 ? p.ws.Gt : p.ws.Ht));
   float *out = reinterpret_cast<float *>(jb.h.ws + (which == 0 ? p.ws.TUt : p.ws.TBt));
-  __nv_bfloat16 *outb = reinterpret_cast<__nv_bfloat16 *>(jb.h.ws + p.ws.TUtb);
+  // fp16 copies (the tensor-core rotations' operand type).
+  __half *outh = reinterpret_cast<__half *>(jb.h.ws + (which == 0 ? p.ws.TUtb : p.ws.TBtb));
   const int m0 = blockIdx.y * GBM, n0 = blockIdx.x * GBN;
+  // Entries outside the leading k x k block are zero: the tensor-core rotations multiply by the
+  // whole r x r matrix.
+  if (k < r)
+    for (int e = threadIdx.x; e < GBM * GBN; e += blockDim.x) {
+      const int q = n0 + e / GBM, l = m0 + e % GBM;
+      if (l < r && q < r && (l >= k || q >= k)) {
+        out[(size_t)q * r + l] = 0.f;
+        outh[(size_t)q * r + l] = __float2half_rn(0.f);
+      }
+    }
+  // B's columns k .. r-1 are cleared before the in-place tensor-core basis rotation (zero after
+  // every fold; clearing keeps a stray non-finite value there out of the products).
+  if (which == 1 && p.tc_basis && k < r) {
+    __nv_bfloat16 *B = static_cast<__nv_bfloat16 *>(jb.h.B);
+    const size_t w = (size_t)(r - k), nth = (size_t)gridDim.x * gridDim.y * blockDim.x;
+    for (size_t e = ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
+         e < (size_t)p.d * w; e += nth)
+      B[(e / w) * r + k + e % w] = __float2bfloat16_rn(0.f);
+  }
   if (m0 >= k || n0 >= k) return;
   tile_gemm<GBM, GBN, GBK, GTM, GTN, true, false>(
       m0, n0, k, k, k, [&](int l, int j) { return Z[(size_t)l * r + j]; },
@@ -278,7 +299,7 @@ __global__ void __launch_bounds__(256, 2) k_reorth_T(const ReorthJob *jobs, Reor
       [&](int l, int q, float acc) {
         const float v = acc * inv;
         out[(size_t)q * r + l] = v;
-        if (which == 0) outb[(size_t)q * r + l] = __float2bfloat16_rn(v);
+        outh[(size_t)q * r + l] = __float2half_rn(v);
       });
 }
 
@@ -292,10 +313,11 @@ __global__ void k_reorth_finalize(const ReorthJob *jobs, ReorthParams p) {
   TS *B = static_cast<TS *>(jb.h.B);
   const float *Bn = reinterpret_cast<const float *>(jb.h.ws + p.ws.Bn);
   const float *sig = reinterpret_cast<const float *>(jb.h.ws + p.ws.sig);
-  for (int e = tid; e < d * r; e += nth) {
-    const int q = e % r;
-    store_checked(&B[e], q < k ? Bn[e] : 0.f, jb.h.meta);
-  }
+  if (!p.tc_basis)  // the tensor-core basis rotation wrote B in place
+    for (int e = tid; e < d * r; e += nth) {
+      const int q = e % r;
+      store_checked(&B[e], q < k ? Bn[e] : 0.f, jb.h.meta);
+    }
   for (int e = tid; e < r; e += nth) jb.h.sigma[e] = e < k ? sig[e] : 0.f;
   if (tid == 0) jb.h.meta[ISKV_META_FOLDS] = 0;
 }
@@ -454,7 +476,10 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
     e = launch_rotate_coords_ffma(reinterpret_cast<const char *>(jobs), q, p.n_cap, s);
   if (e != cudaSuccess) return e;
   stage_mark(s, ST_REORTH_COORDS);
-  e = launch_rotate_basis(reinterpret_cast<const char *>(jobs), q, s);
+  if (p.tc_basis)
+    e = launch_tc_basis(p.basis_dev, p.count, p.d, r, r, s);
+  else
+    e = launch_rotate_basis(reinterpret_cast<const char *>(jobs), q, s);
   if (e != cudaSuccess) return e;
   with_dtype(p.storage, [&](auto ts) {
     k_reorth_finalize<decltype(ts)><<<dim3(32, p.count), 256, 0, s>>>(jobs, p);

@@ -11,7 +11,7 @@ constexpr int NS_ITERS = 5;         // coupled Newton-Schulz iterations
 
 struct ReorthWsLayout {
   size_t scal, gpart_u, gpart_b, G[2], Y[2], Z[2], T[2], Y2[2], Z2[2], M, Gt, Gtb, Ht, sig, TUt,
-      TUtb, TBt, Bn, total;
+      TUtb, TBt, TBtb, Bn, total;
   int nsplit_u, nsplit_b;
 };
 
@@ -25,6 +25,8 @@ struct ReorthParams {
   TcJob *tc_dev;           // their device table
   const TcJob *gram_host;  // tensor-core Gram jobs (host copy) or null
   TcJob *gram_dev;         // their device table
+  int tc_basis;            // 1: B <- B T_B on the tensor cores, in place (jobs in basis_dev)
+  TcJob *basis_dev;
 };
 
 cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStream_t s);

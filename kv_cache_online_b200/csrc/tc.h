@@ -14,9 +14,12 @@ namespace iskv {
 // One tensor-core job: two TMA descriptors plus the pointers its epilogue needs. 64-byte aligned
 // (TMA descriptors must be); lives in the caller's workspace.
 struct alignas(64) TcJob {
-  CUtensorMap mapA;      // U [n_cap][r] bf16, box {64, 128}
-  CUtensorMap mapB;      // rotation: G^T [r][r] bf16, box {64, r}; reconstruction: sigma B [d][r]
-  CUtensorMap mapO;      // reconstruction: out [n_total][d] bf16, box {64, 32} (tile stores)
+  CUtensorMap mapA;      // U [n_cap][r] bf16 (basis rotation: B [d][r]), box {64, 128}
+  CUtensorMap mapB;      // rotation: G^T [r][r] fp16 (basis: H^T [r][kpad]), box {64, r};
+                         // reconstruction: sigma B [d][r]
+  CUtensorMap mapO;      // reconstruction: out [n_total][d] bf16, box {64, 32} (tile stores);
+                         // basis rotation: P [d][bpad] fp16, box {64, 128}
+  CUtensorMap mapS;      // rotations: the output (U or B) bf16, box {64, 32} (tile stores)
   void *U;               // rotation output (in place)
   const int32_t *sc;     // rotation: the job's FS_* scalars
   void *out;             // reconstruction output [n_total][d] bf16
@@ -32,7 +35,10 @@ struct alignas(64) TcJob {
 
 struct TcParams {
   int r, d, n_heads, count, tiles_per_job;
-  int hp, stages;  // reconstruction: heads per CTA, U slab ring depth
+  int hp, stages;  // reconstruction: heads per CTA, U slab ring depth; rotations: A slab ring depth
+  int kslabs;      // rotations: 64-wide K slabs per tile
+  int mode;        // rotations: 0 coordinate (rows n of U), 1 basis (rows d of B)
+  int stg;         // rotations: 1 = each epilogue warp stages 32 x 64 outputs for a tile store
   double theta;
 };
 
@@ -51,6 +57,16 @@ bool encode_gram_job(TcJob &tj, const void *U, int64_t n_cap, const void *B, int
 cudaError_t launch_tc_gram(const TcJob *djobs, const GramParams &p, cudaStream_t s);
 
 bool tc_rotation_supported(int r, int storage);
+
+// Basis rotation of the fold on the tensor cores: B[0:d] <- [B | P] H in place (bf16 factors,
+// fp16 operands), with P (d x bpad) and H^T (r x kpad, kpad = r + bpad) as fp16 in the fold
+// workspace. Job
+// fields: mapA (B, d x r), mapO (Pb, d x bpad), mapB (Htb, r x kpad), U (= B, the output), sc.
+// With bpad = 0 (no mapO) it is the re-orthogonalisation's B <- B T_B.
+bool tc_basis_supported(int r, int bpad, int storage);
+bool encode_basis_job(TcJob &tj, void *B, int d, int r, const void *Pb, int bpad,
+                      const void *Htb, const int32_t *sc, int64_t *meta);
+cudaError_t launch_tc_basis(const TcJob *djobs, int count, int d, int r, int kpad, cudaStream_t s);
 bool tc_recon_supported(int r, int storage, int out_dtype, int head_dim);
 
 bool encode_rotation_job(TcJob &tj, void *U, int64_t n_cap, int r, const void *gtb,

@@ -64,25 +64,63 @@ ISKV_DEV void fail_timeout(Ctl *c, int64_t *meta) {
   if (meta) record_status(meta, ISKV_ERR_TIMEOUT);
 }
 
+// Two bf16 values (low half first) as two fp16 values, each rounded to nearest: exact for
+// magnitudes in fp16's normal range [2^-14, 65504].
+ISKV_DEV uint32_t bf16x2_to_f16x2(uint32_t x) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 // ================================================================================================
-// Coordinate rotation. Job fields: mapA (U), mapB (G^T as bf16, r x r), U, sc (scalars).
-__global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcParams p) {
+// In-place rotations of a factor's rows on the tensor cores (bf16 factors):
+//   mode 0, coordinate rotation (Algorithm 2 step 7; the re-orthogonalisation's U <- U T_U):
+//     U[0:n] <- U[0:n] G, mapA = U, mapB = G^T (r x r);
+//   mode 1, basis rotation (Algorithm 2 step 8; the re-orthogonalisation's B <- B T_B):
+//     B[0:d] <- [B | P] H, mapA = B, mapO = P (d x bpad fp16), mapB = H^T (r x (r + bpad)).
+// The operands are fp16 (11-bit significand): the rotations' entries lie in [-1, 1] and the
+// factors' columns have unit norm, so nothing leaves fp16's range, while bf16 operands (8 bits)
+// would scale every output column by the rounding of its near-one entry: one coherent 2^-9 error
+// per column and rotation, which a trajectory of folds accumulates. A tile is 128 rows; its K
+// slabs 0 .. r/64 - 1 come from mapA as bf16 and are converted to fp16 in shared memory, the
+// rest from mapO as fp16. The rotation's transpose stays resident per history while the A slabs
+// stream through a ring of p.stages 16 KB stages. Warp 0 loads, warp 1 issues the MMAs (M = 128,
+// N = r, accumulators double-buffered in TMEM), warps 2-9 write bf16 rows in place (a tile's rows
+// are read only by that tile), warps 10-13 convert.
+constexpr int ROT_MAX_STAGES = 8;
+constexpr int ROT_THREADS = 448;        // 14 warps
+constexpr int ROT_STG_BYTES = 32 * 128;  // one epilogue warp's staged rows
+
+struct RotCtl {
+  uint64_t a_full[ROT_MAX_STAGES], a_conv[ROT_MAX_STAGES], a_empty[ROT_MAX_STAGES];
+  uint64_t b_full, b_empty;
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t done;
+  uint32_t tmem;
+  int abort;
+};
+
+__global__ void __launch_bounds__(ROT_THREADS, 1) k_rotate_tc(const TcJob *jobs, TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  const int R = p.r, KS = R / 64, N = R;
-  uint8_t *sA = smem;                       // KS slabs x 16 KB
-  uint8_t *sB = smem + KS * SLAB_BYTES;     // KS slabs x (N x 128 B)
-  TcCtl *ctl = reinterpret_cast<TcCtl *>(sB + KS * N * 128);
+  const int R = p.r, KS = p.kslabs, KB = R / 64, N = R, NS = p.stages;
+  uint8_t *sB = smem;                        // KS slabs x (N x 128 B)
+  uint8_t *sA = smem + KS * N * 128;         // NS x 16 KB
+  uint8_t *sStg = sA + NS * SLAB_BYTES;      // p.stg: 8 warps x (32 rows x 128 B), SW128
+  RotCtl *ctl = reinterpret_cast<RotCtl *>(sStg + (p.stg ? 8 * ROT_STG_BYTES : 0));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ncols = N <= 64 ? 128 : (N <= 128 ? 256 : 512);
-  const uint32_t idesc = idesc_bf16_f32(TC_M, N);
+  const uint32_t idesc = idesc_f16_f32(TC_M, N);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 4; ++s) { mbar_init(&ctl->a_full[s], 1); mbar_init(&ctl->a_empty[s], 1); }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&ctl->a_full[s], 1);
+      mbar_init(&ctl->a_conv[s], 4);
+      mbar_init(&ctl->a_empty[s], 1);
+    }
+    mbar_init(&ctl->b_full, 1);
+    mbar_init(&ctl->b_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&ctl->b_full[i], 1);
-      mbar_init(&ctl->b_empty[i], 1);
       mbar_init(&ctl->acc_full[i], 1);
       mbar_init(&ctl->acc_empty[i], 8);
     }
@@ -97,61 +135,101 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
   const uint32_t tmem = ctl->tmem;
   volatile int *abort = &ctl->abort;
   const TileRange tr = my_tiles(p.count, p.tiles_per_job);
-  // Per-thread cache of the current history's scalars: every role tests every tile, and the
+  // Per-thread cache of the current history's row count: every role tests every tile, and the
   // scalars change only with the history, so they are read from global memory once per history.
   int cache_j = -1, cache_n = 0;
   auto rows_of = [&](int j) -> int {
     if (j != cache_j) {
       const int32_t *sc = jobs[j].sc;
       cache_j = j;
-      cache_n = (sc[FS_SKIP] || sc[FS_K_OLD] == 0) ? 0 : sc[FS_N_OLD];
+      cache_n = sc[FS_SKIP] ? 0 : (p.mode ? p.d : (sc[FS_K_OLD] == 0 ? 0 : sc[FS_N_OLD]));
     }
     return cache_n;
   };
 
   if (warp == 0 && lane == 0) {
     // ---------------- producer
-    int cur = -1, nb = 0, na = 0;
-    for (int t = tr.begin; t < tr.end && !*abort; ++t) {
+    int cur = -1, nb = 0;
+    uint32_t gsl = 0;  // A slabs issued so far
+    bool ok = true;
+    for (int t = tr.begin; t < tr.end && ok && !*abort; ++t) {
       const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
       const TcJob &jb = jobs[j];
       if (row0 >= rows_of(j)) continue;
       if (j != cur) {
-        if (nb > 0 && !mbar_wait(&ctl->b_empty[0], (nb - 1) & 1, abort, WAIT_NS)) {
+        if (nb > 0 && !mbar_wait(&ctl->b_empty, (nb - 1) & 1, abort, WAIT_NS)) {
           fail_timeout(ctl, jb.meta);
           break;
         }
         tensormap_acquire(&jb.mapA);
+        if (KS > KB) tensormap_acquire(&jb.mapO);
         tensormap_acquire(&jb.mapB);
-        mbar_arrive_expect_tx(&ctl->b_full[0], KS * N * 128);
-        for (int s = 0; s < KS; ++s) tma_load_2d(sB + s * N * 128, &jb.mapB, s * 64, 0, &ctl->b_full[0]);
+        mbar_arrive_expect_tx(&ctl->b_full, KS * N * 128);
+        for (int s = 0; s < KS; ++s) tma_load_2d(sB + s * N * 128, &jb.mapB, s * 64, 0, &ctl->b_full);
         cur = j;
         ++nb;
       }
-      for (int s = 0; s < KS; ++s) {
-        if (na > 0 && !mbar_wait(&ctl->a_empty[s], (na - 1) & 1, abort, WAIT_NS)) {
+      for (int s = 0; s < KS; ++s, ++gsl) {
+        const uint32_t st = gsl % NS, use = gsl / NS;
+        if (use > 0 && !mbar_wait(&ctl->a_empty[st], (use - 1) & 1, abort, WAIT_NS)) {
           fail_timeout(ctl, jb.meta);
+          ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&ctl->a_full[s], SLAB_BYTES);
-        tma_load_2d(sA + s * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[s]);
+        mbar_arrive_expect_tx(&ctl->a_full[st], SLAB_BYTES);
+        if (s < KB) tma_load_2d(sA + st * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[st]);
+        else tma_load_2d(sA + st * SLAB_BYTES, &jb.mapO, (s - KB) * 64, row0, &ctl->a_full[st]);
       }
-      ++na;
     }
     // Let every load this thread issued land before the CTA can exit.
-    if (na > 0)
-      for (int s = 0; s < KS; ++s) mbar_wait(&ctl->a_full[s], (na - 1) & 1, abort, WAIT_NS / 4);
-    if (nb > 0) mbar_wait(&ctl->b_full[0], (nb - 1) & 1, abort, WAIT_NS / 4);
+    for (uint32_t i = gsl > (uint32_t)NS ? gsl - NS : 0; i < gsl; ++i)
+      mbar_wait(&ctl->a_full[i % NS], (i / NS) & 1, abort, WAIT_NS / 4);
+    if (nb > 0) mbar_wait(&ctl->b_full, (nb - 1) & 1, abort, WAIT_NS / 4);
+  } else if (warp >= 10) {
+    // ---------------- converters: bf16 slabs to fp16 in place (elementwise, so the swizzled
+    // layout is kept); mapO's slabs arrive as fp16.
+    const int ct = threadIdx.x - 10 * 32;  // 0 .. 127
+    uint32_t gsl = 0;
+    for (int t = tr.begin; t < tr.end && !__any_sync(~0u, *abort != 0); ++t) {
+      const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
+      const TcJob &jb = jobs[j];
+      if (row0 >= rows_of(j)) continue;
+      bool ok = true;
+      for (int s = 0; s < KS; ++s, ++gsl) {
+        const uint32_t st = gsl % NS;
+        if (!__all_sync(~0u, mbar_wait(&ctl->a_full[st], (gsl / NS) & 1, abort, WAIT_NS))) {
+          ok = false;
+          break;
+        }
+        if (s < KB) {
+          uint4 *w = reinterpret_cast<uint4 *>(sA + st * SLAB_BYTES);
+#pragma unroll
+          for (int i = 0; i < SLAB_BYTES / 16 / 128; ++i) {
+            uint4 v = w[ct + 128 * i];
+            v.x = bf16x2_to_f16x2(v.x);
+            v.y = bf16x2_to_f16x2(v.y);
+            v.z = bf16x2_to_f16x2(v.z);
+            v.w = bf16x2_to_f16x2(v.w);
+            w[ct + 128 * i] = v;
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->a_conv[st]);
+      }
+      if (!ok) { fail_timeout(ctl, jb.meta); break; }
+    }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     int cur = -1, nb = 0, na = 0;
+    uint32_t gsl = 0;
     for (int t = tr.begin; t < tr.end && !*abort; ++t) {
       const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
       const TcJob &jb = jobs[j];
       if (row0 >= rows_of(j)) continue;
       if (j != cur) {
-        if (cur >= 0) mma_commit(&ctl->b_empty[0]);
-        if (!mbar_wait(&ctl->b_full[0], nb & 1, abort, WAIT_NS)) { fail_timeout(ctl, jb.meta); break; }
+        if (cur >= 0) mma_commit(&ctl->b_empty);
+        if (!mbar_wait(&ctl->b_full, nb & 1, abort, WAIT_NS)) { fail_timeout(ctl, jb.meta); break; }
         cur = j;
         ++nb;
       }
@@ -163,14 +241,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
       fence_after_sync();
       const uint32_t d = tmem + buf * N;
       bool ok = true;
-      for (int s = 0; s < KS && ok; ++s) {
-        if (!mbar_wait(&ctl->a_full[s], na & 1, abort, WAIT_NS)) { ok = false; break; }
+      for (int s = 0; s < KS; ++s, ++gsl) {
+        const uint32_t st = gsl % NS;
+        if (!mbar_wait(&ctl->a_conv[st], (gsl / NS) & 1, abort, WAIT_NS)) {
+          ok = false;
+          break;
+        }
         fence_after_sync();
-        const uint32_t a0 = smem_u32(sA + s * SLAB_BYTES), b0 = smem_u32(sB + s * N * 128);
+        const uint32_t a0 = smem_u32(sA + st * SLAB_BYTES), b0 = smem_u32(sB + s * N * 128);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (s | kk) != 0);
-        mma_commit(&ctl->a_empty[s]);
+        mma_commit(&ctl->a_empty[st]);
       }
       if (!ok) { fail_timeout(ctl, jb.meta); break; }
       mma_commit(&ctl->acc_full[buf]);
@@ -179,10 +261,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
     mma_commit(&ctl->done);
     mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
   } else if (warp >= 2) {
-    // ---------------- epilogue: TMEM -> bf16 -> U rows (in place)
+    // ---------------- epilogue: TMEM -> bf16 -> rows (in place). With p.stg each warp stages
+    // its 32 rows x 64 columns in shared memory (128-byte swizzled) and lane 0 writes them with
+    // one tile store; the last, partial tile of a coordinate rotation keeps per-row stores so
+    // that no row at or beyond n is written.
     const int q = warp & 3, half = (warp - 2) >> 2;
     const int cols = N / 2, c0 = half * cols;
-    int na = 0;
+    uint8_t *stg = sStg + (warp - 2) * ROT_STG_BYTES;
+    bool pending = false;
+    int acq = -1, na = 0;
     // Lanes of a warp take every exit together: tcgen05.ld is a warp-wide instruction.
     for (int t = tr.begin; t < tr.end && !__any_sync(~0u, *abort != 0); ++t) {
       const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
@@ -195,7 +282,48 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
         break;
       }
       fence_after_sync();
-      const int row = row0 + q * 32 + lane;
+      const int rbase = row0 + q * 32, row = rbase + lane;
+      const uint32_t tbase = tmem + buf * N + ((uint32_t)(q * 32) << 16) + c0;
+      if (p.stg && (p.mode || rbase + 32 <= n)) {
+        if (lane == 0 && acq != j) {
+          tensormap_acquire(&jb.mapS);
+          acq = j;
+        }
+        for (int cb = 0; cb < cols; cb += 64) {
+          // The staged rows are free once the previous tile store has read them.
+          if (pending) {
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int cc = 0; cc < 64; cc += 16) {
+            float v[16];
+            tmem_ld16(tbase + cb + cc, v);
+            tmem_ld_wait();
+            uint4 w0, w1;
+            w0.x = pack_bf16(v[0], v[1]);   w0.y = pack_bf16(v[2], v[3]);
+            w0.z = pack_bf16(v[4], v[5]);   w0.w = pack_bf16(v[6], v[7]);
+            w1.x = pack_bf16(v[8], v[9]);   w1.y = pack_bf16(v[10], v[11]);
+            w1.z = pack_bf16(v[12], v[13]); w1.w = pack_bf16(v[14], v[15]);
+            // 16-byte chunk c of a 128-byte staged row sits at chunk c ^ (row & 7).
+            const int ck = cc / 8, sw = lane & 7;
+            *reinterpret_cast<uint4 *>(stg + lane * 128 + 16 * (ck ^ sw)) = w0;
+            *reinterpret_cast<uint4 *>(stg + lane * 128 + 16 * ((ck + 1) ^ sw)) = w1;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&jb.mapS, c0 + cb, rbase, stg);
+            bulk_commit();
+          }
+          pending = true;
+        }
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+        ++na;
+        continue;
+      }
       __nv_bfloat16 *U = static_cast<__nv_bfloat16 *>(jb.U) + (size_t)row * R;
       for (int cc = 0; cc < cols; cc += 16) {
         float v[16];
@@ -217,6 +345,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rot_tc(const TcJob *jobs, TcP
       if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
       ++na;
     }
+    if (lane == 0 && pending) bulk_wait0();
   }
   fence_before_sync();
   __syncthreads();
@@ -874,8 +1003,50 @@ bool tc_recon_supported(int r, int storage, int out_dtype, int head_dim) {
          r >= 64 && r <= 256 && encode_fn() != nullptr;
 }
 
-size_t tc_rot_smem(int r) {
-  return 1024 + (size_t)(r / 64) * SLAB_BYTES + (size_t)(r / 64) * r * 128 + sizeof(TcCtl);
+constexpr size_t kRotSmemCap = 227 * 1024;
+
+// Shared memory of a rotation with `stages` A slabs: the resident transpose (kslabs slabs of
+// r rows x 128 B), the ring, the epilogue's staged rows (stg), the barriers and the 1 KB
+// alignment slack.
+size_t tc_rotate_smem(int r, int kslabs, int stages, int stg) {
+  return 1024 + (size_t)kslabs * r * 128 + (size_t)stages * SLAB_BYTES +
+         (stg ? 8 * ROT_STG_BYTES : 0) + sizeof(RotCtl);
+}
+
+// Ring depth and epilogue form: tile stores (r a multiple of 128, so that a warp's columns are
+// whole 64-column boxes) with at least two ring stages when they fit, else per-row stores; the
+// deepest ring (up to ROT_MAX_STAGES, after the staging) that fits. stages = 0: does not fit.
+void tc_rotate_shape(int r, int kslabs, int &stages, int &stg) {
+  for (stg = (r % 128 == 0) ? 1 : 0; stg >= 0; --stg)
+    for (stages = ROT_MAX_STAGES; stages >= 2; --stages)
+      if (tc_rotate_smem(r, kslabs, stages, stg) <= kRotSmemCap) return;
+  stages = 0;
+  stg = 0;
+}
+
+static cudaError_t launch_rotate(const TcJob *djobs, int count, int r, int d, int kslabs,
+                                 int mode, int tiles_per_job, cudaStream_t s) {
+  TcParams tp;
+  tp.r = r;
+  tp.d = d;
+  tp.n_heads = 0;
+  tp.hp = 0;
+  tp.kslabs = kslabs;
+  tp.mode = mode;
+  tc_rotate_shape(r, kslabs, tp.stages, tp.stg);
+  tp.count = count;
+  tp.tiles_per_job = tiles_per_job;
+  tp.theta = 0.0;
+  if (tp.stages == 0) return cudaErrorInvalidConfiguration;
+  const size_t smem = tc_rotate_smem(r, kslabs, tp.stages, tp.stg);
+  cudaError_t e = cudaFuncSetAttribute(k_rotate_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int total = tp.count * tp.tiles_per_job;
+  const int grid = total < num_sms() ? total : num_sms();
+  k_rotate_tc<<<grid, ROT_THREADS, smem, s>>>(djobs, tp);
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 // Resident basis rows for hp heads, the U slab ring, the output staging rows, the barriers and the
@@ -897,23 +1068,7 @@ void tc_rec_shape(int r, int n_heads, int stg_bytes, int &hp, int &stages) {
 
 cudaError_t launch_tc_rotation(const TcJob *djobs, int count, int r, int64_t n_cap_max,
                                cudaStream_t s) {
-  TcParams tp;
-  tp.r = r;
-  tp.d = 0;
-  tp.n_heads = 0;
-  tp.hp = 0;
-  tp.stages = 0;
-  tp.count = count;
-  tp.tiles_per_job = (int)((n_cap_max + TC_M - 1) / TC_M);
-  tp.theta = 0.0;
-  const size_t smem = tc_rot_smem(r);
-  cudaError_t e = cudaFuncSetAttribute(k_rot_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  const int total = tp.count * tp.tiles_per_job;
-  const int grid = total < num_sms() ? total : num_sms();
-  k_rot_tc<<<grid, TC_THREADS, smem, s>>>(djobs, tp);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_rotate(djobs, count, r, 0, r / 64, 0, (int)((n_cap_max + TC_M - 1) / TC_M), s);
 }
 
 bool encode_rotation_job(TcJob &tj, void *U, int64_t n_cap, int r, const void *gtb,
@@ -921,10 +1076,39 @@ bool encode_rotation_job(TcJob &tj, void *U, int64_t n_cap, int r, const void *g
   std::memset(&tj, 0, sizeof(tj));
   if (!encode_2d(&tj.mapA, U, (uint64_t)n_cap, (uint64_t)r, 128)) return false;
   if (!encode_2d(&tj.mapB, gtb, (uint64_t)r, (uint64_t)r, (uint32_t)r)) return false;
+  if (!encode_2d(&tj.mapS, U, (uint64_t)n_cap, (uint64_t)r, 32)) return false;
   tj.U = U;
   tj.sc = sc;
   tj.meta = meta;
   return true;
+}
+
+static bool basis_fits(int r, int bpad) {
+  int stages, stg;
+  tc_rotate_shape(r, (r + bpad) / 64, stages, stg);
+  return stages > 0;
+}
+
+bool tc_basis_supported(int r, int bpad, int storage) {
+  return storage == ISKV_BF16 && r % 64 == 0 && r >= 64 && r <= 256 && bpad % 64 == 0 &&
+         basis_fits(r, bpad) && encode_fn() != nullptr;
+}
+
+bool encode_basis_job(TcJob &tj, void *B, int d, int r, const void *Pb, int bpad,
+                      const void *Htb, const int32_t *sc, int64_t *meta) {
+  std::memset(&tj, 0, sizeof(tj));
+  if (!encode_2d(&tj.mapA, B, (uint64_t)d, (uint64_t)r, 128)) return false;
+  if (bpad > 0 && !encode_2d(&tj.mapO, Pb, (uint64_t)d, (uint64_t)bpad, 128)) return false;
+  if (!encode_2d(&tj.mapB, Htb, (uint64_t)r, (uint64_t)(r + bpad), (uint32_t)r)) return false;
+  if (!encode_2d(&tj.mapS, B, (uint64_t)d, (uint64_t)r, 32)) return false;
+  tj.U = B;
+  tj.sc = sc;
+  tj.meta = meta;
+  return true;
+}
+
+cudaError_t launch_tc_basis(const TcJob *djobs, int count, int d, int r, int kpad, cudaStream_t s) {
+  return launch_rotate(djobs, count, r, d, kpad / 64, 1, (d + TC_M - 1) / TC_M, s);
 }
 
 bool encode_recon_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void *bsig, int d,

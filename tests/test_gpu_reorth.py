@@ -82,3 +82,39 @@ def test_reorth_partial_rank_after_folds():
     U2, s2, B2, _, (k2, n2, folds, st) = state(h)
     assert (k2, n2, folds, st) == (k, n, 0, 0)
     assert of.rel_fro(of.low_rank_product(U2, s2, B2), of.low_rank_product(U, s, B)) < 1e-4
+
+
+def test_bf16_partial_rank_with_stale_workspace():
+    """A bf16 history of rank k < r_max = 128: the tensor-core rotations of the fold and of the
+    re-orthogonalisation multiply by whole r x (r + b) and r x r operands, so with every workspace
+    filled with NaN bytes before the call, the columns beyond k must come out zero and the factors
+    finite; the represented rows follow the oracle's folds (tau_rel = 1e-2 keeps the rank of the
+    rank-40 rows) and are unchanged by the re-orthogonalisation."""
+    import synth
+    m = kv()
+    d, r, b, n = 256, 128, 64, 512
+    X = stored(synth.lowrank_rows(n, d, 1.0, 0.0, seed=9, rank=40), torch.float32)
+    h = m.LowRankHistory(d, r, n, storage=torch.bfloat16)
+    Xd = torch.as_tensor(X, dtype=torch.float32, device="cuda")
+    wsf = torch.empty(m.fold_workspace_size(1, d, r, b), dtype=torch.uint8, device="cuda")
+    Uo, so, Bo = of.empty_history(d)
+    for i in range(n // b):
+        wsf.fill_(255)
+        m.fold_block(h, Xd[i * b:(i + 1) * b].contiguous(),
+                     torch.arange(i * b, (i + 1) * b, dtype=torch.int32, device="cuda"),
+                     tau_rel=1e-2, ws=wsf)
+        res = of.fold_block(Uo, so, Bo, X[i * b:(i + 1) * b], r, 1e-2)
+        Uo, so, Bo = res.U, res.sigma, res.B
+    U, s, B, _, (k, nn, _, st) = state(h)
+    assert st == 0 and nn == n and k == so.shape[0] and k < r
+    assert bool((h.U[:n, k:] == 0).all()) and bool((h.B[:, k:] == 0).all())
+    assert bool(torch.isfinite(h.U[:n]).all()) and bool(torch.isfinite(h.B).all())
+    assert of.rel_fro(of.low_rank_product(U, s, B), of.low_rank_product(Uo, so, Bo)) < 2e-2
+    wsr = torch.full((m.reorth_workspace_size(1, d, r, n),), 255, dtype=torch.uint8,
+                     device="cuda")
+    m.reorth(h, ws=wsr)
+    U2, s2, B2, _, (k2, n2, folds, st2) = state(h)
+    assert (k2, n2, folds, st2) == (k, n, 0, 0)
+    assert bool((h.U[:n, k:] == 0).all()) and bool((h.B[:, k:] == 0).all())
+    assert bool(torch.isfinite(h.U[:n]).all()) and bool(torch.isfinite(h.B).all())
+    assert of.rel_fro(of.low_rank_product(U2, s2, B2), of.low_rank_product(U, s, B)) < 2e-2
