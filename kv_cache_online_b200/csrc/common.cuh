@@ -110,7 +110,7 @@ ISKV_DEV const JobHead &job_head(const char *jobs, int stride, int i) {
 
 // Byte offsets inside one job's fold workspace.
 struct FoldWsLayout {
-  size_t scal, C, E, C2, P, FP, rho, T, W, Y2, Gt, Gtb, Gbot, Ht, sig, Bn, Pb, Htb, total;
+  size_t scal, C, E, C2, P, FP, rho, T, W, Y2, Gt, Gtb, Gbot, Ht, sig, Bn, Pb, Htb, E1, total;
   int hs;    // row stride (elements) of Ht: r_max + b
   int bpad;  // P's columns as fp16 (Pb), padded to a multiple of 64
   int kpad;  // K extent of the tensor-core basis rotation: r_max + bpad (row stride of Htb, fp16)
@@ -143,6 +143,7 @@ __host__ __device__ inline FoldWsLayout fold_ws_layout(int d, int r, int b) {
   L.kpad = r + L.bpad;
   L.Pb = take(sizeof(__half) * (size_t)d * L.bpad);
   L.Htb = take(sizeof(__half) * (size_t)r * L.kpad);
+  L.E1 = take(sizeof(__nv_bfloat16) * 2 * (size_t)b * d);  // tensor-core projection scratch
   L.total = o;
   return L;
 }

@@ -302,7 +302,7 @@ iskv_status iskv_core_stats(int64_t *out, int32_t reset) {
 size_t iskv_fold_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t b) {
   if (count < 1 || d < 1 || r_max < 1 || b < 1) return 0;
   const FoldWsLayout L = fold_ws_layout(d, r_max, b);
-  return jobs_bytes(count, sizeof(FoldJob)) + 2 * tc_table_bytes(count) + (size_t)count * L.total;
+  return jobs_bytes(count, sizeof(FoldJob)) + 3 * tc_table_bytes(count) + (size_t)count * L.total;
 }
 
 iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const void *const *F,
@@ -351,7 +351,9 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   TcJob *tc_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(FoldJob)));
   TcJob *basis_dev = reinterpret_cast<TcJob *>(base + jobs_bytes(count, sizeof(FoldJob)) +
                                                tc_table_bytes(count));
-  const size_t jb = jobs_bytes(count, sizeof(FoldJob)) + 2 * tc_table_bytes(count);
+  ProjJob *proj_dev = reinterpret_cast<ProjJob *>(base + jobs_bytes(count, sizeof(FoldJob)) +
+                                                  2 * tc_table_bytes(count));
+  const size_t jb = jobs_bytes(count, sizeof(FoldJob)) + 3 * tc_table_bytes(count);
   std::vector<FoldJob> jobs(count);
   int64_t ncap_max = 0;
   for (int32_t i = 0; i < count; ++i) {
@@ -378,6 +380,18 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
                                hs[i].meta))
         return fail(ISKV_ERR_CUDA, "fold: tensor map encoding failed");
   }
+  const bool tc_proj = tc_project_supported(d, r, b, p.storage, f_dtype);
+  std::vector<ProjJob> pj;
+  if (tc_proj) {
+    pj.resize(count);
+    for (int32_t i = 0; i < count; ++i) {
+      char *w = jobs[i].h.ws;
+      if (!encode_project_job(pj[i], hs[i].B, d, r, F[i], b, reinterpret_cast<float *>(w + p.ws.C),
+                              reinterpret_cast<float *>(w + p.ws.E), w + p.ws.E1,
+                              reinterpret_cast<const int32_t *>(w + p.ws.scal), hs[i].meta))
+        return fail(ISKV_ERR_CUDA, "fold: tensor map encoding failed");
+    }
+  }
   std::vector<TcJob> bj;
   if (p.tc_basis) {
     bj.resize(count);
@@ -395,10 +409,12 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   if (e == cudaSuccess && tc_rot) e = upload_jobs(tc_dev, tj.data(), sizeof(TcJob) * count, s);
   if (e == cudaSuccess && p.tc_basis)
     e = upload_jobs(basis_dev, bj.data(), sizeof(TcJob) * count, s);
+  if (e == cudaSuccess && tc_proj) e = upload_jobs(proj_dev, pj.data(), sizeof(ProjJob) * count, s);
   if (e != cudaSuccess) return cuda_fail(e, "fold: upload");
   if ((e = launch_fold_prepare(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: prepare");
   stage_mark(s, ST_UPLOAD);
-  if ((e = launch_fold_project(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: project");
+  e = tc_proj ? launch_tc_project(proj_dev, count, d, r, s) : launch_fold_project(djobs, p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "fold: project");
   stage_mark(s, ST_FOLD_PROJECT);
   if ((e = launch_fold_residual(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: residual");
   stage_mark(s, ST_FOLD_RESIDUAL);

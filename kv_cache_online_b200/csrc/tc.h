@@ -58,6 +58,29 @@ cudaError_t launch_tc_gram(const TcJob *djobs, const GramParams &p, cudaStream_t
 
 bool tc_rotation_supported(int r, int storage);
 
+// Projection of the fold (Algorithm 2 steps 2-3) on the tensor cores: bf16 factors, bf16 block,
+// b = 64, r = 128 or 256, d a multiple of 128 up to 1024; one CTA per history. Outputs C [b][r]
+// and E [b][d] (float32) in the job's fold workspace; E1 [2b][d] bf16 is its scratch.
+struct alignas(64) ProjJob {
+  CUtensorMap mapBm;     // B [d][r] bf16, box {64, 64} (read MN-major: B^T as the A operand)
+  CUtensorMap mapBk;     // B [d][r] bf16, box {64, 128} (read K-major)
+  CUtensorMap mapF;      // F [b][d] bf16, box {64, 64}
+  CUtensorMap mapE1;     // E1 [2b][d] bf16 (hi rows, then lo rows), box {64, 64}
+  __nv_bfloat16 *B;
+  const __nv_bfloat16 *F;
+  float *C, *E;
+  __nv_bfloat16 *E1;
+  const int32_t *sc;     // the job's FS_* scalars
+  int64_t *meta;
+};
+struct ProjParams {
+  int r, d, count;
+};
+bool tc_project_supported(int d, int r, int b, int storage, int f_dtype);
+bool encode_project_job(ProjJob &pj, void *B, int d, int r, const void *F, int b, float *C,
+                        float *E, void *E1, const int32_t *sc, int64_t *meta);
+cudaError_t launch_tc_project(const ProjJob *djobs, int count, int d, int r, cudaStream_t s);
+
 // Basis rotation of the fold on the tensor cores: B[0:d] <- [B | P] H in place (bf16 factors,
 // fp16 operands), with P (d x bpad) and H^T (r x kpad, kpad = r + bpad) as fp16 in the fold
 // workspace. Job

@@ -354,6 +354,272 @@ __global__ void __launch_bounds__(ROT_THREADS, 1) k_rotate_tc(const TcJob *jobs,
 }
 
 // ================================================================================================
+// Projection of the fold (Algorithm 2 steps 2-3) for bf16 factors and a bf16 block F with b = 64:
+// one CTA per history runs four contractions with B, each streaming B from L2 through a ring of
+// 64 KB stages (C^T, C2^T: M = k in 128-row tiles, K = d, B read MN-major; E1, E: M = d in 128-row
+// tiles, K = k, B read K-major; N = b throughout, accumulators in TMEM):
+//   1. C^T  = B^T F^T           F exact in bf16;
+//   2. E1   = F - C B^T         C rounded to bf16 (kept as the MMA operand in shared memory);
+//   3. C2^T = B^T E1^T          E1 as two bf16 terms hi + lo (E1 to about 2^-17);
+//   4. E    = E1 - C2 B^T       C2 rounded to bf16.
+// With B^T B = I, C2 = -(the rounding of C in step 2), so step 4 removes it; what remains in E is
+// the rounding of E1 (2^-17 relative) and of C2 (2^-9 of that rounding), far below the bf16
+// storage of the factors. C (float32, for the core) and E (float32, for the residual QR) go to the
+// workspace; E1's bf16 pair sits in the workspace between steps 2 and 3 (the TMA reads it back).
+constexpr int PROJ_STAGES = 3;
+constexpr int PROJ_STAGE_BYTES = 64 * 1024;
+constexpr int PROJ_B = 64;  // rows of the block
+
+struct ProjCtl {
+  uint64_t full[PROJ_STAGES], empty[PROJ_STAGES];
+  uint64_t pacc;      // steps 1 and 3: accumulators complete
+  uint64_t tacc[8];   // steps 2 and 4: accumulator of d-tile t complete
+  uint64_t c_ready;   // C (step 1) / C2 (step 3) staged as bf16 in shared memory (8 warps)
+  uint64_t e1_ready;  // E1 written to the workspace (8 warps)
+  uint64_t done;
+  uint32_t tmem;
+  int abort;
+};
+
+ISKV_DEV void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(TC_THREADS, 1) k_project_tc(const ProjJob *jobs, ProjParams p) {
+  const ProjJob &jb = jobs[blockIdx.x];
+  if (jb.sc[FS_SKIP]) return;  // uniform over the CTA
+  // The job's pointers, read once: the stores through them could otherwise alias the job table
+  // in the compiler's view and force a reload of each pointer after every store.
+  float *__restrict__ const Cw = jb.C;
+  float *__restrict__ const Ew = jb.E;
+  __nv_bfloat16 *__restrict__ const E1w = jb.E1;
+  const __nv_bfloat16 *__restrict__ const Fr = jb.F;
+  int64_t *const meta = jb.meta;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int R = p.r, D = p.d, KB = R / 64, MH = R / 128, NT = D / 128, ND = D / 64;
+  const int k_old = jb.sc[FS_K_OLD];
+  uint8_t *ring = smem;                                     // PROJ_STAGES x 64 KB
+  uint8_t *sC = smem + PROJ_STAGES * PROJ_STAGE_BYTES;      // KB slabs x (64 rows x 128 B)
+  ProjCtl *ctl = reinterpret_cast<ProjCtl *>(sC + KB * PROJ_B * 128);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tcols = (NT > MH ? NT : MH) * PROJ_B;
+  const uint32_t ncols = tcols <= 32 ? 32 : tcols <= 64 ? 64 : tcols <= 128 ? 128 : tcols <= 256 ? 256 : 512;
+  // bf16 A and B, fp32 D; steps 1/3: A (B^T) MN-major, B operand K-major; steps 2/4: both K-major.
+  const uint32_t idesc_t = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+                           ((uint32_t)(PROJ_B >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+  const uint32_t idesc_n = idesc_bf16_f32(128, PROJ_B);
+
+  // B's columns k_old .. r-1 are cleared (zero after every fold and re-orthogonalisation): the
+  // contractions run over all r columns.
+  if (k_old < R) {
+    __nv_bfloat16 *__restrict__ B = jb.B;
+    const int w = R - k_old;
+    for (int e = threadIdx.x; e < D * w; e += blockDim.x)
+      B[(size_t)(e / w) * R + k_old + e % w] = __float2bfloat16_rn(0.f);
+    fence_proxy_async_global();
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PROJ_STAGES; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    mbar_init(&ctl->pacc, 1);
+    for (int t = 0; t < 8; ++t) mbar_init(&ctl->tacc[t], 1);
+    mbar_init(&ctl->c_ready, 8);
+    mbar_init(&ctl->e1_ready, 8);
+    mbar_init(&ctl->done, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&ctl->tmem, ncols);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int *abort = &ctl->abort;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer: stages of steps 1-4 in order, one ring
+    tensormap_acquire(&jb.mapBm);
+    tensormap_acquire(&jb.mapBk);
+    tensormap_acquire(&jb.mapF);
+    tensormap_acquire(&jb.mapE1);
+    uint32_t g = 0;
+    bool ok = true;
+    for (int step = 0; step < 4 && ok; ++step) {
+      if (step == 2 && !mbar_wait(&ctl->e1_ready, 0, abort, WAIT_NS)) { ok = false; break; }
+      const bool tstep = (step & 1) == 0;  // steps 1 and 3 (K = d)
+      const int n = tstep ? ND : NT;
+      for (int i = 0; i < n; ++i, ++g) {
+        const uint32_t st = g % PROJ_STAGES, use = g / PROJ_STAGES;
+        if (use > 0 && !mbar_wait(&ctl->empty[st], (use - 1) & 1, abort, WAIT_NS)) {
+          ok = false;
+          break;
+        }
+        uint8_t *dst = ring + st * PROJ_STAGE_BYTES;
+        if (tstep) {
+          // B rows [64 i, 64 i + 64) as KB MN-major boxes of 64 columns, then the block's 64
+          // columns [64 i, 64 i + 64): F (step 1) or E1 hi and lo (step 3).
+          const int nb = step == 0 ? 1 : 2;
+          mbar_arrive_expect_tx(&ctl->full[st], KB * 8192 + nb * 8192);
+          for (int sl = 0; sl < KB; ++sl)
+            tma_load_2d(dst + sl * 8192, &jb.mapBm, sl * 64, i * 64, &ctl->full[st]);
+          if (step == 0) {
+            tma_load_2d(dst + 32768, &jb.mapF, i * 64, 0, &ctl->full[st]);
+          } else {
+            tma_load_2d(dst + 32768, &jb.mapE1, i * 64, 0, &ctl->full[st]);
+            tma_load_2d(dst + 40960, &jb.mapE1, i * 64, PROJ_B, &ctl->full[st]);
+          }
+        } else {
+          // B rows [128 i, 128 i + 128) as KB K-major boxes of 64 columns.
+          mbar_arrive_expect_tx(&ctl->full[st], KB * 16384);
+          for (int s = 0; s < KB; ++s)
+            tma_load_2d(dst + s * 16384, &jb.mapBk, s * 64, i * 128, &ctl->full[st]);
+        }
+      }
+    }
+    if (!ok) fail_timeout(ctl, meta);
+    // Let every load this thread issued land before the CTA can exit.
+    for (uint32_t i = g > PROJ_STAGES ? g - PROJ_STAGES : 0; i < g; ++i)
+      mbar_wait(&ctl->full[i % PROJ_STAGES], (i / PROJ_STAGES) & 1, abort, WAIT_NS / 4);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    uint32_t g = 0;
+    bool ok = true;
+    for (int step = 0; step < 4 && ok && !*abort; ++step) {
+      const bool tstep = (step & 1) == 0;
+      // Step 2 needs C staged; step 3 needs TMEM columns of step 2 read out (E1 written);
+      // step 4 needs C2 staged.
+      if (step == 1 && !mbar_wait(&ctl->c_ready, 0, abort, WAIT_NS)) { ok = false; break; }
+      if (step == 2 && !mbar_wait(&ctl->e1_ready, 0, abort, WAIT_NS)) { ok = false; break; }
+      if (step == 3 && !mbar_wait(&ctl->c_ready, 1, abort, WAIT_NS)) { ok = false; break; }
+      fence_after_sync();
+      const int n = tstep ? ND : NT;
+      for (int i = 0; i < n; ++i, ++g) {
+        const uint32_t st = g % PROJ_STAGES;
+        if (!mbar_wait(&ctl->full[st], (g / PROJ_STAGES) & 1, abort, WAIT_NS)) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        const uint32_t base = smem_u32(ring + st * PROJ_STAGE_BYTES);
+        if (tstep) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            for (int h = 0; h < MH; ++h) {
+              const uint64_t adesc = sw128_mn_desc(base + h * 16384 + kk * 2048, 8192);
+              mma_bf16(tmem + h * PROJ_B, adesc, sw128_desc(base + 32768 + kk * 32), idesc_t,
+                       (i | kk) != 0);
+              if (step == 2)
+                mma_bf16(tmem + h * PROJ_B, adesc, sw128_desc(base + 40960 + kk * 32), idesc_t,
+                         true);
+            }
+          }
+        } else {
+          const uint32_t c0 = smem_u32(sC);
+          for (int s = 0; s < KB; ++s)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + i * PROJ_B, sw128_desc(base + s * 16384 + kk * 32),
+                       sw128_desc(c0 + s * 8192 + kk * 32), idesc_n, (s | kk) != 0);
+          mma_commit(&ctl->tacc[i]);
+        }
+        mma_commit(&ctl->empty[st]);
+      }
+      if (ok && tstep) mma_commit(&ctl->pacc);
+    }
+    if (!ok) fail_timeout(ctl, meta);
+    mma_commit(&ctl->done);
+    mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: 8 warps; TMEM lane quarter q = warp & 3
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    const uint32_t lanes = (uint32_t)(q * 32) << 16;
+    bool ok = true;
+    for (int step = 0; step < 4 && ok; ++step) {
+      if ((step & 1) == 0) {
+        // C^T (step 1) or C2^T (step 3) of M-tile `half`: thread = column kc of C.
+        if (half < MH) {
+          ok = __all_sync(~0u, mbar_wait(&ctl->pacc, step >> 1, abort, WAIT_NS));
+          if (!ok) break;
+          fence_after_sync();
+          const int kc = half * 128 + q * 32 + lane;
+          const bool keep = kc < k_old;
+          uint8_t *col = sC + (kc / 64) * 8192 + (kc & 7) * 2;
+          const int ck = (kc & 63) >> 3;
+          for (int c = 0; c < PROJ_B; c += 16) {
+            float v[16];
+            tmem_ld16(tmem + lanes + half * PROJ_B + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const int i = c + u;
+              const float x = keep ? v[u] : 0.f;
+              if (step == 0) Cw[(size_t)i * R + kc] = x;
+              *reinterpret_cast<__nv_bfloat16 *>(col + i * 128 + ((ck ^ (i & 7)) << 4)) =
+                  __float2bfloat16_rn(x);
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->c_ready);
+      } else {
+        // Steps 2 and 4: d-tiles half, half + 2, ...: thread = row dr of B (column of E).
+        for (int t = half; t < NT; t += 2) {
+          ok = __all_sync(~0u, mbar_wait(&ctl->tacc[t], step >> 1, abort, WAIT_NS));
+          if (!ok) break;
+          fence_after_sync();
+          const int dr = t * 128 + q * 32 + lane;
+          // All 64 global loads of the column are issued before any use (one latency per tile).
+          float x[PROJ_B];
+          if (step == 1) {
+#pragma unroll
+            for (int i = 0; i < PROJ_B; ++i) x[i] = __bfloat162float(Fr[(size_t)i * D + dr]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < PROJ_B; ++i) x[i] = Ew[(size_t)i * D + dr];
+          }
+#pragma unroll
+          for (int c = 0; c < PROJ_B; c += 16) {
+            float v[16];
+            tmem_ld16(tmem + lanes + t * PROJ_B + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const size_t at = (size_t)(c + u) * D + dr;
+              const float e = x[c + u] - v[u];
+              Ew[at] = e;
+              if (step == 1) {
+                const __nv_bfloat16 hi = __float2bfloat16_rn(e);
+                E1w[at] = hi;
+                E1w[(size_t)PROJ_B * D + at] = __float2bfloat16_rn(e - __bfloat162float(hi));
+              }
+            }
+          }
+        }
+        if (!ok) break;
+        if (step == 1) {
+          // E1 is read back by the tensor-memory-access unit (the async proxy) in step 3.
+          fence_proxy_async_global();
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->e1_ready);
+        }
+      }
+    }
+    if (!ok) fail_timeout(ctl, meta);
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+// ================================================================================================
 // Reconstruction. Job fields: mapA (U), mapB (sigma-scaled basis, d x r bf16), out, pos, meta.
 //
 // Basis-stationary schedule. Each CTA owns `hp` heads (two when the head count is even) and keeps
@@ -1372,6 +1638,47 @@ cudaError_t launch_tc_gram(const TcJob *djobs, const GramParams &p, cudaStream_t
   e = cudaFuncSetAttribute(k_gram_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_gram_tc<<<p.count * (p.nsu + p.nsb), GRAM_THREADS, smem, s>>>(djobs, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------------
+// Projection of the fold on the tensor cores.
+static_assert(sizeof(ProjJob) <= sizeof(TcJob), "projection jobs use a TcJob-sized table");
+
+bool tc_project_supported(int d, int r, int b, int storage, int f_dtype) {
+  return storage == ISKV_BF16 && f_dtype == ISKV_BF16 && b == PROJ_B && (r == 128 || r == 256) &&
+         d % 128 == 0 && d >= 128 && d <= 1024 && encode_fn() != nullptr;
+}
+
+bool encode_project_job(ProjJob &pj, void *B, int d, int r, const void *F, int b, float *C,
+                        float *E, void *E1, const int32_t *sc, int64_t *meta) {
+  std::memset(&pj, 0, sizeof(pj));
+  if (!encode_2d(&pj.mapBm, B, (uint64_t)d, (uint64_t)r, 64)) return false;
+  if (!encode_2d(&pj.mapBk, B, (uint64_t)d, (uint64_t)r, 128)) return false;
+  if (!encode_2d(&pj.mapF, F, (uint64_t)b, (uint64_t)d, 64)) return false;
+  if (!encode_2d(&pj.mapE1, E1, (uint64_t)(2 * b), (uint64_t)d, 64)) return false;
+  pj.B = static_cast<__nv_bfloat16 *>(B);
+  pj.F = static_cast<const __nv_bfloat16 *>(F);
+  pj.C = C;
+  pj.E = E;
+  pj.E1 = static_cast<__nv_bfloat16 *>(E1);
+  pj.sc = sc;
+  pj.meta = meta;
+  return true;
+}
+
+cudaError_t launch_tc_project(const ProjJob *djobs, int count, int d, int r, cudaStream_t s) {
+  ProjParams pp;
+  pp.r = r;
+  pp.d = d;
+  pp.count = count;
+  const size_t smem = 1024 + (size_t)PROJ_STAGES * PROJ_STAGE_BYTES + (size_t)(r / 64) * PROJ_B * 128 +
+                      sizeof(ProjCtl);
+  cudaError_t e = cudaFuncSetAttribute(k_project_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  k_project_tc<<<count, TC_THREADS, smem, s>>>(djobs, pp);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -84,18 +84,20 @@ def test_reorth_partial_rank_after_folds():
     assert of.rel_fro(of.low_rank_product(U2, s2, B2), of.low_rank_product(U, s, B)) < 1e-4
 
 
-def test_bf16_partial_rank_with_stale_workspace():
-    """A bf16 history of rank k < r_max = 128: the tensor-core rotations of the fold and of the
-    re-orthogonalisation multiply by whole r x (r + b) and r x r operands, so with every workspace
-    filled with NaN bytes before the call, the columns beyond k must come out zero and the factors
-    finite; the represented rows follow the oracle's folds (tau_rel = 1e-2 keeps the rank of the
-    rank-40 rows) and are unchanged by the re-orthogonalisation."""
+@pytest.mark.parametrize("f_dtype", [torch.float32, torch.bfloat16])
+def test_bf16_partial_rank_with_stale_workspace(f_dtype):
+    """A bf16 history of rank k < r_max = 128: the tensor-core projection (bf16 blocks) and
+    rotations of the fold and of the re-orthogonalisation run over all r columns and whole
+    r x (r + b) and r x r operands, so with every workspace filled with NaN bytes before the call,
+    the columns beyond k must come out zero and the factors finite; the represented rows follow
+    the oracle's folds (tau_rel = 1e-2 keeps the rank of the rank-40 rows) and are unchanged by the
+    re-orthogonalisation."""
     import synth
     m = kv()
     d, r, b, n = 256, 128, 64, 512
-    X = stored(synth.lowrank_rows(n, d, 1.0, 0.0, seed=9, rank=40), torch.float32)
+    X = stored(synth.lowrank_rows(n, d, 1.0, 0.0, seed=9, rank=40), f_dtype)
     h = m.LowRankHistory(d, r, n, storage=torch.bfloat16)
-    Xd = torch.as_tensor(X, dtype=torch.float32, device="cuda")
+    Xd = torch.as_tensor(X, dtype=f_dtype, device="cuda")
     wsf = torch.empty(m.fold_workspace_size(1, d, r, b), dtype=torch.uint8, device="cuda")
     Uo, so, Bo = of.empty_history(d)
     for i in range(n // b):
