@@ -629,12 +629,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_project_tc(const ProjJob *job
 // served from L2 to the rest of the group. One MMA of N = hp x 128 covers all of the CTA's heads,
 // so the tensor core reads each A slab once per K step.
 //
-// Output rows go to their positions pos_i. The epilogue stages each head's 128 x 128 bf16 block
-// in shared memory as two 64-column halves in the 128-byte swizzled layout (bank-conflict-free
-// writes); a group of 32 rows whose positions are consecutive -- rows stored in position order,
-// the usual case -- then leaves with two TMA tile stores (32 rows x 64 columns each). Groups with
-// gaps or invalid rows are written from registers.
+// Output rows go to their positions pos_i. Each epilogue warp holds 32 rows and 32 RoPE pairs
+// (columns j and j + 64) of a head; it stages them in shared memory as two 32-column boxes in the
+// 64-byte swizzled layout (bank-conflict-free writes) and, when the 32 rows' positions are
+// consecutive -- rows stored in position order, the usual case -- writes them with two TMA tile
+// stores of its own (no barrier with the warp that holds the other columns). Groups with gaps or
+// invalid rows are written from registers. Tensor memory is released as soon as the unit's last
+// accumulators are in registers, before the staging.
 constexpr int REC_MAX_STAGES = 8;
+// Epilogue warps: two per TMEM lane quarter, 32 RoPE pairs each. (Sixteen warps with 16 pairs
+// each and 32-byte tile stores measured slower.)
+__host__ __device__ constexpr int rec_epilogue_warps(int) { return 8; }
+__host__ __device__ constexpr int rec_threads(int qpk) { return 64 + 32 * rec_epilogue_warps(qpk); }
 constexpr int REC_STG_BYTES = 2 * TC_M * 128;  // lo and hi column halves of one head
 // Attention scores (qpk query heads per KV head): the staging region holds, per warp pair, the
 // query groups of the CTA's (at most two) heads and a 32-row exchange of partial scores.
@@ -683,7 +689,7 @@ struct RecCtl {
 // RoPE'd key row is dotted with the QPK query heads of its KV head and only the scores
 // S[query head][pos] are written; the dense keys never leave the SM.
 template <int QPK>
-__global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcParams p,
+__global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *jobs, TcParams p,
                                                            const __grid_constant__ RopeTab rt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -696,6 +702,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
   RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + rec_stg_bytes(QPK));
   RopeTab *rope_tab = reinterpret_cast<RopeTab *>(ctl + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Epilogue warps: WPQ per TMEM lane quarter, each holding NP of a head's 64 RoPE pairs.
+  constexpr int EPW = rec_epilogue_warps(QPK), WPQ = EPW / 4, NP = 64 / WPQ;
   const int NN = HP * HN;                        // MMA N
   const uint32_t ncols = HP == 2 ? 512 : 256;    // two accumulator buffers of NN columns
   const uint32_t idesc = idesc_bf16_f32(TC_M, NN);
@@ -716,7 +724,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     mbar_init(&ctl->b_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->acc_full[i], 1);
-      mbar_init(&ctl->acc_empty[i], 8);
+      mbar_init(&ctl->acc_empty[i], EPW);
     }
     mbar_init(&ctl->done, 1);
     ctl->abort = 0;
@@ -848,15 +856,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
   } else if (warp >= 2) {
     // ---------------- epilogue: TMEM -> RoPE -> bf16 -> staged rows -> bulk copies to out[pos]
     const int q = warp & 3, half = (warp - 2) >> 2;
-    const int j0 = half * 32;  // this thread's head-local pairs j0 .. j0 + 31 (cols j and j + 64)
+    const int j0 = half * NP;  // this thread's head-local pairs j0 .. j0 + NP - 1 (cols j, j + 64)
     const int srow = q * 32 + lane;
-    uint8_t *stg_lo = sStg + srow * 128, *stg_hi = sStg + TC_M * 128 + srow * 128;
-    const bool issuer = half == 0 && lane == 0;  // issues this lane quarter's tile stores
+    // This warp's staged rows (reconstruction): its 32 rows x NP columns of the lo half and of the
+    // hi half, each a box of 2 NP-byte rows in the matching swizzled layout; lane 0 issues the
+    // warp's tile stores.
+    uint8_t *stg = sStg + (warp - 2) * (2 * 32 * NP * 2);
+    const bool issuer = lane == 0;
+    bool pending = false;  // a tile store of this warp may still be reading the staged rows
     int nc = 0;
-    // The two warps that share rows (q, half 0 and 1) take every decision together through an
-    // AND-reducing named barrier: they meet at named barriers below, and tcgen05.ld is warp-wide.
+    // The warps that share rows (the WPQ warps of lane quarter q) take every decision together
+    // through an AND-reducing named barrier, and tcgen05.ld is warp-wide.
     const int pair_bar = 1 + q;
-    float cs[32], sn[32];
+    constexpr int PB = 32 * WPQ;  // threads at the quarter's barrier
+    float cs[NP], sn[NP];
     // Fields of the history being written, read from global memory once per history rather than
     // once per unit (each read is a dependent global load on the unit's critical path).
     int hj = -1;
@@ -893,7 +906,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
     Cur c = c_first;
     int32_t ps_next = row_pos(c);
     for (;;) {
-      if (!named_and(pair_bar, 64, c.t >= 0 && !*abort)) break;
+      if (!named_and(pair_bar, PB, c.t >= 0 && !*abort)) break;
       const int jj = c.j;
       const int32_t ps_raw = ps_next;
       hist(jj);
@@ -910,10 +923,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       }
       if (rope && valid) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) rope_angle(rope_tab, j0 + i, (uint32_t)ps, cs[i], sn[i]);
-      } else {
+        for (int i = 0; i < NP; ++i) rope_angle(rope_tab, j0 + i, (uint32_t)ps, cs[i], sn[i]);
+      } else if (QPK > 0) {  // the scores apply the (identity) rotation; the rows skip it
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < NP; ++i) {
           cs[i] = 1.f;
           sn[i] = 0.f;
         }
@@ -930,11 +943,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
             qv[((hh * 64 + (f & 63)) * 2 + (f >> 6)) * QPK + g] =
                 qg[(size_t)((member * HP + hh) * QPK + g) * HN + f];
           }
-          named_sync(pair_bar, 64);
+          named_sync(pair_bar, PB);
           q_job = jj;
         }
         const int buf = nc & 1, use = nc >> 1;
-        if (!named_and(pair_bar, 64, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
+        if (!named_and(pair_bar, PB, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
           fail_timeout(ctl, jobs[jj].meta);
           break;
         }
@@ -974,7 +987,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int g = 0; g < QPK; ++g) xch[(lane * 2 + h) * QPK + g] = acc[h][g];
-        named_sync(pair_bar, 64);
+        named_sync(pair_bar, PB);
         if (half == 0 && valid) {
 #pragma unroll
           for (int h = 0; h < 2; ++h)
@@ -1000,7 +1013,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
         acq_j = jj;
       }
       const int buf = nc & 1, use = nc >> 1;
-      if (!named_and(pair_bar, 64, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
+      if (!named_and(pair_bar, PB, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
         fail_timeout(ctl, jb.meta);
         break;
       }
@@ -1009,59 +1022,78 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcP
       for (int h = 0; h < HP; ++h) {
         // The head's 32 RoPE pairs go to packed registers first, so the TMEM loads and the math
         // overlap the previous tile stores still reading the staged rows.
-        uint32_t wl[16], wh[16];
+        uint32_t wl[NP / 2], wh[NP / 2];
 #pragma unroll
-        for (int jb16 = 0; jb16 < 32; jb16 += 16) {
+        for (int jb16 = 0; jb16 < NP; jb16 += 16) {
           float lo[16], hi[16];
           tmem_ld16(base + h * HN + j0 + jb16, lo);
           tmem_ld16(base + h * HN + 64 + j0 + jb16, hi);
           tmem_ld_wait();
+          if (rope) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const float c0 = cs[jb16 + i], s0 = sn[jb16 + i];
-            const float c1 = cs[jb16 + i + 1], s1 = sn[jb16 + i + 1];
-            wl[(jb16 + i) / 2] = pack_bf16(lo[i] * c0 - hi[i] * s0, lo[i + 1] * c1 - hi[i + 1] * s1);
-            wh[(jb16 + i) / 2] = pack_bf16(hi[i] * c0 + lo[i] * s0, hi[i + 1] * c1 + lo[i + 1] * s1);
+            for (int i = 0; i < 16; i += 2) {
+              const float c0 = cs[jb16 + i], s0 = sn[jb16 + i];
+              const float c1 = cs[jb16 + i + 1], s1 = sn[jb16 + i + 1];
+              wl[(jb16 + i) / 2] =
+                  pack_bf16(lo[i] * c0 - hi[i] * s0, lo[i + 1] * c1 - hi[i + 1] * s1);
+              wh[(jb16 + i) / 2] =
+                  pack_bf16(hi[i] * c0 + lo[i] * s0, hi[i + 1] * c1 + lo[i + 1] * s1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              wl[(jb16 + i) / 2] = pack_bf16(lo[i], lo[i + 1]);
+              wh[(jb16 + i) / 2] = pack_bf16(hi[i], hi[i + 1]);
+            }
           }
         }
+        if (h == HP - 1) {
+          // Every accumulator of the unit is in registers: tensor memory can take the next unit
+          // while this warp stages and stores.
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+        }
         if (tiles) {
-          // The staged rows are free once the previous tile stores out of them have been read.
-          if (issuer) bulk_wait_read0();
-          named_sync(pair_bar, 64);
-          // 16-byte chunk c of a 128-byte staged row sits at chunk c ^ (row & 7).
-          const int ck = j0 / 8, sw = srow & 7;
+          // The staged rows are free once this warp's previous tile stores have read them.
+          if (pending) {
+            if (issuer) bulk_wait_read0();
+            __syncwarp();
+          }
+          // Row = lane, 64-byte staged rows: 16-byte chunk u sits at chunk u ^ ((row >> 1) & 3)
+          // (the 64-byte swizzle: address bits 7-8 into bits 4-5).
+          static_assert(QPK > 0 || NP == 32, "staging is laid out for 32 pairs per warp");
+          const int sw = (lane >> 1) & 3;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            *reinterpret_cast<uint4 *>(stg_lo + 16 * ((ck + u) ^ sw)) =
+            *reinterpret_cast<uint4 *>(stg + lane * 64 + 16 * (u ^ sw)) =
                 make_uint4(wl[4 * u], wl[4 * u + 1], wl[4 * u + 2], wl[4 * u + 3]);
-            *reinterpret_cast<uint4 *>(stg_hi + 16 * ((ck + u) ^ sw)) =
+            *reinterpret_cast<uint4 *>(stg + 2048 + lane * 64 + 16 * (u ^ sw)) =
                 make_uint4(wh[4 * u], wh[4 * u + 1], wh[4 * u + 2], wh[4 * u + 3]);
           }
           fence_proxy_async_smem();
-          named_sync(pair_bar, 64);
+          __syncwarp();
           if (issuer) {
-            const int x = (member * HP + h) * HN;
-            tma_store_2d(&jb.mapO, x, (int)first, sStg + q * 32 * 128);
-            tma_store_2d(&jb.mapO, x + 64, (int)first, sStg + TC_M * 128 + q * 32 * 128);
+            const int x = (member * HP + h) * HN + j0;
+            tma_store_2d(&jb.mapO, x, (int)first, stg);
+            tma_store_2d(&jb.mapO, x + 64, (int)first, stg + 2048);
             bulk_commit();
           }
+          pending = true;
         } else if (valid) {
           uint4 *dl = reinterpret_cast<uint4 *>(orow + h * HN + j0);
           uint4 *dh = reinterpret_cast<uint4 *>(orow + h * HN + 64 + j0);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < NP / 8; ++u) {
             dl[u] = make_uint4(wl[4 * u], wl[4 * u + 1], wl[4 * u + 2], wl[4 * u + 3]);
             dh[u] = make_uint4(wh[4 * u], wh[4 * u + 1], wh[4 * u + 2], wh[4 * u + 3]);
           }
         }
       }
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
       ++nc;
       c = cn;
     }
-    if (issuer) bulk_wait0();
+    if (issuer && pending) bulk_wait0();
   }
   fence_before_sync();
   __syncthreads();
@@ -1234,17 +1266,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 row-major matrix [rows][cols], box {64 cols, box_rows}, 128-byte swizzle.
-bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2-D two-byte row-major matrix [rows][cols], box {box_cols, box_rows} (box_cols x 2 bytes no
+// wider than the swizzle span), 128-byte swizzle unless given.
+bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+               uint32_t box_cols = 64, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int num_sms() {
@@ -1383,7 +1417,9 @@ bool encode_recon_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void
   if (!encode_2d(&tj.mapA, U, (uint64_t)n_cap, (uint64_t)r, 128)) return false;
   if (!encode_2d(&tj.mapB, bsig, (uint64_t)d, (uint64_t)r, 128)) return false;
   tj.tiles_ok = n_total >= 32;
-  if (tj.tiles_ok && !encode_2d(&tj.mapO, out, (uint64_t)n_total, (uint64_t)d, 32)) return false;
+  if (tj.tiles_ok && !encode_2d(&tj.mapO, out, (uint64_t)n_total, (uint64_t)d, 32, 32,
+                                CU_TENSOR_MAP_SWIZZLE_64B))
+    return false;
   tj.out = out;
   tj.pos = pos;
   tj.meta = meta;
@@ -1417,7 +1453,7 @@ cudaError_t launch_tc_recon(const TcJob *djobs, const ReconParams &p, cudaStream
   int groups = num_sms() / G;
   if (groups < 1) groups = 1;
   if (groups > total) groups = total;
-  k_rec_tc<0><<<groups * G, TC_THREADS, smem, s>>>(djobs, tp, make_rope_tab(p.theta));
+  k_rec_tc<0><<<groups * G, rec_threads(0), smem, s>>>(djobs, tp, make_rope_tab(p.theta));
   count_launches(1);
   return cudaGetLastError();
 }
@@ -1456,7 +1492,7 @@ static cudaError_t attn_scores_qpk(const TcJob *djobs, const TcParams &tp, int G
   int groups = num_sms() / G;
   if (groups < 1) groups = 1;
   if (groups > total) groups = total;
-  k_rec_tc<QPK><<<groups * G, TC_THREADS, smem, s>>>(djobs, tp, make_rope_tab(tp.theta));
+  k_rec_tc<QPK><<<groups * G, rec_threads(QPK), smem, s>>>(djobs, tp, make_rope_tab(tp.theta));
   count_launches(1);
   return cudaGetLastError();
 }
