@@ -514,6 +514,7 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
   p.tc_host = nullptr;
   p.tc_dev = tc_dev;
   p.gram_host = nullptr;
+  p.gram_nsu = 0;
   p.gram_dev = gram_dev;
   p.tc_basis = tc_basis_supported(r, 0, p.storage) ? 1 : 0;
   p.basis_dev = basis_dev;
@@ -533,6 +534,9 @@ iskv_status iskv_reorth(const iskv_lowrank *hs, int32_t count, void *ws, size_t 
                            jobs[i].h.ws))
         return fail(ISKV_ERR_CUDA, "reorth: tensor map encoding failed");
     p.gram_host = gj.data();
+    // U chunks per job: about one chunk per SM over all jobs (the B chunks are short).
+    int nsu = tc_sm_count() / count;
+    p.gram_nsu = nsu < 1 ? 1 : (nsu > p.ws.nsplit_u ? p.ws.nsplit_u : nsu);
   }
   if (tc_rotation_supported(r, p.storage)) {
     tj.resize(count);
@@ -744,6 +748,7 @@ iskv_status iskv_diagnostics(const iskv_lowrank *hs, int32_t count, const int64_
   p.tc_host = nullptr;
   p.tc_dev = nullptr;
   p.gram_host = nullptr;
+  p.gram_nsu = 0;
   p.gram_dev = gram_dev;
   p.tc_basis = 0;
   p.basis_dev = nullptr;
@@ -755,6 +760,9 @@ iskv_status iskv_diagnostics(const iskv_lowrank *hs, int32_t count, const int64_
                            jobs[i].h.ws))
         return fail(ISKV_ERR_CUDA, "%s: tensor map encoding failed", who);
     p.gram_host = gj.data();
+    // U chunks per job: about one chunk per SM over all jobs (the B chunks are short).
+    int nsu = tc_sm_count() / count;
+    p.gram_nsu = nsu < 1 ? 1 : (nsu > p.ws.nsplit_u ? p.ws.nsplit_u : nsu);
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ReorthJob *djobs = reinterpret_cast<ReorthJob *>(base);

@@ -118,23 +118,35 @@ __global__ void __launch_bounds__(256) k_gram_partial(const ReorthJob *jobs, Reo
       [&](int m, int n, float acc) { G[(size_t)m * r + n] = acc; });
 }
 
-// Sum the partials; then the scale c = trace / k and the Newton-Schulz start Y = G / c, Z = I.
-__global__ void k_gram_reduce(const ReorthJob *jobs, ReorthParams p) {
+// Sum the partials into G (the whole r x r matrix: entries beyond k are zero in every partial,
+// since the factors' columns beyond k are), four floats per thread.
+__global__ void __launch_bounds__(256) k_gram_reduce(const ReorthJob *jobs, ReorthParams p) {
   const int job = blockIdx.y >> 1, which = blockIdx.y & 1;
   const ReorthJob &jb = jobs[job];
   const int32_t *sc = reinterpret_cast<const int32_t *>(jb.h.ws);
   if (sc[FS_SKIP]) return;
-  const int k = sc[FS_K_OLD], r = p.r;
+  // The tensor-core Gram writes a single B chunk's matrix to G itself.
+  if (which == 1 && p.gram_nsu > 0 && p.ws.nsplit_b == 1) return;
+  const int r = p.r;
   const int rows = which == 0 ? sc[FS_N_OLD] : p.d;
-  const int ns = min(which == 0 ? p.ws.nsplit_u : p.ws.nsplit_b,
-                     (rows + REORTH_SPLIT - 1) / REORTH_SPLIT);  // splits that hold rows
-  const float *part = reinterpret_cast<const float *>(jb.h.ws + (which == 0 ? p.ws.gpart_u : p.ws.gpart_b));
-  float *G = reinterpret_cast<float *>(jb.h.ws + p.ws.G[which]);
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < k * k; e += gridDim.x * blockDim.x) {
-    const int i = e / k, j = e % k;
-    float s = 0.f;
-    for (int q = 0; q < ns; ++q) s += part[(size_t)q * r * r + (size_t)i * r + j];
-    G[(size_t)i * r + j] = s;
+  // Splits that hold rows: REORTH_SPLIT-row splits, or the tensor-core Gram's balanced U chunks.
+  const bool bal = which == 0 && p.gram_nsu > 0;
+  const int chunk = bal ? gram_chunk(rows, p.gram_nsu) : REORTH_SPLIT;
+  const int ns = min(bal ? p.gram_nsu : (which == 0 ? p.ws.nsplit_u : p.ws.nsplit_b),
+                     (rows + chunk - 1) / chunk);
+  const float4 *part = reinterpret_cast<const float4 *>(jb.h.ws + (which == 0 ? p.ws.gpart_u : p.ws.gpart_b));
+  float4 *G = reinterpret_cast<float4 *>(jb.h.ws + p.ws.G[which]);
+  const int n4 = r * r / 4;  // r is a multiple of 4 on every path that reaches here
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += gridDim.x * blockDim.x) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < ns; ++q) {
+      const float4 v = part[(size_t)q * n4 + e];
+      a.x += v.x;
+      a.y += v.y;
+      a.z += v.z;
+      a.w += v.w;
+    }
+    G[e] = a;
   }
 }
 
@@ -333,11 +345,12 @@ static cudaError_t reorth_gram(const ReorthJob *jobs, const ReorthParams &p, cud
     gp.r = r;
     gp.d = p.d;
     gp.count = p.count;
-    gp.nsu = W.nsplit_u;
+    gp.nsu = p.gram_nsu;
     gp.nsb = W.nsplit_b;
     gp.split = REORTH_SPLIT;
     gp.off_gu = W.gpart_u;
     gp.off_gb = W.gpart_b;
+    gp.off_g1 = W.G[1];
     cudaError_t e0 = launch_tc_gram(p.gram_dev, gp, s);
     if (e0 != cudaSuccess) return e0;
   } else {

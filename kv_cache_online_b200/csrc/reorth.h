@@ -25,6 +25,7 @@ struct ReorthParams {
   TcJob *tc_dev;           // their device table
   const TcJob *gram_host;  // tensor-core Gram jobs (host copy) or null
   TcJob *gram_dev;         // their device table
+  int gram_nsu;            // tensor-core Gram: U chunks per job (balanced); 0: REORTH_SPLIT rows
   int tc_basis;            // 1: B <- B T_B on the tensor cores, in place (jobs in basis_dev)
   TcJob *basis_dev;
 };

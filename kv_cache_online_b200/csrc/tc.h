@@ -46,11 +46,22 @@ struct TcParams {
 // splits of B rows (`split` rows each); outputs at byte offsets off_gu / off_gb of the job's
 // workspace (TcJob::out), one r x r float32 matrix per split.
 struct GramParams {
-  int r, d, count, nsu, nsb, split;
+  int r, d, count;
+  int nsu;    // U chunks per job: n rows in gram_chunk(n, nsu)-row chunks
+  int nsb;    // B chunks per job of `split` rows
+  int split;
   size_t off_gu, off_gb;
+  size_t off_g1;  // with nsb == 1: B's Gram goes straight to this workspace offset (no partial)
 };
 
+// Rows per U chunk when n rows are split into nsu balanced chunks (whole 64-row stages).
+__host__ __device__ inline int gram_chunk(int n, int nsu) {
+  const int c = (n + nsu - 1) / nsu;
+  return c < 64 ? 64 : (c + 63) / 64 * 64;
+}
+
 bool tc_gram_supported(int r, int storage);
+int tc_sm_count();  // SMs of the current device
 bool encode_gram_job(TcJob &tj, const void *U, int64_t n_cap, const void *B, int d, int r,
                      const int32_t *sc, int64_t *meta, void *ws);
 // The launchers take job tables already uploaded to the device (upload_jobs).

@@ -1109,18 +1109,37 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
 // N = r accumulators in tensor memory); a second kernel sums the partials.
 constexpr int GRAM_THREADS = 192;  // producer warp, MMA warp, 4 epilogue warps
 constexpr int GRAM_STAGES = 4;
+constexpr int GRAM_RING = 6;       // stages of the Gram kernel's ring
 constexpr int GRAM_KT = 64;        // rows per pipeline stage
 
+// Shared memory before the barriers: the stage ring, or the staged 128-row half of a partial
+// (rows padded to r + 4 floats), whichever is larger.
+__host__ __device__ inline int gram_area_bytes(int r) {
+  const int ring = GRAM_RING * (r / 64) * GRAM_KT * 128, stg = 128 * (r + 4) * 4;
+  return ring > stg ? ring : stg;
+}
+
 __global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, GramParams p) {
-  const int per_job = p.nsu + p.nsb;
-  const int job = blockIdx.x / per_job, rem = blockIdx.x % per_job;
-  const int which = rem < p.nsu ? 0 : 1, split = which ? rem - p.nsu : rem;
+  // The U chunks of every job come first (they are the long ones), then the B chunks.
+  const int nU = p.count * p.nsu;
+  int job, which, split;
+  if ((int)blockIdx.x < nU) {
+    job = blockIdx.x / p.nsu;
+    which = 0;
+    split = blockIdx.x % p.nsu;
+  } else {
+    const int b = blockIdx.x - nU;
+    job = b / p.nsb;
+    which = 1;
+    split = b % p.nsb;
+  }
   const TcJob &jb = jobs[job];
   const int32_t *sc = jb.sc;
   const int R = p.r, SL = R / 64, MH = R / 128, N = R;
   const int rows_total = which ? p.d : sc[FS_N_OLD];
-  const int r0 = split * p.split;
-  const int nrows = min(p.split, rows_total - r0);
+  const int chunk = which ? p.split : gram_chunk(rows_total, p.nsu);
+  const int r0 = split * chunk;
+  const int nrows = min(chunk, rows_total - r0);
   if (sc[FS_SKIP] || nrows <= 0 || sc[FS_K_OLD] == 0) return;  // uniform over the CTA
   const int nk = (nrows + GRAM_KT - 1) / GRAM_KT;
   const CUtensorMap *map = which ? &jb.mapB : &jb.mapA;
@@ -1129,14 +1148,14 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   const int STAGE_BYTES = SL * GRAM_KT * 128;
-  TcCtl *ctl = reinterpret_cast<TcCtl *>(smem + GRAM_STAGES * STAGE_BYTES);
-  uint64_t *full = reinterpret_cast<uint64_t *>(ctl + 1);   // [GRAM_STAGES]
-  uint64_t *empty = full + GRAM_STAGES;                      // [GRAM_STAGES]
+  TcCtl *ctl = reinterpret_cast<TcCtl *>(smem + gram_area_bytes(R));
+  uint64_t *full = reinterpret_cast<uint64_t *>(ctl + 1);   // [GRAM_RING]
+  uint64_t *empty = full + GRAM_RING;                      // [GRAM_RING]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ncols = MH * N <= 128 ? 128 : (MH * N <= 256 ? 256 : 512);
   const uint32_t idesc = idesc_bf16_f32_mn(128, N);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < GRAM_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < GRAM_RING; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(&ctl->acc_full[0], 1);
     mbar_init(&ctl->done, 1);
     ctl->abort = 0;
@@ -1152,7 +1171,7 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, 
   if (warp == 0 && lane == 0) {
     tensormap_acquire(map);
     for (int kt = 0; kt < nk && !*abort; ++kt) {
-      const int st = kt % GRAM_STAGES, use = kt / GRAM_STAGES;
+      const int st = kt % GRAM_RING, use = kt / GRAM_RING;
       if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, abort, WAIT_NS)) {
         fail_timeout(ctl, jb.meta);
         break;
@@ -1162,12 +1181,12 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, 
         tma_load_2d(smem + st * STAGE_BYTES + sl * GRAM_KT * 128, map, sl * 64, r0 + kt * GRAM_KT,
                     &full[st]);
     }
-    for (int k = 1; k <= GRAM_STAGES && nk - k >= 0; ++k)
-      mbar_wait(&full[(nk - k) % GRAM_STAGES], ((nk - k) / GRAM_STAGES) & 1, abort, WAIT_NS / 4);
+    for (int k = 1; k <= GRAM_RING && nk - k >= 0; ++k)
+      mbar_wait(&full[(nk - k) % GRAM_RING], ((nk - k) / GRAM_RING) & 1, abort, WAIT_NS / 4);
   } else if (warp == 1 && lane == 0) {
     bool ok = true;
     for (int kt = 0; kt < nk && ok && !*abort; ++kt) {
-      const int st = kt % GRAM_STAGES, use = kt / GRAM_STAGES;
+      const int st = kt % GRAM_RING, use = kt / GRAM_RING;
       if (!mbar_wait(&full[st], use & 1, abort, WAIT_NS)) { ok = false; break; }
       fence_after_sync();
       const uint32_t base = smem_u32(smem + st * STAGE_BYTES);
@@ -1187,26 +1206,43 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, 
     mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
   } else if (warp >= 2) {
     const int q = warp & 3;
+    // A job's single B chunk writes its Gram matrix itself; U chunks write partials.
     float *out = reinterpret_cast<float *>(jb.out) +
-                 (which ? p.off_gb : p.off_gu) / sizeof(float) + (size_t)split * R * R;
-    // One decision per warp: tcgen05.ld is a warp-wide instruction.
-    if (__all_sync(~0u, mbar_wait(&ctl->acc_full[0], 0, abort, WAIT_NS) && !*abort)) {
-      fence_after_sync();
-      for (int h = 0; h < MH; ++h) {
-        const int row = h * 128 + q * 32 + lane;
+                 (which ? (p.nsb == 1 ? p.off_g1 : p.off_gb) : p.off_gu) / sizeof(float) +
+                 (size_t)split * R * R;
+    // Once the accumulators are complete, the stage buffers are idle: each 128-row half of the
+    // partial is staged there (rows of R + 4 floats, so that the 32 rows a warp writes at once
+    // fall in distinct banks) and leaves in whole coalesced rows.
+    float *stg = reinterpret_cast<float *>(smem);
+    const int LDS = R + 4;
+    // One decision per warp: tcgen05.ld is a warp-wide instruction; the four epilogue warps meet
+    // at named barrier 1 whatever they decided.
+    const bool ok = __all_sync(~0u, mbar_wait(&ctl->acc_full[0], 0, abort, WAIT_NS) && !*abort);
+    if (!ok) fail_timeout(ctl, jb.meta);
+    fence_after_sync();
+    for (int h = 0; h < MH; ++h) {
+      if (ok) {
+        float *srow = stg + (size_t)(q * 32 + lane) * LDS;
         for (int c0 = 0; c0 < N; c0 += 16) {
           float v[16];
           tmem_ld16(tmem + h * N + ((uint32_t)(q * 32) << 16) + c0, v);
           tmem_ld_wait();
-          float4 *dst = reinterpret_cast<float4 *>(out + (size_t)row * R + c0);
+          float4 *dst = reinterpret_cast<float4 *>(srow + c0);
           dst[0] = make_float4(v[0], v[1], v[2], v[3]);
           dst[1] = make_float4(v[4], v[5], v[6], v[7]);
           dst[2] = make_float4(v[8], v[9], v[10], v[11]);
           dst[3] = make_float4(v[12], v[13], v[14], v[15]);
         }
       }
-    } else {
-      fail_timeout(ctl, jb.meta);
+      named_sync(1, 128);
+      if (ok)
+        for (int i = 0; i < 32; ++i) {
+          const int row = q * 32 + i;
+          const float4 *src = reinterpret_cast<const float4 *>(stg + (size_t)row * LDS);
+          float4 *dst = reinterpret_cast<float4 *>(out + (size_t)(h * 128 + row) * R);
+          for (int c = lane; c < N / 4; c += 32) dst[c] = src[c];
+        }
+      named_sync(1, 128);
     }
   }
   fence_before_sync();
@@ -1293,6 +1329,8 @@ int num_sms() {
 }
 
 }  // namespace
+
+int tc_sm_count() { return num_sms(); }
 
 bool tc_rotation_supported(int r, int storage) {
   return storage == ISKV_BF16 && r % 64 == 0 && r >= 64 && r <= 256 && encode_fn() != nullptr;
@@ -1669,8 +1707,7 @@ bool encode_gram_job(TcJob &tj, const void *U, int64_t n_cap, const void *B, int
 
 cudaError_t launch_tc_gram(const TcJob *djobs, const GramParams &p, cudaStream_t s) {
   cudaError_t e = cudaSuccess;
-  const size_t smem = 1024 + (size_t)GRAM_STAGES * (p.r / 64) * GRAM_KT * 128 + sizeof(TcCtl) +
-                      2 * GRAM_STAGES * sizeof(uint64_t);
+  const size_t smem = 1024 + gram_area_bytes(p.r) + sizeof(TcCtl) + 2 * GRAM_RING * sizeof(uint64_t);
   e = cudaFuncSetAttribute(k_gram_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_gram_tc<<<p.count * (p.nsu + p.nsb), GRAM_THREADS, smem, s>>>(djobs, p);
