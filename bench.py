@@ -201,6 +201,9 @@ class Workload:
         keys, _ = synth.outlier_prompt_keys(SEL_L, HEADS, HEAD_DIM, seed=4)
         self.keys = torch.as_tensor(keys, dtype=torch.float32).to(dev).to(torch.bfloat16)
         self.sel_out = None
+        self.side = torch.cuda.Stream(dev)
+        self.ev_start = torch.cuda.Event()
+        self.ev_sel = torch.cuda.Event()
         torch.cuda.synchronize(dev)
 
     def _fold(self, g, F, stream=None):
@@ -242,15 +245,23 @@ class Workload:
         return epos, PROMPT + n + WINDOW
 
     def step(self, t, epos, n_total, F=None, stream=None):
-        kv = self.kv
+        """One decode step. The prompt selection reads nothing the fold or the reconstruction
+        writes, so it runs on a second stream beside them (on the SMs the core SVD's last wave of
+        clusters leaves idle); the step ends when both streams have."""
+        kv, torch = self.kv, self.torch
         F = F if F is not None else self.F[t]
-        self._fold(self.n0 // BLK + t, F, stream=stream)
-        kv.reconstruct_batched(self.hists, self.exact, [epos] * len(self.hists), n_total, HEADS,
-                               HEAD_DIM, self.rope, THETA, outs=self.outs,
-                               ws=self._aligned(self.ws_recon), stream=stream)
+        main = stream if stream is not None else torch.cuda.current_stream(self.dev)
+        self.ev_start.record(main)
+        self.side.wait_event(self.ev_start)
         self.sel_out = kv.select_prompt_blocks(self.keys, 8, 128, 4, 32,
                                                ws=self._aligned(self.ws_sel), out=self.sel_out,
-                                               stream=stream)
+                                               stream=self.side)
+        self.ev_sel.record(self.side)
+        self._fold(self.n0 // BLK + t, F, stream=main)
+        kv.reconstruct_batched(self.hists, self.exact, [epos] * len(self.hists), n_total, HEADS,
+                               HEAD_DIM, self.rope, THETA, outs=self.outs,
+                               ws=self._aligned(self.ws_recon), stream=main)
+        main.wait_event(self.ev_sel)
 
 
 ROOFLINE_STAGE = "reconstruct.compressed"
