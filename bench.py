@@ -688,6 +688,10 @@ def run_e2e(wl, kv, torch, dev, stream, pos, first_step, steps, world):
     devK = [torch.empty_like(wl.keys) for _ in range(2)]
     res_sig = torch.empty(cnt, R, dtype=torch.float32).pin_memory()
     res_meta = torch.empty(cnt, 4, dtype=torch.int64).pin_memory()
+    # The histories' sigma and meta words are gathered on the device first, so each step reads
+    # them back with two copies rather than two per history.
+    dev_sig = torch.empty(cnt, R, dtype=torch.float32, device=dev)
+    dev_meta = torch.empty(cnt, 4, dtype=torch.int64, device=dev)
     res_cnt = torch.empty(2 + HEADS, dtype=torch.int64).pin_memory()
     res_pk = torch.empty(SEL_L, dtype=torch.int32).pin_memory()
     res_pv = torch.empty(SEL_L, dtype=torch.int32).pin_memory()
@@ -724,9 +728,10 @@ def run_e2e(wl, kv, torch, dev, stream, pos, first_step, steps, world):
         wl.keys = devK[b]
         wl.step(t, *pos[t], F=devF[b])
         free[b].record(stream)
-        for j, h in enumerate(wl.hists):
-            res_sig[j].copy_(h.sigma, non_blocking=True)
-            res_meta[j].copy_(h.meta, non_blocking=True)
+        torch.stack([h.sigma for h in wl.hists], out=dev_sig)
+        torch.stack([h.meta for h in wl.hists], out=dev_meta)
+        res_sig.copy_(dev_sig, non_blocking=True)
+        res_meta.copy_(dev_meta, non_blocking=True)
         res_cnt.copy_(wl.sel_out["counts"], non_blocking=True)
         res_pk.copy_(wl.sel_out["P_K"], non_blocking=True)
         res_pv.copy_(wl.sel_out["P_V"], non_blocking=True)
