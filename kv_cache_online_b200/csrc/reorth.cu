@@ -14,6 +14,7 @@
 #include "gemm_tile.cuh"
 #include "profiling.h"
 #include "reorth.h"
+#include "tc_sm100.cuh"
 
 namespace iskv {
 
@@ -233,6 +234,236 @@ __global__ void __launch_bounds__(256, 2) k_ns_step(const ReorthJob *jobs, Reort
       [&](int m, int n, float acc) { Xo[(size_t)m * r + n] = acc; });
 }
 
+// The same stages on the tensor cores, for bf16-stored factors (r a multiple of 64 up to 256).
+// Each product is taken in three bf16 MMAs, A_hi B_hi + A_hi B_lo + A_lo B_hi with x = x_hi + x_lo
+// (x_hi = bf16(x), x_lo = bf16(x - x_hi)): about 16 significant bits, far below the bf16 rounding of the factors
+// the re-orthogonalisation serves, and enough for the stopping test (its rounding floor stays
+// near 1e-4 in ||T - I||_F against the 5e-4 threshold). Y, Z and T are polynomials in the Gram
+// matrix, hence symmetric, so the right operand's rows are read as its columns. One CTA takes
+// 128 rows of one product (N = r, K = k): 8 warps convert the float32 K-slabs of both operands
+// into two 96 KB stages of hi / lo tiles (128-byte-swizzled K-major), one thread issues the MMAs
+// into TMEM, and the 8 warps then stage the result through the idle stages and write whole rows.
+constexpr int NS_TC_THREADS = 288;  // 8 converter / epilogue warps + the MMA warp
+constexpr uint64_t NS_WAIT_NS = 2000000000ull;
+
+struct NsTcCtl {
+  uint64_t full[2], empty[2], acc;
+  uint32_t tmem;
+  int abort;
+};
+
+__host__ __device__ constexpr size_t ns_tc_stage_bytes() { return 2 * 128 * 128 + 2 * 256 * 128; }
+__host__ __device__ constexpr size_t ns_tc_smem() {
+  return 1024 + 2 * ns_tc_stage_bytes() + sizeof(NsTcCtl);
+}
+
+// Row `row` of a K-major 128-byte-swizzled tile: 16-byte chunk c of its 128 bytes at chunk
+// c ^ (row & 7).
+ISKV_DEV void ns_put_chunk(uint8_t *tile, int row, int c, uint4 v) {
+  *reinterpret_cast<uint4 *>(tile + row * 128 + ((c ^ (row & 7)) << 4)) = v;
+}
+
+// Eight floats to bf16 hi and lo parts, packed two per word (low half first).
+ISKV_DEV void ns_split8(const float (&x)[8], uint4 &hi, uint4 &lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat16 a = __float2bfloat16_rn(x[2 * i]), b = __float2bfloat16_rn(x[2 * i + 1]);
+    const __nv_bfloat16 c = __float2bfloat16_rn(x[2 * i] - __bfloat162float(a));
+    const __nv_bfloat16 d = __float2bfloat16_rn(x[2 * i + 1] - __bfloat162float(b));
+    h[i] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+    l[i] = (uint32_t)__bfloat16_as_ushort(c) | ((uint32_t)__bfloat16_as_ushort(d) << 16);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+template <int STAGE>
+__global__ void __launch_bounds__(NS_TC_THREADS, 1) k_ns_tc(const ReorthJob *jobs, ReorthParams p,
+                                                           int it, size_t y0, size_t z0, size_t y1,
+                                                           size_t z1, size_t yb0, size_t zb0,
+                                                           size_t yb1, size_t zb1) {
+  using namespace tc;
+  const int per = STAGE == 0 ? 2 : 4;
+  const int job = blockIdx.y / per, rem = blockIdx.y % per, which = rem & 1, g = rem >> 1;
+  const ReorthJob &jb = jobs[job];
+  int32_t *sc = reinterpret_cast<int32_t *>(jb.h.ws);
+  if (sc[FS_SKIP]) return;
+  const int k = sc[FS_K_OLD], R = p.r, m0 = blockIdx.x * 128;
+  if (m0 >= k || ns_converged(sc, it, which)) return;  // uniform over the CTA
+  char *ws = jb.h.ws;
+  const float *Y = reinterpret_cast<const float *>(ws + (which == 0 ? y0 : yb0));
+  const float *Z = reinterpret_cast<const float *>(ws + (which == 0 ? z0 : zb0));
+  const float *Am, *Bm;
+  float *Out;
+  if (STAGE == 0) {
+    Am = Z;
+    Bm = Y;
+    Out = reinterpret_cast<float *>(ws + p.ws.T[which]);
+  } else {
+    const float *T = reinterpret_cast<const float *>(ws + p.ws.T[which]);
+    Am = g == 0 ? Y : T;
+    Bm = g == 0 ? T : Z;
+    Out = reinterpret_cast<float *>(
+        ws + (g == 0 ? (which == 0 ? y1 : yb1) : (which == 0 ? z1 : zb1)));
+  }
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  NsTcCtl *ctl = reinterpret_cast<NsTcCtl *>(smem + 2 * ns_tc_stage_bytes());
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int KS = (k + 63) / 64;
+  const uint32_t idesc = idesc_bf16_f32(128, R);
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->full[i], 8);
+      mbar_init(&ctl->empty[i], 1);
+    }
+    mbar_init(&ctl->acc, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  const uint32_t ncols = R <= 64 ? 64 : (R <= 128 ? 128 : 256);
+  if (warp == 8) tmem_alloc(&ctl->tmem, ncols);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int *abort = &ctl->abort;
+
+  if (warp < 8) {
+    // ---------------- converters: K-slab s of A (rows m0 .. m0+127) and B (rows 0 .. R-1)
+    bool ok = true;
+    for (int s = 0; s < KS && ok; ++s) {
+      const int st = s & 1;
+      if (s >= 2 && !__all_sync(~0u, mbar_wait(&ctl->empty[st], ((s - 2) >> 1) & 1, abort,
+                                               NS_WAIT_NS))) {
+        ok = false;
+        break;
+      }
+      uint8_t *ahi = smem + st * ns_tc_stage_bytes(), *alo = ahi + 128 * 128;
+      uint8_t *bhi = alo + 128 * 128, *blo = bhi + 256 * 128;
+      // A: thread -> (row tid / 2, 32 columns); B: thread -> (row tid, 64 columns). All of a
+      // thread's 16-byte loads are issued before any is converted; entries outside the leading
+      // k x k block count as zero.
+      {
+        const int row = tid >> 1, c0 = (tid & 1) * 32, gm = m0 + row;
+        float4 xa[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          xa[u] = gm < R ? *reinterpret_cast<const float4 *>(Am + (size_t)gm * R + s * 64 + c0 + 4 * u)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 xb[16];
+        const bool brow = tid < R;
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          xb[u] = brow ? *reinterpret_cast<const float4 *>(Bm + (size_t)tid * R + s * 64 + 4 * u)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float x[8] = {xa[2 * u].x, xa[2 * u].y, xa[2 * u].z, xa[2 * u].w,
+                        xa[2 * u + 1].x, xa[2 * u + 1].y, xa[2 * u + 1].z, xa[2 * u + 1].w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (!(gm < k && s * 64 + c0 + u * 8 + e < k)) x[e] = 0.f;
+          uint4 hv, lv;
+          ns_split8(x, hv, lv);
+          ns_put_chunk(ahi, row, (c0 >> 3) + u, hv);
+          ns_put_chunk(alo, row, (c0 >> 3) + u, lv);
+        }
+        if (brow) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float x[8] = {xb[2 * u].x, xb[2 * u].y, xb[2 * u].z, xb[2 * u].w,
+                          xb[2 * u + 1].x, xb[2 * u + 1].y, xb[2 * u + 1].z, xb[2 * u + 1].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (!(tid < k && s * 64 + u * 8 + e < k)) x[e] = 0.f;
+            uint4 hv, lv;
+            ns_split8(x, hv, lv);
+            ns_put_chunk(bhi, tid, u, hv);
+            ns_put_chunk(blo, tid, u, lv);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->full[st]);
+    }
+    if (!ok) {
+      ctl->abort = 1;
+      record_status(jb.h.meta, ISKV_ERR_TIMEOUT);
+    }
+    // ---------------- epilogue: warp (q, half) takes TMEM lanes 32 q and columns 128 half ..
+    const int q = warp & 3, half = warp >> 2, cols = R / 2, c0 = half * cols;
+    const bool ready = ok && __all_sync(~0u, mbar_wait(&ctl->acc, 0, abort, NS_WAIT_NS));
+    fence_after_sync();
+    // The stages are idle once the MMAs are done: rows of R + 4 floats (bank-spread) hold the
+    // 128 x R result before it leaves in whole rows.
+    float *stg = reinterpret_cast<float *>(smem);
+    const int LDS = R + 4, row = q * 32 + lane, gm = m0 + row;
+    float ss = 0.f;
+    if (ready) {
+      for (int cc = 0; cc < cols; cc += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + c0 + cc, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int n = c0 + cc + e;
+          float o = v[e];
+          if (STAGE == 0) {
+            const float t = (gm == n ? 1.5f : 0.f) - 0.5f * o;
+            const float dv = t - (gm == n ? 1.f : 0.f);
+            if (gm < k && n < k) ss = fmaf(dv, dv, ss);
+            o = t;
+          }
+          stg[row * LDS + n] = o;
+        }
+      }
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (ready) {
+      for (int i = warp; i < 128; i += 8) {
+        const int gi = m0 + i;
+        if (gi >= k) continue;
+        for (int n = lane; n < k; n += 32) Out[(size_t)gi * R + n] = stg[i * LDS + n];
+      }
+      if (STAGE == 0) {
+        ss = warp_sum(ss);
+        if (lane == 0) atomicAdd(reinterpret_cast<float *>(sc + RS_DEV + 2 * it + which), ss);
+      }
+    }
+  } else if (lane == 0) {
+    // ---------------- MMA issuer
+    bool ok = true;
+    for (int s = 0; s < KS; ++s) {
+      const int st = s & 1;
+      if (!mbar_wait(&ctl->full[st], (s >> 1) & 1, abort, NS_WAIT_NS)) { ok = false; break; }
+      fence_after_sync();
+      const uint32_t ahi = smem_u32(smem + st * ns_tc_stage_bytes()), alo = ahi + 128 * 128;
+      const uint32_t bhi = alo + 128 * 128, blo = bhi + 256 * 128;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        mma_bf16(tmem, sw128_desc(ahi + kk * 32), sw128_desc(bhi + kk * 32), idesc, (s | kk) != 0);
+        mma_bf16(tmem, sw128_desc(ahi + kk * 32), sw128_desc(blo + kk * 32), idesc, true);
+        mma_bf16(tmem, sw128_desc(alo + kk * 32), sw128_desc(bhi + kk * 32), idesc, true);
+      }
+      mma_commit(&ctl->empty[st]);
+    }
+    if (!ok) {
+      ctl->abort = 1;
+      record_status(jb.h.meta, ISKV_ERR_TIMEOUT);
+    }
+    mma_commit(&ctl->acc);
+    mbar_wait(&ctl->acc, 0, abort, NS_WAIT_NS / 4);
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 8) tmem_dealloc(tmem, ncols);
+}
+
 // Convergence check of the iteration: the last computed T = 1.5 I - 0.5 Z Y must be I to working
 // accuracy, ||T - I||_F <= 1e-3 (the first stage of every computed iteration summed the squares;
 // after an early stop the remaining slots hold 0). Quadratic convergence from a Gram matrix within
@@ -426,11 +657,27 @@ cudaError_t launch_reorth(const ReorthJob *jobs, const ReorthParams &p, cudaStre
   k_ns_init<<<dim3(64, p.count * 2), 256, 0, s>>>(jobs, p);
   size_t y0[2] = {W.Y[0], W.Y[1]}, z0[2] = {W.Z[0], W.Z[1]};
   size_t y1[2] = {W.Y2[0], W.Y2[1]}, z1[2] = {W.Z2[0], W.Z2[1]};
+  const bool ns_tc = p.tc_basis != 0;  // bf16 factors, r a multiple of 64 up to 256
+  if (ns_tc) {
+    cudaError_t e0 = cudaFuncSetAttribute(k_ns_tc<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)ns_tc_smem());
+    if (e0 == cudaSuccess)
+      e0 = cudaFuncSetAttribute(k_ns_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)ns_tc_smem());
+    if (e0 != cudaSuccess) return e0;
+  }
   for (int it = 0; it < NS_ITERS; ++it) {
-    k_ns_step<0><<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p, it, y0[0], z0[0], y1[0],
-                                                         z1[0], y0[1], z0[1], y1[1], z1[1]);
-    k_ns_step<1><<<dim3(tn, tm, p.count * 4), 256, 0, s>>>(jobs, p, it, y0[0], z0[0], y1[0],
-                                                         z1[0], y0[1], z0[1], y1[1], z1[1]);
+    if (ns_tc) {
+      k_ns_tc<0><<<dim3((r + 127) / 128, p.count * 2), NS_TC_THREADS, ns_tc_smem(), s>>>(
+          jobs, p, it, y0[0], z0[0], y1[0], z1[0], y0[1], z0[1], y1[1], z1[1]);
+      k_ns_tc<1><<<dim3((r + 127) / 128, p.count * 4), NS_TC_THREADS, ns_tc_smem(), s>>>(
+          jobs, p, it, y0[0], z0[0], y1[0], z1[0], y0[1], z0[1], y1[1], z1[1]);
+    } else {
+      k_ns_step<0><<<dim3(tn, tm, p.count * 2), 256, 0, s>>>(jobs, p, it, y0[0], z0[0], y1[0],
+                                                           z1[0], y0[1], z0[1], y1[1], z1[1]);
+      k_ns_step<1><<<dim3(tn, tm, p.count * 4), 256, 0, s>>>(jobs, p, it, y0[0], z0[0], y1[0],
+                                                           z1[0], y0[1], z0[1], y1[1], z1[1]);
+    }
     for (int w = 0; w < 2; ++w) {
       size_t t = y0[w]; y0[w] = y1[w]; y1[w] = t;
       t = z0[w]; z0[w] = z1[w]; z1[w] = t;
