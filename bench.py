@@ -202,17 +202,23 @@ class Workload:
         self.keys = torch.as_tensor(keys, dtype=torch.float32).to(dev).to(torch.bfloat16)
         self.sel_out = None
         self.side = torch.cuda.Stream(dev)
+        self.rec_stream = torch.cuda.Stream(dev)
         self.ev_start = torch.cuda.Event()
         self.ev_sel = torch.cuda.Event()
+        self.ev_fold = torch.cuda.Event()
+        self.ev_rec = torch.cuda.Event()
+        self.rec_pending = False
         torch.cuda.synchronize(dev)
 
-    def _fold(self, g, F, stream=None):
+    def _fold(self, g, F, stream=None, factors_ready=None):
         """Fold block g (global block index; rows g*64 .. g*64+63 of every stream) and, when the
-        cadence says so, re-orthogonalise."""
+        cadence says so, re-orthogonalise. With `factors_ready` the fold's factor-writing stages
+        wait for that event (the previous step's reconstruction)."""
         kv = self.kv
         fpos = self.fpos[g * BLK:(g + 1) * BLK]
         kv.fold_block_batched(self.hists, list(F), [fpos] * len(self.hists),
-                              ws=self._aligned(self.ws_fold), stream=stream)
+                              ws=self._aligned(self.ws_fold), stream=stream,
+                              factors_ready=factors_ready)
         if (g + 1) % REORTH_EVERY == 0:
             kv.reorth(self.hists, ws=self._aligned(self.ws_reorth), stream=stream)
 
@@ -245,9 +251,12 @@ class Workload:
         return epos, PROMPT + n + WINDOW
 
     def step(self, t, epos, n_total, F=None, stream=None):
-        """One decode step. The prompt selection reads nothing the fold or the reconstruction
-        writes, so it runs on a second stream beside them (on the SMs the core SVD's last wave of
-        clusters leaves idle); the step ends when both streams have."""
+        """One decode step, pipelined over three streams. The prompt selection reads nothing the
+        fold or the reconstruction writes, so it runs beside them. The step's reconstruction runs on
+        its own stream after the fold (and reorth), and the next step's fold starts beside it: the
+        fold's read-only stages (projection, residual QR, core SVD) overlap the reconstruction,
+        and its rotations and write-back wait for it (iskv_fold_block_batched_after). The step
+        ends when the fold and the selection have; `drain` waits for the last reconstruction."""
         kv, torch = self.kv, self.torch
         F = F if F is not None else self.F[t]
         main = stream if stream is not None else torch.cuda.current_stream(self.dev)
@@ -257,11 +266,22 @@ class Workload:
                                                ws=self._aligned(self.ws_sel), out=self.sel_out,
                                                stream=self.side)
         self.ev_sel.record(self.side)
-        self._fold(self.n0 // BLK + t, F, stream=main)
+        self._fold(self.n0 // BLK + t, F, stream=main,
+                   factors_ready=self.ev_rec if self.rec_pending else None)
+        self.ev_fold.record(main)
+        self.rec_stream.wait_event(self.ev_fold)
         kv.reconstruct_batched(self.hists, self.exact, [epos] * len(self.hists), n_total, HEADS,
                                HEAD_DIM, self.rope, THETA, outs=self.outs,
-                               ws=self._aligned(self.ws_recon), stream=main)
+                               ws=self._aligned(self.ws_recon), stream=self.rec_stream)
+        self.ev_rec.record(self.rec_stream)
+        self.rec_pending = True
         main.wait_event(self.ev_sel)
+
+    def drain(self, stream=None):
+        """Make `stream` wait for the last step's reconstruction."""
+        main = stream if stream is not None else self.torch.cuda.current_stream(self.dev)
+        if self.rec_pending:
+            main.wait_event(self.ev_rec)
 
 
 ROOFLINE_STAGE = "reconstruct.compressed"
@@ -517,6 +537,7 @@ def run_b200(args):
     ev0.record(stream)
     for t in range(args.warmup, steps_total):
         wl.step(t, *pos[t])
+    wl.drain(stream)
     ev1.record(stream)
     barrier()
     clocks = sampler.stop()
@@ -735,6 +756,7 @@ def run_e2e(wl, kv, torch, dev, stream, pos, first_step, steps, world):
         res_cnt.copy_(wl.sel_out["counts"], non_blocking=True)
         res_pk.copy_(wl.sel_out["P_K"], non_blocking=True)
         res_pv.copy_(wl.sel_out["P_V"], non_blocking=True)
+    wl.drain(stream)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - t0

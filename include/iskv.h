@@ -122,6 +122,22 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
                                     float tau_rel, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * The batched fold, pipelined behind readers of the current factors (no counterpart on the
+ * pages; Algorithm 3 runs a step's reconstruction or attention between two folds). The stages
+ * that only read the histories' factors (projection, residual QR and SVD, core SVD) start at once
+ * on `stream`; the stages that change them (basis and coordinate rotations, write-back of U,
+ * sigma, B, positions and meta) first wait for `factors_ready`, a cudaEvent_t the caller records
+ * on the stream of its last reader of those factors (a reconstruction or decode attention issued
+ * on another stream), or NULL. One exception: with bf16 factors and blocks the projection clears
+ * B's columns k .. r_max-1 before the wait; this library leaves those columns zero, so their
+ * values do not change. Arguments and errors otherwise as iskv_fold_block_batched.
+ */
+iskv_status iskv_fold_block_batched_after(const iskv_lowrank *hs, int32_t count,
+                                          const void *const *F, int32_t f_dtype, int32_t b,
+                                          const int32_t *const *f_pos, float tau_rel, void *ws,
+                                          size_t ws_bytes, void *stream, void *factors_ready);
+
+/*
  * Re-orthogonalisation -- Section 4.4: with orthonormal-basis factorisations U = Q_U R_U,
  * B = Q_B R_B, decompose R_U diag(sigma) R_B^T = X diag(sigma') Y^T and set U <- Q_U X,
  * sigma <- sigma', B <- Q_B Y. The product U diag(sigma) B^T is unchanged in exact arithmetic;

@@ -119,8 +119,11 @@ def fold_workspace_size(count, d, r_max, b) -> int:
     return int(_lib.load().iskv_fold_workspace_size(count, d, r_max, b))
 
 
-def fold_block_batched(hists, Fs, f_poss, tau_rel: float = 0.0, ws=None, stream=None):
-    """Algorithm 2 for every history in ``hists`` (one pending block each), in one launch set."""
+def fold_block_batched(hists, Fs, f_poss, tau_rel: float = 0.0, ws=None, stream=None,
+                       factors_ready=None):
+    """Algorithm 2 for every history in ``hists`` (one pending block each), in one launch set.
+    ``factors_ready`` (a ``torch.cuda.Event``) lets the fold's read-only stages start at once and
+    makes its factor-writing stages wait for the event (iskv_fold_block_batched_after)."""
     lib = _lib.load()
     n = len(hists)
     if n == 0:
@@ -138,8 +141,14 @@ def fold_block_batched(hists, Fs, f_poss, tau_rel: float = 0.0, ws=None, stream=
     hs = _handles(hists)
     Fp = (ctypes.c_void_p * n)(*[F.data_ptr() for F in Fs])
     Pp = (ctypes.c_void_p * n)(*[p.data_ptr() for p in f_poss])
-    _lib.check(lib.iskv_fold_block_batched(hs, n, Fp, fdt, b, Pp, float(tau_rel), w.data_ptr(),
-                                           w.numel(), _stream(stream)), "fold_block")
+    if factors_ready is None:
+        _lib.check(lib.iskv_fold_block_batched(hs, n, Fp, fdt, b, Pp, float(tau_rel),
+                                               w.data_ptr(), w.numel(), _stream(stream)),
+                   "fold_block")
+    else:
+        _lib.check(lib.iskv_fold_block_batched_after(hs, n, Fp, fdt, b, Pp, float(tau_rel),
+                                                     w.data_ptr(), w.numel(), _stream(stream),
+                                                     factors_ready.cuda_event), "fold_block")
 
 
 def fold_block(hist, F, f_pos, tau_rel: float = 0.0, ws=None, stream=None):

@@ -46,6 +46,10 @@ SIGNATURES = {
     "iskv_fold_block_batched": (c_i32, [ctypes.POINTER(IskvLowRank), c_i32,
                                         ctypes.POINTER(c_vp), c_i32, c_i32, ctypes.POINTER(c_vp),
                                         c_f32, c_vp, c_sz, c_vp]),
+    "iskv_fold_block_batched_after": (c_i32, [ctypes.POINTER(IskvLowRank), c_i32,
+                                              ctypes.POINTER(c_vp), c_i32, c_i32,
+                                              ctypes.POINTER(c_vp), c_f32, c_vp, c_sz, c_vp,
+                                              c_vp]),
     "iskv_reorth_workspace_size": (c_sz, [c_i32, c_i32, c_i32, c_i64]),
     "iskv_reorth": (c_i32, [ctypes.POINTER(IskvLowRank), c_i32, c_vp, c_sz, c_vp]),
     "iskv_reconstruct_workspace_size": (c_sz, [c_i32, c_i32, c_i32]),

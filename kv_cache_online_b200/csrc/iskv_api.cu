@@ -305,9 +305,10 @@ size_t iskv_fold_workspace_size(int32_t count, int32_t d, int32_t r_max, int32_t
   return jobs_bytes(count, sizeof(FoldJob)) + 3 * tc_table_bytes(count) + (size_t)count * L.total;
 }
 
-iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const void *const *F,
-                                    int32_t f_dtype, int32_t b, const int32_t *const *f_pos,
-                                    float tau_rel, void *ws, size_t ws_bytes, void *stream) {
+static iskv_status fold_batched(const iskv_lowrank *hs, int32_t count, const void *const *F,
+                                int32_t f_dtype, int32_t b, const int32_t *const *f_pos,
+                                float tau_rel, void *ws, size_t ws_bytes, void *stream,
+                                void *factors_ready) {
   const char *who = "iskv_fold_block";
   g_last_error.clear();
   if (!hs || !F || !f_pos) return fail(ISKV_ERR_ARG, "%s: null host array", who);
@@ -422,6 +423,11 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   if ((e = launch_core(cj, fold_core_params(p), s)) != cudaSuccess)
     return cuda_fail(e, "fold: core svd");
   stage_mark(s, ST_FOLD_CORE);
+  // The stages above only read the histories' factors; the rotations and the write-back below
+  // change them, after the caller's readers of the current factors are done.
+  if (factors_ready &&
+      (e = cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(factors_ready), 0)) != cudaSuccess)
+    return cuda_fail(e, "fold: wait for factors_ready");
   const RotParams rp = fold_rot_params(p);
   if (p.tc_basis) {
     e = launch_basis_prep(djobs, p, s);
@@ -441,6 +447,20 @@ iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const
   if ((e = launch_fold_finalize(djobs, p, s)) != cudaSuccess) return cuda_fail(e, "fold: finalize");
   stage_mark(s, ST_FOLD_FINALIZE);
   return ISKV_OK;
+}
+
+iskv_status iskv_fold_block_batched(const iskv_lowrank *hs, int32_t count, const void *const *F,
+                                    int32_t f_dtype, int32_t b, const int32_t *const *f_pos,
+                                    float tau_rel, void *ws, size_t ws_bytes, void *stream) {
+  return fold_batched(hs, count, F, f_dtype, b, f_pos, tau_rel, ws, ws_bytes, stream, nullptr);
+}
+
+iskv_status iskv_fold_block_batched_after(const iskv_lowrank *hs, int32_t count,
+                                          const void *const *F, int32_t f_dtype, int32_t b,
+                                          const int32_t *const *f_pos, float tau_rel, void *ws,
+                                          size_t ws_bytes, void *stream, void *factors_ready) {
+  return fold_batched(hs, count, F, f_dtype, b, f_pos, tau_rel, ws, ws_bytes, stream,
+                      factors_ready);
 }
 
 iskv_status iskv_fold_block(const iskv_lowrank *h, const void *F, int32_t f_dtype, int32_t b,

@@ -150,3 +150,44 @@ def test_nonfinite_block_is_flagged():
     _fold_rows(m, h, X, 16, 2)
     _, _, _, st = h.status()
     assert st & bit(5)
+
+
+def test_fold_after_event_waits_before_writing_factors():
+    """iskv_fold_block_batched_after: a reconstruction issued on another stream, held back there by
+    a long spin, must read the factors from before the fold; the fold's result equals the plain
+    fold's bit for bit."""
+    m = kv()
+    d, r, b, n = 256, 64, 64, 1024
+    import synth
+    X = stored(synth.lowrank_rows(n + b, d, 1.0, 0.02, seed=41), torch.float32)
+    Xd = torch.as_tensor(X, dtype=torch.bfloat16, device="cuda")
+    pos = torch.arange(n + b, dtype=torch.int32, device="cuda")
+
+    def built():
+        h = m.LowRankHistory(d, r, n + b, storage=torch.bfloat16)
+        for i in range(0, n, b):
+            m.fold_block(h, Xd[i:i + b].contiguous(), pos[i:i + b].contiguous())
+        return h
+
+    ha, hb = built(), built()
+    exact = torch.zeros(0, d, dtype=torch.bfloat16, device="cuda")
+    epos = torch.zeros(0, dtype=torch.int32, device="cuda")
+    # The two streams' calls in flight together take workspaces of their own.
+    wsr = torch.empty(m.reconstruct_workspace_size(1, d, r), dtype=torch.uint8, device="cuda")
+    wsf = torch.empty(m.fold_workspace_size(1, d, r, b), dtype=torch.uint8, device="cuda")
+    want = m.reconstruct(ha, exact, epos, n, 2, 128, False, ws=wsr)  # before any new fold
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        torch.cuda._sleep(200_000_000)                               # ~0.1 s at 2 GHz
+        got = m.reconstruct(hb, exact, epos, n, 2, 128, False, ws=wsr, stream=side)
+        ev = torch.cuda.Event()
+        ev.record(side)
+    F = Xd[n:n + b].contiguous()
+    m.fold_block_batched([hb], [F], [pos[n:n + b].contiguous()], ws=wsf, factors_ready=ev)
+    m.fold_block(ha, F, pos[n:n + b].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
+    for x, y in ((ha.U, hb.U), (ha.B, hb.B), (ha.sigma, hb.sigma), (ha.meta, hb.meta)):
+        assert torch.equal(x, y)
