@@ -222,7 +222,8 @@ __global__ void __launch_bounds__(ROT_THREADS, 1) k_rotate_tc(const TcJob *jobs,
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     int cur = -1, nb = 0, na = 0;
-    uint32_t gsl = 0;
+    RingPos rp;
+    const uint64_t da0 = sw128_desc(smem_u32(sA)), db0 = sw128_desc(smem_u32(sB));
     for (int t = tr.begin; t < tr.end && !*abort; ++t) {
       const int j = t / tr.tiles_per_job, row0 = (t % tr.tiles_per_job) * TC_M;
       const TcJob &jb = jobs[j];
@@ -241,18 +242,18 @@ __global__ void __launch_bounds__(ROT_THREADS, 1) k_rotate_tc(const TcJob *jobs,
       fence_after_sync();
       const uint32_t d = tmem + buf * N;
       bool ok = true;
-      for (int s = 0; s < KS; ++s, ++gsl) {
-        const uint32_t st = gsl % NS;
-        if (!mbar_wait(&ctl->a_conv[st], (gsl / NS) & 1, abort, WAIT_NS)) {
+      for (int s = 0; s < KS; ++s) {
+        if (!mbar_wait(&ctl->a_conv[rp.slot], rp.phase, abort, WAIT_NS)) {
           ok = false;
           break;
         }
         fence_after_sync();
-        const uint32_t a0 = smem_u32(sA + st * SLAB_BYTES), b0 = smem_u32(sB + s * N * 128);
+        const uint64_t da = desc_add(da0, rp.slot * SLAB_BYTES), db = desc_add(db0, s * N * 128);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(d, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (s | kk) != 0);
-        mma_commit(&ctl->a_empty[st]);
+          mma_bf16(d, desc_add(da, kk * 32), desc_add(db, kk * 32), idesc, (s | kk) != 0);
+        mma_commit(&ctl->a_empty[rp.slot]);
+        rp.next(NS);
       }
       if (!ok) { fail_timeout(ctl, jb.meta); break; }
       mma_commit(&ctl->acc_full[buf]);
@@ -639,13 +640,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_project_tc(const ProjJob *job
 constexpr int REC_MAX_STAGES = 8;
 // Epilogue warps: two per TMEM lane quarter, 32 RoPE pairs each. (Sixteen warps with 16 pairs
 // each and 32-byte tile stores measured slower.)
-__host__ __device__ constexpr int rec_epilogue_warps(int) { return 8; }
-__host__ __device__ constexpr int rec_threads(int qpk) { return 64 + 32 * rec_epilogue_warps(qpk); }
+constexpr int REC_EPW = 8;
+constexpr int REC_THREADS = 64 + 32 * REC_EPW;
 constexpr int REC_STG_BYTES = 2 * TC_M * 128;  // lo and hi column halves of one head
-// Attention scores (qpk query heads per KV head): the staging region holds, per warp pair, the
-// query groups of the CTA's (at most two) heads and a 32-row exchange of partial scores.
-__host__ __device__ constexpr int attn_pair_floats(int qpk) { return 2 * 64 * 2 * qpk + 32 * 2 * qpk; }
-__host__ __device__ constexpr int rec_stg_bytes(int qpk) { return qpk ? 4 * attn_pair_floats(qpk) * 4 : REC_STG_BYTES; }
 
 // RoPE tables (head_dim 128, 64 frequencies omega_j = theta^(-2j/128)). Angles are reduced in
 // exact integer arithmetic: W_j = omega_j / (2 pi) is held as a 0.64 fixed-point fraction
@@ -685,12 +682,9 @@ struct RecCtl {
   int abort;
 };
 
-// QPK = 0: reconstruction (rows written to out[pos]). QPK > 0: decode-attention scores -- each
-// RoPE'd key row is dotted with the QPK query heads of its KV head and only the scores
-// S[query head][pos] are written; the dense keys never leave the SM.
-template <int QPK>
-__global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *jobs, TcParams p,
-                                                           const __grid_constant__ RopeTab rt) {
+// Reconstruction: rows U (sigma B)^T, RoPE'd at their positions, written to out[pos].
+__global__ void __launch_bounds__(REC_THREADS, 1) k_rec_tc(const TcJob *jobs, TcParams p,
+                                                      const __grid_constant__ RopeTab rt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -699,11 +693,11 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
   uint8_t *sB = smem;                            // KS slabs x (HP x 128 rows) x 128 B, resident
   uint8_t *sA = sB + KS * HP * SLAB_BYTES;       // NA slabs x 16 KB
   uint8_t *sStg = sA + NA * SLAB_BYTES;          // 2 x (128 rows x 128 B), SW128
-  RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + rec_stg_bytes(QPK));
+  RecCtl *ctl = reinterpret_cast<RecCtl *>(sStg + REC_STG_BYTES);
   RopeTab *rope_tab = reinterpret_cast<RopeTab *>(ctl + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Epilogue warps: WPQ per TMEM lane quarter, each holding NP of a head's 64 RoPE pairs.
-  constexpr int EPW = rec_epilogue_warps(QPK), WPQ = EPW / 4, NP = 64 / WPQ;
+  constexpr int EPW = REC_EPW, WPQ = EPW / 4, NP = 64 / WPQ;
   const int NN = HP * HN;                        // MMA N
   const uint32_t ncols = HP == 2 ? 512 : 256;    // two accumulator buffers of NN columns
   const uint32_t idesc = idesc_bf16_f32(TC_M, NN);
@@ -784,6 +778,7 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
   if (warp == 0 && lane == 0) {
     // ---------------- producer: basis rows of this CTA's heads once per history, U slabs per tile
     int na = 0, nb = 0, cur = -1;
+    RingPos rp;
     int64_t *fm = nullptr;  // meta of the history being loaded: where a timeout is recorded
     bool ok = true;
     for (Cur c = c_first; c.t >= 0 && ok && !*abort; c = advance(c)) {
@@ -803,10 +798,11 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
         ++nb;
       }
       for (int s = 0; s < KS; ++s) {
-        const int st = na % NA, use = na / NA;
-        if (use > 0 && !mbar_wait(&ctl->a_empty[st], (use - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
-        mbar_arrive_expect_tx(&ctl->a_full[st], SLAB_BYTES);
-        tma_load_2d(sA + st * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[st]);
+        // The slot's previous use (one lap back) must have been consumed.
+        if (na >= NA && !mbar_wait(&ctl->a_empty[rp.slot], rp.phase ^ 1u, abort, WAIT_NS)) { ok = false; break; }
+        mbar_arrive_expect_tx(&ctl->a_full[rp.slot], SLAB_BYTES);
+        tma_load_2d(sA + rp.slot * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[rp.slot]);
+        rp.next(NA);
         ++na;
       }
     }
@@ -817,9 +813,11 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
       mbar_wait(&ctl->a_full[(na - k) % NA], ((na - k) / NA) & 1, abort, WAIT_NS / 4);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    int na = 0, nb = 0, nc = 0, cur = -1;
+    int nb = 0, nc = 0, cur = -1;
     int64_t *fm = nullptr;
     bool ok = true;
+    RingPos rp;
+    const uint64_t da0 = sw128_desc(smem_u32(sA)), db0 = sw128_desc(smem_u32(sB));
     for (Cur c = c_first; c.t >= 0 && ok && !*abort; c = advance(c)) {
       const int j = c.j;
       fm = jobs[j].meta;
@@ -835,16 +833,15 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
       fence_after_sync();
       const uint32_t d0 = tmem + buf * NN;
       for (int s = 0; s < KS; ++s) {
-        const int st = na % NA;
-        if (!mbar_wait(&ctl->a_full[st], (na / NA) & 1, abort, WAIT_NS)) { ok = false; break; }
+        if (!mbar_wait(&ctl->a_full[rp.slot], rp.phase, abort, WAIT_NS)) { ok = false; break; }
         fence_after_sync();
-        const uint32_t a0 = smem_u32(sA + st * SLAB_BYTES);
-        const uint32_t b0 = smem_u32(sB + s * HP * SLAB_BYTES);
+        const uint64_t da = desc_add(da0, rp.slot * SLAB_BYTES);
+        const uint64_t db = desc_add(db0, s * HP * SLAB_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(d0, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc, (s | kk) != 0);
-        mma_commit(&ctl->a_empty[st]);
-        ++na;
+          mma_bf16(d0, desc_add(da, kk * 32), desc_add(db, kk * 32), idesc, (s | kk) != 0);
+        mma_commit(&ctl->a_empty[rp.slot]);
+        rp.next(NA);
       }
       if (!ok) break;
       mma_commit(&ctl->acc_full[buf]);
@@ -877,16 +874,12 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
     __nv_bfloat16 *h_out = nullptr;
     int64_t h_rows = 0, h_total = 0;
     bool h_rope = false, h_tiles = false;
-    float *h_S = nullptr;
-    float h_scale = 0.f;
     auto hist = [&](int j) {
       if (j != hj) {
         hj = j;
         const TcJob &jb = jobs[j];
         h_pos = jb.pos;
         h_out = static_cast<__nv_bfloat16 *>(jb.out);
-        h_S = jb.S;
-        h_scale = jb.scale;
         h_rows = rows_of(j);
         h_total = jb.n_total;
         h_rope = jb.rope != 0;
@@ -902,7 +895,6 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
       return row < h_rows ? __ldg(h_pos + row) : 0;
     };
     int acq_j = -1;  // history whose output tensor map this thread last acquired
-    int q_job = -1;  // history whose query groups this pair holds (scores mode)
     Cur c = c_first;
     int32_t ps_next = row_pos(c);
     for (;;) {
@@ -924,83 +916,6 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
       if (rope && valid) {
 #pragma unroll
         for (int i = 0; i < NP; ++i) rope_angle(rope_tab, j0 + i, (uint32_t)ps, cs[i], sn[i]);
-      } else if (QPK > 0) {  // the scores apply the (identity) rotation; the rows skip it
-#pragma unroll
-        for (int i = 0; i < NP; ++i) {
-          cs[i] = 1.f;
-          sn[i] = 0.f;
-        }
-      }
-      if constexpr (QPK > 0) {
-        // Scores: the pair keeps the query groups of the CTA's heads in shared memory, laid out
-        // [head][pair j][lo, hi][query] so that each key pair reads its 2 QPK weights contiguously.
-        float *qv = reinterpret_cast<float *>(sStg) + q * attn_pair_floats(QPK);
-        float *xch = qv + 2 * 64 * 2 * QPK;  // [32 rows][2 heads][QPK] partial scores of half 1
-        if (jj != q_job) {  // the same in both warps of the pair; both are past the last reads
-          const float *qg = jobs[jj].q;
-          for (int e = half * 32 + lane; e < HP * QPK * HN; e += 64) {
-            const int hh = e / (QPK * HN), g = (e / HN) % QPK, f = e % HN;
-            qv[((hh * 64 + (f & 63)) * 2 + (f >> 6)) * QPK + g] =
-                qg[(size_t)((member * HP + hh) * QPK + g) * HN + f];
-          }
-          named_sync(pair_bar, PB);
-          q_job = jj;
-        }
-        const int buf = nc & 1, use = nc >> 1;
-        if (!named_and(pair_bar, PB, mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS))) {
-          fail_timeout(ctl, jobs[jj].meta);
-          break;
-        }
-        fence_after_sync();
-        const uint32_t base = tmem + buf * NN + ((uint32_t)(q * 32) << 16);
-        float acc[2][QPK];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int g = 0; g < QPK; ++g) acc[h][g] = 0.f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h >= HP) break;
-#pragma unroll
-          for (int jb16 = 0; jb16 < 32; jb16 += 16) {
-            float lo[16], hi[16];
-            tmem_ld16(base + h * HN + j0 + jb16, lo);
-            tmem_ld16(base + h * HN + 64 + j0 + jb16, hi);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float c0 = cs[jb16 + i], s0 = sn[jb16 + i];
-              const float olo = lo[i] * c0 - hi[i] * s0, ohi = hi[i] * c0 + lo[i] * s0;
-              const float *qj = qv + ((h * 64 + j0 + jb16 + i) * 2) * QPK;
-#pragma unroll
-              for (int g = 0; g < QPK; ++g)
-                acc[h][g] = fmaf(qj[g], olo, fmaf(qj[QPK + g], ohi, acc[h][g]));
-            }
-          }
-        }
-        // The accumulators are in registers: tensor memory can take the next unit.
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
-        if (half == 1)
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int g = 0; g < QPK; ++g) xch[(lane * 2 + h) * QPK + g] = acc[h][g];
-        named_sync(pair_bar, PB);
-        if (half == 0 && valid) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int g = 0; g < QPK; ++g) {
-              if (h >= HP) break;
-              const int qh = (member * HP + h) * QPK + g;
-              h_S[(size_t)qh * n_total + ps] = h_scale * (acc[h][g] + xch[(lane * 2 + h) * QPK + g]);
-            }
-        }
-        ++nc;
-        c = cn;
-        continue;
       }
       __nv_bfloat16 *orow = out + (size_t)(valid ? ps : 0) * D + (size_t)member * HP * HN;
       // This lane quarter's 32 rows go out as tiles when their positions are consecutive (the
@@ -1062,7 +977,7 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
           }
           // Row = lane, 64-byte staged rows: 16-byte chunk u sits at chunk u ^ ((row >> 1) & 3)
           // (the 64-byte swizzle: address bits 7-8 into bits 4-5).
-          static_assert(QPK > 0 || NP == 32, "staging is laid out for 32 pairs per warp");
+          static_assert(NP == 32, "staging is laid out for 32 pairs per warp");
           const int sw = (lane >> 1) & 3;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -1094,6 +1009,389 @@ __global__ void __launch_bounds__(rec_threads(QPK), 1) k_rec_tc(const TcJob *job
       c = cn;
     }
     if (issuer && pending) bulk_wait0();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+// ================================================================================================
+// Decode-attention scores of compressed keys on the tensor cores (bf16 factors, head_dim 128).
+// A first MMA per 128-row tile forms the keys of the CTA's heads, U (sigma B_h)^T, in tensor
+// memory, as in the reconstruction. The epilogue applies RoPE at each row's position and writes
+// the rotated keys back into the same tensor memory as bf16, pair j of a head as one 32-bit
+// column (rotated low component, rotated high component). A second MMA with A in tensor memory
+// contracts them with the head's query group: B = [q_hi; q_lo], N = 16 rows of bf16, the queries
+// split into a bf16 head and a bf16 remainder, so the queries enter with about 16 significant bits
+// and the keys with the bf16 rounding of a reconstructed bf16 cache. Only the scores
+// S[query head][pos] leave the SM.
+struct ScoCtl {
+  uint64_t a_full[REC_MAX_STAGES], a_empty[REC_MAX_STAGES];
+  uint64_t b_full, b_empty;
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t kst_full[2], s_full[2];  // rotated keys written back / query contraction done
+  uint64_t done;
+  uint32_t tmem;
+  int abort;
+};
+constexpr int SCO_EPW = 8;                     // epilogue warps, two per TMEM lane quarter
+constexpr int SCO_THREADS = 64 + 32 * SCO_EPW;
+constexpr int SCO_QN = 16;                     // MMA N of the query contraction
+constexpr int SCO_Q_BYTES = 2 * SCO_QN * 128;  // one head's query operand: two 64-wide K slabs
+
+// Resident basis rows for hp heads, the U slab ring, the query operands, the warps' base angles,
+// barriers, RoPE table.
+size_t tc_sco_smem(int r, int hp, int stages) {
+  return 1024 + (size_t)hp * (r / 64) * SLAB_BYTES + (size_t)stages * SLAB_BYTES +
+         (size_t)hp * SCO_Q_BYTES + SCO_EPW * 32 * sizeof(float2) + sizeof(ScoCtl) +
+         sizeof(RopeTab);
+}
+
+template <int QPK>
+__global__ void __launch_bounds__(SCO_THREADS, 1) k_scores_tc(const TcJob *jobs, TcParams p,
+                                                          const __grid_constant__ RopeTab rt) {
+  static_assert(2 * QPK <= SCO_QN, "query group wider than the contraction");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int R = p.r, KS = R / 64, HP = p.hp, NA = p.stages;
+  constexpr int HN = 128;                   // columns per head
+  uint8_t *sB = smem;                       // KS slabs x (HP x 128 rows) x 128 B, resident
+  uint8_t *sA = sB + KS * HP * SLAB_BYTES;  // NA slabs x 16 KB
+  uint8_t *sQ = sA + NA * SLAB_BYTES;       // HP x [2 K slabs][16 rows][128 B], SW128
+  float2 *sBase = reinterpret_cast<float2 *>(sQ + HP * SCO_Q_BYTES);  // per epilogue warp: 32
+  ScoCtl *ctl = reinterpret_cast<ScoCtl *>(sBase + SCO_EPW * 32);
+  RopeTab *rope_tab = reinterpret_cast<RopeTab *>(ctl + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NN = HP * HN;                      // MMA N of the keys
+  const uint32_t ncols = HP == 2 ? 512 : 256;  // two accumulator buffers of NN columns
+  const uint32_t idesc = idesc_bf16_f32(TC_M, NN);
+  const uint32_t idesc_q = idesc_bf16_f32(TC_M, SCO_QN);
+  const int G = p.n_heads / HP, group = blockIdx.x / G, member = blockIdx.x % G;
+  const int ngroups = gridDim.x / G;
+  const int total = p.count * p.tiles_per_job;
+  const int per = (total + ngroups - 1) / ngroups;
+  const int t_begin = group * per, t_end = min(total, t_begin + per);
+  const int tpj = p.tiles_per_job;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(&ctl->a_full[i], 1);
+      mbar_init(&ctl->a_empty[i], 1);
+    }
+    mbar_init(&ctl->b_full, 1);
+    mbar_init(&ctl->b_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->acc_full[i], 1);
+      mbar_init(&ctl->acc_empty[i], SCO_EPW);
+      mbar_init(&ctl->kst_full[i], SCO_EPW);
+      mbar_init(&ctl->s_full[i], 1);
+    }
+    mbar_init(&ctl->done, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x < 64) {
+    rope_tab->wh[threadIdx.x] = rt.wh[threadIdx.x];
+    rope_tab->wl[threadIdx.x] = rt.wl[threadIdx.x];
+  }
+  if (warp == 1) tmem_alloc(&ctl->tmem, ncols);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = ctl->tmem;
+  volatile int *abort = &ctl->abort;
+  // Tile walk: linear tile t = j * tpj + k (history j, row tile k); every role visits the same
+  // valid tiles (a prefix of each history's tiles, below its current length) in the same order.
+  int cache_j = -1;
+  int64_t cache_n = 0;
+  auto rows_of = [&](int j) -> int64_t {
+    if (j != cache_j) {
+      cache_j = j;
+      cache_n = jobs[j].meta[ISKV_META_N];
+    }
+    return cache_n;
+  };
+  struct Cur {
+    int t, j, k;
+  };
+  auto seek = [&](Cur c) -> Cur {
+    while (c.t < t_end) {
+      if (c.k * TC_M < rows_of(c.j)) return c;
+      c.t += tpj - c.k;
+      ++c.j;
+      c.k = 0;
+    }
+    c.t = -1;
+    return c;
+  };
+  auto advance = [&](Cur c) -> Cur {
+    ++c.t;
+    if (++c.k == tpj) {
+      c.k = 0;
+      ++c.j;
+    }
+    return seek(c);
+  };
+  Cur c_first;
+  c_first.t = t_begin;
+  c_first.j = t_begin / tpj;
+  c_first.k = t_begin - c_first.j * tpj;
+  c_first = seek(c_first);
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer: basis rows of this CTA's heads once per history, U slabs per tile
+    int na = 0, nb = 0, cur = -1;
+    RingPos rp;
+    int64_t *fm = nullptr;
+    bool ok = true;
+    for (Cur c = c_first; c.t >= 0 && ok && !*abort; c = advance(c)) {
+      const int j = c.j, row0 = c.k * TC_M;
+      const TcJob &jb = jobs[j];
+      fm = jb.meta;
+      if (j != cur) {
+        if (nb > 0 && !mbar_wait(&ctl->b_empty, (nb - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
+        tensormap_acquire(&jb.mapA);
+        tensormap_acquire(&jb.mapB);
+        mbar_arrive_expect_tx(&ctl->b_full, KS * HP * SLAB_BYTES);
+        for (int s = 0; s < KS; ++s)
+          for (int h = 0; h < HP; ++h)
+            tma_load_2d(sB + (s * HP + h) * SLAB_BYTES, &jb.mapB, s * 64, (member * HP + h) * HN,
+                        &ctl->b_full);
+        cur = j;
+        ++nb;
+      }
+      for (int s = 0; s < KS; ++s) {
+        // The slot's previous use (one lap back) must have been consumed.
+        if (na >= NA && !mbar_wait(&ctl->a_empty[rp.slot], rp.phase ^ 1u, abort, WAIT_NS)) { ok = false; break; }
+        mbar_arrive_expect_tx(&ctl->a_full[rp.slot], SLAB_BYTES);
+        tma_load_2d(sA + rp.slot * SLAB_BYTES, &jb.mapA, s * 64, row0, &ctl->a_full[rp.slot]);
+        rp.next(NA);
+        ++na;
+      }
+    }
+    if (!ok) fail_timeout(ctl, fm);
+    if (nb > 0) mbar_wait(&ctl->b_full, (nb - 1) & 1, abort, WAIT_NS / 4);
+    for (int k = 1; k <= NA && na - k >= 0; ++k)
+      mbar_wait(&ctl->a_full[(na - k) % NA], ((na - k) / NA) & 1, abort, WAIT_NS / 4);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer: the keys of tile t, then the query contraction of tile t - 1
+    // (whose rotated keys the epilogue writes back while the tensor core forms tile t's keys).
+    int nb = 0, nc = 0, cur = -1;
+    int64_t *fm = nullptr;
+    bool ok = true;
+    int pbuf = -1, puse = 0;
+    RingPos rp;
+    const uint64_t da0 = sw128_desc(smem_u32(sA)), db0 = sw128_desc(smem_u32(sB));
+    const uint64_t dq0 = sw128_desc(smem_u32(sQ));
+    auto contract = [&](int buf, int use) -> bool {
+      if (!mbar_wait(&ctl->kst_full[buf], use & 1, abort, WAIT_NS)) return false;
+      fence_after_sync();
+      for (int h = 0; h < HP; ++h) {
+        const uint32_t a = tmem + buf * NN + h * HN;  // rotated keys: 64 columns, K = 128
+        const uint64_t dq = desc_add(dq0, h * SCO_Q_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(a + 64, a + kk * 8,
+                      desc_add(dq, (kk >> 2) * (SCO_QN * 128) + (kk & 3) * 32), idesc_q, kk != 0);
+      }
+      mma_commit(&ctl->s_full[buf]);
+      return true;
+    };
+    for (Cur c = c_first; c.t >= 0 && ok && !*abort; c = advance(c)) {
+      const int j = c.j;
+      fm = jobs[j].meta;
+      if (j != cur) {
+        if (nb > 0) mma_commit(&ctl->b_empty);
+        if (!mbar_wait(&ctl->b_full, nb & 1, abort, WAIT_NS)) { ok = false; break; }
+        cur = j;
+        ++nb;
+      }
+      const int buf = nc & 1, use = nc >> 1;
+      if (use > 0 && !mbar_wait(&ctl->acc_empty[buf], (use - 1) & 1, abort, WAIT_NS)) { ok = false; break; }
+      fence_after_sync();
+      const uint32_t d0 = tmem + buf * NN;
+      for (int s = 0; s < KS; ++s) {
+        if (!mbar_wait(&ctl->a_full[rp.slot], rp.phase, abort, WAIT_NS)) { ok = false; break; }
+        fence_after_sync();
+        const uint64_t da = desc_add(da0, rp.slot * SLAB_BYTES);
+        const uint64_t db = desc_add(db0, s * HP * SLAB_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(d0, desc_add(da, kk * 32), desc_add(db, kk * 32), idesc, (s | kk) != 0);
+        mma_commit(&ctl->a_empty[rp.slot]);
+        rp.next(NA);
+      }
+      if (!ok) break;
+      mma_commit(&ctl->acc_full[buf]);
+      if (pbuf >= 0 && !contract(pbuf, puse)) { ok = false; break; }
+      pbuf = buf;
+      puse = use;
+      ++nc;
+    }
+    if (ok && pbuf >= 0 && !*abort && !contract(pbuf, puse)) ok = false;
+    if (!ok) fail_timeout(ctl, fm);
+    mma_commit(&ctl->done);
+    mbar_wait(&ctl->done, 0, abort, WAIT_NS / 4);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: TMEM keys -> RoPE -> bf16 keys back to TMEM; scores -> S
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    const int j0 = half * 32;  // this warp's pairs j0 .. j0 + 31 of every head (cols j, j + 64)
+    const int srow = q * 32 + lane;
+    const int et = threadIdx.x - 64;
+    // RoPE by angle addition where a warp's 32 rows sit at consecutive positions p0 + lane: the
+    // rotation by lane omega_j is fixed per thread (computed once), the one by p0 omega_j is
+    // shared by the warp (one angle per lane, exchanged through shared memory). Both angles are
+    // reduced exactly in fixed point; the product adds float32 rounding only.
+    float oc[32], os[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) rope_angle(rope_tab, j0 + i, (uint32_t)lane, oc[i], os[i]);
+    float2 *wbase = sBase + (warp - 2) * 32;
+    int hj = -1;
+    const int32_t *h_pos = nullptr;
+    float *h_S = nullptr;
+    float h_scale = 0.f;
+    int64_t h_rows = 0, h_total = 0;
+    bool h_rope = false;
+    auto hist = [&](int j) {
+      if (j != hj) {
+        hj = j;
+        const TcJob &jb = jobs[j];
+        h_pos = jb.pos;
+        h_S = jb.S;
+        h_scale = jb.scale;
+        h_rows = rows_of(j);
+        h_total = jb.n_total;
+        h_rope = jb.rope != 0;
+      }
+    };
+    auto row_pos = [&](const Cur &c) -> int32_t {
+      if (c.t < 0) return 0;
+      hist(c.j);
+      const int64_t row = (int64_t)c.k * TC_M + srow;
+      return row < h_rows ? __ldg(h_pos + row) : 0;
+    };
+    int q_job = -1;
+    int nc = 0;
+    Cur c = c_first;
+    int32_t ps_next = row_pos(c);
+    for (;;) {
+      if (c.t < 0 || *abort) break;
+      const int jj = c.j;
+      const int32_t ps_raw = ps_next;
+      hist(jj);
+      bool valid = c.k * TC_M + srow < h_rows;
+      const Cur cn = advance(c);
+      ps_next = row_pos(cn);
+      const int64_t ps = valid ? (int64_t)ps_raw : 0;
+      if (valid && (ps < 0 || ps >= h_total)) {
+        record_status(jobs[jj].meta, ISKV_ERR_SHAPE);
+        valid = false;
+      }
+      if (jj != q_job) {
+        // The history's query operand. Row n < QPK: the bf16 head of query n of the CTA's head;
+        // row QPK + n: its bf16 remainder; other rows zero. K index 2j + e holds component
+        // j + 64 e (the column order of the rotated keys). Every contraction that read the
+        // previous operand has completed: this thread waited for its scores.
+        const float *qg = jobs[jj].q;
+        for (int e = et; e < HP * SCO_QN * 64; e += 32 * SCO_EPW) {
+          const int hh = e / (SCO_QN * 64), n = (e >> 6) % SCO_QN, j = e & 63;
+          uint32_t w = 0;
+          if (n < 2 * QPK) {
+            const float *qr = qg + (size_t)((member * HP + hh) * QPK + n % QPK) * HN;
+            float x0 = qr[j], x1 = qr[j + 64];
+            if (n >= QPK) {
+              x0 -= __bfloat162float(__float2bfloat16_rn(x0));
+              x1 -= __bfloat162float(__float2bfloat16_rn(x1));
+            }
+            w = pack_bf16(x0, x1);
+          }
+          // K index 2j: K slab j / 32, byte 4 (j % 32) of the 128-byte row, whose 16-byte chunks
+          // are swizzled by the row (the layout a 128-byte-swizzled TMA box has).
+          const int chunk = (j & 31) >> 2;
+          *reinterpret_cast<uint32_t *>(sQ + hh * SCO_Q_BYTES + (j >> 5) * (SCO_QN * 128) +
+                                        n * 128 + ((chunk ^ (n & 7)) << 4) + 4 * (j & 3)) = w;
+        }
+        fence_proxy_async_smem();
+        q_job = jj;
+      }
+      // 0: no rotation, 1: consecutive positions (angle addition), 2: each row on its own.
+      const int64_t p0 = __shfl_sync(~0u, ps, 0);
+      const int mode = !h_rope ? 0 : __all_sync(~0u, valid && ps == p0 + lane) ? 1 : 2;
+      if (mode == 1) {  // the previous tile's reads of wbase are behind this warp's last __syncwarp
+        float c0, s0;
+        rope_angle(rope_tab, j0 + lane, (uint32_t)p0, c0, s0);
+        wbase[lane] = make_float2(c0, s0);
+        __syncwarp();
+      }
+      const int buf = nc & 1, use = nc >> 1;
+      if (!mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS)) {
+        fail_timeout(ctl, jobs[jj].meta);
+        break;
+      }
+      fence_after_sync();
+      const uint32_t base = tmem + buf * NN + ((uint32_t)(q * 32) << 16);
+#pragma unroll
+      for (int jb16 = 0; jb16 < 32; jb16 += 16) {
+        float cs[16], sn[16];
+        if (mode == 1) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 a = wbase[jb16 + i];
+            cs[i] = a.x * oc[jb16 + i] - a.y * os[jb16 + i];
+            sn[i] = a.y * oc[jb16 + i] + a.x * os[jb16 + i];
+          }
+        } else if (mode == 2 && valid) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            rope_angle(rope_tab, j0 + jb16 + i, (uint32_t)ps, cs[i], sn[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            cs[i] = 1.f;
+            sn[i] = 0.f;
+          }
+        }
+        for (int h = 0; h < HP; ++h) {
+          float lo[16], hi[16];
+          tmem_ld16(base + h * HN + j0 + jb16, lo);
+          tmem_ld16(base + h * HN + 64 + j0 + jb16, hi);
+          tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16(lo[i] * cs[i] - hi[i] * sn[i], hi[i] * cs[i] + lo[i] * sn[i]);
+          // Over this warp's own low-component columns, already read.
+          tmem_st16(base + h * HN + j0 + jb16, w);
+        }
+      }
+      tmem_st_wait();
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->kst_full[buf]);
+      if (!mbar_wait(&ctl->s_full[buf], use & 1, abort, WAIT_NS)) {
+        fail_timeout(ctl, jobs[jj].meta);
+        break;
+      }
+      fence_after_sync();
+      if (half < HP) {  // warp half h reads head h's scores: columns 64 .. 64 + 2 QPK
+        float sc[16];
+        tmem_ld16(base + half * HN + 64, sc);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int g = 0; g < QPK; ++g)
+            h_S[(size_t)((member * HP + half) * QPK + g) * h_total + ps] =
+                h_scale * (sc[g] + sc[QPK + g]);
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+      ++nc;
+      c = cn;
+    }
   }
   fence_before_sync();
   __syncthreads();
@@ -1389,19 +1687,19 @@ static cudaError_t launch_rotate(const TcJob *djobs, int count, int r, int d, in
 
 // Resident basis rows for hp heads, the U slab ring, the output staging rows, the barriers and the
 // RoPE frequencies.
-size_t tc_rec_smem(int r, int hp, int stages, int stg_bytes) {
+size_t tc_rec_smem(int r, int hp, int stages) {
   return 1024 + (size_t)hp * (r / 64) * SLAB_BYTES + (size_t)stages * SLAB_BYTES +
-         (size_t)stg_bytes + sizeof(RecCtl) + sizeof(RopeTab);
+         (size_t)REC_STG_BYTES + sizeof(RecCtl) + sizeof(RopeTab);
 }
 
 constexpr size_t kRecSmemCap = 227 * 1024;
 
 // Heads per CTA and U ring depth for the reconstruction: two heads when the head count is even,
 // and as many 16 KB slabs (up to REC_MAX_STAGES) as the shared memory left over holds.
-void tc_rec_shape(int r, int n_heads, int stg_bytes, int &hp, int &stages) {
-  hp = (n_heads % 2 == 0 && tc_rec_smem(r, 2, 3, stg_bytes) <= kRecSmemCap) ? 2 : 1;
+void tc_rec_shape(int r, int n_heads, int &hp, int &stages) {
+  hp = (n_heads % 2 == 0 && tc_rec_smem(r, 2, 3) <= kRecSmemCap) ? 2 : 1;
   stages = REC_MAX_STAGES;
-  while (stages > 2 && tc_rec_smem(r, hp, stages, stg_bytes) > kRecSmemCap) --stages;
+  while (stages > 2 && tc_rec_smem(r, hp, stages) > kRecSmemCap) --stages;
 }
 
 cudaError_t launch_tc_rotation(const TcJob *djobs, int count, int r, int64_t n_cap_max,
@@ -1480,9 +1778,9 @@ cudaError_t launch_tc_recon(const TcJob *djobs, const ReconParams &p, cudaStream
   tp.count = p.count;
   tp.tiles_per_job = (int)((p.n_cap_max + TC_M - 1) / TC_M);
   tp.theta = p.theta;
-  tc_rec_shape(p.r, p.n_heads, REC_STG_BYTES, tp.hp, tp.stages);
-  const size_t smem = tc_rec_smem(p.r, tp.hp, tp.stages, REC_STG_BYTES);
-  cudaError_t e = cudaFuncSetAttribute(k_rec_tc<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  tc_rec_shape(p.r, p.n_heads, tp.hp, tp.stages);
+  const size_t smem = tc_rec_smem(p.r, tp.hp, tp.stages);
+  cudaError_t e = cudaFuncSetAttribute(k_rec_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Whole groups of n_heads / hp CTAs, as many as fit one per SM (at least one group), and no
   // more groups than row tiles.
@@ -1491,7 +1789,7 @@ cudaError_t launch_tc_recon(const TcJob *djobs, const ReconParams &p, cudaStream
   int groups = num_sms() / G;
   if (groups < 1) groups = 1;
   if (groups > total) groups = total;
-  k_rec_tc<0><<<groups * G, rec_threads(0), smem, s>>>(djobs, tp, make_rope_tab(p.theta));
+  k_rec_tc<<<groups * G, REC_THREADS, smem, s>>>(djobs, tp, make_rope_tab(p.theta));
   count_launches(1);
   return cudaGetLastError();
 }
@@ -1522,15 +1820,15 @@ bool encode_attn_job(TcJob &tj, const void *U, int64_t n_cap, int r, const void 
 
 template <int QPK>
 static cudaError_t attn_scores_qpk(const TcJob *djobs, const TcParams &tp, int G, cudaStream_t s) {
-  const size_t smem = tc_rec_smem(tp.r, tp.hp, tp.stages, rec_stg_bytes(QPK));
-  cudaError_t e = cudaFuncSetAttribute(k_rec_tc<QPK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const size_t smem = tc_sco_smem(tp.r, tp.hp, tp.stages);
+  cudaError_t e = cudaFuncSetAttribute(k_scores_tc<QPK>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int total = tp.count * tp.tiles_per_job;
   int groups = num_sms() / G;
   if (groups < 1) groups = 1;
   if (groups > total) groups = total;
-  k_rec_tc<QPK><<<groups * G, rec_threads(QPK), smem, s>>>(djobs, tp, make_rope_tab(tp.theta));
+  k_scores_tc<QPK><<<groups * G, SCO_THREADS, smem, s>>>(djobs, tp, make_rope_tab(tp.theta));
   count_launches(1);
   return cudaGetLastError();
 }
@@ -1544,7 +1842,10 @@ cudaError_t launch_tc_attn_scores(const TcJob *djobs, const AttnParams &p, cudaS
   tp.tiles_per_job = (int)((p.n_cap_max + TC_M - 1) / TC_M);
   tp.theta = p.theta;
   const int qpk = p.n_q / p.n_kv;
-  tc_rec_shape(p.rk, p.n_kv, rec_stg_bytes(qpk), tp.hp, tp.stages);
+  // Two heads per CTA when the head count is even; as deep a U slab ring as the rest leaves room for.
+  tp.hp = (p.n_kv % 2 == 0 && tc_sco_smem(p.rk, 2, 3) <= kRecSmemCap) ? 2 : 1;
+  tp.stages = REC_MAX_STAGES;
+  while (tp.stages > 2 && tc_sco_smem(p.rk, tp.hp, tp.stages) > kRecSmemCap) --tp.stages;
   const int G = p.n_kv / tp.hp;
   switch (qpk) {
     case 1: return attn_scores_qpk<1>(djobs, tp, G, s);

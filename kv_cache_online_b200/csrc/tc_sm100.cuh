@@ -177,6 +177,24 @@ ISKV_DEV uint64_t sw128_mn_desc(uint32_t smem_addr, uint32_t slab_bytes) {
   return d;
 }
 
+// The descriptor of a tile `bytes` further on (16-byte units in the start-address field; shared
+// memory addresses stay below 2^18, so the field does not overflow).
+ISKV_DEV uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
+// Position in a ring of n pipeline stages: slot and the parity of its current use, advanced
+// without division. An MMA issuer sits on the tensor core's critical path: the tensor pipe
+// holds almost no queue, so every instruction between two MMAs is idle tensor time.
+struct RingPos {
+  int slot = 0;
+  uint32_t phase = 0;
+  ISKV_DEV void next(int n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, both operands MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
@@ -207,6 +225,19 @@ ISKV_DEV void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T: A is M = 128 rows, one per TMEM lane, two 16-bit K elements
+// per 32-bit column (low half first), K-major; one elected thread.
+ISKV_DEV void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                          bool accumulate) {
+  const uint32_t acc = accumulate ? 1u : 0u;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
 // Arrive on `bar` once every MMA this thread issued so far has completed.
 ISKV_DEV void mma_commit(uint64_t *bar) {
   asm volatile(
@@ -230,6 +261,18 @@ ISKV_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 }
 
 ISKV_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 16 consecutive 32-bit columns from registers: thread i writes lane (base lane + i).
+ISKV_DEV void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+ISKV_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 ISKV_DEV uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);

@@ -12,14 +12,15 @@ pytestmark = pytest.mark.gpu
 
 
 def _case(m, *, n, d, r, k, n_kv, hd, n_q, prompt, window, storage, exact_dtype, seed,
-          gap=1, qscale=48.0, theta=500000.0, n_cap=None):
+          gap=1, qscale=48.0, theta=500000.0, n_cap=None, offsets=None):
     """K and V histories at the same positions (compressed rows every `gap` positions after the
-    prompt, the other positions exact), exact prompt and window rows, one query."""
+    prompt, shifted by `offsets` if given, the other positions exact), exact prompt and window
+    rows, one query."""
     g = np.random.Generator(np.random.PCG64(seed))
     Uk, sk, Bk = synthetic_history(n, d, k, seed, 1.2, storage)
     Uv, sv, Bv = synthetic_history(n, d, k, seed + 1, 0.6, storage)
-    n_total = prompt + n * gap + window
-    comp = prompt + gap * np.arange(n)
+    comp = prompt + gap * np.arange(n) + (0 if offsets is None else offsets)
+    n_total = int(comp[-1]) + 1 + window
     exact = np.setdiff1d(np.arange(n_total), comp)
     cap = n + 8 if n_cap is None else n_cap
     hk = m.LowRankHistory(d, r, cap, storage=storage)
@@ -62,6 +63,26 @@ def test_tensor_core_scores_grouped_query_shapes(n_q):
     hk, hv, a, ref = _case(m, n=1000, d=1024, r=256, k=256, n_kv=8, hd=128, n_q=n_q, prompt=512,
                            window=128, storage=torch.bfloat16, exact_dtype=torch.bfloat16,
                            seed=20 + n_q)
+    out = m.decode_attention(hk, hv, a["k_exact"], a["k_exact_pos"], a["v_exact"],
+                             a["v_exact_pos"], a["n_total"], a["q"], 8, 128)
+    assert hk.status()[3] == 0 and hv.status()[3] == 0
+    assert _rel(out.double().cpu().numpy(), ref) < 2e-2
+
+
+@pytest.mark.parametrize("layout", ["consecutive", "gapped", "jumps"])
+def test_tensor_core_scores_position_layouts(layout):
+    """The tensor-core scores kernel rotates a warp's 32 keys by angle addition when their
+    positions are consecutive and each key on its own otherwise: consecutive positions, every
+    third position, and runs broken inside a warp (rows 40 and 150), over a short history whose
+    every key weighs in the softmax, with a ragged last tile."""
+    m = kv()
+    n = 300
+    offsets = None
+    if layout == "jumps":
+        offsets = np.where(np.arange(n) >= 40, 7, 0) + np.where(np.arange(n) >= 150, 13, 0)
+    hk, hv, a, ref = _case(m, n=n, d=1024, r=256, k=256, n_kv=8, hd=128, n_q=32, prompt=8,
+                           window=8, storage=torch.bfloat16, exact_dtype=torch.bfloat16, seed=71,
+                           gap=3 if layout == "gapped" else 1, offsets=offsets)
     out = m.decode_attention(hk, hv, a["k_exact"], a["k_exact_pos"], a["v_exact"],
                              a["v_exact_pos"], a["n_total"], a["q"], 8, 128)
     assert hk.status()[3] == 0 and hv.status()[3] == 0
