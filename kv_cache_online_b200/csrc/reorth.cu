@@ -441,13 +441,15 @@ __global__ void __launch_bounds__(NS_TC_THREADS, 1) k_ns_tc(const ReorthJob *job
       const int st = s & 1;
       if (!mbar_wait(&ctl->full[st], (s >> 1) & 1, abort, NS_WAIT_NS)) { ok = false; break; }
       fence_after_sync();
-      const uint32_t ahi = smem_u32(smem + st * ns_tc_stage_bytes()), alo = ahi + 128 * 128;
-      const uint32_t bhi = alo + 128 * 128, blo = bhi + 256 * 128;
+      const uint64_t ahi = sw128_desc(smem_u32(smem + st * ns_tc_stage_bytes()));
+      const uint64_t alo = desc_add(ahi, 128 * 128), bhi = desc_add(alo, 128 * 128);
+      const uint64_t blo = desc_add(bhi, 256 * 128);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        mma_bf16(tmem, sw128_desc(ahi + kk * 32), sw128_desc(bhi + kk * 32), idesc, (s | kk) != 0);
-        mma_bf16(tmem, sw128_desc(ahi + kk * 32), sw128_desc(blo + kk * 32), idesc, true);
-        mma_bf16(tmem, sw128_desc(alo + kk * 32), sw128_desc(bhi + kk * 32), idesc, true);
+        const uint32_t o = kk * 32;
+        mma_bf16(tmem, desc_add(ahi, o), desc_add(bhi, o), idesc, (s | kk) != 0);
+        mma_bf16(tmem, desc_add(ahi, o), desc_add(blo, o), idesc, true);
+        mma_bf16(tmem, desc_add(alo, o), desc_add(bhi, o), idesc, true);
       }
       mma_commit(&ctl->empty[st]);
     }

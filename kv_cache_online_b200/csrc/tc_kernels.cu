@@ -1276,19 +1276,45 @@ __global__ void __launch_bounds__(SCO_THREADS, 1) k_scores_tc(const TcJob *jobs,
     int nc = 0;
     Cur c = c_first;
     int32_t ps_next = row_pos(c);
-    for (;;) {
-      if (c.t < 0 || *abort) break;
-      const int jj = c.j;
+    // The tile about to be staged, prepared one step ahead (while the previous tile's query
+    // contraction runs): its history, row validity and position, rotation mode, where its scores
+    // go, and (mode 1) the warp's base angles in wbase. The history fields are copied here: the
+    // position prefetch of the tile after it may move the cached fields to the next history.
+    int jj = 0, mode = 0;
+    bool valid = false;
+    int64_t ps = 0, t_total = 0;
+    float *t_S = nullptr;
+    float t_scale = 0.f;
+    Cur cn = c;
+    auto prepare = [&]() {
+      jj = c.j;
       const int32_t ps_raw = ps_next;
       hist(jj);
-      bool valid = c.k * TC_M + srow < h_rows;
-      const Cur cn = advance(c);
-      ps_next = row_pos(cn);
-      const int64_t ps = valid ? (int64_t)ps_raw : 0;
-      if (valid && (ps < 0 || ps >= h_total)) {
+      valid = c.k * TC_M + srow < h_rows;
+      t_S = h_S;
+      t_total = h_total;
+      t_scale = h_scale;
+      const bool rope = h_rope;
+      ps = valid ? (int64_t)ps_raw : 0;
+      if (valid && (ps < 0 || ps >= t_total)) {
         record_status(jobs[jj].meta, ISKV_ERR_SHAPE);
         valid = false;
       }
+      cn = advance(c);
+      ps_next = row_pos(cn);
+      // 0: no rotation, 1: consecutive positions (angle addition), 2: each row on its own.
+      const int64_t p0 = __shfl_sync(~0u, ps, 0);
+      mode = !rope ? 0 : __all_sync(~0u, valid && ps == p0 + lane) ? 1 : 2;
+      if (mode == 1) {  // the last reads of wbase are behind this warp's last __syncwarp
+        float c0, s0;
+        rope_angle(rope_tab, j0 + lane, (uint32_t)p0, c0, s0);
+        wbase[lane] = make_float2(c0, s0);
+        __syncwarp();
+      }
+    };
+    if (c.t >= 0) prepare();
+    for (;;) {
+      if (c.t < 0 || *abort) break;
       if (jj != q_job) {
         // The history's query operand. Row n < QPK: the bf16 head of query n of the CTA's head;
         // row QPK + n: its bf16 remainder; other rows zero. K index 2j + e holds component
@@ -1315,15 +1341,6 @@ __global__ void __launch_bounds__(SCO_THREADS, 1) k_scores_tc(const TcJob *jobs,
         }
         fence_proxy_async_smem();
         q_job = jj;
-      }
-      // 0: no rotation, 1: consecutive positions (angle addition), 2: each row on its own.
-      const int64_t p0 = __shfl_sync(~0u, ps, 0);
-      const int mode = !h_rope ? 0 : __all_sync(~0u, valid && ps == p0 + lane) ? 1 : 2;
-      if (mode == 1) {  // the previous tile's reads of wbase are behind this warp's last __syncwarp
-        float c0, s0;
-        rope_angle(rope_tab, j0 + lane, (uint32_t)p0, c0, s0);
-        wbase[lane] = make_float2(c0, s0);
-        __syncwarp();
       }
       const int buf = nc & 1, use = nc >> 1;
       if (!mbar_wait(&ctl->acc_full[buf], use & 1, abort, WAIT_NS)) {
@@ -1370,8 +1387,17 @@ __global__ void __launch_bounds__(SCO_THREADS, 1) k_scores_tc(const TcJob *jobs,
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->kst_full[buf]);
+      // This tile's scores go where it was prepared to send them; the next tile is prepared
+      // while its contraction runs.
+      const int j_done = jj;
+      float *const s_out = t_S;
+      const int64_t s_total = t_total, s_ps = ps;
+      const float s_scale = t_scale;
+      const bool s_valid = valid;
+      c = cn;
+      if (c.t >= 0) prepare();
       if (!mbar_wait(&ctl->s_full[buf], use & 1, abort, WAIT_NS)) {
-        fail_timeout(ctl, jobs[jj].meta);
+        fail_timeout(ctl, jobs[j_done].meta);
         break;
       }
       fence_after_sync();
@@ -1379,18 +1405,17 @@ __global__ void __launch_bounds__(SCO_THREADS, 1) k_scores_tc(const TcJob *jobs,
         float sc[16];
         tmem_ld16(base + half * HN + 64, sc);
         tmem_ld_wait();
-        if (valid) {
+        if (s_valid) {
 #pragma unroll
           for (int g = 0; g < QPK; ++g)
-            h_S[(size_t)((member * HP + half) * QPK + g) * h_total + ps] =
-                h_scale * (sc[g] + sc[QPK + g]);
+            s_out[(size_t)((member * HP + half) * QPK + g) * s_total + s_ps] =
+                s_scale * (sc[g] + sc[QPK + g]);
         }
       }
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
       ++nc;
-      c = cn;
     }
   }
   fence_before_sync();
@@ -1483,20 +1508,21 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, 
       mbar_wait(&full[(nk - k) % GRAM_RING], ((nk - k) / GRAM_RING) & 1, abort, WAIT_NS / 4);
   } else if (warp == 1 && lane == 0) {
     bool ok = true;
+    RingPos rp;
+    const uint64_t d0 = sw128_mn_desc(smem_u32(smem), GRAM_KT * 128);
     for (int kt = 0; kt < nk && ok && !*abort; ++kt) {
-      const int st = kt % GRAM_RING, use = kt / GRAM_RING;
-      if (!mbar_wait(&full[st], use & 1, abort, WAIT_NS)) { ok = false; break; }
+      if (!mbar_wait(&full[rp.slot], rp.phase, abort, WAIT_NS)) { ok = false; break; }
       fence_after_sync();
-      const uint32_t base = smem_u32(smem + st * STAGE_BYTES);
+      const uint64_t ds = desc_add(d0, rp.slot * STAGE_BYTES);
 #pragma unroll
       for (int kk = 0; kk < GRAM_KT / 16; ++kk) {
-        const uint64_t bdesc = sw128_mn_desc(base + kk * 2048, GRAM_KT * 128);
-        for (int h = 0; h < MH; ++h) {
-          const uint64_t adesc = sw128_mn_desc(base + h * 2 * GRAM_KT * 128 + kk * 2048, GRAM_KT * 128);
-          mma_bf16(tmem + h * N, adesc, bdesc, idesc, (kt | kk) != 0);
-        }
+        const uint64_t bdesc = desc_add(ds, kk * 2048);
+        for (int h = 0; h < MH; ++h)
+          mma_bf16(tmem + h * N, desc_add(bdesc, h * 2 * GRAM_KT * 128), bdesc, idesc,
+                   (kt | kk) != 0);
       }
-      mma_commit(&empty[st]);
+      mma_commit(&empty[rp.slot]);
+      rp.next(GRAM_RING);
     }
     if (!ok) fail_timeout(ctl, jb.meta);
     mma_commit(&ctl->acc_full[0]);
@@ -1923,20 +1949,21 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_pv_tc(const TcJob *jobs, Pv
       mbar_wait(&full[(nk - k) % GRAM_STAGES], ((nk - k) / GRAM_STAGES) & 1, abort, WAIT_NS / 4);
   } else if (warp == 1 && lane == 0) {
     bool ok = true;
+    RingPos rp;
+    const uint64_t d0 = sw128_mn_desc(smem_u32(smem), SLAB);
     for (int kt = 0; kt < nk && ok && !*abort; ++kt) {
-      const int st = kt % GRAM_STAGES, use = kt / GRAM_STAGES;
-      if (!mbar_wait(&full[st], use & 1, abort, WAIT_NS)) { ok = false; break; }
+      if (!mbar_wait(&full[rp.slot], rp.phase, abort, WAIT_NS)) { ok = false; break; }
       fence_after_sync();
-      const uint32_t base = smem_u32(smem + st * STAGE_BYTES);
+      const uint64_t ds = desc_add(d0, rp.slot * STAGE_BYTES);
 #pragma unroll
       for (int kk = 0; kk < GRAM_KT / 16; ++kk) {
-        const uint64_t bdesc = sw128_mn_desc(base + SL * SLAB + kk * 2048, SLAB);
-        for (int h = 0; h < MH; ++h) {
-          const uint64_t adesc = sw128_mn_desc(base + h * 2 * SLAB + kk * 2048, SLAB);
-          mma_bf16(tmem + h * N, adesc, bdesc, idesc, (kt | kk) != 0);
-        }
+        const uint64_t bdesc = desc_add(ds, SL * SLAB + kk * 2048);
+        for (int h = 0; h < MH; ++h)
+          mma_bf16(tmem + h * N, desc_add(ds, h * 2 * SLAB + kk * 2048), bdesc, idesc,
+                   (kt | kk) != 0);
       }
-      mma_commit(&empty[st]);
+      mma_commit(&empty[rp.slot]);
+      rp.next(GRAM_STAGES);
     }
     if (!ok) fail_timeout(ctl, jb.meta);
     mma_commit(&ctl->acc_full[0]);

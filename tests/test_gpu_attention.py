@@ -117,6 +117,29 @@ def test_batched_equals_single():
         assert _rel(o.double().cpu().numpy(), ref) < 2e-2
 
 
+def test_batched_tile_ranges_cross_histories():
+    """Six histories of different lengths, prompts and windows in one call. The tensor-core
+    kernels cut the tiles of all histories into contiguous per-CTA ranges, so ranges run from
+    the end of one history into the next: every history's output must equal its own call."""
+    m = kv()
+    spec = ((1000, 64, 32), (2500, 100, 16), (3100, 8, 64), (1800, 300, 8), (3900, 40, 40),
+            (700, 16, 128))
+    cases = [_case(m, n=n, d=1024, r=256, k=256, n_kv=8, hd=128, n_q=32, prompt=pr, window=wi,
+                   storage=torch.bfloat16, exact_dtype=torch.bfloat16, seed=90 + i, n_cap=4096)
+             for i, (n, pr, wi) in enumerate(spec)]
+    outs = m.decode_attention_batched(
+        [c[0] for c in cases], [c[1] for c in cases], [c[2]["k_exact"] for c in cases],
+        [c[2]["k_exact_pos"] for c in cases], [c[2]["v_exact"] for c in cases],
+        [c[2]["v_exact_pos"] for c in cases], [c[2]["n_total"] for c in cases],
+        [c[2]["q"] for c in cases], 8, 128)
+    for (hk, hv, a, ref), o in zip(cases, outs):
+        single = m.decode_attention(hk, hv, a["k_exact"], a["k_exact_pos"], a["v_exact"],
+                                    a["v_exact_pos"], a["n_total"], a["q"], 8, 128)
+        assert hk.status()[3] == 0 and hv.status()[3] == 0
+        assert torch.equal(single, o)
+        assert _rel(o.double().cpu().numpy(), ref) < 2e-2
+
+
 def test_key_without_value_is_flagged():
     """A key position whose value row is missing leaves probability mass unaccounted: SHAPE."""
     m = kv()
