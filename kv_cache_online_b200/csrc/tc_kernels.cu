@@ -1508,21 +1508,20 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_gram_tc(const TcJob *jobs, 
       mbar_wait(&full[(nk - k) % GRAM_RING], ((nk - k) / GRAM_RING) & 1, abort, WAIT_NS / 4);
   } else if (warp == 1 && lane == 0) {
     bool ok = true;
-    RingPos rp;
-    const uint64_t d0 = sw128_mn_desc(smem_u32(smem), GRAM_KT * 128);
     for (int kt = 0; kt < nk && ok && !*abort; ++kt) {
-      if (!mbar_wait(&full[rp.slot], rp.phase, abort, WAIT_NS)) { ok = false; break; }
+      const int st = kt % GRAM_RING, use = kt / GRAM_RING;
+      if (!mbar_wait(&full[st], use & 1, abort, WAIT_NS)) { ok = false; break; }
       fence_after_sync();
-      const uint64_t ds = desc_add(d0, rp.slot * STAGE_BYTES);
+      const uint32_t base = smem_u32(smem + st * STAGE_BYTES);
 #pragma unroll
       for (int kk = 0; kk < GRAM_KT / 16; ++kk) {
-        const uint64_t bdesc = desc_add(ds, kk * 2048);
-        for (int h = 0; h < MH; ++h)
-          mma_bf16(tmem + h * N, desc_add(bdesc, h * 2 * GRAM_KT * 128), bdesc, idesc,
-                   (kt | kk) != 0);
+        const uint64_t bdesc = sw128_mn_desc(base + kk * 2048, GRAM_KT * 128);
+        for (int h = 0; h < MH; ++h) {
+          const uint64_t adesc = sw128_mn_desc(base + h * 2 * GRAM_KT * 128 + kk * 2048, GRAM_KT * 128);
+          mma_bf16(tmem + h * N, adesc, bdesc, idesc, (kt | kk) != 0);
+        }
       }
-      mma_commit(&empty[rp.slot]);
-      rp.next(GRAM_RING);
+      mma_commit(&empty[st]);
     }
     if (!ok) fail_timeout(ctl, jb.meta);
     mma_commit(&ctl->acc_full[0]);
@@ -1949,21 +1948,20 @@ __global__ void __launch_bounds__(GRAM_THREADS, 1) k_pv_tc(const TcJob *jobs, Pv
       mbar_wait(&full[(nk - k) % GRAM_STAGES], ((nk - k) / GRAM_STAGES) & 1, abort, WAIT_NS / 4);
   } else if (warp == 1 && lane == 0) {
     bool ok = true;
-    RingPos rp;
-    const uint64_t d0 = sw128_mn_desc(smem_u32(smem), SLAB);
     for (int kt = 0; kt < nk && ok && !*abort; ++kt) {
-      if (!mbar_wait(&full[rp.slot], rp.phase, abort, WAIT_NS)) { ok = false; break; }
+      const int st = kt % GRAM_STAGES, use = kt / GRAM_STAGES;
+      if (!mbar_wait(&full[st], use & 1, abort, WAIT_NS)) { ok = false; break; }
       fence_after_sync();
-      const uint64_t ds = desc_add(d0, rp.slot * STAGE_BYTES);
+      const uint32_t base = smem_u32(smem + st * STAGE_BYTES);
 #pragma unroll
       for (int kk = 0; kk < GRAM_KT / 16; ++kk) {
-        const uint64_t bdesc = desc_add(ds, SL * SLAB + kk * 2048);
-        for (int h = 0; h < MH; ++h)
-          mma_bf16(tmem + h * N, desc_add(ds, h * 2 * SLAB + kk * 2048), bdesc, idesc,
-                   (kt | kk) != 0);
+        const uint64_t bdesc = sw128_mn_desc(base + SL * SLAB + kk * 2048, SLAB);
+        for (int h = 0; h < MH; ++h) {
+          const uint64_t adesc = sw128_mn_desc(base + h * 2 * SLAB + kk * 2048, SLAB);
+          mma_bf16(tmem + h * N, adesc, bdesc, idesc, (kt | kk) != 0);
+        }
       }
-      mma_commit(&empty[rp.slot]);
-      rp.next(GRAM_STAGES);
+      mma_commit(&empty[st]);
     }
     if (!ok) fail_timeout(ctl, jb.meta);
     mma_commit(&ctl->acc_full[0]);
