@@ -578,7 +578,8 @@ def run_b200(args):
     rl_hbm = {"kernel": ROOFLINE_STAGE, "bound": "hbm",
               "achieved": stages[ROOFLINE_STAGE]["achieved_gbs"], "peak": hbm, "unit": "GB/s",
               "frac": stages[ROOFLINE_STAGE]["frac_hbm"],
-              "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+              "peak_source": ("MEASURED_PEAKS.json hbm_gbs (burst copy)" if peak_kind == "measured"
+                              else "fallback 6650 GB/s (no MEASURED_PEAKS.json)"),
               "traffic": traffic}
     if earlier is not None:
         rl_hbm["traffic_earlier_capture"] = earlier
