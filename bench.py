@@ -457,8 +457,9 @@ def fp32_peak_tflops(sm_mhz):
 
 def core_roofline(stats, stage, peak_tflops):
     """Achieved float32 rate of the core SVD stage: the flops the kernel executed (counted on the
-    device: pair inner products and applied rotations) over its measured time, and the survey's
-    algorithmic count 7 (k + b)^3 flops per sweep per core for comparison."""
+    device: pair inner products and applied rotations) over its measured time, and for comparison
+    the usual estimate of about 7 (k + b)^3 flops per one-sided Jacobi sweep of a (k + b)-column
+    core."""
     if not stats["cores"] or stage is None:
         return None
     ms = stage["ms_per_call"] * stage["calls"]
@@ -773,7 +774,7 @@ def run_e2e(wl, kv, torch, dev, stream, pos, first_step, steps, world):
 
 
 # ------------------------------------------------------------------------------------------------
-# CPU oracle legs (the baseline the task asks for; never a target).
+# CPU oracle legs: the float64 oracle timed on the host cores, a reported baseline (never a target).
 
 _KEYS = {}
 SEL_SLICE = SEL_L // (2 * LAYERS)  # one history's share of the step's prompt selection
